@@ -1,0 +1,264 @@
+/*
+ * pa_oracle.c -- plain fp64 CPU oracle for paged decode attention and the two
+ * cache operations that feed it.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the tests, the package's smoke() entry and the
+ * bench's CPU-baseline / reference arm may load this library.  It shares no code
+ * with the CUDA path (no headers, no helpers, no tables) and is deliberately
+ * slow: every loop follows the definition of the operation, with no blocking,
+ * no online softmax and no split over partitions.
+ *
+ * Sources (web pages on vLLM / PagedAttention):
+ *  - "详解vLLM推理引擎架构" (tbr8.org), section "PagedAttention 的核心思想":
+ *    the KV cache is cut into fixed-size blocks of 16 or 32 tokens; a per-sequence
+ *    block table maps logical block b to a physical block anywhere in the pool.
+ *  - same page, section "Copy-on-Write 与内存共享": a write to a block whose
+ *    refcount exceeds 1 first copies the block (copy_block(old, new)).
+ *  - "vLLM 深度解读" (luoboask.github.io), section 3 "PagedAttention CUDA Kernel":
+ *    k_cache / v_cache are [num_blocks, block_size, num_kv_heads, head_size];
+ *    q and out are [num_seqs, num_heads, head_size]; the element of token t of a
+ *    sequence lives at physical_block*block_size*num_kv_heads*head_size
+ *    + (t % block_size)*num_kv_heads*head_size + head*head_size, with
+ *    physical_block = block_table[t / block_size]; the score is
+ *    scale * sum_d q[d]*k[d] and the result is softmax(scores) applied to V.
+ *  - "vLLM 深度解读", section 7 (Llama attention): new K/V are stored into the
+ *    paged cache before attention runs, so the context includes the new token.
+ *
+ * Readings where the pages are silent or inconsistent:
+ *  - the printed kernel indexes K with the query head although it receives
+ *    num_kv_heads; under grouped-query attention query head hq reads KV head
+ *    hq / (num_q_heads / num_kv_heads) (contiguous groups);
+ *  - the softmax is the textbook one, computed here in two passes in fp64 with
+ *    libm exp; a sequence of length 0 yields an all-zero output row;
+ *  - a negative slot in slot_mapping means "no write".
+ *
+ * Parity pins for every function live in tests/test_oracle_pins.py.
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+enum { OR_F32 = 0, OR_F16 = 1, OR_BF16 = 2 };
+
+enum {
+  OR_OK = 0,
+  OR_ERR_ARG = -1,      /* bad sizes, dtype or null pointer */
+  OR_ERR_RANGE = -2,    /* an index (block id, slot, pair) is out of range */
+  OR_ERR_NOMEM = -3,
+};
+
+/* IEEE-754 binary16 -> double, from the format's definition:
+ * 1 sign bit, 5 exponent bits (bias 15), 10 fraction bits; exponent 0 encodes
+ * subnormals m * 2^-24, exponent 31 encodes inf / NaN. */
+double oracle_f16_to_f64(uint16_t h) {
+  int sign = (h >> 15) & 1;
+  int e = (h >> 10) & 0x1f;
+  int m = h & 0x3ff;
+  double v;
+  if (e == 0) {
+    v = ldexp((double)m, -24);
+  } else if (e == 31) {
+    v = m ? NAN : INFINITY;
+  } else {
+    v = ldexp((double)(m + 1024), e - 25);
+  }
+  return sign ? -v : v;
+}
+
+/* bfloat16 -> double: a bfloat16 is the upper half of an IEEE binary32. */
+double oracle_bf16_to_f64(uint16_t b) {
+  uint32_t u = (uint32_t)b << 16;
+  float f;
+  memcpy(&f, &u, sizeof f);
+  return (double)f;
+}
+
+static double load_elem(const void* base, int64_t idx, int dtype) {
+  switch (dtype) {
+    case OR_F32: return (double)((const float*)base)[idx];
+    case OR_F16: return oracle_f16_to_f64(((const uint16_t*)base)[idx]);
+    default:     return oracle_bf16_to_f64(((const uint16_t*)base)[idx]);
+  }
+}
+
+/* copy_blocks: apply the (src, dst) pairs in order; each pair duplicates the
+ * whole physical block src into dst, for the K cache and for the V cache. */
+int oracle_copy_blocks(uint8_t* k_cache, uint8_t* v_cache, const int32_t* pairs,
+                       int64_t num_pairs, int64_t num_blocks, int64_t block_bytes) {
+  if (num_pairs < 0 || block_bytes <= 0 || num_blocks <= 0) return OR_ERR_ARG;
+  if (num_pairs > 0 && (!k_cache || !v_cache || !pairs)) return OR_ERR_ARG;
+  for (int64_t p = 0; p < num_pairs; ++p) {
+    int64_t src = pairs[2 * p], dst = pairs[2 * p + 1];
+    if (src < 0 || src >= num_blocks || dst < 0 || dst >= num_blocks) return OR_ERR_RANGE;
+  }
+  for (int64_t p = 0; p < num_pairs; ++p) {
+    int64_t src = pairs[2 * p], dst = pairs[2 * p + 1];
+    memmove(k_cache + dst * block_bytes, k_cache + src * block_bytes, (size_t)block_bytes);
+    memmove(v_cache + dst * block_bytes, v_cache + src * block_bytes, (size_t)block_bytes);
+  }
+  return OR_OK;
+}
+
+/* reshape_and_cache: token t with slot s >= 0 goes to physical block s / block_size,
+ * position s % block_size, for every KV head.  k / v are [num_tokens, num_kv_heads,
+ * head_dim] with a row stride of token_stride elements between tokens. */
+int oracle_reshape_and_cache(const uint8_t* k, const uint8_t* v, uint8_t* k_cache,
+                             uint8_t* v_cache, const int64_t* slot_mapping,
+                             int64_t num_tokens, int num_kv_heads, int head_dim,
+                             int block_size, int64_t num_blocks, int elem_bytes,
+                             int64_t k_token_stride, int64_t v_token_stride) {
+  if (num_tokens < 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 ||
+      num_blocks <= 0 || elem_bytes <= 0)
+    return OR_ERR_ARG;
+  if (num_tokens > 0 && (!k || !v || !k_cache || !v_cache || !slot_mapping)) return OR_ERR_ARG;
+  for (int64_t t = 0; t < num_tokens; ++t) {
+    int64_t s = slot_mapping[t];
+    if (s >= num_blocks * block_size) return OR_ERR_RANGE;
+  }
+  const int64_t row = (int64_t)head_dim * elem_bytes;
+  for (int64_t t = 0; t < num_tokens; ++t) {
+    int64_t s = slot_mapping[t];
+    if (s < 0) continue;
+    int64_t blk = s / block_size, pos = s % block_size;
+    for (int h = 0; h < num_kv_heads; ++h) {
+      int64_t dst = ((blk * block_size + pos) * num_kv_heads + h) * row;
+      memcpy(k_cache + dst, k + (t * k_token_stride + (int64_t)h * head_dim) * elem_bytes, (size_t)row);
+      memcpy(v_cache + dst, v + (t * v_token_stride + (int64_t)h * head_dim) * elem_bytes, (size_t)row);
+    }
+  }
+  return OR_OK;
+}
+
+typedef struct {
+  double* out;
+  const void* q;
+  int q_dtype;
+  const void* k_cache;
+  const void* v_cache;
+  int kv_dtype;
+  const int32_t* block_tables;
+  const int32_t* seq_lens;
+  int num_q_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq;
+  double scale;
+  int seq_begin, seq_end;
+  int status;
+} decode_job;
+
+/* Offset (in elements) of element d of token t's KV row for kv head h, reached
+ * through the sequence's block table -- the index formula of the kernel on the
+ * "vLLM 深度解读" page, with the KV head in place of the query head. */
+static int64_t kv_offset(const int32_t* table, int t, int h, int d, int block_size,
+                         int num_kv_heads, int head_dim) {
+  int64_t phys = table[t / block_size];
+  return phys * block_size * num_kv_heads * head_dim + (int64_t)(t % block_size) * num_kv_heads * head_dim +
+         (int64_t)h * head_dim + d;
+}
+
+static void* decode_worker(void* arg) {
+  decode_job* J = (decode_job*)arg;
+  const int G = J->num_q_heads / J->num_kv_heads;
+  const int D = J->head_dim;
+  double* scores = NULL;
+  size_t cap = 0;
+  for (int i = J->seq_begin; i < J->seq_end; ++i) {
+    const int L = J->seq_lens[i];
+    const int32_t* table = J->block_tables + (int64_t)i * J->max_blocks_per_seq;
+    if ((size_t)L > cap) {
+      free(scores);
+      cap = (size_t)L;
+      scores = (double*)malloc(cap * sizeof(double));
+      if (!scores) { J->status = OR_ERR_NOMEM; return NULL; }
+    }
+    for (int hq = 0; hq < J->num_q_heads; ++hq) {
+      const int h = hq / G;                       /* KV head shared by this query head */
+      const int64_t qo = ((int64_t)i * J->num_q_heads + hq) * D;
+      double* o = J->out + qo;
+      for (int d = 0; d < D; ++d) o[d] = 0.0;
+      if (L == 0) continue;
+      /* pass 1: scores and their maximum */
+      double m = -INFINITY;
+      for (int t = 0; t < L; ++t) {
+        double s = 0.0;
+        for (int d = 0; d < D; ++d)
+          s += load_elem(J->q, qo + d, J->q_dtype) *
+               load_elem(J->k_cache, kv_offset(table, t, h, d, J->block_size, J->num_kv_heads, D), J->kv_dtype);
+        s *= J->scale;
+        scores[t] = s;
+        if (s > m) m = s;
+      }
+      /* pass 2: softmax weights and the weighted sum of V rows */
+      double z = 0.0;
+      for (int t = 0; t < L; ++t) {
+        double w = exp(scores[t] - m);
+        z += w;
+        for (int d = 0; d < D; ++d)
+          o[d] += w * load_elem(J->v_cache, kv_offset(table, t, h, d, J->block_size, J->num_kv_heads, D), J->kv_dtype);
+      }
+      for (int d = 0; d < D; ++d) o[d] /= z;
+    }
+  }
+  free(scores);
+  return NULL;
+}
+
+/* Decode attention: out[i, hq, :] = softmax_t(scale * q[i,hq,:] . K_t) V_t over the
+ * seq_lens[i] tokens of sequence i, K_t / V_t gathered through block_tables.
+ * out is fp64 [num_seqs, num_q_heads, head_dim].  Sequences are split across
+ * num_threads POSIX threads; each output element is computed by one thread in
+ * the same order whatever the thread count. */
+int oracle_decode(double* out, const void* q, int q_dtype, const void* k_cache,
+                  const void* v_cache, int kv_dtype, const int32_t* block_tables,
+                  const int32_t* seq_lens, int num_seqs, int num_q_heads, int num_kv_heads,
+                  int head_dim, int block_size, int max_blocks_per_seq, int64_t num_blocks,
+                  float scale, int num_threads) {
+  if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 ||
+      max_blocks_per_seq < 0 || num_blocks <= 0)
+    return OR_ERR_ARG;
+  if (num_q_heads % num_kv_heads) return OR_ERR_ARG;
+  if (q_dtype < OR_F32 || q_dtype > OR_BF16 || kv_dtype < OR_F32 || kv_dtype > OR_BF16) return OR_ERR_ARG;
+  if (num_seqs == 0) return OR_OK;
+  if (!out || !q || !k_cache || !v_cache || !block_tables || !seq_lens) return OR_ERR_ARG;
+  /* every block the definition will touch must exist */
+  for (int i = 0; i < num_seqs; ++i) {
+    int L = seq_lens[i];
+    if (L < 0 || (int64_t)L > (int64_t)max_blocks_per_seq * block_size) return OR_ERR_RANGE;
+    int nb = (L + block_size - 1) / block_size;
+    for (int b = 0; b < nb; ++b) {
+      int32_t p = block_tables[(int64_t)i * max_blocks_per_seq + b];
+      if (p < 0 || p >= num_blocks) return OR_ERR_RANGE;
+    }
+  }
+  if (num_threads < 1) num_threads = 1;
+  if (num_threads > num_seqs) num_threads = num_seqs;
+  decode_job* jobs = (decode_job*)calloc((size_t)num_threads, sizeof(decode_job));
+  pthread_t* tids = (pthread_t*)calloc((size_t)num_threads, sizeof(pthread_t));
+  if (!jobs || !tids) { free(jobs); free(tids); return OR_ERR_NOMEM; }
+  for (int w = 0; w < num_threads; ++w) {
+    decode_job* J = &jobs[w];
+    J->out = out; J->q = q; J->q_dtype = q_dtype; J->k_cache = k_cache; J->v_cache = v_cache;
+    J->kv_dtype = kv_dtype; J->block_tables = block_tables; J->seq_lens = seq_lens;
+    J->num_q_heads = num_q_heads; J->num_kv_heads = num_kv_heads; J->head_dim = head_dim;
+    J->block_size = block_size; J->max_blocks_per_seq = max_blocks_per_seq;
+    J->scale = (double)scale;
+    J->seq_begin = (int)((int64_t)num_seqs * w / num_threads);
+    J->seq_end = (int)((int64_t)num_seqs * (w + 1) / num_threads);
+    J->status = OR_OK;
+  }
+  int status = OR_OK;
+  int started = 0;
+  for (int w = 1; w < num_threads; ++w) {
+    if (pthread_create(&tids[w], NULL, decode_worker, &jobs[w]) != 0) break;
+    started = w;
+  }
+  decode_worker(&jobs[0]);
+  for (int w = 1; w <= started; ++w) pthread_join(tids[w], NULL);
+  /* any range not covered by a started thread runs here */
+  for (int w = started + 1; w < num_threads; ++w) decode_worker(&jobs[w]);
+  for (int w = 0; w < num_threads; ++w)
+    if (jobs[w].status != OR_OK) status = jobs[w].status;
+  free(jobs);
+  free(tids);
+  return status;
+}

@@ -1,0 +1,373 @@
+"""Seeded synthetic decode-step workloads shaped like the models on the vLLM pages.
+
+This module only builds inputs: sequence lengths, block tables (through the
+refcounted allocator in ``block_manager``), the pre-step paged K/V pool, the step's
+new K/V tokens with their slots, the copy-on-write pairs and the queries.  It holds
+none of the attention arithmetic and is shared, as the single input source, by the
+tests, the bench and the oracle-side checks.
+
+A decode step, as the Llama attention layer on "vLLM 深度解读" (section 7) orders it:
+  1. copy_blocks    -- duplicate every shared block that a sequence is about to
+                       write into (copy-on-write, "详解vLLM推理引擎架构", "Copy-on-Write");
+  2. reshape_and_cache -- store the step's new K/V tokens into their slots;
+  3. decode         -- attend with one query per sequence over seq_lens[i] tokens,
+                       the new ones included.
+
+Value recipe: every K, V and q element is drawn from N(0, 1) in float32 and rounded
+to nearest-even into the stored dtype (fp16 / bf16; fp32 q stays as drawn).  Pool
+positions that no sequence has written hold a NaN pattern, so any stray read of them
+poisons the output.  Each config draws from ``numpy.random.default_rng([seed, stream])``
+with seed = 3270 + config index and separate streams for lengths, placement, q,
+history K/V and new K/V, so logical values do not depend on the block size or the pool.
+"""
+from __future__ import annotations
+
+import concurrent.futures
+import dataclasses
+import math
+import os
+from typing import Dict, List, Optional, Sequence, Tuple
+
+import numpy as np
+
+from .block_manager import BlockAllocator, BlockTable, tables_to_array
+
+ELEM_BYTES = {"f32": 4, "f16": 2, "bf16": 2}
+NAN_BITS = {"f16": 0x7E00, "bf16": 0x7FC0}
+
+# random streams
+_S_LENS, _S_PLACE, _S_Q, _S_HIST, _S_NEW, _S_EXTRA = range(6)
+
+
+def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:
+    """Round float32 to bfloat16 (nearest, ties to even); returns the uint16 bit patterns."""
+    u = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32)
+    bias = ((u >> np.uint32(16)) & np.uint32(1)) + np.uint32(0x7FFF)
+    return ((u + bias) >> np.uint32(16)).astype(np.uint16)
+
+
+def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:
+    return (np.asarray(b, dtype=np.uint16).astype(np.uint32) << np.uint32(16)).view(np.float32)
+
+
+def to_storage(x: np.ndarray, dtype: str) -> np.ndarray:
+    """float32 values -> storage array (float32, or uint16 bit patterns for f16 / bf16)."""
+    if dtype == "f32":
+        return np.ascontiguousarray(x, dtype=np.float32)
+    if dtype == "f16":
+        return np.ascontiguousarray(x, dtype=np.float32).astype(np.float16).view(np.uint16)
+    if dtype == "bf16":
+        return f32_to_bf16_bits(x)
+    raise ValueError(f"unknown dtype {dtype!r}")
+
+
+def storage_to_f32(a: np.ndarray, dtype: str) -> np.ndarray:
+    if dtype == "f32":
+        return np.asarray(a, dtype=np.float32)
+    if dtype == "f16":
+        return np.asarray(a, dtype=np.uint16).view(np.float16).astype(np.float32)
+    if dtype == "bf16":
+        return bf16_bits_to_f32(a)
+    raise ValueError(f"unknown dtype {dtype!r}")
+
+
+_CHUNK = 1 << 22
+
+
+def _draw(key: Tuple[int, ...], shape, dtype: str) -> np.ndarray:
+    """N(0,1) values rounded into ``dtype`` storage, generated in fixed 4 Mi-element chunks.
+
+    Chunk c is drawn from default_rng(key + (c,)), so the values depend only on ``key``
+    and the element count, never on the thread count.
+    """
+    n = int(np.prod(shape, dtype=np.int64))
+    out = np.empty(n, dtype=np.float32 if dtype == "f32" else np.uint16)
+
+    def fill(c: int) -> None:
+        lo, hi = c * _CHUNK, min(n, (c + 1) * _CHUNK)
+        x = np.random.default_rng(list(key) + [c]).standard_normal(hi - lo, dtype=np.float32)
+        out[lo:hi] = to_storage(x, dtype)
+
+    chunks = range(-(-n // _CHUNK))
+    if n > _CHUNK:
+        with concurrent.futures.ThreadPoolExecutor(max_workers=min(16, os.cpu_count() or 1)) as ex:
+            list(ex.map(fill, chunks))
+    else:
+        for c in chunks:
+            fill(c)
+    return out.reshape(shape)
+
+
+@dataclasses.dataclass
+class Group:
+    """Sequences that share a prefix: member 0 owns the prefix, members 1.. fork from it.
+
+    prefix: tokens cached before the step (shared by every member).
+    step_tokens: tokens each member appends in this step (through reshape_and_cache).
+    """
+    prefix: int
+    step_tokens: List[int]
+
+
+@dataclasses.dataclass
+class Workload:
+    name: str
+    num_seqs: int
+    num_q_heads: int
+    num_kv_heads: int
+    head_dim: int
+    block_size: int
+    num_blocks: int
+    q_dtype: str
+    kv_dtype: str
+    scale: float                  # float32 value of 1/sqrt(head_dim)
+    q: np.ndarray                 # [N, Hq, D]
+    k_cache: np.ndarray           # [NB, bs, Hkv, D], state before the step
+    v_cache: np.ndarray
+    block_tables: np.ndarray      # int32 [N, MB], padded with -1
+    seq_lens: np.ndarray          # int32 [N], after the step
+    new_k: np.ndarray             # [T, Hkv, D]
+    new_v: np.ndarray
+    slot_mapping: np.ndarray      # int64 [T]
+    copy_pairs: np.ndarray        # int32 [P, 2]
+    notes: Dict[str, object] = dataclasses.field(default_factory=dict)
+
+    @property
+    def max_blocks_per_seq(self) -> int:
+        return int(self.block_tables.shape[1])
+
+    @property
+    def group_size(self) -> int:
+        return self.num_q_heads // self.num_kv_heads
+
+    @property
+    def kv_row_bytes(self) -> int:
+        """Bytes of one token's K (or V) row over all KV heads."""
+        return self.num_kv_heads * self.head_dim * ELEM_BYTES[self.kv_dtype]
+
+    @property
+    def block_bytes(self) -> int:
+        return self.block_size * self.kv_row_bytes
+
+    def total_tokens(self) -> int:
+        return int(self.seq_lens.astype(np.int64).sum())
+
+    def kv_bytes_logical(self) -> int:
+        """K+V bytes decode reads: each (token, KV head) of each sequence counted once."""
+        return 2 * self.total_tokens() * self.kv_row_bytes
+
+    def kv_bytes_unique(self) -> int:
+        """K+V bytes of distinct physical token slots reached by any sequence (shared blocks once)."""
+        used: Dict[int, int] = {}
+        bs = self.block_size
+        for i in range(self.num_seqs):
+            L = int(self.seq_lens[i])
+            nb = -(-L // bs)
+            for b in range(nb):
+                phys = int(self.block_tables[i, b])
+                n = min(bs, L - b * bs)
+                if used.get(phys, 0) < n:
+                    used[phys] = n
+        return 2 * sum(used.values()) * self.kv_row_bytes
+
+    def num_partitions(self, partition_size: int = 512) -> int:
+        L = self.seq_lens.astype(np.int64)
+        return int(((L + partition_size - 1) // partition_size).sum())
+
+    def io_bytes(self) -> Dict[str, int]:
+        """Algorithmic bytes of one decode call other than K/V."""
+        q_bytes = self.q.nbytes
+        return {"q": q_bytes, "block_tables": int(sum(-(-int(L) // self.block_size) for L in self.seq_lens)) * 4,
+                "seq_lens": self.num_seqs * 4}
+
+
+def build_groups(name: str, groups: Sequence[Group], *, num_q_heads: int, num_kv_heads: int,
+                 head_dim: int, block_size: int, q_dtype: str, kv_dtype: str, seed: int,
+                 pool_factor: float = 1.25, num_blocks: Optional[int] = None,
+                 notes: Optional[dict] = None) -> Workload:
+    """Materialise a decode step from groups of prefix-sharing sequences.
+
+    Sequence order is group by group, member by member.  The pool holds
+    ``num_blocks`` blocks, or ceil(pool_factor * blocks the step needs).
+    """
+    if num_q_heads % num_kv_heads:
+        raise ValueError("num_q_heads must be a multiple of num_kv_heads")
+    for g in groups:
+        if g.prefix < 0 or not g.step_tokens or min(g.step_tokens) < 0:
+            raise ValueError("bad group")
+    bs = block_size
+
+    def run(allocator: BlockAllocator):
+        tables: List[BlockTable] = []
+        prefix_slots: List[np.ndarray] = []
+        step_slots: List[List[np.ndarray]] = []
+        for g in groups:
+            parent = BlockTable(bs)
+            prefix_slots.append(parent.append_tokens(g.prefix, allocator))
+            members = [parent]
+            for _ in g.step_tokens[1:]:
+                child = BlockTable(bs)
+                child.fork_from(parent, allocator)
+                members.append(child)
+            step_slots.append([m.append_tokens(n, allocator) for m, n in zip(members, g.step_tokens)])
+            tables.extend(members)
+        return tables, prefix_slots, step_slots
+
+    # dry run on an identity-ordered pool large enough for anything: counts the blocks needed
+    upper = sum(-(-g.prefix // bs) + sum(-(-n // bs) + 1 for n in g.step_tokens) for g in groups) + 1
+    probe = BlockAllocator(upper, bs)
+    run(probe)
+    need = upper - probe.get_num_free_blocks()
+    if num_blocks is None:
+        num_blocks = max(1, int(math.ceil(pool_factor * need)))
+    if num_blocks < need:
+        raise ValueError(f"pool of {num_blocks} blocks is smaller than the {need} the step needs")
+
+    place_rng = np.random.default_rng([seed, _S_PLACE])
+    allocator = BlockAllocator(num_blocks, bs, rng=place_rng)
+    tables, prefix_slots, step_slots = run(allocator)
+    pairs = allocator.take_pending_copies()
+
+    N = len(tables)
+    Hkv, D = num_kv_heads, head_dim
+    q = _draw((seed, _S_Q), (N, num_q_heads, head_dim), q_dtype)
+
+    # history: every group's prefix tokens, in group order, K then V
+    nan = NAN_BITS[kv_dtype]
+    k_cache = np.full((num_blocks, bs, Hkv, D), nan, dtype=np.uint16)
+    v_cache = np.full((num_blocks, bs, Hkv, D), nan, dtype=np.uint16)
+    hist_slots = np.concatenate([np.zeros(0, np.int64)] + prefix_slots)
+    H = len(hist_slots)
+    if H:
+        k_cache.reshape(num_blocks * bs, Hkv, D)[hist_slots] = _draw((seed, _S_HIST, 0), (H, Hkv, D), kv_dtype)
+        v_cache.reshape(num_blocks * bs, Hkv, D)[hist_slots] = _draw((seed, _S_HIST, 1), (H, Hkv, D), kv_dtype)
+
+    all_slots = np.concatenate([np.zeros(0, np.int64)] +
+                               [s for per_group in step_slots for s in per_group]).astype(np.int64)
+    T = len(all_slots)
+    new_k = _draw((seed, _S_NEW, 0), (T, Hkv, D), kv_dtype)
+    new_v = _draw((seed, _S_NEW, 1), (T, Hkv, D), kv_dtype)
+
+    seq_lens = np.asarray([t.num_tokens for t in tables], dtype=np.int32)
+    block_tables = tables_to_array(tables)
+    info = {"groups": len(groups), "blocks_needed": int(need), "cow_pairs": int(len(pairs)),
+            "new_tokens": int(T), "pool_factor": pool_factor}
+    if notes:
+        info.update(notes)
+    return Workload(name=name, num_seqs=N, num_q_heads=num_q_heads, num_kv_heads=num_kv_heads,
+                    head_dim=head_dim, block_size=bs, num_blocks=num_blocks, q_dtype=q_dtype,
+                    kv_dtype=kv_dtype, scale=float(np.float32(1.0 / math.sqrt(head_dim))), q=q,
+                    k_cache=k_cache, v_cache=v_cache, block_tables=block_tables, seq_lens=seq_lens,
+                    new_k=new_k, new_v=new_v, slot_mapping=all_slots, copy_pairs=pairs, notes=info)
+
+
+def independent(name: str, seq_lens: Sequence[int], **kw) -> Workload:
+    """Each sequence on its own; seq_lens are post-step lengths, the last token stored in the step."""
+    groups = [Group(prefix=max(int(L) - 1, 0), step_tokens=[1 if L > 0 else 0]) for L in seq_lens]
+    return build_groups(name, groups, **kw)
+
+
+# ---------------------------------------------------------------------------------------
+# The five named decode configurations.
+# ---------------------------------------------------------------------------------------
+CONFIG_NAMES = ("tiny", "7b", "13b", "8b", "70b")
+CONFIG_INDEX = {n: i + 1 for i, n in enumerate(CONFIG_NAMES)}
+
+
+def config_seed(name: str) -> int:
+    return 3270 + CONFIG_INDEX[name]
+
+
+def _tiny(seed: int, block_size: int) -> Workload:
+    # 4 sequences, post-step lengths uniform in [1, 64]; sequence 3 is a fork of sequence 2
+    # (parallel sampling), so the step's first write into their shared partial block is the
+    # one copy-on-write pair.  Fixed pool of 64 blocks.
+    rng = np.random.default_rng([seed, _S_LENS])
+    L = [int(x) for x in rng.integers(1, 65, size=2)]
+    while True:
+        L2 = int(rng.integers(1, 65))
+        if (L2 - 1) % block_size != 0:
+            break
+    groups = [Group(L[0] - 1, [1]), Group(L[1] - 1, [1]), Group(L2 - 1, [1, 1])]
+    return build_groups("tiny", groups, num_q_heads=2, num_kv_heads=2, head_dim=64,
+                        block_size=block_size, q_dtype="f32", kv_dtype="f16", seed=seed,
+                        num_blocks=64, notes={"lens": "uniform[1,64]; seq 3 forks seq 2"})
+
+
+def _7b(seed: int, block_size: int, num_seqs: int = 64) -> Workload:
+    rng = np.random.default_rng([seed, _S_LENS])
+    L = rng.integers(128, 2049, size=num_seqs)
+    return independent("7b", L, num_q_heads=32, num_kv_heads=32, head_dim=128, block_size=block_size,
+                       q_dtype="bf16", kv_dtype="bf16", seed=seed,
+                       notes={"lens": "uniform[128,2048]"})
+
+
+def _13b(seed: int, block_size: int, num_seqs: int = 128) -> Workload:
+    rng = np.random.default_rng([seed, _S_LENS])
+    L = rng.integers(16, 2049, size=num_seqs)
+    return independent(f"13b-bs{block_size}", L, num_q_heads=40, num_kv_heads=40, head_dim=128,
+                       block_size=block_size, q_dtype="f16", kv_dtype="f16", seed=seed,
+                       notes={"lens": "uniform[16,2048]"})
+
+
+def lognormal_lengths(rng: np.random.Generator, n: int, median: float = 1024.0, sigma: float = 1.0,
+                      lo: int = 32, hi: int = 8192) -> np.ndarray:
+    z = rng.standard_normal(n)
+    return np.clip(np.rint(np.exp(math.log(median) + sigma * z)), lo, hi).astype(np.int64)
+
+
+def _8b(seed: int, block_size: int, num_seqs: int = 256) -> Workload:
+    rng = np.random.default_rng([seed, _S_LENS])
+    L = lognormal_lengths(rng, num_seqs)
+    return independent("8b", L, num_q_heads=32, num_kv_heads=8, head_dim=128, block_size=block_size,
+                       q_dtype="bf16", kv_dtype="bf16", seed=seed,
+                       notes={"lens": "lognormal(median 1024, sigma 1.0) clipped to [32, 8192]"})
+
+
+def _70b(seed: int, block_size: int, num_groups: int = 64, samples: int = 4,
+         prefix: int = 4096, long_len: int = 32768, num_long: int = 4) -> Workload:
+    # 64 groups x 4 samples.  Each group's parent holds prefix + r_g tokens, r_g uniform in
+    # [1, bs-1], so its last shared block is partial; the samples fork from it and each
+    # appends its own suffix (uniform in [1, 512] tokens) in the step: the first three
+    # writers into the shared partial block copy it, the fourth writes in place.  Four
+    # standalone 32768-token sequences ride in the same batch.
+    rng = np.random.default_rng([seed, _S_LENS])
+    groups = []
+    for _ in range(num_groups):
+        r = int(rng.integers(1, block_size))
+        suffix = [int(x) for x in rng.integers(1, 513, size=samples)]
+        groups.append(Group(prefix + r, suffix))
+    groups += [Group(long_len - 1, [1]) for _ in range(num_long)]
+    return build_groups("70b", groups, num_q_heads=64, num_kv_heads=8, head_dim=128,
+                        block_size=block_size, q_dtype="bf16", kv_dtype="bf16", seed=seed,
+                        notes={"lens": "64 groups x 4 samples: prefix 4096+r (r in [1,bs-1]) + "
+                                       "suffix uniform[1,512]; plus 4 x 32768"})
+
+
+_BUILDERS = {"tiny": _tiny, "7b": _7b, "13b": _13b, "8b": _8b, "70b": _70b}
+_DEFAULT_BS = {"tiny": 16, "7b": 16, "13b": 16, "8b": 16, "70b": 16}
+
+
+def make_config(name: str, block_size: Optional[int] = None, seed: Optional[int] = None,
+                **overrides) -> Workload:
+    """Build one of the named decode configs ("tiny", "7b", "13b", "8b", "70b")."""
+    if name not in _BUILDERS:
+        raise KeyError(f"unknown config {name!r}; choose from {CONFIG_NAMES}")
+    bs = block_size or _DEFAULT_BS[name]
+    return _BUILDERS[name](config_seed(name) if seed is None else seed, bs, **overrides)
+
+
+def apply_step_host(w: Workload) -> Tuple[np.ndarray, np.ndarray]:
+    """The post-step caches computed with plain numpy indexing (no kernel, no oracle).
+
+    Used only to give tests an independent expectation of the cache state.
+    """
+    kc, vc = w.k_cache.copy(), w.v_cache.copy()
+    for s, d in w.copy_pairs:
+        kc[d] = kc[s]
+        vc[d] = vc[s]
+    NB, bs, Hkv, D = kc.shape
+    keep = w.slot_mapping >= 0
+    kc.reshape(NB * bs, Hkv, D)[w.slot_mapping[keep]] = w.new_k[keep]
+    vc.reshape(NB * bs, Hkv, D)[w.slot_mapping[keep]] = w.new_v[keep]
+    return kc, vc

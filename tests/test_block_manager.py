@@ -1,0 +1,167 @@
+"""Host block manager and workload generator (CPU only).
+
+Pins: ceil(num_tokens / block_size) blocks per table and the exhausted-pool error
+("vLLM 深度解读", section 2); fork shares blocks and copy-on-write copies only a
+block whose refcount exceeds 1, then drops one reference from it ("详解vLLM推理引擎架构",
+"Copy-on-Write 与内存共享"); the seeded free list gives a shuffled placement.
+"""
+import numpy as np
+import pytest
+
+from paged_kv_cache_327_b200 import workload as W
+from paged_kv_cache_327_b200.block_manager import (BlockAllocator, BlockTable, NoFreeBlocksError,
+                                                   tables_to_array)
+
+
+def test_required_blocks_is_ceil():
+    t = BlockTable(16)
+    assert [t.get_num_required_blocks(n) for n in (0, 1, 15, 16, 17, 32, 33)] == [0, 1, 1, 1, 2, 2, 3]
+    t32 = BlockTable(32)
+    assert t32.get_num_required_blocks(33) == 2
+
+
+def test_allocator_exhaustion_raises_and_free_returns():
+    a = BlockAllocator(3, 16, seed=1)
+    got = [a.allocate() for _ in range(3)]
+    assert sorted(got) == [0, 1, 2]
+    with pytest.raises(NoFreeBlocksError):
+        a.allocate()
+    a.free(got[1])
+    assert a.get_num_free_blocks() == 1
+    assert a.allocate() == got[1]
+
+
+def test_seeded_placement_is_shuffled_and_reproducible():
+    a = [BlockAllocator(64, 16, seed=7).allocate() for _ in range(1)]
+    b1 = BlockAllocator(64, 16, seed=7)
+    b2 = BlockAllocator(64, 16, seed=7)
+    s1 = [b1.allocate() for _ in range(64)]
+    s2 = [b2.allocate() for _ in range(64)]
+    assert s1 == s2 and sorted(s1) == list(range(64)) and s1 != list(range(64))
+    assert a[0] == s1[0]
+
+
+def test_append_slots_allocates_when_block_full():
+    a = BlockAllocator(10, 4, seed=None)
+    t = BlockTable(4)
+    slots = t.append_tokens(9, a)
+    assert len(t) == 3 and t.num_tokens == 9
+    blocks = t.get_physical_blocks()
+    assert list(slots) == [blocks[j // 4] * 4 + j % 4 for j in range(9)]
+    # token-at-a-time gives the same slots
+    a2 = BlockAllocator(10, 4, seed=None)
+    t2 = BlockTable(4)
+    assert [t2.append_token(a2) for _ in range(9)] == list(slots)
+
+
+def test_fork_and_copy_on_write_counts():
+    a = BlockAllocator(16, 4, seed=3)
+    parent = BlockTable(4)
+    parent.append_tokens(6, a)                      # 2 blocks, last one half full
+    kids = []
+    for _ in range(3):
+        c = BlockTable(4)
+        c.fork_from(parent, a)
+        kids.append(c)
+    last = parent.get_block_number(1)
+    assert a.get_refcount(last) == 4 and a.get_refcount(parent.get_block_number(0)) == 4
+    # writers 1..3 copy (refcount 4 -> 3 -> 2 -> 1), the last one writes in place
+    for t in [parent] + kids:
+        t.append_token(a)
+    pairs = a.take_pending_copies()
+    assert len(pairs) == 3 and all(p[0] == last for p in pairs)
+    assert len({int(p[1]) for p in pairs}) == 3 and last not in {int(p[1]) for p in pairs}
+    assert a.get_refcount(last) == 1
+    assert kids[-1].get_block_number(1) == last
+    # the full first block stays shared
+    assert a.get_refcount(parent.get_block_number(0)) == 4
+
+
+def test_write_to_unshared_block_copies_nothing():
+    a = BlockAllocator(4, 4, seed=0)
+    t = BlockTable(4)
+    t.append_tokens(2, a)
+    t.write_to_block(0, a)
+    assert len(a.take_pending_copies()) == 0
+
+
+def test_refcount_underflow_raises():
+    a = BlockAllocator(2, 4)
+    b = a.allocate()
+    a.free(b)
+    with pytest.raises(ValueError):
+        a.free(b)
+
+
+def test_tables_to_array_pads():
+    a = BlockAllocator(8, 4, seed=2)
+    t1, t2 = BlockTable(4), BlockTable(4)
+    t1.append_tokens(9, a)
+    t2.append_tokens(1, a)
+    arr = tables_to_array([t1, t2])
+    assert arr.shape == (2, 3) and arr.dtype == np.int32 and list(arr[1, 1:]) == [-1, -1]
+
+
+def test_tiny_config_has_one_cow_pair_and_poisoned_pool():
+    w = W.make_config("tiny")
+    assert w.num_seqs == 4 and w.num_blocks == 64 and len(w.copy_pairs) == 1
+    assert w.q.dtype == np.float32 and w.kv_dtype == "f16"
+    assert all(1 <= L <= 64 for L in w.seq_lens)
+    assert w.seq_lens[2] == w.seq_lens[3]
+    # the CoW destination is unwritten (NaN) before the step
+    dst = int(w.copy_pairs[0, 1])
+    assert np.all(w.k_cache[dst] == W.NAN_BITS["f16"])
+    # after copy + store, every position a sequence reads is finite
+    kc, vc = W.apply_step_host(w)
+    for i in range(w.num_seqs):
+        L = int(w.seq_lens[i])
+        for j in range(L):
+            phys = w.block_tables[i, j // 16]
+            assert np.all(np.isfinite(W.storage_to_f32(kc[phys, j % 16], "f16")))
+
+
+def test_workload_draws_do_not_depend_on_block_size():
+    a = W.independent("x", [40, 3, 77], num_q_heads=4, num_kv_heads=2, head_dim=64, block_size=16,
+                      q_dtype="bf16", kv_dtype="bf16", seed=9)
+    b = W.independent("x", [40, 3, 77], num_q_heads=4, num_kv_heads=2, head_dim=64, block_size=32,
+                      q_dtype="bf16", kv_dtype="bf16", seed=9)
+    assert np.array_equal(a.q, b.q) and np.array_equal(a.new_k, b.new_k)
+    for w in (a, b):
+        kc, _ = W.apply_step_host(w)
+        flat = kc.reshape(-1, 2, 64)
+        w.__dict__["_logical"] = np.concatenate(
+            [flat[w.block_tables[i, np.arange(L) // w.block_size] * w.block_size + np.arange(L) % w.block_size]
+             for i, L in enumerate(w.seq_lens)])
+    assert np.array_equal(a._logical, b._logical)
+
+
+def test_bf16_rounding_is_nearest_even():
+    x = np.array([1.0, 1.0 + 2**-8, 1.0 + 3 * 2**-8, 1.0 + 2**-9, -2.5, 3.0e-39], np.float32)
+    got = W.bf16_bits_to_f32(W.f32_to_bf16_bits(x))
+    import torch
+    ref = torch.from_numpy(x).to(torch.bfloat16).float().numpy()
+    assert np.array_equal(got, ref)
+
+
+@pytest.mark.parametrize("name", ["7b", "13b", "8b", "70b"])
+def test_named_config_shapes(name):
+    w = W.make_config(name)
+    G = {"7b": 1, "13b": 1, "8b": 4, "70b": 8}[name]
+    assert w.group_size == G and w.head_dim == 128
+    L = w.seq_lens
+    if name == "7b":
+        assert w.num_seqs == 64 and L.min() >= 128 and L.max() <= 2048
+    if name == "13b":
+        assert w.num_seqs == 128 and L.min() >= 16 and L.max() <= 2048
+    if name == "8b":
+        assert w.num_seqs == 256 and L.min() >= 32 and L.max() <= 8192
+        assert 700 < np.median(L) < 1400
+    if name == "70b":
+        assert w.num_seqs == 260 and len(w.copy_pairs) == 192
+        assert sorted(L)[-4:] == [32768] * 4
+        assert w.kv_bytes_unique() < w.kv_bytes_logical() / 2
+    assert w.num_blocks >= int(np.ceil(1.25 * w.notes["blocks_needed"]))
+    # no block is referenced by two different sequences unless it is a shared prefix block
+    if name != "70b":
+        used = np.concatenate([w.block_tables[i, :-(-int(l) // w.block_size)] for i, l in enumerate(L)])
+        assert len(np.unique(used)) == len(used)
