@@ -1,0 +1,410 @@
+#!/usr/bin/env python
+"""Paged decode attention throughput on B200.
+
+One step = the whole hot path over one batch: copy_blocks (copy-on-write pairs, when the
+workload has any) -> reshape_and_cache (the step's new tokens) -> pa_decode.  The default
+workload is the Llama-3-8B-shaped GQA decode: 256 sequences, 32 query / 8 KV heads,
+head_dim 128, block size 16, lognormal lengths (median 1024, sigma 1) clipped to
+[32, 8192], bf16, shuffled physical placement, 512-token split-K partitions.
+
+value      = decode K+V bytes (each token's K and V rows of each KV head, once) / step time
+e2e        = the same bytes / time of a step whose inputs start in pinned host memory
+             (H2D of q, new K/V, slots, block tables, lengths, pairs) and whose output is
+             read back to the host, all through the C ABI
+roofline   = pa_decode alone: algorithmic bytes (K+V + q + out + block tables + lengths)
+             per call / its mean CUDA-event duration inside the timed loop, vs the
+             measured HBM copy bandwidth
+cpu_baseline / --impl reference = the fp64 C oracle on the host cores, on a bounded
+             sample of the same workload
+
+Multi-GPU (torchrun): every rank runs its own batch (seeded by rank) on its own GPU, no
+collective on the data path ("replicas", weak scaling); the time is the max over ranks.
+"""
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from paged_kv_cache_327_b200 import workload as W  # noqa: E402
+
+METRIC = "paged decode attention KV GB/s (% of HBM peak); seq-tokens/s, 8B-GQA decode"
+KERNEL_SOURCES = ["paged_kv_cache_327_b200/csrc/pa_decode.cuh", "paged_kv_cache_327_b200/csrc/pa_ptx.cuh",
+                  "paged_kv_cache_327_b200/csrc/pa_api.cu"]
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse_args():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=3000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", default="8b", choices=list(W.CONFIG_NAMES))
+    ap.add_argument("--block-size", type=int, default=None)
+    ap.add_argument("--partition-size", type=int, default=0)
+    ap.add_argument("--out-dtype", default=None, help="f32 | f16 | bf16 (default: the query dtype)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target oracle time for cpu_baseline")
+    ap.add_argument("--ref-seconds", type=float, default=150.0, help="target total time of --impl reference")
+    return ap.parse_args()
+
+
+def workload_label(w: W.Workload) -> str:
+    return (f"{w.name}: {w.num_seqs} seqs, {w.num_q_heads}/{w.num_kv_heads} heads, head_dim {w.head_dim}, "
+            f"block {w.block_size}, {w.notes.get('lens', '')}, q {w.q_dtype}, kv {w.kv_dtype}")
+
+
+def measured_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured (MEASURED_PEAKS.json hbm_gbs)"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback 6.65 TB/s (no MEASURED_PEAKS.json)"
+
+
+def sources_digest():
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(config: str):
+    """dram bytes per pa_decode partition-kernel launch from the committed ncu summary, if it was
+    taken on the current kernel sources (otherwise None)."""
+    path = os.path.join(ROOT, "profiles", f"pa_decode_partition_{config}.md")
+    if not os.path.exists(path):
+        return None
+    vals = {}
+    for line in open(path, encoding="utf-8"):
+        if line.startswith("traffic_bytes_per_launch:") or line.startswith("kernel_sources_sha256_16:"):
+            k, v = line.split(":", 1)
+            vals[k.strip()] = v.strip()
+    if vals.get("kernel_sources_sha256_16") != sources_digest():
+        return None
+    try:
+        return int(float(vals["traffic_bytes_per_launch"]))
+    except (KeyError, ValueError):
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons every 200 ms while it runs."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.path = None
+        self.t_window = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200",
+                 "-i", str(self.dev)], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def mark(self, t0, t1):
+        self.t_window = (t0, t1)
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((float(parts[1]), float(parts[2]), float(parts[3]), parts[5:9]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        loaded = [r for r in rows if r[2] > 0.5 * max(x[2] for x in rows)] or rows
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in loaded for i, v in enumerate(r[3]) if v.lower().startswith("active")})
+        return {"sm_mhz": statistics.median(r[0] for r in loaded), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": reasons, "samples": len(loaded)}
+
+
+def oracle_sample_rate(w: W.Workload, seconds: float, start: int = 0):
+    """Time the fp64 oracle on consecutive sequences (from `start`, wrapping) until ~`seconds` of work.
+
+    Returns (KV bytes processed, seconds, threads, sequence count)."""
+    import oracle
+
+    threads = oracle.default_threads()
+    kc, vc = W.apply_step_host(w)
+    row = 2 * w.kv_row_bytes
+    order = [(start + i) % w.num_seqs for i in range(w.num_seqs)]
+    # pilot: one sequence of median length to size the sample
+    med = int(np.argsort(w.seq_lens)[w.num_seqs // 2])
+    t = time.perf_counter()
+    oracle.decode(np.ascontiguousarray(w.q[[med]]), w.q_dtype, kc, vc, w.kv_dtype,
+                  np.ascontiguousarray(w.block_tables[[med]]), w.seq_lens[[med]], w.scale, num_threads=1)
+    per_token = (time.perf_counter() - t) / max(1, int(w.seq_lens[med]))
+    budget_tokens = seconds * threads / max(per_token, 1e-12)
+    pick, tok = [], 0
+    for i in order:
+        if tok >= budget_tokens and pick:
+            break
+        pick.append(i)
+        tok += int(w.seq_lens[i])
+    idx = np.asarray(pick)
+    t = time.perf_counter()
+    oracle.decode(np.ascontiguousarray(w.q[idx]), w.q_dtype, kc, vc, w.kv_dtype,
+                  np.ascontiguousarray(w.block_tables[idx]), np.ascontiguousarray(w.seq_lens[idx]), w.scale,
+                  num_threads=threads)
+    dt = time.perf_counter() - t
+    return tok * row, dt, threads, len(idx)
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    w = W.make_config(args.config, block_size=args.block_size)
+    per_step = max(0.5, args.ref_seconds / max(1, args.steps + args.warmup))
+    start = 0
+    for _ in range(args.warmup):
+        _, _, _, n = oracle_sample_rate(w, per_step, start)
+        start += n
+    total_b, total_t, threads, seqs = 0, 0.0, 1, 0
+    for _ in range(args.steps):
+        b, t, threads, n = oracle_sample_rate(w, per_step, start)
+        start += n
+        total_b += b
+        total_t += t
+        seqs += n
+    value = total_b / total_t / 1e9
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * total_t / args.steps, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": workload_label(w)},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
+                         "sample": f"{seqs} sequences over {args.steps} steps (consecutive windows of the batch), "
+                                   f"fp64 two-pass softmax, decode only"},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours(args):
+    from paged_kv_cache_327_b200 import binding as B
+    from paged_kv_cache_327_b200 import build as pkg_build
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        print(f"warning: --gpus {args.gpus} but WORLD_SIZE {world}", file=sys.stderr)
+    pkg_build.build()
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+
+    seed = W.config_seed(args.config) + 1000 * rank
+    w = W.make_config(args.config, block_size=args.block_size, seed=seed)
+    out_dtype = args.out_dtype or w.q_dtype
+    dw = B.device_workload(w, f"cuda:{local}")
+    ws = B.DecodeWorkspace.for_workload(dw, args.partition_size)
+    out = torch.empty((w.num_seqs, w.num_q_heads, w.head_dim), dtype=B._NAME_TORCH[out_dtype], device="cuda")
+    stream = torch.cuda.current_stream()
+
+    kv_bytes = w.kv_bytes_logical()
+    io = w.io_bytes()
+    out_bytes = out.numel() * out.element_size()
+    decode_bytes = kv_bytes + io["q"] + io["block_tables"] + io["seq_lens"] + out_bytes
+    launches_per_step = (1 if len(w.copy_pairs) else 0) + (1 if len(w.slot_mapping) else 0) + 3
+
+    def step():
+        B.run_step(dw, out, ws, args.partition_size, stream)
+
+    # ---- warm-up (also checks the device error word once)
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    if B.pa_get_device_error() != B.PA_DEV_OK:
+        raise RuntimeError("device error during warm-up")
+
+    clocks = ClockSampler(torch.cuda.current_device()) if rank == 0 else None
+    if clocks:
+        clocks.start()
+        time.sleep(0.5)
+    # ---- timed region: K steps, events around every decode call
+    ev_dec = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    wall0 = time.time()
+    t_start.record(stream)
+    for i in range(args.steps):
+        if len(w.copy_pairs):
+            B.pa_copy_blocks(dw.k_cache, dw.v_cache, dw.copy_pairs, stream=stream)
+        if len(w.slot_mapping):
+            B.pa_reshape_and_cache(dw.new_k, dw.new_v, dw.k_cache, dw.v_cache, dw.slot_mapping, stream=stream)
+        ev_dec[i][0].record(stream)
+        B.pa_decode(out, dw.q, dw.k_cache, dw.v_cache, dw.block_tables, dw.seq_lens, w.scale, ws.tensor,
+                    args.partition_size, stream)
+        ev_dec[i][1].record(stream)
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    wall1 = time.time()
+    if dist:
+        dist.barrier()
+    elapsed_ms = t_start.elapsed_time(t_end)
+    dec_ms = [a.elapsed_time(b) for a, b in ev_dec]
+    if clocks:
+        clocks.mark(wall0, wall1)
+    if dist:
+        t = torch.tensor([elapsed_ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms = float(t.item())
+    if B.pa_get_device_error() != B.PA_DEV_OK:
+        raise RuntimeError("device error during the timed region")
+
+    # ---- e2e: inputs from pinned host memory, result back to the host, every step
+    host = {
+        "q": B.from_torch(dw.q), "new_k": B.from_torch(dw.new_k), "new_v": B.from_torch(dw.new_v),
+    }
+    pin = lambda t: t.cpu().pin_memory()
+    h_q, h_k, h_v = pin(dw.q), pin(dw.new_k), pin(dw.new_v)
+    h_slots, h_bt, h_sl, h_pairs = pin(dw.slot_mapping), pin(dw.block_tables), pin(dw.seq_lens), pin(dw.copy_pairs)
+    h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in (h_q, h_k, h_v, h_slots, h_bt, h_sl, h_pairs))
+    d2h = h_out.numel() * h_out.element_size()
+    del host
+    e2e_steps = max(1, min(args.steps, 500))
+
+    def e2e_step():
+        dw.q.copy_(h_q, non_blocking=True)
+        dw.new_k.copy_(h_k, non_blocking=True)
+        dw.new_v.copy_(h_v, non_blocking=True)
+        dw.slot_mapping.copy_(h_slots, non_blocking=True)
+        dw.block_tables.copy_(h_bt, non_blocking=True)
+        dw.seq_lens.copy_(h_sl, non_blocking=True)
+        dw.copy_pairs.copy_(h_pairs, non_blocking=True)
+        step()
+        h_out.copy_(out, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    if dist:
+        t = torch.tensor([e2e_ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+
+    clock_info = clocks.stop() if clocks else None
+
+    # ---- L2-flushed decode timing (outside the timed region; a cross-check of the roofline)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    flushed = []
+    for _ in range(10):
+        flush.fill_(1)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        B.pa_decode(out, dw.q, dw.k_cache, dw.v_cache, dw.block_tables, dw.seq_lens, w.scale, ws.tensor,
+                    args.partition_size, stream)
+        b.record(stream)
+        torch.cuda.synchronize()
+        flushed.append(a.elapsed_time(b))
+    del flush
+
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+
+    ms_step = elapsed_ms / args.steps
+    value = world * kv_bytes / (ms_step * 1e-3) / 1e9
+    peak, peak_src = measured_peak()
+    dec_mean = float(np.mean(dec_ms))
+    achieved = decode_bytes / (dec_mean * 1e-3) / 1e9
+    cpu = None
+    if not args.no_cpu_baseline and world == 1:
+        b, t, threads, n = oracle_sample_rate(w, args.cpu_seconds)
+        cpu = {"value": round(b / t / 1e9, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
+               "sample": f"first {n} of {w.num_seqs} sequences ({b / 1e9:.3f} GB of K+V), decode only, "
+                         f"fp64 two-pass softmax, {t:.1f} s"}
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_step, 5), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": w.kv_dtype, "data": "synthetic",
+        "config": {"workload": workload_label(w), "kv_bytes_per_step": kv_bytes,
+                   "seq_tokens_per_step": w.total_tokens(), "new_tokens_per_step": int(len(w.slot_mapping)),
+                   "cow_pairs_per_step": int(len(w.copy_pairs)), "out_dtype": out_dtype,
+                   "partition_size": args.partition_size or 512,
+                   "l2": f"inputs larger than L2 (K+V {kv_bytes / 1e9:.2f} GB vs 126 MB L2); no flush in the "
+                         f"timed loop", "parallelism": f"replicas x{world}" if world > 1 else "1 GPU"},
+        "seq_tokens_per_s": round(world * w.total_tokens() / (ms_step * 1e-3), 1),
+        "pct_of_hbm_peak": round(100 * value / world / peak, 2),
+        "e2e": {"value": round(world * kv_bytes / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 5)},
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4), "traffic": recorded_traffic(args.config),
+                     "kernel": "pa_decode call (plan + partition + reduce kernels)",
+                     "algorithmic_bytes_per_launch": decode_bytes, "launch_ms_mean": round(dec_mean, 5),
+                     "launch_ms_l2_flushed_median": round(float(np.median(flushed)), 5),
+                     "peak_source": peak_src},
+        "cpu_baseline": cpu,
+        "clocks": clock_info,
+        "gpu_launches": launches_per_step * args.steps,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,142 @@
+/*
+ * pa.h -- C ABI of libpa.so: paged KV-cache decode attention for NVIDIA B200 (sm_100a).
+ *
+ * The operations come from web pages describing vLLM's PagedAttention:
+ *   - "详解vLLM推理引擎架构" (tbr8.org), "PagedAttention 的核心思想": the KV cache is
+ *     cut into fixed-size blocks of 16 or 32 tokens scattered over a physical pool and
+ *     reached through a per-sequence block table; "Copy-on-Write 与内存共享": a shared
+ *     block is copied before it is written.
+ *   - "vLLM 深度解读" (luoboask.github.io), section 3 ("PagedAttention CUDA Kernel"):
+ *     the cache and query layouts and the per-token score / softmax / weighted sum;
+ *     section 7 (Llama attention): new K/V are stored into the cache, then attention
+ *     runs over the context including them.
+ *
+ * Conventions shared by every entry point
+ *   - Every pointer argument is a DEVICE pointer unless its name starts with host_.
+ *     The caller owns all memory (including the decode workspace); the library never
+ *     allocates device memory and keeps no per-call state.
+ *   - Tensors are dense and row-major (C order) unless a stride argument says otherwise.
+ *   - Element types are pa_dtype values.  Caches and the decode query must start on a
+ *     16-byte boundary.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default stream)
+ *     and never synchronise.  Arguments are validated on the host first: an invalid
+ *     call returns a negative pa_status and launches nothing.  PA_ERR_CUDA reports a
+ *     launch failure (the CUDA error is left for cudaGetLastError()).
+ *   - Data-dependent faults found by the kernels (a block id, slot or pair outside the
+ *     pool, a sequence longer than its table) never touch memory out of range: the
+ *     offending access is skipped, the affected outputs are NaN, and the first such
+ *     fault is recorded in a process-wide device error word that pa_get_device_error()
+ *     returns.  A wait that exceeds its bound records PA_DEV_TIMEOUT the same way.
+ */
+#ifndef PA_H_
+#define PA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define PA_API __attribute__((visibility("default")))
+#else
+#define PA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum { PA_F32 = 0, PA_F16 = 1, PA_BF16 = 2 } pa_dtype;
+
+typedef enum {
+  PA_OK = 0,
+  PA_ERR_INVALID = -1,     /* null pointer, bad size, misaligned pointer */
+  PA_ERR_UNSUPPORTED = -2, /* valid but not implemented: head_dim, block_size, dtype mix, group size */
+  PA_ERR_WORKSPACE = -3,   /* workspace missing or smaller than pa_decode_workspace_size() */
+  PA_ERR_CUDA = -4         /* a CUDA runtime call or kernel launch failed */
+} pa_status;
+
+/* codes returned by pa_get_device_error() */
+typedef enum {
+  PA_DEV_OK = 0,
+  PA_DEV_BAD_BLOCK_ID = 1, /* a block-table entry a sequence needs is outside [0, num_blocks) */
+  PA_DEV_BAD_SEQ_LEN = 2,  /* seq_lens[i] < 0 or > max_blocks_per_seq * block_size */
+  PA_DEV_BAD_SLOT = 3,     /* slot_mapping[t] >= num_blocks * block_size */
+  PA_DEV_BAD_PAIR = 4,     /* a copy_blocks pair names a block outside [0, num_blocks) */
+  PA_DEV_TIMEOUT = 5       /* a bounded wait on an asynchronous copy gave up */
+} pa_device_error;
+
+/* Bytes of device workspace pa_decode needs, an upper bound valid for any seq_lens whose
+ * entries are all <= max_seq_len.  pa_decode itself requires the bound for
+ * max_seq_len = max_blocks_per_seq * block_size.  partition_size 0 means the default (512).
+ * Returns 0 for invalid arguments. */
+PA_API size_t pa_decode_workspace_size(int num_seqs, int num_q_heads, int head_dim, int max_seq_len,
+                                int partition_size);
+
+/* Paged decode attention ("vLLM 深度解读", section 3; grouped-query reading: query head hq
+ * uses KV head hq / (num_q_heads / num_kv_heads)).  For every sequence i and query head hq:
+ *   out[i, hq, :] = sum_t softmax_t(scale * q[i, hq, :] . K_t) * V_t,  t < seq_lens[i],
+ * where token t lives in physical block block_tables[i, t / block_size], position
+ * t % block_size, and K_t = k_cache[phys, t % block_size, hq / G, :] (V_t likewise).
+ *   out          [num_seqs, num_q_heads, head_dim], out_dtype (f32, f16 or bf16)
+ *   q            [num_seqs, num_q_heads, head_dim], q_dtype == kv_dtype or f32
+ *   k_cache, v_cache  [num_blocks, block_size, num_kv_heads, head_dim], kv_dtype (f16 or bf16)
+ *   block_tables int32 [num_seqs, max_blocks_per_seq]; entries past a sequence's
+ *                ceil(seq_lens[i] / block_size) blocks are never read
+ *   seq_lens     int32 [num_seqs]; 0 gives an all-zero output row
+ *   supported: head_dim 64 or 128, block_size 16 or 32, G = num_q_heads / num_kv_heads
+ *   from 1 to 8.  partition_size (0 = 512) must be a multiple of block_size and at
+ *   most 32 * block_size: sequences longer than one partition are split into
+ *   partitions whose partial softmax states are merged by a second kernel
+ *   (deterministic: the split depends only on seq_lens[i]).
+ *   workspace    device scratch of >= pa_decode_workspace_size(num_seqs, num_q_heads,
+ *                head_dim, max_blocks_per_seq * block_size, partition_size) bytes, 256-byte
+ *                aligned; its contents need no initialisation and are overwritten. */
+PA_API int pa_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
+              const int32_t* block_tables, const int32_t* seq_lens, int num_seqs,
+              int num_q_heads, int num_kv_heads, int head_dim, int block_size, float scale,
+              int max_blocks_per_seq, int64_t num_blocks, int q_dtype, int kv_dtype,
+              int out_dtype, int partition_size, void* workspace, size_t workspace_bytes,
+              void* stream);
+
+/* Store the step's new tokens into the paged cache ("vLLM 深度解读", section 7).
+ * For each token t with slot = slot_mapping[t] >= 0:
+ *   k_cache[slot / block_size, slot % block_size, h, :] = k[t, h, :]  for every KV head h
+ * (and v likewise); a negative slot skips the token.
+ *   k, v          [num_tokens, num_kv_heads, head_dim] rows, kv_dtype, token t at element
+ *                 offset t * k_token_stride (v_token_stride for v); 0 = num_kv_heads * head_dim
+ *   slot_mapping  int64 [num_tokens]
+ * Slots must be distinct (two tokens on one slot race).  Bit-exact byte copies. */
+PA_API int pa_reshape_and_cache(const void* k, const void* v, void* k_cache, void* v_cache,
+                         const int64_t* slot_mapping, int num_tokens, int num_kv_heads,
+                         int head_dim, int block_size, int64_t num_blocks, int kv_dtype,
+                         int64_t k_token_stride, int64_t v_token_stride, void* stream);
+
+/* Copy-on-write block duplication ("详解vLLM推理引擎架构", "Copy-on-Write 与内存共享"):
+ * for each pair p, physical block src_dst_pairs[p][0] of k_cache is copied over block
+ * src_dst_pairs[p][1] (and the same for v_cache), block_bytes bytes each
+ * (= block_size * num_kv_heads * head_dim * element size, a multiple of 16).
+ *   src_dst_pairs  int32 [num_pairs, 2], device
+ *   host_pairs     optional host copy of the same pairs: when given, the call checks that
+ *                  every id is in range, that no destination repeats and that no
+ *                  destination is also a source (so the result does not depend on the
+ *                  order the copies run in), returning PA_ERR_INVALID otherwise.  When
+ *                  NULL those preconditions are the caller's; out-of-range ids are still
+ *                  skipped and reported through pa_get_device_error(). */
+PA_API int pa_copy_blocks(void* k_cache, void* v_cache, const int32_t* src_dst_pairs, int num_pairs,
+                   int64_t num_blocks, size_t block_bytes, const int32_t* host_pairs,
+                   void* stream);
+
+/* Static description of a pa_status value. */
+PA_API const char* pa_strerror(int status);
+
+/* Synchronises `stream`, returns the first pa_device_error recorded on the current device
+ * since the last call (or a negative pa_status if reading it failed) and clears it. */
+PA_API int pa_get_device_error(void* stream);
+
+/* ABI version of this header (major * 100 + minor). */
+PA_API int pa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PA_H_ */

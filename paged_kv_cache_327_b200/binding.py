@@ -1,0 +1,215 @@
+"""ctypes binding of libpa.so (include/pa.h), with the ABI's own names.
+
+Argument marshalling only: torch tensors are turned into device pointers, sizes and
+pa_dtype codes, and every computation happens in the library's CUDA kernels.  Loading
+fails loudly (ImportError) when libpa.so has not been built; there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import dataclasses
+import os
+from typing import Optional
+
+import numpy as np
+import torch
+
+from . import workload as W
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libpa.so")
+
+PA_F32, PA_F16, PA_BF16 = 0, 1, 2
+PA_OK, PA_ERR_INVALID, PA_ERR_UNSUPPORTED, PA_ERR_WORKSPACE, PA_ERR_CUDA = 0, -1, -2, -3, -4
+PA_DEV_OK, PA_DEV_BAD_BLOCK_ID, PA_DEV_BAD_SEQ_LEN, PA_DEV_BAD_SLOT, PA_DEV_BAD_PAIR, PA_DEV_TIMEOUT = range(6)
+
+EXPORTED = ("pa_decode_workspace_size", "pa_decode", "pa_reshape_and_cache", "pa_copy_blocks",
+            "pa_strerror", "pa_get_device_error", "pa_version")
+
+_TORCH_CODE = {torch.float32: PA_F32, torch.float16: PA_F16, torch.bfloat16: PA_BF16}
+_NAME_CODE = {"f32": PA_F32, "f16": PA_F16, "bf16": PA_BF16}
+_NAME_TORCH = {"f32": torch.float32, "f16": torch.float16, "bf16": torch.bfloat16}
+
+_lib = None
+
+
+def load_library(path: str = _LIB_PATH):
+    """Load libpa.so once and declare the ABI's signatures."""
+    global _lib
+    if _lib is not None and path == _LIB_PATH:
+        return _lib
+    if not os.path.exists(path):
+        raise ImportError(f"{path} is missing: build it with `python paged_kv_cache_327_b200/build.py` "
+                          "(the CUDA path has no fallback)")
+    lib = ctypes.CDLL(path)
+    P, I, I64, SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t
+    lib.pa_decode_workspace_size.argtypes = [I, I, I, I, I]
+    lib.pa_decode_workspace_size.restype = SZ
+    lib.pa_decode.argtypes = [P, P, P, P, P, P, I, I, I, I, I, ctypes.c_float, I, I64, I, I, I, I, P, SZ, P]
+    lib.pa_decode.restype = I
+    lib.pa_reshape_and_cache.argtypes = [P, P, P, P, P, I, I, I, I, I64, I, I64, I64, P]
+    lib.pa_reshape_and_cache.restype = I
+    lib.pa_copy_blocks.argtypes = [P, P, P, I, I64, SZ, P, P]
+    lib.pa_copy_blocks.restype = I
+    lib.pa_strerror.argtypes = [I]
+    lib.pa_strerror.restype = ctypes.c_char_p
+    lib.pa_get_device_error.argtypes = [P]
+    lib.pa_get_device_error.restype = I
+    lib.pa_version.argtypes = []
+    lib.pa_version.restype = I
+    if path == _LIB_PATH:
+        _lib = lib
+    return lib
+
+
+class PAError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {pa_strerror(status)} (status {status})")
+
+
+def pa_strerror(status: int) -> str:
+    return load_library().pa_strerror(int(status)).decode()
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _check(rc: int, what: str) -> None:
+    if rc != PA_OK:
+        raise PAError(rc, what)
+
+
+def pa_decode_workspace_size(num_seqs: int, num_q_heads: int, head_dim: int, max_seq_len: int,
+                             partition_size: int = 0) -> int:
+    return int(load_library().pa_decode_workspace_size(num_seqs, num_q_heads, head_dim, max_seq_len,
+                                                       partition_size))
+
+
+def pa_decode(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+              block_tables: torch.Tensor, seq_lens: torch.Tensor, scale: float, workspace: torch.Tensor,
+              partition_size: int = 0, stream=None) -> None:
+    """out[N,Hq,D] <- paged decode attention (see include/pa.h); shapes give the sizes."""
+    N, Hq, D = q.shape
+    NB, bs, Hkv, D2 = k_cache.shape
+    if D2 != D or tuple(out.shape) != (N, Hq, D) or v_cache.shape != k_cache.shape:
+        raise ValueError("shape mismatch between q, out and the caches")
+    for t in (out, q, k_cache, v_cache, block_tables, seq_lens, workspace):
+        if not t.is_contiguous():
+            raise ValueError("tensors must be contiguous")
+    if block_tables.dtype != torch.int32 or seq_lens.dtype != torch.int32:
+        raise TypeError("block_tables and seq_lens must be int32")
+    rc = load_library().pa_decode(
+        _ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), _ptr(seq_lens), N, Hq, Hkv, D, bs,
+        ctypes.c_float(scale), block_tables.shape[1], NB, _TORCH_CODE[q.dtype], _TORCH_CODE[k_cache.dtype],
+        _TORCH_CODE[out.dtype], partition_size, _ptr(workspace), workspace.numel() * workspace.element_size(),
+        _stream(stream))
+    _check(rc, "pa_decode")
+
+
+def pa_reshape_and_cache(k: torch.Tensor, v: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                         slot_mapping: torch.Tensor, stream=None) -> None:
+    """k_cache/v_cache[slot // bs, slot % bs] <- k/v[t] for each token t with slot >= 0."""
+    T, Hkv, D = k.shape
+    NB, bs = k_cache.shape[:2]
+    if slot_mapping.dtype != torch.int64:
+        raise TypeError("slot_mapping must be int64")
+    rc = load_library().pa_reshape_and_cache(
+        _ptr(k), _ptr(v), _ptr(k_cache), _ptr(v_cache), _ptr(slot_mapping), T, Hkv, D, bs, NB,
+        _TORCH_CODE[k_cache.dtype], k.stride(0), v.stride(0), _stream(stream))
+    _check(rc, "pa_reshape_and_cache")
+
+
+def pa_copy_blocks(k_cache: torch.Tensor, v_cache: torch.Tensor, src_dst_pairs: torch.Tensor,
+                   host_pairs: Optional[np.ndarray] = None, stream=None) -> None:
+    """Copy physical block pairs[p,0] over pairs[p,1] in both caches (copy-on-write)."""
+    P = src_dst_pairs.shape[0]
+    NB = k_cache.shape[0]
+    block_bytes = k_cache[0].numel() * k_cache.element_size()
+    hp = None
+    if host_pairs is not None:
+        hp = np.ascontiguousarray(host_pairs, dtype=np.int32)
+    rc = load_library().pa_copy_blocks(
+        _ptr(k_cache), _ptr(v_cache), _ptr(src_dst_pairs), P, NB, block_bytes,
+        ctypes.c_void_p(hp.ctypes.data) if hp is not None else ctypes.c_void_p(0), _stream(stream))
+    _check(rc, "pa_copy_blocks")
+
+
+def pa_get_device_error(stream=None) -> int:
+    return int(load_library().pa_get_device_error(_stream(stream)))
+
+
+# ---------------------------------------------------------------------------------------
+# convenience: a workload on the device and one decode step through the ABI
+# ---------------------------------------------------------------------------------------
+def to_torch(a: np.ndarray, dtype: str, device) -> torch.Tensor:
+    """Storage array (float32, or uint16 bit patterns) -> torch tensor of the named dtype."""
+    if dtype == "f32":
+        t = torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32))
+    else:
+        t = torch.from_numpy(np.ascontiguousarray(a, dtype=np.uint16).view(np.int16)).view(_NAME_TORCH[dtype])
+    return t.to(device)
+
+
+def from_torch(t: torch.Tensor) -> np.ndarray:
+    """torch tensor -> storage array (float32, or uint16 bit patterns for 16-bit types)."""
+    t = t.detach().cpu().contiguous()
+    if t.dtype == torch.float32:
+        return t.numpy()
+    return t.view(torch.int16).numpy().view(np.uint16)
+
+
+@dataclasses.dataclass
+class DeviceWorkload:
+    w: W.Workload
+    q: torch.Tensor
+    k_cache: torch.Tensor
+    v_cache: torch.Tensor
+    block_tables: torch.Tensor
+    seq_lens: torch.Tensor
+    new_k: torch.Tensor
+    new_v: torch.Tensor
+    slot_mapping: torch.Tensor
+    copy_pairs: torch.Tensor
+
+
+def device_workload(w: W.Workload, device="cuda") -> DeviceWorkload:
+    return DeviceWorkload(
+        w=w, q=to_torch(w.q, w.q_dtype, device), k_cache=to_torch(w.k_cache, w.kv_dtype, device),
+        v_cache=to_torch(w.v_cache, w.kv_dtype, device),
+        block_tables=torch.from_numpy(w.block_tables).to(device),
+        seq_lens=torch.from_numpy(w.seq_lens).to(device), new_k=to_torch(w.new_k, w.kv_dtype, device),
+        new_v=to_torch(w.new_v, w.kv_dtype, device), slot_mapping=torch.from_numpy(w.slot_mapping).to(device),
+        copy_pairs=torch.from_numpy(np.ascontiguousarray(w.copy_pairs, dtype=np.int32).reshape(-1, 2)).to(device))
+
+
+class DecodeWorkspace:
+    """Caller-owned decode workspace sized by pa_decode_workspace_size()."""
+
+    def __init__(self, num_seqs, num_q_heads, head_dim, max_seq_len, partition_size=0, device="cuda"):
+        n = pa_decode_workspace_size(num_seqs, num_q_heads, head_dim, max_seq_len, partition_size)
+        if n == 0:
+            raise ValueError("invalid workspace request")
+        self.tensor = torch.empty(n, dtype=torch.uint8, device=device)
+
+    @classmethod
+    def for_workload(cls, dw: DeviceWorkload, partition_size=0):
+        w = dw.w
+        return cls(w.num_seqs, w.num_q_heads, w.head_dim, w.max_blocks_per_seq * w.block_size, partition_size,
+                   device=dw.q.device)
+
+
+def run_step(dw: DeviceWorkload, out: torch.Tensor, ws: DecodeWorkspace, partition_size=0, stream=None) -> None:
+    """One decode step: copy_blocks -> reshape_and_cache -> decode (all through the C ABI)."""
+    if dw.copy_pairs.shape[0]:
+        pa_copy_blocks(dw.k_cache, dw.v_cache, dw.copy_pairs, stream=stream)
+    if dw.slot_mapping.shape[0]:
+        pa_reshape_and_cache(dw.new_k, dw.new_v, dw.k_cache, dw.v_cache, dw.slot_mapping, stream=stream)
+    pa_decode(out, dw.q, dw.k_cache, dw.v_cache, dw.block_tables, dw.seq_lens, dw.w.scale, ws.tensor,
+              partition_size=partition_size, stream=stream)

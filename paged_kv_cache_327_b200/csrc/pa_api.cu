@@ -1,0 +1,298 @@
+// pa_api.cu -- the C ABI of libpa.so (declared in include/pa.h): host-side validation,
+// workspace layout, TMA descriptor encoding and kernel launches.  Every step of the
+// computation runs in the CUDA kernels of pa_decode.cuh / pa_cache.cuh; there is no CPU
+// fallback.  The library allocates no device memory.
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <climits>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+#include <unordered_set>
+
+#include "pa.h"
+#include "pa_cache.cuh"
+
+namespace {
+
+constexpr int kDefaultPartition = 512;
+constexpr int kMaxDevices = 64;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+int elem_bytes(int dt) { return dt == PA_F32 ? 4 : 2; }
+
+struct WsLayout {
+  size_t counters, seq_nparts, items, part_ml, part_acc, total;
+};
+
+WsLayout ws_layout(int64_t num_seqs, int64_t num_q_heads, int64_t head_dim, int64_t max_parts) {
+  WsLayout L{};
+  size_t o = 0;
+  L.counters = o;
+  o += 256;
+  L.seq_nparts = o;
+  o += align256(static_cast<size_t>(num_seqs) * 4);
+  L.items = o;
+  o += align256(static_cast<size_t>(num_seqs * max_parts) * sizeof(pa::WorkItem));
+  L.part_ml = o;
+  o += align256(static_cast<size_t>(num_seqs * max_parts * num_q_heads) * sizeof(float2));
+  L.part_acc = o;
+  o += align256(static_cast<size_t>(num_seqs * max_parts * num_q_heads * head_dim) * sizeof(float));
+  L.total = o;
+  return L;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// Per-device launch facts, looked up once.
+struct DeviceInfo {
+  int sm_count = 0;
+  bool smem_set[32] = {};
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mu;
+
+int current_device_info(int* dev, DeviceInfo** info) {
+  if (cudaGetDevice(dev) != cudaSuccess || *dev < 0 || *dev >= kMaxDevices) return PA_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  DeviceInfo& d = g_dev[*dev];
+  if (d.sm_count == 0 && cudaDeviceGetAttribute(&d.sm_count, cudaDevAttrMultiProcessorCount, *dev) != cudaSuccess)
+    return PA_ERR_CUDA;
+  *info = &d;
+  return PA_OK;
+}
+
+// KV cache [num_blocks, block_size, num_kv_heads, head_dim] seen as a 3-D tensor
+// (64 elements, head_dim/64 * num_kv_heads column halves, num_blocks * block_size rows);
+// one box = block_size rows of one 128-byte column half, 128-byte swizzle.
+int encode_kv_map(CUtensorMap* map, const void* base, int kv_dtype, int64_t num_blocks, int block_size,
+                  int num_kv_heads, int head_dim) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+  if (!enc) return PA_ERR_CUDA;
+  const cuuint64_t dims[3] = {64, static_cast<cuuint64_t>(head_dim / 64) * num_kv_heads,
+                              static_cast<cuuint64_t>(num_blocks) * block_size};
+  const cuuint64_t strides[2] = {128, static_cast<cuuint64_t>(num_kv_heads) * head_dim * 2};
+  const cuuint32_t box[3] = {64, 1, static_cast<cuuint32_t>(block_size)};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r =
+      enc(map, kv_dtype == PA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3,
+          const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? PA_OK : PA_ERR_CUDA;
+}
+
+template <int BS, int D, typename KT, bool QF32>
+int launch_partition(const pa::DecodeParams& p, const CUtensorMap& tmk, const CUtensorMap& tmv,
+                     int64_t max_items, DeviceInfo* info, int slot_id, cudaStream_t stream) {
+  using C = pa::DecodeCfg<BS, D, KT, QF32>;
+  auto kern = pa::pa_decode_partition_kernel<BS, D, KT, QF32>;
+  if (!info->smem_set[slot_id]) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
+      return PA_ERR_CUDA;
+    info->smem_set[slot_id] = true;
+  }
+  int64_t ctas = (max_items + C::NWARP - 1) / C::NWARP;
+  if (ctas > info->sm_count) ctas = info->sm_count;
+  if (ctas < 1) ctas = 1;
+  kern<<<static_cast<unsigned>(ctas), C::NWARP * 32, C::SMEM_BYTES, stream>>>(tmk, tmv, p);
+  return cudaPeekAtLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+template <int BS, int D>
+int dispatch_kv(const pa::DecodeParams& p, const CUtensorMap& tmk, const CUtensorMap& tmv, int64_t max_items,
+                DeviceInfo* info, int kv_dtype, bool qf32, int base_id, cudaStream_t stream) {
+  if (kv_dtype == PA_BF16)
+    return qf32 ? launch_partition<BS, D, __nv_bfloat16, true>(p, tmk, tmv, max_items, info, base_id + 0, stream)
+                : launch_partition<BS, D, __nv_bfloat16, false>(p, tmk, tmv, max_items, info, base_id + 1, stream);
+  return qf32 ? launch_partition<BS, D, __half, true>(p, tmk, tmv, max_items, info, base_id + 2, stream)
+              : launch_partition<BS, D, __half, false>(p, tmk, tmv, max_items, info, base_id + 3, stream);
+}
+
+}  // namespace
+
+extern "C" {
+
+int pa_version(void) { return 100; }
+
+const char* pa_strerror(int status) {
+  switch (status) {
+    case PA_OK: return "success";
+    case PA_ERR_INVALID: return "invalid argument (null or misaligned pointer, or a size out of range)";
+    case PA_ERR_UNSUPPORTED: return "unsupported configuration (head_dim, block_size, dtype or group size)";
+    case PA_ERR_WORKSPACE: return "workspace missing or smaller than pa_decode_workspace_size()";
+    case PA_ERR_CUDA: return "a CUDA runtime call or kernel launch failed";
+    default: return "unknown pa_status";
+  }
+}
+
+size_t pa_decode_workspace_size(int num_seqs, int num_q_heads, int head_dim, int max_seq_len,
+                                int partition_size) {
+  if (num_seqs < 0 || num_q_heads <= 0 || head_dim <= 0 || max_seq_len < 0 || partition_size < 0) return 0;
+  const int P = partition_size ? partition_size : kDefaultPartition;
+  const int64_t max_parts = std::max<int64_t>(1, (static_cast<int64_t>(max_seq_len) + P - 1) / P);
+  return ws_layout(num_seqs, num_q_heads, head_dim, max_parts).total;
+}
+
+int pa_decode(void* out, const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,
+              const int32_t* seq_lens, int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+              int block_size, float scale, int max_blocks_per_seq, int64_t num_blocks, int q_dtype,
+              int kv_dtype, int out_dtype, int partition_size, void* workspace, size_t workspace_bytes,
+              void* stream) {
+  if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 ||
+      max_blocks_per_seq <= 0 || num_blocks <= 0 || partition_size < 0 || !std::isfinite(scale))
+    return PA_ERR_INVALID;
+  if (num_q_heads % num_kv_heads) return PA_ERR_INVALID;
+  const int G = num_q_heads / num_kv_heads;
+  if (G > 8) return PA_ERR_UNSUPPORTED;
+  if (head_dim != 64 && head_dim != 128) return PA_ERR_UNSUPPORTED;
+  if (block_size != 16 && block_size != 32) return PA_ERR_UNSUPPORTED;
+  if (kv_dtype != PA_F16 && kv_dtype != PA_BF16) return PA_ERR_UNSUPPORTED;
+  if (q_dtype != kv_dtype && q_dtype != PA_F32) return PA_ERR_UNSUPPORTED;
+  if (out_dtype != PA_F32 && out_dtype != PA_F16 && out_dtype != PA_BF16) return PA_ERR_UNSUPPORTED;
+  const int P = partition_size ? partition_size : kDefaultPartition;
+  if (P % block_size || P / block_size > 32) return PA_ERR_UNSUPPORTED;
+  if (num_blocks > INT_MAX / block_size) return PA_ERR_INVALID;
+  const int64_t max_len = static_cast<int64_t>(max_blocks_per_seq) * block_size;
+  if (max_len > INT_MAX) return PA_ERR_INVALID;
+  if (num_seqs == 0) return PA_OK;
+  if (!out || !q || !k_cache || !v_cache || !block_tables || !seq_lens) return PA_ERR_INVALID;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache)) return PA_ERR_INVALID;
+  const int64_t max_parts = std::max<int64_t>(1, (max_len + P - 1) / P);
+  const WsLayout L = ws_layout(num_seqs, num_q_heads, head_dim, max_parts);
+  if (!workspace || workspace_bytes < L.total) return PA_ERR_WORKSPACE;
+  if (reinterpret_cast<uintptr_t>(workspace) & 255u) return PA_ERR_INVALID;
+
+  int dev;
+  DeviceInfo* info;
+  if (current_device_info(&dev, &info) != PA_OK) return PA_ERR_CUDA;
+  CUtensorMap tmk, tmv;
+  if (encode_kv_map(&tmk, k_cache, kv_dtype, num_blocks, block_size, num_kv_heads, head_dim) != PA_OK ||
+      encode_kv_map(&tmv, v_cache, kv_dtype, num_blocks, block_size, num_kv_heads, head_dim) != PA_OK)
+    return PA_ERR_CUDA;
+
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  pa::DecodeParams p{};
+  p.out = out;
+  p.q = q;
+  p.block_tables = block_tables;
+  p.seq_lens = seq_lens;
+  p.num_seqs = num_seqs;
+  p.num_q_heads = num_q_heads;
+  p.num_kv_heads = num_kv_heads;
+  p.group = G;
+  p.head_dim = head_dim;
+  p.block_size = block_size;
+  p.max_blocks_per_seq = max_blocks_per_seq;
+  p.num_blocks = static_cast<int>(num_blocks);
+  p.partition_size = P;
+  p.max_parts = static_cast<int>(max_parts);
+  p.out_dtype = out_dtype;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.counters = reinterpret_cast<unsigned int*>(ws + L.counters);
+  p.seq_nparts = reinterpret_cast<int*>(ws + L.seq_nparts);
+  p.items = reinterpret_cast<pa::WorkItem*>(ws + L.items);
+  p.part_ml = reinterpret_cast<float2*>(ws + L.part_ml);
+  p.part_acc = reinterpret_cast<float*>(ws + L.part_acc);
+
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  pa::pa_decode_plan_kernel<<<1, 1024, 0, st>>>(p);
+  if (cudaPeekAtLastError() != cudaSuccess) return PA_ERR_CUDA;
+
+  const int64_t max_items = static_cast<int64_t>(num_seqs) * max_parts * num_kv_heads;
+  const bool qf32 = q_dtype == PA_F32;
+  int rc;
+  if (block_size == 16)
+    rc = head_dim == 128 ? dispatch_kv<16, 128>(p, tmk, tmv, max_items, info, kv_dtype, qf32, 0, st)
+                         : dispatch_kv<16, 64>(p, tmk, tmv, max_items, info, kv_dtype, qf32, 4, st);
+  else
+    rc = head_dim == 128 ? dispatch_kv<32, 128>(p, tmk, tmv, max_items, info, kv_dtype, qf32, 8, st)
+                         : dispatch_kv<32, 64>(p, tmk, tmv, max_items, info, kv_dtype, qf32, 12, st);
+  if (rc != PA_OK) return rc;
+
+  pa::pa_decode_reduce_kernel<<<dim3(static_cast<unsigned>(num_seqs), static_cast<unsigned>(num_kv_heads)), 128, 0,
+                                st>>>(p);
+  return cudaPeekAtLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+int pa_reshape_and_cache(const void* k, const void* v, void* k_cache, void* v_cache, const int64_t* slot_mapping,
+                         int num_tokens, int num_kv_heads, int head_dim, int block_size, int64_t num_blocks,
+                         int kv_dtype, int64_t k_token_stride, int64_t v_token_stride, void* stream) {
+  if (num_tokens < 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 || num_blocks <= 0 ||
+      k_token_stride < 0 || v_token_stride < 0)
+    return PA_ERR_INVALID;
+  if (kv_dtype != PA_F16 && kv_dtype != PA_BF16 && kv_dtype != PA_F32) return PA_ERR_UNSUPPORTED;
+  const int es = elem_bytes(kv_dtype);
+  const int64_t row = static_cast<int64_t>(num_kv_heads) * head_dim;
+  if ((row * es) % 16) return PA_ERR_UNSUPPORTED;
+  if (!k_token_stride) k_token_stride = row;
+  if (!v_token_stride) v_token_stride = row;
+  if (k_token_stride < row || v_token_stride < row || (k_token_stride * es) % 16 || (v_token_stride * es) % 16)
+    return PA_ERR_INVALID;
+  if (num_tokens == 0) return PA_OK;
+  if (!k || !v || !k_cache || !v_cache || !slot_mapping) return PA_ERR_INVALID;
+  if (!aligned16(k) || !aligned16(v) || !aligned16(k_cache) || !aligned16(v_cache)) return PA_ERR_INVALID;
+  int dev;
+  DeviceInfo* info;
+  if (current_device_info(&dev, &info) != PA_OK) return PA_ERR_CUDA;
+  const int grid = static_cast<int>(std::min<int64_t>(num_tokens, 64LL * info->sm_count));
+  pa::pa_reshape_and_cache_kernel<<<grid, 128, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint8_t*>(k), static_cast<const uint8_t*>(v), static_cast<uint8_t*>(k_cache),
+      static_cast<uint8_t*>(v_cache), slot_mapping, num_tokens, row * es, k_token_stride * es, v_token_stride * es,
+      num_blocks * block_size);
+  return cudaPeekAtLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+int pa_copy_blocks(void* k_cache, void* v_cache, const int32_t* src_dst_pairs, int num_pairs, int64_t num_blocks,
+                   size_t block_bytes, const int32_t* host_pairs, void* stream) {
+  if (num_pairs < 0 || num_blocks <= 0 || block_bytes == 0 || block_bytes % 16) return PA_ERR_INVALID;
+  if (num_pairs == 0) return PA_OK;
+  if (!k_cache || !v_cache || !src_dst_pairs) return PA_ERR_INVALID;
+  if (!aligned16(k_cache) || !aligned16(v_cache)) return PA_ERR_INVALID;
+  if (host_pairs) {
+    std::unordered_set<int32_t> dsts, srcs;
+    for (int i = 0; i < num_pairs; ++i) {
+      const int32_t s = host_pairs[2 * i], d = host_pairs[2 * i + 1];
+      if (s < 0 || s >= num_blocks || d < 0 || d >= num_blocks || s == d) return PA_ERR_INVALID;
+      if (!dsts.insert(d).second) return PA_ERR_INVALID;
+      srcs.insert(s);
+    }
+    for (int32_t d : dsts)
+      if (srcs.count(d)) return PA_ERR_INVALID;
+  }
+  const int64_t vecs = static_cast<int64_t>(block_bytes / 16);
+  const int chunks = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(16, vecs / (256 * 4))));
+  pa::pa_copy_blocks_kernel<<<dim3(static_cast<unsigned>(num_pairs), 2, static_cast<unsigned>(chunks)), 256, 0,
+                              static_cast<cudaStream_t>(stream)>>>(static_cast<uint8_t*>(k_cache),
+                                                                   static_cast<uint8_t*>(v_cache), src_dst_pairs,
+                                                                   num_blocks, static_cast<int64_t>(block_bytes));
+  return cudaPeekAtLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+int pa_get_device_error(void* stream) {
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return PA_ERR_CUDA;
+  unsigned int code = 0;
+  if (cudaMemcpyFromSymbol(&code, pa::g_dev_error, sizeof(code)) != cudaSuccess) return PA_ERR_CUDA;
+  const unsigned int zero = 0;
+  if (cudaMemcpyToSymbol(pa::g_dev_error, &zero, sizeof(zero)) != cudaSuccess) return PA_ERR_CUDA;
+  return static_cast<int>(code);
+}
+
+}  // extern "C"

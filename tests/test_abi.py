@@ -1,0 +1,107 @@
+"""The C ABI on a machine without a GPU: the library loads, exports every entry point
+that include/pa.h declares, and rejects invalid arguments on the host before any CUDA
+call (no compute is launched here)."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+from paged_kv_cache_327_b200 import binding as B
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "pa.h")
+
+
+def declared_symbols():
+    text = open(HEADER, encoding="utf-8").read()
+    return re.findall(r"^PA_API\s+[\w\s\*]+?\b(pa_\w+)\s*\(", text, flags=re.M)
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from paged_kv_cache_327_b200 import build
+    build.build()
+    return B.load_library()
+
+
+def test_header_declares_the_entry_points():
+    names = declared_symbols()
+    assert set(names) == set(B.EXPORTED), names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_symbols():
+        assert hasattr(lib, name), f"{name} not exported"
+
+
+def test_version_and_strerror(lib):
+    assert lib.pa_version() == 100
+    for st in (B.PA_OK, B.PA_ERR_INVALID, B.PA_ERR_UNSUPPORTED, B.PA_ERR_WORKSPACE, B.PA_ERR_CUDA):
+        assert len(B.pa_strerror(st)) > 5
+    assert "unknown" in B.pa_strerror(12345)
+
+
+def test_workspace_size(lib):
+    ws = B.pa_decode_workspace_size
+    assert ws(0, 1, 128, 0) > 0
+    assert ws(-1, 32, 128, 100) == 0 and ws(4, 0, 128, 100) == 0
+    a = ws(256, 32, 128, 8192)
+    # 16 partitions of 512 per sequence: the fp32 partial outputs dominate
+    assert a >= 256 * 16 * 32 * 128 * 4
+    assert ws(256, 32, 128, 8192, 256) > a
+    assert ws(256, 32, 128, 8193) > a
+
+
+FAKE = 0x10000  # a 16-byte aligned non-null address that is never dereferenced
+
+
+def decode_call(lib, **kw):
+    a = dict(out=FAKE, q=FAKE, k=FAKE, v=FAKE, bt=FAKE, sl=FAKE, N=4, Hq=8, Hkv=2, D=128, bs=16, scale=0.1,
+             MB=8, NB=64, qd=2, kd=2, od=0, P=0, ws=FAKE, wsb=0, stream=0)
+    a.update(kw)
+    V = ctypes.c_void_p
+    return lib.pa_decode(V(a["out"]), V(a["q"]), V(a["k"]), V(a["v"]), V(a["bt"]), V(a["sl"]), a["N"], a["Hq"],
+                         a["Hkv"], a["D"], a["bs"], ctypes.c_float(a["scale"]), a["MB"], a["NB"], a["qd"], a["kd"],
+                         a["od"], a["P"], V(a["ws"]), a["wsb"], V(a["stream"]))
+
+
+def test_decode_argument_validation(lib):
+    assert decode_call(lib, N=0) == B.PA_OK                      # nothing to do, no CUDA call
+    assert decode_call(lib, Hq=6, Hkv=4) == B.PA_ERR_INVALID     # heads not a multiple
+    assert decode_call(lib, Hq=32, Hkv=2) == B.PA_ERR_UNSUPPORTED  # G = 16
+    assert decode_call(lib, D=96) == B.PA_ERR_UNSUPPORTED
+    assert decode_call(lib, bs=8) == B.PA_ERR_UNSUPPORTED
+    assert decode_call(lib, kd=0, qd=0) == B.PA_ERR_UNSUPPORTED  # fp32 cache
+    assert decode_call(lib, qd=1) == B.PA_ERR_UNSUPPORTED        # f16 q with bf16 cache
+    assert decode_call(lib, od=7) == B.PA_ERR_UNSUPPORTED
+    assert decode_call(lib, P=24) == B.PA_ERR_UNSUPPORTED        # not a multiple of the block size
+    assert decode_call(lib, P=1024) == B.PA_ERR_UNSUPPORTED      # more than 32 blocks per partition
+    assert decode_call(lib, scale=float("nan")) == B.PA_ERR_INVALID
+    assert decode_call(lib, q=0) == B.PA_ERR_INVALID
+    assert decode_call(lib, k=FAKE + 8) == B.PA_ERR_INVALID      # misaligned cache
+    assert decode_call(lib, wsb=100) == B.PA_ERR_WORKSPACE
+    need = B.pa_decode_workspace_size(4, 8, 128, 8 * 16)
+    assert decode_call(lib, wsb=need - 1) == B.PA_ERR_WORKSPACE
+    assert decode_call(lib, ws=FAKE + 16, wsb=need) == B.PA_ERR_INVALID   # workspace not 256-aligned
+
+
+def test_cache_op_argument_validation(lib):
+    V = ctypes.c_void_p
+    r = lib.pa_reshape_and_cache
+    assert r(V(FAKE), V(FAKE), V(FAKE), V(FAKE), V(FAKE), 0, 8, 128, 16, 10, 2, 0, 0, V(0)) == B.PA_OK
+    assert r(V(FAKE), V(FAKE), V(FAKE), V(FAKE), V(FAKE), 3, 8, 128, 16, 10, 2, 100, 0, V(0)) == B.PA_ERR_INVALID
+    assert r(V(FAKE), V(FAKE), V(FAKE), V(FAKE), V(FAKE), 3, 1, 4, 16, 10, 2, 0, 0, V(0)) == B.PA_ERR_UNSUPPORTED
+    assert r(V(0), V(FAKE), V(FAKE), V(FAKE), V(FAKE), 3, 8, 128, 16, 10, 2, 0, 0, V(0)) == B.PA_ERR_INVALID
+    c = lib.pa_copy_blocks
+    assert c(V(FAKE), V(FAKE), V(FAKE), 0, 10, 4096, V(0), V(0)) == B.PA_OK
+    assert c(V(FAKE), V(FAKE), V(FAKE), 1, 10, 4008, V(0), V(0)) == B.PA_ERR_INVALID   # not a multiple of 16
+    for bad in ([[1, 2], [3, 2]], [[1, 2], [2, 3]], [[1, 10]], [[4, 4]], [[-1, 2]]):
+        hp = np.asarray(bad, np.int32)
+        assert c(V(FAKE), V(FAKE), V(FAKE), len(hp), 10, 4096, V(hp.ctypes.data), V(0)) == B.PA_ERR_INVALID, bad
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    with pytest.raises(ImportError):
+        B.load_library(str(tmp_path / "libpa.so"))
