@@ -52,6 +52,7 @@ def parse_args():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", default="8b", choices=list(W.CONFIG_NAMES))
     ap.add_argument("--block-size", type=int, default=None)
+    ap.add_argument("--num-seqs", type=int, default=None, help="smaller batch of the same config (profiling)")
     ap.add_argument("--partition-size", type=int, default=0)
     ap.add_argument("--out-dtype", default=None, help="f32 | f16 | bf16 (default: the query dtype)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -177,12 +178,16 @@ def oracle_sample_rate(w: W.Workload, seconds: float, start: int = 0):
         pick.append(i)
         tok += int(w.seq_lens[i])
     idx = np.asarray(pick)
-    t = time.perf_counter()
-    oracle.decode(np.ascontiguousarray(w.q[idx]), w.q_dtype, kc, vc, w.kv_dtype,
-                  np.ascontiguousarray(w.block_tables[idx]), np.ascontiguousarray(w.seq_lens[idx]), w.scale,
-                  num_threads=threads)
-    dt = time.perf_counter() - t
-    return tok * row, dt, threads, len(idx)
+    q, bt, sl = (np.ascontiguousarray(w.q[idx]), np.ascontiguousarray(w.block_tables[idx]),
+                 np.ascontiguousarray(w.seq_lens[idx]))
+    passes, t = 0, time.perf_counter()
+    while True:  # whole passes over the sample until the time budget is used
+        oracle.decode(q, w.q_dtype, kc, vc, w.kv_dtype, bt, sl, w.scale, num_threads=threads)
+        passes += 1
+        dt = time.perf_counter() - t
+        if dt >= 0.8 * seconds:
+            break
+    return passes * tok * row, dt, threads, passes * len(idx)
 
 
 def run_reference(args):
@@ -237,7 +242,8 @@ def run_ours(args):
                                 device_id=torch.device("cuda", local))
 
     seed = W.config_seed(args.config) + 1000 * rank
-    w = W.make_config(args.config, block_size=args.block_size, seed=seed)
+    extra = {"num_seqs": args.num_seqs} if args.num_seqs else {}
+    w = W.make_config(args.config, block_size=args.block_size, seed=seed, **extra)
     out_dtype = args.out_dtype or w.q_dtype
     dw = B.device_workload(w, f"cuda:{local}")
     ws = B.DecodeWorkspace.for_workload(dw, args.partition_size)
@@ -369,8 +375,8 @@ def run_ours(args):
     if not args.no_cpu_baseline and world == 1:
         b, t, threads, n = oracle_sample_rate(w, args.cpu_seconds)
         cpu = {"value": round(b / t / 1e9, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
-               "sample": f"first {n} of {w.num_seqs} sequences ({b / 1e9:.3f} GB of K+V), decode only, "
-                         f"fp64 two-pass softmax, {t:.1f} s"}
+               "sample": f"{n} sequence decodes from the start of the batch of {w.num_seqs} "
+                         f"({b / 1e9:.3f} GB of K+V), decode only, fp64 two-pass softmax, {t:.1f} s"}
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_step, 5), "higher_is_better": True, "scaling": "weak",

@@ -208,6 +208,7 @@ def test_bad_seq_len_and_slot_and_pair_are_reported():
     w = W.independent("bad", [40, 20], num_q_heads=2, num_kv_heads=2, head_dim=64, block_size=16,
                       q_dtype="f16", kv_dtype="f16", seed=6)
     dw = B.device_workload(w)
+    B.pa_reshape_and_cache(dw.new_k, dw.new_v, dw.k_cache, dw.v_cache, dw.slot_mapping)
     dw.seq_lens[0] = w.max_blocks_per_seq * 16 + 1
     out = torch.zeros((2, 2, 64), dtype=torch.float32, device="cuda")
     ws = B.DecodeWorkspace.for_workload(dw)
