@@ -27,16 +27,17 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 int elem_bytes(int dt) { return dt == PA_F32 ? 4 : 2; }
 
 struct WsLayout {
-  size_t counters, seq_nparts, items, part_ml, part_acc, total;
+  size_t counters, merge_cnt, items, part_ml, part_acc, total;
 };
 
+// merge counters are sized by num_q_heads (>= num_kv_heads), so the size needs no KV-head count
 WsLayout ws_layout(int64_t num_seqs, int64_t num_q_heads, int64_t head_dim, int64_t max_parts) {
   WsLayout L{};
   size_t o = 0;
   L.counters = o;
   o += 256;
-  L.seq_nparts = o;
-  o += align256(static_cast<size_t>(num_seqs) * 4);
+  L.merge_cnt = o;
+  o += align256(static_cast<size_t>(num_seqs * num_q_heads) * 4);
   L.items = o;
   o += align256(static_cast<size_t>(num_seqs * max_parts) * sizeof(pa::WorkItem));
   L.part_ml = o;
@@ -111,7 +112,19 @@ int launch_partition(const pa::DecodeParams& p, const CUtensorMap& tmk, const CU
   int64_t ctas = (max_items + C::NWARP - 1) / C::NWARP;
   if (ctas > info->sm_count) ctas = info->sm_count;
   if (ctas < 1) ctas = 1;
-  kern<<<static_cast<unsigned>(ctas), C::NWARP * 32, C::SMEM_BYTES, stream>>>(tmk, tmv, p);
+  // programmatic dependent launch: the prologue overlaps the plan kernel, which the
+  // partition kernel waits for (griddepcontrol.wait) before reading anything
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(ctas));
+  cfg.blockDim = dim3(C::NWARP * 32);
+  cfg.dynamicSmemBytes = C::SMEM_BYTES;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kern, tmk, tmv, p) != cudaSuccess) return PA_ERR_CUDA;
   return cudaPeekAtLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
@@ -175,6 +188,7 @@ int pa_decode(void* out, const void* q, const void* k_cache, const void* v_cache
   if (!out || !q || !k_cache || !v_cache || !block_tables || !seq_lens) return PA_ERR_INVALID;
   if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache)) return PA_ERR_INVALID;
   const int64_t max_parts = std::max<int64_t>(1, (max_len + P - 1) / P);
+  if (max_parts > 32767) return PA_ERR_UNSUPPORTED;
   const WsLayout L = ws_layout(num_seqs, num_q_heads, head_dim, max_parts);
   if (!workspace || workspace_bytes < L.total) return PA_ERR_WORKSPACE;
   if (reinterpret_cast<uintptr_t>(workspace) & 255u) return PA_ERR_INVALID;
@@ -206,13 +220,13 @@ int pa_decode(void* out, const void* q, const void* k_cache, const void* v_cache
   p.out_dtype = out_dtype;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.counters = reinterpret_cast<unsigned int*>(ws + L.counters);
-  p.seq_nparts = reinterpret_cast<int*>(ws + L.seq_nparts);
+  p.merge_cnt = reinterpret_cast<int*>(ws + L.merge_cnt);
   p.items = reinterpret_cast<pa::WorkItem*>(ws + L.items);
   p.part_ml = reinterpret_cast<float2*>(ws + L.part_ml);
   p.part_acc = reinterpret_cast<float*>(ws + L.part_acc);
 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  pa::pa_decode_plan_kernel<<<1, 1024, 0, st>>>(p);
+  pa::pa_decode_plan_kernel<<<1, pa::kPlanThreads, 0, st>>>(p);
   if (cudaPeekAtLastError() != cudaSuccess) return PA_ERR_CUDA;
 
   const int64_t max_items = static_cast<int64_t>(num_seqs) * max_parts * num_kv_heads;
@@ -224,11 +238,7 @@ int pa_decode(void* out, const void* q, const void* k_cache, const void* v_cache
   else
     rc = head_dim == 128 ? dispatch_kv<32, 128>(p, tmk, tmv, max_items, info, kv_dtype, qf32, 8, st)
                          : dispatch_kv<32, 64>(p, tmk, tmv, max_items, info, kv_dtype, qf32, 12, st);
-  if (rc != PA_OK) return rc;
-
-  pa::pa_decode_reduce_kernel<<<dim3(static_cast<unsigned>(num_seqs), static_cast<unsigned>(num_kv_heads)), 128, 0,
-                                st>>>(p);
-  return cudaPeekAtLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+  return rc;
 }
 
 int pa_reshape_and_cache(const void* k, const void* v, void* k_cache, void* v_cache, const int64_t* slot_mapping,

@@ -164,3 +164,14 @@ __device__ __forceinline__ float fast_exp2(float x) {
 }
 
 }  // namespace pa
+
+namespace pa {
+
+// Programmatic dependent launch: let the next kernel in the stream start its prologue,
+// and wait (in the dependent kernel) until the previous kernel's results are visible.
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+}  // namespace pa
