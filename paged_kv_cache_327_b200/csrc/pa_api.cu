@@ -27,17 +27,14 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 int elem_bytes(int dt) { return dt == PA_F32 ? 4 : 2; }
 
 struct WsLayout {
-  size_t counters, merge_cnt, items, part_ml, part_acc, total;
+  size_t counters, items, part_ml, part_acc, total;
 };
 
-// merge counters are sized by num_q_heads (>= num_kv_heads), so the size needs no KV-head count
 WsLayout ws_layout(int64_t num_seqs, int64_t num_q_heads, int64_t head_dim, int64_t max_parts) {
   WsLayout L{};
   size_t o = 0;
   L.counters = o;
   o += 256;
-  L.merge_cnt = o;
-  o += align256(static_cast<size_t>(num_seqs * num_q_heads) * 4);
   L.items = o;
   o += align256(static_cast<size_t>(num_seqs * max_parts) * sizeof(pa::WorkItem));
   L.part_ml = o;
@@ -220,7 +217,6 @@ int pa_decode(void* out, const void* q, const void* k_cache, const void* v_cache
   p.out_dtype = out_dtype;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.counters = reinterpret_cast<unsigned int*>(ws + L.counters);
-  p.merge_cnt = reinterpret_cast<int*>(ws + L.merge_cnt);
   p.items = reinterpret_cast<pa::WorkItem*>(ws + L.items);
   p.part_ml = reinterpret_cast<float2*>(ws + L.part_ml);
   p.part_acc = reinterpret_cast<float*>(ws + L.part_acc);
@@ -238,7 +234,21 @@ int pa_decode(void* out, const void* q, const void* k_cache, const void* v_cache
   else
     rc = head_dim == 128 ? dispatch_kv<32, 128>(p, tmk, tmv, max_items, info, kv_dtype, qf32, 8, st)
                          : dispatch_kv<32, 64>(p, tmk, tmv, max_items, info, kv_dtype, qf32, 12, st);
-  return rc;
+  if (rc != PA_OK) return rc;
+  {  // merge kernel: waits (griddepcontrol.wait) for the partition kernel's partial results
+    const int64_t warps = static_cast<int64_t>(num_seqs) * num_q_heads;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>((warps + pa::kMergeWarps - 1) / pa::kMergeWarps));
+    cfg.blockDim = dim3(pa::kMergeWarps * 32);
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, pa::pa_decode_merge_kernel, p) != cudaSuccess) return PA_ERR_CUDA;
+  }
+  return cudaPeekAtLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
 int pa_reshape_and_cache(const void* k, const void* v, void* k_cache, void* v_cache, const int64_t* slot_mapping,

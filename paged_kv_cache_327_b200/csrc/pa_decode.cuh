@@ -7,8 +7,8 @@
 //
 // How (B200 design, not the page's one-CTA-per-(seq, head) scalar loop):
 //  * plan kernel (one CTA): turns seq_lens into a work list of (sequence, partition)
-//    pairs -- full 512-token partitions first, ragged tails last -- zeroes the work and
-//    merge counters, and writes the rows of empty or invalid sequences;
+//    pairs -- full 512-token partitions first, ragged tails last -- zeroes the work
+//    counter, and writes the rows of empty or invalid sequences;
 //  * partition kernel: persistent, one CTA per SM, NC consumer warps each fed by its own
 //    producer warp.  A work item is (sequence, partition, KV head), taken from an atomic
 //    counter.  The producer resolves the item's block-table entries and streams its
@@ -24,11 +24,12 @@
 //      O^T[D x G]   += V^T[D x tokens] . P^T[tokens x G]  (P^T via movmatrix.trans)
 //      l[G]         += 1^T . P^T                          (one more MMA, no shuffles)
 //    A sequence that fits one partition writes `out` directly.  Longer ones write the
-//    partition's (max, sum, unnormalised O); the warp that completes the last
-//    partition of a (sequence, KV head) merges them with the log-sum-exp rescale.
-// The partition boundaries depend only on seq_lens[i], each item is computed the same
-// way whatever warp runs it, and merges run in partition order, so results are
-// deterministic and batch-invariant.
+//    partition's (max, sum, unnormalised O) to the workspace and nothing else: no fence,
+//    atomic or merge ever stalls a consumer's page stream;
+//  * merge kernel: one warp per (sequence, query head) of a multi-partition sequence
+//    combines its partitions with the log-sum-exp rescale, in partition order.
+// The partition boundaries depend only on seq_lens[i] and each item is computed the same
+// way whatever warp runs it, so results are deterministic and batch-invariant.
 #pragma once
 
 #include <math_constants.h>
@@ -74,7 +75,6 @@ struct DecodeParams {
   float scale_log2;  // scale * log2(e)
   // workspace views
   unsigned int* counters;  // [0] next work item, [1] number of (sequence, partition) pairs
-  int* merge_cnt;          // [num_seqs * num_kv_heads]: partitions finished so far
   WorkItem* items;         // [num_seqs * max_parts]
   float2* part_ml;         // [num_seqs * max_parts * num_q_heads]: (max in log2 units, sum)
   float* part_acc;         // [num_seqs * max_parts * num_q_heads * head_dim]
@@ -129,7 +129,6 @@ __global__ void __launch_bounds__(kPlanThreads) pa_decode_plan_kernel(const Deco
   __shared__ int s_warp[33];
   const int N = p.num_seqs, P = p.partition_size;
   const int max_len = p.max_blocks_per_seq * p.block_size;
-  for (int i = threadIdx.x; i < N * p.num_kv_heads; i += blockDim.x) p.merge_cnt[i] = 0;
   int local = 0;
   for (int i = threadIdx.x; i < N; i += blockDim.x) {
     const int L = p.seq_lens[i];
@@ -241,48 +240,6 @@ __global__ void __launch_bounds__(DecodeCfg<BS, D, KT, QF32>::NWARP * 32, 1)
   pdl_wait();  // the plan kernel's work list and counters are visible from here on
 
   const int G = p.group, Hkv = p.num_kv_heads, Hq = p.num_q_heads;
-
-  // merge the np partitions of (seq, kvh): out = sum_k w_k O_k / sum_k w_k l_k, w_k = 2^(m_k - M)
-  auto merge = [&](int seq, int kvh, int np) {
-    const int64_t base = static_cast<int64_t>(seq) * p.max_parts;
-    for (int g = 0; g < G; ++g) {
-      const int hq = kvh * G + g;
-      float M = -CUDART_INF_F;
-      for (int k = lane; k < np; k += 32) M = fmaxf(M, __ldcg(&p.part_ml[(base + k) * Hq + hq].x));
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(FULL, M, o));
-      float den = 0.f;
-      for (int k = lane; k < np; k += 32) {
-        const float2 ml = __ldcg(&p.part_ml[(base + k) * Hq + hq]);
-        den += fast_exp2(ml.x - M) * ml.y;
-      }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(FULL, den, o);
-      constexpr int PER = D / 32;  // elements per lane
-      float num[PER];
-#pragma unroll
-      for (int e = 0; e < PER; ++e) num[e] = 0.f;
-      for (int k = 0; k < np; ++k) {
-        const float wk = fast_exp2(__ldcg(&p.part_ml[(base + k) * Hq + hq].x) - M);
-        const float* src = p.part_acc + ((base + k) * Hq + hq) * D + lane * PER;
-        if constexpr (PER == 4) {
-          const float4 a = __ldcg(reinterpret_cast<const float4*>(src));
-          num[0] += wk * a.x;
-          num[1] += wk * a.y;
-          num[2] += wk * a.z;
-          num[3] += wk * a.w;
-        } else {
-          const float2 a = __ldcg(reinterpret_cast<const float2*>(src));
-          num[0] += wk * a.x;
-          num[1] += wk * a.y;
-        }
-      }
-      const float inv = 1.f / den;
-      const int64_t o = (static_cast<int64_t>(seq) * Hq + hq) * D + lane * PER;
-#pragma unroll
-      for (int e = 0; e < PER; ++e) store_out(p.out, o + e, num[e] * inv, p.out_dtype);
-    }
-  };
 
   if (warp >= C::NC) {
     // ============================== producer ==============================
@@ -536,16 +493,6 @@ __global__ void __launch_bounds__(DecodeCfg<BS, D, KT, QF32>::NWARP * 32, 1)
       if (g0 < G) __stcg(&p.part_ml[pidx * Hq + hq0], poisoned ? make_float2(0.f, nan) : make_float2(mu0, l0));
       if (g1 < G) __stcg(&p.part_ml[pidx * Hq + hq1], poisoned ? make_float2(0.f, nan) : make_float2(mu1, l1));
     }
-    // the warp that completes the last partition of (seq, kvh) merges them
-    __threadfence();
-    __syncwarp();
-    int done = 0;
-    if (lane == 0) done = atomicAdd(&p.merge_cnt[seq * Hkv + kvh], 1);
-    done = __shfl_sync(FULL, done, 0);
-    if (done == np - 1) {
-      __threadfence();
-      merge(seq, kvh, np);
-    }
   };
 
   uint32_t n = 0;
@@ -580,6 +527,46 @@ __global__ void __launch_bounds__(DecodeCfg<BS, D, KT, QF32>::NWARP * 32, 1)
     record_error(DEV_TIMEOUT);
     *abort_flag = 1;
   }
+}
+
+// ------------------------------------------------------------------------------ merge
+// One warp per (sequence, query head) of a sequence with more than one partition:
+// out = sum_k 2^(m_k - M) O_k / sum_k 2^(m_k - M) l_k, M = max_k m_k, partitions in order.
+constexpr int kMergeWarps = 8;
+__global__ void __launch_bounds__(kMergeWarps * 32) pa_decode_merge_kernel(const DecodeParams p) {
+  pdl_wait();  // the partition kernel's partial results are visible from here on
+  const int lane = threadIdx.x & 31;
+  const int64_t pair = static_cast<int64_t>(blockIdx.x) * kMergeWarps + (threadIdx.x >> 5);
+  const int Hq = p.num_q_heads, D = p.head_dim, P = p.partition_size;
+  if (pair >= static_cast<int64_t>(p.num_seqs) * Hq) return;
+  const int seq = static_cast<int>(pair / Hq), hq = static_cast<int>(pair % Hq);
+  const int L = p.seq_lens[seq];
+  if (L <= P || L > p.max_blocks_per_seq * p.block_size) return;  // direct, empty or invalid rows
+  const int np = (L + P - 1) / P;
+  const int64_t base = static_cast<int64_t>(seq) * p.max_parts;
+  float M = -CUDART_INF_F;
+  for (int k = lane; k < np; k += 32) M = fmaxf(M, __ldcg(&p.part_ml[(base + k) * Hq + hq].x));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+  float num[4] = {0.f, 0.f, 0.f, 0.f}, den = 0.f;
+  const int per = D >> 5;  // 2 or 4 elements per lane
+#pragma unroll 4
+  for (int k = 0; k < np; ++k) {
+    const float2 ml = __ldcg(&p.part_ml[(base + k) * Hq + hq]);
+    const float* src = p.part_acc + ((base + k) * Hq + hq) * D + lane;
+    float a[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) a[j] = j < per ? __ldcg(src + 32 * j) : 0.f;
+    const float w = fast_exp2(ml.x - M);
+    den += w * ml.y;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) num[j] += w * a[j];
+  }
+  const float inv = 1.f / den;
+  const int64_t o = (static_cast<int64_t>(seq) * Hq + hq) * D + lane;
+#pragma unroll
+  for (int j = 0; j < 4; ++j)
+    if (j < per) store_out(p.out, o + 32 * j, num[j] * inv, p.out_dtype);
 }
 
 }  // namespace pa
