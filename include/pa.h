@@ -51,7 +51,9 @@ typedef enum {
   PA_ERR_INVALID = -1,     /* null pointer, bad size, misaligned pointer */
   PA_ERR_UNSUPPORTED = -2, /* valid but not implemented: head_dim, block_size, dtype mix, group size */
   PA_ERR_WORKSPACE = -3,   /* workspace missing or smaller than pa_decode_workspace_size() */
-  PA_ERR_CUDA = -4         /* a CUDA runtime call or kernel launch failed */
+  PA_ERR_CUDA = -4,        /* a CUDA runtime call or kernel launch failed */
+  PA_ERR_TOO_LARGE = -5    /* pa_decode_static_workspace: the call needs more scratch than
+                              PA_DECODE_STATIC_WORKSPACE_BYTES */
 } pa_status;
 
 /* codes returned by pa_get_device_error() */
@@ -134,6 +136,39 @@ PA_API int pa_get_device_error(void* stream);
 
 /* ABI version of this header (major * 100 + minor). */
 PA_API int pa_version(void);
+
+/* Size of the library's built-in decode scratch buffer used by pa_decode_static_workspace. */
+#define PA_DECODE_STATIC_WORKSPACE_BYTES (64ull << 20)
+
+/* pa_decode without a caller-provided workspace (the pages have no counterpart: this is
+ * an interface convenience, not part of the method).
+ *
+ * Who needs it: callers that cannot allocate device memory at the time they decode.  A
+ * serving engine typically hands almost all free HBM to its paged KV-cache pool at start-up
+ * (the pool is sized to a fraction of device memory), so a later cudaMalloc for scratch can
+ * fail or force the pool to shrink; a plugin embedded in a host framework may have no
+ * allocator of its own at all.  Such callers still pass the inputs and the output (exactly as
+ * for pa_decode, minus workspace / workspace_bytes); the scratch comes from one buffer of
+ * PA_DECODE_STATIC_WORKSPACE_BYTES (64 MiB) compiled into the library as a device global,
+ * which every GPU that loads the library holds until the process exits.
+ *
+ * Behaviour:
+ *   - The computation, arguments, layouts and results are those of pa_decode.
+ *   - A call whose workspace requirement, pa_decode_workspace_size(num_seqs, num_q_heads,
+ *     head_dim, max_blocks_per_seq * block_size, partition_size), exceeds
+ *     PA_DECODE_STATIC_WORKSPACE_BYTES returns PA_ERR_TOO_LARGE and launches nothing.
+ *   - The first call on each device looks up that device's address of the buffer (a host
+ *     runtime call); make that first call before any stream capture on the device.
+ *   - Nothing is allocated or freed, by this call or by anything it calls.
+ *   - All calls on a device share the one buffer and it keeps the previous call's contents;
+ *     what must start at zero is reset by the call itself.  Calls whose kernels can overlap
+ *     on the GPU (different streams, different host threads) race on the buffer: serialise
+ *     them, e.g. by issuing them on one stream. */
+PA_API int pa_decode_static_workspace(void* out, const void* q, const void* k_cache, const void* v_cache,
+                                      const int32_t* block_tables, const int32_t* seq_lens, int num_seqs,
+                                      int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                                      float scale, int max_blocks_per_seq, int64_t num_blocks, int q_dtype,
+                                      int kv_dtype, int out_dtype, int partition_size, void* stream);
 
 #ifdef __cplusplus
 }

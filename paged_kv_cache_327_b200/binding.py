@@ -23,7 +23,9 @@ PA_OK, PA_ERR_INVALID, PA_ERR_UNSUPPORTED, PA_ERR_WORKSPACE, PA_ERR_CUDA = 0, -1
 PA_DEV_OK, PA_DEV_BAD_BLOCK_ID, PA_DEV_BAD_SEQ_LEN, PA_DEV_BAD_SLOT, PA_DEV_BAD_PAIR, PA_DEV_TIMEOUT = range(6)
 
 EXPORTED = ("pa_decode_workspace_size", "pa_decode", "pa_reshape_and_cache", "pa_copy_blocks",
-            "pa_strerror", "pa_get_device_error", "pa_version")
+            "pa_strerror", "pa_get_device_error", "pa_version", "pa_decode_static_workspace")
+PA_ERR_TOO_LARGE = -5
+PA_DECODE_STATIC_WORKSPACE_BYTES = 64 << 20
 
 _TORCH_CODE = {torch.float32: PA_F32, torch.float16: PA_F16, torch.bfloat16: PA_BF16}
 _NAME_CODE = {"f32": PA_F32, "f16": PA_F16, "bf16": PA_BF16}
@@ -56,6 +58,8 @@ def load_library(path: str = _LIB_PATH):
     lib.pa_get_device_error.restype = I
     lib.pa_version.argtypes = []
     lib.pa_version.restype = I
+    lib.pa_decode_static_workspace.argtypes = [P, P, P, P, P, P, I, I, I, I, I, ctypes.c_float, I, I64, I, I, I, I, P]
+    lib.pa_decode_static_workspace.restype = I
     if path == _LIB_PATH:
         _lib = lib
     return lib
@@ -111,6 +115,32 @@ def pa_decode(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor, v_cache
         _TORCH_CODE[out.dtype], partition_size, _ptr(workspace), workspace.numel() * workspace.element_size(),
         _stream(stream))
     _check(rc, "pa_decode")
+
+
+def pa_decode_static_workspace(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                               block_tables: torch.Tensor, seq_lens: torch.Tensor, scale: float,
+                               partition_size: int = 0, stream=None) -> None:
+    """pa_decode with the library's built-in scratch buffer instead of a caller workspace.
+
+    For callers that cannot allocate device memory when they decode (for example when the
+    KV-cache pool already holds nearly all free HBM).  Raises PAError (PA_ERR_TOO_LARGE) when
+    the call needs more than PA_DECODE_STATIC_WORKSPACE_BYTES of scratch.  Calls that could
+    run concurrently on the GPU share that buffer and must be serialised (one stream).
+    """
+    N, Hq, D = q.shape
+    NB, bs, Hkv, D2 = k_cache.shape
+    if D2 != D or tuple(out.shape) != (N, Hq, D) or v_cache.shape != k_cache.shape:
+        raise ValueError("shape mismatch between q, out and the caches")
+    for t in (out, q, k_cache, v_cache, block_tables, seq_lens):
+        if not t.is_contiguous():
+            raise ValueError("tensors must be contiguous")
+    if block_tables.dtype != torch.int32 or seq_lens.dtype != torch.int32:
+        raise TypeError("block_tables and seq_lens must be int32")
+    rc = load_library().pa_decode_static_workspace(
+        _ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), _ptr(seq_lens), N, Hq, Hkv, D, bs,
+        ctypes.c_float(scale), block_tables.shape[1], NB, _TORCH_CODE[q.dtype], _TORCH_CODE[k_cache.dtype],
+        _TORCH_CODE[out.dtype], partition_size, _stream(stream))
+    _check(rc, "pa_decode_static_workspace")
 
 
 def pa_reshape_and_cache(k: torch.Tensor, v: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,

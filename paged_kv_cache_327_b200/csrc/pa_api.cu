@@ -148,6 +148,7 @@ const char* pa_strerror(int status) {
     case PA_ERR_UNSUPPORTED: return "unsupported configuration (head_dim, block_size, dtype or group size)";
     case PA_ERR_WORKSPACE: return "workspace missing or smaller than pa_decode_workspace_size()";
     case PA_ERR_CUDA: return "a CUDA runtime call or kernel launch failed";
+    case PA_ERR_TOO_LARGE: return "the call needs more scratch than the built-in 64 MiB decode buffer";
     default: return "unknown pa_status";
   }
 }
@@ -316,3 +317,46 @@ int pa_get_device_error(void* stream) {
 }
 
 }  // extern "C"
+
+// ------------------------------------------------------------------------------------------
+// pa_decode_static_workspace: pa_decode with its scratch in a device global of this file, for
+// callers that cannot allocate device memory when they decode (see include/pa.h).
+// ------------------------------------------------------------------------------------------
+static __device__ __align__(256) unsigned char g_pa_static_workspace[PA_DECODE_STATIC_WORKSPACE_BYTES];
+
+namespace {
+void* g_static_ws_addr[kMaxDevices];  // device address of g_pa_static_workspace, per device
+std::mutex g_static_ws_mu;
+}  // namespace
+
+extern "C" int pa_decode_static_workspace(void* out, const void* q, const void* k_cache, const void* v_cache,
+                                          const int32_t* block_tables, const int32_t* seq_lens, int num_seqs,
+                                          int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                                          float scale, int max_blocks_per_seq, int64_t num_blocks, int q_dtype,
+                                          int kv_dtype, int out_dtype, int partition_size, void* stream) {
+  // argument errors are reported by pa_decode itself; only the size limit is checked here
+  if (num_seqs > 0 && num_q_heads > 0 && head_dim > 0 && block_size > 0 && max_blocks_per_seq > 0 &&
+      partition_size >= 0) {
+    const int64_t max_len = static_cast<int64_t>(max_blocks_per_seq) * block_size;
+    if (max_len <= INT_MAX) {
+      const size_t need = pa_decode_workspace_size(num_seqs, num_q_heads, head_dim, static_cast<int>(max_len),
+                                                   partition_size);
+      if (need > PA_DECODE_STATIC_WORKSPACE_BYTES) return PA_ERR_TOO_LARGE;
+    }
+  }
+  void* ws = nullptr;
+  if (num_seqs > 0) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return PA_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_static_ws_mu);
+    if (!g_static_ws_addr[dev]) {  // once per device, with that device current
+      void* addr = nullptr;
+      if (cudaGetSymbolAddress(&addr, g_pa_static_workspace) != cudaSuccess || !addr) return PA_ERR_CUDA;
+      g_static_ws_addr[dev] = addr;
+    }
+    ws = g_static_ws_addr[dev];
+  }
+  return pa_decode(out, q, k_cache, v_cache, block_tables, seq_lens, num_seqs, num_q_heads, num_kv_heads, head_dim,
+                   block_size, scale, max_blocks_per_seq, num_blocks, q_dtype, kv_dtype, out_dtype, partition_size,
+                   ws, ws ? PA_DECODE_STATIC_WORKSPACE_BYTES : 0, stream);
+}
