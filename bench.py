@@ -75,6 +75,25 @@ def measured_peak():
         return FALLBACK_HBM_GBS, "fallback 6.65 TB/s (no MEASURED_PEAKS.json)"
 
 
+def rank_seed(config: str, rank: int) -> int:
+    """Each replica decodes its own batch: the config's seed offset by the rank."""
+    return W.config_seed(config) + 1000 * rank
+
+
+def max_over_ranks(x: float, dist=None, device="cpu") -> float:
+    """The slowest rank's value (time is taken as the max over ranks); identity without a group."""
+    if dist is None:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(bytes_per_rank: int, world: int, seconds: float) -> float:
+    """Whole-job GB/s: every rank processes bytes_per_rank in `seconds` (the max over ranks)."""
+    return world * bytes_per_rank / seconds / 1e9
+
+
 def sources_digest():
     h = hashlib.sha256()
     for rel in KERNEL_SOURCES:
@@ -241,7 +260,7 @@ def run_ours(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
 
-    seed = W.config_seed(args.config) + 1000 * rank
+    seed = rank_seed(args.config, rank)
     extra = {"num_seqs": args.num_seqs} if args.num_seqs else {}
     w = W.make_config(args.config, block_size=args.block_size, seed=seed, **extra)
     out_dtype = args.out_dtype or w.q_dtype
@@ -296,10 +315,7 @@ def run_ours(args):
     dec_ms = [a.elapsed_time(b) for a, b in ev_dec]
     if clocks:
         clocks.mark(wall0, wall1)
-    if dist:
-        t = torch.tensor([elapsed_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
+    elapsed_ms = max_over_ranks(elapsed_ms, dist, "cuda")
     if B.pa_get_device_error() != B.PA_DEV_OK:
         raise RuntimeError("device error during the timed region")
 
@@ -339,10 +355,7 @@ def run_ours(args):
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1) / e2e_steps
-    if dist:
-        t = torch.tensor([e2e_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e2e_ms, dist, "cuda")
 
     clock_info = clocks.stop() if clocks else None
 
@@ -367,7 +380,7 @@ def run_ours(args):
         return 0
 
     ms_step = elapsed_ms / args.steps
-    value = world * kv_bytes / (ms_step * 1e-3) / 1e9
+    value = job_throughput(kv_bytes, world, ms_step * 1e-3)
     peak, peak_src = measured_peak()
     dec_mean = float(np.mean(dec_ms))
     achieved = decode_bytes / (dec_mean * 1e-3) / 1e9
@@ -389,7 +402,7 @@ def run_ours(args):
                          f"timed loop", "parallelism": f"replicas x{world}" if world > 1 else "1 GPU"},
         "seq_tokens_per_s": round(world * w.total_tokens() / (ms_step * 1e-3), 1),
         "pct_of_hbm_peak": round(100 * value / world / peak, 2),
-        "e2e": {"value": round(world * kv_bytes / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+        "e2e": {"value": round(job_throughput(kv_bytes, world, e2e_ms * 1e-3), 2), "unit": "GB/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 5)},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "traffic": recorded_traffic(args.config),
