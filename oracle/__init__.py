@@ -14,6 +14,9 @@ What each function follows (web pages on vLLM / PagedAttention):
     stores each new token's K/V into its slot before attention runs).
   * ``copy_blocks`` -- "详解vLLM推理引擎架构", section "Copy-on-Write 与内存共享"
     (copy_block(old, new) before writing a shared block).
+  * ``reshape_and_cache_e4m3`` / ``decode(..., kv_dtype="e4m3")`` -- the FP8 KV cache of
+    "详解vLLM推理引擎架构", section "量化集成与部署" (--kv-cache-dtype fp8), read as OCP E4M3
+    codes with one fp32 scale for K and one for V.
 
 Every function is pinned in ``tests/test_oracle_pins.py`` against things other
 than itself: the pages' block-table example, closed forms, torch's
@@ -28,8 +31,8 @@ import numpy as np
 
 from . import build as _build
 
-DTYPES = {"f32": 0, "f16": 1, "bf16": 2}
-ELEM_BYTES = {"f32": 4, "f16": 2, "bf16": 2}
+DTYPES = {"f32": 0, "f16": 1, "bf16": 2, "e4m3": 3}
+ELEM_BYTES = {"f32": 4, "f16": 2, "bf16": 2, "e4m3": 1}
 
 _lib = None
 
@@ -51,6 +54,16 @@ def _load(path=None):
     lib.oracle_reshape_and_cache.restype = i32
     lib.oracle_copy_blocks.argtypes = [P, P, P, i64, i64, i64]
     lib.oracle_copy_blocks.restype = i32
+    lib.oracle_decode_scaled.argtypes = [P, P, i32, P, P, i32, P, P, i32, i32, i32, i32, i32, i32, i64,
+                                         ctypes.c_float, ctypes.c_float, ctypes.c_float, i32]
+    lib.oracle_decode_scaled.restype = i32
+    lib.oracle_reshape_and_cache_e4m3.argtypes = [P, P, P, P, P, i64, i32, i32, i32, i64, i32,
+                                                  ctypes.c_float, ctypes.c_float, i64, i64]
+    lib.oracle_reshape_and_cache_e4m3.restype = i32
+    lib.oracle_e4m3_to_f64.argtypes = [ctypes.c_uint8]
+    lib.oracle_e4m3_to_f64.restype = ctypes.c_double
+    lib.oracle_f32_to_e4m3.argtypes = [ctypes.c_float]
+    lib.oracle_f32_to_e4m3.restype = ctypes.c_uint8
     lib.oracle_f16_to_f64.argtypes = [ctypes.c_uint16]
     lib.oracle_f16_to_f64.restype = ctypes.c_double
     lib.oracle_bf16_to_f64.argtypes = [ctypes.c_uint16]
@@ -69,7 +82,7 @@ def _ptr(a: np.ndarray):
 
 
 def _check_storage(a: np.ndarray, dtype: str, name: str):
-    want = np.float32 if dtype == "f32" else np.uint16
+    want = {"f32": np.float32, "e4m3": np.uint8}.get(dtype, np.uint16)
     if a.dtype != want:
         raise TypeError(f"{name}: {dtype} data must be stored as {np.dtype(want)}, got {a.dtype}")
     if not a.flags.c_contiguous:
@@ -84,12 +97,13 @@ def default_threads() -> int:
 
 
 def decode(q, q_dtype, k_cache, v_cache, kv_dtype, block_tables, seq_lens, scale,
-           num_threads=None, lib=None):
+           num_threads=None, lib=None, k_scale=1.0, v_scale=1.0):
     """fp64 paged decode attention.
 
     q: [N, Hq, D] (float32 for "f32", uint16 bit patterns for "f16"/"bf16");
-    k_cache, v_cache: [NB, bs, Hkv, D] in kv_dtype storage; block_tables int32
-    [N, MB]; seq_lens int32 [N].  Returns float64 [N, Hq, D].
+    k_cache, v_cache: [NB, bs, Hkv, D] in kv_dtype storage (uint8 codes for "e4m3", whose
+    values are code * k_scale and code * v_scale); block_tables int32 [N, MB]; seq_lens
+    int32 [N].  Returns float64 [N, Hq, D].
     """
     lib = lib or _load()
     _check_storage(q, q_dtype, "q")
@@ -105,10 +119,16 @@ def decode(q, q_dtype, k_cache, v_cache, kv_dtype, block_tables, seq_lens, scale
         raise ValueError("block_tables must be [N, MB] and seq_lens [N]")
     MB = block_tables.shape[1]
     out = np.zeros((N, Hq, D), dtype=np.float64)
-    rc = lib.oracle_decode(_ptr(out), _ptr(q), DTYPES[q_dtype], _ptr(k_cache), _ptr(v_cache),
-                           DTYPES[kv_dtype], _ptr(block_tables), _ptr(seq_lens), N, Hq, Hkv, D, bs,
-                           MB, NB, ctypes.c_float(scale),
-                           num_threads if num_threads else default_threads())
+    threads = num_threads if num_threads else default_threads()
+    if kv_dtype == "e4m3":
+        rc = lib.oracle_decode_scaled(_ptr(out), _ptr(q), DTYPES[q_dtype], _ptr(k_cache), _ptr(v_cache),
+                                      DTYPES[kv_dtype], _ptr(block_tables), _ptr(seq_lens), N, Hq, Hkv, D, bs,
+                                      MB, NB, ctypes.c_float(scale), ctypes.c_float(k_scale),
+                                      ctypes.c_float(v_scale), threads)
+    else:
+        rc = lib.oracle_decode(_ptr(out), _ptr(q), DTYPES[q_dtype], _ptr(k_cache), _ptr(v_cache),
+                               DTYPES[kv_dtype], _ptr(block_tables), _ptr(seq_lens), N, Hq, Hkv, D, bs,
+                               MB, NB, ctypes.c_float(scale), threads)
     if rc != 0:
         raise OracleError(f"oracle_decode failed with status {rc}")
     return out
@@ -131,6 +151,26 @@ def reshape_and_cache(k, v, k_cache, v_cache, slot_mapping, kv_dtype, lib=None):
         raise OracleError(f"oracle_reshape_and_cache failed with status {rc}")
 
 
+def reshape_and_cache_e4m3(k, v, k_cache, v_cache, slot_mapping, in_dtype, k_scale, v_scale, lib=None):
+    """In place: quantise token t's K/V rows ([T, Hkv, D], in_dtype) to E4M3 codes
+    e4m3(x / scale) at slot slot_mapping[t] of the uint8 caches (skip if < 0)."""
+    lib = lib or _load()
+    _check_storage(k, in_dtype, "k")
+    _check_storage(v, in_dtype, "v")
+    _check_storage(k_cache, "e4m3", "k_cache")
+    _check_storage(v_cache, "e4m3", "v_cache")
+    slot_mapping = np.ascontiguousarray(slot_mapping, dtype=np.int64)
+    T, Hkv, D = k.shape
+    NB, bs, Hkv2, D2 = k_cache.shape
+    if (Hkv2, D2) != (Hkv, D) or v.shape != k.shape or slot_mapping.shape != (T,):
+        raise ValueError("shape mismatch")
+    rc = lib.oracle_reshape_and_cache_e4m3(_ptr(k), _ptr(v), _ptr(k_cache), _ptr(v_cache), _ptr(slot_mapping),
+                                           T, Hkv, D, bs, NB, DTYPES[in_dtype], ctypes.c_float(k_scale),
+                                           ctypes.c_float(v_scale), Hkv * D, Hkv * D)
+    if rc != 0:
+        raise OracleError(f"oracle_reshape_and_cache_e4m3 failed with status {rc}")
+
+
 def copy_blocks(k_cache, v_cache, pairs, lib=None):
     """In place: for each (src, dst) row of pairs, in order, copy physical block src to dst."""
     lib = lib or _load()
@@ -151,3 +191,11 @@ def f16_to_f64(bits: int) -> float:
 
 def bf16_to_f64(bits: int) -> float:
     return _load().oracle_bf16_to_f64(bits)
+
+
+def e4m3_to_f64(code: int) -> float:
+    return _load().oracle_e4m3_to_f64(code)
+
+
+def f32_to_e4m3(x: float) -> int:
+    return int(_load().oracle_f32_to_e4m3(x))

@@ -23,6 +23,9 @@
  *    scale * sum_d q[d]*k[d] and the result is softmax(scores) applied to V.
  *  - "vLLM 深度解读", section 7 (Llama attention): new K/V are stored into the
  *    paged cache before attention runs, so the context includes the new token.
+ *  - "详解vLLM推理引擎架构", section "量化集成与部署": the KV cache may be stored in FP8
+ *    (--kv-cache-dtype fp8).  The page names no format; read here as OCP E4M3 with one
+ *    fp32 scale for K and one for V: stored code = e4m3(x / scale), value = code * scale.
  *
  * Readings where the pages are silent or inconsistent:
  *  - the printed kernel indexes K with the query head although it receives
@@ -40,7 +43,7 @@
 #include <stdlib.h>
 #include <string.h>
 
-enum { OR_F32 = 0, OR_F16 = 1, OR_BF16 = 2 };
+enum { OR_F32 = 0, OR_F16 = 1, OR_BF16 = 2, OR_E4M3 = 3 };
 
 enum {
   OR_OK = 0,
@@ -75,10 +78,47 @@ double oracle_bf16_to_f64(uint16_t b) {
   return (double)f;
 }
 
+/* FP8 E4M3 (the OCP "e4m3fn" format) -> double, from the format's definition:
+ * 1 sign bit, 4 exponent bits (bias 7), 3 fraction bits; exponent 0 encodes subnormals
+ * m * 2^-9; there is no infinity and S.1111.111 is NaN; the largest finite value is 448. */
+double oracle_e4m3_to_f64(uint8_t c) {
+  int sign = (c >> 7) & 1;
+  int e = (c >> 3) & 0xf;
+  int m = c & 7;
+  double v;
+  if (e == 15 && m == 7) return NAN;
+  if (e == 0) v = ldexp((double)m, -9);
+  else v = ldexp((double)(8 + m), e - 10);
+  return sign ? -v : v;
+}
+
+/* float -> FP8 E4M3: round to nearest, ties to even, saturating to +-448; NaN -> 0x7f.
+ * The value is scaled to an integer count of the quantum of its binade (2^-9 below 2^-6,
+ * otherwise 2^(exponent - 3)) and rounded with rint (default rounding: ties to even); a
+ * count of 16 carries into the next binade, which the code layout does by itself. */
+uint8_t oracle_f32_to_e4m3(float x) {
+  if (isnan(x)) return 0x7f;
+  uint8_t sign = signbit(x) ? 0x80 : 0;
+  double a = fabs((double)x);
+  if (a > 448.0) return sign | 0x7e;
+  if (a == 0.0) return sign;
+  int E;
+  frexp(a, &E);              /* a = f * 2^E, f in [0.5, 1): a's binade is 2^(E-1) */
+  int code;
+  if (E - 1 < -6) {
+    code = (int)rint(a / ldexp(1.0, -9));                 /* subnormal quantum 2^-9 */
+  } else {
+    int q = (int)rint(a / ldexp(1.0, E - 1 - 3));        /* 8 <= q <= 16 */
+    code = ((E - 1 + 7) << 3) + (q - 8);
+  }
+  return sign | (uint8_t)code;
+}
+
 static double load_elem(const void* base, int64_t idx, int dtype) {
   switch (dtype) {
     case OR_F32: return (double)((const float*)base)[idx];
     case OR_F16: return oracle_f16_to_f64(((const uint16_t*)base)[idx]);
+    case OR_E4M3: return oracle_e4m3_to_f64(((const uint8_t*)base)[idx]);
     default:     return oracle_bf16_to_f64(((const uint16_t*)base)[idx]);
   }
 }
@@ -131,6 +171,39 @@ int oracle_reshape_and_cache(const uint8_t* k, const uint8_t* v, uint8_t* k_cach
   return OR_OK;
 }
 
+/* reshape_and_cache into an FP8 E4M3 cache with per-tensor scales: each element x of the
+ * new token (in_dtype f32 / f16 / bf16) is stored as e4m3(x / scale), the division done
+ * in fp32 (round to nearest); the slot rule is the one of oracle_reshape_and_cache. */
+int oracle_reshape_and_cache_e4m3(const void* k, const void* v, uint8_t* k_cache, uint8_t* v_cache,
+                                  const int64_t* slot_mapping, int64_t num_tokens, int num_kv_heads,
+                                  int head_dim, int block_size, int64_t num_blocks, int in_dtype,
+                                  float k_scale, float v_scale, int64_t k_token_stride,
+                                  int64_t v_token_stride) {
+  if (num_tokens < 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 || num_blocks <= 0)
+    return OR_ERR_ARG;
+  if (in_dtype < OR_F32 || in_dtype > OR_BF16) return OR_ERR_ARG;
+  if (num_tokens > 0 && (!k || !v || !k_cache || !v_cache || !slot_mapping)) return OR_ERR_ARG;
+  for (int64_t t = 0; t < num_tokens; ++t)
+    if (slot_mapping[t] >= num_blocks * block_size) return OR_ERR_RANGE;
+  for (int64_t t = 0; t < num_tokens; ++t) {
+    int64_t s = slot_mapping[t];
+    if (s < 0) continue;
+    int64_t blk = s / block_size, pos = s % block_size;
+    for (int h = 0; h < num_kv_heads; ++h) {
+      int64_t dst = ((blk * block_size + pos) * num_kv_heads + h) * head_dim;
+      for (int d = 0; d < head_dim; ++d) {
+        float xk = (float)load_elem(k, t * k_token_stride + (int64_t)h * head_dim + d, in_dtype);
+        float xv = (float)load_elem(v, t * v_token_stride + (int64_t)h * head_dim + d, in_dtype);
+        float qk = xk / k_scale;
+        float qv = xv / v_scale;
+        k_cache[dst + d] = oracle_f32_to_e4m3(qk);
+        v_cache[dst + d] = oracle_f32_to_e4m3(qv);
+      }
+    }
+  }
+  return OR_OK;
+}
+
 typedef struct {
   double* out;
   const void* q;
@@ -142,6 +215,7 @@ typedef struct {
   const int32_t* seq_lens;
   int num_q_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq;
   double scale;
+  double k_scale, v_scale;   /* dequantisation scales of an E4M3 cache (1 otherwise) */
   int seq_begin, seq_end;
   int status;
 } decode_job;
@@ -184,6 +258,7 @@ static void* decode_worker(void* arg) {
         for (int d = 0; d < D; ++d)
           s += load_elem(J->q, qo + d, J->q_dtype) *
                load_elem(J->k_cache, kv_offset(table, t, h, d, J->block_size, J->num_kv_heads, D), J->kv_dtype);
+        if (J->kv_dtype == OR_E4M3) s *= J->k_scale;   /* K_t = code * k_scale */
         s *= J->scale;
         scores[t] = s;
         if (s > m) m = s;
@@ -197,6 +272,8 @@ static void* decode_worker(void* arg) {
           o[d] += w * load_elem(J->v_cache, kv_offset(table, t, h, d, J->block_size, J->num_kv_heads, D), J->kv_dtype);
       }
       for (int d = 0; d < D; ++d) o[d] /= z;
+      if (J->kv_dtype == OR_E4M3)                      /* V_t = code * v_scale */
+        for (int d = 0; d < D; ++d) o[d] *= J->v_scale;
     }
   }
   free(scores);
@@ -208,16 +285,34 @@ static void* decode_worker(void* arg) {
  * out is fp64 [num_seqs, num_q_heads, head_dim].  Sequences are split across
  * num_threads POSIX threads; each output element is computed by one thread in
  * the same order whatever the thread count. */
+int oracle_decode_scaled(double* out, const void* q, int q_dtype, const void* k_cache,
+                         const void* v_cache, int kv_dtype, const int32_t* block_tables,
+                         const int32_t* seq_lens, int num_seqs, int num_q_heads, int num_kv_heads,
+                         int head_dim, int block_size, int max_blocks_per_seq, int64_t num_blocks,
+                         float scale, float k_scale, float v_scale, int num_threads);
+
 int oracle_decode(double* out, const void* q, int q_dtype, const void* k_cache,
                   const void* v_cache, int kv_dtype, const int32_t* block_tables,
                   const int32_t* seq_lens, int num_seqs, int num_q_heads, int num_kv_heads,
                   int head_dim, int block_size, int max_blocks_per_seq, int64_t num_blocks,
                   float scale, int num_threads) {
+  return oracle_decode_scaled(out, q, q_dtype, k_cache, v_cache, kv_dtype, block_tables, seq_lens,
+                              num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
+                              max_blocks_per_seq, num_blocks, scale, 1.0f, 1.0f, num_threads);
+}
+
+/* Decode attention over a cache of any element type; for an E4M3 cache the stored codes are
+ * multiplied by k_scale (keys) and v_scale (values) -- the scales are ignored otherwise. */
+int oracle_decode_scaled(double* out, const void* q, int q_dtype, const void* k_cache,
+                         const void* v_cache, int kv_dtype, const int32_t* block_tables,
+                         const int32_t* seq_lens, int num_seqs, int num_q_heads, int num_kv_heads,
+                         int head_dim, int block_size, int max_blocks_per_seq, int64_t num_blocks,
+                         float scale, float k_scale, float v_scale, int num_threads) {
   if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 ||
       max_blocks_per_seq < 0 || num_blocks <= 0)
     return OR_ERR_ARG;
   if (num_q_heads % num_kv_heads) return OR_ERR_ARG;
-  if (q_dtype < OR_F32 || q_dtype > OR_BF16 || kv_dtype < OR_F32 || kv_dtype > OR_BF16) return OR_ERR_ARG;
+  if (q_dtype < OR_F32 || q_dtype > OR_BF16 || kv_dtype < OR_F32 || kv_dtype > OR_E4M3) return OR_ERR_ARG;
   if (num_seqs == 0) return OR_OK;
   if (!out || !q || !k_cache || !v_cache || !block_tables || !seq_lens) return OR_ERR_ARG;
   /* every block the definition will touch must exist */
@@ -242,6 +337,8 @@ int oracle_decode(double* out, const void* q, int q_dtype, const void* k_cache,
     J->num_q_heads = num_q_heads; J->num_kv_heads = num_kv_heads; J->head_dim = head_dim;
     J->block_size = block_size; J->max_blocks_per_seq = max_blocks_per_seq;
     J->scale = (double)scale;
+    J->k_scale = (double)k_scale;
+    J->v_scale = (double)v_scale;
     J->seq_begin = (int)((int64_t)num_seqs * w / num_threads);
     J->seq_end = (int)((int64_t)num_seqs * (w + 1) / num_threads);
     J->status = OR_OK;

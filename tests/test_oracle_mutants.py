@@ -35,12 +35,23 @@ MUTANTS = {
     "f16_hidden_bit": ("ldexp((double)(m + 1024), e - 25)", "ldexp((double)(m + 512), e - 25)"),
     "bf16_shift": ("uint32_t u = (uint32_t)b << 16;", "uint32_t u = (uint32_t)b << 15;"),
     "reshape_block_pos_swapped": ("int64_t blk = s / block_size, pos = s % block_size;",
-                                  "int64_t blk = s % block_size, pos = s / block_size;"),
-    "reshape_negative_slot_written": ("if (s < 0) continue;", "if (s < 0) s = 0;"),
+                                  "int64_t blk = s % block_size, pos = s / block_size;", 0),
+    "reshape_negative_slot_written": ("if (s < 0) continue;", "if (s < 0) s = 0;", 0),
+    "e4m3_store_block_pos_swapped": ("int64_t blk = s / block_size, pos = s % block_size;",
+                                     "int64_t blk = s % block_size, pos = s / block_size;", 1),
+    "e4m3_store_negative_slot_written": ("if (s < 0) continue;", "if (s < 0) s = 0;", 1),
     "reshape_ignores_head": ("k + (t * k_token_stride + (int64_t)h * head_dim) * elem_bytes",
                              "k + (t * k_token_stride) * elem_bytes"),
     "copy_direction": ("memmove(k_cache + dst * block_bytes, k_cache + src * block_bytes",
                        "memmove(k_cache + src * block_bytes, k_cache + dst * block_bytes"),
+    "e4m3_bias": ("else v = ldexp((double)(8 + m), e - 10);", "else v = ldexp((double)(8 + m), e - 9);"),
+    "e4m3_nan_rule": ("if (e == 15 && m == 7) return NAN;", "if (e == 15) return NAN;"),
+    "e4m3_truncates": ("int q = (int)rint(a / ldexp(1.0, E - 1 - 3));", "int q = (int)floor(a / ldexp(1.0, E - 1 - 3));"),
+    "e4m3_no_saturation": ("if (a > 448.0) return sign | 0x7e;", "if (a > 448.0) return sign | 0x7f;"),
+    "e4m3_subnormal_quantum": ("code = (int)rint(a / ldexp(1.0, -9));", "code = (int)rint(a / ldexp(1.0, -10));"),
+    "e4m3_store_multiplies": ("float qk = xk / k_scale;", "float qk = xk * k_scale;"),
+    "e4m3_k_scale_dropped": ("if (J->kv_dtype == OR_E4M3) s *= J->k_scale;", ""),
+    "e4m3_v_scale_dropped": ("for (int d = 0; d < D; ++d) o[d] *= J->v_scale;", ";"),
     "copy_skips_v": ("    memmove(v_cache + dst * block_bytes, v_cache + src * block_bytes, (size_t)block_bytes);\n",
                      ""),
 }
@@ -64,11 +75,18 @@ sys.exit(1 if failed else 0)
 
 @pytest.mark.parametrize("name", sorted(MUTANTS))
 def test_pins_catch_mutant(name, tmp_path):
-    find, repl = MUTANTS[name]
+    find, repl, *which = MUTANTS[name]
     src = open(SRC, encoding="utf-8").read()
-    assert src.count(find) == 1, f"mutant {name}: pattern must occur exactly once"
+    if which:  # the pattern occurs more than once: mutate the given occurrence only
+        idx = -1
+        for _ in range(which[0] + 1):
+            idx = src.index(find, idx + 1)
+        mutated = src[:idx] + repl + src[idx + len(find):]
+    else:
+        assert src.count(find) == 1, f"mutant {name}: pattern must occur exactly once"
+        mutated = src.replace(find, repl)
     mutant_c = tmp_path / f"{name}.c"
-    mutant_c.write_text(src.replace(find, repl), encoding="utf-8")
+    mutant_c.write_text(mutated, encoding="utf-8")
     lib = tmp_path / f"{name}.so"
     subprocess.run(["gcc", "-std=c11", "-O2", "-fPIC", "-shared", "-pthread", "-D_GNU_SOURCE",
                     str(mutant_c), "-o", str(lib), "-lm"], check=True)

@@ -311,9 +311,116 @@ def check_copy_blocks(lib):
     assert np.array_equal(kc, ek) and np.array_equal(vc, ev)
 
 
+# ------------------------------------------------------------------ FP8 (E4M3) KV cache
+E4M3_FINITE = [c for c in range(256) if (c & 0x7f) != 0x7f]
+
+
+def _e4m3_values():
+    return torch.arange(256, dtype=torch.int32).to(torch.uint8).view(torch.float8_e4m3fn).double().numpy()
+
+
+def brute_force_e4m3(x: float) -> int:
+    """Nearest finite E4M3 code by exhaustive search; ties to the even code; |x| > 448 saturates."""
+    vals = _e4m3_values()
+    if abs(x) > 448.0:
+        return 0xFE if x < 0 else 0x7E
+    best, bd = None, None
+    for c in E4M3_FINITE:
+        if (c >> 7) != (1 if math.copysign(1.0, x) < 0 else 0):
+            continue
+        d = abs(float(vals[c]) - x)
+        if bd is None or d < bd or (d == bd and (c & 1) == 0 and (best & 1) == 1):
+            best, bd = c, d
+    return best
+
+
+def check_e4m3_decode(lib):
+    ref = _e4m3_values()
+    got = np.array([lib.oracle_e4m3_to_f64(c) for c in range(256)])
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(got), nan) and np.array_equal(got[~nan], ref[~nan])
+    assert lib.oracle_e4m3_to_f64(0x7E) == 448.0 and lib.oracle_e4m3_to_f64(0x01) == 2.0 ** -9
+
+
+def check_e4m3_encode(lib):
+    rng = _rng(71)
+    vals = _e4m3_values()
+    pos = np.sort(np.unique(vals[[c for c in E4M3_FINITE if c < 0x80]]))
+    mids = ((pos[1:] + pos[:-1]) / 2).astype(np.float32)      # exact ties between neighbours
+    xs = np.concatenate([rng.standard_normal(300).astype(np.float32) * 10 ** rng.uniform(-3, 2.5, 300).astype(np.float32),
+                         mids, -mids, pos.astype(np.float32), np.float32([0.0, -0.0, 447.9, 448.0, 449.0, 460.0,
+                                                                          465.0, 1e6, -1e6, 2.0 ** -10, 2.0 ** -11])])
+    for x in xs:
+        got = lib.oracle_f32_to_e4m3(ctypes_float(x))
+        want = brute_force_e4m3(float(x))
+        assert got == want, (float(x), got, want)
+    # in range, torch's round-to-nearest-even cast agrees
+    inr = xs[np.abs(xs) <= 448]
+    t = torch.from_numpy(inr).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    got = np.array([lib.oracle_f32_to_e4m3(ctypes_float(x)) for x in inr], dtype=np.uint8)
+    assert np.array_equal(got, t)
+
+
+def ctypes_float(x):
+    import ctypes
+    return ctypes.c_float(float(x))
+
+
+def check_reshape_and_cache_e4m3(lib):
+    rng = _rng(72)
+    NB, bs, H, D, T = 5, 16, 2, 64, 12
+    for in_dt in ("bf16", "f16", "f32"):
+        kc = rng.integers(0, 256, size=(NB, bs, H, D), dtype=np.uint8)
+        vc = rng.integers(0, 256, size=(NB, bs, H, D), dtype=np.uint8)
+        k = W.to_storage(rng.standard_normal((T, H, D), dtype=np.float32) * 3, in_dt)
+        v = W.to_storage(rng.standard_normal((T, H, D), dtype=np.float32) * 3, in_dt)
+        ks, vs = np.float32(0.0371), np.float32(0.0459)   # |x / scale| stays below 448
+        slots = rng.choice(NB * bs, size=T, replace=False).astype(np.int64)
+        slots[4] = -1
+        ek, ev = kc.copy(), vc.copy()
+        keep = slots >= 0
+        qk = (torch.from_numpy(W.storage_to_f32(k, in_dt)) / torch.tensor(ks)).to(torch.float8_e4m3fn)
+        qv = (torch.from_numpy(W.storage_to_f32(v, in_dt)) / torch.tensor(vs)).to(torch.float8_e4m3fn)
+        ek.reshape(NB * bs, H, D)[slots[keep]] = qk.view(torch.uint8).numpy()[keep]
+        ev.reshape(NB * bs, H, D)[slots[keep]] = qv.view(torch.uint8).numpy()[keep]
+        oracle.reshape_and_cache_e4m3(k, v, kc, vc, slots, in_dt, float(ks), float(vs), lib=lib)
+        assert np.array_equal(kc, ek) and np.array_equal(vc, ev), in_dt
+
+
+def check_decode_e4m3_vs_sdpa(lib):
+    rng = _rng(73)
+    for n, (lens, Hq, Hkv, D, bs, qd) in enumerate([([40, 1, 77], 8, 2, 128, 16, "bf16"),
+                                                     ([33, 130], 4, 4, 64, 32, "f32")]):
+        ks, vs = 0.0123, 0.0211
+        codes_k = [rng.choice(E4M3_FINITE, size=(L, Hkv, D)).astype(np.uint8) for L in lens]
+        codes_v = [rng.choice(E4M3_FINITE, size=(L, Hkv, D)).astype(np.uint8) for L in lens]
+        vals = _e4m3_values()
+        Ks = [vals[c] * np.float64(np.float32(ks)) for c in codes_k]
+        Vs = [vals[c] * np.float64(np.float32(vs)) for c in codes_v]
+        NB = sum(-(-L // bs) for L in lens) + 2
+        kc = np.zeros((NB, bs, Hkv, D), np.uint8)
+        vc = np.zeros_like(kc)
+        perm = list(_rng(74 + n).permutation(NB))
+        bt = np.full((len(lens), max(-(-L // bs) for L in lens)), -1, np.int32)
+        for i, L in enumerate(lens):
+            for b in range(-(-L // bs)):
+                phys = perm.pop(0)
+                bt[i, b] = phys
+                m = min(bs, L - b * bs)
+                kc[phys, :m] = codes_k[i][b * bs:b * bs + m]
+                vc[phys, :m] = codes_v[i][b * bs:b * bs + m]
+        q32 = W.storage_to_f32(W.to_storage(rng.standard_normal((len(lens), Hq, D), dtype=np.float32), qd), qd)
+        scale = float(np.float32(1 / math.sqrt(D)))
+        got = oracle.decode(W.to_storage(q32, qd), qd, kc, vc, "e4m3", bt, np.asarray(lens, np.int32), scale,
+                            lib=lib, k_scale=ks, v_scale=vs)
+        ref = sdpa_reference(q32, Ks, Vs, scale, Hq // Hkv)
+        assert np.max(np.abs(got - ref)) < 1e-12, n
+
+
 ALL_CHECKS = [check_f16_decode, check_bf16_decode, check_decode_vs_sdpa, check_closed_forms,
               check_page_block_table_example, check_invariants, check_cow_leaves_parent,
-              check_reshape_and_cache, check_copy_blocks]
+              check_reshape_and_cache, check_copy_blocks, check_e4m3_decode, check_e4m3_encode,
+              check_reshape_and_cache_e4m3, check_decode_e4m3_vs_sdpa]
 
 
 @pytest.fixture(scope="module")
