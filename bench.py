@@ -55,6 +55,8 @@ def parse_args():
     ap.add_argument("--num-seqs", type=int, default=None, help="smaller batch of the same config (profiling)")
     ap.add_argument("--partition-size", type=int, default=0)
     ap.add_argument("--out-dtype", default=None, help="f32 | f16 | bf16 (default: the query dtype)")
+    ap.add_argument("--kv-dtype", default=None, choices=["e4m3"],
+                    help="e4m3: the same config over an FP8 KV cache (per-tensor K/V scales)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target oracle time for cpu_baseline")
     ap.add_argument("--ref-seconds", type=float, default=150.0, help="target total time of --impl reference")
@@ -62,8 +64,9 @@ def parse_args():
 
 
 def workload_label(w: W.Workload) -> str:
+    kv = w.kv_dtype if w.kv_dtype != "e4m3" else f"e4m3 (scales {w.k_scale:.4g}/{w.v_scale:.4g}, new tokens {w.new_kv_dtype})"
     return (f"{w.name}: {w.num_seqs} seqs, {w.num_q_heads}/{w.num_kv_heads} heads, head_dim {w.head_dim}, "
-            f"block {w.block_size}, {w.notes.get('lens', '')}, q {w.q_dtype}, kv {w.kv_dtype}")
+            f"block {w.block_size}, {w.notes.get('lens', '')}, q {w.q_dtype}, kv {kv}")
 
 
 def measured_peak():
@@ -173,6 +176,19 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(loaded)}
 
 
+def oracle_post_step(w: W.Workload):
+    """The cache state after the step, by the oracle's own cache operations."""
+    import oracle
+
+    kc, vc = w.k_cache.copy(), w.v_cache.copy()
+    oracle.copy_blocks(kc, vc, w.copy_pairs)
+    if w.kv_dtype == "e4m3":
+        oracle.reshape_and_cache_e4m3(w.new_k, w.new_v, kc, vc, w.slot_mapping, w.new_kv_dtype, w.k_scale, w.v_scale)
+    else:
+        oracle.reshape_and_cache(w.new_k, w.new_v, kc, vc, w.slot_mapping, w.kv_dtype)
+    return kc, vc
+
+
 def oracle_sample_rate(w: W.Workload, seconds: float, start: int = 0):
     """Time the fp64 oracle on consecutive sequences (from `start`, wrapping) until ~`seconds` of work.
 
@@ -180,14 +196,15 @@ def oracle_sample_rate(w: W.Workload, seconds: float, start: int = 0):
     import oracle
 
     threads = oracle.default_threads()
-    kc, vc = W.apply_step_host(w)
+    kc, vc = oracle_post_step(w)
+    dec = dict(k_scale=w.k_scale, v_scale=w.v_scale)
     row = 2 * w.kv_row_bytes
     order = [(start + i) % w.num_seqs for i in range(w.num_seqs)]
     # pilot: one sequence of median length to size the sample
     med = int(np.argsort(w.seq_lens)[w.num_seqs // 2])
     t = time.perf_counter()
     oracle.decode(np.ascontiguousarray(w.q[[med]]), w.q_dtype, kc, vc, w.kv_dtype,
-                  np.ascontiguousarray(w.block_tables[[med]]), w.seq_lens[[med]], w.scale, num_threads=1)
+                  np.ascontiguousarray(w.block_tables[[med]]), w.seq_lens[[med]], w.scale, num_threads=1, **dec)
     per_token = (time.perf_counter() - t) / max(1, int(w.seq_lens[med]))
     budget_tokens = seconds * threads / max(per_token, 1e-12)
     pick, tok = [], 0
@@ -201,7 +218,7 @@ def oracle_sample_rate(w: W.Workload, seconds: float, start: int = 0):
                  np.ascontiguousarray(w.seq_lens[idx]))
     passes, t = 0, time.perf_counter()
     while True:  # whole passes over the sample until the time budget is used
-        oracle.decode(q, w.q_dtype, kc, vc, w.kv_dtype, bt, sl, w.scale, num_threads=threads)
+        oracle.decode(q, w.q_dtype, kc, vc, w.kv_dtype, bt, sl, w.scale, num_threads=threads, **dec)
         passes += 1
         dt = time.perf_counter() - t
         if dt >= 0.8 * seconds:
@@ -213,7 +230,7 @@ def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
-    w = W.make_config(args.config, block_size=args.block_size)
+    w = W.make_config(args.config, block_size=args.block_size, kv_dtype=args.kv_dtype)
     per_step = max(0.5, args.ref_seconds / max(1, args.steps + args.warmup))
     start = 0
     for _ in range(args.warmup):
@@ -262,7 +279,7 @@ def run_ours(args):
 
     seed = rank_seed(args.config, rank)
     extra = {"num_seqs": args.num_seqs} if args.num_seqs else {}
-    w = W.make_config(args.config, block_size=args.block_size, seed=seed, **extra)
+    w = W.make_config(args.config, block_size=args.block_size, seed=seed, kv_dtype=args.kv_dtype, **extra)
     out_dtype = args.out_dtype or w.q_dtype
     dw = B.device_workload(w, f"cuda:{local}")
     ws = B.DecodeWorkspace.for_workload(dw, args.partition_size)
@@ -300,14 +317,30 @@ def run_ours(args):
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     wall0 = time.time()
     t_start.record(stream)
+    fp8 = w.kv_dtype == "e4m3"
+
+    def store():
+        if fp8:
+            B.pa_reshape_and_cache_fp8(dw.new_k, dw.new_v, dw.k_cache, dw.v_cache, dw.slot_mapping, w.k_scale,
+                                       w.v_scale, stream=stream)
+        else:
+            B.pa_reshape_and_cache(dw.new_k, dw.new_v, dw.k_cache, dw.v_cache, dw.slot_mapping, stream=stream)
+
+    def decode():
+        if fp8:
+            B.pa_decode_fp8(out, dw.q, dw.k_cache, dw.v_cache, dw.block_tables, dw.seq_lens, w.scale, w.k_scale,
+                            w.v_scale, ws.tensor, args.partition_size, stream)
+        else:
+            B.pa_decode(out, dw.q, dw.k_cache, dw.v_cache, dw.block_tables, dw.seq_lens, w.scale, ws.tensor,
+                        args.partition_size, stream)
+
     for i in range(args.steps):
         if len(w.copy_pairs):
             B.pa_copy_blocks(dw.k_cache, dw.v_cache, dw.copy_pairs, stream=stream)
         if len(w.slot_mapping):
-            B.pa_reshape_and_cache(dw.new_k, dw.new_v, dw.k_cache, dw.v_cache, dw.slot_mapping, stream=stream)
+            store()
         ev_dec[i][0].record(stream)
-        B.pa_decode(out, dw.q, dw.k_cache, dw.v_cache, dw.block_tables, dw.seq_lens, w.scale, ws.tensor,
-                    args.partition_size, stream)
+        decode()
         ev_dec[i][1].record(stream)
     t_end.record(stream)
     torch.cuda.synchronize()
@@ -369,8 +402,7 @@ def run_ours(args):
         flush.fill_(1)
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
-        B.pa_decode(out, dw.q, dw.k_cache, dw.v_cache, dw.block_tables, dw.seq_lens, w.scale, ws.tensor,
-                    args.partition_size, stream)
+        decode()
         b.record(stream)
         torch.cuda.synchronize()
         flushed.append(a.elapsed_time(b))

@@ -44,7 +44,8 @@
 extern "C" {
 #endif
 
-typedef enum { PA_F32 = 0, PA_F16 = 1, PA_BF16 = 2 } pa_dtype;
+/* PA_FP8_E4M3: OCP FP8 E4M3 codes, one byte per element, dequantised as code * scale */
+typedef enum { PA_F32 = 0, PA_F16 = 1, PA_BF16 = 2, PA_FP8_E4M3 = 3 } pa_dtype;
 
 typedef enum {
   PA_OK = 0,
@@ -91,13 +92,29 @@ PA_API size_t pa_decode_workspace_size(int num_seqs, int num_q_heads, int head_d
  *   (deterministic: the split depends only on seq_lens[i]).
  *   workspace    device scratch of >= pa_decode_workspace_size(num_seqs, num_q_heads,
  *                head_dim, max_blocks_per_seq * block_size, partition_size) bytes, 256-byte
- *                aligned; its contents need no initialisation and are overwritten. */
+ *                aligned; its contents need no initialisation and are overwritten.
+ *   An FP8 cache needs its scales: kv_dtype PA_FP8_E4M3 returns PA_ERR_UNSUPPORTED here
+ *   (use pa_decode_fp8). */
 PA_API int pa_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
               const int32_t* block_tables, const int32_t* seq_lens, int num_seqs,
               int num_q_heads, int num_kv_heads, int head_dim, int block_size, float scale,
               int max_blocks_per_seq, int64_t num_blocks, int q_dtype, int kv_dtype,
               int out_dtype, int partition_size, void* workspace, size_t workspace_bytes,
               void* stream);
+
+/* pa_decode over an FP8 E4M3 cache ("详解vLLM推理引擎架构", section "量化集成与部署":
+ * --kv-cache-dtype fp8; the page gives no format -- read as OCP E4M3 codes with one fp32
+ * scale for K and one for V).  K_t = code * k_scale and V_t = code * v_scale; everything
+ * else is pa_decode.  k_cache, v_cache: [num_blocks, block_size, num_kv_heads, 128] bytes
+ * (head_dim 128 only); q_dtype f32, f16 or bf16; scales finite and > 0.  The tensor-core
+ * products run in f16: an f32 query is split into two f16 parts (hi + lo), a 16-bit query is
+ * converted to f16 (exact for |q| in [2^-14, 65504]). */
+PA_API int pa_decode_fp8(void* out, const void* q, const void* k_cache, const void* v_cache,
+                         const int32_t* block_tables, const int32_t* seq_lens, int num_seqs,
+                         int num_q_heads, int num_kv_heads, int head_dim, int block_size, float scale,
+                         float k_scale, float v_scale, int max_blocks_per_seq, int64_t num_blocks,
+                         int q_dtype, int out_dtype, int partition_size, void* workspace,
+                         size_t workspace_bytes, void* stream);
 
 /* Store the step's new tokens into the paged cache ("vLLM 深度解读", section 7).
  * For each token t with slot = slot_mapping[t] >= 0:
@@ -111,6 +128,17 @@ PA_API int pa_reshape_and_cache(const void* k, const void* v, void* k_cache, voi
                          const int64_t* slot_mapping, int num_tokens, int num_kv_heads,
                          int head_dim, int block_size, int64_t num_blocks, int kv_dtype,
                          int64_t k_token_stride, int64_t v_token_stride, void* stream);
+
+/* pa_reshape_and_cache into an FP8 E4M3 cache: element x of k[t] (v[t]), in in_dtype f32,
+ * f16 or bf16, is stored as e4m3(x / k_scale) (v_scale for v): the division rounded to
+ * nearest in fp32, the conversion rounded to nearest even and saturated to +-448.  The slot
+ * rule, strides (in elements of in_dtype) and error behaviour are those of
+ * pa_reshape_and_cache; num_kv_heads * head_dim must be a multiple of 16. */
+PA_API int pa_reshape_and_cache_fp8(const void* k, const void* v, void* k_cache, void* v_cache,
+                                    const int64_t* slot_mapping, int num_tokens, int num_kv_heads,
+                                    int head_dim, int block_size, int64_t num_blocks, int in_dtype,
+                                    float k_scale, float v_scale, int64_t k_token_stride,
+                                    int64_t v_token_stride, void* stream);
 
 /* Copy-on-write block duplication ("详解vLLM推理引擎架构", "Copy-on-Write 与内存共享"):
  * for each pair p, physical block src_dst_pairs[p][0] of k_cache is copied over block

@@ -18,12 +18,13 @@ from . import workload as W
 
 _LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libpa.so")
 
-PA_F32, PA_F16, PA_BF16 = 0, 1, 2
+PA_F32, PA_F16, PA_BF16, PA_FP8_E4M3 = 0, 1, 2, 3
 PA_OK, PA_ERR_INVALID, PA_ERR_UNSUPPORTED, PA_ERR_WORKSPACE, PA_ERR_CUDA = 0, -1, -2, -3, -4
 PA_DEV_OK, PA_DEV_BAD_BLOCK_ID, PA_DEV_BAD_SEQ_LEN, PA_DEV_BAD_SLOT, PA_DEV_BAD_PAIR, PA_DEV_TIMEOUT = range(6)
 
 EXPORTED = ("pa_decode_workspace_size", "pa_decode", "pa_reshape_and_cache", "pa_copy_blocks",
-            "pa_strerror", "pa_get_device_error", "pa_version", "pa_decode_static_workspace")
+            "pa_strerror", "pa_get_device_error", "pa_version", "pa_decode_static_workspace",
+            "pa_decode_fp8", "pa_reshape_and_cache_fp8")
 PA_ERR_TOO_LARGE = -5
 PA_DECODE_STATIC_WORKSPACE_BYTES = 64 << 20
 
@@ -60,6 +61,11 @@ def load_library(path: str = _LIB_PATH):
     lib.pa_version.restype = I
     lib.pa_decode_static_workspace.argtypes = [P, P, P, P, P, P, I, I, I, I, I, ctypes.c_float, I, I64, I, I, I, I, P]
     lib.pa_decode_static_workspace.restype = I
+    F = ctypes.c_float
+    lib.pa_decode_fp8.argtypes = [P, P, P, P, P, P, I, I, I, I, I, F, F, F, I, I64, I, I, I, P, SZ, P]
+    lib.pa_decode_fp8.restype = I
+    lib.pa_reshape_and_cache_fp8.argtypes = [P, P, P, P, P, I, I, I, I, I64, I, F, F, I64, I64, P]
+    lib.pa_reshape_and_cache_fp8.restype = I
     if path == _LIB_PATH:
         _lib = lib
     return lib
@@ -143,6 +149,38 @@ def pa_decode_static_workspace(out: torch.Tensor, q: torch.Tensor, k_cache: torc
     _check(rc, "pa_decode_static_workspace")
 
 
+def pa_decode_fp8(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                  block_tables: torch.Tensor, seq_lens: torch.Tensor, scale: float, k_scale: float, v_scale: float,
+                  workspace: torch.Tensor, partition_size: int = 0, stream=None) -> None:
+    """pa_decode over an FP8 E4M3 cache (uint8 tensors of codes; value = code * scale)."""
+    N, Hq, D = q.shape
+    NB, bs, Hkv, D2 = k_cache.shape
+    if D2 != D or tuple(out.shape) != (N, Hq, D) or v_cache.shape != k_cache.shape:
+        raise ValueError("shape mismatch between q, out and the caches")
+    if k_cache.dtype != torch.uint8 or v_cache.dtype != torch.uint8:
+        raise TypeError("FP8 caches are uint8 tensors of E4M3 codes")
+    rc = load_library().pa_decode_fp8(
+        _ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), _ptr(seq_lens), N, Hq, Hkv, D, bs,
+        ctypes.c_float(scale), ctypes.c_float(k_scale), ctypes.c_float(v_scale), block_tables.shape[1], NB,
+        _TORCH_CODE[q.dtype], _TORCH_CODE[out.dtype], partition_size, _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(rc, "pa_decode_fp8")
+
+
+def pa_reshape_and_cache_fp8(k: torch.Tensor, v: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                             slot_mapping: torch.Tensor, k_scale: float, v_scale: float, stream=None) -> None:
+    """Quantise token rows k/v[t] to E4M3 codes e4m3(x / scale) at their slots (skip if < 0)."""
+    T, Hkv, D = k.shape
+    NB, bs = k_cache.shape[:2]
+    if slot_mapping.dtype != torch.int64:
+        raise TypeError("slot_mapping must be int64")
+    rc = load_library().pa_reshape_and_cache_fp8(
+        _ptr(k), _ptr(v), _ptr(k_cache), _ptr(v_cache), _ptr(slot_mapping), T, Hkv, D, bs, NB,
+        _TORCH_CODE[k.dtype], ctypes.c_float(k_scale), ctypes.c_float(v_scale), k.stride(0), v.stride(0),
+        _stream(stream))
+    _check(rc, "pa_reshape_and_cache_fp8")
+
+
 def pa_reshape_and_cache(k: torch.Tensor, v: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
                          slot_mapping: torch.Tensor, stream=None) -> None:
     """k_cache/v_cache[slot // bs, slot % bs] <- k/v[t] for each token t with slot >= 0."""
@@ -179,9 +217,11 @@ def pa_get_device_error(stream=None) -> int:
 # convenience: a workload on the device and one decode step through the ABI
 # ---------------------------------------------------------------------------------------
 def to_torch(a: np.ndarray, dtype: str, device) -> torch.Tensor:
-    """Storage array (float32, or uint16 bit patterns) -> torch tensor of the named dtype."""
+    """Storage array (float32, uint16 bit patterns, or uint8 E4M3 codes) -> torch tensor."""
     if dtype == "f32":
         t = torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32))
+    elif dtype == "e4m3":
+        t = torch.from_numpy(np.ascontiguousarray(a, dtype=np.uint8))
     else:
         t = torch.from_numpy(np.ascontiguousarray(a, dtype=np.uint16).view(np.int16)).view(_NAME_TORCH[dtype])
     return t.to(device)
@@ -190,7 +230,7 @@ def to_torch(a: np.ndarray, dtype: str, device) -> torch.Tensor:
 def from_torch(t: torch.Tensor) -> np.ndarray:
     """torch tensor -> storage array (float32, or uint16 bit patterns for 16-bit types)."""
     t = t.detach().cpu().contiguous()
-    if t.dtype == torch.float32:
+    if t.dtype in (torch.float32, torch.uint8):
         return t.numpy()
     return t.view(torch.int16).numpy().view(np.uint16)
 
@@ -214,8 +254,8 @@ def device_workload(w: W.Workload, device="cuda") -> DeviceWorkload:
         w=w, q=to_torch(w.q, w.q_dtype, device), k_cache=to_torch(w.k_cache, w.kv_dtype, device),
         v_cache=to_torch(w.v_cache, w.kv_dtype, device),
         block_tables=torch.from_numpy(w.block_tables).to(device),
-        seq_lens=torch.from_numpy(w.seq_lens).to(device), new_k=to_torch(w.new_k, w.kv_dtype, device),
-        new_v=to_torch(w.new_v, w.kv_dtype, device), slot_mapping=torch.from_numpy(w.slot_mapping).to(device),
+        seq_lens=torch.from_numpy(w.seq_lens).to(device), new_k=to_torch(w.new_k, w.new_kv_dtype, device),
+        new_v=to_torch(w.new_v, w.new_kv_dtype, device), slot_mapping=torch.from_numpy(w.slot_mapping).to(device),
         copy_pairs=torch.from_numpy(np.ascontiguousarray(w.copy_pairs, dtype=np.int32).reshape(-1, 2)).to(device))
 
 
@@ -237,8 +277,16 @@ class DecodeWorkspace:
 
 def run_step(dw: DeviceWorkload, out: torch.Tensor, ws: DecodeWorkspace, partition_size=0, stream=None) -> None:
     """One decode step: copy_blocks -> reshape_and_cache -> decode (all through the C ABI)."""
+    w = dw.w
     if dw.copy_pairs.shape[0]:
         pa_copy_blocks(dw.k_cache, dw.v_cache, dw.copy_pairs, stream=stream)
+    if w.kv_dtype == "e4m3":
+        if dw.slot_mapping.shape[0]:
+            pa_reshape_and_cache_fp8(dw.new_k, dw.new_v, dw.k_cache, dw.v_cache, dw.slot_mapping, w.k_scale,
+                                     w.v_scale, stream=stream)
+        pa_decode_fp8(out, dw.q, dw.k_cache, dw.v_cache, dw.block_tables, dw.seq_lens, w.scale, w.k_scale,
+                      w.v_scale, ws.tensor, partition_size=partition_size, stream=stream)
+        return
     if dw.slot_mapping.shape[0]:
         pa_reshape_and_cache(dw.new_k, dw.new_v, dw.k_cache, dw.v_cache, dw.slot_mapping, stream=stream)
     pa_decode(out, dw.q, dw.k_cache, dw.v_cache, dw.block_tables, dw.seq_lens, dw.w.scale, ws.tensor,

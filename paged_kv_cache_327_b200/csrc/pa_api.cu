@@ -24,7 +24,7 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-int elem_bytes(int dt) { return dt == PA_F32 ? 4 : 2; }
+int elem_bytes(int dt) { return dt == PA_F32 ? 4 : dt == PA_FP8_E4M3 ? 1 : 2; }
 
 struct WsLayout {
   size_t counters, items, part_ml, part_acc, total;
@@ -62,7 +62,7 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 // Per-device launch facts, looked up once.
 struct DeviceInfo {
   int sm_count = 0;
-  bool smem_set[32] = {};
+  bool smem_set[64] = {};
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_mu;
@@ -78,29 +78,34 @@ int current_device_info(int* dev, DeviceInfo** info) {
 }
 
 // KV cache [num_blocks, block_size, num_kv_heads, head_dim] seen as a 3-D tensor
-// (64 elements, head_dim/64 * num_kv_heads column halves, num_blocks * block_size rows);
-// one box = block_size rows of one 128-byte column half, 128-byte swizzle.
+// (128 bytes of a row, head_dim * elem / 128 * num_kv_heads 128-byte column blocks,
+// num_blocks * block_size rows); one box = block_size rows of one 128-byte column block,
+// 128-byte swizzle.
 int encode_kv_map(CUtensorMap* map, const void* base, int kv_dtype, int64_t num_blocks, int block_size,
                   int num_kv_heads, int head_dim) {
   PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
   if (!enc) return PA_ERR_CUDA;
-  const cuuint64_t dims[3] = {64, static_cast<cuuint64_t>(head_dim / 64) * num_kv_heads,
+  const int es = elem_bytes(kv_dtype);
+  const cuuint64_t inner = 128 / es;
+  const cuuint64_t dims[3] = {inner, static_cast<cuuint64_t>(head_dim * es / 128) * num_kv_heads,
                               static_cast<cuuint64_t>(num_blocks) * block_size};
-  const cuuint64_t strides[2] = {128, static_cast<cuuint64_t>(num_kv_heads) * head_dim * 2};
-  const cuuint32_t box[3] = {64, 1, static_cast<cuuint32_t>(block_size)};
+  const cuuint64_t strides[2] = {128, static_cast<cuuint64_t>(num_kv_heads) * head_dim * es};
+  const cuuint32_t box[3] = {static_cast<cuuint32_t>(inner), 1, static_cast<cuuint32_t>(block_size)};
   const cuuint32_t estr[3] = {1, 1, 1};
-  const CUresult r =
-      enc(map, kv_dtype == PA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3,
-          const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  const CUtensorMapDataType dt = kv_dtype == PA_BF16   ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                 : kv_dtype == PA_F16  ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
+                                                       : CU_TENSOR_MAP_DATA_TYPE_UINT8;
+  const CUresult r = enc(map, dt, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? PA_OK : PA_ERR_CUDA;
 }
 
-template <int BS, int D, typename KT, bool QF32>
+template <int BS, int D, typename KT, typename QT>
 int launch_partition(const pa::DecodeParams& p, const CUtensorMap& tmk, const CUtensorMap& tmv,
                      int64_t max_items, DeviceInfo* info, int slot_id, cudaStream_t stream) {
-  using C = pa::DecodeCfg<BS, D, KT, QF32>;
-  auto kern = pa::pa_decode_partition_kernel<BS, D, KT, QF32>;
+  using C = pa::DecodeCfg<BS, D, KT, QT>;
+  auto kern = pa::pa_decode_partition_kernel<BS, D, KT, QT>;
   if (!info->smem_set[slot_id]) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
       return PA_ERR_CUDA;
@@ -125,14 +130,28 @@ int launch_partition(const pa::DecodeParams& p, const CUtensorMap& tmk, const CU
   return cudaPeekAtLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
+// one shared-memory attribute flag per kernel instantiation
+constexpr int kInstPerShape = 8;
+
 template <int BS, int D>
 int dispatch_kv(const pa::DecodeParams& p, const CUtensorMap& tmk, const CUtensorMap& tmv, int64_t max_items,
-                DeviceInfo* info, int kv_dtype, bool qf32, int base_id, cudaStream_t stream) {
+                DeviceInfo* info, int kv_dtype, int q_dtype, int base_id, cudaStream_t stream) {
+  const bool qf32 = q_dtype == PA_F32;
   if (kv_dtype == PA_BF16)
-    return qf32 ? launch_partition<BS, D, __nv_bfloat16, true>(p, tmk, tmv, max_items, info, base_id + 0, stream)
-                : launch_partition<BS, D, __nv_bfloat16, false>(p, tmk, tmv, max_items, info, base_id + 1, stream);
-  return qf32 ? launch_partition<BS, D, __half, true>(p, tmk, tmv, max_items, info, base_id + 2, stream)
-              : launch_partition<BS, D, __half, false>(p, tmk, tmv, max_items, info, base_id + 3, stream);
+    return qf32 ? launch_partition<BS, D, __nv_bfloat16, float>(p, tmk, tmv, max_items, info, base_id + 0, stream)
+                : launch_partition<BS, D, __nv_bfloat16, __nv_bfloat16>(p, tmk, tmv, max_items, info, base_id + 1,
+                                                                        stream);
+  if (kv_dtype == PA_F16)
+    return qf32 ? launch_partition<BS, D, __half, float>(p, tmk, tmv, max_items, info, base_id + 2, stream)
+                : launch_partition<BS, D, __half, __half>(p, tmk, tmv, max_items, info, base_id + 3, stream);
+  if constexpr (D == 128) {  // an FP8 row of head_dim 128 fills one 128-byte TMA box
+    if (q_dtype == PA_F32)
+      return launch_partition<BS, D, pa::fp8e4m3, float>(p, tmk, tmv, max_items, info, base_id + 4, stream);
+    if (q_dtype == PA_F16)
+      return launch_partition<BS, D, pa::fp8e4m3, __half>(p, tmk, tmv, max_items, info, base_id + 5, stream);
+    return launch_partition<BS, D, pa::fp8e4m3, __nv_bfloat16>(p, tmk, tmv, max_items, info, base_id + 6, stream);
+  }
+  return PA_ERR_UNSUPPORTED;
 }
 
 }  // namespace
@@ -161,21 +180,32 @@ size_t pa_decode_workspace_size(int num_seqs, int num_q_heads, int head_dim, int
   return ws_layout(num_seqs, num_q_heads, head_dim, max_parts).total;
 }
 
-int pa_decode(void* out, const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,
-              const int32_t* seq_lens, int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
-              int block_size, float scale, int max_blocks_per_seq, int64_t num_blocks, int q_dtype,
-              int kv_dtype, int out_dtype, int partition_size, void* workspace, size_t workspace_bytes,
-              void* stream) {
+}  // extern "C"
+
+namespace {
+
+// pa_decode and pa_decode_fp8: kv_dtype F16 / BF16 (scales unused) or FP8_E4M3
+int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,
+                const int32_t* seq_lens, int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                int block_size, float scale, float k_scale, float v_scale, int max_blocks_per_seq,
+                int64_t num_blocks, int q_dtype, int kv_dtype, int out_dtype, int partition_size, void* workspace,
+                size_t workspace_bytes, void* stream) {
   if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 ||
-      max_blocks_per_seq <= 0 || num_blocks <= 0 || partition_size < 0 || !std::isfinite(scale))
+      max_blocks_per_seq <= 0 || num_blocks <= 0 || partition_size < 0 || !std::isfinite(scale) ||
+      !std::isfinite(k_scale) || !std::isfinite(v_scale) || k_scale <= 0.f || v_scale <= 0.f)
     return PA_ERR_INVALID;
   if (num_q_heads % num_kv_heads) return PA_ERR_INVALID;
   const int G = num_q_heads / num_kv_heads;
   if (G > 8) return PA_ERR_UNSUPPORTED;
   if (head_dim != 64 && head_dim != 128) return PA_ERR_UNSUPPORTED;
   if (block_size != 16 && block_size != 32) return PA_ERR_UNSUPPORTED;
-  if (kv_dtype != PA_F16 && kv_dtype != PA_BF16) return PA_ERR_UNSUPPORTED;
-  if (q_dtype != kv_dtype && q_dtype != PA_F32) return PA_ERR_UNSUPPORTED;
+  if (kv_dtype == PA_FP8_E4M3) {
+    if (head_dim != 128) return PA_ERR_UNSUPPORTED;
+    if (q_dtype != PA_F32 && q_dtype != PA_F16 && q_dtype != PA_BF16) return PA_ERR_UNSUPPORTED;
+  } else {
+    if (kv_dtype != PA_F16 && kv_dtype != PA_BF16) return PA_ERR_UNSUPPORTED;
+    if (q_dtype != kv_dtype && q_dtype != PA_F32) return PA_ERR_UNSUPPORTED;
+  }
   if (out_dtype != PA_F32 && out_dtype != PA_F16 && out_dtype != PA_BF16) return PA_ERR_UNSUPPORTED;
   const int P = partition_size ? partition_size : kDefaultPartition;
   if (P % block_size || P / block_size > 32) return PA_ERR_UNSUPPORTED;
@@ -216,7 +246,9 @@ int pa_decode(void* out, const void* q, const void* k_cache, const void* v_cache
   p.partition_size = P;
   p.max_parts = static_cast<int>(max_parts);
   p.out_dtype = out_dtype;
-  p.scale_log2 = scale * 1.4426950408889634f;
+  const bool fp8 = kv_dtype == PA_FP8_E4M3;
+  p.scale_log2 = scale * (fp8 ? k_scale : 1.f) * 1.4426950408889634f;
+  p.v_scale = fp8 ? v_scale : 1.f;
   p.counters = reinterpret_cast<unsigned int*>(ws + L.counters);
   p.items = reinterpret_cast<pa::WorkItem*>(ws + L.items);
   p.part_ml = reinterpret_cast<float2*>(ws + L.part_ml);
@@ -227,14 +259,14 @@ int pa_decode(void* out, const void* q, const void* k_cache, const void* v_cache
   if (cudaPeekAtLastError() != cudaSuccess) return PA_ERR_CUDA;
 
   const int64_t max_items = static_cast<int64_t>(num_seqs) * max_parts * num_kv_heads;
-  const bool qf32 = q_dtype == PA_F32;
   int rc;
   if (block_size == 16)
-    rc = head_dim == 128 ? dispatch_kv<16, 128>(p, tmk, tmv, max_items, info, kv_dtype, qf32, 0, st)
-                         : dispatch_kv<16, 64>(p, tmk, tmv, max_items, info, kv_dtype, qf32, 4, st);
+    rc = head_dim == 128 ? dispatch_kv<16, 128>(p, tmk, tmv, max_items, info, kv_dtype, q_dtype, 0, st)
+                         : dispatch_kv<16, 64>(p, tmk, tmv, max_items, info, kv_dtype, q_dtype, kInstPerShape, st);
   else
-    rc = head_dim == 128 ? dispatch_kv<32, 128>(p, tmk, tmv, max_items, info, kv_dtype, qf32, 8, st)
-                         : dispatch_kv<32, 64>(p, tmk, tmv, max_items, info, kv_dtype, qf32, 12, st);
+    rc = head_dim == 128
+             ? dispatch_kv<32, 128>(p, tmk, tmv, max_items, info, kv_dtype, q_dtype, 2 * kInstPerShape, st)
+             : dispatch_kv<32, 64>(p, tmk, tmv, max_items, info, kv_dtype, q_dtype, 3 * kInstPerShape, st);
   if (rc != PA_OK) return rc;
   {  // merge kernel: waits (griddepcontrol.wait) for the partition kernel's partial results
     const int64_t warps = static_cast<int64_t>(num_seqs) * num_q_heads;
@@ -250,6 +282,31 @@ int pa_decode(void* out, const void* q, const void* k_cache, const void* v_cache
     if (cudaLaunchKernelEx(&cfg, pa::pa_decode_merge_kernel, p) != cudaSuccess) return PA_ERR_CUDA;
   }
   return cudaPeekAtLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+int pa_decode(void* out, const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,
+              const int32_t* seq_lens, int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+              int block_size, float scale, int max_blocks_per_seq, int64_t num_blocks, int q_dtype,
+              int kv_dtype, int out_dtype, int partition_size, void* workspace, size_t workspace_bytes,
+              void* stream) {
+  if (kv_dtype == PA_FP8_E4M3) return PA_ERR_UNSUPPORTED;  // needs its scales: pa_decode_fp8
+  return decode_impl(out, q, k_cache, v_cache, block_tables, seq_lens, num_seqs, num_q_heads, num_kv_heads,
+                     head_dim, block_size, scale, 1.f, 1.f, max_blocks_per_seq, num_blocks, q_dtype, kv_dtype,
+                     out_dtype, partition_size, workspace, workspace_bytes, stream);
+}
+
+int pa_decode_fp8(void* out, const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,
+                  const int32_t* seq_lens, int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                  int block_size, float scale, float k_scale, float v_scale, int max_blocks_per_seq,
+                  int64_t num_blocks, int q_dtype, int out_dtype, int partition_size, void* workspace,
+                  size_t workspace_bytes, void* stream) {
+  return decode_impl(out, q, k_cache, v_cache, block_tables, seq_lens, num_seqs, num_q_heads, num_kv_heads,
+                     head_dim, block_size, scale, k_scale, v_scale, max_blocks_per_seq, num_blocks, q_dtype,
+                     PA_FP8_E4M3, out_dtype, partition_size, workspace, workspace_bytes, stream);
 }
 
 int pa_reshape_and_cache(const void* k, const void* v, void* k_cache, void* v_cache, const int64_t* slot_mapping,
@@ -277,6 +334,49 @@ int pa_reshape_and_cache(const void* k, const void* v, void* k_cache, void* v_ca
       static_cast<const uint8_t*>(k), static_cast<const uint8_t*>(v), static_cast<uint8_t*>(k_cache),
       static_cast<uint8_t*>(v_cache), slot_mapping, num_tokens, row * es, k_token_stride * es, v_token_stride * es,
       num_blocks * block_size);
+  return cudaPeekAtLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+int pa_reshape_and_cache_fp8(const void* k, const void* v, void* k_cache, void* v_cache,
+                             const int64_t* slot_mapping, int num_tokens, int num_kv_heads, int head_dim,
+                             int block_size, int64_t num_blocks, int in_dtype, float k_scale, float v_scale,
+                             int64_t k_token_stride, int64_t v_token_stride, void* stream) {
+  if (num_tokens < 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 || num_blocks <= 0 ||
+      k_token_stride < 0 || v_token_stride < 0 || !std::isfinite(k_scale) || !std::isfinite(v_scale) ||
+      k_scale <= 0.f || v_scale <= 0.f)
+    return PA_ERR_INVALID;
+  if (in_dtype != PA_F32 && in_dtype != PA_F16 && in_dtype != PA_BF16) return PA_ERR_UNSUPPORTED;
+  const int64_t row = static_cast<int64_t>(num_kv_heads) * head_dim;
+  if (row % 16) return PA_ERR_UNSUPPORTED;  // 8 elements per thread, 16-byte aligned cache rows
+  if (!k_token_stride) k_token_stride = row;
+  if (!v_token_stride) v_token_stride = row;
+  if (k_token_stride < row || v_token_stride < row) return PA_ERR_INVALID;
+  if (num_tokens == 0) return PA_OK;
+  if (!k || !v || !k_cache || !v_cache || !slot_mapping) return PA_ERR_INVALID;
+  const int es = elem_bytes(in_dtype);
+  if (!aligned16(k_cache) || !aligned16(v_cache) || !aligned16(k) || !aligned16(v) || (k_token_stride * es) % 16 ||
+      (v_token_stride * es) % 16)
+    return PA_ERR_INVALID;
+  int dev;
+  DeviceInfo* info;
+  if (current_device_info(&dev, &info) != PA_OK) return PA_ERR_CUDA;
+  const int grid = static_cast<int>(std::min<int64_t>(num_tokens, 64LL * info->sm_count));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* kc = static_cast<uint8_t*>(k_cache);
+  uint8_t* vc = static_cast<uint8_t*>(v_cache);
+  const int64_t slots = num_blocks * block_size;
+  if (in_dtype == PA_BF16)
+    pa::pa_reshape_and_cache_fp8_kernel<__nv_bfloat16><<<grid, 128, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(v), kc, vc, slot_mapping, num_tokens,
+        row, k_token_stride, v_token_stride, slots, k_scale, v_scale);
+  else if (in_dtype == PA_F16)
+    pa::pa_reshape_and_cache_fp8_kernel<__half><<<grid, 128, 0, st>>>(
+        static_cast<const __half*>(k), static_cast<const __half*>(v), kc, vc, slot_mapping, num_tokens, row,
+        k_token_stride, v_token_stride, slots, k_scale, v_scale);
+  else
+    pa::pa_reshape_and_cache_fp8_kernel<float><<<grid, 128, 0, st>>>(
+        static_cast<const float*>(k), static_cast<const float*>(v), kc, vc, slot_mapping, num_tokens, row,
+        k_token_stride, v_token_stride, slots, k_scale, v_scale);
   return cudaPeekAtLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 

@@ -39,6 +39,57 @@ __global__ void __launch_bounds__(128)
   }
 }
 
+// Store into an FP8 E4M3 cache: each element x of the token's K (V) row becomes the code
+// e4m3(x / scale), the division rounded to nearest in fp32, the conversion rounded to
+// nearest even and saturated to +-448.  A thread converts 8 consecutive elements.
+template <typename IT>
+__device__ __forceinline__ void load8(const IT* p, float (&x)[8]) {
+  if constexpr (std::is_same<IT, float>::value) {
+    const float4 a = __ldg(reinterpret_cast<const float4*>(p)), b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+    x[0] = a.x, x[1] = a.y, x[2] = a.z, x[3] = a.w, x[4] = b.x, x[5] = b.y, x[6] = b.z, x[7] = b.w;
+  } else {
+    const uint4 u = __ldg(reinterpret_cast<const uint4*>(p));
+    const IT* e = reinterpret_cast<const IT*>(&u);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) x[j] = to_float(e[j]);
+  }
+}
+
+__device__ __forceinline__ uint32_t e4m3x4(float a, float b, float c, float d) {
+  const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3);  // a: low byte
+  const uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(c, d), __NV_SATFINITE, __NV_E4M3);
+  return (lo & 0xffffu) | (hi << 16);
+}
+
+template <typename IT>
+__global__ void __launch_bounds__(128)
+    pa_reshape_and_cache_fp8_kernel(const IT* __restrict__ k, const IT* __restrict__ v,
+                                    uint8_t* __restrict__ kc, uint8_t* __restrict__ vc,
+                                    const int64_t* __restrict__ slots, int num_tokens, int64_t row,
+                                    int64_t k_stride, int64_t v_stride, int64_t num_slots, float k_scale,
+                                    float v_scale) {
+  for (int t = blockIdx.x; t < num_tokens; t += gridDim.x) {
+    const int64_t s = slots[t];
+    if (s < 0) continue;
+    if (s >= num_slots) {
+      if (threadIdx.x == 0) record_error(DEV_BAD_SLOT);
+      continue;
+    }
+    for (int64_t i = threadIdx.x * 8; i < row; i += blockDim.x * 8) {
+#pragma unroll
+      for (int which = 0; which < 2; ++which) {
+        float x[8];
+        load8((which ? v + t * v_stride : k + t * k_stride) + i, x);
+        const float sc = which ? v_scale : k_scale;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) x[j] = __fdiv_rn(x[j], sc);
+        const uint2 w = make_uint2(e4m3x4(x[0], x[1], x[2], x[3]), e4m3x4(x[4], x[5], x[6], x[7]));
+        *reinterpret_cast<uint2*>((which ? vc : kc) + s * row + i) = w;
+      }
+    }
+  }
+}
+
 // grid: (num_pairs, 2 [K, V], chunks)
 __global__ void __launch_bounds__(256)
     pa_copy_blocks_kernel(uint8_t* __restrict__ kc, uint8_t* __restrict__ vc,

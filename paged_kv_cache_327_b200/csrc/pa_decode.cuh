@@ -32,7 +32,10 @@
 // way whatever warp runs it, so results are deterministic and batch-invariant.
 #pragma once
 
+#include <cuda_fp8.h>
 #include <math_constants.h>
+
+#include <type_traits>
 
 #include "pa_ptx.cuh"
 
@@ -72,7 +75,8 @@ struct DecodeParams {
   int num_seqs, num_q_heads, num_kv_heads, group;
   int head_dim, block_size, max_blocks_per_seq, num_blocks;
   int partition_size, max_parts, out_dtype, pad;
-  float scale_log2;  // scale * log2(e)
+  float scale_log2;  // scale * log2(e) (* k_scale for an FP8 cache)
+  float v_scale;     // multiplies the output (FP8 cache); 1 otherwise
   // workspace views
   unsigned int* counters;  // [0] next work item, [1] number of (sequence, partition) pairs
   WorkItem* items;         // [num_seqs * max_parts]
@@ -170,12 +174,56 @@ __global__ void __launch_bounds__(kPlanThreads) pa_decode_plan_kernel(const Deco
 }
 
 // ------------------------------------------------------------------------------ partition kernel
-template <int BS, int D, typename KT, bool QF32>
+// Tag of a KV cache holding FP8 E4M3 codes (one byte per element).  Its tiles are turned into
+// f16 in registers, so its tensor-core work runs in f16; the query is then split into two f16
+// parts (hi + lo) to keep its precision.
+struct fp8e4m3 {};
+
+template <typename KT>
+struct KvTraits {
+  using mma_t = KT;
+  static constexpr int bytes = 2;
+  static constexpr bool fp8 = false;
+};
+template <>
+struct KvTraits<fp8e4m3> {
+  using mma_t = __half;
+  static constexpr int bytes = 1;
+  static constexpr bool fp8 = true;
+};
+
+template <typename T>
+__device__ __forceinline__ float to_float(T x);
+template <>
+__device__ __forceinline__ float to_float<float>(float x) { return x; }
+template <>
+__device__ __forceinline__ float to_float<__half>(__half x) { return __half2float(x); }
+template <>
+__device__ __forceinline__ float to_float<__nv_bfloat16>(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+// two E4M3 codes (low byte first) -> two f16 (exact: every E4M3 value is an f16 value)
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t v) {
+  const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(v & 0xffffu), __NV_E4M3);
+  return static_cast<uint32_t>(h.x) | (static_cast<uint32_t>(h.y) << 16);
+}
+
+__device__ __forceinline__ uint32_t lds_u16(uint32_t addr) {
+  unsigned short v;
+  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(addr));
+  return v;
+}
+
+template <int BS, int D, typename KT, typename QT>
 struct DecodeCfg {
-  static constexpr int HALVES = D / 64;                 // 64-element (128-byte) column halves
+  static constexpr bool FP8 = KvTraits<KT>::fp8;
+  static constexpr int HALVES = D * KvTraits<KT>::bytes / 128;  // 128-byte column blocks of a row
   static constexpr int BOX_BYTES = BS * 128;            // one TMA box: BS rows x 128 bytes
   static constexpr int PAGE_BYTES = BOX_BYTES * HALVES; // one KV head of one block
-  static constexpr int QE = QF32 ? 4 : 2;
+  static constexpr int QE = sizeof(QT);
+  // an fp32 query is split into hi + lo parts of the operand type; a 16-bit query over an FP8
+  // cache is converted to f16 once (exact for |q| in [2^-14, 65504])
+  static constexpr bool QSPLIT = std::is_same<QT, float>::value;
+  static constexpr bool QCONV = FP8 && !QSPLIT;
   static constexpr int Q_BYTES = 8 * D * QE;            // up to 8 grouped query rows
   static constexpr int SLOT_BYTES = ((2 * PAGE_BYTES + Q_BYTES + 1023) / 1024) * 1024;
   static constexpr int NC = 4;                          // consumer warps (one producer each)
@@ -191,6 +239,7 @@ struct DecodeCfg {
   static constexpr int KS = D / 16;     // 16-wide steps over head_dim
   static_assert(D == 64 || D == 128, "head_dim");
   static_assert(BS == 16 || BS == 32, "block_size");
+  static_assert(HALVES >= 1, "an FP8 row must fill a 128-byte box (head_dim 128)");
 };
 
 // byte offset, inside a page, of the 16-byte chunk holding (row t, columns d0..d0+7)
@@ -203,11 +252,12 @@ __device__ __forceinline__ uint32_t swz(int t, int d0) {
 // meta word: ntok (bits 0-7) | flags (bits 8-15) | partitions of the sequence (bits 16-31)
 constexpr int F_FIRST = 1, F_LAST = 2, F_BAD = 4, F_END = 8;
 
-template <int BS, int D, typename KT, bool QF32>
-__global__ void __launch_bounds__(DecodeCfg<BS, D, KT, QF32>::NWARP * 32, 1)
+template <int BS, int D, typename KT, typename QT>
+__global__ void __launch_bounds__(DecodeCfg<BS, D, KT, QT>::NWARP * 32, 1)
     pa_decode_partition_kernel(const __grid_constant__ CUtensorMap tmk,
                                const __grid_constant__ CUtensorMap tmv, const DecodeParams p) {
-  using C = DecodeCfg<BS, D, KT, QF32>;
+  using C = DecodeCfg<BS, D, KT, QT>;
+  using MA = typename KvTraits<KT>::mma_t;  // element type of the tensor-core operands
   constexpr unsigned FULL = 0xffffffffu;
 
   extern __shared__ uint8_t smem_raw[];
@@ -333,33 +383,53 @@ __global__ void __launch_bounds__(DecodeCfg<BS, D, KT, QF32>::NWARP * 32, 1)
     voff[k] = swz<C::BOX_BYTES>(lr + ((lm >> 1) << 3), k * 16 + ((lm & 1) << 3));
   }
   const float sl = p.scale_log2;
-  const uint32_t ones = pack2<KT>(1.f, 1.f);
+  const uint32_t ones = pack2<MA>(1.f, 1.f);
+  // FP8 tiles: per-lane offsets of the K rows for ldmatrix (row lr + 8 (lm & 1), 16-byte chunk
+  // 2 kb + (lm >> 1)) and the swizzle terms of the V rows 2c (+8) and 2c+1 (+8) a lane reads
+  uint32_t koff8[C::FP8 ? C::KS / 2 : 1];
+  int vx0 = 0, vx1 = 0;
+  if constexpr (C::FP8) {
+#pragma unroll
+    for (int kq = 0; kq < C::KS / 2; ++kq) {
+      const int t = lr + ((lm & 1) << 3);
+      koff8[kq] = t * 128 + ((((2 * kq + (lm >> 1)) ^ (t & 7))) << 4);
+    }
+    vx0 = c2 & 7;
+    vx1 = (c2 + 1) & 7;
+  }
 
   float mu0 = -CUDART_INF_F, mu1 = -CUDART_INF_F;  // running maxima (log2 units), columns c2, c2+1
   float acc[C::KS][4] = {};
   float lacc[4] = {0.f, 0.f, 0.f, 0.f};
   uint32_t qf[C::KS][2];
-  uint32_t ql[QF32 ? C::KS : 1][2];
+  uint32_t ql[C::QSPLIT ? C::KS : 1][2];
+  (void)ql;
   bool poisoned = false;
 
   auto load_q = [&](const uint8_t* qs) {
-    if constexpr (!QF32) {
+    if constexpr (!C::QSPLIT && !C::QCONV) {
 #pragma unroll
       for (int k2 = 0; k2 < C::KS; k2 += 2) {
         const int d0 = (k2 + (lm >> 1)) * 16 + ((lm & 1) << 3);
         ldsm_x4(smem_u32(qs + (lr * D + d0) * 2), qf[k2][0], qf[k2][1], qf[k2 + 1][0], qf[k2 + 1][1]);
       }
     } else {
-      const float* qv = reinterpret_cast<const float*>(qs);
+      const QT* qv = reinterpret_cast<const QT*>(qs);
 #pragma unroll
       for (int kk = 0; kk < C::KS; ++kk) {
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-          const float2 x = *reinterpret_cast<const float2*>(qv + r0 * D + kk * 16 + h * 8 + c2);
-          const uint32_t hi = pack2<KT>(x.x, x.y);
-          const float2 hf = unpack2<KT>(hi);
+          // FP8 tiles are unpacked as 4 consecutive columns 16 kk + 4c .. +3 per lane
+          // (pairs h = 0, 1); the query takes the same order.  Otherwise the usual
+          // m16n8k16 columns 16 kk + 2c (+1) and + 8.
+          const int d = C::FP8 ? kk * 16 + 2 * c2 + 2 * h : kk * 16 + h * 8 + c2;
+          const float x0 = to_float(qv[r0 * D + d]), x1 = to_float(qv[r0 * D + d + 1]);
+          const uint32_t hi = pack2<MA>(x0, x1);
           qf[kk][h] = hi;
-          ql[kk][h] = pack2<KT>(x.x - hf.x, x.y - hf.y);
+          if constexpr (C::QSPLIT) {
+            const float2 hf = unpack2<MA>(hi);
+            ql[kk][h] = pack2<MA>(x0 - hf.x, x1 - hf.y);
+          }
         }
       }
     }
@@ -371,17 +441,38 @@ __global__ void __launch_bounds__(DecodeCfg<BS, D, KT, QF32>::NWARP * 32, 1)
 #pragma unroll
     for (int mt = 0; mt < C::MT; ++mt) {
       float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb2[4] = {0.f, 0.f, 0.f, 0.f};
+      if constexpr (C::FP8) {
+        // one ldmatrix.x4 holds 32 columns of 16 rows: lane gets 4 codes of row r0 (r0 + 8)
 #pragma unroll
-      for (int kk = 0; kk < C::KS; ++kk) {
-        uint32_t a0, a1, a2, a3;
-        ldsm_x4(kb + mt * 2048 + koff[kk], a0, a1, a2, a3);
-        if constexpr (QF32) {
-          Mma<KT>::run(sa, a0, a1, a2, a3, qf[kk][0], qf[kk][1]);
-          Mma<KT>::run(sb2, a0, a1, a2, a3, ql[kk][0], ql[kk][1]);
-        } else if (kk & 1) {
-          Mma<KT>::run(sb2, a0, a1, a2, a3, qf[kk][0], qf[kk][1]);
-        } else {
-          Mma<KT>::run(sa, a0, a1, a2, a3, qf[kk][0], qf[kk][1]);
+        for (int kq = 0; kq < C::KS / 2; ++kq) {
+          uint32_t r[4];
+          ldsm_x4(kb + mt * 2048 + koff8[kq], r[0], r[1], r[2], r[3]);
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int kk = 2 * kq + h;
+            const uint32_t a0 = e4m3x2_to_f16x2(r[2 * h]), a1 = e4m3x2_to_f16x2(r[2 * h + 1]);
+            const uint32_t a2 = e4m3x2_to_f16x2(r[2 * h] >> 16), a3 = e4m3x2_to_f16x2(r[2 * h + 1] >> 16);
+            if constexpr (C::QSPLIT) {
+              Mma<MA>::run(sa, a0, a1, a2, a3, qf[kk][0], qf[kk][1]);
+              Mma<MA>::run(sb2, a0, a1, a2, a3, ql[kk][0], ql[kk][1]);
+            } else {
+              Mma<MA>::run(h ? sb2 : sa, a0, a1, a2, a3, qf[kk][0], qf[kk][1]);
+            }
+          }
+        }
+      } else {
+#pragma unroll
+        for (int kk = 0; kk < C::KS; ++kk) {
+          uint32_t a0, a1, a2, a3;
+          ldsm_x4(kb + mt * 2048 + koff[kk], a0, a1, a2, a3);
+          if constexpr (C::QSPLIT) {
+            Mma<MA>::run(sa, a0, a1, a2, a3, qf[kk][0], qf[kk][1]);
+            Mma<MA>::run(sb2, a0, a1, a2, a3, ql[kk][0], ql[kk][1]);
+          } else if (kk & 1) {
+            Mma<MA>::run(sb2, a0, a1, a2, a3, qf[kk][0], qf[kk][1]);
+          } else {
+            Mma<MA>::run(sa, a0, a1, a2, a3, qf[kk][0], qf[kk][1]);
+          }
         }
       }
 #pragma unroll
@@ -426,16 +517,48 @@ __global__ void __launch_bounds__(DecodeCfg<BS, D, KT, QF32>::NWARP * 32, 1)
     }
 #pragma unroll
     for (int mt = 0; mt < C::MT; ++mt) {
-      const uint32_t plo = pack2<KT>(fast_exp2(fmaf(s[mt][0], sl, -mu0)), fast_exp2(fmaf(s[mt][1], sl, -mu1)));
-      const uint32_t phi = pack2<KT>(fast_exp2(fmaf(s[mt][2], sl, -mu0)), fast_exp2(fmaf(s[mt][3], sl, -mu1)));
+      const uint32_t plo = pack2<MA>(fast_exp2(fmaf(s[mt][0], sl, -mu0)), fast_exp2(fmaf(s[mt][1], sl, -mu1)));
+      const uint32_t phi = pack2<MA>(fast_exp2(fmaf(s[mt][2], sl, -mu0)), fast_exp2(fmaf(s[mt][3], sl, -mu1)));
       const uint32_t b0 = movmatrix_t(plo), b1 = movmatrix_t(phi);
-      Mma<KT>::run(lacc, ones, ones, ones, ones, b0, b1);  // row sums of the weights as the MMA sees them
-      if (ntok >= (mt + 1) * 16) {
+      Mma<MA>::run(lacc, ones, ones, ones, ones, b0, b1);  // row sums of the weights as the MMA sees them
+      if constexpr (C::FP8) {
+        // V^T tile (16 columns x 16 tokens) from the codes: a lane reads the 16-bit column pair
+        // (2 r0, 2 r0 + 1) of tokens 2c, 2c+1, 2c+8, 2c+9 and pairs the tokens up by byte
+        // permutation; accumulator rows r0 / r0 + 8 are columns 2 r0 / 2 r0 + 1.
+        const int tk = mt * 16 + c2;
+        const uint32_t row0 = vb + (mt * 16 + c2) * 128 + 2 * r0;
+        auto v_tiles = [&](uint32_t mlo, uint32_t mhi, auto masked) {
+#pragma unroll
+          for (int dt = 0; dt < C::KS; ++dt) {
+            const uint32_t u0 = lds_u16(row0 + (((dt ^ vx0)) << 4));
+            const uint32_t u1 = lds_u16(row0 + 128 + (((dt ^ vx1)) << 4));
+            const uint32_t u2 = lds_u16(row0 + 8 * 128 + (((dt ^ vx0)) << 4));
+            const uint32_t u3 = lds_u16(row0 + 9 * 128 + (((dt ^ vx1)) << 4));
+            const uint32_t w01 = __byte_perm(u0, u1, 0x5140), w23 = __byte_perm(u2, u3, 0x5140);
+            uint32_t a0 = e4m3x2_to_f16x2(w01), a1 = e4m3x2_to_f16x2(w01 >> 16);
+            uint32_t a2 = e4m3x2_to_f16x2(w23), a3 = e4m3x2_to_f16x2(w23 >> 16);
+            if constexpr (decltype(masked)::value) {
+              a0 &= mlo;
+              a1 &= mlo;
+              a2 &= mhi;
+              a3 &= mhi;
+            }
+            Mma<MA>::run(acc[dt], a0, a1, a2, a3, b0, b1);
+          }
+        };
+        if (ntok >= (mt + 1) * 16) {
+          v_tiles(FULL, FULL, std::false_type{});
+        } else {
+          const uint32_t mlo = (tk < ntok ? 0x0000ffffu : 0u) | (tk + 1 < ntok ? 0xffff0000u : 0u);
+          const uint32_t mhi = (tk + 8 < ntok ? 0x0000ffffu : 0u) | (tk + 9 < ntok ? 0xffff0000u : 0u);
+          v_tiles(mlo, mhi, std::true_type{});
+        }
+      } else if (ntok >= (mt + 1) * 16) {
 #pragma unroll
         for (int dt = 0; dt < C::KS; ++dt) {
           uint32_t a0, a1, a2, a3;
           ldsm_x4_t(vb + mt * 2048 + voff[dt], a0, a1, a2, a3);
-          Mma<KT>::run(acc[dt], a0, a1, a2, a3, b0, b1);
+          Mma<MA>::run(acc[dt], a0, a1, a2, a3, b0, b1);
         }
       } else {
         // V rows past the end may hold anything (even NaN): zero them, 0 * NaN would poison
@@ -446,7 +569,7 @@ __global__ void __launch_bounds__(DecodeCfg<BS, D, KT, QF32>::NWARP * 32, 1)
         for (int dt = 0; dt < C::KS; ++dt) {
           uint32_t a0, a1, a2, a3;
           ldsm_x4_t(vb + mt * 2048 + voff[dt], a0, a1, a2, a3);
-          Mma<KT>::run(acc[dt], a0 & mlo, a1 & mlo, a2 & mhi, a3 & mhi, b0, b1);
+          Mma<MA>::run(acc[dt], a0 & mlo, a1 & mlo, a2 & mhi, a3 & mhi, b0, b1);
         }
       }
     }
@@ -457,19 +580,22 @@ __global__ void __launch_bounds__(DecodeCfg<BS, D, KT, QF32>::NWARP * 32, 1)
     const int hq0 = kvh * G + g0, hq1 = hq0 + 1;
     const float nan = CUDART_NAN_F;
     const float l0 = lacc[0], l1 = lacc[1];  // every row of the ones-MMA holds the column sums
+    // accumulator rows r0 and r0 + 8 of tile dt are columns d and d + dd
+    const int dd = C::FP8 ? 1 : 8;
+    const float vs = p.v_scale;
     if (np == 1) {
-      const float i0 = poisoned ? nan : 1.f / l0, i1 = poisoned ? nan : 1.f / l1;
+      const float i0 = poisoned ? nan : vs / l0, i1 = poisoned ? nan : vs / l1;
       const int64_t o0 = (static_cast<int64_t>(seq) * Hq + hq0) * D, o1 = o0 + D;
 #pragma unroll
       for (int dt = 0; dt < C::KS; ++dt) {
-        const int d = dt * 16 + r0;
+        const int d = dt * 16 + (C::FP8 ? 2 * r0 : r0);
         if (g0 < G) {
           store_out(p.out, o0 + d, acc[dt][0] * i0, p.out_dtype);
-          store_out(p.out, o0 + d + 8, acc[dt][2] * i0, p.out_dtype);
+          store_out(p.out, o0 + d + dd, acc[dt][2] * i0, p.out_dtype);
         }
         if (g1 < G) {
           store_out(p.out, o1 + d, acc[dt][1] * i1, p.out_dtype);
-          store_out(p.out, o1 + d + 8, acc[dt][3] * i1, p.out_dtype);
+          store_out(p.out, o1 + d + dd, acc[dt][3] * i1, p.out_dtype);
         }
       }
       return;
@@ -479,14 +605,14 @@ __global__ void __launch_bounds__(DecodeCfg<BS, D, KT, QF32>::NWARP * 32, 1)
     float* pa1 = pa0 + D;
 #pragma unroll
     for (int dt = 0; dt < C::KS; ++dt) {
-      const int d = dt * 16 + r0;
+      const int d = dt * 16 + (C::FP8 ? 2 * r0 : r0);
       if (g0 < G) {
-        __stcg(pa0 + d, poisoned ? nan : acc[dt][0]);
-        __stcg(pa0 + d + 8, poisoned ? nan : acc[dt][2]);
+        __stcg(pa0 + d, poisoned ? nan : acc[dt][0] * vs);
+        __stcg(pa0 + d + dd, poisoned ? nan : acc[dt][2] * vs);
       }
       if (g1 < G) {
-        __stcg(pa1 + d, poisoned ? nan : acc[dt][1]);
-        __stcg(pa1 + d + 8, poisoned ? nan : acc[dt][3]);
+        __stcg(pa1 + d, poisoned ? nan : acc[dt][1] * vs);
+        __stcg(pa1 + d + dd, poisoned ? nan : acc[dt][3] * vs);
       }
     }
     if (lane < 4) {

@@ -32,8 +32,12 @@ import numpy as np
 
 from .block_manager import BlockAllocator, BlockTable, tables_to_array
 
-ELEM_BYTES = {"f32": 4, "f16": 2, "bf16": 2}
-NAN_BITS = {"f16": 0x7E00, "bf16": 0x7FC0}
+ELEM_BYTES = {"f32": 4, "f16": 2, "bf16": 2, "e4m3": 1}
+NAN_BITS = {"f16": 0x7E00, "bf16": 0x7FC0, "e4m3": 0x7F}
+
+# Default per-tensor scales of an FP8 (E4M3) cache for N(0,1) data: |x| / scale stays well
+# inside the format's +-448 for every draw (|x| < 7).
+FP8_K_SCALE, FP8_V_SCALE = 0.0171, 0.0193
 
 # random streams
 _S_LENS, _S_PLACE, _S_Q, _S_HIST, _S_NEW, _S_EXTRA = range(6)
@@ -74,6 +78,15 @@ def storage_to_f32(a: np.ndarray, dtype: str) -> np.ndarray:
 _CHUNK = 1 << 22
 
 
+def to_e4m3_codes(x: np.ndarray, scale: float) -> np.ndarray:
+    """float32 values -> FP8 E4M3 codes of x / scale (torch's round-to-nearest-even cast),
+    clamped to the format's +-448 first."""
+    import torch
+    y = torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32)) / torch.tensor(np.float32(scale))
+    y = torch.clamp(y, -448.0, 448.0)
+    return y.to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+
+
 def _draw(key: Tuple[int, ...], shape, dtype: str) -> np.ndarray:
     """N(0,1) values rounded into ``dtype`` storage, generated in fixed 4 Mi-element chunks.
 
@@ -81,12 +94,15 @@ def _draw(key: Tuple[int, ...], shape, dtype: str) -> np.ndarray:
     and the element count, never on the thread count.
     """
     n = int(np.prod(shape, dtype=np.int64))
-    out = np.empty(n, dtype=np.float32 if dtype == "f32" else np.uint16)
+    fp8_scale = None
+    if isinstance(dtype, tuple):  # ("e4m3", scale): codes of N(0,1) / scale
+        dtype, fp8_scale = dtype
+    out = np.empty(n, dtype={"f32": np.float32, "e4m3": np.uint8}.get(dtype, np.uint16))
 
     def fill(c: int) -> None:
         lo, hi = c * _CHUNK, min(n, (c + 1) * _CHUNK)
         x = np.random.default_rng(list(key) + [c]).standard_normal(hi - lo, dtype=np.float32)
-        out[lo:hi] = to_storage(x, dtype)
+        out[lo:hi] = to_e4m3_codes(x, fp8_scale) if dtype == "e4m3" else to_storage(x, dtype)
 
     chunks = range(-(-n // _CHUNK))
     if n > _CHUNK:
@@ -131,6 +147,13 @@ class Workload:
     slot_mapping: np.ndarray      # int64 [T]
     copy_pairs: np.ndarray        # int32 [P, 2]
     notes: Dict[str, object] = dataclasses.field(default_factory=dict)
+    new_dtype: str = ""           # dtype of new_k / new_v ("" = kv_dtype)
+    k_scale: float = 1.0          # FP8 cache: value = code * scale
+    v_scale: float = 1.0
+
+    @property
+    def new_kv_dtype(self) -> str:
+        return self.new_dtype or self.kv_dtype
 
     @property
     def max_blocks_per_seq(self) -> int:
@@ -184,11 +207,14 @@ class Workload:
 def build_groups(name: str, groups: Sequence[Group], *, num_q_heads: int, num_kv_heads: int,
                  head_dim: int, block_size: int, q_dtype: str, kv_dtype: str, seed: int,
                  pool_factor: float = 1.25, num_blocks: Optional[int] = None,
-                 notes: Optional[dict] = None) -> Workload:
+                 notes: Optional[dict] = None, new_dtype: str = "bf16",
+                 k_scale: float = FP8_K_SCALE, v_scale: float = FP8_V_SCALE) -> Workload:
     """Materialise a decode step from groups of prefix-sharing sequences.
 
     Sequence order is group by group, member by member.  The pool holds
-    ``num_blocks`` blocks, or ceil(pool_factor * blocks the step needs).
+    ``num_blocks`` blocks, or ceil(pool_factor * blocks the step needs).  With kv_dtype
+    "e4m3" the pool holds FP8 codes of N(0,1) / scale, and the step's new tokens are
+    ``new_dtype`` values that the step itself quantises.
     """
     if num_q_heads % num_kv_heads:
         raise ValueError("num_q_heads must be a multiple of num_kv_heads")
@@ -234,19 +260,24 @@ def build_groups(name: str, groups: Sequence[Group], *, num_q_heads: int, num_kv
 
     # history: every group's prefix tokens, in group order, K then V
     nan = NAN_BITS[kv_dtype]
-    k_cache = np.full((num_blocks, bs, Hkv, D), nan, dtype=np.uint16)
-    v_cache = np.full((num_blocks, bs, Hkv, D), nan, dtype=np.uint16)
+    fp8 = kv_dtype == "e4m3"
+    pool_t = np.uint8 if fp8 else np.uint16
+    k_cache = np.full((num_blocks, bs, Hkv, D), nan, dtype=pool_t)
+    v_cache = np.full((num_blocks, bs, Hkv, D), nan, dtype=pool_t)
     hist_slots = np.concatenate([np.zeros(0, np.int64)] + prefix_slots)
     H = len(hist_slots)
+    kdt = ("e4m3", k_scale) if fp8 else kv_dtype
+    vdt = ("e4m3", v_scale) if fp8 else kv_dtype
     if H:
-        k_cache.reshape(num_blocks * bs, Hkv, D)[hist_slots] = _draw((seed, _S_HIST, 0), (H, Hkv, D), kv_dtype)
-        v_cache.reshape(num_blocks * bs, Hkv, D)[hist_slots] = _draw((seed, _S_HIST, 1), (H, Hkv, D), kv_dtype)
+        k_cache.reshape(num_blocks * bs, Hkv, D)[hist_slots] = _draw((seed, _S_HIST, 0), (H, Hkv, D), kdt)
+        v_cache.reshape(num_blocks * bs, Hkv, D)[hist_slots] = _draw((seed, _S_HIST, 1), (H, Hkv, D), vdt)
 
     all_slots = np.concatenate([np.zeros(0, np.int64)] +
                                [s for per_group in step_slots for s in per_group]).astype(np.int64)
     T = len(all_slots)
-    new_k = _draw((seed, _S_NEW, 0), (T, Hkv, D), kv_dtype)
-    new_v = _draw((seed, _S_NEW, 1), (T, Hkv, D), kv_dtype)
+    ndt = new_dtype if fp8 else kv_dtype
+    new_k = _draw((seed, _S_NEW, 0), (T, Hkv, D), ndt)
+    new_v = _draw((seed, _S_NEW, 1), (T, Hkv, D), ndt)
 
     seq_lens = np.asarray([t.num_tokens for t in tables], dtype=np.int32)
     block_tables = tables_to_array(tables)
@@ -258,13 +289,22 @@ def build_groups(name: str, groups: Sequence[Group], *, num_q_heads: int, num_kv
                     head_dim=head_dim, block_size=bs, num_blocks=num_blocks, q_dtype=q_dtype,
                     kv_dtype=kv_dtype, scale=float(np.float32(1.0 / math.sqrt(head_dim))), q=q,
                     k_cache=k_cache, v_cache=v_cache, block_tables=block_tables, seq_lens=seq_lens,
-                    new_k=new_k, new_v=new_v, slot_mapping=all_slots, copy_pairs=pairs, notes=info)
+                    new_k=new_k, new_v=new_v, slot_mapping=all_slots, copy_pairs=pairs, notes=info,
+                    new_dtype=ndt, k_scale=float(np.float32(k_scale)) if fp8 else 1.0,
+                    v_scale=float(np.float32(v_scale)) if fp8 else 1.0)
 
 
 def independent(name: str, seq_lens: Sequence[int], **kw) -> Workload:
     """Each sequence on its own; seq_lens are post-step lengths, the last token stored in the step."""
     groups = [Group(prefix=max(int(L) - 1, 0), step_tokens=[1 if L > 0 else 0]) for L in seq_lens]
     return build_groups(name, groups, **kw)
+
+
+def _fp8_kw(kw: dict) -> dict:
+    """Inside make_config(kv_dtype="e4m3"): the config's own dtype becomes the new tokens' dtype."""
+    if _FP8_OVERRIDE:
+        kw = dict(kw, new_dtype=kw["kv_dtype"], kv_dtype="e4m3")
+    return kw
 
 
 # ---------------------------------------------------------------------------------------
@@ -297,17 +337,17 @@ def _tiny(seed: int, block_size: int) -> Workload:
 def _7b(seed: int, block_size: int, num_seqs: int = 64) -> Workload:
     rng = np.random.default_rng([seed, _S_LENS])
     L = rng.integers(128, 2049, size=num_seqs)
-    return independent("7b", L, num_q_heads=32, num_kv_heads=32, head_dim=128, block_size=block_size,
-                       q_dtype="bf16", kv_dtype="bf16", seed=seed,
-                       notes={"lens": "uniform[128,2048]"})
+    return independent("7b", L, **_fp8_kw(dict(num_q_heads=32, num_kv_heads=32, head_dim=128, block_size=block_size,
+                                               q_dtype="bf16", kv_dtype="bf16", seed=seed,
+                                               notes={"lens": "uniform[128,2048]"})))
 
 
 def _13b(seed: int, block_size: int, num_seqs: int = 128) -> Workload:
     rng = np.random.default_rng([seed, _S_LENS])
     L = rng.integers(16, 2049, size=num_seqs)
-    return independent(f"13b-bs{block_size}", L, num_q_heads=40, num_kv_heads=40, head_dim=128,
-                       block_size=block_size, q_dtype="f16", kv_dtype="f16", seed=seed,
-                       notes={"lens": "uniform[16,2048]"})
+    return independent(f"13b-bs{block_size}", L, **_fp8_kw(dict(num_q_heads=40, num_kv_heads=40, head_dim=128,
+                                                             block_size=block_size, q_dtype="f16", kv_dtype="f16",
+                                                             seed=seed, notes={"lens": "uniform[16,2048]"})))
 
 
 def lognormal_lengths(rng: np.random.Generator, n: int, median: float = 1024.0, sigma: float = 1.0,
@@ -319,9 +359,10 @@ def lognormal_lengths(rng: np.random.Generator, n: int, median: float = 1024.0, 
 def _8b(seed: int, block_size: int, num_seqs: int = 256) -> Workload:
     rng = np.random.default_rng([seed, _S_LENS])
     L = lognormal_lengths(rng, num_seqs)
-    return independent("8b", L, num_q_heads=32, num_kv_heads=8, head_dim=128, block_size=block_size,
-                       q_dtype="bf16", kv_dtype="bf16", seed=seed,
-                       notes={"lens": "lognormal(median 1024, sigma 1.0) clipped to [32, 8192]"})
+    return independent("8b", L, **_fp8_kw(dict(num_q_heads=32, num_kv_heads=8, head_dim=128, block_size=block_size,
+                                               q_dtype="bf16", kv_dtype="bf16", seed=seed,
+                                               notes={"lens": "lognormal(median 1024, sigma 1.0) clipped to "
+                                                              "[32, 8192]"})))
 
 
 def _70b(seed: int, block_size: int, num_groups: int = 64, samples: int = 4,
@@ -338,10 +379,12 @@ def _70b(seed: int, block_size: int, num_groups: int = 64, samples: int = 4,
         suffix = [int(x) for x in rng.integers(1, 513, size=samples)]
         groups.append(Group(prefix + r, suffix))
     groups += [Group(long_len - 1, [1]) for _ in range(num_long)]
-    return build_groups("70b", groups, num_q_heads=64, num_kv_heads=8, head_dim=128,
-                        block_size=block_size, q_dtype="bf16", kv_dtype="bf16", seed=seed,
-                        notes={"lens": "64 groups x 4 samples: prefix 4096+r (r in [1,bs-1]) + "
-                                       "suffix uniform[1,512]; plus 4 x 32768"})
+    return build_groups("70b", groups, **_fp8_kw(dict(num_q_heads=64, num_kv_heads=8, head_dim=128,
+                                                      block_size=block_size, q_dtype="bf16", kv_dtype="bf16",
+                                                      seed=seed,
+                                                      notes={"lens": "64 groups x 4 samples: prefix 4096+r "
+                                                                     "(r in [1,bs-1]) + suffix uniform[1,512]; "
+                                                                     "plus 4 x 32768"})))
 
 
 _BUILDERS = {"tiny": _tiny, "7b": _7b, "13b": _13b, "8b": _8b, "70b": _70b}
@@ -349,19 +392,34 @@ _DEFAULT_BS = {"tiny": 16, "7b": 16, "13b": 16, "8b": 16, "70b": 16}
 
 
 def make_config(name: str, block_size: Optional[int] = None, seed: Optional[int] = None,
-                **overrides) -> Workload:
-    """Build one of the named decode configs ("tiny", "7b", "13b", "8b", "70b")."""
+                kv_dtype: Optional[str] = None, **overrides) -> Workload:
+    """Build one of the named decode configs ("tiny", "7b", "13b", "8b", "70b").
+
+    kv_dtype="e4m3" gives the same config over an FP8 cache (head_dim 128 configs): the
+    history is stored as FP8 codes, the step's new tokens stay in the config's dtype.
+    """
     if name not in _BUILDERS:
         raise KeyError(f"unknown config {name!r}; choose from {CONFIG_NAMES}")
     bs = block_size or _DEFAULT_BS[name]
-    return _BUILDERS[name](config_seed(name) if seed is None else seed, bs, **overrides)
+    global _FP8_OVERRIDE
+    _FP8_OVERRIDE = kv_dtype == "e4m3"
+    try:
+        return _BUILDERS[name](config_seed(name) if seed is None else seed, bs, **overrides)
+    finally:
+        _FP8_OVERRIDE = False
+
+
+_FP8_OVERRIDE = False
 
 
 def apply_step_host(w: Workload) -> Tuple[np.ndarray, np.ndarray]:
     """The post-step caches computed with plain numpy indexing (no kernel, no oracle).
 
-    Used only to give tests an independent expectation of the cache state.
+    Used only to give tests an independent expectation of the cache state.  Not defined for
+    an FP8 cache, whose step quantises the new tokens.
     """
+    if w.kv_dtype == "e4m3":
+        raise ValueError("the post-step state of an FP8 cache needs the quantising store")
     kc, vc = w.k_cache.copy(), w.v_cache.copy()
     for s, d in w.copy_pairs:
         kc[d] = kc[s]
