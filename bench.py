@@ -50,6 +50,8 @@ def parse_args():
     ap.add_argument("--steps", type=int, default=3000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--op", choices=["step", "swap"], default="step",
+                    help="step: the decode step (default); swap: swap_blocks to / from pinned host memory")
     ap.add_argument("--config", default="8b", choices=list(W.CONFIG_NAMES))
     ap.add_argument("--block-size", type=int, default=None)
     ap.add_argument("--num-seqs", type=int, default=None, help="smaller batch of the same config (profiling)")
@@ -453,10 +455,68 @@ def run_ours(args):
     return 0
 
 
+def run_swap(args):
+    """swap_blocks: a quarter of the config's sequences swapped out to pinned host memory and back,
+    against plain bulk copies between the same kinds of memory (the host link's roofline)."""
+    from paged_kv_cache_327_b200 import binding as B
+    from paged_kv_cache_327_b200 import build as pkg_build
+
+    pkg_build.build()
+    w = W.make_config(args.config, block_size=args.block_size, kv_dtype=args.kv_dtype)
+    dw = B.device_workload(w)
+    bs = w.block_size
+    seqs = range(w.num_seqs // 4)
+    blocks = np.asarray([int(b) for i in seqs for b in w.block_tables[i, :-(-int(w.seq_lens[i]) // bs)]], np.int32)
+    n = len(blocks)
+    hk = torch.empty((n,) + tuple(dw.k_cache.shape[1:]), dtype=dw.k_cache.dtype).pin_memory()
+    hv = torch.empty_like(hk).pin_memory()
+    out_pairs = torch.from_numpy(np.stack([blocks, np.arange(n, dtype=np.int32)], 1)).cuda()
+    in_pairs = torch.from_numpy(np.stack([np.arange(n, dtype=np.int32), blocks], 1)).cuda()
+    nbytes = 2 * n * w.block_bytes
+    stream = torch.cuda.current_stream()
+
+    def timed(fn, reps):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(True), torch.cuda.Event(True)
+        a.record(stream)
+        for _ in range(reps):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / reps * 1e-3
+
+    reps = max(3, min(args.steps, 50))
+    t_out = timed(lambda: B.pa_swap_blocks(hk, hv, dw.k_cache, dw.v_cache, out_pairs, stream=stream), reps)
+    t_in = timed(lambda: B.pa_swap_blocks(dw.k_cache, dw.v_cache, hk, hv, in_pairs, stream=stream), reps)
+    assert B.pa_get_device_error() == B.PA_DEV_OK
+    dbuf = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    hbuf = torch.empty(nbytes, dtype=torch.uint8).pin_memory()
+    t_d2h = timed(lambda: hbuf.copy_(dbuf, non_blocking=True), reps)
+    t_h2d = timed(lambda: dbuf.copy_(hbuf, non_blocking=True), reps)
+    line = {
+        "metric": "swap_blocks GB/s between the GPU pool and pinned host memory", "op": "swap",
+        "value": round(nbytes / t_in / 1e9, 2), "unit": "GB/s", "n_gpus": 1, "steps": reps,
+        "higher_is_better": True, "data": "synthetic", "dtype": w.kv_dtype,
+        "config": {"workload": workload_label(w), "blocks": n, "block_bytes": w.block_bytes, "bytes_per_swap": nbytes},
+        "swap_out_gbs": round(nbytes / t_out / 1e9, 2), "swap_in_gbs": round(nbytes / t_in / 1e9, 2),
+        "roofline": {"bound": "host link", "unit": "GB/s",
+                     "peak_d2h": round(nbytes / t_d2h / 1e9, 2), "peak_h2d": round(nbytes / t_h2d / 1e9, 2),
+                     "frac_out": round(t_d2h / t_out, 4), "frac_in": round(t_h2d / t_in, 4),
+                     "peak_source": "cudaMemcpyAsync of one contiguous pinned buffer of the same size, this run"},
+        "gpu_launches": 2 * reps,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     args = parse_args()
     if args.impl == "reference":
         return run_reference(args)
+    if args.op == "swap":
+        return run_swap(args)
     return run_ours(args)
 
 

@@ -155,6 +155,22 @@ PA_API int pa_copy_blocks(void* k_cache, void* v_cache, const int32_t* src_dst_p
                    int64_t num_blocks, size_t block_bytes, const int32_t* host_pairs,
                    void* stream);
 
+/* Swap KV blocks between two pools -- preemption ("详解vLLM推理引擎架构", scheduler section:
+ * when GPU memory runs short the KV cache of low-priority requests is moved to CPU memory and
+ * brought back later; --swap-space).  For each pair p, block src_dst_pairs[p][0] of
+ * (src_k_cache, src_v_cache) is copied to block src_dst_pairs[p][1] of (dst_k_cache,
+ * dst_v_cache), block_bytes bytes each (a multiple of 16; any element type).
+ *   pools        either side may be device memory or pinned host memory that the device
+ *                addresses directly (cudaHostAlloc / cudaHostRegister, mapped); 16-byte aligned
+ *   src_dst_pairs int32 [num_pairs, 2], device-addressable (device or pinned host memory)
+ * One kernel launch for all pairs.  Destinations should be distinct; ids outside
+ * [0, num_src_blocks) / [0, num_dst_blocks) are skipped and reported through
+ * pa_get_device_error(). */
+PA_API int pa_swap_blocks(void* dst_k_cache, void* dst_v_cache, const void* src_k_cache,
+                          const void* src_v_cache, const int32_t* src_dst_pairs, int num_pairs,
+                          int64_t num_src_blocks, int64_t num_dst_blocks, size_t block_bytes,
+                          void* stream);
+
 /* Static description of a pa_status value. */
 PA_API const char* pa_strerror(int status);
 

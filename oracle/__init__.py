@@ -14,6 +14,8 @@ What each function follows (web pages on vLLM / PagedAttention):
     stores each new token's K/V into its slot before attention runs).
   * ``copy_blocks`` -- "详解vLLM推理引擎架构", section "Copy-on-Write 与内存共享"
     (copy_block(old, new) before writing a shared block).
+  * ``swap_blocks`` -- "详解vLLM推理引擎架构", scheduler section (preempted requests' KV
+    cache swapped out to CPU memory and back).
   * ``reshape_and_cache_e4m3`` / ``decode(..., kv_dtype="e4m3")`` -- the FP8 KV cache of
     "详解vLLM推理引擎架构", section "量化集成与部署" (--kv-cache-dtype fp8), read as OCP E4M3
     codes with one fp32 scale for K and one for V.
@@ -64,6 +66,8 @@ def _load(path=None):
     lib.oracle_e4m3_to_f64.restype = ctypes.c_double
     lib.oracle_f32_to_e4m3.argtypes = [ctypes.c_float]
     lib.oracle_f32_to_e4m3.restype = ctypes.c_uint8
+    lib.oracle_swap_blocks.argtypes = [P, P, P, P, P, i64, i64, i64, i64]
+    lib.oracle_swap_blocks.restype = i32
     lib.oracle_f16_to_f64.argtypes = [ctypes.c_uint16]
     lib.oracle_f16_to_f64.restype = ctypes.c_double
     lib.oracle_bf16_to_f64.argtypes = [ctypes.c_uint16]
@@ -183,6 +187,23 @@ def copy_blocks(k_cache, v_cache, pairs, lib=None):
                                 block_bytes)
     if rc != 0:
         raise OracleError(f"oracle_copy_blocks failed with status {rc}")
+
+
+def swap_blocks(dst_k, dst_v, src_k, src_v, pairs, lib=None):
+    """In place: for each (src, dst) row of pairs, in order, copy block src of the source pool
+    (src_k, src_v) to block dst of the destination pool (dst_k, dst_v)."""
+    lib = lib or _load()
+    for a in (dst_k, dst_v, src_k, src_v):
+        if not a.flags.c_contiguous:
+            raise ValueError("pools must be C-contiguous")
+    pairs = np.ascontiguousarray(pairs, dtype=np.int32).reshape(-1, 2)
+    block_bytes = src_k.nbytes // src_k.shape[0]
+    if dst_k.nbytes // dst_k.shape[0] != block_bytes:
+        raise ValueError("the pools' blocks differ in size")
+    rc = lib.oracle_swap_blocks(_ptr(dst_k), _ptr(dst_v), _ptr(src_k), _ptr(src_v), _ptr(pairs), pairs.shape[0],
+                                src_k.shape[0], dst_k.shape[0], block_bytes)
+    if rc != 0:
+        raise OracleError(f"oracle_swap_blocks failed with status {rc}")
 
 
 def f16_to_f64(bits: int) -> float:

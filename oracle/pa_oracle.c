@@ -141,6 +141,28 @@ int oracle_copy_blocks(uint8_t* k_cache, uint8_t* v_cache, const int32_t* pairs,
   return OR_OK;
 }
 
+/* swap_blocks: block pairs[p][0] of the source pool is copied to block pairs[p][1] of the
+ * destination pool (K and V), for every pair in order -- moving a preempted sequence's blocks
+ * to CPU memory and back ("详解vLLM推理引擎架构", scheduler section: the KV cache of
+ * low-priority requests is swapped out to CPU memory when GPU memory runs short and
+ * swapped back later; --swap-space). */
+int oracle_swap_blocks(uint8_t* dst_k, uint8_t* dst_v, const uint8_t* src_k, const uint8_t* src_v,
+                       const int32_t* pairs, int64_t num_pairs, int64_t num_src_blocks,
+                       int64_t num_dst_blocks, int64_t block_bytes) {
+  if (num_pairs < 0 || block_bytes <= 0 || num_src_blocks <= 0 || num_dst_blocks <= 0) return OR_ERR_ARG;
+  if (num_pairs > 0 && (!dst_k || !dst_v || !src_k || !src_v || !pairs)) return OR_ERR_ARG;
+  for (int64_t p = 0; p < num_pairs; ++p) {
+    int64_t s = pairs[2 * p], d = pairs[2 * p + 1];
+    if (s < 0 || s >= num_src_blocks || d < 0 || d >= num_dst_blocks) return OR_ERR_RANGE;
+  }
+  for (int64_t p = 0; p < num_pairs; ++p) {
+    int64_t s = pairs[2 * p], d = pairs[2 * p + 1];
+    memcpy(dst_k + d * block_bytes, src_k + s * block_bytes, (size_t)block_bytes);
+    memcpy(dst_v + d * block_bytes, src_v + s * block_bytes, (size_t)block_bytes);
+  }
+  return OR_OK;
+}
+
 /* reshape_and_cache: token t with slot s >= 0 goes to physical block s / block_size,
  * position s % block_size, for every KV head.  k / v are [num_tokens, num_kv_heads,
  * head_dim] with a row stride of token_stride elements between tokens. */

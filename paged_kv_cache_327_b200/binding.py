@@ -24,7 +24,7 @@ PA_DEV_OK, PA_DEV_BAD_BLOCK_ID, PA_DEV_BAD_SEQ_LEN, PA_DEV_BAD_SLOT, PA_DEV_BAD_
 
 EXPORTED = ("pa_decode_workspace_size", "pa_decode", "pa_reshape_and_cache", "pa_copy_blocks",
             "pa_strerror", "pa_get_device_error", "pa_version", "pa_decode_static_workspace",
-            "pa_decode_fp8", "pa_reshape_and_cache_fp8")
+            "pa_decode_fp8", "pa_reshape_and_cache_fp8", "pa_swap_blocks")
 PA_ERR_TOO_LARGE = -5
 PA_DECODE_STATIC_WORKSPACE_BYTES = 64 << 20
 
@@ -66,6 +66,8 @@ def load_library(path: str = _LIB_PATH):
     lib.pa_decode_fp8.restype = I
     lib.pa_reshape_and_cache_fp8.argtypes = [P, P, P, P, P, I, I, I, I, I64, I, F, F, I64, I64, P]
     lib.pa_reshape_and_cache_fp8.restype = I
+    lib.pa_swap_blocks.argtypes = [P, P, P, P, P, I, I64, I64, SZ, P]
+    lib.pa_swap_blocks.restype = I
     if path == _LIB_PATH:
         _lib = lib
     return lib
@@ -207,6 +209,22 @@ def pa_copy_blocks(k_cache: torch.Tensor, v_cache: torch.Tensor, src_dst_pairs: 
         _ptr(k_cache), _ptr(v_cache), _ptr(src_dst_pairs), P, NB, block_bytes,
         ctypes.c_void_p(hp.ctypes.data) if hp is not None else ctypes.c_void_p(0), _stream(stream))
     _check(rc, "pa_copy_blocks")
+
+
+def pa_swap_blocks(dst_k: torch.Tensor, dst_v: torch.Tensor, src_k: torch.Tensor, src_v: torch.Tensor,
+                   src_dst_pairs: torch.Tensor, stream=None) -> None:
+    """Copy block pairs[p,0] of the source pool to block pairs[p,1] of the destination pool.
+
+    Either pool may be a pinned host tensor (``pin_memory()``), which the device addresses
+    directly; ``src_dst_pairs`` (int32 [P, 2]) must be on the device or in pinned memory.
+    """
+    block_bytes = src_k[0].numel() * src_k.element_size()
+    if dst_k[0].numel() * dst_k.element_size() != block_bytes:
+        raise ValueError("the pools' blocks differ in size")
+    rc = load_library().pa_swap_blocks(_ptr(dst_k), _ptr(dst_v), _ptr(src_k), _ptr(src_v), _ptr(src_dst_pairs),
+                                       src_dst_pairs.shape[0], src_k.shape[0], dst_k.shape[0], block_bytes,
+                                       _stream(stream))
+    _check(rc, "pa_swap_blocks")
 
 
 def pa_get_device_error(stream=None) -> int:

@@ -22,7 +22,10 @@ Readings where the pages are silent or inconsistent:
     ``free`` drops one reference and returns the block to the pool at zero;
   * block copies are not executed on the host: ``copy_block`` records a (src, dst)
     pair that the device operation ``pa_copy_blocks`` carries out before the step's
-    writes.
+    writes;
+  * preemption ("详解vLLM推理引擎架构", scheduler section: a low-priority request's KV cache
+    is moved to CPU memory and back): ``swap_out`` / ``swap_in`` move whole sequence groups
+    between a GPU and a CPU allocator and return the block pairs for ``pa_swap_blocks``.
 """
 from __future__ import annotations
 
@@ -203,3 +206,34 @@ def tables_to_array(tables: Iterable[BlockTable], max_blocks: Optional[int] = No
             raise ValueError("a table is wider than max_blocks")
         out[i, :len(blocks)] = blocks
     return out
+
+
+def _move_tables(tables: Iterable[BlockTable], src: BlockAllocator, dst: BlockAllocator) -> np.ndarray:
+    """Move every block the tables reference from pool ``src`` to pool ``dst``.
+
+    A block shared by several of the tables moves once and stays shared (its new refcount is
+    the number of references among the tables).  Returns the (src, dst) block pairs, in first-
+    reference order, and repoints the tables to the new ids.
+    """
+    mapping = {}
+    pairs = []
+    for t in tables:
+        for i, b in enumerate(t._blocks):
+            if b in mapping:
+                dst.increment_refcount(mapping[b])
+            else:
+                mapping[b] = dst.allocate()
+                pairs.append((b, mapping[b]))
+            t._blocks[i] = mapping[b]
+            src.free(b)
+    return np.asarray(pairs, dtype=np.int32).reshape(-1, 2)
+
+
+def swap_out(tables: Iterable[BlockTable], gpu: BlockAllocator, cpu: BlockAllocator) -> np.ndarray:
+    """Preempt a sequence group: its blocks move to the CPU pool (pairs gpu -> cpu)."""
+    return _move_tables(tables, gpu, cpu)
+
+
+def swap_in(tables: Iterable[BlockTable], cpu: BlockAllocator, gpu: BlockAllocator) -> np.ndarray:
+    """Resume a swapped sequence group: its blocks move back to the GPU pool (pairs cpu -> gpu)."""
+    return _move_tables(tables, cpu, gpu)

@@ -406,6 +406,25 @@ int pa_copy_blocks(void* k_cache, void* v_cache, const int32_t* src_dst_pairs, i
   return cudaPeekAtLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
+int pa_swap_blocks(void* dst_k_cache, void* dst_v_cache, const void* src_k_cache, const void* src_v_cache,
+                   const int32_t* src_dst_pairs, int num_pairs, int64_t num_src_blocks, int64_t num_dst_blocks,
+                   size_t block_bytes, void* stream) {
+  if (num_pairs < 0 || num_src_blocks <= 0 || num_dst_blocks <= 0 || block_bytes == 0 || block_bytes % 16)
+    return PA_ERR_INVALID;
+  if (num_pairs == 0) return PA_OK;
+  if (!dst_k_cache || !dst_v_cache || !src_k_cache || !src_v_cache || !src_dst_pairs) return PA_ERR_INVALID;
+  if (!aligned16(dst_k_cache) || !aligned16(dst_v_cache) || !aligned16(src_k_cache) || !aligned16(src_v_cache))
+    return PA_ERR_INVALID;
+  const int64_t vecs = static_cast<int64_t>(block_bytes / 16);
+  const int chunks = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(16, vecs / (256 * 4))));
+  pa::pa_swap_blocks_kernel<<<dim3(static_cast<unsigned>(num_pairs), 2, static_cast<unsigned>(chunks)), 256, 0,
+                              static_cast<cudaStream_t>(stream)>>>(
+      static_cast<uint8_t*>(dst_k_cache), static_cast<uint8_t*>(dst_v_cache), static_cast<const uint8_t*>(src_k_cache),
+      static_cast<const uint8_t*>(src_v_cache), src_dst_pairs, num_src_blocks, num_dst_blocks,
+      static_cast<int64_t>(block_bytes));
+  return cudaPeekAtLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
 int pa_get_device_error(void* stream) {
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (cudaStreamSynchronize(st) != cudaSuccess) return PA_ERR_CUDA;

@@ -110,3 +110,36 @@ __global__ void __launch_bounds__(256)
 }
 
 }  // namespace pa
+
+namespace pa {
+
+// Swap: block pairs[p][0] of the source pool goes to block pairs[p][1] of the destination pool
+// (K and V).  Either pool may be pinned host memory the device addresses directly, so each
+// thread keeps four independent 16-byte loads in flight to cover the host link's latency.
+// grid: (num_pairs, 2 [K, V], chunks)
+__global__ void __launch_bounds__(256)
+    pa_swap_blocks_kernel(uint8_t* __restrict__ dk, uint8_t* __restrict__ dv, const uint8_t* __restrict__ sk,
+                          const uint8_t* __restrict__ sv, const int32_t* __restrict__ pairs, int64_t num_src,
+                          int64_t num_dst, int64_t block_bytes) {
+  const int64_t src = pairs[2 * static_cast<int64_t>(blockIdx.x)];
+  const int64_t dst = pairs[2 * static_cast<int64_t>(blockIdx.x) + 1];
+  if (src < 0 || src >= num_src || dst < 0 || dst >= num_dst) {
+    if (threadIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0) record_error(DEV_BAD_PAIR);
+    return;
+  }
+  const uint4* s = reinterpret_cast<const uint4*>((blockIdx.y ? sv : sk) + src * block_bytes);
+  uint4* d = reinterpret_cast<uint4*>((blockIdx.y ? dv : dk) + dst * block_bytes);
+  const int64_t vecs = block_bytes >> 4;
+  const int64_t stride = static_cast<int64_t>(blockDim.x) * gridDim.z;
+  int64_t i = threadIdx.x + static_cast<int64_t>(blockIdx.z) * blockDim.x;
+  for (; i + 3 * stride < vecs; i += 4 * stride) {
+    const uint4 a = s[i], b = s[i + stride], c = s[i + 2 * stride], e = s[i + 3 * stride];
+    d[i] = a;
+    d[i + stride] = b;
+    d[i + 2 * stride] = c;
+    d[i + 3 * stride] = e;
+  }
+  for (; i < vecs; i += stride) d[i] = s[i];
+}
+
+}  // namespace pa

@@ -165,3 +165,29 @@ def test_named_config_shapes(name):
     if name != "70b":
         used = np.concatenate([w.block_tables[i, :-(-int(l) // w.block_size)] for i, l in enumerate(L)])
         assert len(np.unique(used)) == len(used)
+
+
+def test_swap_out_and_in_move_groups_and_keep_sharing():
+    from paged_kv_cache_327_b200.block_manager import swap_in, swap_out
+    gpu = BlockAllocator(16, 4, seed=11)
+    cpu = BlockAllocator(8, 4, seed=12)
+    parent = BlockTable(4)
+    parent.append_tokens(9, gpu)                      # 3 blocks
+    child = BlockTable(4)
+    child.fork_from(parent, gpu)
+    child.append_token(gpu)                           # copy-on-write of the partial block
+    gpu.take_pending_copies()
+    before_free = gpu.get_num_free_blocks()
+    old = (parent.get_physical_blocks(), child.get_physical_blocks())
+    pairs = swap_out([parent, child], gpu, cpu)
+    # 2 shared full blocks + 2 private last blocks = 4 distinct blocks move once each
+    assert len(pairs) == 4 and len(set(pairs[:, 0])) == 4 and len(set(pairs[:, 1])) == 4
+    assert gpu.get_num_free_blocks() == before_free + 4
+    m = {int(a): int(b) for a, b in pairs}
+    assert parent.get_physical_blocks() == [m[b] for b in old[0]]
+    assert child.get_physical_blocks() == [m[b] for b in old[1]]
+    assert cpu.get_refcount(parent.get_block_number(0)) == 2          # still shared on the CPU side
+    back = swap_in([parent, child], cpu, gpu)
+    assert len(back) == 4 and cpu.get_num_free_blocks() == 8
+    assert gpu.get_refcount(parent.get_block_number(0)) == 2
+    assert parent.get_block_number(0) == child.get_block_number(0)

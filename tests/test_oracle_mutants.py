@@ -52,6 +52,9 @@ MUTANTS = {
     "e4m3_store_multiplies": ("float qk = xk / k_scale;", "float qk = xk * k_scale;"),
     "e4m3_k_scale_dropped": ("if (J->kv_dtype == OR_E4M3) s *= J->k_scale;", ""),
     "e4m3_v_scale_dropped": ("for (int d = 0; d < D; ++d) o[d] *= J->v_scale;", ";"),
+    "swap_direction": ("memcpy(dst_k + d * block_bytes, src_k + s * block_bytes, (size_t)block_bytes);",
+                       "memcpy(dst_k + s * block_bytes, src_k + d * block_bytes, (size_t)block_bytes);"),
+    "swap_skips_v": ("    memcpy(dst_v + d * block_bytes, src_v + s * block_bytes, (size_t)block_bytes);\n", ""),
     "copy_skips_v": ("    memmove(v_cache + dst * block_bytes, v_cache + src * block_bytes, (size_t)block_bytes);\n",
                      ""),
 }

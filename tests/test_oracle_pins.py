@@ -417,7 +417,23 @@ def check_decode_e4m3_vs_sdpa(lib):
         assert np.max(np.abs(got - ref)) < 1e-12, n
 
 
-ALL_CHECKS = [check_f16_decode, check_bf16_decode, check_decode_vs_sdpa, check_closed_forms,
+def check_swap_blocks(lib):
+    rng = _rng(81)
+    src_k = rng.integers(0, 256, size=(7, 16, 2, 64, 2), dtype=np.uint8)
+    src_v = rng.integers(0, 256, size=src_k.shape, dtype=np.uint8)
+    dst_k = rng.integers(0, 256, size=(5, 16, 2, 64, 2), dtype=np.uint8)
+    dst_v = rng.integers(0, 256, size=dst_k.shape, dtype=np.uint8)
+    pairs = np.asarray([[6, 0], [2, 4], [0, 1]], np.int32)
+    ek, ev = dst_k.copy(), dst_v.copy()
+    for s_, d_ in pairs:
+        ek[d_], ev[d_] = src_k[s_], src_v[s_]
+    sk, sv = src_k.copy(), src_v.copy()
+    oracle.swap_blocks(dst_k, dst_v, src_k, src_v, pairs, lib=lib)
+    assert np.array_equal(dst_k, ek) and np.array_equal(dst_v, ev)
+    assert np.array_equal(src_k, sk) and np.array_equal(src_v, sv), "the source pool is left as it was"
+
+
+ALL_CHECKS = [check_swap_blocks, check_f16_decode, check_bf16_decode, check_decode_vs_sdpa, check_closed_forms,
               check_page_block_table_example, check_invariants, check_cow_leaves_parent,
               check_reshape_and_cache, check_copy_blocks, check_e4m3_decode, check_e4m3_encode,
               check_reshape_and_cache_e4m3, check_decode_e4m3_vs_sdpa]
