@@ -59,6 +59,9 @@ def _load(path=None):
     lib.oracle_decode_scaled.argtypes = [P, P, i32, P, P, i32, P, P, i32, i32, i32, i32, i32, i32, i64,
                                          ctypes.c_float, ctypes.c_float, ctypes.c_float, i32]
     lib.oracle_decode_scaled.restype = i32
+    lib.oracle_decode_multi.argtypes = [P, P, i32, P, P, i32, P, P, i32, i32, i32, i32, i32, i32, i32, i64,
+                                        ctypes.c_float, i32]
+    lib.oracle_decode_multi.restype = i32
     lib.oracle_reshape_and_cache_e4m3.argtypes = [P, P, P, P, P, i64, i32, i32, i32, i64, i32,
                                                   ctypes.c_float, ctypes.c_float, i64, i64]
     lib.oracle_reshape_and_cache_e4m3.restype = i32
@@ -135,6 +138,40 @@ def decode(q, q_dtype, k_cache, v_cache, kv_dtype, block_tables, seq_lens, scale
                                MB, NB, ctypes.c_float(scale), threads)
     if rc != 0:
         raise OracleError(f"oracle_decode failed with status {rc}")
+    return out
+
+
+def decode_multi(q, q_dtype, k_cache, v_cache, kv_dtype, block_tables, seq_lens, scale, num_threads=None,
+                 lib=None):
+    """fp64 causal multi-token attention over the paged cache.
+
+    q: [N, T, Hq, D] in q_dtype storage; query token t of sequence i is the token at position
+    seq_lens[i] - T + t and attends to tokens 0 .. seq_lens[i] - T + t (a sequence holds 0
+    or at least T tokens).  Caches, block_tables and seq_lens as in decode (16-bit or f32
+    caches).  Returns float64 [N, T, Hq, D].
+    """
+    lib = lib or _load()
+    _check_storage(q, q_dtype, "q")
+    _check_storage(k_cache, kv_dtype, "k_cache")
+    _check_storage(v_cache, kv_dtype, "v_cache")
+    if kv_dtype == "e4m3":
+        raise ValueError("decode_multi takes a 16-bit or f32 cache")
+    block_tables = np.ascontiguousarray(block_tables, dtype=np.int32)
+    seq_lens = np.ascontiguousarray(seq_lens, dtype=np.int32)
+    N, T, Hq, D = q.shape
+    NB, bs, Hkv, D2 = k_cache.shape
+    if D2 != D or v_cache.shape != k_cache.shape:
+        raise ValueError("shape mismatch between q and the caches")
+    if block_tables.ndim != 2 or block_tables.shape[0] != N or seq_lens.shape != (N,):
+        raise ValueError("block_tables must be [N, MB] and seq_lens [N]")
+    MB = block_tables.shape[1]
+    out = np.zeros((N, T, Hq, D), dtype=np.float64)
+    threads = num_threads if num_threads else default_threads()
+    rc = lib.oracle_decode_multi(_ptr(out), _ptr(q), DTYPES[q_dtype], _ptr(k_cache), _ptr(v_cache),
+                                 DTYPES[kv_dtype], _ptr(block_tables), _ptr(seq_lens), N, T, Hq, Hkv, D, bs, MB,
+                                 NB, ctypes.c_float(scale), threads)
+    if rc != 0:
+        raise OracleError(f"oracle_decode_multi failed with status {rc}")
     return out
 
 

@@ -26,6 +26,11 @@
  *  - "详解vLLM推理引擎架构", section "量化集成与部署": the KV cache may be stored in FP8
  *    (--kv-cache-dtype fp8).  The page names no format; read here as OCP E4M3 with one
  *    fp32 scale for K and one for V: stored code = e4m3(x / scale), value = code * scale.
+ *  - same page, sections "量化集成与部署" (speculative decoding: the large model checks N
+ *    draft tokens at once) and "Chunked Prefill" (a prompt is processed in chunks): several
+ *    query tokens of one sequence attend to the paged cache in one call.  The page gives no
+ *    formula; read as causal attention of the sequence's last T tokens, already in the
+ *    cache: query token tq (position L - T + tq) sees tokens 0 .. L - T + tq.
  *
  * Readings where the pages are silent or inconsistent:
  *  - the printed kernel indexes K with the query head although it receives
@@ -235,6 +240,7 @@ typedef struct {
   int kv_dtype;
   const int32_t* block_tables;
   const int32_t* seq_lens;
+  int num_q_tokens;          /* query tokens per sequence (1 = decode) */
   int num_q_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq;
   double scale;
   double k_scale, v_scale;   /* dequantisation scales of an E4M3 cache (1 otherwise) */
@@ -267,15 +273,19 @@ static void* decode_worker(void* arg) {
       scores = (double*)malloc(cap * sizeof(double));
       if (!scores) { J->status = OR_ERR_NOMEM; return NULL; }
     }
+    const int T = J->num_q_tokens;
+    for (int tq = 0; tq < T; ++tq)
     for (int hq = 0; hq < J->num_q_heads; ++hq) {
       const int h = hq / G;                       /* KV head shared by this query head */
-      const int64_t qo = ((int64_t)i * J->num_q_heads + hq) * D;
+      const int64_t qo = (((int64_t)i * T + tq) * J->num_q_heads + hq) * D;
       double* o = J->out + qo;
       for (int d = 0; d < D; ++d) o[d] = 0.0;
       if (L == 0) continue;
+      /* query token tq sits at position L - T + tq and sees the tokens up to its own */
+      const int n = L - T + tq + 1;
       /* pass 1: scores and their maximum */
       double m = -INFINITY;
-      for (int t = 0; t < L; ++t) {
+      for (int t = 0; t < n; ++t) {
         double s = 0.0;
         for (int d = 0; d < D; ++d)
           s += load_elem(J->q, qo + d, J->q_dtype) *
@@ -287,7 +297,7 @@ static void* decode_worker(void* arg) {
       }
       /* pass 2: softmax weights and the weighted sum of V rows */
       double z = 0.0;
-      for (int t = 0; t < L; ++t) {
+      for (int t = 0; t < n; ++t) {
         double w = exp(scores[t] - m);
         z += w;
         for (int d = 0; d < D; ++d)
@@ -301,6 +311,12 @@ static void* decode_worker(void* arg) {
   free(scores);
   return NULL;
 }
+
+static int decode_common(double* out, const void* q, int q_dtype, const void* k_cache,
+                         const void* v_cache, int kv_dtype, const int32_t* block_tables,
+                         const int32_t* seq_lens, int num_seqs, int num_q_tokens, int num_q_heads,
+                         int num_kv_heads, int head_dim, int block_size, int max_blocks_per_seq,
+                         int64_t num_blocks, float scale, float k_scale, float v_scale, int num_threads);
 
 /* Decode attention: out[i, hq, :] = softmax_t(scale * q[i,hq,:] . K_t) V_t over the
  * seq_lens[i] tokens of sequence i, K_t / V_t gathered through block_tables.
@@ -330,8 +346,32 @@ int oracle_decode_scaled(double* out, const void* q, int q_dtype, const void* k_
                          const int32_t* seq_lens, int num_seqs, int num_q_heads, int num_kv_heads,
                          int head_dim, int block_size, int max_blocks_per_seq, int64_t num_blocks,
                          float scale, float k_scale, float v_scale, int num_threads) {
-  if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 ||
-      max_blocks_per_seq < 0 || num_blocks <= 0)
+  return decode_common(out, q, q_dtype, k_cache, v_cache, kv_dtype, block_tables, seq_lens, num_seqs, 1,
+                       num_q_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq, num_blocks, scale,
+                       k_scale, v_scale, num_threads);
+}
+
+/* Multi-token causal attention over the paged cache: q and out are
+ * [num_seqs, num_q_tokens, num_q_heads, head_dim]; query token tq of sequence i is the
+ * token at position seq_lens[i] - num_q_tokens + tq and attends to the tokens 0 .. that
+ * position.  A sequence must hold 0 or at least num_q_tokens tokens. */
+int oracle_decode_multi(double* out, const void* q, int q_dtype, const void* k_cache,
+                        const void* v_cache, int kv_dtype, const int32_t* block_tables,
+                        const int32_t* seq_lens, int num_seqs, int num_q_tokens, int num_q_heads,
+                        int num_kv_heads, int head_dim, int block_size, int max_blocks_per_seq,
+                        int64_t num_blocks, float scale, int num_threads) {
+  return decode_common(out, q, q_dtype, k_cache, v_cache, kv_dtype, block_tables, seq_lens, num_seqs,
+                       num_q_tokens, num_q_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq,
+                       num_blocks, scale, 1.0f, 1.0f, num_threads);
+}
+
+static int decode_common(double* out, const void* q, int q_dtype, const void* k_cache,
+                         const void* v_cache, int kv_dtype, const int32_t* block_tables,
+                         const int32_t* seq_lens, int num_seqs, int num_q_tokens, int num_q_heads,
+                         int num_kv_heads, int head_dim, int block_size, int max_blocks_per_seq,
+                         int64_t num_blocks, float scale, float k_scale, float v_scale, int num_threads) {
+  if (num_seqs < 0 || num_q_tokens <= 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 ||
+      block_size <= 0 || max_blocks_per_seq < 0 || num_blocks <= 0)
     return OR_ERR_ARG;
   if (num_q_heads % num_kv_heads) return OR_ERR_ARG;
   if (q_dtype < OR_F32 || q_dtype > OR_BF16 || kv_dtype < OR_F32 || kv_dtype > OR_E4M3) return OR_ERR_ARG;
@@ -341,6 +381,7 @@ int oracle_decode_scaled(double* out, const void* q, int q_dtype, const void* k_
   for (int i = 0; i < num_seqs; ++i) {
     int L = seq_lens[i];
     if (L < 0 || (int64_t)L > (int64_t)max_blocks_per_seq * block_size) return OR_ERR_RANGE;
+    if (L > 0 && L < num_q_tokens) return OR_ERR_RANGE;
     int nb = (L + block_size - 1) / block_size;
     for (int b = 0; b < nb; ++b) {
       int32_t p = block_tables[(int64_t)i * max_blocks_per_seq + b];
@@ -356,6 +397,7 @@ int oracle_decode_scaled(double* out, const void* q, int q_dtype, const void* k_
     decode_job* J = &jobs[w];
     J->out = out; J->q = q; J->q_dtype = q_dtype; J->k_cache = k_cache; J->v_cache = v_cache;
     J->kv_dtype = kv_dtype; J->block_tables = block_tables; J->seq_lens = seq_lens;
+    J->num_q_tokens = num_q_tokens;
     J->num_q_heads = num_q_heads; J->num_kv_heads = num_kv_heads; J->head_dim = head_dim;
     J->block_size = block_size; J->max_blocks_per_seq = max_blocks_per_seq;
     J->scale = (double)scale;

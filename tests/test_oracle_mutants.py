@@ -17,15 +17,20 @@ SRC = os.path.join(ROOT, "oracle", "pa_oracle.c")
 
 MUTANTS = {
     "gqa_head_map": ("const int h = hq / G;", "const int h = hq % J->num_kv_heads;"),
-    "q_uses_kv_head": ("const int64_t qo = ((int64_t)i * J->num_q_heads + hq) * D;",
-                       "const int64_t qo = ((int64_t)i * J->num_q_heads + hq / G) * D;"),
+    "q_uses_kv_head": ("const int64_t qo = (((int64_t)i * T + tq) * J->num_q_heads + hq) * D;",
+                       "const int64_t qo = (((int64_t)i * T + tq) * J->num_q_heads + hq / G) * D;"),
+    "q_token_index": ("const int64_t qo = (((int64_t)i * T + tq) * J->num_q_heads + hq) * D;",
+                      "const int64_t qo = (((int64_t)i * T) * J->num_q_heads + hq) * D;"),
+    "causal_off_by_one": ("const int n = L - T + tq + 1;", "const int n = L - T + tq;"),
+    "causal_ignored": ("const int n = L - T + tq + 1;", "const int n = L;"),
+    "causal_reversed": ("const int n = L - T + tq + 1;", "const int n = L - tq;"),
     "table_index_mod": ("int64_t phys = table[t / block_size];", "int64_t phys = table[t % block_size];"),
     "token_in_block_div": ("(int64_t)(t % block_size) * num_kv_heads * head_dim",
                            "(int64_t)(t / block_size) * num_kv_heads * head_dim"),
     "head_stride": ("(int64_t)h * head_dim + d;", "(int64_t)h * block_size + d;"),
     "no_scale": ("        s *= J->scale;\n", "\n"),
-    "drop_last_token": ("      for (int t = 0; t < L; ++t) {\n        double w",
-                        "      for (int t = 0; t + 1 < L; ++t) {\n        double w"),
+    "drop_last_token": ("      for (int t = 0; t < n; ++t) {\n        double w",
+                        "      for (int t = 0; t + 1 < n; ++t) {\n        double w"),
     "no_normalisation": ("for (int d = 0; d < D; ++d) o[d] /= z;", ""),
     "k_from_v_cache": ("load_elem(J->k_cache, kv_offset", "load_elem(J->v_cache, kv_offset"),
     "no_max_shift": ("double w = exp(scores[t] - m);", "double w = exp(scores[t]);"),

@@ -15,7 +15,12 @@ What pins what:
     blocks 0, 1, 2 -> physical 5, 12, 3); invariants (placement permutation, shared
     prefix == private copy, copy-on-write leaves the parent unchanged, GQA == MHA
     with repeated KV, block size 16 == 32);
-  * reshape_and_cache / copy_blocks -- numpy fancy-index assignment.
+  * reshape_and_cache / copy_blocks -- numpy fancy-index assignment;
+  * multi-token causal attention -- torch SDPA in fp64 with an explicit causal mask
+    (query token t of a sequence of L tokens sees positions 0 .. L - T + t) on contiguous
+    K/V scattered into the pool; a closed form (zero keys: each query token averages V
+    over exactly the positions it sees); and the reduction of every query token to a
+    single-token decode of the sequence cut after the token's own position.
 """
 import json
 import math
@@ -433,10 +438,88 @@ def check_swap_blocks(lib):
     assert np.array_equal(src_k, sk) and np.array_equal(src_v, sv), "the source pool is left as it was"
 
 
+MULTI_CASES = [
+    # lens, T, Hq, Hkv, D, bs, q_dtype, kv_dtype
+    ([5, 17, 40, 0], 5, 4, 2, 64, 16, "f32", "f16"),
+    ([33, 64, 4], 4, 8, 2, 128, 16, "bf16", "bf16"),
+    ([70, 3], 3, 6, 3, 128, 32, "f16", "f16"),
+    ([20, 48], 8, 4, 1, 64, 32, "bf16", "bf16"),
+]
+
+
+def random_multi_case(seed, lens, T, Hq, Hkv, D, bs, q_dtype, kv_dtype):
+    rng = _rng(seed)
+    q32 = W.storage_to_f32(W.to_storage(rng.standard_normal((len(lens), T, Hq, D), dtype=np.float32), q_dtype),
+                           q_dtype)
+    Ks, Vs = [], []
+    for L in lens:
+        Ks.append(W.storage_to_f32(W.to_storage(rng.standard_normal((L, Hkv, D), dtype=np.float32), kv_dtype), kv_dtype))
+        Vs.append(W.storage_to_f32(W.to_storage(rng.standard_normal((L, Hkv, D), dtype=np.float32), kv_dtype), kv_dtype))
+    kc, vc, bt, sl = paged_from_logical(Ks, Vs, bs, sum(-(-L // bs) for L in lens) + 2, rng, kv_dtype)
+    return W.to_storage(q32, q_dtype), q32, Ks, Vs, kc, vc, bt, sl
+
+
+def causal_sdpa_reference(q32, Ks, Vs, scale, G):
+    """torch SDPA in fp64 with a boolean mask: query token t sees key positions <= L - T + t."""
+    N, T = q32.shape[:2]
+    outs = []
+    for i, (K, V) in enumerate(zip(Ks, Vs)):
+        L = len(K)
+        if L == 0:
+            outs.append(np.zeros(q32.shape[1:], np.float64))
+            continue
+        qi = torch.from_numpy(q32[i].astype(np.float64)).permute(1, 0, 2)[None]   # [1,Hq,T,D]
+        k = torch.from_numpy(K.astype(np.float64)).permute(1, 0, 2)[None]        # [1,Hkv,L,D]
+        v = torch.from_numpy(V.astype(np.float64)).permute(1, 0, 2)[None]
+        mask = torch.arange(L)[None, :] <= (L - T + torch.arange(T))[:, None]    # [T, L]
+        o = torch.nn.functional.scaled_dot_product_attention(qi, k, v, attn_mask=mask, scale=scale,
+                                                             enable_gqa=G > 1)
+        outs.append(o[0].permute(1, 0, 2).numpy())                               # [T,Hq,D]
+    return np.stack(outs)
+
+
+def check_multi_vs_sdpa(lib, cases=MULTI_CASES):
+    for n, (lens, T, Hq, Hkv, D, bs, qd, kd) in enumerate(cases):
+        q, q32, Ks, Vs, kc, vc, bt, sl = random_multi_case(300 + n, lens, T, Hq, Hkv, D, bs, qd, kd)
+        scale = float(np.float32(1 / math.sqrt(D)))
+        got = oracle.decode_multi(q, qd, kc, vc, kd, bt, sl, scale, num_threads=2, lib=lib)
+        ref = causal_sdpa_reference(q32, Ks, Vs, scale, Hq // Hkv)
+        err = np.max(np.abs(got - ref))
+        assert err < 1e-12, f"case {n}: multi-token oracle vs causal SDPA max|err| = {err}"
+
+
+def check_multi_causal_closed_form(lib):
+    """Zero keys make every visible score equal: query token t of a sequence of L tokens
+    returns the mean of V over positions 0 .. L - T + t, exactly the positions it sees."""
+    rng = _rng(17)
+    T, L, D, bs = 6, 37, 64, 16
+    K = np.zeros((L, 1, D), np.float32)
+    V = rng.integers(-8, 9, size=(L, 1, D)).astype(np.float32)
+    kc, vc, bt, sl = paged_from_logical([K], [V], bs, 6, rng, "f16")
+    q = W.to_storage(rng.standard_normal((1, T, 1, D), dtype=np.float32), "f32")
+    got = oracle.decode_multi(q, "f32", kc, vc, "f16", bt, sl, 0.3, num_threads=1, lib=lib)[0, :, 0]
+    for t in range(T):
+        want = V[:L - T + t + 1, 0].astype(np.float64).mean(axis=0)
+        assert np.max(np.abs(got[t] - want)) < 1e-12, f"query token {t}"
+
+
+def check_multi_reduces_to_decode(lib):
+    """Query token t equals a one-token decode of the sequence cut after position L - T + t."""
+    lens, T = [9, 40, 0, 4], 4
+    q, q32, Ks, Vs, kc, vc, bt, sl = random_multi_case(77, lens, T, 4, 2, 64, 16, "bf16", "bf16")
+    got = oracle.decode_multi(q, "bf16", kc, vc, "bf16", bt, sl, 0.125, num_threads=1, lib=lib)
+    for t in range(T):
+        cut = np.where(sl > 0, sl - T + t + 1, 0).astype(np.int32)
+        one = oracle.decode(np.ascontiguousarray(q[:, t]), "bf16", kc, vc, "bf16", bt, cut, 0.125, num_threads=1,
+                            lib=lib)
+        assert np.array_equal(got[:, t], one), f"query token {t}"
+
+
 ALL_CHECKS = [check_swap_blocks, check_f16_decode, check_bf16_decode, check_decode_vs_sdpa, check_closed_forms,
               check_page_block_table_example, check_invariants, check_cow_leaves_parent,
               check_reshape_and_cache, check_copy_blocks, check_e4m3_decode, check_e4m3_encode,
-              check_reshape_and_cache_e4m3, check_decode_e4m3_vs_sdpa]
+              check_reshape_and_cache_e4m3, check_decode_e4m3_vs_sdpa, check_multi_vs_sdpa,
+              check_multi_causal_closed_form, check_multi_reduces_to_decode]
 
 
 @pytest.fixture(scope="module")
@@ -467,3 +550,7 @@ def test_oracle_rejects_bad_indices(lib):
         oracle.copy_blocks(kc, vc, np.asarray([[0, kc.shape[0]]], np.int32), lib=lib)
     with pytest.raises(oracle.OracleError):
         oracle.reshape_and_cache(kc[0], vc[0], kc, vc, np.full(16, kc.shape[0] * 16, np.int64), "f16", lib=lib)
+    # a sequence must hold at least its query tokens
+    qm = np.zeros((2, 6, 2, 64), np.uint16)
+    with pytest.raises(oracle.OracleError):
+        oracle.decode_multi(qm, "f16", kc, vc, "f16", bt, sl, 0.125, lib=lib)
