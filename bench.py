@@ -59,6 +59,9 @@ def parse_args():
     ap.add_argument("--out-dtype", default=None, help="f32 | f16 | bf16 (default: the query dtype)")
     ap.add_argument("--kv-dtype", default=None, choices=["e4m3"],
                     help="e4m3: the same config over an FP8 KV cache (per-tensor K/V scales)")
+    ap.add_argument("--qtok", type=int, default=1,
+                    help="query tokens per sequence: T > 1 runs causal multi-token attention (pa_decode_multi) "
+                         "over the same config, the step storing each sequence's last T tokens")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target oracle time for cpu_baseline")
     ap.add_argument("--ref-seconds", type=float, default=150.0, help="target total time of --impl reference")
@@ -67,8 +70,9 @@ def parse_args():
 
 def workload_label(w: W.Workload) -> str:
     kv = w.kv_dtype if w.kv_dtype != "e4m3" else f"e4m3 (scales {w.k_scale:.4g}/{w.v_scale:.4g}, new tokens {w.new_kv_dtype})"
+    qt = f", {w.num_q_tokens} query tokens per seq (causal)" if w.num_q_tokens > 1 else ""
     return (f"{w.name}: {w.num_seqs} seqs, {w.num_q_heads}/{w.num_kv_heads} heads, head_dim {w.head_dim}, "
-            f"block {w.block_size}, {w.notes.get('lens', '')}, q {w.q_dtype}, kv {kv}")
+            f"block {w.block_size}, {w.notes.get('lens', '')}, q {w.q_dtype}, kv {kv}{qt}")
 
 
 def measured_peak():
@@ -107,10 +111,17 @@ def sources_digest():
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(config: str):
-    """dram bytes per pa_decode partition-kernel launch from the committed ncu summary, if it was
+def profile_name(args) -> str:
+    """Name of the committed ncu summary of this run's partition kernel: config, cache dtype and
+    query tokens (pa_decode_partition_8b, pa_decode_partition_8b_e4m3, pa_decode_partition_8b_T5)."""
+    return (f"pa_decode_partition_{args.config}" + (f"_{args.kv_dtype}" if args.kv_dtype else "")
+            + (f"_T{args.qtok}" if args.qtok > 1 else ""))
+
+
+def recorded_traffic(name: str):
+    """dram bytes per partition-kernel launch from the committed ncu summary `name`, if it was
     taken on the current kernel sources (otherwise None)."""
-    path = os.path.join(ROOT, "profiles", f"pa_decode_partition_{config}.md")
+    path = os.path.join(ROOT, "profiles", f"{name}.md")
     if not os.path.exists(path):
         return None
     vals = {}
@@ -199,14 +210,19 @@ def oracle_sample_rate(w: W.Workload, seconds: float, start: int = 0):
 
     threads = oracle.default_threads()
     kc, vc = oracle_post_step(w)
-    dec = dict(k_scale=w.k_scale, v_scale=w.v_scale)
+    if w.num_q_tokens > 1:
+        def run(q, bt, sl, num_threads):
+            return oracle.decode_multi(q, w.q_dtype, kc, vc, w.kv_dtype, bt, sl, w.scale, num_threads=num_threads)
+    else:
+        def run(q, bt, sl, num_threads):
+            return oracle.decode(q, w.q_dtype, kc, vc, w.kv_dtype, bt, sl, w.scale, num_threads=num_threads,
+                                 k_scale=w.k_scale, v_scale=w.v_scale)
     row = 2 * w.kv_row_bytes
     order = [(start + i) % w.num_seqs for i in range(w.num_seqs)]
     # pilot: one sequence of median length to size the sample
     med = int(np.argsort(w.seq_lens)[w.num_seqs // 2])
     t = time.perf_counter()
-    oracle.decode(np.ascontiguousarray(w.q[[med]]), w.q_dtype, kc, vc, w.kv_dtype,
-                  np.ascontiguousarray(w.block_tables[[med]]), w.seq_lens[[med]], w.scale, num_threads=1, **dec)
+    run(np.ascontiguousarray(w.q[[med]]), np.ascontiguousarray(w.block_tables[[med]]), w.seq_lens[[med]], 1)
     per_token = (time.perf_counter() - t) / max(1, int(w.seq_lens[med]))
     budget_tokens = seconds * threads / max(per_token, 1e-12)
     pick, tok = [], 0
@@ -220,7 +236,7 @@ def oracle_sample_rate(w: W.Workload, seconds: float, start: int = 0):
                  np.ascontiguousarray(w.seq_lens[idx]))
     passes, t = 0, time.perf_counter()
     while True:  # whole passes over the sample until the time budget is used
-        oracle.decode(q, w.q_dtype, kc, vc, w.kv_dtype, bt, sl, w.scale, num_threads=threads, **dec)
+        run(q, bt, sl, threads)
         passes += 1
         dt = time.perf_counter() - t
         if dt >= 0.8 * seconds:
@@ -232,7 +248,8 @@ def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
-    w = W.make_config(args.config, block_size=args.block_size, kv_dtype=args.kv_dtype)
+    qkw = {"num_q_tokens": args.qtok} if args.qtok > 1 else {}
+    w = W.make_config(args.config, block_size=args.block_size, kv_dtype=args.kv_dtype, **qkw)
     per_step = max(0.5, args.ref_seconds / max(1, args.steps + args.warmup))
     start = 0
     for _ in range(args.warmup):
@@ -253,7 +270,7 @@ def run_reference(args):
         "config": {"workload": workload_label(w)},
         "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
                          "sample": f"{seqs} sequences over {args.steps} steps (consecutive windows of the batch), "
-                                   f"fp64 two-pass softmax, decode only"},
+                                   f"fp64 two-pass softmax, attention only"},
         "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -281,11 +298,13 @@ def run_ours(args):
 
     seed = rank_seed(args.config, rank)
     extra = {"num_seqs": args.num_seqs} if args.num_seqs else {}
+    if args.qtok > 1:
+        extra["num_q_tokens"] = args.qtok
     w = W.make_config(args.config, block_size=args.block_size, seed=seed, kv_dtype=args.kv_dtype, **extra)
     out_dtype = args.out_dtype or w.q_dtype
     dw = B.device_workload(w, f"cuda:{local}")
     ws = B.DecodeWorkspace.for_workload(dw, args.partition_size)
-    out = torch.empty((w.num_seqs, w.num_q_heads, w.head_dim), dtype=B._NAME_TORCH[out_dtype], device="cuda")
+    out = torch.empty(tuple(dw.q.shape), dtype=B._NAME_TORCH[out_dtype], device="cuda")
     stream = torch.cuda.current_stream()
 
     kv_bytes = w.kv_bytes_logical()
@@ -329,7 +348,10 @@ def run_ours(args):
             B.pa_reshape_and_cache(dw.new_k, dw.new_v, dw.k_cache, dw.v_cache, dw.slot_mapping, stream=stream)
 
     def decode():
-        if fp8:
+        if w.num_q_tokens > 1:
+            B.pa_decode_multi(out, dw.q, dw.k_cache, dw.v_cache, dw.block_tables, dw.seq_lens, w.scale, ws.tensor,
+                              args.partition_size, stream)
+        elif fp8:
             B.pa_decode_fp8(out, dw.q, dw.k_cache, dw.v_cache, dw.block_tables, dw.seq_lens, w.scale, w.k_scale,
                             w.v_scale, ws.tensor, args.partition_size, stream)
         else:
@@ -426,7 +448,7 @@ def run_ours(args):
         b, t, threads, n = oracle_sample_rate(w, args.cpu_seconds)
         cpu = {"value": round(b / t / 1e9, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
                "sample": f"{n} sequence decodes from the start of the batch of {w.num_seqs} "
-                         f"({b / 1e9:.3f} GB of K+V), decode only, fp64 two-pass softmax, {t:.1f} s"}
+                         f"({b / 1e9:.3f} GB of K+V), attention only, fp64 two-pass softmax, {t:.1f} s"}
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_step, 5), "higher_is_better": True, "scaling": "weak",
@@ -438,12 +460,14 @@ def run_ours(args):
                    "l2": f"inputs larger than L2 (K+V {kv_bytes / 1e9:.2f} GB vs 126 MB L2); no flush in the "
                          f"timed loop", "parallelism": f"replicas x{world}" if world > 1 else "1 GPU"},
         "seq_tokens_per_s": round(world * w.total_tokens() / (ms_step * 1e-3), 1),
+        "query_tokens_per_s": round(world * w.num_seqs * w.num_q_tokens / (ms_step * 1e-3), 1),
         "pct_of_hbm_peak": round(100 * value / world / peak, 2),
         "e2e": {"value": round(job_throughput(kv_bytes, world, e2e_ms * 1e-3), 2), "unit": "GB/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 5)},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
-                     "frac": round(achieved / peak, 4), "traffic": recorded_traffic(args.config),
-                     "kernel": "pa_decode call (plan + partition + reduce kernels)",
+                     "frac": round(achieved / peak, 4), "traffic": recorded_traffic(profile_name(args)),
+                     "kernel": ("pa_decode_multi" if w.num_q_tokens > 1 else "pa_decode")
+                               + " call (plan + partition + merge kernels)",
                      "algorithmic_bytes_per_launch": decode_bytes, "launch_ms_mean": round(dec_mean, 5),
                      "launch_ms_l2_flushed_median": round(float(np.median(flushed)), 5),
                      "peak_source": peak_src},

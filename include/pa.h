@@ -116,6 +116,30 @@ PA_API int pa_decode_fp8(void* out, const void* q, const void* k_cache, const vo
                          int q_dtype, int out_dtype, int partition_size, void* workspace,
                          size_t workspace_bytes, void* stream);
 
+/* Multi-token paged attention: several query tokens per sequence, causal ("详解vLLM推理引擎
+ *架构", section "量化集成与部署": speculative decoding verifies N draft tokens in one pass of
+ * the large model; section "Chunked Prefill": a prompt is processed in chunks interleaved
+ * with decode steps).  The pages give no formula; the reading taken is the plain causal one:
+ * the T = num_q_tokens query tokens of sequence i are its last T tokens, already stored in the
+ * cache, and query token t (position seq_lens[i] - T + t) attends to tokens 0 ..
+ * seq_lens[i] - T + t:
+ *   out[i, t, hq, :] = sum_{s <= L - T + t} softmax_s(scale * q[i, t, hq, :] . K_s) * V_s,
+ * with L = seq_lens[i] and K_s, V_s, G and the block-table lookup as in pa_decode.
+ *   out  [num_seqs, num_q_tokens, num_q_heads, head_dim], out_dtype (f32, f16 or bf16)
+ *   q    [num_seqs, num_q_tokens, num_q_heads, head_dim], q_dtype
+ *   seq_lens[i] = 0 gives all-zero rows; 0 < seq_lens[i] < num_q_tokens is invalid (its rows
+ *   are NaN and pa_get_device_error reports PA_DEV_BAD_SEQ_LEN).
+ *   supported: num_q_tokens * G <= 8 on every dtype pair pa_decode takes; up to 32 with
+ *   head_dim 128 and q_dtype == kv_dtype (f16 or bf16).  Everything else as pa_decode; the
+ *   workspace is pa_decode_workspace_size(num_seqs, num_q_tokens * num_q_heads, head_dim,
+ *   max_blocks_per_seq * block_size, partition_size).  num_q_tokens 1 is pa_decode. */
+PA_API int pa_decode_multi(void* out, const void* q, const void* k_cache, const void* v_cache,
+                           const int32_t* block_tables, const int32_t* seq_lens, int num_seqs,
+                           int num_q_tokens, int num_q_heads, int num_kv_heads, int head_dim,
+                           int block_size, float scale, int max_blocks_per_seq, int64_t num_blocks,
+                           int q_dtype, int kv_dtype, int out_dtype, int partition_size, void* workspace,
+                           size_t workspace_bytes, void* stream);
+
 /* Store the step's new tokens into the paged cache ("vLLM 深度解读", section 7).
  * For each token t with slot = slot_mapping[t] >= 0:
  *   k_cache[slot / block_size, slot % block_size, h, :] = k[t, h, :]  for every KV head h

@@ -24,7 +24,7 @@ PA_DEV_OK, PA_DEV_BAD_BLOCK_ID, PA_DEV_BAD_SEQ_LEN, PA_DEV_BAD_SLOT, PA_DEV_BAD_
 
 EXPORTED = ("pa_decode_workspace_size", "pa_decode", "pa_reshape_and_cache", "pa_copy_blocks",
             "pa_strerror", "pa_get_device_error", "pa_version", "pa_decode_static_workspace",
-            "pa_decode_fp8", "pa_reshape_and_cache_fp8", "pa_swap_blocks")
+            "pa_decode_fp8", "pa_reshape_and_cache_fp8", "pa_swap_blocks", "pa_decode_multi")
 PA_ERR_TOO_LARGE = -5
 PA_DECODE_STATIC_WORKSPACE_BYTES = 64 << 20
 
@@ -68,6 +68,8 @@ def load_library(path: str = _LIB_PATH):
     lib.pa_reshape_and_cache_fp8.restype = I
     lib.pa_swap_blocks.argtypes = [P, P, P, P, P, I, I64, I64, SZ, P]
     lib.pa_swap_blocks.restype = I
+    lib.pa_decode_multi.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, F, I, I64, I, I, I, I, P, SZ, P]
+    lib.pa_decode_multi.restype = I
     if path == _LIB_PATH:
         _lib = lib
     return lib
@@ -123,6 +125,32 @@ def pa_decode(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor, v_cache
         _TORCH_CODE[out.dtype], partition_size, _ptr(workspace), workspace.numel() * workspace.element_size(),
         _stream(stream))
     _check(rc, "pa_decode")
+
+
+def pa_decode_multi(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                    block_tables: torch.Tensor, seq_lens: torch.Tensor, scale: float, workspace: torch.Tensor,
+                    partition_size: int = 0, stream=None) -> None:
+    """out[N,T,Hq,D] <- causal attention of each sequence's last T tokens over the paged cache.
+
+    Query token t of sequence i sits at position seq_lens[i] - T + t and attends to positions
+    0 .. seq_lens[i] - T + t (see include/pa.h).  The workspace is that of pa_decode for
+    T * Hq query heads (DecodeWorkspace.for_multi).
+    """
+    N, T, Hq, D = q.shape
+    NB, bs, Hkv, D2 = k_cache.shape
+    if D2 != D or tuple(out.shape) != (N, T, Hq, D) or v_cache.shape != k_cache.shape:
+        raise ValueError("shape mismatch between q, out and the caches")
+    for t in (out, q, k_cache, v_cache, block_tables, seq_lens, workspace):
+        if not t.is_contiguous():
+            raise ValueError("tensors must be contiguous")
+    if block_tables.dtype != torch.int32 or seq_lens.dtype != torch.int32:
+        raise TypeError("block_tables and seq_lens must be int32")
+    rc = load_library().pa_decode_multi(
+        _ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), _ptr(seq_lens), N, T, Hq, Hkv, D, bs,
+        ctypes.c_float(scale), block_tables.shape[1], NB, _TORCH_CODE[q.dtype], _TORCH_CODE[k_cache.dtype],
+        _TORCH_CODE[out.dtype], partition_size, _ptr(workspace), workspace.numel() * workspace.element_size(),
+        _stream(stream))
+    _check(rc, "pa_decode_multi")
 
 
 def pa_decode_static_workspace(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
@@ -289,12 +317,20 @@ class DecodeWorkspace:
     @classmethod
     def for_workload(cls, dw: DeviceWorkload, partition_size=0):
         w = dw.w
-        return cls(w.num_seqs, w.num_q_heads, w.head_dim, w.max_blocks_per_seq * w.block_size, partition_size,
-                   device=dw.q.device)
+        return cls(w.num_seqs, w.num_q_tokens * w.num_q_heads, w.head_dim, w.max_blocks_per_seq * w.block_size,
+                   partition_size, device=dw.q.device)
+
+    @classmethod
+    def for_multi(cls, num_seqs, num_q_tokens, num_q_heads, head_dim, max_seq_len, partition_size=0,
+                  device="cuda"):
+        """Workspace of pa_decode_multi: pa_decode's for num_q_tokens * num_q_heads heads."""
+        return cls(num_seqs, num_q_tokens * num_q_heads, head_dim, max_seq_len, partition_size, device=device)
 
 
 def run_step(dw: DeviceWorkload, out: torch.Tensor, ws: DecodeWorkspace, partition_size=0, stream=None) -> None:
-    """One decode step: copy_blocks -> reshape_and_cache -> decode (all through the C ABI)."""
+    """One decode step: copy_blocks -> reshape_and_cache -> decode (all through the C ABI).
+
+    A workload with several query tokens per sequence runs pa_decode_multi as its decode."""
     w = dw.w
     if dw.copy_pairs.shape[0]:
         pa_copy_blocks(dw.k_cache, dw.v_cache, dw.copy_pairs, stream=stream)
@@ -307,5 +343,9 @@ def run_step(dw: DeviceWorkload, out: torch.Tensor, ws: DecodeWorkspace, partiti
         return
     if dw.slot_mapping.shape[0]:
         pa_reshape_and_cache(dw.new_k, dw.new_v, dw.k_cache, dw.v_cache, dw.slot_mapping, stream=stream)
+    if w.num_q_tokens > 1:
+        pa_decode_multi(out, dw.q, dw.k_cache, dw.v_cache, dw.block_tables, dw.seq_lens, w.scale, ws.tensor,
+                        partition_size=partition_size, stream=stream)
+        return
     pa_decode(out, dw.q, dw.k_cache, dw.v_cache, dw.block_tables, dw.seq_lens, dw.w.scale, ws.tensor,
               partition_size=partition_size, stream=stream)

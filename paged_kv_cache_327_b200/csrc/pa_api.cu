@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <atomic>
 #include <climits>
 #include <cmath>
 #include <cstdint>
@@ -62,7 +63,6 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 // Per-device launch facts, looked up once.
 struct DeviceInfo {
   int sm_count = 0;
-  bool smem_set[64] = {};
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_mu;
@@ -101,15 +101,16 @@ int encode_kv_map(CUtensorMap* map, const void* base, int kv_dtype, int64_t num_
   return r == CUDA_SUCCESS ? PA_OK : PA_ERR_CUDA;
 }
 
-template <int BS, int D, typename KT, typename QT>
+template <int BS, int D, typename KT, typename QT, int NT>
 int launch_partition(const pa::DecodeParams& p, const CUtensorMap& tmk, const CUtensorMap& tmv,
-                     int64_t max_items, DeviceInfo* info, int slot_id, cudaStream_t stream) {
-  using C = pa::DecodeCfg<BS, D, KT, QT>;
-  auto kern = pa::pa_decode_partition_kernel<BS, D, KT, QT>;
-  if (!info->smem_set[slot_id]) {
+                     int64_t max_items, int dev, DeviceInfo* info, cudaStream_t stream) {
+  using C = pa::DecodeCfg<BS, D, KT, QT, NT>;
+  auto kern = pa::pa_decode_partition_kernel<BS, D, KT, QT, NT>;
+  static std::atomic<bool> smem_set[kMaxDevices];  // per instantiation and device
+  if (!smem_set[dev].load(std::memory_order_acquire)) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
       return PA_ERR_CUDA;
-    info->smem_set[slot_id] = true;
+    smem_set[dev].store(true, std::memory_order_release);
   }
   int64_t ctas = (max_items + C::NWARP - 1) / C::NWARP;
   if (ctas > info->sm_count) ctas = info->sm_count;
@@ -130,26 +131,43 @@ int launch_partition(const pa::DecodeParams& p, const CUtensorMap& tmk, const CU
   return cudaPeekAtLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
-// one shared-memory attribute flag per kernel instantiation
-constexpr int kInstPerShape = 8;
-
+// Kernel instantiation for (block_size, head_dim, KV dtype, query dtype, query rows per item):
+// items of up to 8 query rows run on every dtype pair; wider items (several query tokens, NT
+// 8-row tiles) on a 16-bit cache with a query of the same type, head_dim 128.
 template <int BS, int D>
 int dispatch_kv(const pa::DecodeParams& p, const CUtensorMap& tmk, const CUtensorMap& tmv, int64_t max_items,
-                DeviceInfo* info, int kv_dtype, int q_dtype, int base_id, cudaStream_t stream) {
+                int dev, DeviceInfo* info, int kv_dtype, int q_dtype, cudaStream_t stream) {
   const bool qf32 = q_dtype == PA_F32;
+  const int nt = (p.item_cols + 7) / 8;
+  if (nt > 1) {
+    if constexpr (D == 128) {
+      if (kv_dtype == PA_BF16 && q_dtype == PA_BF16) {
+        using T = __nv_bfloat16;
+        if (nt == 2) return launch_partition<BS, D, T, T, 2>(p, tmk, tmv, max_items, dev, info, stream);
+        if (nt == 3) return launch_partition<BS, D, T, T, 3>(p, tmk, tmv, max_items, dev, info, stream);
+        return launch_partition<BS, D, T, T, 4>(p, tmk, tmv, max_items, dev, info, stream);
+      }
+      if (kv_dtype == PA_F16 && q_dtype == PA_F16) {
+        using T = __half;
+        if (nt == 2) return launch_partition<BS, D, T, T, 2>(p, tmk, tmv, max_items, dev, info, stream);
+        if (nt == 3) return launch_partition<BS, D, T, T, 3>(p, tmk, tmv, max_items, dev, info, stream);
+        return launch_partition<BS, D, T, T, 4>(p, tmk, tmv, max_items, dev, info, stream);
+      }
+    }
+    return PA_ERR_UNSUPPORTED;
+  }
   if (kv_dtype == PA_BF16)
-    return qf32 ? launch_partition<BS, D, __nv_bfloat16, float>(p, tmk, tmv, max_items, info, base_id + 0, stream)
-                : launch_partition<BS, D, __nv_bfloat16, __nv_bfloat16>(p, tmk, tmv, max_items, info, base_id + 1,
-                                                                        stream);
+    return qf32 ? launch_partition<BS, D, __nv_bfloat16, float, 1>(p, tmk, tmv, max_items, dev, info, stream)
+                : launch_partition<BS, D, __nv_bfloat16, __nv_bfloat16, 1>(p, tmk, tmv, max_items, dev, info, stream);
   if (kv_dtype == PA_F16)
-    return qf32 ? launch_partition<BS, D, __half, float>(p, tmk, tmv, max_items, info, base_id + 2, stream)
-                : launch_partition<BS, D, __half, __half>(p, tmk, tmv, max_items, info, base_id + 3, stream);
+    return qf32 ? launch_partition<BS, D, __half, float, 1>(p, tmk, tmv, max_items, dev, info, stream)
+                : launch_partition<BS, D, __half, __half, 1>(p, tmk, tmv, max_items, dev, info, stream);
   if constexpr (D == 128) {  // an FP8 row of head_dim 128 fills one 128-byte TMA box
     if (q_dtype == PA_F32)
-      return launch_partition<BS, D, pa::fp8e4m3, float>(p, tmk, tmv, max_items, info, base_id + 4, stream);
+      return launch_partition<BS, D, pa::fp8e4m3, float, 1>(p, tmk, tmv, max_items, dev, info, stream);
     if (q_dtype == PA_F16)
-      return launch_partition<BS, D, pa::fp8e4m3, __half>(p, tmk, tmv, max_items, info, base_id + 5, stream);
-    return launch_partition<BS, D, pa::fp8e4m3, __nv_bfloat16>(p, tmk, tmv, max_items, info, base_id + 6, stream);
+      return launch_partition<BS, D, pa::fp8e4m3, __half, 1>(p, tmk, tmv, max_items, dev, info, stream);
+    return launch_partition<BS, D, pa::fp8e4m3, __nv_bfloat16, 1>(p, tmk, tmv, max_items, dev, info, stream);
   }
   return PA_ERR_UNSUPPORTED;
 }
@@ -184,19 +202,25 @@ size_t pa_decode_workspace_size(int num_seqs, int num_q_heads, int head_dim, int
 
 namespace {
 
-// pa_decode and pa_decode_fp8: kv_dtype F16 / BF16 (scales unused) or FP8_E4M3
+// pa_decode, pa_decode_fp8 and pa_decode_multi: kv_dtype F16 / BF16 (scales unused) or
+// FP8_E4M3; qtok query tokens per sequence (1 = decode)
 int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,
-                const int32_t* seq_lens, int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                const int32_t* seq_lens, int num_seqs, int qtok, int num_q_heads, int num_kv_heads, int head_dim,
                 int block_size, float scale, float k_scale, float v_scale, int max_blocks_per_seq,
                 int64_t num_blocks, int q_dtype, int kv_dtype, int out_dtype, int partition_size, void* workspace,
                 size_t workspace_bytes, void* stream) {
-  if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 ||
+  if (num_seqs < 0 || qtok <= 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 ||
       max_blocks_per_seq <= 0 || num_blocks <= 0 || partition_size < 0 || !std::isfinite(scale) ||
       !std::isfinite(k_scale) || !std::isfinite(v_scale) || k_scale <= 0.f || v_scale <= 0.f)
     return PA_ERR_INVALID;
   if (num_q_heads % num_kv_heads) return PA_ERR_INVALID;
   const int G = num_q_heads / num_kv_heads;
   if (G > 8) return PA_ERR_UNSUPPORTED;
+  // an item holds qtok * G query rows: up to 8 on every dtype pair, up to 32 on a 16-bit
+  // cache with a query of its own type and head_dim 128
+  if (static_cast<int64_t>(qtok) * G > 32) return PA_ERR_UNSUPPORTED;
+  if (qtok * G > 8 && (head_dim != 128 || kv_dtype == PA_FP8_E4M3 || q_dtype != kv_dtype))
+    return PA_ERR_UNSUPPORTED;
   if (head_dim != 64 && head_dim != 128) return PA_ERR_UNSUPPORTED;
   if (block_size != 16 && block_size != 32) return PA_ERR_UNSUPPORTED;
   if (kv_dtype == PA_FP8_E4M3) {
@@ -217,7 +241,8 @@ int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cac
   if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache)) return PA_ERR_INVALID;
   const int64_t max_parts = std::max<int64_t>(1, (max_len + P - 1) / P);
   if (max_parts > 32767) return PA_ERR_UNSUPPORTED;
-  const WsLayout L = ws_layout(num_seqs, num_q_heads, head_dim, max_parts);
+  // partial results are kept per (query token, query head): the workspace of qtok * num_q_heads heads
+  const WsLayout L = ws_layout(num_seqs, static_cast<int64_t>(qtok) * num_q_heads, head_dim, max_parts);
   if (!workspace || workspace_bytes < L.total) return PA_ERR_WORKSPACE;
   if (reinterpret_cast<uintptr_t>(workspace) & 255u) return PA_ERR_INVALID;
 
@@ -246,6 +271,8 @@ int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cac
   p.partition_size = P;
   p.max_parts = static_cast<int>(max_parts);
   p.out_dtype = out_dtype;
+  p.qtok = qtok;
+  p.item_cols = qtok * G;
   const bool fp8 = kv_dtype == PA_FP8_E4M3;
   p.scale_log2 = scale * (fp8 ? k_scale : 1.f) * 1.4426950408889634f;
   p.v_scale = fp8 ? v_scale : 1.f;
@@ -261,15 +288,14 @@ int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cac
   const int64_t max_items = static_cast<int64_t>(num_seqs) * max_parts * num_kv_heads;
   int rc;
   if (block_size == 16)
-    rc = head_dim == 128 ? dispatch_kv<16, 128>(p, tmk, tmv, max_items, info, kv_dtype, q_dtype, 0, st)
-                         : dispatch_kv<16, 64>(p, tmk, tmv, max_items, info, kv_dtype, q_dtype, kInstPerShape, st);
+    rc = head_dim == 128 ? dispatch_kv<16, 128>(p, tmk, tmv, max_items, dev, info, kv_dtype, q_dtype, st)
+                         : dispatch_kv<16, 64>(p, tmk, tmv, max_items, dev, info, kv_dtype, q_dtype, st);
   else
-    rc = head_dim == 128
-             ? dispatch_kv<32, 128>(p, tmk, tmv, max_items, info, kv_dtype, q_dtype, 2 * kInstPerShape, st)
-             : dispatch_kv<32, 64>(p, tmk, tmv, max_items, info, kv_dtype, q_dtype, 3 * kInstPerShape, st);
+    rc = head_dim == 128 ? dispatch_kv<32, 128>(p, tmk, tmv, max_items, dev, info, kv_dtype, q_dtype, st)
+                         : dispatch_kv<32, 64>(p, tmk, tmv, max_items, dev, info, kv_dtype, q_dtype, st);
   if (rc != PA_OK) return rc;
   {  // merge kernel: waits (griddepcontrol.wait) for the partition kernel's partial results
-    const int64_t warps = static_cast<int64_t>(num_seqs) * num_q_heads;
+    const int64_t warps = static_cast<int64_t>(num_seqs) * qtok * num_q_heads;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>((warps + pa::kMergeWarps - 1) / pa::kMergeWarps));
     cfg.blockDim = dim3(pa::kMergeWarps * 32);
@@ -294,7 +320,7 @@ int pa_decode(void* out, const void* q, const void* k_cache, const void* v_cache
               int kv_dtype, int out_dtype, int partition_size, void* workspace, size_t workspace_bytes,
               void* stream) {
   if (kv_dtype == PA_FP8_E4M3) return PA_ERR_UNSUPPORTED;  // needs its scales: pa_decode_fp8
-  return decode_impl(out, q, k_cache, v_cache, block_tables, seq_lens, num_seqs, num_q_heads, num_kv_heads,
+  return decode_impl(out, q, k_cache, v_cache, block_tables, seq_lens, num_seqs, 1, num_q_heads, num_kv_heads,
                      head_dim, block_size, scale, 1.f, 1.f, max_blocks_per_seq, num_blocks, q_dtype, kv_dtype,
                      out_dtype, partition_size, workspace, workspace_bytes, stream);
 }
@@ -304,9 +330,20 @@ int pa_decode_fp8(void* out, const void* q, const void* k_cache, const void* v_c
                   int block_size, float scale, float k_scale, float v_scale, int max_blocks_per_seq,
                   int64_t num_blocks, int q_dtype, int out_dtype, int partition_size, void* workspace,
                   size_t workspace_bytes, void* stream) {
-  return decode_impl(out, q, k_cache, v_cache, block_tables, seq_lens, num_seqs, num_q_heads, num_kv_heads,
+  return decode_impl(out, q, k_cache, v_cache, block_tables, seq_lens, num_seqs, 1, num_q_heads, num_kv_heads,
                      head_dim, block_size, scale, k_scale, v_scale, max_blocks_per_seq, num_blocks, q_dtype,
                      PA_FP8_E4M3, out_dtype, partition_size, workspace, workspace_bytes, stream);
+}
+
+int pa_decode_multi(void* out, const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,
+                    const int32_t* seq_lens, int num_seqs, int num_q_tokens, int num_q_heads, int num_kv_heads,
+                    int head_dim, int block_size, float scale, int max_blocks_per_seq, int64_t num_blocks,
+                    int q_dtype, int kv_dtype, int out_dtype, int partition_size, void* workspace,
+                    size_t workspace_bytes, void* stream) {
+  if (kv_dtype == PA_FP8_E4M3) return PA_ERR_UNSUPPORTED;
+  return decode_impl(out, q, k_cache, v_cache, block_tables, seq_lens, num_seqs, num_q_tokens, num_q_heads,
+                     num_kv_heads, head_dim, block_size, scale, 1.f, 1.f, max_blocks_per_seq, num_blocks, q_dtype,
+                     kv_dtype, out_dtype, partition_size, workspace, workspace_bytes, stream);
 }
 
 int pa_reshape_and_cache(const void* k, const void* v, void* k_cache, void* v_cache, const int64_t* slot_mapping,

@@ -64,7 +64,7 @@ constexpr uint32_t kWaitLimit = 1u << 20;
 constexpr float kRescaleThreshold = 8.0f;
 
 struct WorkItem {
-  int seq, part, len, pad;
+  int seq, part, len, members;  // members: sequences seq .. seq + members - 1 share the item
 };
 
 struct DecodeParams {
@@ -74,14 +74,15 @@ struct DecodeParams {
   const int32_t* seq_lens;
   int num_seqs, num_q_heads, num_kv_heads, group;
   int head_dim, block_size, max_blocks_per_seq, num_blocks;
-  int partition_size, max_parts, out_dtype, pad;
+  int partition_size, max_parts, out_dtype, qtok;  // qtok: query tokens per sequence (1 = decode)
+  int item_cols;     // query rows of an item: members * qtok * group
   float scale_log2;  // scale * log2(e) (* k_scale for an FP8 cache)
   float v_scale;     // multiplies the output (FP8 cache); 1 otherwise
   // workspace views
   unsigned int* counters;  // [0] next work item, [1] number of (sequence, partition) pairs
   WorkItem* items;         // [num_seqs * max_parts]
-  float2* part_ml;         // [num_seqs * max_parts * num_q_heads]: (max in log2 units, sum)
-  float* part_acc;         // [num_seqs * max_parts * num_q_heads * head_dim]
+  float2* part_ml;         // [num_seqs * max_parts * qtok * num_q_heads]: (max in log2 units, sum)
+  float* part_acc;         // [num_seqs * max_parts * qtok * num_q_heads * head_dim]
 };
 
 __device__ __forceinline__ void store_out(void* out, int64_t idx, float v, int dt) {
@@ -136,7 +137,7 @@ __global__ void __launch_bounds__(kPlanThreads) pa_decode_plan_kernel(const Deco
   int local = 0;
   for (int i = threadIdx.x; i < N; i += blockDim.x) {
     const int L = p.seq_lens[i];
-    if (L >= 0 && L <= max_len) local += L / P;
+    if (L >= 0 && L <= max_len && (L == 0 || L >= p.qtok)) local += L / P;
   }
   int n_full;
   block_exclusive_scan(local, s_warp, &n_full);
@@ -146,7 +147,8 @@ __global__ void __launch_bounds__(kPlanThreads) pa_decode_plan_kernel(const Deco
     int L = 0, nf = 0, nt = 0;
     if (i < N) {
       L = p.seq_lens[i];
-      const bool valid = L >= 0 && L <= max_len;
+      // a sequence holds its qtok query tokens: 0 < L < qtok is invalid
+      const bool valid = L >= 0 && L <= max_len && (L == 0 || L >= p.qtok);
       if (valid) {
         nf = L / P;
         nt = (L % P) ? 1 : 0;
@@ -155,15 +157,15 @@ __global__ void __launch_bounds__(kPlanThreads) pa_decode_plan_kernel(const Deco
       }
       if (!valid || L == 0) {  // no work item: the row is zero (empty) or NaN (invalid)
         const float v = valid ? 0.f : CUDART_NAN_F;
-        const int64_t row = static_cast<int64_t>(p.num_q_heads) * p.head_dim;
+        const int64_t row = static_cast<int64_t>(p.qtok) * p.num_q_heads * p.head_dim;
         for (int64_t e = 0; e < row; ++e) store_out(p.out, i * row + e, v, p.out_dtype);
       }
     }
     int tf, tt;
     const int of = block_exclusive_scan(nf, s_warp, &tf);
     const int ot = block_exclusive_scan(nt, s_warp, &tt);
-    for (int k = 0; k < nf; ++k) p.items[base_full + of + k] = WorkItem{i, k, L, 0};
-    if (nt) p.items[n_full + base_tail + ot] = WorkItem{i, nf, L, 0};
+    for (int k = 0; k < nf; ++k) p.items[base_full + of + k] = WorkItem{i, k, L, 1};
+    if (nt) p.items[n_full + base_tail + ot] = WorkItem{i, nf, L, 1};
     base_full += tf;
     base_tail += tt;
   }
@@ -213,7 +215,7 @@ __device__ __forceinline__ uint32_t lds_u16(uint32_t addr) {
   return v;
 }
 
-template <int BS, int D, typename KT, typename QT>
+template <int BS, int D, typename KT, typename QT, int NT>
 struct DecodeCfg {
   static constexpr bool FP8 = KvTraits<KT>::fp8;
   static constexpr int HALVES = D * KvTraits<KT>::bytes / 128;  // 128-byte column blocks of a row
@@ -224,15 +226,16 @@ struct DecodeCfg {
   // cache is converted to f16 once (exact for |q| in [2^-14, 65504])
   static constexpr bool QSPLIT = std::is_same<QT, float>::value;
   static constexpr bool QCONV = FP8 && !QSPLIT;
-  static constexpr int Q_BYTES = 8 * D * QE;            // up to 8 grouped query rows
-  static constexpr int SLOT_BYTES = ((2 * PAGE_BYTES + Q_BYTES + 1023) / 1024) * 1024;
+  static constexpr int COLS = 8 * NT;                   // query rows per item (MMA N dimension)
+  static constexpr int QBUF_BYTES = ((COLS * D * QE + 1023) / 1024) * 1024;  // per consumer
+  static constexpr int SLOT_BYTES = 2 * PAGE_BYTES;     // K page then V page
   static constexpr int NC = 4;                          // consumer warps (one producer each)
   static constexpr int NWARP = 2 * NC;
   static constexpr int SMEM_BUDGET = 200 * 1024;
-  static constexpr int NSLOT_FIT = SMEM_BUDGET / (NC * SLOT_BYTES);
+  static constexpr int NSLOT_FIT = (SMEM_BUDGET / NC - QBUF_BYTES) / SLOT_BYTES;
   static constexpr int NSLOT = NSLOT_FIT > 8 ? 8 : (NSLOT_FIT < 2 ? 2 : NSLOT_FIT);
-  static constexpr int RING_BYTES = NC * NSLOT * SLOT_BYTES;
-  static constexpr int BAR_BYTES = NC * NSLOT * 16;     // full + empty barrier per slot
+  static constexpr int RING_BYTES = NC * (NSLOT * SLOT_BYTES + QBUF_BYTES);
+  static constexpr int BAR_BYTES = NC * (2 * NSLOT + 2) * 8;  // full + empty per slot, qfree (+pad)
   static constexpr int META_BYTES = NC * NSLOT * 16;
   static constexpr int SMEM_BYTES = 1024 + RING_BYTES + BAR_BYTES + META_BYTES + 16 * NC;
   static constexpr int MT = BS / 16;    // 16-token MMA tiles per page
@@ -240,6 +243,8 @@ struct DecodeCfg {
   static_assert(D == 64 || D == 128, "head_dim");
   static_assert(BS == 16 || BS == 32, "block_size");
   static_assert(HALVES >= 1, "an FP8 row must fill a 128-byte box (head_dim 128)");
+  static_assert(NT == 1 || (!FP8 && !QSPLIT), "wide items: 16-bit cache and query");
+  static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
 };
 
 // byte offset, inside a page, of the 16-byte chunk holding (row t, columns d0..d0+7)
@@ -249,14 +254,19 @@ __device__ __forceinline__ uint32_t swz(int t, int d0) {
   return (d0 >> 6) * BOX_BYTES + t * 128 + ((((d0 & 63) >> 3) ^ (t & 7)) << 4);
 }
 
-// meta word: ntok (bits 0-7) | flags (bits 8-15) | partitions of the sequence (bits 16-31)
+// slot metadata: x = seq, y = part | page << 16, z = kvh | ntok << 16 | flags << 24, w = len
 constexpr int F_FIRST = 1, F_LAST = 2, F_BAD = 4, F_END = 8;
 
-template <int BS, int D, typename KT, typename QT>
-__global__ void __launch_bounds__(DecodeCfg<BS, D, KT, QT>::NWARP * 32, 1)
+// The query rows ("columns") of one work item are (member m, query token t, head g) for
+// m < members, t < qtok, g < G, in that order: column c = (m * qtok + t) * G + g.  A plain decode
+// has one member and one query token; multi-token attention has qtok > 1 (query token t sits at
+// position len - qtok + t and attends causally); a shared-prefix item has members > 1 (the
+// sequences seq .. seq + members - 1 share the item's tokens).
+template <int BS, int D, typename KT, typename QT, int NT>
+__global__ void __launch_bounds__(DecodeCfg<BS, D, KT, QT, NT>::NWARP * 32, 1)
     pa_decode_partition_kernel(const __grid_constant__ CUtensorMap tmk,
                                const __grid_constant__ CUtensorMap tmv, const DecodeParams p) {
-  using C = DecodeCfg<BS, D, KT, QT>;
+  using C = DecodeCfg<BS, D, KT, QT, NT>;
   using MA = typename KvTraits<KT>::mma_t;  // element type of the tensor-core operands
   constexpr unsigned FULL = 0xffffffffu;
 
@@ -264,24 +274,21 @@ __global__ void __launch_bounds__(DecodeCfg<BS, D, KT, QT>::NWARP * 32, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int c = warp % C::NC;  // consumer index of this warp's pair
-  uint8_t* ring = smem + c * C::NSLOT * C::SLOT_BYTES;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::RING_BYTES) + c * 2 * C::NSLOT;
+  uint8_t* ring = smem + c * (C::NSLOT * C::SLOT_BYTES + C::QBUF_BYTES);
+  uint8_t* qbuf = ring + C::NSLOT * C::SLOT_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::RING_BYTES) + c * (2 * C::NSLOT + 2);
   uint64_t* empty = full + C::NSLOT;
+  uint64_t* qfree = empty + C::NSLOT;
   int4* meta = reinterpret_cast<int4*>(smem + C::RING_BYTES + C::BAR_BYTES) + c * C::NSLOT;
   volatile int* flags_base = reinterpret_cast<volatile int*>(smem + C::RING_BYTES + C::BAR_BYTES + C::META_BYTES);
   volatile int* abort_flag = flags_base + 4 * c;
 
-  if (warp < C::NC) {
-    // query rows >= G of every slot stay zero: the bulk copy only ever writes rows < G
-    for (int s = 0; s < C::NSLOT; ++s) {
-      uint4* qz = reinterpret_cast<uint4*>(ring + s * C::SLOT_BYTES + 2 * C::PAGE_BYTES);
-      for (int i = lane; i < C::Q_BYTES / 16; i += 32) qz[i] = make_uint4(0, 0, 0, 0);
-    }
-  }
   if (threadIdx.x == 0) {
-    uint64_t* all = reinterpret_cast<uint64_t*>(smem + C::RING_BYTES);
-    for (int s = 0; s < 2 * C::NC * C::NSLOT; ++s) mbar_init(&all[s], 1);
-    for (int i = 0; i < C::NC; ++i) flags_base[4 * i] = 0;
+    for (int i = 0; i < C::NC; ++i) {
+      uint64_t* b = reinterpret_cast<uint64_t*>(smem + C::RING_BYTES) + i * (2 * C::NSLOT + 2);
+      for (int s = 0; s < 2 * C::NSLOT + 1; ++s) mbar_init(&b[s], 1);
+      flags_base[4 * i] = 0;
+    }
     fence_mbar_init();
     prefetch_tensormap(&tmk);
     prefetch_tensormap(&tmv);
@@ -289,13 +296,14 @@ __global__ void __launch_bounds__(DecodeCfg<BS, D, KT, QT>::NWARP * 32, 1)
   __syncthreads();
   pdl_wait();  // the plan kernel's work list and counters are visible from here on
 
-  const int G = p.group, Hkv = p.num_kv_heads, Hq = p.num_q_heads;
+  const int G = p.group, Hkv = p.num_kv_heads, Hq = p.num_q_heads, T = p.qtok;
 
   if (warp >= C::NC) {
     // ============================== producer ==============================
     const unsigned total = p.counters[1] * static_cast<unsigned>(Hkv);
     const uint64_t pol = policy_evict_first();
-    uint32_t n = 0;  // pages issued into this ring
+    uint32_t n = 0;      // pages issued into this ring
+    uint32_t items = 0;  // items started (the query buffer is refilled once per item)
     bool stop = false;
     auto acquire_slot = [&](int slot) -> bool {  // wait until the consumer freed `slot`
       if (n < C::NSLOT) return true;
@@ -312,7 +320,7 @@ __global__ void __launch_bounds__(DecodeCfg<BS, D, KT, QT>::NWARP * 32, 1)
       const int tok0 = it.part * p.partition_size;
       const int tok1 = min(it.len, tok0 + p.partition_size);
       const int npages = (tok1 - tok0 + BS - 1) / BS;
-      const int nparts = (it.len + p.partition_size - 1) / p.partition_size;
+      const int rows = it.members * T;  // (member, query token) pairs of the item: G query rows each
       int bt = 0;
       bool bad = false;
       if (lane < npages) {
@@ -321,6 +329,13 @@ __global__ void __launch_bounds__(DecodeCfg<BS, D, KT, QT>::NWARP * 32, 1)
       }
       bad = __any_sync(FULL, bad);
       if (bad && lane == 0) record_error(DEV_BAD_BLOCK_ID);
+      if (items >= 1) {  // the consumer has taken the previous item's query rows
+        const bool ok = mbar_wait_bounded(qfree, (items - 1) & 1u, kWaitLimit);
+        if (!__all_sync(FULL, ok) || *abort_flag) {
+          stop = true;
+          break;
+        }
+      }
       for (int pg = 0; pg < npages; ++pg) {
         const int phys = __shfl_sync(FULL, bt, pg);
         const int slot = static_cast<int>(n % C::NSLOT);
@@ -328,15 +343,16 @@ __global__ void __launch_bounds__(DecodeCfg<BS, D, KT, QT>::NWARP * 32, 1)
           stop = true;
           break;
         }
+        const bool first = pg == 0;
         if (lane == 0) {
           uint8_t* sb = ring + slot * C::SLOT_BYTES;
           const int ntok = min(BS, tok1 - (tok0 + pg * BS));
-          const int flags = (pg == 0 ? F_FIRST : 0) | (pg == npages - 1 ? F_LAST : 0) | (bad ? F_BAD : 0);
-          meta[slot] = make_int4(it.seq, it.part, kvh, ntok | (flags << 8) | (nparts << 16));
+          const int flags = (first ? F_FIRST : 0) | (pg == npages - 1 ? F_LAST : 0) | (bad ? F_BAD : 0);
+          meta[slot] = make_int4(it.seq, it.part | (pg << 16), kvh | (ntok << 16) | (flags << 24), it.len);
           if (bad) {
             mbar_arrive(&full[slot]);
           } else {
-            const uint32_t qbytes = pg == 0 ? static_cast<uint32_t>(G * D * C::QE) : 0u;
+            const uint32_t qbytes = first ? static_cast<uint32_t>(rows * G * D * C::QE) : 0u;
             mbar_arrive_expect_tx(&full[slot], 2 * C::PAGE_BYTES + qbytes);
 #pragma unroll
             for (int h = 0; h < C::HALVES; ++h) {
@@ -344,20 +360,27 @@ __global__ void __launch_bounds__(DecodeCfg<BS, D, KT, QT>::NWARP * 32, 1)
               tma_load_3d(sb + C::PAGE_BYTES + h * C::BOX_BYTES, &tmv, 0, kvh * C::HALVES + h, phys * BS,
                           &full[slot], pol);
             }
-            if (qbytes)
-              bulk_load(sb + 2 * C::PAGE_BYTES,
-                        static_cast<const uint8_t*>(p.q) + (static_cast<int64_t>(it.seq) * Hq + kvh * G) * D * C::QE,
-                        qbytes, &full[slot]);
+          }
+        }
+        if (first && !bad) {
+          __syncwarp();  // the expected byte count is set before any copy can complete
+          if (lane < rows) {  // query rows of (member, token) lane: G contiguous heads
+            const int m = lane / T, t = lane - m * T;
+            bulk_load(qbuf + lane * G * D * C::QE,
+                      static_cast<const uint8_t*>(p.q) +
+                          ((static_cast<int64_t>(it.seq + m) * T + t) * Hq + kvh * G) * D * C::QE,
+                      static_cast<uint32_t>(G * D * C::QE), &full[slot]);
           }
         }
         ++n;
       }
+      ++items;
     }
     if (!stop) {  // tell the consumer there is no more work
       const int slot = static_cast<int>(n % C::NSLOT);
       if (acquire_slot(slot)) {
         if (lane == 0) {
-          meta[slot] = make_int4(0, 0, 0, F_END << 8);
+          meta[slot] = make_int4(0, 0, F_END << 24, 0);
           mbar_arrive(&full[slot]);
         }
       } else {
@@ -366,6 +389,7 @@ __global__ void __launch_bounds__(DecodeCfg<BS, D, KT, QT>::NWARP * 32, 1)
     }
     if (stop) {
       if (lane == 0) record_error(DEV_TIMEOUT);
+      // copies this warp issued may still be landing: wait for them before the CTA exits
       for (uint32_t k = n > C::NSLOT ? n - C::NSLOT : 0; k < n; ++k)
         mbar_wait_bounded(&full[k % C::NSLOT], (k / C::NSLOT) & 1u, kWaitLimit);
     }
@@ -375,13 +399,13 @@ __global__ void __launch_bounds__(DecodeCfg<BS, D, KT, QT>::NWARP * 32, 1)
   // ============================== consumer ==============================
   const int lr = lane & 7, lm = lane >> 3;  // ldmatrix: row inside an 8x8 matrix, matrix index
   const int r0 = lane >> 2, c2 = (lane & 3) * 2;
-  // per-lane swizzled offsets of the ldmatrix rows (the same in every slot and 16-row tile)
-  uint32_t koff[C::KS], voff[C::KS];
-#pragma unroll
-  for (int k = 0; k < C::KS; ++k) {
-    koff[k] = swz<C::BOX_BYTES>(lr + ((lm & 1) << 3), k * 16 + ((lm >> 1) << 3));
-    voff[k] = swz<C::BOX_BYTES>(lr + ((lm >> 1) << 3), k * 16 + ((lm & 1) << 3));
-  }
+  // per-lane swizzled offsets of the ldmatrix rows (the same in every slot and 16-row tile).
+  // Step k adds 2k to the 16-byte chunk index, an even number, so under the XOR swizzle its
+  // offset is the step-0 offset XOR (k mod 4) << 5, plus the 128-byte column block k / 4.
+  const uint32_t koff0 = swz<C::BOX_BYTES>(lr + ((lm & 1) << 3), (lm >> 1) << 3);
+  const uint32_t voff0 = swz<C::BOX_BYTES>(lr + ((lm >> 1) << 3), (lm & 1) << 3);
+  auto koff = [&](int k) { return (koff0 ^ ((k & 3) << 5)) + (k >> 2) * C::BOX_BYTES; };
+  auto voff = [&](int k) { return (voff0 ^ ((k & 3) << 5)) + (k >> 2) * C::BOX_BYTES; };
   const float sl = p.scale_log2;
   const uint32_t ones = pack2<MA>(1.f, 1.f);
   // FP8 tiles: per-lane offsets of the K rows for ldmatrix (row lr + 8 (lm & 1), 16-byte chunk
@@ -398,23 +422,33 @@ __global__ void __launch_bounds__(DecodeCfg<BS, D, KT, QT>::NWARP * 32, 1)
     vx1 = (c2 + 1) & 7;
   }
 
-  float mu0 = -CUDART_INF_F, mu1 = -CUDART_INF_F;  // running maxima (log2 units), columns c2, c2+1
-  float acc[C::KS][4] = {};
-  float lacc[4] = {0.f, 0.f, 0.f, 0.f};
-  uint32_t qf[C::KS][2];
+  float mu[NT][2];  // running maxima (log2 units) of columns nt * 8 + c2, + 1
+  float acc[C::KS][NT][4] = {};
+  float lacc[NT][4] = {};
+  uint32_t qf[C::KS][NT][2];
   uint32_t ql[C::QSPLIT ? C::KS : 1][2];
   (void)ql;
   bool poisoned = false;
+  int ncol = G;  // query rows of the current item
 
-  auto load_q = [&](const uint8_t* qs) {
+  auto load_q = [&]() {  // query rows of the item from the consumer's buffer; rows >= ncol are zero
     if constexpr (!C::QSPLIT && !C::QCONV) {
 #pragma unroll
-      for (int k2 = 0; k2 < C::KS; k2 += 2) {
-        const int d0 = (k2 + (lm >> 1)) * 16 + ((lm & 1) << 3);
-        ldsm_x4(smem_u32(qs + (lr * D + d0) * 2), qf[k2][0], qf[k2][1], qf[k2 + 1][0], qf[k2 + 1][1]);
+      for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+        for (int k2 = 0; k2 < C::KS; k2 += 2) {
+          const int d0 = (k2 + (lm >> 1)) * 16 + ((lm & 1) << 3);
+          ldsm_x4(smem_u32(qbuf + ((nt * 8 + lr) * D + d0) * 2), qf[k2][nt][0], qf[k2][nt][1], qf[k2 + 1][nt][0],
+                  qf[k2 + 1][nt][1]);
+        }
+        if (nt * 8 + r0 >= ncol) {
+#pragma unroll
+          for (int k = 0; k < C::KS; ++k) qf[k][nt][0] = qf[k][nt][1] = 0u;
+        }
       }
     } else {
-      const QT* qv = reinterpret_cast<const QT*>(qs);
+      const QT* qv = reinterpret_cast<const QT*>(qbuf);
+      const bool live = r0 < ncol;
 #pragma unroll
       for (int kk = 0; kk < C::KS; ++kk) {
 #pragma unroll
@@ -423,9 +457,9 @@ __global__ void __launch_bounds__(DecodeCfg<BS, D, KT, QT>::NWARP * 32, 1)
           // (pairs h = 0, 1); the query takes the same order.  Otherwise the usual
           // m16n8k16 columns 16 kk + 2c (+1) and + 8.
           const int d = C::FP8 ? kk * 16 + 2 * c2 + 2 * h : kk * 16 + h * 8 + c2;
-          const float x0 = to_float(qv[r0 * D + d]), x1 = to_float(qv[r0 * D + d + 1]);
+          const float x0 = live ? to_float(qv[r0 * D + d]) : 0.f, x1 = live ? to_float(qv[r0 * D + d + 1]) : 0.f;
           const uint32_t hi = pack2<MA>(x0, x1);
-          qf[kk][h] = hi;
+          qf[kk][0][h] = hi;
           if constexpr (C::QSPLIT) {
             const float2 hf = unpack2<MA>(hi);
             ql[kk][h] = pack2<MA>(x0 - hf.x, x1 - hf.y);
@@ -435,189 +469,239 @@ __global__ void __launch_bounds__(DecodeCfg<BS, D, KT, QT>::NWARP * 32, 1)
     }
   };
 
-  auto page_math = [&](const uint8_t* sb, int ntok) {
+  // One page: S^T = K . Q^T, online-softmax update, O^T += V^T . P^T.  The softmax state is
+  // updated once per chunk of MC 16-token tiles: the whole page for items of up to 16 query
+  // rows, each tile on its own for wider items (their scores would not fit in registers).
+  auto page_math = [&](const uint8_t* sb, int ntok, int kpos0, int len) {
     const uint32_t kb = smem_u32(sb), vb = kb + C::PAGE_BYTES;
-    float s[C::MT][4];
+    constexpr int MC = NT > 2 ? 1 : C::MT;
 #pragma unroll
-    for (int mt = 0; mt < C::MT; ++mt) {
-      float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb2[4] = {0.f, 0.f, 0.f, 0.f};
-      if constexpr (C::FP8) {
-        // one ldmatrix.x4 holds 32 columns of 16 rows: lane gets 4 codes of row r0 (r0 + 8)
+    for (int m0 = 0; m0 < C::MT; m0 += MC) {
+      float s[MC][NT][4];
 #pragma unroll
-        for (int kq = 0; kq < C::KS / 2; ++kq) {
-          uint32_t r[4];
-          ldsm_x4(kb + mt * 2048 + koff8[kq], r[0], r[1], r[2], r[3]);
+      for (int mi = 0; mi < MC; ++mi) {
+        const int mt = m0 + mi;
+        float sa[NT][4] = {}, sb2[NT][4] = {};
+        if constexpr (C::FP8) {
+          // one ldmatrix.x4 holds 32 columns of 16 rows: lane gets 4 codes of row r0 (r0 + 8)
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const int kk = 2 * kq + h;
-            const uint32_t a0 = e4m3x2_to_f16x2(r[2 * h]), a1 = e4m3x2_to_f16x2(r[2 * h + 1]);
-            const uint32_t a2 = e4m3x2_to_f16x2(r[2 * h] >> 16), a3 = e4m3x2_to_f16x2(r[2 * h + 1] >> 16);
-            if constexpr (C::QSPLIT) {
-              Mma<MA>::run(sa, a0, a1, a2, a3, qf[kk][0], qf[kk][1]);
-              Mma<MA>::run(sb2, a0, a1, a2, a3, ql[kk][0], ql[kk][1]);
-            } else {
-              Mma<MA>::run(h ? sb2 : sa, a0, a1, a2, a3, qf[kk][0], qf[kk][1]);
+          for (int kq = 0; kq < C::KS / 2; ++kq) {
+            uint32_t r[4];
+            ldsm_x4(kb + mt * 2048 + koff8[kq], r[0], r[1], r[2], r[3]);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const int kk = 2 * kq + h;
+              const uint32_t a0 = e4m3x2_to_f16x2(r[2 * h]), a1 = e4m3x2_to_f16x2(r[2 * h + 1]);
+              const uint32_t a2 = e4m3x2_to_f16x2(r[2 * h] >> 16), a3 = e4m3x2_to_f16x2(r[2 * h + 1] >> 16);
+              if constexpr (C::QSPLIT) {
+                Mma<MA>::run(sa[0], a0, a1, a2, a3, qf[kk][0][0], qf[kk][0][1]);
+                Mma<MA>::run(sb2[0], a0, a1, a2, a3, ql[kk][0], ql[kk][1]);
+              } else {
+                Mma<MA>::run(h ? sb2[0] : sa[0], a0, a1, a2, a3, qf[kk][0][0], qf[kk][0][1]);
+              }
+            }
+          }
+        } else {
+#pragma unroll
+          for (int kk = 0; kk < C::KS; ++kk) {
+            uint32_t a0, a1, a2, a3;
+            ldsm_x4(kb + mt * 2048 + koff(kk), a0, a1, a2, a3);
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+              if constexpr (C::QSPLIT) {
+                Mma<MA>::run(sa[nt], a0, a1, a2, a3, qf[kk][nt][0], qf[kk][nt][1]);
+                Mma<MA>::run(sb2[nt], a0, a1, a2, a3, ql[kk][0], ql[kk][1]);
+              } else if (kk & 1) {
+                Mma<MA>::run(sb2[nt], a0, a1, a2, a3, qf[kk][nt][0], qf[kk][nt][1]);
+              } else {
+                Mma<MA>::run(sa[nt], a0, a1, a2, a3, qf[kk][nt][0], qf[kk][nt][1]);
+              }
             }
           }
         }
-      } else {
 #pragma unroll
-        for (int kk = 0; kk < C::KS; ++kk) {
-          uint32_t a0, a1, a2, a3;
-          ldsm_x4(kb + mt * 2048 + koff[kk], a0, a1, a2, a3);
-          if constexpr (C::QSPLIT) {
-            Mma<MA>::run(sa, a0, a1, a2, a3, qf[kk][0], qf[kk][1]);
-            Mma<MA>::run(sb2, a0, a1, a2, a3, ql[kk][0], ql[kk][1]);
-          } else if (kk & 1) {
-            Mma<MA>::run(sb2, a0, a1, a2, a3, qf[kk][0], qf[kk][1]);
-          } else {
-            Mma<MA>::run(sa, a0, a1, a2, a3, qf[kk][0], qf[kk][1]);
-          }
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) s[mi][nt][e] = sa[nt][e] + sb2[nt][e];
+      }
+      if (ntok < BS) {  // tokens past the end of the partition do not take part
+#pragma unroll
+        for (int mi = 0; mi < MC; ++mi)
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+              if ((m0 + mi) * 16 + r0 + 8 * h >= ntok) s[mi][nt][2 * h] = s[mi][nt][2 * h + 1] = -CUDART_INF_F;
+      }
+      if (T > 1 && kpos0 + BS > len - T) {
+        // causal: query token t (position len - T + t) sees keys up to its own position
+#pragma unroll
+        for (int mi = 0; mi < MC; ++mi)
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int col = nt * 8 + c2 + (e & 1);
+              const int t = (col / G) % T;
+              if (kpos0 + (m0 + mi) * 16 + r0 + 8 * (e >> 1) > len - T + t) s[mi][nt][e] = -CUDART_INF_F;
+            }
+      }
+      // raw (unscaled) maxima of this lane's entries; scale > 0 commutes with max
+      float x[NT][2];
+      bool raise = false;
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        x[nt][0] = x[nt][1] = -CUDART_INF_F;
+#pragma unroll
+        for (int mi = 0; mi < MC; ++mi) {
+          x[nt][0] = fmaxf(x[nt][0], fmaxf(s[mi][nt][0], s[mi][nt][2]));
+          x[nt][1] = fmaxf(x[nt][1], fmaxf(s[mi][nt][1], s[mi][nt][3]));
         }
+        raise |= x[nt][0] * sl > mu[nt][0] + kRescaleThreshold || x[nt][1] * sl > mu[nt][1] + kRescaleThreshold;
       }
+      if (__any_sync(FULL, raise)) {
 #pragma unroll
-      for (int e = 0; e < 4; ++e) s[mt][e] = sa[e] + sb2[e];
-    }
-    if (ntok < BS) {  // tokens past the end of the partition do not take part
+        for (int nt = 0; nt < NT; ++nt) {
 #pragma unroll
-      for (int mt = 0; mt < C::MT; ++mt)
-#pragma unroll
-        for (int h = 0; h < 2; ++h)
-          if (mt * 16 + r0 + 8 * h >= ntok) s[mt][2 * h] = s[mt][2 * h + 1] = -CUDART_INF_F;
-    }
-    // raw (unscaled) maxima of this lane's entries; scale > 0 commutes with max
-    float x0 = -CUDART_INF_F, x1 = -CUDART_INF_F;
-#pragma unroll
-    for (int mt = 0; mt < C::MT; ++mt) {
-      x0 = fmaxf(x0, fmaxf(s[mt][0], s[mt][2]));
-      x1 = fmaxf(x1, fmaxf(s[mt][1], s[mt][3]));
-    }
-    const bool raise = x0 * sl > mu0 + kRescaleThreshold || x1 * sl > mu1 + kRescaleThreshold;
-    if (__any_sync(FULL, raise)) {
-#pragma unroll
-      for (int o = 4; o < 32; o <<= 1) {
-        x0 = fmaxf(x0, __shfl_xor_sync(FULL, x0, o));
-        x1 = fmaxf(x1, __shfl_xor_sync(FULL, x1, o));
-      }
-      const float n0 = fmaxf(mu0, x0 * sl), n1 = fmaxf(mu1, x1 * sl);
-      const float al0 = fast_exp2(mu0 - n0), al1 = fast_exp2(mu1 - n1);
-      mu0 = n0;
-      mu1 = n1;
-#pragma unroll
-      for (int dt = 0; dt < C::KS; ++dt) {
-        acc[dt][0] *= al0;
-        acc[dt][1] *= al1;
-        acc[dt][2] *= al0;
-        acc[dt][3] *= al1;
-      }
-      lacc[0] *= al0;
-      lacc[1] *= al1;
-      lacc[2] *= al0;
-      lacc[3] *= al1;
-    }
-#pragma unroll
-    for (int mt = 0; mt < C::MT; ++mt) {
-      const uint32_t plo = pack2<MA>(fast_exp2(fmaf(s[mt][0], sl, -mu0)), fast_exp2(fmaf(s[mt][1], sl, -mu1)));
-      const uint32_t phi = pack2<MA>(fast_exp2(fmaf(s[mt][2], sl, -mu0)), fast_exp2(fmaf(s[mt][3], sl, -mu1)));
-      const uint32_t b0 = movmatrix_t(plo), b1 = movmatrix_t(phi);
-      Mma<MA>::run(lacc, ones, ones, ones, ones, b0, b1);  // row sums of the weights as the MMA sees them
-      if constexpr (C::FP8) {
-        // V^T tile (16 columns x 16 tokens) from the codes: a lane reads the 16-bit column pair
-        // (2 r0, 2 r0 + 1) of tokens 2c, 2c+1, 2c+8, 2c+9 and pairs the tokens up by byte
-        // permutation; accumulator rows r0 / r0 + 8 are columns 2 r0 / 2 r0 + 1.
-        const int tk = mt * 16 + c2;
-        const uint32_t row0 = vb + (mt * 16 + c2) * 128 + 2 * r0;
-        auto v_tiles = [&](uint32_t mlo, uint32_t mhi, auto masked) {
+          for (int o = 4; o < 32; o <<= 1) {
+            x[nt][0] = fmaxf(x[nt][0], __shfl_xor_sync(FULL, x[nt][0], o));
+            x[nt][1] = fmaxf(x[nt][1], __shfl_xor_sync(FULL, x[nt][1], o));
+          }
+          const float n0 = fmaxf(mu[nt][0], x[nt][0] * sl), n1 = fmaxf(mu[nt][1], x[nt][1] * sl);
+          // a column that has seen only masked scores keeps -inf; its weights stay 0
+          const float al0 = n0 == -CUDART_INF_F ? 1.f : fast_exp2(mu[nt][0] - n0);
+          const float al1 = n1 == -CUDART_INF_F ? 1.f : fast_exp2(mu[nt][1] - n1);
+          mu[nt][0] = n0;
+          mu[nt][1] = n1;
 #pragma unroll
           for (int dt = 0; dt < C::KS; ++dt) {
-            const uint32_t u0 = lds_u16(row0 + (((dt ^ vx0)) << 4));
-            const uint32_t u1 = lds_u16(row0 + 128 + (((dt ^ vx1)) << 4));
-            const uint32_t u2 = lds_u16(row0 + 8 * 128 + (((dt ^ vx0)) << 4));
-            const uint32_t u3 = lds_u16(row0 + 9 * 128 + (((dt ^ vx1)) << 4));
-            const uint32_t w01 = __byte_perm(u0, u1, 0x5140), w23 = __byte_perm(u2, u3, 0x5140);
-            uint32_t a0 = e4m3x2_to_f16x2(w01), a1 = e4m3x2_to_f16x2(w01 >> 16);
-            uint32_t a2 = e4m3x2_to_f16x2(w23), a3 = e4m3x2_to_f16x2(w23 >> 16);
-            if constexpr (decltype(masked)::value) {
-              a0 &= mlo;
-              a1 &= mlo;
-              a2 &= mhi;
-              a3 &= mhi;
-            }
-            Mma<MA>::run(acc[dt], a0, a1, a2, a3, b0, b1);
+            acc[dt][nt][0] *= al0;
+            acc[dt][nt][1] *= al1;
+            acc[dt][nt][2] *= al0;
+            acc[dt][nt][3] *= al1;
           }
-        };
-        if (ntok >= (mt + 1) * 16) {
-          v_tiles(FULL, FULL, std::false_type{});
-        } else {
-          const uint32_t mlo = (tk < ntok ? 0x0000ffffu : 0u) | (tk + 1 < ntok ? 0xffff0000u : 0u);
-          const uint32_t mhi = (tk + 8 < ntok ? 0x0000ffffu : 0u) | (tk + 9 < ntok ? 0xffff0000u : 0u);
-          v_tiles(mlo, mhi, std::true_type{});
-        }
-      } else if (ntok >= (mt + 1) * 16) {
-#pragma unroll
-        for (int dt = 0; dt < C::KS; ++dt) {
-          uint32_t a0, a1, a2, a3;
-          ldsm_x4_t(vb + mt * 2048 + voff[dt], a0, a1, a2, a3);
-          Mma<MA>::run(acc[dt], a0, a1, a2, a3, b0, b1);
-        }
-      } else {
-        // V rows past the end may hold anything (even NaN): zero them, 0 * NaN would poison
-        const int tk = mt * 16 + c2;
-        const uint32_t mlo = (tk < ntok ? 0x0000ffffu : 0u) | (tk + 1 < ntok ? 0xffff0000u : 0u);
-        const uint32_t mhi = (tk + 8 < ntok ? 0x0000ffffu : 0u) | (tk + 9 < ntok ? 0xffff0000u : 0u);
-#pragma unroll
-        for (int dt = 0; dt < C::KS; ++dt) {
-          uint32_t a0, a1, a2, a3;
-          ldsm_x4_t(vb + mt * 2048 + voff[dt], a0, a1, a2, a3);
-          Mma<MA>::run(acc[dt], a0 & mlo, a1 & mlo, a2 & mhi, a3 & mhi, b0, b1);
+          lacc[nt][0] *= al0;
+          lacc[nt][1] *= al1;
+          lacc[nt][2] *= al0;
+          lacc[nt][3] *= al1;
         }
       }
-    }
+#pragma unroll
+      for (int mi = 0; mi < MC; ++mi) {
+        const int mt = m0 + mi;
+        uint32_t b0[NT], b1[NT];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          // a column with no visible key yet (mu = -inf) gets weight 0, not 2^(-inf + inf)
+          const float u0 = mu[nt][0] == -CUDART_INF_F ? 0.f : mu[nt][0];
+          const float u1 = mu[nt][1] == -CUDART_INF_F ? 0.f : mu[nt][1];
+          const uint32_t plo =
+              pack2<MA>(fast_exp2(fmaf(s[mi][nt][0], sl, -u0)), fast_exp2(fmaf(s[mi][nt][1], sl, -u1)));
+          const uint32_t phi =
+              pack2<MA>(fast_exp2(fmaf(s[mi][nt][2], sl, -u0)), fast_exp2(fmaf(s[mi][nt][3], sl, -u1)));
+          b0[nt] = movmatrix_t(plo);
+          b1[nt] = movmatrix_t(phi);
+          Mma<MA>::run(lacc[nt], ones, ones, ones, ones, b0[nt], b1[nt]);  // row sums of the weights the MMA sees
+        }
+        if constexpr (C::FP8) {
+          // V^T tile (16 columns x 16 tokens) from the codes: a lane reads the 16-bit column pair
+          // (2 r0, 2 r0 + 1) of tokens 2c, 2c+1, 2c+8, 2c+9 and pairs the tokens up by byte
+          // permutation; accumulator rows r0 / r0 + 8 are columns 2 r0 / 2 r0 + 1.
+          const int tk = mt * 16 + c2;
+          const uint32_t row0 = vb + (mt * 16 + c2) * 128 + 2 * r0;
+          auto v_tiles = [&](uint32_t mlo, uint32_t mhi, auto masked) {
+#pragma unroll
+            for (int dt = 0; dt < C::KS; ++dt) {
+              const uint32_t u0 = lds_u16(row0 + (((dt ^ vx0)) << 4));
+              const uint32_t u1 = lds_u16(row0 + 128 + (((dt ^ vx1)) << 4));
+              const uint32_t u2 = lds_u16(row0 + 8 * 128 + (((dt ^ vx0)) << 4));
+              const uint32_t u3 = lds_u16(row0 + 9 * 128 + (((dt ^ vx1)) << 4));
+              const uint32_t w01 = __byte_perm(u0, u1, 0x5140), w23 = __byte_perm(u2, u3, 0x5140);
+              uint32_t a0 = e4m3x2_to_f16x2(w01), a1 = e4m3x2_to_f16x2(w01 >> 16);
+              uint32_t a2 = e4m3x2_to_f16x2(w23), a3 = e4m3x2_to_f16x2(w23 >> 16);
+              if constexpr (decltype(masked)::value) {
+                a0 &= mlo;
+                a1 &= mlo;
+                a2 &= mhi;
+                a3 &= mhi;
+              }
+              Mma<MA>::run(acc[dt][0], a0, a1, a2, a3, b0[0], b1[0]);
+            }
+          };
+          if (ntok >= (mt + 1) * 16) {
+            v_tiles(FULL, FULL, std::false_type{});
+          } else {
+            const uint32_t mlo = (tk < ntok ? 0x0000ffffu : 0u) | (tk + 1 < ntok ? 0xffff0000u : 0u);
+            const uint32_t mhi = (tk + 8 < ntok ? 0x0000ffffu : 0u) | (tk + 9 < ntok ? 0xffff0000u : 0u);
+            v_tiles(mlo, mhi, std::true_type{});
+          }
+        } else if (ntok >= (mt + 1) * 16) {
+#pragma unroll
+          for (int dt = 0; dt < C::KS; ++dt) {
+            uint32_t a0, a1, a2, a3;
+            ldsm_x4_t(vb + mt * 2048 + voff(dt), a0, a1, a2, a3);
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) Mma<MA>::run(acc[dt][nt], a0, a1, a2, a3, b0[nt], b1[nt]);
+          }
+        } else {
+          // V rows past the end may hold anything (even NaN): zero them, 0 * NaN would poison
+          const int tk = mt * 16 + c2;
+          const uint32_t mlo = (tk < ntok ? 0x0000ffffu : 0u) | (tk + 1 < ntok ? 0xffff0000u : 0u);
+          const uint32_t mhi = (tk + 8 < ntok ? 0x0000ffffu : 0u) | (tk + 9 < ntok ? 0xffff0000u : 0u);
+#pragma unroll
+          for (int dt = 0; dt < C::KS; ++dt) {
+            uint32_t a0, a1, a2, a3;
+            ldsm_x4_t(vb + mt * 2048 + voff(dt), a0, a1, a2, a3);
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+              Mma<MA>::run(acc[dt][nt], a0 & mlo, a1 & mlo, a2 & mhi, a3 & mhi, b0[nt], b1[nt]);
+          }
+        }
+      }
+    }  // chunk of MC tiles
   };
 
+  // Write the item's result.  Column col = (m * T + t) * G + g is query head kvh * G + g of
+  // query token t of sequence seq + m; its "virtual head" (T query tokens x Hq heads) is
+  // t * Hq + kvh * G + g.
   auto finalize = [&](int seq, int part, int kvh, int np) {
-    const int g0 = c2, g1 = c2 + 1;
-    const int hq0 = kvh * G + g0, hq1 = hq0 + 1;
     const float nan = CUDART_NAN_F;
-    const float l0 = lacc[0], l1 = lacc[1];  // every row of the ones-MMA holds the column sums
     // accumulator rows r0 and r0 + 8 of tile dt are columns d and d + dd
     const int dd = C::FP8 ? 1 : 8;
     const float vs = p.v_scale;
-    if (np == 1) {
-      const float i0 = poisoned ? nan : vs / l0, i1 = poisoned ? nan : vs / l1;
-      const int64_t o0 = (static_cast<int64_t>(seq) * Hq + hq0) * D, o1 = o0 + D;
+    const int HV = T * Hq;
 #pragma unroll
-      for (int dt = 0; dt < C::KS; ++dt) {
-        const int d = dt * 16 + (C::FP8 ? 2 * r0 : r0);
-        if (g0 < G) {
-          store_out(p.out, o0 + d, acc[dt][0] * i0, p.out_dtype);
-          store_out(p.out, o0 + d + dd, acc[dt][2] * i0, p.out_dtype);
-        }
-        if (g1 < G) {
-          store_out(p.out, o1 + d, acc[dt][1] * i1, p.out_dtype);
-          store_out(p.out, o1 + d + dd, acc[dt][3] * i1, p.out_dtype);
-        }
-      }
-      return;
-    }
-    const int64_t pidx = static_cast<int64_t>(seq) * p.max_parts + part;
-    float* pa0 = p.part_acc + (pidx * Hq + hq0) * D;
-    float* pa1 = pa0 + D;
+    for (int nt = 0; nt < NT; ++nt) {
 #pragma unroll
-    for (int dt = 0; dt < C::KS; ++dt) {
-      const int d = dt * 16 + (C::FP8 ? 2 * r0 : r0);
-      if (g0 < G) {
-        __stcg(pa0 + d, poisoned ? nan : acc[dt][0] * vs);
-        __stcg(pa0 + d + dd, poisoned ? nan : acc[dt][2] * vs);
+      for (int j = 0; j < 2; ++j) {
+        const int col = nt * 8 + c2 + j;
+        if (col >= ncol) continue;
+        const int g = col % G, mt_ = col / G;
+        const int m = mt_ / T, t = mt_ - m * T;
+        const int vh = t * Hq + kvh * G + g;
+        const float l = lacc[nt][j];  // every row of the ones-MMA holds the column sums
+        if (np == 1) {
+          const float inv = poisoned ? nan : vs / l;
+          const int64_t o = (static_cast<int64_t>(seq + m) * HV + vh) * D;
+#pragma unroll
+          for (int dt = 0; dt < C::KS; ++dt) {
+            const int d = dt * 16 + (C::FP8 ? 2 * r0 : r0);
+            store_out(p.out, o + d, acc[dt][nt][j] * inv, p.out_dtype);
+            store_out(p.out, o + d + dd, acc[dt][nt][2 + j] * inv, p.out_dtype);
+          }
+        } else {
+          const int64_t pidx = static_cast<int64_t>(seq + m) * p.max_parts + part;
+          float* pa = p.part_acc + (pidx * HV + vh) * D;
+#pragma unroll
+          for (int dt = 0; dt < C::KS; ++dt) {
+            const int d = dt * 16 + (C::FP8 ? 2 * r0 : r0);
+            __stcg(pa + d, poisoned ? nan : acc[dt][nt][j] * vs);
+            __stcg(pa + d + dd, poisoned ? nan : acc[dt][nt][2 + j] * vs);
+          }
+          if (r0 == 0)
+            __stcg(&p.part_ml[pidx * HV + vh], poisoned ? make_float2(0.f, nan) : make_float2(mu[nt][j], l));
+        }
       }
-      if (g1 < G) {
-        __stcg(pa1 + d, poisoned ? nan : acc[dt][1] * vs);
-        __stcg(pa1 + d + dd, poisoned ? nan : acc[dt][3] * vs);
-      }
-    }
-    if (lane < 4) {
-      if (g0 < G) __stcg(&p.part_ml[pidx * Hq + hq0], poisoned ? make_float2(0.f, nan) : make_float2(mu0, l0));
-      if (g1 < G) __stcg(&p.part_ml[pidx * Hq + hq1], poisoned ? make_float2(0.f, nan) : make_float2(mu1, l1));
     }
   };
 
@@ -632,21 +716,28 @@ __global__ void __launch_bounds__(DecodeCfg<BS, D, KT, QT>::NWARP * 32, 1)
       break;
     }
     const int4 mt = meta[slot];
-    const int ntok = mt.w & 0xff, flags = (mt.w >> 8) & 0xff, np = mt.w >> 16;
+    const int kvh = mt.z & 0xffff, ntok = (mt.z >> 16) & 0xff, flags = (mt.z >> 24) & 0xff;
     if (flags & F_END) break;
+    const int part = mt.y & 0xffff, pg = mt.y >> 16, len = mt.w;
     const uint8_t* sb = ring + slot * C::SLOT_BYTES;
     if (flags & F_FIRST) {
-      mu0 = mu1 = -CUDART_INF_F;
 #pragma unroll
-      for (int dt = 0; dt < C::KS; ++dt) acc[dt][0] = acc[dt][1] = acc[dt][2] = acc[dt][3] = 0.f;
-      lacc[0] = lacc[1] = lacc[2] = lacc[3] = 0.f;
+      for (int nt = 0; nt < NT; ++nt) {
+        mu[nt][0] = mu[nt][1] = -CUDART_INF_F;
+        lacc[nt][0] = lacc[nt][1] = lacc[nt][2] = lacc[nt][3] = 0.f;
+#pragma unroll
+        for (int dt = 0; dt < C::KS; ++dt) acc[dt][nt][0] = acc[dt][nt][1] = acc[dt][nt][2] = acc[dt][nt][3] = 0.f;
+      }
       poisoned = (flags & F_BAD) != 0;
-      if (!poisoned) load_q(sb + 2 * C::PAGE_BYTES);
+      ncol = p.item_cols;  // the same for every item of a call
+      if (!poisoned) load_q();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(qfree);  // the query buffer may take the next item's rows
     }
-    if (!poisoned) page_math(sb, ntok);
+    if (!poisoned) page_math(sb, ntok, part * p.partition_size + pg * BS, len);
     __syncwarp();  // every lane is done reading the slot before it is handed back
     if (lane == 0) mbar_arrive(&empty[slot]);
-    if (flags & F_LAST) finalize(mt.x, mt.y, mt.z, np);
+    if (flags & F_LAST) finalize(mt.x, part, kvh, (len + p.partition_size - 1) / p.partition_size);
     ++n;
   }
   if (!ok && lane == 0) {
@@ -656,14 +747,15 @@ __global__ void __launch_bounds__(DecodeCfg<BS, D, KT, QT>::NWARP * 32, 1)
 }
 
 // ------------------------------------------------------------------------------ merge
-// One warp per (sequence, query head) of a sequence with more than one partition:
+// One warp per (sequence, virtual head = query token x query head) of a sequence with more
+// than one partition:
 // out = sum_k 2^(m_k - M) O_k / sum_k 2^(m_k - M) l_k, M = max_k m_k, partitions in order.
 constexpr int kMergeWarps = 8;
 __global__ void __launch_bounds__(kMergeWarps * 32) pa_decode_merge_kernel(const DecodeParams p) {
   pdl_wait();  // the partition kernel's partial results are visible from here on
   const int lane = threadIdx.x & 31;
   const int64_t pair = static_cast<int64_t>(blockIdx.x) * kMergeWarps + (threadIdx.x >> 5);
-  const int Hq = p.num_q_heads, D = p.head_dim, P = p.partition_size;
+  const int Hq = p.qtok * p.num_q_heads, D = p.head_dim, P = p.partition_size;
   if (pair >= static_cast<int64_t>(p.num_seqs) * Hq) return;
   const int seq = static_cast<int>(pair / Hq), hq = static_cast<int>(pair % Hq);
   const int L = p.seq_lens[seq];

@@ -137,7 +137,7 @@ class Workload:
     q_dtype: str
     kv_dtype: str
     scale: float                  # float32 value of 1/sqrt(head_dim)
-    q: np.ndarray                 # [N, Hq, D]
+    q: np.ndarray                 # [N, Hq, D]; [N, T, Hq, D] with T = num_q_tokens > 1
     k_cache: np.ndarray           # [NB, bs, Hkv, D], state before the step
     v_cache: np.ndarray
     block_tables: np.ndarray      # int32 [N, MB], padded with -1
@@ -150,6 +150,7 @@ class Workload:
     new_dtype: str = ""           # dtype of new_k / new_v ("" = kv_dtype)
     k_scale: float = 1.0          # FP8 cache: value = code * scale
     v_scale: float = 1.0
+    num_q_tokens: int = 1         # query tokens per sequence: the last T tokens, stored in the step
 
     @property
     def new_kv_dtype(self) -> str:
@@ -208,13 +209,15 @@ def build_groups(name: str, groups: Sequence[Group], *, num_q_heads: int, num_kv
                  head_dim: int, block_size: int, q_dtype: str, kv_dtype: str, seed: int,
                  pool_factor: float = 1.25, num_blocks: Optional[int] = None,
                  notes: Optional[dict] = None, new_dtype: str = "bf16",
-                 k_scale: float = FP8_K_SCALE, v_scale: float = FP8_V_SCALE) -> Workload:
+                 k_scale: float = FP8_K_SCALE, v_scale: float = FP8_V_SCALE, num_q_tokens: int = 1) -> Workload:
     """Materialise a decode step from groups of prefix-sharing sequences.
 
     Sequence order is group by group, member by member.  The pool holds
     ``num_blocks`` blocks, or ceil(pool_factor * blocks the step needs).  With kv_dtype
     "e4m3" the pool holds FP8 codes of N(0,1) / scale, and the step's new tokens are
-    ``new_dtype`` values that the step itself quantises.
+    ``new_dtype`` values that the step itself quantises.  With num_q_tokens T > 1 the
+    queries are [N, T, Hq, D]: each sequence's step appends T tokens (or none, for an empty
+    sequence), which its T query tokens then attend to causally.
     """
     if num_q_heads % num_kv_heads:
         raise ValueError("num_q_heads must be a multiple of num_kv_heads")
@@ -256,7 +259,12 @@ def build_groups(name: str, groups: Sequence[Group], *, num_q_heads: int, num_kv
 
     N = len(tables)
     Hkv, D = num_kv_heads, head_dim
-    q = _draw((seed, _S_Q), (N, num_q_heads, head_dim), q_dtype)
+    if num_q_tokens > 1 and any(n not in (0, num_q_tokens) for g in groups for n in g.step_tokens):
+        raise ValueError("with several query tokens every sequence appends exactly that many tokens (or none)")
+    # the [N, Hq, D] draw of one query token is the [N, 1, Hq, D] draw
+    q = _draw((seed, _S_Q), (N, num_q_tokens, num_q_heads, head_dim), q_dtype)
+    if num_q_tokens == 1:
+        q = q.reshape(N, num_q_heads, head_dim)
 
     # history: every group's prefix tokens, in group order, K then V
     nan = NAN_BITS[kv_dtype]
@@ -291,13 +299,17 @@ def build_groups(name: str, groups: Sequence[Group], *, num_q_heads: int, num_kv
                     k_cache=k_cache, v_cache=v_cache, block_tables=block_tables, seq_lens=seq_lens,
                     new_k=new_k, new_v=new_v, slot_mapping=all_slots, copy_pairs=pairs, notes=info,
                     new_dtype=ndt, k_scale=float(np.float32(k_scale)) if fp8 else 1.0,
-                    v_scale=float(np.float32(v_scale)) if fp8 else 1.0)
+                    v_scale=float(np.float32(v_scale)) if fp8 else 1.0, num_q_tokens=num_q_tokens)
 
 
-def independent(name: str, seq_lens: Sequence[int], **kw) -> Workload:
-    """Each sequence on its own; seq_lens are post-step lengths, the last token stored in the step."""
-    groups = [Group(prefix=max(int(L) - 1, 0), step_tokens=[1 if L > 0 else 0]) for L in seq_lens]
-    return build_groups(name, groups, **kw)
+def independent(name: str, seq_lens: Sequence[int], num_q_tokens: int = 1, **kw) -> Workload:
+    """Each sequence on its own; seq_lens are post-step lengths, the last num_q_tokens tokens
+    stored in the step (a sequence holds 0 or at least num_q_tokens tokens)."""
+    T = num_q_tokens
+    if any(0 < int(L) < T for L in seq_lens):
+        raise ValueError("a sequence must hold 0 or at least num_q_tokens tokens")
+    groups = [Group(prefix=max(int(L) - T, 0), step_tokens=[T if L > 0 else 0]) for L in seq_lens]
+    return build_groups(name, groups, num_q_tokens=T, **kw)
 
 
 def _fp8_kw(kw: dict) -> dict:
@@ -334,18 +346,18 @@ def _tiny(seed: int, block_size: int) -> Workload:
                         num_blocks=64, notes={"lens": "uniform[1,64]; seq 3 forks seq 2"})
 
 
-def _7b(seed: int, block_size: int, num_seqs: int = 64) -> Workload:
+def _7b(seed: int, block_size: int, num_seqs: int = 64, num_q_tokens: int = 1) -> Workload:
     rng = np.random.default_rng([seed, _S_LENS])
     L = rng.integers(128, 2049, size=num_seqs)
-    return independent("7b", L, **_fp8_kw(dict(num_q_heads=32, num_kv_heads=32, head_dim=128, block_size=block_size,
+    return independent("7b", L, num_q_tokens, **_fp8_kw(dict(num_q_heads=32, num_kv_heads=32, head_dim=128, block_size=block_size,
                                                q_dtype="bf16", kv_dtype="bf16", seed=seed,
                                                notes={"lens": "uniform[128,2048]"})))
 
 
-def _13b(seed: int, block_size: int, num_seqs: int = 128) -> Workload:
+def _13b(seed: int, block_size: int, num_seqs: int = 128, num_q_tokens: int = 1) -> Workload:
     rng = np.random.default_rng([seed, _S_LENS])
     L = rng.integers(16, 2049, size=num_seqs)
-    return independent(f"13b-bs{block_size}", L, **_fp8_kw(dict(num_q_heads=40, num_kv_heads=40, head_dim=128,
+    return independent(f"13b-bs{block_size}", L, num_q_tokens, **_fp8_kw(dict(num_q_heads=40, num_kv_heads=40, head_dim=128,
                                                              block_size=block_size, q_dtype="f16", kv_dtype="f16",
                                                              seed=seed, notes={"lens": "uniform[16,2048]"})))
 
@@ -356,10 +368,10 @@ def lognormal_lengths(rng: np.random.Generator, n: int, median: float = 1024.0, 
     return np.clip(np.rint(np.exp(math.log(median) + sigma * z)), lo, hi).astype(np.int64)
 
 
-def _8b(seed: int, block_size: int, num_seqs: int = 256) -> Workload:
+def _8b(seed: int, block_size: int, num_seqs: int = 256, num_q_tokens: int = 1) -> Workload:
     rng = np.random.default_rng([seed, _S_LENS])
     L = lognormal_lengths(rng, num_seqs)
-    return independent("8b", L, **_fp8_kw(dict(num_q_heads=32, num_kv_heads=8, head_dim=128, block_size=block_size,
+    return independent("8b", L, num_q_tokens, **_fp8_kw(dict(num_q_heads=32, num_kv_heads=8, head_dim=128, block_size=block_size,
                                                q_dtype="bf16", kv_dtype="bf16", seed=seed,
                                                notes={"lens": "lognormal(median 1024, sigma 1.0) clipped to "
                                                               "[32, 8192]"})))
@@ -397,6 +409,8 @@ def make_config(name: str, block_size: Optional[int] = None, seed: Optional[int]
 
     kv_dtype="e4m3" gives the same config over an FP8 cache (head_dim 128 configs): the
     history is stored as FP8 codes, the step's new tokens stay in the config's dtype.
+    num_q_tokens=T ("7b", "13b", "8b") gives the multi-token step: the same lengths, the last
+    T tokens of every sequence stored in the step and attended to causally by T queries.
     """
     if name not in _BUILDERS:
         raise KeyError(f"unknown config {name!r}; choose from {CONFIG_NAMES}")

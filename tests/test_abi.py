@@ -105,3 +105,29 @@ def test_cache_op_argument_validation(lib):
 def test_missing_library_fails_loudly(tmp_path):
     with pytest.raises(ImportError):
         B.load_library(str(tmp_path / "libpa.so"))
+
+
+def multi_call(lib, **kw):
+    a = dict(out=FAKE, q=FAKE, k=FAKE, v=FAKE, bt=FAKE, sl=FAKE, N=4, T=4, Hq=8, Hkv=2, D=128, bs=16, scale=0.1,
+             MB=8, NB=64, qd=2, kd=2, od=0, P=0, ws=FAKE, wsb=0, stream=0)
+    a.update(kw)
+    V = ctypes.c_void_p
+    return lib.pa_decode_multi(V(a["out"]), V(a["q"]), V(a["k"]), V(a["v"]), V(a["bt"]), V(a["sl"]), a["N"],
+                               a["T"], a["Hq"], a["Hkv"], a["D"], a["bs"], ctypes.c_float(a["scale"]), a["MB"],
+                               a["NB"], a["qd"], a["kd"], a["od"], a["P"], V(a["ws"]), a["wsb"], V(a["stream"]))
+
+
+def test_multi_argument_validation(lib):
+    assert multi_call(lib, N=0) == B.PA_OK
+    assert multi_call(lib, T=0) == B.PA_ERR_INVALID
+    assert multi_call(lib, T=9) == B.PA_ERR_UNSUPPORTED            # 9 tokens x 4 heads > 32 query rows
+    assert multi_call(lib, D=64) == B.PA_ERR_UNSUPPORTED           # > 8 rows needs head_dim 128
+    assert multi_call(lib, qd=0) == B.PA_ERR_UNSUPPORTED           # > 8 rows needs q_dtype == kv_dtype
+    assert multi_call(lib, kd=3) == B.PA_ERR_UNSUPPORTED           # FP8 cache
+    assert multi_call(lib, T=2, qd=0) == B.PA_ERR_WORKSPACE        # 8 rows: any dtype pair; then the workspace
+    assert multi_call(lib, T=2, D=64) == B.PA_ERR_WORKSPACE
+    # the workspace is pa_decode's for T * Hq heads
+    need = B.pa_decode_workspace_size(4, 4 * 8, 128, 8 * 16)
+    assert need > B.pa_decode_workspace_size(4, 8, 128, 8 * 16)
+    assert multi_call(lib, wsb=need - 1) == B.PA_ERR_WORKSPACE
+    assert multi_call(lib, ws=FAKE + 16, wsb=need) == B.PA_ERR_INVALID  # passes the size check, not 256-aligned
