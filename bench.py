@@ -62,6 +62,9 @@ def parse_args():
     ap.add_argument("--qtok", type=int, default=1,
                     help="query tokens per sequence: T > 1 runs causal multi-token attention (pa_decode_multi) "
                          "over the same config, the step storing each sequence's last T tokens")
+    ap.add_argument("--prefix", action="store_true",
+                    help="prefix-aware decode (pa_decode_prefix): sequences sharing their first blocks read them "
+                         "once; the groups come from the block tables")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target oracle time for cpu_baseline")
     ap.add_argument("--ref-seconds", type=float, default=150.0, help="target total time of --impl reference")
@@ -115,7 +118,7 @@ def profile_name(args) -> str:
     """Name of the committed ncu summary of this run's partition kernel: config, cache dtype and
     query tokens (pa_decode_partition_8b, pa_decode_partition_8b_e4m3, pa_decode_partition_8b_T5)."""
     return (f"pa_decode_partition_{args.config}" + (f"_{args.kv_dtype}" if args.kv_dtype else "")
-            + (f"_T{args.qtok}" if args.qtok > 1 else ""))
+            + (f"_T{args.qtok}" if args.qtok > 1 else "") + ("_prefix" if args.prefix else ""))
 
 
 def recorded_traffic(name: str):
@@ -306,6 +309,15 @@ def run_ours(args):
     ws = B.DecodeWorkspace.for_workload(dw, args.partition_size)
     out = torch.empty(tuple(dw.q.shape), dtype=B._NAME_TORCH[out_dtype], device="cuda")
     stream = torch.cuda.current_stream()
+    groups_np = np.zeros((0, 3), np.int32)
+    if args.prefix:
+        from paged_kv_cache_327_b200 import block_manager as BM
+
+        if w.num_q_tokens > 1 or w.kv_dtype == "e4m3":
+            raise SystemExit("--prefix runs single-token decode over a 16-bit cache")
+        groups_np = BM.find_prefix_groups(w.block_tables, w.seq_lens, w.block_size)
+    groups = torch.from_numpy(groups_np).to(f"cuda:{local}")
+    max_members = B.max_prefix_members(w.num_q_heads, w.num_kv_heads)
 
     kv_bytes = w.kv_bytes_logical()
     # with shared prefix blocks a physical byte is read once per sharer but fetched from HBM
@@ -317,7 +329,34 @@ def run_ours(args):
     launches_per_step = (1 if len(w.copy_pairs) else 0) + (1 if len(w.slot_mapping) else 0) + 3
 
     def step():
-        B.run_step(dw, out, ws, args.partition_size, stream)
+        if len(w.copy_pairs):
+            B.pa_copy_blocks(dw.k_cache, dw.v_cache, dw.copy_pairs, stream=stream)
+        if len(w.slot_mapping):
+            store()
+        decode()
+
+    fp8 = w.kv_dtype == "e4m3"
+
+    def store():
+        if fp8:
+            B.pa_reshape_and_cache_fp8(dw.new_k, dw.new_v, dw.k_cache, dw.v_cache, dw.slot_mapping, w.k_scale,
+                                       w.v_scale, stream=stream)
+        else:
+            B.pa_reshape_and_cache(dw.new_k, dw.new_v, dw.k_cache, dw.v_cache, dw.slot_mapping, stream=stream)
+
+    def decode():
+        if args.prefix:
+            B.pa_decode_prefix(out, dw.q, dw.k_cache, dw.v_cache, dw.block_tables, dw.seq_lens, w.scale, ws.tensor,
+                               groups, max_members, args.partition_size, stream)
+        elif w.num_q_tokens > 1:
+            B.pa_decode_multi(out, dw.q, dw.k_cache, dw.v_cache, dw.block_tables, dw.seq_lens, w.scale, ws.tensor,
+                              args.partition_size, stream)
+        elif fp8:
+            B.pa_decode_fp8(out, dw.q, dw.k_cache, dw.v_cache, dw.block_tables, dw.seq_lens, w.scale, w.k_scale,
+                            w.v_scale, ws.tensor, args.partition_size, stream)
+        else:
+            B.pa_decode(out, dw.q, dw.k_cache, dw.v_cache, dw.block_tables, dw.seq_lens, w.scale, ws.tensor,
+                        args.partition_size, stream)
 
     # ---- warm-up (also checks the device error word once)
     for _ in range(max(3, args.warmup)):
@@ -338,26 +377,6 @@ def run_ours(args):
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     wall0 = time.time()
     t_start.record(stream)
-    fp8 = w.kv_dtype == "e4m3"
-
-    def store():
-        if fp8:
-            B.pa_reshape_and_cache_fp8(dw.new_k, dw.new_v, dw.k_cache, dw.v_cache, dw.slot_mapping, w.k_scale,
-                                       w.v_scale, stream=stream)
-        else:
-            B.pa_reshape_and_cache(dw.new_k, dw.new_v, dw.k_cache, dw.v_cache, dw.slot_mapping, stream=stream)
-
-    def decode():
-        if w.num_q_tokens > 1:
-            B.pa_decode_multi(out, dw.q, dw.k_cache, dw.v_cache, dw.block_tables, dw.seq_lens, w.scale, ws.tensor,
-                              args.partition_size, stream)
-        elif fp8:
-            B.pa_decode_fp8(out, dw.q, dw.k_cache, dw.v_cache, dw.block_tables, dw.seq_lens, w.scale, w.k_scale,
-                            w.v_scale, ws.tensor, args.partition_size, stream)
-        else:
-            B.pa_decode(out, dw.q, dw.k_cache, dw.v_cache, dw.block_tables, dw.seq_lens, w.scale, ws.tensor,
-                        args.partition_size, stream)
-
     for i in range(args.steps):
         if len(w.copy_pairs):
             B.pa_copy_blocks(dw.k_cache, dw.v_cache, dw.copy_pairs, stream=stream)
@@ -386,8 +405,9 @@ def run_ours(args):
     pin = lambda t: t.cpu().pin_memory()
     h_q, h_k, h_v = pin(dw.q), pin(dw.new_k), pin(dw.new_v)
     h_slots, h_bt, h_sl, h_pairs = pin(dw.slot_mapping), pin(dw.block_tables), pin(dw.seq_lens), pin(dw.copy_pairs)
+    h_groups = pin(groups)
     h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    h2d = sum(t.numel() * t.element_size() for t in (h_q, h_k, h_v, h_slots, h_bt, h_sl, h_pairs))
+    h2d = sum(t.numel() * t.element_size() for t in (h_q, h_k, h_v, h_slots, h_bt, h_sl, h_pairs, h_groups))
     d2h = h_out.numel() * h_out.element_size()
     del host
     e2e_steps = max(1, min(args.steps, 500))
@@ -400,6 +420,7 @@ def run_ours(args):
         dw.block_tables.copy_(h_bt, non_blocking=True)
         dw.seq_lens.copy_(h_sl, non_blocking=True)
         dw.copy_pairs.copy_(h_pairs, non_blocking=True)
+        groups.copy_(h_groups, non_blocking=True)
         step()
         h_out.copy_(out, non_blocking=True)
 
@@ -457,6 +478,9 @@ def run_ours(args):
                    "seq_tokens_per_step": w.total_tokens(), "new_tokens_per_step": int(len(w.slot_mapping)),
                    "cow_pairs_per_step": int(len(w.copy_pairs)), "out_dtype": out_dtype,
                    "partition_size": args.partition_size or 512,
+                   "prefix_groups": (f"{len(groups_np)} groups, {int(groups_np[:, 1].sum())} sequences, shared "
+                                     f"tokens {sorted(set(int(x) for x in groups_np[:, 2]))}, max_members "
+                                     f"{max_members}") if args.prefix else None,
                    "l2": f"inputs larger than L2 (K+V {kv_bytes / 1e9:.2f} GB vs 126 MB L2); no flush in the "
                          f"timed loop", "parallelism": f"replicas x{world}" if world > 1 else "1 GPU"},
         "seq_tokens_per_s": round(world * w.total_tokens() / (ms_step * 1e-3), 1),
@@ -466,7 +490,8 @@ def run_ours(args):
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 5)},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "traffic": recorded_traffic(profile_name(args)),
-                     "kernel": ("pa_decode_multi" if w.num_q_tokens > 1 else "pa_decode")
+                     "kernel": ("pa_decode_prefix" if args.prefix else
+                                "pa_decode_multi" if w.num_q_tokens > 1 else "pa_decode")
                                + " call (plan + partition + merge kernels)",
                      "algorithmic_bytes_per_launch": decode_bytes, "launch_ms_mean": round(dec_mean, 5),
                      "launch_ms_l2_flushed_median": round(float(np.median(flushed)), 5),

@@ -64,7 +64,10 @@ typedef enum {
   PA_DEV_BAD_SEQ_LEN = 2,  /* seq_lens[i] < 0 or > max_blocks_per_seq * block_size */
   PA_DEV_BAD_SLOT = 3,     /* slot_mapping[t] >= num_blocks * block_size */
   PA_DEV_BAD_PAIR = 4,     /* a copy_blocks pair names a block outside [0, num_blocks) */
-  PA_DEV_TIMEOUT = 5       /* a bounded wait on an asynchronous copy gave up */
+  PA_DEV_TIMEOUT = 5,      /* a bounded wait on an asynchronous copy gave up */
+  PA_DEV_BAD_PREFIX = 6    /* pa_decode_prefix: a prefix group is malformed (it is then ignored), or
+                              its members' block tables differ inside the shared tokens (their
+                              rows are NaN) */
 } pa_device_error;
 
 /* Bytes of device workspace pa_decode needs, an upper bound valid for any seq_lens whose
@@ -86,8 +89,8 @@ PA_API size_t pa_decode_workspace_size(int num_seqs, int num_q_heads, int head_d
  *                ceil(seq_lens[i] / block_size) blocks are never read
  *   seq_lens     int32 [num_seqs]; 0 gives an all-zero output row
  *   supported: head_dim 64 or 128, block_size 16 or 32, G = num_q_heads / num_kv_heads
- *   from 1 to 8.  partition_size (0 = 512) must be a multiple of block_size and at
- *   most 32 * block_size: sequences longer than one partition are split into
+ *   from 1 to 8, num_kv_heads up to 255.  partition_size (0 = 512) must be a multiple of
+ *   block_size and at most 32 * block_size: sequences longer than one partition are split into
  *   partitions whose partial softmax states are merged by a second kernel
  *   (deterministic: the split depends only on seq_lens[i]).
  *   workspace    device scratch of >= pa_decode_workspace_size(num_seqs, num_q_heads,
@@ -116,8 +119,8 @@ PA_API int pa_decode_fp8(void* out, const void* q, const void* k_cache, const vo
                          int q_dtype, int out_dtype, int partition_size, void* workspace,
                          size_t workspace_bytes, void* stream);
 
-/* Multi-token paged attention: several query tokens per sequence, causal ("详解vLLM推理引擎
- *架构", section "量化集成与部署": speculative decoding verifies N draft tokens in one pass of
+/* Multi-token paged attention: several query tokens per sequence, causal
+ * ("详解vLLM推理引擎架构", section "量化集成与部署": speculative decoding verifies N draft tokens in one pass of
  * the large model; section "Chunked Prefill": a prompt is processed in chunks interleaved
  * with decode steps).  The pages give no formula; the reading taken is the plain causal one:
  * the T = num_q_tokens query tokens of sequence i are its last T tokens, already stored in the
@@ -139,6 +142,34 @@ PA_API int pa_decode_multi(void* out, const void* q, const void* k_cache, const 
                            int block_size, float scale, int max_blocks_per_seq, int64_t num_blocks,
                            int q_dtype, int kv_dtype, int out_dtype, int partition_size, void* workspace,
                            size_t workspace_bytes, void* stream);
+
+/* pa_decode with prefix groups: sequences that share their first blocks read them once
+ * ("详解vLLM推理引擎架构", section "Copy-on-Write 与内存共享": parallel samples of one prompt
+ * share the prompt's physical blocks through refcounted block-table entries; the same page,
+ * Prefix Caching: requests with a common system prompt share its blocks).  The result is
+ * pa_decode's, up to rounding: for each group the shared tokens are attended once for the
+ * query rows of all its members (one pass over each shared block per KV head), each member's
+ * own tokens once for that member, and the partial softmax states are merged per sequence.
+ *   prefix_groups  device int32 [num_groups][3] = (first, members, shared): sequences first ..
+ *                  first + members - 1 hold the same physical blocks for their first `shared`
+ *                  tokens; groups disjoint; shared a multiple of block_size and <= every
+ *                  member's seq_lens.  A group breaking these rules (both groups of an
+ *                  overlapping pair) is ignored
+ *                  (its sequences decode alone) and PA_DEV_BAD_PREFIX is recorded; members whose
+ *                  block-table entries differ inside the shared tokens get NaN rows and the
+ *                  same error.
+ *   max_members    members one shared pass serves (larger groups are split): max_members * G
+ *                  query rows per KV head, at most 32; above 8 rows only with head_dim 128 and
+ *                  q_dtype == kv_dtype (f16 or bf16).
+ * Caches f16 or bf16; everything else, the workspace included, as pa_decode.  num_groups 0 is
+ * pa_decode. */
+PA_API int pa_decode_prefix(void* out, const void* q, const void* k_cache, const void* v_cache,
+                            const int32_t* block_tables, const int32_t* seq_lens, int num_seqs,
+                            int num_q_heads, int num_kv_heads, int head_dim, int block_size, float scale,
+                            int max_blocks_per_seq, int64_t num_blocks, int q_dtype, int kv_dtype,
+                            int out_dtype, int partition_size, const int32_t* prefix_groups,
+                            int num_groups, int max_members, void* workspace, size_t workspace_bytes,
+                            void* stream);
 
 /* Store the step's new tokens into the paged cache ("vLLM 深度解读", section 7).
  * For each token t with slot = slot_mapping[t] >= 0:

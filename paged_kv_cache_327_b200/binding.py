@@ -20,11 +20,12 @@ _LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libpa.so")
 
 PA_F32, PA_F16, PA_BF16, PA_FP8_E4M3 = 0, 1, 2, 3
 PA_OK, PA_ERR_INVALID, PA_ERR_UNSUPPORTED, PA_ERR_WORKSPACE, PA_ERR_CUDA = 0, -1, -2, -3, -4
-PA_DEV_OK, PA_DEV_BAD_BLOCK_ID, PA_DEV_BAD_SEQ_LEN, PA_DEV_BAD_SLOT, PA_DEV_BAD_PAIR, PA_DEV_TIMEOUT = range(6)
+(PA_DEV_OK, PA_DEV_BAD_BLOCK_ID, PA_DEV_BAD_SEQ_LEN, PA_DEV_BAD_SLOT, PA_DEV_BAD_PAIR, PA_DEV_TIMEOUT,
+ PA_DEV_BAD_PREFIX) = range(7)
 
 EXPORTED = ("pa_decode_workspace_size", "pa_decode", "pa_reshape_and_cache", "pa_copy_blocks",
             "pa_strerror", "pa_get_device_error", "pa_version", "pa_decode_static_workspace",
-            "pa_decode_fp8", "pa_reshape_and_cache_fp8", "pa_swap_blocks", "pa_decode_multi")
+            "pa_decode_fp8", "pa_reshape_and_cache_fp8", "pa_swap_blocks", "pa_decode_multi", "pa_decode_prefix")
 PA_ERR_TOO_LARGE = -5
 PA_DECODE_STATIC_WORKSPACE_BYTES = 64 << 20
 
@@ -70,6 +71,8 @@ def load_library(path: str = _LIB_PATH):
     lib.pa_swap_blocks.restype = I
     lib.pa_decode_multi.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, F, I, I64, I, I, I, I, P, SZ, P]
     lib.pa_decode_multi.restype = I
+    lib.pa_decode_prefix.argtypes = [P, P, P, P, P, P, I, I, I, I, I, F, I, I64, I, I, I, I, P, I, I, P, SZ, P]
+    lib.pa_decode_prefix.restype = I
     if path == _LIB_PATH:
         _lib = lib
     return lib
@@ -151,6 +154,38 @@ def pa_decode_multi(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor, v
         _TORCH_CODE[out.dtype], partition_size, _ptr(workspace), workspace.numel() * workspace.element_size(),
         _stream(stream))
     _check(rc, "pa_decode_multi")
+
+
+def pa_decode_prefix(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                     block_tables: torch.Tensor, seq_lens: torch.Tensor, scale: float, workspace: torch.Tensor,
+                     prefix_groups: torch.Tensor, max_members: int, partition_size: int = 0, stream=None) -> None:
+    """pa_decode where each prefix group's shared blocks are read once for all its members.
+
+    prefix_groups: device int32 [num_groups, 3] rows (first, members, shared tokens), e.g. from
+    block_manager.find_prefix_groups; max_members * (Hq / Hkv) <= 32 (see include/pa.h).
+    """
+    N, Hq, D = q.shape
+    NB, bs, Hkv, D2 = k_cache.shape
+    if D2 != D or tuple(out.shape) != (N, Hq, D) or v_cache.shape != k_cache.shape:
+        raise ValueError("shape mismatch between q, out and the caches")
+    for t in (out, q, k_cache, v_cache, block_tables, seq_lens, workspace, prefix_groups):
+        if not t.is_contiguous():
+            raise ValueError("tensors must be contiguous")
+    if block_tables.dtype != torch.int32 or seq_lens.dtype != torch.int32 or prefix_groups.dtype != torch.int32:
+        raise TypeError("block_tables, seq_lens and prefix_groups must be int32")
+    if prefix_groups.numel() and (prefix_groups.dim() != 2 or prefix_groups.shape[1] != 3):
+        raise ValueError("prefix_groups must be [num_groups, 3]")
+    rc = load_library().pa_decode_prefix(
+        _ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), _ptr(seq_lens), N, Hq, Hkv, D, bs,
+        ctypes.c_float(scale), block_tables.shape[1], NB, _TORCH_CODE[q.dtype], _TORCH_CODE[k_cache.dtype],
+        _TORCH_CODE[out.dtype], partition_size, _ptr(prefix_groups), prefix_groups.shape[0] if prefix_groups.numel()
+        else 0, max_members, _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(rc, "pa_decode_prefix")
+
+
+def max_prefix_members(num_q_heads: int, num_kv_heads: int) -> int:
+    """Largest max_members pa_decode_prefix takes: 32 query rows per KV head in one shared pass."""
+    return max(1, 32 // (num_q_heads // num_kv_heads))
 
 
 def pa_decode_static_workspace(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,

@@ -237,3 +237,34 @@ def swap_out(tables: Iterable[BlockTable], gpu: BlockAllocator, cpu: BlockAlloca
 def swap_in(tables: Iterable[BlockTable], cpu: BlockAllocator, gpu: BlockAllocator) -> np.ndarray:
     """Resume a swapped sequence group: its blocks move back to the GPU pool (pairs cpu -> gpu)."""
     return _move_tables(tables, cpu, gpu)
+
+
+def find_prefix_groups(block_tables: np.ndarray, seq_lens: np.ndarray, block_size: int) -> np.ndarray:
+    """Prefix groups for ``pa_decode_prefix``: runs of consecutive sequences whose tables start
+    with the same physical blocks (forks of one parent, or requests that reuse one cached prompt:
+    "详解vLLM推理引擎架构", "Copy-on-Write 与内存共享" and "Prefix Caching").
+
+    Returns int32 [num_groups, 3] rows (first, members, shared): sequences first .. first +
+    members - 1 (members >= 2) hold the same blocks for their first ``shared`` tokens, a
+    positive multiple of block_size no larger than any member's length.  A block that is
+    shared but only partly filled by some member is left out of ``shared`` (those tokens are
+    read per sequence).
+    """
+    bt = np.asarray(block_tables)
+    lens = np.asarray(seq_lens, dtype=np.int64)
+    N = len(lens)
+    rows = []
+    i = 0
+    while i < N:
+        full_i = int(lens[i]) // block_size
+        j = i + 1
+        common = full_i
+        while j < N and full_i > 0 and int(lens[j]) >= block_size and bt[j, 0] == bt[i, 0]:
+            n = min(common, int(lens[j]) // block_size)
+            same = bt[j, :n] == bt[i, :n]
+            common = n if same.all() else int(np.argmin(same))
+            j += 1
+        if j - i >= 2 and common > 0:
+            rows.append((i, j - i, common * block_size))
+        i = j
+    return np.asarray(rows, dtype=np.int32).reshape(-1, 3)

@@ -28,14 +28,24 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 int elem_bytes(int dt) { return dt == PA_F32 ? 4 : dt == PA_FP8_E4M3 ? 1 : 2; }
 
 struct WsLayout {
-  size_t counters, items, part_ml, part_acc, total;
+  size_t counters, seq_parts, seq_shared, seq_sub, items, part_ml, part_acc, total;
 };
+
+// Partitions a sequence of up to max_len tokens can produce: its own ceil(max_len / P), plus one
+// when a shared prefix ends inside a partition (shared and own tokens are partitioned apart).
+int64_t max_parts_for(int64_t max_len, int P) { return (max_len + P - 1) / P + 1; }
 
 WsLayout ws_layout(int64_t num_seqs, int64_t num_q_heads, int64_t head_dim, int64_t max_parts) {
   WsLayout L{};
   size_t o = 0;
   L.counters = o;
   o += 256;
+  L.seq_parts = o;
+  o += align256(static_cast<size_t>(num_seqs) * sizeof(int));
+  L.seq_shared = o;
+  o += align256(static_cast<size_t>(num_seqs) * sizeof(int));
+  L.seq_sub = o;
+  o += align256(static_cast<size_t>(num_seqs) * sizeof(int));
   L.items = o;
   o += align256(static_cast<size_t>(num_seqs * max_parts) * sizeof(pa::WorkItem));
   L.part_ml = o;
@@ -101,13 +111,20 @@ int encode_kv_map(CUtensorMap* map, const void* base, int kv_dtype, int64_t num_
   return r == CUDA_SUCCESS ? PA_OK : PA_ERR_CUDA;
 }
 
-template <int BS, int D, typename KT, typename QT, int NT>
+template <int BS, int D, typename KT, typename QT, int NT, bool PAIR>
 int launch_partition(const pa::DecodeParams& p, const CUtensorMap& tmk, const CUtensorMap& tmv,
                      int64_t max_items, int dev, DeviceInfo* info, cudaStream_t stream) {
-  using C = pa::DecodeCfg<BS, D, KT, QT, NT>;
-  auto kern = pa::pa_decode_partition_kernel<BS, D, KT, QT, NT>;
+  using C = pa::DecodeCfg<BS, D, KT, QT, NT, PAIR>;
+  auto kern = pa::pa_decode_partition_kernel<BS, D, KT, QT, NT, PAIR>;
   static std::atomic<bool> smem_set[kMaxDevices];  // per instantiation and device
   if (!smem_set[dev].load(std::memory_order_acquire)) {
+    if (PAIR) {
+      // the warps' setmaxnreg split must fit the registers the block is launched with, or the
+      // consumers' increase would wait for ever: never launch such a build
+      cudaFuncAttributes fa{};
+      if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return PA_ERR_CUDA;
+      if (fa.numRegs < C::REG_LAUNCH) return PA_ERR_UNSUPPORTED;
+    }
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
       return PA_ERR_CUDA;
     smem_set[dev].store(true, std::memory_order_release);
@@ -132,42 +149,41 @@ int launch_partition(const pa::DecodeParams& p, const CUtensorMap& tmk, const CU
 }
 
 // Kernel instantiation for (block_size, head_dim, KV dtype, query dtype, query rows per item):
-// items of up to 8 query rows run on every dtype pair; wider items (several query tokens, NT
-// 8-row tiles) on a 16-bit cache with a query of the same type, head_dim 128.
+// items of up to 8 query rows run on every dtype pair with one consumer warp per ring; wider
+// items (several query tokens, or the members of a shared prefix) on a 16-bit cache with a query
+// of the same type, head_dim 128, with two consumer warps per ring of 1 or 2 eight-row tiles.
 template <int BS, int D>
 int dispatch_kv(const pa::DecodeParams& p, const CUtensorMap& tmk, const CUtensorMap& tmv, int64_t max_items,
-                int dev, DeviceInfo* info, int kv_dtype, int q_dtype, cudaStream_t stream) {
+                int dev, DeviceInfo* info, int kv_dtype, int q_dtype, int cols, cudaStream_t stream) {
   const bool qf32 = q_dtype == PA_F32;
-  const int nt = (p.item_cols + 7) / 8;
+  const int nt = (cols + 7) / 8;
   if (nt > 1) {
     if constexpr (D == 128) {
       if (kv_dtype == PA_BF16 && q_dtype == PA_BF16) {
         using T = __nv_bfloat16;
-        if (nt == 2) return launch_partition<BS, D, T, T, 2>(p, tmk, tmv, max_items, dev, info, stream);
-        if (nt == 3) return launch_partition<BS, D, T, T, 3>(p, tmk, tmv, max_items, dev, info, stream);
-        return launch_partition<BS, D, T, T, 4>(p, tmk, tmv, max_items, dev, info, stream);
+        if (nt == 2) return launch_partition<BS, D, T, T, 1, true>(p, tmk, tmv, max_items, dev, info, stream);
+        return launch_partition<BS, D, T, T, 2, true>(p, tmk, tmv, max_items, dev, info, stream);
       }
       if (kv_dtype == PA_F16 && q_dtype == PA_F16) {
         using T = __half;
-        if (nt == 2) return launch_partition<BS, D, T, T, 2>(p, tmk, tmv, max_items, dev, info, stream);
-        if (nt == 3) return launch_partition<BS, D, T, T, 3>(p, tmk, tmv, max_items, dev, info, stream);
-        return launch_partition<BS, D, T, T, 4>(p, tmk, tmv, max_items, dev, info, stream);
+        if (nt == 2) return launch_partition<BS, D, T, T, 1, true>(p, tmk, tmv, max_items, dev, info, stream);
+        return launch_partition<BS, D, T, T, 2, true>(p, tmk, tmv, max_items, dev, info, stream);
       }
     }
     return PA_ERR_UNSUPPORTED;
   }
   if (kv_dtype == PA_BF16)
-    return qf32 ? launch_partition<BS, D, __nv_bfloat16, float, 1>(p, tmk, tmv, max_items, dev, info, stream)
-                : launch_partition<BS, D, __nv_bfloat16, __nv_bfloat16, 1>(p, tmk, tmv, max_items, dev, info, stream);
+    return qf32 ? launch_partition<BS, D, __nv_bfloat16, float, 1, false>(p, tmk, tmv, max_items, dev, info, stream)
+                : launch_partition<BS, D, __nv_bfloat16, __nv_bfloat16, 1, false>(p, tmk, tmv, max_items, dev, info, stream);
   if (kv_dtype == PA_F16)
-    return qf32 ? launch_partition<BS, D, __half, float, 1>(p, tmk, tmv, max_items, dev, info, stream)
-                : launch_partition<BS, D, __half, __half, 1>(p, tmk, tmv, max_items, dev, info, stream);
+    return qf32 ? launch_partition<BS, D, __half, float, 1, false>(p, tmk, tmv, max_items, dev, info, stream)
+                : launch_partition<BS, D, __half, __half, 1, false>(p, tmk, tmv, max_items, dev, info, stream);
   if constexpr (D == 128) {  // an FP8 row of head_dim 128 fills one 128-byte TMA box
     if (q_dtype == PA_F32)
-      return launch_partition<BS, D, pa::fp8e4m3, float, 1>(p, tmk, tmv, max_items, dev, info, stream);
+      return launch_partition<BS, D, pa::fp8e4m3, float, 1, false>(p, tmk, tmv, max_items, dev, info, stream);
     if (q_dtype == PA_F16)
-      return launch_partition<BS, D, pa::fp8e4m3, __half, 1>(p, tmk, tmv, max_items, dev, info, stream);
-    return launch_partition<BS, D, pa::fp8e4m3, __nv_bfloat16, 1>(p, tmk, tmv, max_items, dev, info, stream);
+      return launch_partition<BS, D, pa::fp8e4m3, __half, 1, false>(p, tmk, tmv, max_items, dev, info, stream);
+    return launch_partition<BS, D, pa::fp8e4m3, __nv_bfloat16, 1, false>(p, tmk, tmv, max_items, dev, info, stream);
   }
   return PA_ERR_UNSUPPORTED;
 }
@@ -194,33 +210,37 @@ size_t pa_decode_workspace_size(int num_seqs, int num_q_heads, int head_dim, int
                                 int partition_size) {
   if (num_seqs < 0 || num_q_heads <= 0 || head_dim <= 0 || max_seq_len < 0 || partition_size < 0) return 0;
   const int P = partition_size ? partition_size : kDefaultPartition;
-  const int64_t max_parts = std::max<int64_t>(1, (static_cast<int64_t>(max_seq_len) + P - 1) / P);
-  return ws_layout(num_seqs, num_q_heads, head_dim, max_parts).total;
+  return ws_layout(num_seqs, num_q_heads, head_dim, max_parts_for(max_seq_len, P)).total;
 }
 
 }  // extern "C"
 
 namespace {
 
-// pa_decode, pa_decode_fp8 and pa_decode_multi: kv_dtype F16 / BF16 (scales unused) or
-// FP8_E4M3; qtok query tokens per sequence (1 = decode)
+// pa_decode, pa_decode_fp8, pa_decode_multi and pa_decode_prefix: kv_dtype F16 / BF16 (scales
+// unused) or FP8_E4M3; qtok query tokens per sequence (1 = decode); num_groups prefix groups
+// (device int32 [num_groups][3]) whose shared items cover up to max_members sequences
 int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,
                 const int32_t* seq_lens, int num_seqs, int qtok, int num_q_heads, int num_kv_heads, int head_dim,
                 int block_size, float scale, float k_scale, float v_scale, int max_blocks_per_seq,
-                int64_t num_blocks, int q_dtype, int kv_dtype, int out_dtype, int partition_size, void* workspace,
-                size_t workspace_bytes, void* stream) {
+                int64_t num_blocks, int q_dtype, int kv_dtype, int out_dtype, int partition_size,
+                const int32_t* groups, int num_groups, int max_members, void* workspace, size_t workspace_bytes,
+                void* stream) {
   if (num_seqs < 0 || qtok <= 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 ||
       max_blocks_per_seq <= 0 || num_blocks <= 0 || partition_size < 0 || !std::isfinite(scale) ||
-      !std::isfinite(k_scale) || !std::isfinite(v_scale) || k_scale <= 0.f || v_scale <= 0.f)
+      !std::isfinite(k_scale) || !std::isfinite(v_scale) || k_scale <= 0.f || v_scale <= 0.f || num_groups < 0 ||
+      max_members < 1)
     return PA_ERR_INVALID;
   if (num_q_heads % num_kv_heads) return PA_ERR_INVALID;
   const int G = num_q_heads / num_kv_heads;
-  if (G > 8) return PA_ERR_UNSUPPORTED;
-  // an item holds qtok * G query rows: up to 8 on every dtype pair, up to 32 on a 16-bit
-  // cache with a query of its own type and head_dim 128
-  if (static_cast<int64_t>(qtok) * G > 32) return PA_ERR_UNSUPPORTED;
-  if (qtok * G > 8 && (head_dim != 128 || kv_dtype == PA_FP8_E4M3 || q_dtype != kv_dtype))
-    return PA_ERR_UNSUPPORTED;
+  if (G > 8 || num_kv_heads > 255) return PA_ERR_UNSUPPORTED;
+  if (num_groups == 0) max_members = 1;
+  if (max_members > 1 && qtok > 1) return PA_ERR_UNSUPPORTED;  // shared items are single-token decode
+  // an item holds qtok * G (or max_members * G) query rows: up to 8 on every dtype pair, up to
+  // 32 on a 16-bit cache with a query of its own type and head_dim 128
+  const int64_t cols = static_cast<int64_t>(qtok) * max_members * G;
+  if (cols > 32) return PA_ERR_UNSUPPORTED;
+  if (cols > 8 && (head_dim != 128 || kv_dtype == PA_FP8_E4M3 || q_dtype != kv_dtype)) return PA_ERR_UNSUPPORTED;
   if (head_dim != 64 && head_dim != 128) return PA_ERR_UNSUPPORTED;
   if (block_size != 16 && block_size != 32) return PA_ERR_UNSUPPORTED;
   if (kv_dtype == PA_FP8_E4M3) {
@@ -237,9 +257,10 @@ int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cac
   const int64_t max_len = static_cast<int64_t>(max_blocks_per_seq) * block_size;
   if (max_len > INT_MAX) return PA_ERR_INVALID;
   if (num_seqs == 0) return PA_OK;
-  if (!out || !q || !k_cache || !v_cache || !block_tables || !seq_lens) return PA_ERR_INVALID;
+  if (!out || !q || !k_cache || !v_cache || !block_tables || !seq_lens || (num_groups && !groups))
+    return PA_ERR_INVALID;
   if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache)) return PA_ERR_INVALID;
-  const int64_t max_parts = std::max<int64_t>(1, (max_len + P - 1) / P);
+  const int64_t max_parts = max_parts_for(max_len, P);
   if (max_parts > 32767) return PA_ERR_UNSUPPORTED;
   // partial results are kept per (query token, query head): the workspace of qtok * num_q_heads heads
   const WsLayout L = ws_layout(num_seqs, static_cast<int64_t>(qtok) * num_q_heads, head_dim, max_parts);
@@ -272,12 +293,17 @@ int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cac
   p.max_parts = static_cast<int>(max_parts);
   p.out_dtype = out_dtype;
   p.qtok = qtok;
-  p.item_cols = qtok * G;
+  p.groups = groups;
+  p.num_groups = num_groups;
+  p.max_members = max_members;
   const bool fp8 = kv_dtype == PA_FP8_E4M3;
   p.scale_log2 = scale * (fp8 ? k_scale : 1.f) * 1.4426950408889634f;
   p.v_scale = fp8 ? v_scale : 1.f;
   p.counters = reinterpret_cast<unsigned int*>(ws + L.counters);
   p.items = reinterpret_cast<pa::WorkItem*>(ws + L.items);
+  p.seq_parts = reinterpret_cast<int*>(ws + L.seq_parts);
+  p.seq_shared = reinterpret_cast<int*>(ws + L.seq_shared);
+  p.seq_sub = reinterpret_cast<int*>(ws + L.seq_sub);
   p.part_ml = reinterpret_cast<float2*>(ws + L.part_ml);
   p.part_acc = reinterpret_cast<float*>(ws + L.part_acc);
 
@@ -287,12 +313,13 @@ int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cac
 
   const int64_t max_items = static_cast<int64_t>(num_seqs) * max_parts * num_kv_heads;
   int rc;
+  const int c = static_cast<int>(cols);
   if (block_size == 16)
-    rc = head_dim == 128 ? dispatch_kv<16, 128>(p, tmk, tmv, max_items, dev, info, kv_dtype, q_dtype, st)
-                         : dispatch_kv<16, 64>(p, tmk, tmv, max_items, dev, info, kv_dtype, q_dtype, st);
+    rc = head_dim == 128 ? dispatch_kv<16, 128>(p, tmk, tmv, max_items, dev, info, kv_dtype, q_dtype, c, st)
+                         : dispatch_kv<16, 64>(p, tmk, tmv, max_items, dev, info, kv_dtype, q_dtype, c, st);
   else
-    rc = head_dim == 128 ? dispatch_kv<32, 128>(p, tmk, tmv, max_items, dev, info, kv_dtype, q_dtype, st)
-                         : dispatch_kv<32, 64>(p, tmk, tmv, max_items, dev, info, kv_dtype, q_dtype, st);
+    rc = head_dim == 128 ? dispatch_kv<32, 128>(p, tmk, tmv, max_items, dev, info, kv_dtype, q_dtype, c, st)
+                         : dispatch_kv<32, 64>(p, tmk, tmv, max_items, dev, info, kv_dtype, q_dtype, c, st);
   if (rc != PA_OK) return rc;
   {  // merge kernel: waits (griddepcontrol.wait) for the partition kernel's partial results
     const int64_t warps = static_cast<int64_t>(num_seqs) * qtok * num_q_heads;
@@ -322,7 +349,7 @@ int pa_decode(void* out, const void* q, const void* k_cache, const void* v_cache
   if (kv_dtype == PA_FP8_E4M3) return PA_ERR_UNSUPPORTED;  // needs its scales: pa_decode_fp8
   return decode_impl(out, q, k_cache, v_cache, block_tables, seq_lens, num_seqs, 1, num_q_heads, num_kv_heads,
                      head_dim, block_size, scale, 1.f, 1.f, max_blocks_per_seq, num_blocks, q_dtype, kv_dtype,
-                     out_dtype, partition_size, workspace, workspace_bytes, stream);
+                     out_dtype, partition_size, nullptr, 0, 1, workspace, workspace_bytes, stream);
 }
 
 int pa_decode_fp8(void* out, const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,
@@ -332,7 +359,7 @@ int pa_decode_fp8(void* out, const void* q, const void* k_cache, const void* v_c
                   size_t workspace_bytes, void* stream) {
   return decode_impl(out, q, k_cache, v_cache, block_tables, seq_lens, num_seqs, 1, num_q_heads, num_kv_heads,
                      head_dim, block_size, scale, k_scale, v_scale, max_blocks_per_seq, num_blocks, q_dtype,
-                     PA_FP8_E4M3, out_dtype, partition_size, workspace, workspace_bytes, stream);
+                     PA_FP8_E4M3, out_dtype, partition_size, nullptr, 0, 1, workspace, workspace_bytes, stream);
 }
 
 int pa_decode_multi(void* out, const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,
@@ -343,7 +370,20 @@ int pa_decode_multi(void* out, const void* q, const void* k_cache, const void* v
   if (kv_dtype == PA_FP8_E4M3) return PA_ERR_UNSUPPORTED;
   return decode_impl(out, q, k_cache, v_cache, block_tables, seq_lens, num_seqs, num_q_tokens, num_q_heads,
                      num_kv_heads, head_dim, block_size, scale, 1.f, 1.f, max_blocks_per_seq, num_blocks, q_dtype,
-                     kv_dtype, out_dtype, partition_size, workspace, workspace_bytes, stream);
+                     kv_dtype, out_dtype, partition_size, nullptr, 0, 1, workspace, workspace_bytes, stream);
+}
+
+int pa_decode_prefix(void* out, const void* q, const void* k_cache, const void* v_cache,
+                     const int32_t* block_tables, const int32_t* seq_lens, int num_seqs, int num_q_heads,
+                     int num_kv_heads, int head_dim, int block_size, float scale, int max_blocks_per_seq,
+                     int64_t num_blocks, int q_dtype, int kv_dtype, int out_dtype, int partition_size,
+                     const int32_t* prefix_groups, int num_groups, int max_members, void* workspace,
+                     size_t workspace_bytes, void* stream) {
+  if (kv_dtype == PA_FP8_E4M3) return PA_ERR_UNSUPPORTED;
+  return decode_impl(out, q, k_cache, v_cache, block_tables, seq_lens, num_seqs, 1, num_q_heads, num_kv_heads,
+                     head_dim, block_size, scale, 1.f, 1.f, max_blocks_per_seq, num_blocks, q_dtype, kv_dtype,
+                     out_dtype, partition_size, prefix_groups, num_groups, max_members, workspace,
+                     workspace_bytes, stream);
 }
 
 int pa_reshape_and_cache(const void* k, const void* v, void* k_cache, void* v_cache, const int64_t* slot_mapping,

@@ -48,6 +48,7 @@ enum : unsigned {
   DEV_BAD_SLOT = 3,
   DEV_BAD_PAIR = 4,
   DEV_TIMEOUT = 5,
+  DEV_BAD_PREFIX = 6,
 };
 
 enum : int { DT_F32 = 0, DT_F16 = 1, DT_BF16 = 2 };
@@ -63,9 +64,12 @@ constexpr uint32_t kWaitLimit = 1u << 20;
 // running maximum is raised only when a score exceeds it by more than this (log2 units)
 constexpr float kRescaleThreshold = 8.0f;
 
+// A work item: tokens [tok0, tok1) of sequence seq (and of the members - 1 sequences after it,
+// which share those tokens' blocks), for every KV head; pm = part | members << 16 | WI_DIRECT.
 struct WorkItem {
-  int seq, part, len, members;  // members: sequences seq .. seq + members - 1 share the item
+  int seq, tok0, tok1, pm;
 };
+constexpr int WI_DIRECT = 1 << 30;  // the sequence's only item: write `out`, not a partial result
 
 struct DecodeParams {
   void* out;
@@ -75,12 +79,18 @@ struct DecodeParams {
   int num_seqs, num_q_heads, num_kv_heads, group;
   int head_dim, block_size, max_blocks_per_seq, num_blocks;
   int partition_size, max_parts, out_dtype, qtok;  // qtok: query tokens per sequence (1 = decode)
-  int item_cols;     // query rows of an item: members * qtok * group
+  // prefix groups, int32 [num_groups][3] = (first sequence, members, shared tokens): sequences
+  // first .. first + members - 1 hold the same blocks for their first `shared` tokens
+  const int32_t* groups;
+  int num_groups, max_members;  // a shared item covers at most max_members sequences
   float scale_log2;  // scale * log2(e) (* k_scale for an FP8 cache)
   float v_scale;     // multiplies the output (FP8 cache); 1 otherwise
   // workspace views
-  unsigned int* counters;  // [0] next work item, [1] number of (sequence, partition) pairs
+  unsigned int* counters;  // [0] next work item, [1] number of work items
   WorkItem* items;         // [num_seqs * max_parts]
+  int* seq_parts;          // [num_seqs]: partial results of the sequence (0: written directly, or no work)
+  int* seq_shared;         // [num_seqs]: tokens shared through a valid prefix group (plan scratch)
+  int* seq_sub;            // [num_seqs]: members of the shared items this sequence leads (plan scratch)
   float2* part_ml;         // [num_seqs * max_parts * qtok * num_q_heads]: (max in log2 units, sum)
   float* part_acc;         // [num_seqs * max_parts * qtok * num_q_heads * head_dim]
 };
@@ -127,51 +137,137 @@ __device__ int block_exclusive_scan(int v, int* s_warp, int* total) {
 
 constexpr int kPlanThreads = 256;
 
+__device__ __forceinline__ int block_sum(int v, int* s_warp) {
+  int total;
+  block_exclusive_scan(v, s_warp, &total);
+  return total;
+}
+
+// Work list of one call.  Per sequence i of length L (valid: 0 <= L <= max_len and L = 0 or
+// L >= qtok) with S shared tokens (0 outside a prefix group):
+//   * shared items: a sequence that leads up to max_members members of a group gets one item
+//     per partition of tokens [0, S), covering all those members;
+//   * own items: tokens [S, L) in partitions of P tokens (full ones, then a ragged tail).
+// The partial results of sequence i are numbered shared partitions first, then its own; a
+// sequence with no shared tokens and one partition writes `out` directly.  Items are listed
+// shared first (the widest), then full partitions, then tails.
 __global__ void __launch_bounds__(kPlanThreads) pa_decode_plan_kernel(const DecodeParams p) {
   // the partition kernel may start its prologue now; it waits for this grid before
   // touching anything written here
   pdl_launch_dependents();
   __shared__ int s_warp[33];
-  const int N = p.num_seqs, P = p.partition_size;
+  const int N = p.num_seqs, P = p.partition_size, BS = p.block_size;
   const int max_len = p.max_blocks_per_seq * p.block_size;
-  int local = 0;
-  for (int i = threadIdx.x; i < N; i += blockDim.x) {
-    const int L = p.seq_lens[i];
-    if (L >= 0 && L <= max_len && (L == 0 || L >= p.qtok)) local += L / P;
+  auto valid_len = [&](int L) { return L >= 0 && L <= max_len && (L == 0 || L >= p.qtok); };
+
+  if (p.num_groups > 0) {
+    // A group is used if it is in range, its shared tokens are whole blocks that every member
+    // holds, and no other group claims any of its sequences; otherwise it is reported and its
+    // sequences decode alone.  seq_sub first counts the claims on each sequence.
+    auto well_formed = [&](int g) {
+      const int first = p.groups[3 * g], M = p.groups[3 * g + 1], S = p.groups[3 * g + 2];
+      bool ok = first >= 0 && M >= 1 && first <= N - M && S >= 0 && S % BS == 0;
+      for (int m = 0; ok && m < M; ++m) {
+        const int L = p.seq_lens[first + m];
+        ok = valid_len(L) && S <= L;
+      }
+      return ok;
+    };
+    for (int i = threadIdx.x; i < N; i += blockDim.x) p.seq_shared[i] = p.seq_sub[i] = 0;
+    __syncthreads();
+    for (int g = threadIdx.x; g < p.num_groups; g += blockDim.x) {
+      if (!well_formed(g)) {
+        record_error(DEV_BAD_PREFIX);
+        continue;
+      }
+      for (int m = 0; m < p.groups[3 * g + 1]; ++m) atomicAdd(&p.seq_sub[p.groups[3 * g] + m], 1);
+    }
+    __syncthreads();
+    for (int g = threadIdx.x; g < p.num_groups; g += blockDim.x) {
+      if (!well_formed(g)) continue;
+      const int first = p.groups[3 * g], M = p.groups[3 * g + 1], S = p.groups[3 * g + 2];
+      bool alone = true;
+      for (int m = 0; m < M; ++m) alone &= p.seq_sub[first + m] == 1;
+      if (!alone) {
+        record_error(DEV_BAD_PREFIX);
+        continue;
+      }
+      if (S > 0 && M > 1)
+        for (int m = 0; m < M; ++m) p.seq_shared[first + m] = S;
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < N; i += blockDim.x) p.seq_sub[i] = 0;
+    __syncthreads();
+    for (int g = threadIdx.x; g < p.num_groups; g += blockDim.x) {
+      if (!well_formed(g)) continue;
+      const int first = p.groups[3 * g], M = p.groups[3 * g + 1], S = p.groups[3 * g + 2];
+      if (S == 0 || M == 1 || p.seq_shared[first] != S) continue;  // unused, or lost a claim
+      for (int m = 0; m < M; m += p.max_members) p.seq_sub[first + m] = min(p.max_members, M - m);
+    }
+    __syncthreads();
   }
-  int n_full;
-  block_exclusive_scan(local, s_warp, &n_full);
-  int base_full = 0, base_tail = 0;
+
+  struct Counts {
+    int L, S, sub, ns, nf, nt, nps;
+  };
+  auto counts = [&](int i) {
+    Counts c{};
+    c.L = p.seq_lens[i];
+    if (!valid_len(c.L)) return c;
+    c.S = p.num_groups > 0 ? p.seq_shared[i] : 0;
+    c.sub = p.num_groups > 0 ? p.seq_sub[i] : 0;
+    c.nps = (c.S + P - 1) / P;
+    c.ns = c.sub > 0 ? c.nps : 0;
+    c.nf = (c.L - c.S) / P;
+    c.nt = ((c.L - c.S) % P) ? 1 : 0;
+    return c;
+  };
+
+  int loc_s = 0, loc_f = 0;
+  for (int i = threadIdx.x; i < N; i += blockDim.x) {
+    const Counts c = counts(i);
+    loc_s += c.ns;
+    loc_f += c.nf;
+  }
+  const int n_shared = block_sum(loc_s, s_warp);
+  const int n_full = block_sum(loc_f, s_warp);
+  int base_s = 0, base_f = 0, base_t = 0;
   for (int start = 0; start < N; start += blockDim.x) {
     const int i = start + threadIdx.x;
-    int L = 0, nf = 0, nt = 0;
+    Counts c{};
     if (i < N) {
-      L = p.seq_lens[i];
-      // a sequence holds its qtok query tokens: 0 < L < qtok is invalid
-      const bool valid = L >= 0 && L <= max_len && (L == 0 || L >= p.qtok);
-      if (valid) {
-        nf = L / P;
-        nt = (L % P) ? 1 : 0;
-      } else {
-        record_error(DEV_BAD_SEQ_LEN);
-      }
-      if (!valid || L == 0) {  // no work item: the row is zero (empty) or NaN (invalid)
+      c = counts(i);
+      const bool valid = valid_len(c.L);
+      if (!valid) record_error(DEV_BAD_SEQ_LEN);
+      if (!valid || c.L == 0) {  // no work item: the rows are zero (empty) or NaN (invalid)
         const float v = valid ? 0.f : CUDART_NAN_F;
         const int64_t row = static_cast<int64_t>(p.qtok) * p.num_q_heads * p.head_dim;
         for (int64_t e = 0; e < row; ++e) store_out(p.out, i * row + e, v, p.out_dtype);
       }
+      const int parts = c.nps + c.nf + c.nt;
+      const bool direct = c.S == 0 && parts == 1;
+      p.seq_parts[i] = direct ? 0 : parts;
     }
-    int tf, tt;
-    const int of = block_exclusive_scan(nf, s_warp, &tf);
-    const int ot = block_exclusive_scan(nt, s_warp, &tt);
-    for (int k = 0; k < nf; ++k) p.items[base_full + of + k] = WorkItem{i, k, L, 1};
-    if (nt) p.items[n_full + base_tail + ot] = WorkItem{i, nf, L, 1};
-    base_full += tf;
-    base_tail += tt;
+    int ts, tf, tt;
+    const int os = block_exclusive_scan(c.ns, s_warp, &ts);
+    const int of = block_exclusive_scan(c.nf, s_warp, &tf);
+    const int ot = block_exclusive_scan(c.nt, s_warp, &tt);
+    const int dflag = (c.S == 0 && c.nf + c.nt == 1) ? WI_DIRECT : 0;
+    for (int k = 0; k < c.ns; ++k)
+      p.items[base_s + os + k] = WorkItem{i, k * P, min(c.S, (k + 1) * P), k | (c.sub << 16)};
+    for (int k = 0; k < c.nf; ++k)
+      p.items[n_shared + base_f + of + k] =
+          WorkItem{i, c.S + k * P, c.S + (k + 1) * P, (c.nps + k) | (1 << 16) | dflag};
+    if (c.nt)
+      p.items[n_shared + n_full + base_t + ot] =
+          WorkItem{i, c.S + c.nf * P, c.L, (c.nps + c.nf) | (1 << 16) | dflag};
+    base_s += ts;
+    base_f += tf;
+    base_t += tt;
   }
   if (threadIdx.x == 0) {
     p.counters[0] = 0;
-    p.counters[1] = static_cast<unsigned>(n_full + base_tail);
+    p.counters[1] = static_cast<unsigned>(n_shared + n_full + base_t);
   }
 }
 
@@ -215,7 +311,10 @@ __device__ __forceinline__ uint32_t lds_u16(uint32_t addr) {
   return v;
 }
 
-template <int BS, int D, typename KT, typename QT, int NT>
+// NT: 8-column MMA tiles per consumer warp; PAIR: two consumer warps share each ring, the
+// second taking the item's query rows after the first's 8 * NT (for items of up to 32 rows:
+// twice the warps hide the latency of the longer per-page work).
+template <int BS, int D, typename KT, typename QT, int NT, bool PAIR>
 struct DecodeCfg {
   static constexpr bool FP8 = KvTraits<KT>::fp8;
   static constexpr int HALVES = D * KvTraits<KT>::bytes / 128;  // 128-byte column blocks of a row
@@ -226,11 +325,17 @@ struct DecodeCfg {
   // cache is converted to f16 once (exact for |q| in [2^-14, 65504])
   static constexpr bool QSPLIT = std::is_same<QT, float>::value;
   static constexpr bool QCONV = FP8 && !QSPLIT;
-  static constexpr int COLS = 8 * NT;                   // query rows per item (MMA N dimension)
-  static constexpr int QBUF_BYTES = ((COLS * D * QE + 1023) / 1024) * 1024;  // per consumer
+  static constexpr int CONS = PAIR ? 2 : 1;             // consumer warps per ring
+  static constexpr int COLS = 8 * NT * CONS;            // query rows per item (MMA N dimension)
+  static constexpr int QBUF_BYTES = ((COLS * D * QE + 1023) / 1024) * 1024;  // per ring
   static constexpr int SLOT_BYTES = 2 * PAGE_BYTES;     // K page then V page
-  static constexpr int NC = 4;                          // consumer warps (one producer each)
-  static constexpr int NWARP = 2 * NC;
+  static constexpr int NC = 4;                          // rings, one producer warp each
+  static constexpr int NCONS = NC * CONS;               // consumer warps: ring = warp % NC
+  static constexpr int NWARP = NCONS + NC;
+  // registers per thread: at launch (65536 / threads), and after setmaxnreg in a paired kernel
+  static constexpr int REG_LAUNCH = PAIR ? 168 : 255, REG_PRODUCER = 56, REG_CONSUMER = 224;
+  static_assert(!PAIR || NC * 32 * REG_PRODUCER + NCONS * 32 * REG_CONSUMER <= NWARP * 32 * REG_LAUNCH,
+                "register split exceeds the launch allocation");
   static constexpr int SMEM_BUDGET = 200 * 1024;
   static constexpr int NSLOT_FIT = (SMEM_BUDGET / NC - QBUF_BYTES) / SLOT_BYTES;
   static constexpr int NSLOT = NSLOT_FIT > 8 ? 8 : (NSLOT_FIT < 2 ? 2 : NSLOT_FIT);
@@ -243,7 +348,7 @@ struct DecodeCfg {
   static_assert(D == 64 || D == 128, "head_dim");
   static_assert(BS == 16 || BS == 32, "block_size");
   static_assert(HALVES >= 1, "an FP8 row must fill a 128-byte box (head_dim 128)");
-  static_assert(NT == 1 || (!FP8 && !QSPLIT), "wide items: 16-bit cache and query");
+  static_assert((NT == 1 && !PAIR) || (!FP8 && !QSPLIT), "wide items: 16-bit cache and query");
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
 };
 
@@ -254,26 +359,27 @@ __device__ __forceinline__ uint32_t swz(int t, int d0) {
   return (d0 >> 6) * BOX_BYTES + t * 128 + ((((d0 & 63) >> 3) ^ (t & 7)) << 4);
 }
 
-// slot metadata: x = seq, y = part | page << 16, z = kvh | ntok << 16 | flags << 24, w = len
-constexpr int F_FIRST = 1, F_LAST = 2, F_BAD = 4, F_END = 8;
+// slot metadata: x = seq, y = part | page << 16, z = kvh | ntok << 8 | members << 16 | flags << 24,
+// w = position of the page's first token relative to the first query token (len - qtok)
+constexpr int F_FIRST = 1, F_LAST = 2, F_BAD = 4, F_END = 8, F_DIRECT = 16;
 
 // The query rows ("columns") of one work item are (member m, query token t, head g) for
 // m < members, t < qtok, g < G, in that order: column c = (m * qtok + t) * G + g.  A plain decode
 // has one member and one query token; multi-token attention has qtok > 1 (query token t sits at
 // position len - qtok + t and attends causally); a shared-prefix item has members > 1 (the
 // sequences seq .. seq + members - 1 share the item's tokens).
-template <int BS, int D, typename KT, typename QT, int NT>
-__global__ void __launch_bounds__(DecodeCfg<BS, D, KT, QT, NT>::NWARP * 32, 1)
+template <int BS, int D, typename KT, typename QT, int NT, bool PAIR>
+__global__ void __launch_bounds__(DecodeCfg<BS, D, KT, QT, NT, PAIR>::NWARP * 32, 1)
     pa_decode_partition_kernel(const __grid_constant__ CUtensorMap tmk,
                                const __grid_constant__ CUtensorMap tmv, const DecodeParams p) {
-  using C = DecodeCfg<BS, D, KT, QT, NT>;
+  using C = DecodeCfg<BS, D, KT, QT, NT, PAIR>;
   using MA = typename KvTraits<KT>::mma_t;  // element type of the tensor-core operands
   constexpr unsigned FULL = 0xffffffffu;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int c = warp % C::NC;  // consumer index of this warp's pair
+  const int c = warp % C::NC;  // ring of this warp (its consumers and producer share a scheduler)
   uint8_t* ring = smem + c * (C::NSLOT * C::SLOT_BYTES + C::QBUF_BYTES);
   uint8_t* qbuf = ring + C::NSLOT * C::SLOT_BYTES;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::RING_BYTES) + c * (2 * C::NSLOT + 2);
@@ -286,7 +392,8 @@ __global__ void __launch_bounds__(DecodeCfg<BS, D, KT, QT, NT>::NWARP * 32, 1)
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::NC; ++i) {
       uint64_t* b = reinterpret_cast<uint64_t*>(smem + C::RING_BYTES) + i * (2 * C::NSLOT + 2);
-      for (int s = 0; s < 2 * C::NSLOT + 1; ++s) mbar_init(&b[s], 1);
+      // full: the producer's arrival (+ bytes); empty and qfree: one arrival per consumer warp
+      for (int s = 0; s < 2 * C::NSLOT + 1; ++s) mbar_init(&b[s], s < C::NSLOT ? 1 : C::CONS);
       flags_base[4 * i] = 0;
     }
     fence_mbar_init();
@@ -298,8 +405,9 @@ __global__ void __launch_bounds__(DecodeCfg<BS, D, KT, QT, NT>::NWARP * 32, 1)
 
   const int G = p.group, Hkv = p.num_kv_heads, Hq = p.num_q_heads, T = p.qtok;
 
-  if (warp >= C::NC) {
+  if (warp >= C::NCONS) {
     // ============================== producer ==============================
+    if constexpr (PAIR) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(C::REG_PRODUCER));
     const unsigned total = p.counters[1] * static_cast<unsigned>(Hkv);
     const uint64_t pol = policy_evict_first();
     uint32_t n = 0;      // pages issued into this ring
@@ -317,18 +425,29 @@ __global__ void __launch_bounds__(DecodeCfg<BS, D, KT, QT, NT>::NWARP * 32, 1)
       if (w >= total) break;
       const WorkItem it = p.items[w / Hkv];
       const int kvh = static_cast<int>(w % Hkv);
-      const int tok0 = it.part * p.partition_size;
-      const int tok1 = min(it.len, tok0 + p.partition_size);
+      const int part = it.pm & 0xffff, members = (it.pm >> 16) & 0xff;
+      const int tok0 = it.tok0, tok1 = it.tok1;
       const int npages = (tok1 - tok0 + BS - 1) / BS;
-      const int rows = it.members * T;  // (member, query token) pairs of the item: G query rows each
+      const int rows = members * T;  // (member, query token) pairs of the item: G query rows each
+      // key positions relative to the first query token (causal masking of several query tokens)
+      const int rel0 = T > 1 ? tok0 - (p.seq_lens[it.seq] - T) : 0;
       int bt = 0;
-      bool bad = false;
+      bool bad = false, mismatch = false;
       if (lane < npages) {
-        bt = p.block_tables[static_cast<int64_t>(it.seq) * p.max_blocks_per_seq + tok0 / BS + lane];
+        const int64_t col = tok0 / BS + lane;
+        bt = p.block_tables[static_cast<int64_t>(it.seq) * p.max_blocks_per_seq + col];
         bad = bt < 0 || bt >= p.num_blocks;
+        // the members of a shared item must hold the same blocks
+        for (int m = 1; m < members; ++m)
+          mismatch |= p.block_tables[static_cast<int64_t>(it.seq + m) * p.max_blocks_per_seq + col] != bt;
       }
       bad = __any_sync(FULL, bad);
-      if (bad && lane == 0) record_error(DEV_BAD_BLOCK_ID);
+      mismatch = __any_sync(FULL, mismatch);
+      if (lane == 0) {
+        if (bad) record_error(DEV_BAD_BLOCK_ID);
+        if (mismatch) record_error(DEV_BAD_PREFIX);
+      }
+      bad |= mismatch;
       if (items >= 1) {  // the consumer has taken the previous item's query rows
         const bool ok = mbar_wait_bounded(qfree, (items - 1) & 1u, kWaitLimit);
         if (!__all_sync(FULL, ok) || *abort_flag) {
@@ -347,8 +466,10 @@ __global__ void __launch_bounds__(DecodeCfg<BS, D, KT, QT, NT>::NWARP * 32, 1)
         if (lane == 0) {
           uint8_t* sb = ring + slot * C::SLOT_BYTES;
           const int ntok = min(BS, tok1 - (tok0 + pg * BS));
-          const int flags = (first ? F_FIRST : 0) | (pg == npages - 1 ? F_LAST : 0) | (bad ? F_BAD : 0);
-          meta[slot] = make_int4(it.seq, it.part | (pg << 16), kvh | (ntok << 16) | (flags << 24), it.len);
+          const int flags = (first ? F_FIRST : 0) | (pg == npages - 1 ? F_LAST : 0) | (bad ? F_BAD : 0) |
+                            ((it.pm & WI_DIRECT) ? F_DIRECT : 0);
+          meta[slot] = make_int4(it.seq, part | (pg << 16), kvh | (ntok << 8) | (members << 16) | (flags << 24),
+                                 rel0 + pg * BS);
           if (bad) {
             mbar_arrive(&full[slot]);
           } else {
@@ -397,6 +518,8 @@ __global__ void __launch_bounds__(DecodeCfg<BS, D, KT, QT, NT>::NWARP * 32, 1)
   }
 
   // ============================== consumer ==============================
+  if constexpr (PAIR) asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(C::REG_CONSUMER));
+  const int col0 = (warp / C::NC) * NT * 8;  // first query row (column) of this consumer
   const int lr = lane & 7, lm = lane >> 3;  // ldmatrix: row inside an 8x8 matrix, matrix index
   const int r0 = lane >> 2, c2 = (lane & 3) * 2;
   // per-lane swizzled offsets of the ldmatrix rows (the same in every slot and 16-row tile).
@@ -438,10 +561,10 @@ __global__ void __launch_bounds__(DecodeCfg<BS, D, KT, QT, NT>::NWARP * 32, 1)
 #pragma unroll
         for (int k2 = 0; k2 < C::KS; k2 += 2) {
           const int d0 = (k2 + (lm >> 1)) * 16 + ((lm & 1) << 3);
-          ldsm_x4(smem_u32(qbuf + ((nt * 8 + lr) * D + d0) * 2), qf[k2][nt][0], qf[k2][nt][1], qf[k2 + 1][nt][0],
-                  qf[k2 + 1][nt][1]);
+          ldsm_x4(smem_u32(qbuf + ((col0 + nt * 8 + lr) * D + d0) * 2), qf[k2][nt][0], qf[k2][nt][1],
+                  qf[k2 + 1][nt][0], qf[k2 + 1][nt][1]);
         }
-        if (nt * 8 + r0 >= ncol) {
+        if (col0 + nt * 8 + r0 >= ncol) {
 #pragma unroll
           for (int k = 0; k < C::KS; ++k) qf[k][nt][0] = qf[k][nt][1] = 0u;
         }
@@ -472,9 +595,15 @@ __global__ void __launch_bounds__(DecodeCfg<BS, D, KT, QT, NT>::NWARP * 32, 1)
   // One page: S^T = K . Q^T, online-softmax update, O^T += V^T . P^T.  The softmax state is
   // updated once per chunk of MC 16-token tiles: the whole page for items of up to 16 query
   // rows, each tile on its own for wider items (their scores would not fit in registers).
-  auto page_math = [&](const uint8_t* sb, int ntok, int kpos0, int len) {
+  // na: the number NA of 8-column tiles that hold the current item's query rows (NT, or 1 for an
+  // item of at most 8 rows -- items of one call differ in width when shared items cover several
+  // sequences); the tiles past NA are skipped.  The choice is made once per page, so the tile
+  // loops stay unrolled and branch-free.
+  auto page_math = [&](const uint8_t* sb, int ntok, int rel, auto na) {
+    constexpr int NA = decltype(na)::value;
+    auto on = [](int nt) { return nt < NA; };
     const uint32_t kb = smem_u32(sb), vb = kb + C::PAGE_BYTES;
-    constexpr int MC = NT > 2 ? 1 : C::MT;
+    constexpr int MC = NA > 1 ? 1 : C::MT;
 #pragma unroll
     for (int m0 = 0; m0 < C::MT; m0 += MC) {
       float s[MC][NT][4];
@@ -508,6 +637,7 @@ __global__ void __launch_bounds__(DecodeCfg<BS, D, KT, QT, NT>::NWARP * 32, 1)
             ldsm_x4(kb + mt * 2048 + koff(kk), a0, a1, a2, a3);
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
+              if (!on(nt)) continue;
               if constexpr (C::QSPLIT) {
                 Mma<MA>::run(sa[nt], a0, a1, a2, a3, qf[kk][nt][0], qf[kk][nt][1]);
                 Mma<MA>::run(sb2[nt], a0, a1, a2, a3, ql[kk][0], ql[kk][1]);
@@ -533,17 +663,18 @@ __global__ void __launch_bounds__(DecodeCfg<BS, D, KT, QT, NT>::NWARP * 32, 1)
             for (int h = 0; h < 2; ++h)
               if ((m0 + mi) * 16 + r0 + 8 * h >= ntok) s[mi][nt][2 * h] = s[mi][nt][2 * h + 1] = -CUDART_INF_F;
       }
-      if (T > 1 && kpos0 + BS > len - T) {
-        // causal: query token t (position len - T + t) sees keys up to its own position
+      if (T > 1 && rel + BS > 1) {
+        // causal: query token t sees keys up to its own position (rel: the page's first key
+        // relative to query token 0)
 #pragma unroll
         for (int mi = 0; mi < MC; ++mi)
 #pragma unroll
           for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-              const int col = nt * 8 + c2 + (e & 1);
+              const int col = col0 + nt * 8 + c2 + (e & 1);
               const int t = (col / G) % T;
-              if (kpos0 + (m0 + mi) * 16 + r0 + 8 * (e >> 1) > len - T + t) s[mi][nt][e] = -CUDART_INF_F;
+              if (rel + (m0 + mi) * 16 + r0 + 8 * (e >> 1) > t) s[mi][nt][e] = -CUDART_INF_F;
             }
       }
       // raw (unscaled) maxima of this lane's entries; scale > 0 commutes with max
@@ -557,11 +688,13 @@ __global__ void __launch_bounds__(DecodeCfg<BS, D, KT, QT, NT>::NWARP * 32, 1)
           x[nt][0] = fmaxf(x[nt][0], fmaxf(s[mi][nt][0], s[mi][nt][2]));
           x[nt][1] = fmaxf(x[nt][1], fmaxf(s[mi][nt][1], s[mi][nt][3]));
         }
-        raise |= x[nt][0] * sl > mu[nt][0] + kRescaleThreshold || x[nt][1] * sl > mu[nt][1] + kRescaleThreshold;
+        if (on(nt))
+          raise |= x[nt][0] * sl > mu[nt][0] + kRescaleThreshold || x[nt][1] * sl > mu[nt][1] + kRescaleThreshold;
       }
       if (__any_sync(FULL, raise)) {
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
+          if (!on(nt)) continue;
 #pragma unroll
           for (int o = 4; o < 32; o <<= 1) {
             x[nt][0] = fmaxf(x[nt][0], __shfl_xor_sync(FULL, x[nt][0], o));
@@ -592,6 +725,8 @@ __global__ void __launch_bounds__(DecodeCfg<BS, D, KT, QT, NT>::NWARP * 32, 1)
         uint32_t b0[NT], b1[NT];
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
+          b0[nt] = b1[nt] = 0u;
+          if (!on(nt)) continue;
           // a column with no visible key yet (mu = -inf) gets weight 0, not 2^(-inf + inf)
           const float u0 = mu[nt][0] == -CUDART_INF_F ? 0.f : mu[nt][0];
           const float u1 = mu[nt][1] == -CUDART_INF_F ? 0.f : mu[nt][1];
@@ -641,7 +776,8 @@ __global__ void __launch_bounds__(DecodeCfg<BS, D, KT, QT, NT>::NWARP * 32, 1)
             uint32_t a0, a1, a2, a3;
             ldsm_x4_t(vb + mt * 2048 + voff(dt), a0, a1, a2, a3);
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt) Mma<MA>::run(acc[dt][nt], a0, a1, a2, a3, b0[nt], b1[nt]);
+            for (int nt = 0; nt < NT; ++nt)
+              if (on(nt)) Mma<MA>::run(acc[dt][nt], a0, a1, a2, a3, b0[nt], b1[nt]);
           }
         } else {
           // V rows past the end may hold anything (even NaN): zero them, 0 * NaN would poison
@@ -654,7 +790,7 @@ __global__ void __launch_bounds__(DecodeCfg<BS, D, KT, QT, NT>::NWARP * 32, 1)
             ldsm_x4_t(vb + mt * 2048 + voff(dt), a0, a1, a2, a3);
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt)
-              Mma<MA>::run(acc[dt][nt], a0 & mlo, a1 & mlo, a2 & mhi, a3 & mhi, b0[nt], b1[nt]);
+              if (on(nt)) Mma<MA>::run(acc[dt][nt], a0 & mlo, a1 & mlo, a2 & mhi, a3 & mhi, b0[nt], b1[nt]);
           }
         }
       }
@@ -664,7 +800,7 @@ __global__ void __launch_bounds__(DecodeCfg<BS, D, KT, QT, NT>::NWARP * 32, 1)
   // Write the item's result.  Column col = (m * T + t) * G + g is query head kvh * G + g of
   // query token t of sequence seq + m; its "virtual head" (T query tokens x Hq heads) is
   // t * Hq + kvh * G + g.
-  auto finalize = [&](int seq, int part, int kvh, int np) {
+  auto finalize = [&](int seq, int part, int kvh, bool direct) {
     const float nan = CUDART_NAN_F;
     // accumulator rows r0 and r0 + 8 of tile dt are columns d and d + dd
     const int dd = C::FP8 ? 1 : 8;
@@ -674,13 +810,13 @@ __global__ void __launch_bounds__(DecodeCfg<BS, D, KT, QT, NT>::NWARP * 32, 1)
     for (int nt = 0; nt < NT; ++nt) {
 #pragma unroll
       for (int j = 0; j < 2; ++j) {
-        const int col = nt * 8 + c2 + j;
+        const int col = col0 + nt * 8 + c2 + j;
         if (col >= ncol) continue;
         const int g = col % G, mt_ = col / G;
         const int m = mt_ / T, t = mt_ - m * T;
         const int vh = t * Hq + kvh * G + g;
         const float l = lacc[nt][j];  // every row of the ones-MMA holds the column sums
-        if (np == 1) {
+        if (direct) {
           const float inv = poisoned ? nan : vs / l;
           const int64_t o = (static_cast<int64_t>(seq + m) * HV + vh) * D;
 #pragma unroll
@@ -716,9 +852,9 @@ __global__ void __launch_bounds__(DecodeCfg<BS, D, KT, QT, NT>::NWARP * 32, 1)
       break;
     }
     const int4 mt = meta[slot];
-    const int kvh = mt.z & 0xffff, ntok = (mt.z >> 16) & 0xff, flags = (mt.z >> 24) & 0xff;
+    const int kvh = mt.z & 0xff, ntok = (mt.z >> 8) & 0xff, flags = (mt.z >> 24) & 0xff;
     if (flags & F_END) break;
-    const int part = mt.y & 0xffff, pg = mt.y >> 16, len = mt.w;
+    const int part = mt.y & 0xffff;
     const uint8_t* sb = ring + slot * C::SLOT_BYTES;
     if (flags & F_FIRST) {
 #pragma unroll
@@ -729,15 +865,21 @@ __global__ void __launch_bounds__(DecodeCfg<BS, D, KT, QT, NT>::NWARP * 32, 1)
         for (int dt = 0; dt < C::KS; ++dt) acc[dt][nt][0] = acc[dt][nt][1] = acc[dt][nt][2] = acc[dt][nt][3] = 0.f;
       }
       poisoned = (flags & F_BAD) != 0;
-      ncol = p.item_cols;  // the same for every item of a call
+      ncol = ((mt.z >> 16) & 0xff) * T * G;  // members x query tokens x grouped heads
       if (!poisoned) load_q();
       __syncwarp();
       if (lane == 0) mbar_arrive(qfree);  // the query buffer may take the next item's rows
     }
-    if (!poisoned) page_math(sb, ntok, part * p.partition_size + pg * BS, len);
+    const int mycols = ncol - col0;  // query rows of the item in this consumer's tiles
+    if (!poisoned && mycols > 0) {
+      if (NT > 1 && mycols <= 8)
+        page_math(sb, ntok, mt.w, std::integral_constant<int, 1>{});
+      else
+        page_math(sb, ntok, mt.w, std::integral_constant<int, NT>{});
+    }
     __syncwarp();  // every lane is done reading the slot before it is handed back
     if (lane == 0) mbar_arrive(&empty[slot]);
-    if (flags & F_LAST) finalize(mt.x, part, kvh, (len + p.partition_size - 1) / p.partition_size);
+    if (flags & F_LAST) finalize(mt.x, part, kvh, (flags & F_DIRECT) != 0);
     ++n;
   }
   if (!ok && lane == 0) {
@@ -747,20 +889,19 @@ __global__ void __launch_bounds__(DecodeCfg<BS, D, KT, QT, NT>::NWARP * 32, 1)
 }
 
 // ------------------------------------------------------------------------------ merge
-// One warp per (sequence, virtual head = query token x query head) of a sequence with more
-// than one partition:
+// One warp per (sequence, virtual head = query token x query head) of a sequence whose items
+// wrote partial results (shared partitions first, then its own):
 // out = sum_k 2^(m_k - M) O_k / sum_k 2^(m_k - M) l_k, M = max_k m_k, partitions in order.
 constexpr int kMergeWarps = 8;
 __global__ void __launch_bounds__(kMergeWarps * 32) pa_decode_merge_kernel(const DecodeParams p) {
   pdl_wait();  // the partition kernel's partial results are visible from here on
   const int lane = threadIdx.x & 31;
   const int64_t pair = static_cast<int64_t>(blockIdx.x) * kMergeWarps + (threadIdx.x >> 5);
-  const int Hq = p.qtok * p.num_q_heads, D = p.head_dim, P = p.partition_size;
+  const int Hq = p.qtok * p.num_q_heads, D = p.head_dim;
   if (pair >= static_cast<int64_t>(p.num_seqs) * Hq) return;
   const int seq = static_cast<int>(pair / Hq), hq = static_cast<int>(pair % Hq);
-  const int L = p.seq_lens[seq];
-  if (L <= P || L > p.max_blocks_per_seq * p.block_size) return;  // direct, empty or invalid rows
-  const int np = (L + P - 1) / P;
+  const int np = p.seq_parts[seq];
+  if (np == 0) return;  // written directly, or empty / invalid
   const int64_t base = static_cast<int64_t>(seq) * p.max_parts;
   float M = -CUDART_INF_F;
   for (int k = lane; k < np; k += 32) M = fmaxf(M, __ldcg(&p.part_ml[(base + k) * Hq + hq].x));

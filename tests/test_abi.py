@@ -131,3 +131,31 @@ def test_multi_argument_validation(lib):
     assert need > B.pa_decode_workspace_size(4, 8, 128, 8 * 16)
     assert multi_call(lib, wsb=need - 1) == B.PA_ERR_WORKSPACE
     assert multi_call(lib, ws=FAKE + 16, wsb=need) == B.PA_ERR_INVALID  # passes the size check, not 256-aligned
+
+
+def prefix_call(lib, **kw):
+    a = dict(out=FAKE, q=FAKE, k=FAKE, v=FAKE, bt=FAKE, sl=FAKE, N=4, Hq=16, Hkv=2, D=128, bs=16, scale=0.1,
+             MB=8, NB=64, qd=2, kd=2, od=0, P=0, groups=FAKE, ng=1, mm=4, ws=FAKE, wsb=0, stream=0)
+    a.update(kw)
+    V = ctypes.c_void_p
+    return lib.pa_decode_prefix(V(a["out"]), V(a["q"]), V(a["k"]), V(a["v"]), V(a["bt"]), V(a["sl"]), a["N"],
+                                a["Hq"], a["Hkv"], a["D"], a["bs"], ctypes.c_float(a["scale"]), a["MB"], a["NB"],
+                                a["qd"], a["kd"], a["od"], a["P"], V(a["groups"]), a["ng"], a["mm"], V(a["ws"]),
+                                a["wsb"], V(a["stream"]))
+
+
+def test_prefix_argument_validation(lib):
+    assert prefix_call(lib, N=0) == B.PA_OK
+    assert prefix_call(lib, ng=-1) == B.PA_ERR_INVALID
+    assert prefix_call(lib, mm=0) == B.PA_ERR_INVALID
+    assert prefix_call(lib, groups=0) == B.PA_ERR_INVALID          # groups promised, none given
+    assert prefix_call(lib, mm=5) == B.PA_ERR_UNSUPPORTED           # 5 members x 8 heads > 32 rows
+    assert prefix_call(lib, kd=3) == B.PA_ERR_UNSUPPORTED           # FP8 cache
+    assert prefix_call(lib, qd=0) == B.PA_ERR_UNSUPPORTED           # 32 rows need q_dtype == kv_dtype
+    assert prefix_call(lib, Hq=512, Hkv=256) == B.PA_ERR_UNSUPPORTED  # more than 255 KV heads
+    assert prefix_call(lib, mm=1, qd=0) == B.PA_ERR_WORKSPACE       # 8 rows: any dtype pair
+    assert prefix_call(lib, ng=0, mm=99, qd=0) == B.PA_ERR_WORKSPACE  # no groups: max_members unused
+    need = B.pa_decode_workspace_size(4, 16, 128, 8 * 16)
+    assert prefix_call(lib, wsb=need - 1) == B.PA_ERR_WORKSPACE
+    assert prefix_call(lib, ws=FAKE + 16, wsb=need) == B.PA_ERR_INVALID
+    assert B.max_prefix_members(64, 8) == 4 and B.max_prefix_members(32, 8) == 8 and B.max_prefix_members(8, 8) == 32

@@ -7,6 +7,7 @@ block whose refcount exceeds 1, then drops one reference from it ("详解vLLM推
 """
 import numpy as np
 import pytest
+from paged_kv_cache_327_b200 import block_manager as BM
 
 from paged_kv_cache_327_b200 import workload as W
 from paged_kv_cache_327_b200.block_manager import (BlockAllocator, BlockTable, NoFreeBlocksError,
@@ -191,3 +192,58 @@ def test_swap_out_and_in_move_groups_and_keep_sharing():
     assert len(back) == 4 and cpu.get_num_free_blocks() == 8
     assert gpu.get_refcount(parent.get_block_number(0)) == 2
     assert parent.get_block_number(0) == child.get_block_number(0)
+
+
+# ---------------------------------------------------------------------------------------------
+# prefix groups (input of pa_decode_prefix)
+# ---------------------------------------------------------------------------------------------
+def test_prefix_groups_of_the_70b_batch():
+    from paged_kv_cache_327_b200 import workload as W
+    w = W.make_config("70b")
+    g = BM.find_prefix_groups(w.block_tables, w.seq_lens, w.block_size)
+    # 64 parents of 4096 + r tokens (r < 16) forked into 4 samples; the partial block is
+    # copied on write, so exactly the 256 full blocks are shared; the long sequences stand alone
+    assert g.shape == (64, 3)
+    assert np.array_equal(g[:, 0], np.arange(0, 256, 4)) and np.all(g[:, 1] == 4) and np.all(g[:, 2] == 4096)
+    for first, m, S in g:
+        nb = S // w.block_size
+        for k in range(1, m):
+            assert np.array_equal(w.block_tables[first + k, :nb], w.block_tables[first, :nb])
+        # the next block is no longer shared by all members
+        assert len({int(w.block_tables[first + k, nb]) for k in range(m)}) > 1
+
+
+def test_prefix_groups_edge_cases():
+    bs = 16
+    bt = np.array([[7, 8, 9, -1],      # 0: leader
+                   [7, 8, 3, -1],      # 1: shares 2 blocks with 0
+                   [7, 8, 9, 4],       # 2: shares 3 with 0, but the run's common part is 2 blocks
+                   [5, 6, -1, -1],     # 3: alone
+                   [1, 2, -1, -1],     # 4: shares block 1 only partly filled by 5
+                   [1, 2, -1, -1],     # 5
+                   [10, -1, -1, -1],   # 6: shares a block 7 does not fill
+                   [10, -1, -1, -1],   # 7
+                   [11, 12, -1, -1],   # 8: same table as 9 but not next to it in order
+                   [13, -1, -1, -1],   # 9
+                   [11, 12, -1, -1]],  # 10
+                  np.int32)
+    lens = np.array([40, 40, 60, 20, 32, 20, 16, 10, 30, 5, 30], np.int32)
+    g = BM.find_prefix_groups(bt, lens, bs)
+    assert g.tolist() == [[0, 3, 32], [4, 2, 16]]
+
+
+def test_prefix_groups_of_forks_built_by_the_allocator():
+    bs = 16
+    alloc = BM.BlockAllocator(64, bs, seed=4)
+    parent = BM.BlockTable(bs)
+    parent.append_tokens(40, alloc)           # 2 full blocks + 8 tokens
+    kids = []
+    for _ in range(3):
+        k = BM.BlockTable(bs)
+        k.fork_from(parent, alloc)
+        kids.append(k)
+    for t in [parent] + kids:
+        t.append_tokens(5, alloc)             # copy-on-write of the partial third block
+    tables = [parent] + kids
+    g = BM.find_prefix_groups(BM.tables_to_array(tables), np.array([t.num_tokens for t in tables]), bs)
+    assert g.tolist() == [[0, 4, 32]]
