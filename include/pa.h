@@ -70,10 +70,11 @@ typedef enum {
                               rows are NaN) */
 } pa_device_error;
 
-/* Bytes of device workspace pa_decode needs, an upper bound valid for any seq_lens whose
- * entries are all <= max_seq_len.  pa_decode itself requires the bound for
- * max_seq_len = max_blocks_per_seq * block_size.  partition_size 0 means the default (512).
- * Returns 0 for invalid arguments. */
+/* Bytes of device workspace the decode entry points need: an upper bound valid for any seq_lens
+ * whose entries are all <= max_seq_len, with or without prefix groups.  A call is always
+ * accepted with the bound for max_seq_len = max_blocks_per_seq * block_size (pa_decode_multi:
+ * num_q_heads = num_q_tokens * the query heads); plain decode may need less.  partition_size 0
+ * means the default (512).  Returns 0 for invalid arguments. */
 PA_API size_t pa_decode_workspace_size(int num_seqs, int num_q_heads, int head_dim, int max_seq_len,
                                 int partition_size);
 
@@ -132,8 +133,9 @@ PA_API int pa_decode_fp8(void* out, const void* q, const void* k_cache, const vo
  *   q    [num_seqs, num_q_tokens, num_q_heads, head_dim], q_dtype
  *   seq_lens[i] = 0 gives all-zero rows; 0 < seq_lens[i] < num_q_tokens is invalid (its rows
  *   are NaN and pa_get_device_error reports PA_DEV_BAD_SEQ_LEN).
- *   supported: num_q_tokens * G <= 8 on every dtype pair pa_decode takes; up to 32 with
- *   head_dim 128 and q_dtype == kv_dtype (f16 or bf16).  Everything else as pa_decode; the
+ *   supported: q_dtype == kv_dtype (f16 or bf16); num_q_tokens * G <= 8 with head_dim 64 or
+ *   128, up to 32 with head_dim 128 (num_q_tokens 1: every dtype pair of pa_decode).
+ *   Everything else as pa_decode; the
  *   workspace is pa_decode_workspace_size(num_seqs, num_q_tokens * num_q_heads, head_dim,
  *   max_blocks_per_seq * block_size, partition_size).  num_q_tokens 1 is pa_decode. */
 PA_API int pa_decode_multi(void* out, const void* q, const void* k_cache, const void* v_cache,

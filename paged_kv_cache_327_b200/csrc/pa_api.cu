@@ -11,6 +11,7 @@
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <type_traits>
 #include <unordered_set>
 
 #include "pa.h"
@@ -32,8 +33,11 @@ struct WsLayout {
 };
 
 // Partitions a sequence of up to max_len tokens can produce: its own ceil(max_len / P), plus one
-// when a shared prefix ends inside a partition (shared and own tokens are partitioned apart).
-int64_t max_parts_for(int64_t max_len, int P) { return (max_len + P - 1) / P + 1; }
+// with prefix groups, where a shared prefix may end inside a partition (shared and own tokens
+// are partitioned apart).  The workspace size covers both.
+int64_t max_parts_for(int64_t max_len, int P, bool groups = true) {
+  return std::max<int64_t>(1, (max_len + P - 1) / P + (groups ? 1 : 0));
+}
 
 WsLayout ws_layout(int64_t num_seqs, int64_t num_q_heads, int64_t head_dim, int64_t max_parts) {
   WsLayout L{};
@@ -111,11 +115,11 @@ int encode_kv_map(CUtensorMap* map, const void* base, int kv_dtype, int64_t num_
   return r == CUDA_SUCCESS ? PA_OK : PA_ERR_CUDA;
 }
 
-template <int BS, int D, typename KT, typename QT, int NT, bool PAIR>
+template <int BS, int D, typename KT, typename QT, int NT, bool PAIR, bool CAUSAL>
 int launch_partition(const pa::DecodeParams& p, const CUtensorMap& tmk, const CUtensorMap& tmv,
                      int64_t max_items, int dev, DeviceInfo* info, cudaStream_t stream) {
-  using C = pa::DecodeCfg<BS, D, KT, QT, NT, PAIR>;
-  auto kern = pa::pa_decode_partition_kernel<BS, D, KT, QT, NT, PAIR>;
+  using C = pa::DecodeCfg<BS, D, KT, QT, NT, PAIR, CAUSAL>;
+  auto kern = pa::pa_decode_partition_kernel<BS, D, KT, QT, NT, PAIR, CAUSAL>;
   static std::atomic<bool> smem_set[kMaxDevices];  // per instantiation and device
   if (!smem_set[dev].load(std::memory_order_acquire)) {
     if (PAIR) {
@@ -148,42 +152,52 @@ int launch_partition(const pa::DecodeParams& p, const CUtensorMap& tmk, const CU
   return cudaPeekAtLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
-// Kernel instantiation for (block_size, head_dim, KV dtype, query dtype, query rows per item):
-// items of up to 8 query rows run on every dtype pair with one consumer warp per ring; wider
-// items (several query tokens, or the members of a shared prefix) on a 16-bit cache with a query
-// of the same type, head_dim 128, with two consumer warps per ring of 1 or 2 eight-row tiles.
+// Kernel instantiation for (block_size, head_dim, KV dtype, query dtype, query rows per item,
+// several query tokens): single-token items of up to 8 query rows run on every dtype pair with one
+// consumer warp per ring; multi-token items of up to 8 rows on a 16-bit cache with a query of the
+// same type; wider items (several query tokens, or the members of a shared prefix) on a 16-bit
+// cache with a query of the same type, head_dim 128, with two consumer warps per ring of 1 or 2
+// eight-row tiles.
 template <int BS, int D>
 int dispatch_kv(const pa::DecodeParams& p, const CUtensorMap& tmk, const CUtensorMap& tmv, int64_t max_items,
                 int dev, DeviceInfo* info, int kv_dtype, int q_dtype, int cols, cudaStream_t stream) {
   const bool qf32 = q_dtype == PA_F32;
   const int nt = (cols + 7) / 8;
+  // one instantiation: KV element type K, query type Q, tiles per consumer N, paired, causal
+  auto run = [&](auto k, auto q, auto n, auto pair, auto causal) {
+    using K = decltype(k);
+    using Q = decltype(q);
+    return launch_partition<BS, D, K, Q, decltype(n)::value, decltype(pair)::value, decltype(causal)::value>(
+        p, tmk, tmv, max_items, dev, info, stream);
+  };
+  using bf16 = __nv_bfloat16;
+  using f16 = __half;
+  using One = std::integral_constant<int, 1>;
+  using Two = std::integral_constant<int, 2>;
+  using Yes = std::true_type;
+  using No = std::false_type;
+  if (nt == 1 && p.qtok > 1) {
+    if (kv_dtype == PA_BF16 && q_dtype == PA_BF16) return run(bf16{}, bf16{}, One{}, No{}, Yes{});
+    if (kv_dtype == PA_F16 && q_dtype == PA_F16) return run(f16{}, f16{}, One{}, No{}, Yes{});
+    return PA_ERR_UNSUPPORTED;
+  }
   if (nt > 1) {
     if constexpr (D == 128) {
-      if (kv_dtype == PA_BF16 && q_dtype == PA_BF16) {
-        using T = __nv_bfloat16;
-        if (nt == 2) return launch_partition<BS, D, T, T, 1, true>(p, tmk, tmv, max_items, dev, info, stream);
-        return launch_partition<BS, D, T, T, 2, true>(p, tmk, tmv, max_items, dev, info, stream);
-      }
-      if (kv_dtype == PA_F16 && q_dtype == PA_F16) {
-        using T = __half;
-        if (nt == 2) return launch_partition<BS, D, T, T, 1, true>(p, tmk, tmv, max_items, dev, info, stream);
-        return launch_partition<BS, D, T, T, 2, true>(p, tmk, tmv, max_items, dev, info, stream);
-      }
+      if (kv_dtype == PA_BF16 && q_dtype == PA_BF16)
+        return nt == 2 ? run(bf16{}, bf16{}, One{}, Yes{}, Yes{}) : run(bf16{}, bf16{}, Two{}, Yes{}, Yes{});
+      if (kv_dtype == PA_F16 && q_dtype == PA_F16)
+        return nt == 2 ? run(f16{}, f16{}, One{}, Yes{}, Yes{}) : run(f16{}, f16{}, Two{}, Yes{}, Yes{});
     }
     return PA_ERR_UNSUPPORTED;
   }
   if (kv_dtype == PA_BF16)
-    return qf32 ? launch_partition<BS, D, __nv_bfloat16, float, 1, false>(p, tmk, tmv, max_items, dev, info, stream)
-                : launch_partition<BS, D, __nv_bfloat16, __nv_bfloat16, 1, false>(p, tmk, tmv, max_items, dev, info, stream);
+    return qf32 ? run(bf16{}, float{}, One{}, No{}, No{}) : run(bf16{}, bf16{}, One{}, No{}, No{});
   if (kv_dtype == PA_F16)
-    return qf32 ? launch_partition<BS, D, __half, float, 1, false>(p, tmk, tmv, max_items, dev, info, stream)
-                : launch_partition<BS, D, __half, __half, 1, false>(p, tmk, tmv, max_items, dev, info, stream);
+    return qf32 ? run(f16{}, float{}, One{}, No{}, No{}) : run(f16{}, f16{}, One{}, No{}, No{});
   if constexpr (D == 128) {  // an FP8 row of head_dim 128 fills one 128-byte TMA box
-    if (q_dtype == PA_F32)
-      return launch_partition<BS, D, pa::fp8e4m3, float, 1, false>(p, tmk, tmv, max_items, dev, info, stream);
-    if (q_dtype == PA_F16)
-      return launch_partition<BS, D, pa::fp8e4m3, __half, 1, false>(p, tmk, tmv, max_items, dev, info, stream);
-    return launch_partition<BS, D, pa::fp8e4m3, __nv_bfloat16, 1, false>(p, tmk, tmv, max_items, dev, info, stream);
+    if (q_dtype == PA_F32) return run(pa::fp8e4m3{}, float{}, One{}, No{}, No{});
+    if (q_dtype == PA_F16) return run(pa::fp8e4m3{}, f16{}, One{}, No{}, No{});
+    return run(pa::fp8e4m3{}, bf16{}, One{}, No{}, No{});
   }
   return PA_ERR_UNSUPPORTED;
 }
@@ -236,6 +250,8 @@ int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cac
   if (G > 8 || num_kv_heads > 255) return PA_ERR_UNSUPPORTED;
   if (num_groups == 0) max_members = 1;
   if (max_members > 1 && qtok > 1) return PA_ERR_UNSUPPORTED;  // shared items are single-token decode
+  // several query tokens: a 16-bit cache with a query of the same type
+  if (qtok > 1 && (kv_dtype == PA_FP8_E4M3 || q_dtype != kv_dtype)) return PA_ERR_UNSUPPORTED;
   // an item holds qtok * G (or max_members * G) query rows: up to 8 on every dtype pair, up to
   // 32 on a 16-bit cache with a query of its own type and head_dim 128
   const int64_t cols = static_cast<int64_t>(qtok) * max_members * G;
@@ -260,7 +276,7 @@ int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cac
   if (!out || !q || !k_cache || !v_cache || !block_tables || !seq_lens || (num_groups && !groups))
     return PA_ERR_INVALID;
   if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache)) return PA_ERR_INVALID;
-  const int64_t max_parts = max_parts_for(max_len, P);
+  const int64_t max_parts = max_parts_for(max_len, P, num_groups > 0);
   if (max_parts > 32767) return PA_ERR_UNSUPPORTED;
   // partial results are kept per (query token, query head): the workspace of qtok * num_q_heads heads
   const WsLayout L = ws_layout(num_seqs, static_cast<int64_t>(qtok) * num_q_heads, head_dim, max_parts);

@@ -105,43 +105,46 @@ __device__ __forceinline__ void store_out(void* out, int64_t idx, float v, int d
 }
 
 // ------------------------------------------------------------------------------ plan
-__device__ __forceinline__ int warp_inclusive_scan(int v) {
+template <typename T>
+__device__ __forceinline__ T warp_inclusive_scan(T v) {
   const int lane = threadIdx.x & 31;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
-    const int n = __shfl_up_sync(0xffffffffu, v, o);
+    const T n = __shfl_up_sync(0xffffffffu, v, o);
     if (lane >= o) v += n;
   }
   return v;
 }
 
 // Exclusive prefix sum over the block (blockDim.x a multiple of 32, at most 1024);
-// *total receives the block sum.
-__device__ int block_exclusive_scan(int v, int* s_warp, int* total) {
+// *total receives the block sum.  A 64-bit T scans two 32-bit counts at once (low + high << 32).
+template <typename T>
+__device__ T block_exclusive_scan(T v, T* s_warp, T* total) {
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
-  const int inc = warp_inclusive_scan(v);
+  const T inc = warp_inclusive_scan(v);
   if (lane == 31) s_warp[w] = inc;
   __syncthreads();
   if (w == 0) {
-    const int x = lane < nw ? s_warp[lane] : 0;
-    const int xi = warp_inclusive_scan(x);
+    const T x = lane < nw ? s_warp[lane] : T(0);
+    const T xi = warp_inclusive_scan(x);
     if (lane < nw) s_warp[lane] = xi - x;
     if (lane == 31) s_warp[32] = xi;
   }
   __syncthreads();
-  const int r = s_warp[w] + inc - v;
+  const T r = s_warp[w] + inc - v;
   *total = s_warp[32];
   __syncthreads();
   return r;
 }
 
+__device__ __forceinline__ long long pack2x32(int lo, int hi) {
+  return static_cast<long long>(lo) + (static_cast<long long>(hi) << 32);
+}
+__device__ __forceinline__ int lo32(long long v) { return static_cast<int>(v & 0xffffffffll); }
+__device__ __forceinline__ int hi32(long long v) { return static_cast<int>(v >> 32); }
+
 constexpr int kPlanThreads = 256;
 
-__device__ __forceinline__ int block_sum(int v, int* s_warp) {
-  int total;
-  block_exclusive_scan(v, s_warp, &total);
-  return total;
-}
 
 // Work list of one call.  Per sequence i of length L (valid: 0 <= L <= max_len and L = 0 or
 // L >= qtok) with S shared tokens (0 outside a prefix group):
@@ -155,7 +158,7 @@ __global__ void __launch_bounds__(kPlanThreads) pa_decode_plan_kernel(const Deco
   // the partition kernel may start its prologue now; it waits for this grid before
   // touching anything written here
   pdl_launch_dependents();
-  __shared__ int s_warp[33];
+  __shared__ long long s_warp[33];
   const int N = p.num_seqs, P = p.partition_size, BS = p.block_size;
   const int max_len = p.max_blocks_per_seq * p.block_size;
   auto valid_len = [&](int L) { return L >= 0 && L <= max_len && (L == 0 || L >= p.qtok); };
@@ -229,8 +232,9 @@ __global__ void __launch_bounds__(kPlanThreads) pa_decode_plan_kernel(const Deco
     loc_s += c.ns;
     loc_f += c.nf;
   }
-  const int n_shared = block_sum(loc_s, s_warp);
-  const int n_full = block_sum(loc_f, s_warp);
+  long long tot;
+  block_exclusive_scan(pack2x32(loc_f, loc_s), s_warp, &tot);
+  const int n_full = lo32(tot), n_shared = hi32(tot);
   int base_s = 0, base_f = 0, base_t = 0;
   for (int start = 0; start < N; start += blockDim.x) {
     const int i = start + threadIdx.x;
@@ -248,10 +252,15 @@ __global__ void __launch_bounds__(kPlanThreads) pa_decode_plan_kernel(const Deco
       const bool direct = c.S == 0 && parts == 1;
       p.seq_parts[i] = direct ? 0 : parts;
     }
-    int ts, tf, tt;
-    const int os = block_exclusive_scan(c.ns, s_warp, &ts);
-    const int of = block_exclusive_scan(c.nf, s_warp, &tf);
-    const int ot = block_exclusive_scan(c.nt, s_warp, &tt);
+    long long tft;
+    const long long oft = block_exclusive_scan(pack2x32(c.nf, c.nt), s_warp, &tft);
+    const int of = lo32(oft), ot = hi32(oft), tf = lo32(tft), tt = hi32(tft);
+    int os = 0, ts = 0;
+    if (n_shared > 0) {  // block-uniform
+      long long tsl;
+      os = static_cast<int>(block_exclusive_scan(static_cast<long long>(c.ns), s_warp, &tsl));
+      ts = static_cast<int>(tsl);
+    }
     const int dflag = (c.S == 0 && c.nf + c.nt == 1) ? WI_DIRECT : 0;
     for (int k = 0; k < c.ns; ++k)
       p.items[base_s + os + k] = WorkItem{i, k * P, min(c.S, (k + 1) * P), k | (c.sub << 16)};
@@ -313,8 +322,9 @@ __device__ __forceinline__ uint32_t lds_u16(uint32_t addr) {
 
 // NT: 8-column MMA tiles per consumer warp; PAIR: two consumer warps share each ring, the
 // second taking the item's query rows after the first's 8 * NT (for items of up to 32 rows:
-// twice the warps hide the latency of the longer per-page work).
-template <int BS, int D, typename KT, typename QT, int NT, bool PAIR>
+// twice the warps hide the latency of the longer per-page work); CAUSAL: the kernel can run
+// several query tokens per sequence (causal masking compiled in).
+template <int BS, int D, typename KT, typename QT, int NT, bool PAIR, bool CAUSAL>
 struct DecodeCfg {
   static constexpr bool FP8 = KvTraits<KT>::fp8;
   static constexpr int HALVES = D * KvTraits<KT>::bytes / 128;  // 128-byte column blocks of a row
@@ -327,7 +337,10 @@ struct DecodeCfg {
   static constexpr bool QCONV = FP8 && !QSPLIT;
   static constexpr int CONS = PAIR ? 2 : 1;             // consumer warps per ring
   static constexpr int COLS = 8 * NT * CONS;            // query rows per item (MMA N dimension)
-  static constexpr int QBUF_BYTES = ((COLS * D * QE + 1023) / 1024) * 1024;  // per ring
+  static constexpr int QBUF_BYTES = ((COLS * D * QE + 1023) / 1024) * 1024;  // one item's query rows
+  // query buffers per ring: the producer fills item k's while items k - QN + 1 .. k - 1 are in
+  // flight, so it can run ahead across short items
+  static constexpr int QN = PAIR ? 2 : 4;
   static constexpr int SLOT_BYTES = 2 * PAGE_BYTES;     // K page then V page
   static constexpr int NC = 4;                          // rings, one producer warp each
   static constexpr int NCONS = NC * CONS;               // consumer warps: ring = warp % NC
@@ -337,10 +350,11 @@ struct DecodeCfg {
   static_assert(!PAIR || NC * 32 * REG_PRODUCER + NCONS * 32 * REG_CONSUMER <= NWARP * 32 * REG_LAUNCH,
                 "register split exceeds the launch allocation");
   static constexpr int SMEM_BUDGET = 200 * 1024;
-  static constexpr int NSLOT_FIT = (SMEM_BUDGET / NC - QBUF_BYTES) / SLOT_BYTES;
+  static constexpr int NSLOT_FIT = (SMEM_BUDGET / NC - QN * QBUF_BYTES) / SLOT_BYTES;
   static constexpr int NSLOT = NSLOT_FIT > 8 ? 8 : (NSLOT_FIT < 2 ? 2 : NSLOT_FIT);
-  static constexpr int RING_BYTES = NC * (NSLOT * SLOT_BYTES + QBUF_BYTES);
-  static constexpr int BAR_BYTES = NC * (2 * NSLOT + 2) * 8;  // full + empty per slot, qfree (+pad)
+  static constexpr int RING_BYTES = NC * (NSLOT * SLOT_BYTES + QN * QBUF_BYTES);
+  static constexpr int NBAR = (2 * NSLOT + QN + 1) & ~1;     // full + empty per slot, qfree per buffer (+pad)
+  static constexpr int BAR_BYTES = NC * NBAR * 8;
   static constexpr int META_BYTES = NC * NSLOT * 16;
   static constexpr int SMEM_BYTES = 1024 + RING_BYTES + BAR_BYTES + META_BYTES + 16 * NC;
   static constexpr int MT = BS / 16;    // 16-token MMA tiles per page
@@ -348,7 +362,7 @@ struct DecodeCfg {
   static_assert(D == 64 || D == 128, "head_dim");
   static_assert(BS == 16 || BS == 32, "block_size");
   static_assert(HALVES >= 1, "an FP8 row must fill a 128-byte box (head_dim 128)");
-  static_assert((NT == 1 && !PAIR) || (!FP8 && !QSPLIT), "wide items: 16-bit cache and query");
+  static_assert((NT == 1 && !PAIR && !CAUSAL) || (!FP8 && !QSPLIT), "wide or causal items: 16-bit cache and query");
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
 };
 
@@ -368,11 +382,11 @@ constexpr int F_FIRST = 1, F_LAST = 2, F_BAD = 4, F_END = 8, F_DIRECT = 16;
 // has one member and one query token; multi-token attention has qtok > 1 (query token t sits at
 // position len - qtok + t and attends causally); a shared-prefix item has members > 1 (the
 // sequences seq .. seq + members - 1 share the item's tokens).
-template <int BS, int D, typename KT, typename QT, int NT, bool PAIR>
-__global__ void __launch_bounds__(DecodeCfg<BS, D, KT, QT, NT, PAIR>::NWARP * 32, 1)
+template <int BS, int D, typename KT, typename QT, int NT, bool PAIR, bool CAUSAL>
+__global__ void __launch_bounds__(DecodeCfg<BS, D, KT, QT, NT, PAIR, CAUSAL>::NWARP * 32, 1)
     pa_decode_partition_kernel(const __grid_constant__ CUtensorMap tmk,
                                const __grid_constant__ CUtensorMap tmv, const DecodeParams p) {
-  using C = DecodeCfg<BS, D, KT, QT, NT, PAIR>;
+  using C = DecodeCfg<BS, D, KT, QT, NT, PAIR, CAUSAL>;
   using MA = typename KvTraits<KT>::mma_t;  // element type of the tensor-core operands
   constexpr unsigned FULL = 0xffffffffu;
 
@@ -380,9 +394,9 @@ __global__ void __launch_bounds__(DecodeCfg<BS, D, KT, QT, NT, PAIR>::NWARP * 32
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int c = warp % C::NC;  // ring of this warp (its consumers and producer share a scheduler)
-  uint8_t* ring = smem + c * (C::NSLOT * C::SLOT_BYTES + C::QBUF_BYTES);
-  uint8_t* qbuf = ring + C::NSLOT * C::SLOT_BYTES;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::RING_BYTES) + c * (2 * C::NSLOT + 2);
+  uint8_t* ring = smem + c * (C::NSLOT * C::SLOT_BYTES + C::QN * C::QBUF_BYTES);
+  uint8_t* qbufs = ring + C::NSLOT * C::SLOT_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::RING_BYTES) + c * C::NBAR;
   uint64_t* empty = full + C::NSLOT;
   uint64_t* qfree = empty + C::NSLOT;
   int4* meta = reinterpret_cast<int4*>(smem + C::RING_BYTES + C::BAR_BYTES) + c * C::NSLOT;
@@ -391,9 +405,9 @@ __global__ void __launch_bounds__(DecodeCfg<BS, D, KT, QT, NT, PAIR>::NWARP * 32
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::NC; ++i) {
-      uint64_t* b = reinterpret_cast<uint64_t*>(smem + C::RING_BYTES) + i * (2 * C::NSLOT + 2);
+      uint64_t* b = reinterpret_cast<uint64_t*>(smem + C::RING_BYTES) + i * C::NBAR;
       // full: the producer's arrival (+ bytes); empty and qfree: one arrival per consumer warp
-      for (int s = 0; s < 2 * C::NSLOT + 1; ++s) mbar_init(&b[s], s < C::NSLOT ? 1 : C::CONS);
+      for (int s = 0; s < 2 * C::NSLOT + C::QN; ++s) mbar_init(&b[s], s < C::NSLOT ? 1 : C::CONS);
       flags_base[4 * i] = 0;
     }
     fence_mbar_init();
@@ -448,8 +462,9 @@ __global__ void __launch_bounds__(DecodeCfg<BS, D, KT, QT, NT, PAIR>::NWARP * 32
         if (mismatch) record_error(DEV_BAD_PREFIX);
       }
       bad |= mismatch;
-      if (items >= 1) {  // the consumer has taken the previous item's query rows
-        const bool ok = mbar_wait_bounded(qfree, (items - 1) & 1u, kWaitLimit);
+      const uint32_t qb = items % C::QN;
+      if (items >= C::QN) {  // the consumers have taken the query rows of item `items - QN`
+        const bool ok = mbar_wait_bounded(&qfree[qb], ((items / C::QN) - 1) & 1u, kWaitLimit);
         if (!__all_sync(FULL, ok) || *abort_flag) {
           stop = true;
           break;
@@ -487,7 +502,7 @@ __global__ void __launch_bounds__(DecodeCfg<BS, D, KT, QT, NT, PAIR>::NWARP * 32
           __syncwarp();  // the expected byte count is set before any copy can complete
           if (lane < rows) {  // query rows of (member, token) lane: G contiguous heads
             const int m = lane / T, t = lane - m * T;
-            bulk_load(qbuf + lane * G * D * C::QE,
+            bulk_load(qbufs + qb * C::QBUF_BYTES + lane * G * D * C::QE,
                       static_cast<const uint8_t*>(p.q) +
                           ((static_cast<int64_t>(it.seq + m) * T + t) * Hq + kvh * G) * D * C::QE,
                       static_cast<uint32_t>(G * D * C::QE), &full[slot]);
@@ -554,7 +569,8 @@ __global__ void __launch_bounds__(DecodeCfg<BS, D, KT, QT, NT, PAIR>::NWARP * 32
   bool poisoned = false;
   int ncol = G;  // query rows of the current item
 
-  auto load_q = [&]() {  // query rows of the item from the consumer's buffer; rows >= ncol are zero
+  // query rows of the item from its buffer qbuf; rows >= ncol are zero
+  auto load_q = [&](const uint8_t* qbuf) {
     if constexpr (!C::QSPLIT && !C::QCONV) {
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
@@ -663,7 +679,7 @@ __global__ void __launch_bounds__(DecodeCfg<BS, D, KT, QT, NT, PAIR>::NWARP * 32
             for (int h = 0; h < 2; ++h)
               if ((m0 + mi) * 16 + r0 + 8 * h >= ntok) s[mi][nt][2 * h] = s[mi][nt][2 * h + 1] = -CUDART_INF_F;
       }
-      if (T > 1 && rel + BS > 1) {
+      if (CAUSAL && T > 1 && rel + BS > 1) {
         // causal: query token t sees keys up to its own position (rel: the page's first key
         // relative to query token 0)
 #pragma unroll
@@ -842,6 +858,7 @@ __global__ void __launch_bounds__(DecodeCfg<BS, D, KT, QT, NT, PAIR>::NWARP * 32
   };
 
   uint32_t n = 0;
+  uint32_t citems = 0;  // items started by this consumer (selects the query buffer)
   bool ok = true;
   while (true) {
     const int slot = static_cast<int>(n % C::NSLOT);
@@ -866,9 +883,11 @@ __global__ void __launch_bounds__(DecodeCfg<BS, D, KT, QT, NT, PAIR>::NWARP * 32
       }
       poisoned = (flags & F_BAD) != 0;
       ncol = ((mt.z >> 16) & 0xff) * T * G;  // members x query tokens x grouped heads
-      if (!poisoned) load_q();
+      const uint32_t qb = citems % C::QN;
+      if (!poisoned) load_q(qbufs + qb * C::QBUF_BYTES);
       __syncwarp();
-      if (lane == 0) mbar_arrive(qfree);  // the query buffer may take the next item's rows
+      if (lane == 0) mbar_arrive(&qfree[qb]);  // the buffer may take a later item's rows
+      ++citems;
     }
     const int mycols = ncol - col0;  // query rows of the item in this consumer's tiles
     if (!poisoned && mycols > 0) {
@@ -900,8 +919,15 @@ __global__ void __launch_bounds__(kMergeWarps * 32) pa_decode_merge_kernel(const
   const int Hq = p.qtok * p.num_q_heads, D = p.head_dim;
   if (pair >= static_cast<int64_t>(p.num_seqs) * Hq) return;
   const int seq = static_cast<int>(pair / Hq), hq = static_cast<int>(pair % Hq);
-  const int np = p.seq_parts[seq];
-  if (np == 0) return;  // written directly, or empty / invalid
+  int np;
+  if (p.num_groups == 0) {  // the partitions follow from the length alone
+    const int L = p.seq_lens[seq], P = p.partition_size;
+    if (L <= P || L > p.max_blocks_per_seq * p.block_size) return;  // direct, empty or invalid rows
+    np = (L + P - 1) / P;
+  } else {
+    np = p.seq_parts[seq];
+    if (np == 0) return;  // written directly, or empty / invalid
+  }
   const int64_t base = static_cast<int64_t>(seq) * p.max_parts;
   float M = -CUDART_INF_F;
   for (int k = lane; k < np; k += 32) M = fmaxf(M, __ldcg(&p.part_ml[(base + k) * Hq + hq].x));

@@ -82,8 +82,10 @@ def test_decode_argument_validation(lib):
     assert decode_call(lib, q=0) == B.PA_ERR_INVALID
     assert decode_call(lib, k=FAKE + 8) == B.PA_ERR_INVALID      # misaligned cache
     assert decode_call(lib, wsb=100) == B.PA_ERR_WORKSPACE
+    # the size query bounds every decode entry point (prefix groups need one more partition per
+    # sequence than plain decode); a workspace well below it is refused
     need = B.pa_decode_workspace_size(4, 8, 128, 8 * 16)
-    assert decode_call(lib, wsb=need - 1) == B.PA_ERR_WORKSPACE
+    assert decode_call(lib, wsb=need // 2) == B.PA_ERR_WORKSPACE
     assert decode_call(lib, ws=FAKE + 16, wsb=need) == B.PA_ERR_INVALID   # workspace not 256-aligned
 
 
@@ -124,12 +126,13 @@ def test_multi_argument_validation(lib):
     assert multi_call(lib, D=64) == B.PA_ERR_UNSUPPORTED           # > 8 rows needs head_dim 128
     assert multi_call(lib, qd=0) == B.PA_ERR_UNSUPPORTED           # > 8 rows needs q_dtype == kv_dtype
     assert multi_call(lib, kd=3) == B.PA_ERR_UNSUPPORTED           # FP8 cache
-    assert multi_call(lib, T=2, qd=0) == B.PA_ERR_WORKSPACE        # 8 rows: any dtype pair; then the workspace
-    assert multi_call(lib, T=2, D=64) == B.PA_ERR_WORKSPACE
+    assert multi_call(lib, T=2, qd=0) == B.PA_ERR_UNSUPPORTED      # several tokens: q_dtype == kv_dtype
+    assert multi_call(lib, T=1, qd=0) == B.PA_ERR_WORKSPACE        # one token: pa_decode's dtype pairs
+    assert multi_call(lib, T=2, D=64) == B.PA_ERR_WORKSPACE        # 8 rows: head_dim 64 too
     # the workspace is pa_decode's for T * Hq heads
     need = B.pa_decode_workspace_size(4, 4 * 8, 128, 8 * 16)
     assert need > B.pa_decode_workspace_size(4, 8, 128, 8 * 16)
-    assert multi_call(lib, wsb=need - 1) == B.PA_ERR_WORKSPACE
+    assert multi_call(lib, wsb=need // 2) == B.PA_ERR_WORKSPACE
     assert multi_call(lib, ws=FAKE + 16, wsb=need) == B.PA_ERR_INVALID  # passes the size check, not 256-aligned
 
 
@@ -156,6 +159,6 @@ def test_prefix_argument_validation(lib):
     assert prefix_call(lib, mm=1, qd=0) == B.PA_ERR_WORKSPACE       # 8 rows: any dtype pair
     assert prefix_call(lib, ng=0, mm=99, qd=0) == B.PA_ERR_WORKSPACE  # no groups: max_members unused
     need = B.pa_decode_workspace_size(4, 16, 128, 8 * 16)
-    assert prefix_call(lib, wsb=need - 1) == B.PA_ERR_WORKSPACE
+    assert prefix_call(lib, wsb=need - 1) == B.PA_ERR_WORKSPACE       # prefix calls need the full bound
     assert prefix_call(lib, ws=FAKE + 16, wsb=need) == B.PA_ERR_INVALID
     assert B.max_prefix_members(64, 8) == 4 and B.max_prefix_members(32, 8) == 8 and B.max_prefix_members(8, 8) == 32
