@@ -115,14 +115,14 @@ int encode_kv_map(CUtensorMap* map, const void* base, int kv_dtype, int64_t num_
   return r == CUDA_SUCCESS ? PA_OK : PA_ERR_CUDA;
 }
 
-template <int BS, int D, typename KT, typename QT, int NT, bool PAIR, bool CAUSAL>
+template <int BS, int D, typename KT, typename QT, int NT, bool PAIR, bool CAUSAL, int NR>
 int launch_partition(const pa::DecodeParams& p, const CUtensorMap& tmk, const CUtensorMap& tmv,
                      int64_t max_items, int dev, DeviceInfo* info, cudaStream_t stream) {
-  using C = pa::DecodeCfg<BS, D, KT, QT, NT, PAIR, CAUSAL>;
-  auto kern = pa::pa_decode_partition_kernel<BS, D, KT, QT, NT, PAIR, CAUSAL>;
+  using C = pa::DecodeCfg<BS, D, KT, QT, NT, PAIR, CAUSAL, NR>;
+  auto kern = pa::pa_decode_partition_kernel<BS, D, KT, QT, NT, PAIR, CAUSAL, NR>;
   static std::atomic<bool> smem_set[kMaxDevices];  // per instantiation and device
   if (!smem_set[dev].load(std::memory_order_acquire)) {
-    if (PAIR) {
+    if (C::SPLIT) {
       // the warps' setmaxnreg split must fit the registers the block is launched with, or the
       // consumers' increase would wait for ever: never launch such a build
       cudaFuncAttributes fa{};
@@ -163,11 +163,13 @@ int dispatch_kv(const pa::DecodeParams& p, const CUtensorMap& tmk, const CUtenso
                 int dev, DeviceInfo* info, int kv_dtype, int q_dtype, int cols, cudaStream_t stream) {
   const bool qf32 = q_dtype == PA_F32;
   const int nt = (cols + 7) / 8;
-  // one instantiation: KV element type K, query type Q, tiles per consumer N, paired, causal
+  // one instantiation: KV element type K, query type Q, tiles per consumer N, paired, causal;
+  // an FP8 cache runs 8 rings per CTA
   auto run = [&](auto k, auto q, auto n, auto pair, auto causal) {
     using K = decltype(k);
     using Q = decltype(q);
-    return launch_partition<BS, D, K, Q, decltype(n)::value, decltype(pair)::value, decltype(causal)::value>(
+    constexpr int NR = std::is_same<K, pa::fp8e4m3>::value ? 8 : 4;
+    return launch_partition<BS, D, K, Q, decltype(n)::value, decltype(pair)::value, decltype(causal)::value, NR>(
         p, tmk, tmv, max_items, dev, info, stream);
   };
   using bf16 = __nv_bfloat16;

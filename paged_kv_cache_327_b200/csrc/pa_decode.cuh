@@ -323,8 +323,10 @@ __device__ __forceinline__ uint32_t lds_u16(uint32_t addr) {
 // NT: 8-column MMA tiles per consumer warp; PAIR: two consumer warps share each ring, the
 // second taking the item's query rows after the first's 8 * NT (for items of up to 32 rows:
 // twice the warps hide the latency of the longer per-page work); CAUSAL: the kernel can run
-// several query tokens per sequence (causal masking compiled in).
-template <int BS, int D, typename KT, typename QT, int NT, bool PAIR, bool CAUSAL>
+// several query tokens per sequence (causal masking compiled in); NR: rings per CTA, each with
+// its own producer warp (8 rings put two independent consumers on every scheduler, for the
+// FP8 cache whose consumers convert every tile).
+template <int BS, int D, typename KT, typename QT, int NT, bool PAIR, bool CAUSAL, int NR = 4>
 struct DecodeCfg {
   static constexpr bool FP8 = KvTraits<KT>::fp8;
   static constexpr int HALVES = D * KvTraits<KT>::bytes / 128;  // 128-byte column blocks of a row
@@ -340,15 +342,20 @@ struct DecodeCfg {
   static constexpr int QBUF_BYTES = ((COLS * D * QE + 1023) / 1024) * 1024;  // one item's query rows
   // query buffers per ring: the producer fills item k's while items k - QN + 1 .. k - 1 are in
   // flight, so it can run ahead across short items
-  static constexpr int QN = PAIR ? 2 : 4;
+  static constexpr int QN = (PAIR || NR > 4) ? 2 : 4;
   static constexpr int SLOT_BYTES = 2 * PAGE_BYTES;     // K page then V page
-  static constexpr int NC = 4;                          // rings, one producer warp each
+  static constexpr int NC = NR;                         // rings, one producer warp each
   static constexpr int NCONS = NC * CONS;               // consumer warps: ring = warp % NC
   static constexpr int NWARP = NCONS + NC;
-  // registers per thread: at launch (65536 / threads), and after setmaxnreg in a paired kernel
-  static constexpr int REG_LAUNCH = PAIR ? 168 : 255, REG_PRODUCER = 56, REG_CONSUMER = 224;
-  static_assert(!PAIR || NC * 32 * REG_PRODUCER + NCONS * 32 * REG_CONSUMER <= NWARP * 32 * REG_LAUNCH,
+  // registers per thread: at launch (65536 / threads, a multiple of 8), and -- with more than 8
+  // warps -- after setmaxnreg moves the producers' share to the consumers
+  static constexpr bool SPLIT = NWARP > 8;
+  static constexpr int REG_LAUNCH = SPLIT ? (65536 / (NWARP * 32)) & ~7 : 255;
+  static constexpr int REG_PRODUCER = 56;
+  static constexpr int REG_CONSUMER = SPLIT ? ((NWARP * REG_LAUNCH - NC * REG_PRODUCER) / NCONS) & ~7 : 255;
+  static_assert(!SPLIT || NC * 32 * REG_PRODUCER + NCONS * 32 * REG_CONSUMER <= NWARP * 32 * REG_LAUNCH,
                 "register split exceeds the launch allocation");
+  static_assert(!SPLIT || (NC % 4 == 0 && NCONS % 4 == 0), "setmaxnreg acts on whole warpgroups");
   static constexpr int SMEM_BUDGET = 200 * 1024;
   static constexpr int NSLOT_FIT = (SMEM_BUDGET / NC - QN * QBUF_BYTES) / SLOT_BYTES;
   static constexpr int NSLOT = NSLOT_FIT > 8 ? 8 : (NSLOT_FIT < 2 ? 2 : NSLOT_FIT);
@@ -382,11 +389,11 @@ constexpr int F_FIRST = 1, F_LAST = 2, F_BAD = 4, F_END = 8, F_DIRECT = 16;
 // has one member and one query token; multi-token attention has qtok > 1 (query token t sits at
 // position len - qtok + t and attends causally); a shared-prefix item has members > 1 (the
 // sequences seq .. seq + members - 1 share the item's tokens).
-template <int BS, int D, typename KT, typename QT, int NT, bool PAIR, bool CAUSAL>
-__global__ void __launch_bounds__(DecodeCfg<BS, D, KT, QT, NT, PAIR, CAUSAL>::NWARP * 32, 1)
+template <int BS, int D, typename KT, typename QT, int NT, bool PAIR, bool CAUSAL, int NR>
+__global__ void __launch_bounds__(DecodeCfg<BS, D, KT, QT, NT, PAIR, CAUSAL, NR>::NWARP * 32, 1)
     pa_decode_partition_kernel(const __grid_constant__ CUtensorMap tmk,
                                const __grid_constant__ CUtensorMap tmv, const DecodeParams p) {
-  using C = DecodeCfg<BS, D, KT, QT, NT, PAIR, CAUSAL>;
+  using C = DecodeCfg<BS, D, KT, QT, NT, PAIR, CAUSAL, NR>;
   using MA = typename KvTraits<KT>::mma_t;  // element type of the tensor-core operands
   constexpr unsigned FULL = 0xffffffffu;
 
@@ -421,7 +428,7 @@ __global__ void __launch_bounds__(DecodeCfg<BS, D, KT, QT, NT, PAIR, CAUSAL>::NW
 
   if (warp >= C::NCONS) {
     // ============================== producer ==============================
-    if constexpr (PAIR) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(C::REG_PRODUCER));
+    if constexpr (C::SPLIT) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(C::REG_PRODUCER));
     const unsigned total = p.counters[1] * static_cast<unsigned>(Hkv);
     const uint64_t pol = policy_evict_first();
     uint32_t n = 0;      // pages issued into this ring
@@ -533,7 +540,7 @@ __global__ void __launch_bounds__(DecodeCfg<BS, D, KT, QT, NT, PAIR, CAUSAL>::NW
   }
 
   // ============================== consumer ==============================
-  if constexpr (PAIR) asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(C::REG_CONSUMER));
+  if constexpr (C::SPLIT) asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(C::REG_CONSUMER));
   const int col0 = (warp / C::NC) * NT * 8;  // first query row (column) of this consumer
   const int lr = lane & 7, lm = lane >> 3;  // ldmatrix: row inside an 8x8 matrix, matrix index
   const int r0 = lane >> 2, c2 = (lane & 3) * 2;
