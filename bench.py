@@ -54,7 +54,8 @@ def parse_args():
                     help="step: the decode step (default); swap: swap_blocks to / from pinned host memory")
     ap.add_argument("--config", default="8b", choices=list(W.CONFIG_NAMES))
     ap.add_argument("--block-size", type=int, default=None)
-    ap.add_argument("--num-seqs", type=int, default=None, help="smaller batch of the same config (profiling)")
+    ap.add_argument("--num-seqs", type=int, default=None,
+                    help="smaller batch of the same config (profiling; 70b: that many shared-prefix samples)")
     ap.add_argument("--partition-size", type=int, default=0)
     ap.add_argument("--out-dtype", default=None, help="f32 | f16 | bf16 (default: the query dtype)")
     ap.add_argument("--kv-dtype", default=None, choices=["e4m3"],
@@ -300,7 +301,9 @@ def run_ours(args):
                                 device_id=torch.device("cuda", local))
 
     seed = rank_seed(args.config, rank)
-    extra = {"num_seqs": args.num_seqs} if args.num_seqs else {}
+    extra = {}
+    if args.num_seqs:  # the 70b batch shrinks by whole groups of 4 samples
+        extra = {"num_groups": max(1, args.num_seqs // 4)} if args.config == "70b" else {"num_seqs": args.num_seqs}
     if args.qtok > 1:
         extra["num_q_tokens"] = args.qtok
     w = W.make_config(args.config, block_size=args.block_size, seed=seed, kv_dtype=args.kv_dtype, **extra)
