@@ -154,7 +154,8 @@ PA_API int pa_decode_multi(void* out, const void* q, const void* k_cache, const 
  * own tokens once for that member, and the partial softmax states are merged per sequence.
  *   prefix_groups  device int32 [num_groups][3] = (first, members, shared): sequences first ..
  *                  first + members - 1 hold the same physical blocks for their first `shared`
- *                  tokens; groups disjoint; shared a multiple of block_size and <= every
+ *                  tokens; groups disjoint (so num_groups <= num_seqs, else
+ *                  PA_ERR_INVALID); shared a multiple of block_size and <= every
  *                  member's seq_lens.  A group breaking these rules (both groups of an
  *                  overlapping pair) is ignored
  *                  (its sequences decode alone) and PA_DEV_BAD_PREFIX is recorded; members whose

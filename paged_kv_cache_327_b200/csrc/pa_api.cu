@@ -277,6 +277,7 @@ int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cac
   if (num_seqs == 0) return PA_OK;
   if (!out || !q || !k_cache || !v_cache || !block_tables || !seq_lens || (num_groups && !groups))
     return PA_ERR_INVALID;
+  if (num_groups > num_seqs) return PA_ERR_INVALID;  // disjoint groups of at least one sequence
   if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache)) return PA_ERR_INVALID;
   const int64_t max_parts = max_parts_for(max_len, P, num_groups > 0);
   if (max_parts > 32767) return PA_ERR_UNSUPPORTED;

@@ -166,32 +166,37 @@ __global__ void __launch_bounds__(kPlanThreads) pa_decode_plan_kernel(const Deco
   if (p.num_groups > 0) {
     // A group is used if it is in range, its shared tokens are whole blocks that every member
     // holds, and no other group claims any of its sequences; otherwise it is reported and its
-    // sequences decode alone.  seq_sub first counts the claims on each sequence.
-    auto well_formed = [&](int g) {
-      const int first = p.groups[3 * g], M = p.groups[3 * g + 1], S = p.groups[3 * g + 2];
-      bool ok = first >= 0 && M >= 1 && first <= N - M && S >= 0 && S % BS == 0;
-      for (int m = 0; ok && m < M; ++m) {
-        const int L = p.seq_lens[first + m];
-        ok = valid_len(L) && S <= L;
-      }
-      return ok;
-    };
+    // sequences decode alone.  seq_sub first counts the claims on each sequence; each group's
+    // verdict is kept in the (not yet written) work list, one int per group (num_groups <= N).
+    int* verdict = reinterpret_cast<int*>(p.items);
     for (int i = threadIdx.x; i < N; i += blockDim.x) p.seq_shared[i] = p.seq_sub[i] = 0;
     __syncthreads();
     for (int g = threadIdx.x; g < p.num_groups; g += blockDim.x) {
-      if (!well_formed(g)) {
+      const int first = p.groups[3 * g], M = p.groups[3 * g + 1], S = p.groups[3 * g + 2];
+      bool ok = first >= 0 && M >= 1 && first <= N - M && S >= 0 && S % BS == 0;
+      if (ok) {
+#pragma unroll 4
+        for (int m = 0; m < M; ++m) {  // independent loads: no early exit
+          const int L = p.seq_lens[first + m];
+          ok &= valid_len(L) && S <= L;
+        }
+      }
+      verdict[g] = ok;
+      if (!ok) {
         record_error(DEV_BAD_PREFIX);
         continue;
       }
-      for (int m = 0; m < p.groups[3 * g + 1]; ++m) atomicAdd(&p.seq_sub[p.groups[3 * g] + m], 1);
+      for (int m = 0; m < M; ++m) atomicAdd(&p.seq_sub[first + m], 1);
     }
     __syncthreads();
     for (int g = threadIdx.x; g < p.num_groups; g += blockDim.x) {
-      if (!well_formed(g)) continue;
+      if (!verdict[g]) continue;
       const int first = p.groups[3 * g], M = p.groups[3 * g + 1], S = p.groups[3 * g + 2];
       bool alone = true;
+#pragma unroll 4
       for (int m = 0; m < M; ++m) alone &= p.seq_sub[first + m] == 1;
       if (!alone) {
+        verdict[g] = 0;
         record_error(DEV_BAD_PREFIX);
         continue;
       }
@@ -202,12 +207,12 @@ __global__ void __launch_bounds__(kPlanThreads) pa_decode_plan_kernel(const Deco
     for (int i = threadIdx.x; i < N; i += blockDim.x) p.seq_sub[i] = 0;
     __syncthreads();
     for (int g = threadIdx.x; g < p.num_groups; g += blockDim.x) {
-      if (!well_formed(g)) continue;
+      if (!verdict[g]) continue;
       const int first = p.groups[3 * g], M = p.groups[3 * g + 1], S = p.groups[3 * g + 2];
-      if (S == 0 || M == 1 || p.seq_shared[first] != S) continue;  // unused, or lost a claim
+      if (S == 0 || M == 1) continue;
       for (int m = 0; m < M; m += p.max_members) p.seq_sub[first + m] = min(p.max_members, M - m);
     }
-    __syncthreads();
+    __syncthreads();  // the verdicts are dead from here on: the work list overwrites them
   }
 
   struct Counts {

@@ -34,21 +34,25 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
+// Suspend-time hint of one poll, in ns: a waiting thread sleeps (instead of issuing) until the
+// phase completes or this time has passed.
+constexpr uint32_t kPollSuspendNs = 1000;
+
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t done;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(done)
-      : "r"(smem_u32(bar)), "r"(parity)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(kPollSuspendNs)
       : "memory");
   return done != 0;
 }
 
 // Wait for the phase with the given parity to complete; gives up after `limit` polls.
-// Each try_wait may itself suspend the thread for a bounded, implementation-defined time,
-// so a limit of a few million polls is far beyond any healthy copy and far below a hang.
+// Each try_wait suspends the thread for at most kPollSuspendNs, so 2^20 polls give up after
+// about a second: far beyond any healthy copy and far below a hang.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, uint32_t limit) {
   for (uint32_t i = 0; i < limit; ++i)
     if (mbar_try_wait(bar, parity)) return true;

@@ -152,6 +152,7 @@ def test_prefix_argument_validation(lib):
     assert prefix_call(lib, ng=-1) == B.PA_ERR_INVALID
     assert prefix_call(lib, mm=0) == B.PA_ERR_INVALID
     assert prefix_call(lib, groups=0) == B.PA_ERR_INVALID          # groups promised, none given
+    assert prefix_call(lib, ng=5) == B.PA_ERR_INVALID              # more groups than sequences
     assert prefix_call(lib, mm=5) == B.PA_ERR_UNSUPPORTED           # 5 members x 8 heads > 32 rows
     assert prefix_call(lib, kd=3) == B.PA_ERR_UNSUPPORTED           # FP8 cache
     assert prefix_call(lib, qd=0) == B.PA_ERR_UNSUPPORTED           # 32 rows need q_dtype == kv_dtype
