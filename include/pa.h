@@ -236,6 +236,13 @@ PA_API const char* pa_strerror(int status);
  * since the last call (or a negative pa_status if reading it failed) and clears it. */
 PA_API int pa_get_device_error(void* stream);
 
+/* Diagnostic: runs, on one warp, the bounded mbarrier wait every kernel of the library uses,
+ * on a barrier that nothing ever arrives on, for at most `polls` polls (1 .. 2^20; each poll
+ * sleeps at most 1 us).  The wait gives up, records PA_DEV_TIMEOUT in the device error word
+ * and the kernel returns: this exercises the library's failure path without a fault or hang.
+ * Returns PA_ERR_INVALID for polls out of range, else the launch status. */
+PA_API int pa_selftest_wait_timeout(int polls, void* stream);
+
 /* ABI version of this header (major * 100 + minor). */
 PA_API int pa_version(void);
 

@@ -25,7 +25,8 @@ PA_OK, PA_ERR_INVALID, PA_ERR_UNSUPPORTED, PA_ERR_WORKSPACE, PA_ERR_CUDA = 0, -1
 
 EXPORTED = ("pa_decode_workspace_size", "pa_decode", "pa_reshape_and_cache", "pa_copy_blocks",
             "pa_strerror", "pa_get_device_error", "pa_version", "pa_decode_static_workspace",
-            "pa_decode_fp8", "pa_reshape_and_cache_fp8", "pa_swap_blocks", "pa_decode_multi", "pa_decode_prefix")
+            "pa_decode_fp8", "pa_reshape_and_cache_fp8", "pa_swap_blocks", "pa_decode_multi", "pa_decode_prefix",
+            "pa_selftest_wait_timeout")
 PA_ERR_TOO_LARGE = -5
 PA_DECODE_STATIC_WORKSPACE_BYTES = 64 << 20
 
@@ -73,6 +74,8 @@ def load_library(path: str = _LIB_PATH):
     lib.pa_decode_multi.restype = I
     lib.pa_decode_prefix.argtypes = [P, P, P, P, P, P, I, I, I, I, I, F, I, I64, I, I, I, I, P, I, I, P, SZ, P]
     lib.pa_decode_prefix.restype = I
+    lib.pa_selftest_wait_timeout.argtypes = [I, P]
+    lib.pa_selftest_wait_timeout.restype = I
     if path == _LIB_PATH:
         _lib = lib
     return lib
@@ -288,6 +291,11 @@ def pa_swap_blocks(dst_k: torch.Tensor, dst_v: torch.Tensor, src_k: torch.Tensor
                                        src_dst_pairs.shape[0], src_k.shape[0], dst_k.shape[0], block_bytes,
                                        _stream(stream))
     _check(rc, "pa_swap_blocks")
+
+
+def pa_selftest_wait_timeout(polls: int, stream=None) -> None:
+    """Run the library's bounded wait on a barrier nothing completes (see include/pa.h)."""
+    _check(load_library().pa_selftest_wait_timeout(int(polls), _stream(stream)), "pa_selftest_wait_timeout")
 
 
 def pa_get_device_error(stream=None) -> int:

@@ -521,6 +521,12 @@ int pa_swap_blocks(void* dst_k_cache, void* dst_v_cache, const void* src_k_cache
   return cudaPeekAtLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
+int pa_selftest_wait_timeout(int polls, void* stream) {
+  if (polls < 1 || polls > static_cast<int>(pa::kWaitLimit)) return PA_ERR_INVALID;
+  pa::pa_selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(static_cast<uint32_t>(polls));
+  return cudaPeekAtLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
 int pa_get_device_error(void* stream) {
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (cudaStreamSynchronize(st) != cudaSuccess) return PA_ERR_CUDA;

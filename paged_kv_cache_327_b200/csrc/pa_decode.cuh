@@ -919,11 +919,27 @@ __global__ void __launch_bounds__(DecodeCfg<BS, D, KT, QT, NT, PAIR, CAUSAL, NR>
   }
 }
 
+// ------------------------------------------------------------------------------ self-test
+// A wait that nothing completes: the bounded wait gives up after `polls` polls, records
+// DEV_TIMEOUT and the kernel returns (the failure path of every wait in this library).
+__global__ void __launch_bounds__(32) pa_selftest_wait_kernel(uint32_t polls) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+  }
+  __syncwarp();
+  const bool ok = mbar_wait_bounded(&bar, 0, polls);  // phase 0 never completes
+  if (!__all_sync(0xffffffffu, ok) && threadIdx.x == 0) record_error(DEV_TIMEOUT);
+}
+
 // ------------------------------------------------------------------------------ merge
 // One warp per (sequence, virtual head = query token x query head) of a sequence whose items
 // wrote partial results (shared partitions first, then its own):
-// out = sum_k 2^(m_k - M) O_k / sum_k 2^(m_k - M) l_k, M = max_k m_k, partitions in order.
+// out = sum_k 2^(m_k - M) O_k / sum_k 2^(m_k - M) l_k, M = max_k m_k, partitions in order (a
+// fixed interleaved order for sequences of more than kMergeSplit partitions).
 constexpr int kMergeWarps = 8;
+constexpr int kMergeSplit = 16;  // above this many partitions a warp merges four at a time
 __global__ void __launch_bounds__(kMergeWarps * 32) pa_decode_merge_kernel(const DecodeParams p) {
   pdl_wait();  // the partition kernel's partial results are visible from here on
   const int lane = threadIdx.x & 31;
@@ -947,6 +963,55 @@ __global__ void __launch_bounds__(kMergeWarps * 32) pa_decode_merge_kernel(const
   for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
   float num[4] = {0.f, 0.f, 0.f, 0.f}, den = 0.f;
   const int per = D >> 5;  // 2 or 4 elements per lane
+  if (np > kMergeSplit) {
+    // many partitions: four groups of 8 lanes take every fourth partition, a lane holding D / 8
+    // consecutive elements, so that several partitions are in flight; the groups' sums are added
+    // in a fixed order
+    const int grp = lane >> 3, cl = lane & 7, nv = D >> 5;  // float4 per lane
+    float4 acc4[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) acc4[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 2
+    for (int k = grp; k < np; k += 4) {
+      const float2 ml = __ldcg(&p.part_ml[(base + k) * Hq + hq]);
+      const float4* src = reinterpret_cast<const float4*>(p.part_acc + ((base + k) * Hq + hq) * D) + cl * nv;
+      float4 a[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) a[j] = j < nv ? __ldcg(src + j) : make_float4(0.f, 0.f, 0.f, 0.f);
+      const float w = fast_exp2(ml.x - M);
+      den += w * ml.y;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        acc4[j].x += w * a[j].x;
+        acc4[j].y += w * a[j].y;
+        acc4[j].z += w * a[j].z;
+        acc4[j].w += w * a[j].w;
+      }
+    }
+#pragma unroll
+    for (int o = 8; o < 32; o <<= 1) {
+      den += __shfl_xor_sync(0xffffffffu, den, o);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        acc4[j].x += __shfl_xor_sync(0xffffffffu, acc4[j].x, o);
+        acc4[j].y += __shfl_xor_sync(0xffffffffu, acc4[j].y, o);
+        acc4[j].z += __shfl_xor_sync(0xffffffffu, acc4[j].z, o);
+        acc4[j].w += __shfl_xor_sync(0xffffffffu, acc4[j].w, o);
+      }
+    }
+    if (grp != 0) return;
+    const float inv = 1.f / den;
+    const int64_t o = (static_cast<int64_t>(seq) * Hq + hq) * D + cl * nv * 4;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      if (j >= nv) break;
+      store_out(p.out, o + 4 * j + 0, acc4[j].x * inv, p.out_dtype);
+      store_out(p.out, o + 4 * j + 1, acc4[j].y * inv, p.out_dtype);
+      store_out(p.out, o + 4 * j + 2, acc4[j].z * inv, p.out_dtype);
+      store_out(p.out, o + 4 * j + 3, acc4[j].w * inv, p.out_dtype);
+    }
+    return;
+  }
 #pragma unroll 4
   for (int k = 0; k < np; ++k) {
     const float2 ml = __ldcg(&p.part_ml[(base + k) * Hq + hq]);

@@ -163,3 +163,8 @@ def test_prefix_argument_validation(lib):
     assert prefix_call(lib, wsb=need - 1) == B.PA_ERR_WORKSPACE       # prefix calls need the full bound
     assert prefix_call(lib, ws=FAKE + 16, wsb=need) == B.PA_ERR_INVALID
     assert B.max_prefix_members(64, 8) == 4 and B.max_prefix_members(32, 8) == 8 and B.max_prefix_members(8, 8) == 32
+
+
+def test_selftest_argument_checks(lib):
+    assert lib.pa_selftest_wait_timeout(0, ctypes.c_void_p(0)) == B.PA_ERR_INVALID
+    assert lib.pa_selftest_wait_timeout((1 << 20) + 1, ctypes.c_void_p(0)) == B.PA_ERR_INVALID
