@@ -313,10 +313,13 @@ __device__ __forceinline__ float to_float<__half>(__half x) { return __half2floa
 template <>
 __device__ __forceinline__ float to_float<__nv_bfloat16>(__nv_bfloat16 x) { return __bfloat162float(x); }
 
-// two E4M3 codes (low byte first) -> two f16 (exact: every E4M3 value is an f16 value)
-__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t v) {
-  const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(v & 0xffffu), __NV_E4M3);
-  return static_cast<uint32_t>(h.x) | (static_cast<uint32_t>(h.y) << 16);
+// four E4M3 codes (byte 0 first) -> f16 pairs (bytes 0, 1) and (bytes 2, 3), exact (every E4M3
+// value is an f16 value); the two halves of the word are converted in place, with no shift
+__device__ __forceinline__ void e4m3x4_to_f16x2x2(uint32_t v, uint32_t& lo, uint32_t& hi) {
+  asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %2;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %0, l;\n\tcvt.rn.f16x2.e4m3x2 %1, h;\n\t}"
+      : "=r"(lo), "=r"(hi)
+      : "r"(v));
 }
 
 __device__ __forceinline__ uint32_t lds_u16(uint32_t addr) {
@@ -648,8 +651,9 @@ __global__ void __launch_bounds__(DecodeCfg<BS, D, KT, QT, NT, PAIR, CAUSAL, NR>
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
               const int kk = 2 * kq + h;
-              const uint32_t a0 = e4m3x2_to_f16x2(r[2 * h]), a1 = e4m3x2_to_f16x2(r[2 * h + 1]);
-              const uint32_t a2 = e4m3x2_to_f16x2(r[2 * h] >> 16), a3 = e4m3x2_to_f16x2(r[2 * h + 1] >> 16);
+              uint32_t a0, a1, a2, a3;
+              e4m3x4_to_f16x2x2(r[2 * h], a0, a2);
+              e4m3x4_to_f16x2x2(r[2 * h + 1], a1, a3);
               if constexpr (C::QSPLIT) {
                 Mma<MA>::run(sa[0], a0, a1, a2, a3, qf[kk][0][0], qf[kk][0][1]);
                 Mma<MA>::run(sb2[0], a0, a1, a2, a3, ql[kk][0], ql[kk][1]);
@@ -780,8 +784,9 @@ __global__ void __launch_bounds__(DecodeCfg<BS, D, KT, QT, NT, PAIR, CAUSAL, NR>
               const uint32_t u2 = lds_u16(row0 + 8 * 128 + (((dt ^ vx0)) << 4));
               const uint32_t u3 = lds_u16(row0 + 9 * 128 + (((dt ^ vx1)) << 4));
               const uint32_t w01 = __byte_perm(u0, u1, 0x5140), w23 = __byte_perm(u2, u3, 0x5140);
-              uint32_t a0 = e4m3x2_to_f16x2(w01), a1 = e4m3x2_to_f16x2(w01 >> 16);
-              uint32_t a2 = e4m3x2_to_f16x2(w23), a3 = e4m3x2_to_f16x2(w23 >> 16);
+              uint32_t a0, a1, a2, a3;
+              e4m3x4_to_f16x2x2(w01, a0, a1);
+              e4m3x4_to_f16x2x2(w23, a2, a3);
               if constexpr (decltype(masked)::value) {
                 a0 &= mlo;
                 a1 &= mlo;
