@@ -6,30 +6,34 @@
 // block block_tables[i][t / block_size] at position t % block_size, KV head hq / G.
 //
 // How (B200 design, not the page's one-CTA-per-(seq, head) scalar loop):
-//  * plan kernel (one CTA): turns seq_lens into a work list of (sequence, partition)
-//    pairs -- full 512-token partitions first, ragged tails last -- zeroes the work
-//    counter, and writes the rows of empty or invalid sequences;
-//  * partition kernel: persistent, one CTA per SM, NC consumer warps each fed by its own
-//    producer warp.  A work item is (sequence, partition, KV head), taken from an atomic
-//    counter.  The producer resolves the item's block-table entries and streams its
-//    pages into the consumer's ring of shared-memory slots: one TMA per 64-column half
-//    of the K and V page (box = block_size rows x 128 B, 128-byte swizzle, L2
-//    evict-first) plus a bulk copy of the G query rows with the first page, counted on
-//    the slot's "full" mbarrier; the consumer frees the slot through its "empty"
-//    mbarrier.  Per page the G grouped query heads share one read of K and V:
-//      S^T[tokens x G] = K[tokens x D] . Q^T[D x G]       (mma.sync m16n8k16, fp32 acc)
-//      online softmax per query head: exp2 of scale*log2(e)-scaled scores, with the
-//      running maximum raised (and the accumulators rescaled) only when a score exceeds
-//      it by more than 2^8 -- the result is the same softmax, the rescale is rare
-//      O^T[D x G]   += V^T[D x tokens] . P^T[tokens x G]  (P^T via movmatrix.trans)
-//      l[G]         += 1^T . P^T                          (one more MMA, no shuffles)
-//    A sequence that fits one partition writes `out` directly.  Longer ones write the
-//    partition's (max, sum, unnormalised O) to the workspace and nothing else: no fence,
-//    atomic or merge ever stalls a consumer's page stream;
-//  * merge kernel: one warp per (sequence, query head) of a multi-partition sequence
-//    combines its partitions with the log-sum-exp rescale, in partition order.
-// The partition boundaries depend only on seq_lens[i] and each item is computed the same
-// way whatever warp runs it, so results are deterministic and batch-invariant.
+//  * plan kernel (one CTA): turns seq_lens (and prefix groups, if any) into a work list --
+//    shared-prefix items first, then full 512-token partitions, then ragged tails -- zeroes
+//    the work counter, and writes the rows of empty or invalid sequences;
+//  * partition kernel: persistent, one CTA per SM, with NR rings (4, or 8 for an FP8 cache),
+//    each fed by its own producer warp and drained by one consumer warp (two for items of more
+//    than 8 query rows).  A work item is (sequence(s), token range, KV head), taken from an
+//    atomic counter.  The producer resolves the item's block-table entries and streams its
+//    pages into the ring of shared-memory slots: one TMA per 128-byte column block of the K
+//    and V page (box = block_size rows x 128 B, 128-byte swizzle, L2 evict-first) plus bulk
+//    copies of the item's query rows with the first page, counted on the slot's "full"
+//    mbarrier; the consumers free the slot through its "empty" mbarrier.  Per page, all query
+//    rows of the item (the G grouped heads, times the query tokens or the members of a shared
+//    prefix) share one read of K and V:
+//      S^T[tokens x rows] = K[tokens x D] . Q^T[D x rows]     (mma.sync m16n8k16, fp32 acc)
+//      online softmax per row: exp2 of scale*log2(e)-scaled scores, with the running maximum
+//      raised (and the accumulators rescaled) only when a score exceeds it by more than 2^8
+//      -- the result is the same softmax, the rescale is rare; causal masking when the
+//      sequence has several query tokens
+//      O^T[D x rows] += V^T[D x tokens] . P^T[tokens x rows]  (P^T via movmatrix.trans)
+//      l[rows]       += 1^T . P^T                             (one more MMA, no shuffles)
+//    A sequence whose only item is one partition writes `out` directly.  Other items write
+//    their (max, sum, unnormalised O) to the workspace and nothing else: no fence, atomic or
+//    merge ever stalls a consumer's page stream;
+//  * merge kernel: one warp per (sequence, query row) of a sequence with partial results
+//    combines them with the log-sum-exp rescale, in a fixed order.
+// The split depends only on seq_lens[i] (and the prefix groups) and each item is computed the
+// same way whatever warp runs it, so results are deterministic; without prefix groups they are
+// also batch-invariant.
 #pragma once
 
 #include <cuda_fp8.h>
