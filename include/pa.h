@@ -133,8 +133,10 @@ PA_API int pa_decode_fp8(void* out, const void* q, const void* k_cache, const vo
  *   q    [num_seqs, num_q_tokens, num_q_heads, head_dim], q_dtype
  *   seq_lens[i] = 0 gives all-zero rows; 0 < seq_lens[i] < num_q_tokens is invalid (its rows
  *   are NaN and pa_get_device_error reports PA_DEV_BAD_SEQ_LEN).
- *   supported: q_dtype == kv_dtype (f16 or bf16); num_q_tokens * G <= 8 with head_dim 64 or
- *   128, up to 32 with head_dim 128 (num_q_tokens 1: every dtype pair of pa_decode).
+ *   supported: q_dtype == kv_dtype (f16 or bf16) for num_q_tokens > 1 (num_q_tokens 1: every
+ *   dtype pair of pa_decode), num_q_tokens up to 65536.  A work item holds up to 32 query rows
+ *   (query tokens x grouped heads) per KV head, 8 with head_dim 64: with more query tokens, the
+ *   tokens are split into column groups and each K/V page is read once per group.
  *   Everything else as pa_decode; the
  *   workspace is pa_decode_workspace_size(num_seqs, num_q_tokens * num_q_heads, head_dim,
  *   max_blocks_per_seq * block_size, partition_size).  num_q_tokens 1 is pa_decode. */

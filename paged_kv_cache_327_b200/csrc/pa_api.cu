@@ -39,6 +39,8 @@ int64_t max_parts_for(int64_t max_len, int P, bool groups = true) {
   return std::max<int64_t>(1, (max_len + P - 1) / P + (groups ? 1 : 0));
 }
 
+// num_q_heads: query heads x query tokens.  Items: one per (sequence, partition, column group);
+// a column group holds at least a sixteenth of the query rows, hence the factor.
 WsLayout ws_layout(int64_t num_seqs, int64_t num_q_heads, int64_t head_dim, int64_t max_parts) {
   WsLayout L{};
   size_t o = 0;
@@ -51,7 +53,7 @@ WsLayout ws_layout(int64_t num_seqs, int64_t num_q_heads, int64_t head_dim, int6
   L.seq_sub = o;
   o += align256(static_cast<size_t>(num_seqs) * sizeof(int));
   L.items = o;
-  o += align256(static_cast<size_t>(num_seqs * max_parts) * sizeof(pa::WorkItem));
+  o += align256(static_cast<size_t>(num_seqs * max_parts * ((num_q_heads + 15) / 16)) * sizeof(pa::WorkItem));
   L.part_ml = o;
   o += align256(static_cast<size_t>(num_seqs * max_parts * num_q_heads) * sizeof(float2));
   L.part_acc = o;
@@ -254,9 +256,14 @@ int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cac
   if (max_members > 1 && qtok > 1) return PA_ERR_UNSUPPORTED;  // shared items are single-token decode
   // several query tokens: a 16-bit cache with a query of the same type
   if (qtok > 1 && (kv_dtype == PA_FP8_E4M3 || q_dtype != kv_dtype)) return PA_ERR_UNSUPPORTED;
-  // an item holds qtok * G (or max_members * G) query rows: up to 8 on every dtype pair, up to
+  if (qtok > 65536 || static_cast<int64_t>(qtok) * num_q_heads * head_dim > INT_MAX) return PA_ERR_UNSUPPORTED;
+  // query tokens per item: all of them, or column groups of up to 32 query rows per KV head
+  // (8 with head_dim 64, whose items run on the one-consumer kernels)
+  const int max_rows = head_dim == 128 ? 32 : 8;
+  const int qtok_item = qtok * G <= max_rows ? qtok : std::max(1, max_rows / G);
+  // an item holds qtok_item * G (or max_members * G) query rows: up to 8 on every dtype pair, up to
   // 32 on a 16-bit cache with a query of its own type and head_dim 128
-  const int64_t cols = static_cast<int64_t>(qtok) * max_members * G;
+  const int64_t cols = static_cast<int64_t>(qtok_item) * max_members * G;
   if (cols > 32) return PA_ERR_UNSUPPORTED;
   if (cols > 8 && (head_dim != 128 || kv_dtype == PA_FP8_E4M3 || q_dtype != kv_dtype)) return PA_ERR_UNSUPPORTED;
   if (head_dim != 64 && head_dim != 128) return PA_ERR_UNSUPPORTED;
@@ -312,6 +319,7 @@ int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cac
   p.max_parts = static_cast<int>(max_parts);
   p.out_dtype = out_dtype;
   p.qtok = qtok;
+  p.qtok_item = qtok_item;
   p.groups = groups;
   p.num_groups = num_groups;
   p.max_members = max_members;
@@ -330,7 +338,8 @@ int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cac
   pa::pa_decode_plan_kernel<<<1, pa::kPlanThreads, 0, st>>>(p);
   if (cudaPeekAtLastError() != cudaSuccess) return PA_ERR_CUDA;
 
-  const int64_t max_items = static_cast<int64_t>(num_seqs) * max_parts * num_kv_heads;
+  const int64_t max_items =
+      static_cast<int64_t>(num_seqs) * max_parts * ((qtok + qtok_item - 1) / qtok_item) * num_kv_heads;
   int rc;
   const int c = static_cast<int>(cols);
   if (block_size == 16)

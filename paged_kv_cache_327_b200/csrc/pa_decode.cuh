@@ -69,9 +69,12 @@ constexpr uint32_t kWaitLimit = 1u << 20;
 constexpr float kRescaleThreshold = 8.0f;
 
 // A work item: tokens [tok0, tok1) of sequence seq (and of the members - 1 sequences after it,
-// which share those tokens' blocks), for every KV head; pm = part | members << 16 | WI_DIRECT.
-struct WorkItem {
+// which share those tokens' blocks), for every KV head, for the query tokens t0 .. t0 + tq - 1
+// of the sequence (a sequence with more query tokens than one item holds is split into column
+// groups); pm = part | members << 16 | WI_DIRECT.
+struct __align__(16) WorkItem {
   int seq, tok0, tok1, pm;
+  int t0, tq, pad0, pad1;
 };
 constexpr int WI_DIRECT = 1 << 30;  // the sequence's only item: write `out`, not a partial result
 
@@ -83,6 +86,7 @@ struct DecodeParams {
   int num_seqs, num_q_heads, num_kv_heads, group;
   int head_dim, block_size, max_blocks_per_seq, num_blocks;
   int partition_size, max_parts, out_dtype, qtok;  // qtok: query tokens per sequence (1 = decode)
+  int qtok_item;     // query tokens of one item (qtok, or fewer: then several column groups)
   // prefix groups, int32 [num_groups][3] = (first sequence, members, shared tokens): sequences
   // first .. first + members - 1 hold the same blocks for their first `shared` tokens
   const int32_t* groups;
@@ -91,7 +95,7 @@ struct DecodeParams {
   float v_scale;     // multiplies the output (FP8 cache); 1 otherwise
   // workspace views
   unsigned int* counters;  // [0] next work item, [1] number of work items
-  WorkItem* items;         // [num_seqs * max_parts]
+  WorkItem* items;         // [num_seqs * max_parts * column groups]
   int* seq_parts;          // [num_seqs]: partial results of the sequence (0: written directly, or no work)
   int* seq_shared;         // [num_seqs]: tokens shared through a valid prefix group (plan scratch)
   int* seq_sub;            // [num_seqs]: members of the shared items this sequence leads (plan scratch)
@@ -219,6 +223,8 @@ __global__ void __launch_bounds__(kPlanThreads) pa_decode_plan_kernel(const Deco
     __syncthreads();  // the verdicts are dead from here on: the work list overwrites them
   }
 
+  // column groups: the qtok query tokens of a sequence are split into items of qtok_item tokens
+  const int Tc = p.qtok_item, ncg = (p.qtok + Tc - 1) / Tc;
   struct Counts {
     int L, S, sub, ns, nf, nt, nps;
   };
@@ -239,7 +245,7 @@ __global__ void __launch_bounds__(kPlanThreads) pa_decode_plan_kernel(const Deco
   for (int i = threadIdx.x; i < N; i += blockDim.x) {
     const Counts c = counts(i);
     loc_s += c.ns;
-    loc_f += c.nf;
+    loc_f += c.nf * ncg;
   }
   long long tot;
   block_exclusive_scan(pack2x32(loc_f, loc_s), s_warp, &tot);
@@ -262,7 +268,7 @@ __global__ void __launch_bounds__(kPlanThreads) pa_decode_plan_kernel(const Deco
       p.seq_parts[i] = direct ? 0 : parts;
     }
     long long tft;
-    const long long oft = block_exclusive_scan(pack2x32(c.nf, c.nt), s_warp, &tft);
+    const long long oft = block_exclusive_scan(pack2x32(c.nf * ncg, c.nt * ncg), s_warp, &tft);
     const int of = lo32(oft), ot = hi32(oft), tf = lo32(tft), tt = hi32(tft);
     int os = 0, ts = 0;
     if (n_shared > 0) {  // block-uniform
@@ -271,14 +277,19 @@ __global__ void __launch_bounds__(kPlanThreads) pa_decode_plan_kernel(const Deco
       ts = static_cast<int>(tsl);
     }
     const int dflag = (c.S == 0 && c.nf + c.nt == 1) ? WI_DIRECT : 0;
+    // shared items have one query token (prefix groups are single-token decode)
     for (int k = 0; k < c.ns; ++k)
-      p.items[base_s + os + k] = WorkItem{i, k * P, min(c.S, (k + 1) * P), k | (c.sub << 16)};
+      p.items[base_s + os + k] = WorkItem{i, k * P, min(c.S, (k + 1) * P), k | (c.sub << 16), 0, 1, 0, 0};
     for (int k = 0; k < c.nf; ++k)
-      p.items[n_shared + base_f + of + k] =
-          WorkItem{i, c.S + k * P, c.S + (k + 1) * P, (c.nps + k) | (1 << 16) | dflag};
+      for (int j = 0; j < ncg; ++j)
+        p.items[n_shared + base_f + of + k * ncg + j] =
+            WorkItem{i, c.S + k * P, c.S + (k + 1) * P, (c.nps + k) | (1 << 16) | dflag, j * Tc,
+                     min(Tc, p.qtok - j * Tc), 0, 0};
     if (c.nt)
-      p.items[n_shared + n_full + base_t + ot] =
-          WorkItem{i, c.S + c.nf * P, c.L, (c.nps + c.nf) | (1 << 16) | dflag};
+      for (int j = 0; j < ncg; ++j)
+        p.items[n_shared + n_full + base_t + ot + j] =
+            WorkItem{i, c.S + c.nf * P, c.L, (c.nps + c.nf) | (1 << 16) | dflag, j * Tc,
+                     min(Tc, p.qtok - j * Tc), 0, 0};
     base_s += ts;
     base_f += tf;
     base_t += tt;
@@ -374,7 +385,7 @@ struct DecodeCfg {
   static constexpr int RING_BYTES = NC * (NSLOT * SLOT_BYTES + QN * QBUF_BYTES);
   static constexpr int NBAR = (2 * NSLOT + QN + 1) & ~1;     // full + empty per slot, qfree per buffer (+pad)
   static constexpr int BAR_BYTES = NC * NBAR * 8;
-  static constexpr int META_BYTES = NC * NSLOT * 16;
+  static constexpr int META_BYTES = NC * NSLOT * 32;    // two int4 per slot
   static constexpr int SMEM_BYTES = 1024 + RING_BYTES + BAR_BYTES + META_BYTES + 16 * NC;
   static constexpr int MT = BS / 16;    // 16-token MMA tiles per page
   static constexpr int KS = D / 16;     // 16-wide steps over head_dim
@@ -392,8 +403,10 @@ __device__ __forceinline__ uint32_t swz(int t, int d0) {
   return (d0 >> 6) * BOX_BYTES + t * 128 + ((((d0 & 63) >> 3) ^ (t & 7)) << 4);
 }
 
-// slot metadata: x = seq, y = part | page << 16, z = kvh | ntok << 8 | members << 16 | flags << 24,
-// w = position of the page's first token relative to the first query token (len - qtok)
+// slot metadata, two int4 per slot: [0] x = seq, y = part | page << 16,
+// z = kvh | ntok << 8 | rows << 16 | flags << 24 (rows: members x query tokens of the item),
+// w = position of the page's first token relative to the item's first query token;
+// [1] x = the item's first query token t0
 constexpr int F_FIRST = 1, F_LAST = 2, F_BAD = 4, F_END = 8, F_DIRECT = 16;
 
 // The query rows ("columns") of one work item are (member m, query token t, head g) for
@@ -418,7 +431,7 @@ __global__ void __launch_bounds__(DecodeCfg<BS, D, KT, QT, NT, PAIR, CAUSAL, NR>
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::RING_BYTES) + c * C::NBAR;
   uint64_t* empty = full + C::NSLOT;
   uint64_t* qfree = empty + C::NSLOT;
-  int4* meta = reinterpret_cast<int4*>(smem + C::RING_BYTES + C::BAR_BYTES) + c * C::NSLOT;
+  int4* meta = reinterpret_cast<int4*>(smem + C::RING_BYTES + C::BAR_BYTES) + 2 * c * C::NSLOT;
   volatile int* flags_base = reinterpret_cast<volatile int*>(smem + C::RING_BYTES + C::BAR_BYTES + C::META_BYTES);
   volatile int* abort_flag = flags_base + 4 * c;
 
@@ -461,9 +474,11 @@ __global__ void __launch_bounds__(DecodeCfg<BS, D, KT, QT, NT, PAIR, CAUSAL, NR>
       const int part = it.pm & 0xffff, members = (it.pm >> 16) & 0xff;
       const int tok0 = it.tok0, tok1 = it.tok1;
       const int npages = (tok1 - tok0 + BS - 1) / BS;
-      const int rows = members * T;  // (member, query token) pairs of the item: G query rows each
-      // key positions relative to the first query token (causal masking of several query tokens)
-      const int rel0 = T > 1 ? tok0 - (p.seq_lens[it.seq] - T) : 0;
+      const int t0 = it.t0, tq = it.tq;
+      const int rows = members * tq;  // (member, query token) pairs of the item: G query rows each
+      // key positions relative to the item's first query token, at position len - T + t0
+      // (causal masking of several query tokens)
+      const int rel0 = T > 1 ? tok0 - (p.seq_lens[it.seq] - T + t0) : 0;
       int bt = 0;
       bool bad = false, mismatch = false;
       if (lane < npages) {
@@ -502,8 +517,9 @@ __global__ void __launch_bounds__(DecodeCfg<BS, D, KT, QT, NT, PAIR, CAUSAL, NR>
           const int ntok = min(BS, tok1 - (tok0 + pg * BS));
           const int flags = (first ? F_FIRST : 0) | (pg == npages - 1 ? F_LAST : 0) | (bad ? F_BAD : 0) |
                             ((it.pm & WI_DIRECT) ? F_DIRECT : 0);
-          meta[slot] = make_int4(it.seq, part | (pg << 16), kvh | (ntok << 8) | (members << 16) | (flags << 24),
-                                 rel0 + pg * BS);
+          meta[2 * slot] = make_int4(it.seq, part | (pg << 16), kvh | (ntok << 8) | (rows << 16) | (flags << 24),
+                                     rel0 + pg * BS);
+          meta[2 * slot + 1] = make_int4(t0, 0, 0, 0);
           if (bad) {
             mbar_arrive(&full[slot]);
           } else {
@@ -520,7 +536,7 @@ __global__ void __launch_bounds__(DecodeCfg<BS, D, KT, QT, NT, PAIR, CAUSAL, NR>
         if (first && !bad) {
           __syncwarp();  // the expected byte count is set before any copy can complete
           if (lane < rows) {  // query rows of (member, token) lane: G contiguous heads
-            const int m = lane / T, t = lane - m * T;
+            const int m = lane / tq, t = t0 + lane - m * tq;
             bulk_load(qbufs + qb * C::QBUF_BYTES + lane * G * D * C::QE,
                       static_cast<const uint8_t*>(p.q) +
                           ((static_cast<int64_t>(it.seq + m) * T + t) * Hq + kvh * G) * D * C::QE,
@@ -535,7 +551,7 @@ __global__ void __launch_bounds__(DecodeCfg<BS, D, KT, QT, NT, PAIR, CAUSAL, NR>
       const int slot = static_cast<int>(n % C::NSLOT);
       if (acquire_slot(slot)) {
         if (lane == 0) {
-          meta[slot] = make_int4(0, 0, F_END << 24, 0);
+          meta[2 * slot] = make_int4(0, 0, F_END << 24, 0);
           mbar_arrive(&full[slot]);
         }
       } else {
@@ -586,7 +602,8 @@ __global__ void __launch_bounds__(DecodeCfg<BS, D, KT, QT, NT, PAIR, CAUSAL, NR>
   uint32_t ql[C::QSPLIT ? C::KS : 1][2];
   (void)ql;
   bool poisoned = false;
-  int ncol = G;  // query rows of the current item
+  int ncol = G;       // query rows of the current item
+  int item_t0 = 0;    // its first query token
 
   // query rows of the item from its buffer qbuf; rows >= ncol are zero
   auto load_q = [&](const uint8_t* qbuf) {
@@ -709,7 +726,7 @@ __global__ void __launch_bounds__(DecodeCfg<BS, D, KT, QT, NT, PAIR, CAUSAL, NR>
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
               const int col = col0 + nt * 8 + c2 + (e & 1);
-              const int t = (col / G) % T;
+              const int t = col / G;  // the item's query token (one member when T > 1)
               if (rel + (m0 + mi) * 16 + r0 + 8 * (e >> 1) > t) s[mi][nt][e] = -CUDART_INF_F;
             }
       }
@@ -850,7 +867,8 @@ __global__ void __launch_bounds__(DecodeCfg<BS, D, KT, QT, NT, PAIR, CAUSAL, NR>
         const int col = col0 + nt * 8 + c2 + j;
         if (col >= ncol) continue;
         const int g = col % G, mt_ = col / G;
-        const int m = mt_ / T, t = mt_ - m * T;
+        // several query tokens: one member, token t0 + mt_; otherwise member mt_, token 0
+        const int m = T > 1 ? 0 : mt_, t = T > 1 ? item_t0 + mt_ : 0;
         const int vh = t * Hq + kvh * G + g;
         const float l = lacc[nt][j];  // every row of the ones-MMA holds the column sums
         if (direct) {
@@ -889,7 +907,7 @@ __global__ void __launch_bounds__(DecodeCfg<BS, D, KT, QT, NT, PAIR, CAUSAL, NR>
       ok = false;
       break;
     }
-    const int4 mt = meta[slot];
+    const int4 mt = meta[2 * slot];
     const int kvh = mt.z & 0xff, ntok = (mt.z >> 8) & 0xff, flags = (mt.z >> 24) & 0xff;
     if (flags & F_END) break;
     const int part = mt.y & 0xffff;
@@ -903,7 +921,8 @@ __global__ void __launch_bounds__(DecodeCfg<BS, D, KT, QT, NT, PAIR, CAUSAL, NR>
         for (int dt = 0; dt < C::KS; ++dt) acc[dt][nt][0] = acc[dt][nt][1] = acc[dt][nt][2] = acc[dt][nt][3] = 0.f;
       }
       poisoned = (flags & F_BAD) != 0;
-      ncol = ((mt.z >> 16) & 0xff) * T * G;  // members x query tokens x grouped heads
+      ncol = ((mt.z >> 16) & 0xff) * G;  // (members x query tokens of the item) x grouped heads
+      item_t0 = meta[2 * slot + 1].x;
       const uint32_t qb = citems % C::QN;
       if (!poisoned) load_q(qbufs + qb * C::QBUF_BYTES);
       __syncwarp();

@@ -348,7 +348,7 @@ def _tiny(seed: int, block_size: int) -> Workload:
 
 def _7b(seed: int, block_size: int, num_seqs: int = 64, num_q_tokens: int = 1) -> Workload:
     rng = np.random.default_rng([seed, _S_LENS])
-    L = rng.integers(128, 2049, size=num_seqs)
+    L = np.maximum(rng.integers(128, 2049, size=num_seqs), num_q_tokens)
     return independent("7b", L, num_q_tokens, **_fp8_kw(dict(num_q_heads=32, num_kv_heads=32, head_dim=128, block_size=block_size,
                                                q_dtype="bf16", kv_dtype="bf16", seed=seed,
                                                notes={"lens": "uniform[128,2048]"})))
@@ -356,7 +356,7 @@ def _7b(seed: int, block_size: int, num_seqs: int = 64, num_q_tokens: int = 1) -
 
 def _13b(seed: int, block_size: int, num_seqs: int = 128, num_q_tokens: int = 1) -> Workload:
     rng = np.random.default_rng([seed, _S_LENS])
-    L = rng.integers(16, 2049, size=num_seqs)
+    L = np.maximum(rng.integers(16, 2049, size=num_seqs), num_q_tokens)
     return independent(f"13b-bs{block_size}", L, num_q_tokens, **_fp8_kw(dict(num_q_heads=40, num_kv_heads=40, head_dim=128,
                                                              block_size=block_size, q_dtype="f16", kv_dtype="f16",
                                                              seed=seed, notes={"lens": "uniform[16,2048]"})))
@@ -370,7 +370,7 @@ def lognormal_lengths(rng: np.random.Generator, n: int, median: float = 1024.0, 
 
 def _8b(seed: int, block_size: int, num_seqs: int = 256, num_q_tokens: int = 1) -> Workload:
     rng = np.random.default_rng([seed, _S_LENS])
-    L = lognormal_lengths(rng, num_seqs)
+    L = np.maximum(lognormal_lengths(rng, num_seqs), num_q_tokens)
     return independent("8b", L, num_q_tokens, **_fp8_kw(dict(num_q_heads=32, num_kv_heads=8, head_dim=128, block_size=block_size,
                                                q_dtype="bf16", kv_dtype="bf16", seed=seed,
                                                notes={"lens": "lognormal(median 1024, sigma 1.0) clipped to "
@@ -409,8 +409,9 @@ def make_config(name: str, block_size: Optional[int] = None, seed: Optional[int]
 
     kv_dtype="e4m3" gives the same config over an FP8 cache (head_dim 128 configs): the
     history is stored as FP8 codes, the step's new tokens stay in the config's dtype.
-    num_q_tokens=T ("7b", "13b", "8b") gives the multi-token step: the same lengths, the last
-    T tokens of every sequence stored in the step and attended to causally by T queries.
+    num_q_tokens=T ("7b", "13b", "8b") gives the multi-token step: the same lengths (raised to T
+    where shorter), the last T tokens of every sequence stored in the step and attended to
+    causally by T queries.
     """
     if name not in _BUILDERS:
         raise KeyError(f"unknown config {name!r}; choose from {CONFIG_NAMES}")

@@ -122,9 +122,10 @@ def multi_call(lib, **kw):
 def test_multi_argument_validation(lib):
     assert multi_call(lib, N=0) == B.PA_OK
     assert multi_call(lib, T=0) == B.PA_ERR_INVALID
-    assert multi_call(lib, T=9) == B.PA_ERR_UNSUPPORTED            # 9 tokens x 4 heads > 32 query rows
-    assert multi_call(lib, D=64) == B.PA_ERR_UNSUPPORTED           # > 8 rows needs head_dim 128
-    assert multi_call(lib, qd=0) == B.PA_ERR_UNSUPPORTED           # > 8 rows needs q_dtype == kv_dtype
+    assert multi_call(lib, T=9) == B.PA_ERR_WORKSPACE              # 36 rows: two column groups of tokens
+    assert multi_call(lib, T=100000) == B.PA_ERR_UNSUPPORTED       # more than 65536 query tokens
+    assert multi_call(lib, D=64) == B.PA_ERR_WORKSPACE             # head_dim 64: groups of 8 rows
+    assert multi_call(lib, qd=0) == B.PA_ERR_UNSUPPORTED           # several tokens need q_dtype == kv_dtype
     assert multi_call(lib, kd=3) == B.PA_ERR_UNSUPPORTED           # FP8 cache
     assert multi_call(lib, T=2, qd=0) == B.PA_ERR_UNSUPPORTED      # several tokens: q_dtype == kv_dtype
     assert multi_call(lib, T=1, qd=0) == B.PA_ERR_WORKSPACE        # one token: pa_decode's dtype pairs

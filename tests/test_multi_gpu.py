@@ -5,6 +5,7 @@ attend causally: query token t of a sequence of L tokens sees positions 0 .. L -
 Tolerances are those of single-token decode (2e-3 with fp16 KV, 1e-2 with bf16 KV, plus
 half an ulp of a 16-bit output): the kernel's arithmetic per (query row, key) is the same.
 Cases cover items of 1 to 4 eight-row query tiles (T x G = 2 .. 32 query rows per KV head),
+sequences with more query rows than an item holds (split into column groups of tokens),
 both block sizes, partition tails that lie wholly after some query tokens' positions (those
 rows see none of the tail partition's keys), empty sequences, sequences of exactly T tokens,
 and an invalid length 0 < L < T.
@@ -75,6 +76,11 @@ CASES = [
     (16, 2, 4, 128, 32, "f16", "f32", 256),    # 32 rows: four tiles, block size 32
     (64, 8, 4, 128, 16, "bf16", "bf16", 0),    # 32 rows (G = 8)
     (32, 8, 8, 128, 32, "bf16", "f32", 128),   # 32 rows, short partitions
+    # more query rows than one item holds: the query tokens are split into column groups
+    (32, 8, 16, 128, 16, "bf16", "f32", 0),    # 64 rows: 2 groups of 8 tokens
+    (64, 8, 9, 128, 16, "bf16", "bf16", 0),    # G = 8: groups of 4, 4 and 1 tokens
+    (8, 8, 40, 128, 32, "f16", "f32", 256),    # MHA: groups of 32 and 8 tokens
+    (8, 2, 11, 64, 16, "bf16", "f32", 0),      # head_dim 64: groups of 2 tokens (8 rows)
 ]
 
 
