@@ -337,11 +337,12 @@ __device__ __forceinline__ void e4m3x4_to_f16x2x2(uint32_t v, uint32_t& lo, uint
       : "r"(v));
 }
 
-__device__ __forceinline__ uint32_t lds_u16(uint32_t addr) {
-  unsigned short v;
-  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(addr));
+__device__ __forceinline__ uint32_t lds_u32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
   return v;
 }
+
 
 // NT: 8-column MMA tiles per consumer warp; PAIR: two consumer warps share each ring, the
 // second taking the item's query rows after the first's 8 * NT (for items of up to 32 rows:
@@ -792,29 +793,36 @@ __global__ void __launch_bounds__(DecodeCfg<BS, D, KT, QT, NT, PAIR, CAUSAL, NR>
           Mma<MA>::run(lacc[nt], ones, ones, ones, ones, b0[nt], b1[nt]);  // row sums of the weights the MMA sees
         }
         if constexpr (C::FP8) {
-          // V^T tile (16 columns x 16 tokens) from the codes: a lane reads the 16-bit column pair
-          // (2 r0, 2 r0 + 1) of tokens 2c, 2c+1, 2c+8, 2c+9 and pairs the tokens up by byte
-          // permutation; accumulator rows r0 / r0 + 8 are columns 2 r0 / 2 r0 + 1.
+          // V^T tiles (16 columns x 16 tokens) from the codes, two MMA steps per load: in step
+          // pair sp a lane reads one 32-bit word -- columns d .. d + 3 with
+          // d = 32 sp + 16 (r0 >> 2) + 4 (r0 & 3) -- of tokens 2c, 2c+1, 2c+8, 2c+9, and pairs
+          // the tokens up by byte permutation: step 2 sp takes columns d, d + 1 (accumulator
+          // rows r0, r0 + 8), step 2 sp + 1 columns d + 2, d + 3.
           const int tk = mt * 16 + c2;
-          const uint32_t row0 = vb + (mt * 16 + c2) * 128 + 2 * r0;
+          const uint32_t rowa = vb + (mt * 16 + c2) * 128 + 4 * (r0 & 3);  // tokens 2c (+8)
+          const uint32_t rowb = rowa + 128;                                  // tokens 2c+1 (+9)
           auto v_tiles = [&](uint32_t mlo, uint32_t mhi, auto masked) {
 #pragma unroll
-            for (int dt = 0; dt < C::KS; ++dt) {
-              const uint32_t u0 = lds_u16(row0 + (((dt ^ vx0)) << 4));
-              const uint32_t u1 = lds_u16(row0 + 128 + (((dt ^ vx1)) << 4));
-              const uint32_t u2 = lds_u16(row0 + 8 * 128 + (((dt ^ vx0)) << 4));
-              const uint32_t u3 = lds_u16(row0 + 9 * 128 + (((dt ^ vx1)) << 4));
-              const uint32_t w01 = __byte_perm(u0, u1, 0x5140), w23 = __byte_perm(u2, u3, 0x5140);
-              uint32_t a0, a1, a2, a3;
-              e4m3x4_to_f16x2x2(w01, a0, a1);
-              e4m3x4_to_f16x2x2(w23, a2, a3);
-              if constexpr (decltype(masked)::value) {
-                a0 &= mlo;
-                a1 &= mlo;
-                a2 &= mhi;
-                a3 &= mhi;
+            for (int sp = 0; sp < C::KS / 2; ++sp) {
+              const int chunk = 2 * sp + (r0 >> 2);  // 16-byte chunk of the row holding the word
+              const uint32_t w0 = lds_u32(rowa + ((chunk ^ vx0) << 4));
+              const uint32_t w1 = lds_u32(rowb + ((chunk ^ vx1) << 4));
+              const uint32_t w2 = lds_u32(rowa + 8 * 128 + ((chunk ^ vx0) << 4));
+              const uint32_t w3 = lds_u32(rowb + 8 * 128 + ((chunk ^ vx1) << 4));
+#pragma unroll
+              for (int h = 0; h < 2; ++h) {
+                const uint32_t sel = h ? 0x7362u : 0x5140u;  // columns d, d+1 or d+2, d+3
+                uint32_t a0, a1, a2, a3;
+                e4m3x4_to_f16x2x2(__byte_perm(w0, w1, sel), a0, a1);
+                e4m3x4_to_f16x2x2(__byte_perm(w2, w3, sel), a2, a3);
+                if constexpr (decltype(masked)::value) {
+                  a0 &= mlo;
+                  a1 &= mlo;
+                  a2 &= mhi;
+                  a3 &= mhi;
+                }
+                Mma<MA>::run(acc[2 * sp + h][0], a0, a1, a2, a3, b0[0], b1[0]);
               }
-              Mma<MA>::run(acc[dt][0], a0, a1, a2, a3, b0[0], b1[0]);
             }
           };
           if (ntok >= (mt + 1) * 16) {
@@ -856,8 +864,11 @@ __global__ void __launch_bounds__(DecodeCfg<BS, D, KT, QT, NT, PAIR, CAUSAL, NR>
   // t * Hq + kvh * G + g.
   auto finalize = [&](int seq, int part, int kvh, bool direct) {
     const float nan = CUDART_NAN_F;
-    // accumulator rows r0 and r0 + 8 of tile dt are columns d and d + dd
+    // accumulator rows r0 and r0 + 8 of tile dt are columns d = vcol(dt) and d + dd
     const int dd = C::FP8 ? 1 : 8;
+    auto vcol = [&](int dt) {
+      return C::FP8 ? 32 * (dt >> 1) + 16 * (r0 >> 2) + 4 * (r0 & 3) + 2 * (dt & 1) : dt * 16 + r0;
+    };
     const float vs = p.v_scale;
     const int HV = T * Hq;
 #pragma unroll
@@ -876,7 +887,7 @@ __global__ void __launch_bounds__(DecodeCfg<BS, D, KT, QT, NT, PAIR, CAUSAL, NR>
           const int64_t o = (static_cast<int64_t>(seq + m) * HV + vh) * D;
 #pragma unroll
           for (int dt = 0; dt < C::KS; ++dt) {
-            const int d = dt * 16 + (C::FP8 ? 2 * r0 : r0);
+            const int d = vcol(dt);
             store_out(p.out, o + d, acc[dt][nt][j] * inv, p.out_dtype);
             store_out(p.out, o + d + dd, acc[dt][nt][2 + j] * inv, p.out_dtype);
           }
@@ -885,7 +896,7 @@ __global__ void __launch_bounds__(DecodeCfg<BS, D, KT, QT, NT, PAIR, CAUSAL, NR>
           float* pa = p.part_acc + (pidx * HV + vh) * D;
 #pragma unroll
           for (int dt = 0; dt < C::KS; ++dt) {
-            const int d = dt * 16 + (C::FP8 ? 2 * r0 : r0);
+            const int d = vcol(dt);
             __stcg(pa + d, poisoned ? nan : acc[dt][nt][j] * vs);
             __stcg(pa + d + dd, poisoned ? nan : acc[dt][nt][2 + j] * vs);
           }
