@@ -40,7 +40,7 @@ from paged_kv_cache_327_b200 import workload as W  # noqa: E402
 
 METRIC = "paged decode attention KV GB/s (% of HBM peak); seq-tokens/s, 8B-GQA decode"
 KERNEL_SOURCES = ["paged_kv_cache_327_b200/csrc/pa_decode.cuh", "paged_kv_cache_327_b200/csrc/pa_ptx.cuh",
-                  "paged_kv_cache_327_b200/csrc/pa_api.cu"]
+                  "paged_kv_cache_327_b200/csrc/pa_decode_tc.cuh", "paged_kv_cache_327_b200/csrc/pa_api.cu"]
 FALLBACK_HBM_GBS = 6650.0
 
 
@@ -66,6 +66,9 @@ def parse_args():
     ap.add_argument("--prefix", action="store_true",
                     help="prefix-aware decode (pa_decode_prefix): sequences sharing their first blocks read them "
                          "once; the groups come from the block tables")
+    ap.add_argument("--wide-kernel", choices=["mma", "tcgen05"], default="mma",
+                    help="kernel for items of more than 8 query rows per KV head (--qtok, --prefix): the warp-MMA "
+                         "kernel (default) or the 5th-generation tensor-core kernel")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target oracle time for cpu_baseline")
     ap.add_argument("--ref-seconds", type=float, default=150.0, help="target total time of --impl reference")
@@ -124,7 +127,8 @@ def profile_name(args) -> str:
     """Name of the committed ncu summary of this run's partition kernel: config, cache dtype and
     query tokens (pa_decode_partition_8b, pa_decode_partition_8b_e4m3, pa_decode_partition_8b_T5)."""
     return (f"pa_decode_partition_{args.config}" + (f"_{args.kv_dtype}" if args.kv_dtype else "")
-            + (f"_T{args.qtok}" if args.qtok > 1 else "") + ("_prefix" if args.prefix else ""))
+            + (f"_T{args.qtok}" if args.qtok > 1 else "") + ("_prefix" if args.prefix else "")
+            + ("_tcgen05" if getattr(args, "wide_kernel", "mma") == "tcgen05" else ""))
 
 
 def recorded_traffic(name: str):
@@ -297,6 +301,7 @@ def run_ours(args):
         print(f"warning: --gpus {args.gpus} but WORLD_SIZE {world}", file=sys.stderr)
     pkg_build.build()
     torch.cuda.set_device(local)
+    B.set_wide_kernel(args.wide_kernel)
     dist = None
     if world > 1:
         import datetime
@@ -522,6 +527,7 @@ def run_ours(args):
                    "seq_tokens_per_step": w.total_tokens(), "new_tokens_per_step": int(len(w.slot_mapping)),
                    "cow_pairs_per_step": int(len(w.copy_pairs)), "out_dtype": out_dtype,
                    "partition_size": args.partition_size or 512,
+                   "wide_kernel": args.wide_kernel if (w.num_q_tokens > 1 or args.prefix) else None,
                    "prefix_groups": (f"{len(groups_np)} groups, {int(groups_np[:, 1].sum())} sequences, shared "
                                      f"tokens {sorted(set(int(x) for x in groups_np[:, 2]))}, max_members "
                                      f"{max_members}") if args.prefix else None,

@@ -245,6 +245,24 @@ PA_API int pa_get_device_error(void* stream);
  * Returns PA_ERR_INVALID for polls out of range, else the launch status. */
 PA_API int pa_selftest_wait_timeout(int polls, void* stream);
 
+/* Process-wide options.
+ *
+ * PA_OPT_WIDE_KERNEL chooses the kernel for work items of more than 8 query rows per KV head (the
+ * query tokens of pa_decode_multi, or the members of a pa_decode_prefix group) on a 16-bit cache
+ * with head_dim 128 and block_size 16:
+ *   PA_WIDE_MMA (default)  the persistent warp-MMA kernel: two consumer warps per ring share
+ *                          each staged page;
+ *   PA_WIDE_TCGEN05        the 5th-generation tensor-core kernel: chunks of 8 pages, S^T = K.Q^T
+ *                          and O^T += V^T.P^T accumulate in tensor memory, one loading warp, one
+ *                          MMA-issuing warp and four softmax warps per CTA.
+ * Both match the same oracle within the attention tolerances; on B200 the first is the faster
+ * of the two for every shape measured.  Other paths ignore the option.
+ * Returns PA_OK, or PA_ERR_INVALID for an unknown option or value (nothing changes then). */
+#define PA_OPT_WIDE_KERNEL 1
+#define PA_WIDE_MMA 0
+#define PA_WIDE_TCGEN05 1
+PA_API int pa_set_option(int option, int value);
+
 /* ABI version of this header (major * 100 + minor). */
 PA_API int pa_version(void);
 

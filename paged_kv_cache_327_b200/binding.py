@@ -26,7 +26,7 @@ PA_OK, PA_ERR_INVALID, PA_ERR_UNSUPPORTED, PA_ERR_WORKSPACE, PA_ERR_CUDA = 0, -1
 EXPORTED = ("pa_decode_workspace_size", "pa_decode", "pa_reshape_and_cache", "pa_copy_blocks",
             "pa_strerror", "pa_get_device_error", "pa_version", "pa_decode_static_workspace",
             "pa_decode_fp8", "pa_reshape_and_cache_fp8", "pa_swap_blocks", "pa_decode_multi", "pa_decode_prefix",
-            "pa_selftest_wait_timeout")
+            "pa_selftest_wait_timeout", "pa_set_option")
 PA_ERR_TOO_LARGE = -5
 PA_DECODE_STATIC_WORKSPACE_BYTES = 64 << 20
 
@@ -76,6 +76,8 @@ def load_library(path: str = _LIB_PATH):
     lib.pa_decode_prefix.restype = I
     lib.pa_selftest_wait_timeout.argtypes = [I, P]
     lib.pa_selftest_wait_timeout.restype = I
+    lib.pa_set_option.argtypes = [I, I]
+    lib.pa_set_option.restype = I
     if path == _LIB_PATH:
         _lib = lib
     return lib
@@ -296,6 +298,22 @@ def pa_swap_blocks(dst_k: torch.Tensor, dst_v: torch.Tensor, src_k: torch.Tensor
 def pa_selftest_wait_timeout(polls: int, stream=None) -> None:
     """Run the library's bounded wait on a barrier nothing completes (see include/pa.h)."""
     _check(load_library().pa_selftest_wait_timeout(int(polls), _stream(stream)), "pa_selftest_wait_timeout")
+
+
+PA_OPT_WIDE_KERNEL = 1
+WIDE_KERNELS = {"mma": 0, "tcgen05": 1}
+
+
+def pa_set_option(option: int, value: int) -> None:
+    """Process-wide library option (see include/pa.h)."""
+    _check(load_library().pa_set_option(int(option), int(value)), "pa_set_option")
+
+
+def set_wide_kernel(name: str) -> None:
+    """Kernel for items of more than 8 query rows per KV head: "mma" (default) or "tcgen05"."""
+    if name not in WIDE_KERNELS:
+        raise ValueError(f"wide kernel must be one of {sorted(WIDE_KERNELS)}, not {name!r}")
+    pa_set_option(PA_OPT_WIDE_KERNEL, WIDE_KERNELS[name])
 
 
 def pa_get_device_error(stream=None) -> int:

@@ -16,6 +16,7 @@
 
 #include "pa.h"
 #include "pa_cache.cuh"
+#include "pa_decode_tc.cuh"
 
 namespace {
 
@@ -154,6 +155,38 @@ int launch_partition(const pa::DecodeParams& p, const CUtensorMap& tmk, const CU
   return cudaPeekAtLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
+// The tensor-core kernel for wide items (block size 16, head_dim 128, 16-bit cache and query).
+// kernel for items of more than 8 query rows (PA_OPT_WIDE_KERNEL)
+std::atomic<int> g_wide_kernel{PA_WIDE_MMA};
+
+template <typename KT, int N>
+int launch_tc(const pa::DecodeParams& p, const CUtensorMap& tmk, const CUtensorMap& tmv, int64_t max_items,
+              int dev, DeviceInfo* info, cudaStream_t stream) {
+  using C = pa::TcCfg<KT, N>;
+  auto kern = pa::pa_decode_tc_kernel<KT, N, true>;
+  static std::atomic<bool> smem_set[kMaxDevices];
+  if (!smem_set[dev].load(std::memory_order_acquire)) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
+      return PA_ERR_CUDA;
+    smem_set[dev].store(true, std::memory_order_release);
+  }
+  int64_t ctas = max_items;  // one ring (and one CTA) per SM
+  if (ctas > info->sm_count) ctas = info->sm_count;
+  if (ctas < 1) ctas = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(ctas));
+  cfg.blockDim = dim3(C::NTHREADS);
+  cfg.dynamicSmemBytes = C::SMEM_BYTES;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kern, tmk, tmv, p) != cudaSuccess) return PA_ERR_CUDA;
+  return cudaPeekAtLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
 // Kernel instantiation for (block_size, head_dim, KV dtype, query dtype, query rows per item,
 // several query tokens): single-token items of up to 8 query rows run on every dtype pair with one
 // consumer warp per ring; multi-token items of up to 8 rows on a 16-bit cache with a query of the
@@ -186,6 +219,16 @@ int dispatch_kv(const pa::DecodeParams& p, const CUtensorMap& tmk, const CUtenso
     return PA_ERR_UNSUPPORTED;
   }
   if (nt > 1) {
+    if constexpr (D == 128 && BS == 16) {  // 5th-generation tensor-core kernel, when chosen
+      if (g_wide_kernel.load(std::memory_order_relaxed) == PA_WIDE_TCGEN05) {
+        if (kv_dtype == PA_BF16 && q_dtype == PA_BF16)
+          return cols <= 16 ? launch_tc<bf16, 16>(p, tmk, tmv, max_items, dev, info, stream)
+                            : launch_tc<bf16, 32>(p, tmk, tmv, max_items, dev, info, stream);
+        if (kv_dtype == PA_F16 && q_dtype == PA_F16)
+          return cols <= 16 ? launch_tc<f16, 16>(p, tmk, tmv, max_items, dev, info, stream)
+                            : launch_tc<f16, 32>(p, tmk, tmv, max_items, dev, info, stream);
+      }
+    }
     if constexpr (D == 128) {
       if (kv_dtype == PA_BF16 && q_dtype == PA_BF16)
         return nt == 2 ? run(bf16{}, bf16{}, One{}, Yes{}, Yes{}) : run(bf16{}, bf16{}, Two{}, Yes{}, Yes{});
@@ -209,6 +252,14 @@ int dispatch_kv(const pa::DecodeParams& p, const CUtensorMap& tmk, const CUtenso
 }  // namespace
 
 extern "C" {
+
+int pa_set_option(int option, int value) {
+  if (option == PA_OPT_WIDE_KERNEL && (value == PA_WIDE_MMA || value == PA_WIDE_TCGEN05)) {
+    g_wide_kernel.store(value, std::memory_order_relaxed);
+    return PA_OK;
+  }
+  return PA_ERR_INVALID;
+}
 
 int pa_version(void) { return 100; }
 

@@ -410,6 +410,127 @@ __device__ __forceinline__ uint32_t swz(int t, int d0) {
 // [1] x = the item's first query token t0
 constexpr int F_FIRST = 1, F_LAST = 2, F_BAD = 4, F_END = 8, F_DIRECT = 16;
 
+// The producer warp of one ring: takes work items from the shared counter and streams their pages
+// (K and V of one KV head, by TMA) and query rows (bulk copies) into the ring's slots, with each
+// slot's metadata; ends the stream with an F_END slot.  C gives the slot geometry.
+template <class C, int BS, int D>
+__device__ __forceinline__ void produce(const DecodeParams& p, const CUtensorMap& tmk, const CUtensorMap& tmv,
+                                        uint8_t* ring, uint8_t* qbufs, uint64_t* full, uint64_t* empty,
+                                        uint64_t* qfree, int4* meta, volatile int* abort_flag, int lane) {
+  constexpr unsigned FULL = 0xffffffffu;
+  const int G = p.group, Hkv = p.num_kv_heads, Hq = p.num_q_heads, T = p.qtok;
+  const unsigned total = p.counters[1] * static_cast<unsigned>(Hkv);
+  const uint64_t pol = policy_evict_first();
+  uint32_t n = 0;      // pages issued into this ring
+  uint32_t items = 0;  // items started (the query buffer is refilled once per item)
+  bool stop = false;
+  auto acquire_slot = [&](int slot) -> bool {  // wait until the consumer freed `slot`
+    if (n < C::NSLOT) return true;
+    const bool ok = mbar_wait_bounded(&empty[slot], ((n / C::NSLOT) - 1) & 1u, kWaitLimit);
+    return __all_sync(FULL, ok) && !*abort_flag;
+  };
+  while (!stop) {
+    unsigned w = 0;
+    if (lane == 0) w = atomicAdd(&p.counters[0], 1u);
+    w = __shfl_sync(FULL, w, 0);
+    if (w >= total) break;
+    const WorkItem it = p.items[w / Hkv];
+    const int kvh = static_cast<int>(w % Hkv);
+    const int part = it.pm & 0xffff, members = (it.pm >> 16) & 0xff;
+    const int tok0 = it.tok0, tok1 = it.tok1;
+    const int npages = (tok1 - tok0 + BS - 1) / BS;
+    const int t0 = it.t0, tq = it.tq;
+    const int rows = members * tq;  // (member, query token) pairs of the item: G query rows each
+    // key positions relative to the item's first query token, at position len - T + t0
+    // (causal masking of several query tokens)
+    const int rel0 = T > 1 ? tok0 - (p.seq_lens[it.seq] - T + t0) : 0;
+    int bt = 0;
+    bool bad = false, mismatch = false;
+    if (lane < npages) {
+      const int64_t col = tok0 / BS + lane;
+      bt = p.block_tables[static_cast<int64_t>(it.seq) * p.max_blocks_per_seq + col];
+      bad = bt < 0 || bt >= p.num_blocks;
+      // the members of a shared item must hold the same blocks
+      for (int m = 1; m < members; ++m)
+        mismatch |= p.block_tables[static_cast<int64_t>(it.seq + m) * p.max_blocks_per_seq + col] != bt;
+    }
+    bad = __any_sync(FULL, bad);
+    mismatch = __any_sync(FULL, mismatch);
+    if (lane == 0) {
+      if (bad) record_error(DEV_BAD_BLOCK_ID);
+      if (mismatch) record_error(DEV_BAD_PREFIX);
+    }
+    bad |= mismatch;
+    const uint32_t qb = items % C::QN;
+    if (items >= C::QN) {  // the consumers have taken the query rows of item `items - QN`
+      const bool ok = mbar_wait_bounded(&qfree[qb], ((items / C::QN) - 1) & 1u, kWaitLimit);
+      if (!__all_sync(FULL, ok) || *abort_flag) {
+        stop = true;
+        break;
+      }
+    }
+    for (int pg = 0; pg < npages; ++pg) {
+      const int phys = __shfl_sync(FULL, bt, pg);
+      const int slot = static_cast<int>(n % C::NSLOT);
+      if (!acquire_slot(slot)) {
+        stop = true;
+        break;
+      }
+      const bool first = pg == 0;
+      if (lane == 0) {
+        uint8_t* sb = ring + slot * C::SLOT_BYTES;
+        const int ntok = min(BS, tok1 - (tok0 + pg * BS));
+        const int flags = (first ? F_FIRST : 0) | (pg == npages - 1 ? F_LAST : 0) | (bad ? F_BAD : 0) |
+                          ((it.pm & WI_DIRECT) ? F_DIRECT : 0);
+        meta[2 * slot] = make_int4(it.seq, part | (pg << 16), kvh | (ntok << 8) | (rows << 16) | (flags << 24),
+                                   rel0 + pg * BS);
+        meta[2 * slot + 1] = make_int4(t0, 0, 0, 0);
+        if (bad) {
+          mbar_arrive(&full[slot]);
+        } else {
+          const uint32_t qbytes = first ? static_cast<uint32_t>(rows * G * D * C::QE) : 0u;
+          mbar_arrive_expect_tx(&full[slot], 2 * C::PAGE_BYTES + qbytes);
+#pragma unroll
+          for (int h = 0; h < C::HALVES; ++h) {
+            tma_load_3d(sb + h * C::BOX_BYTES, &tmk, 0, kvh * C::HALVES + h, phys * BS, &full[slot], pol);
+            tma_load_3d(sb + C::PAGE_BYTES + h * C::BOX_BYTES, &tmv, 0, kvh * C::HALVES + h, phys * BS,
+                        &full[slot], pol);
+          }
+        }
+      }
+      if (first && !bad) {
+        __syncwarp();  // the expected byte count is set before any copy can complete
+        if (lane < rows) {  // query rows of (member, token) lane: G contiguous heads
+          const int m = lane / tq, t = t0 + lane - m * tq;
+          bulk_load(qbufs + qb * C::QBUF_BYTES + lane * G * D * C::QE,
+                    static_cast<const uint8_t*>(p.q) +
+                        ((static_cast<int64_t>(it.seq + m) * T + t) * Hq + kvh * G) * D * C::QE,
+                    static_cast<uint32_t>(G * D * C::QE), &full[slot]);
+        }
+      }
+      ++n;
+    }
+    ++items;
+  }
+  if (!stop) {  // tell the consumer there is no more work
+    const int slot = static_cast<int>(n % C::NSLOT);
+    if (acquire_slot(slot)) {
+      if (lane == 0) {
+        meta[2 * slot] = make_int4(0, 0, F_END << 24, 0);
+        mbar_arrive(&full[slot]);
+      }
+    } else {
+      stop = true;
+    }
+  }
+  if (stop) {
+    if (lane == 0) record_error(DEV_TIMEOUT);
+    // copies this warp issued may still be landing: wait for them before the CTA exits
+    for (uint32_t k = n > C::NSLOT ? n - C::NSLOT : 0; k < n; ++k)
+      mbar_wait_bounded(&full[k % C::NSLOT], (k / C::NSLOT) & 1u, kWaitLimit);
+  }
+}
+
 // The query rows ("columns") of one work item are (member m, query token t, head g) for
 // m < members, t < qtok, g < G, in that order: column c = (m * qtok + t) * G + g.  A plain decode
 // has one member and one query token; multi-token attention has qtok > 1 (query token t sits at
@@ -450,121 +571,12 @@ __global__ void __launch_bounds__(DecodeCfg<BS, D, KT, QT, NT, PAIR, CAUSAL, NR>
   __syncthreads();
   pdl_wait();  // the plan kernel's work list and counters are visible from here on
 
-  const int G = p.group, Hkv = p.num_kv_heads, Hq = p.num_q_heads, T = p.qtok;
+  const int G = p.group, Hq = p.num_q_heads, T = p.qtok;
 
   if (warp >= C::NCONS) {
     // ============================== producer ==============================
     if constexpr (C::SPLIT) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(C::REG_PRODUCER));
-    const unsigned total = p.counters[1] * static_cast<unsigned>(Hkv);
-    const uint64_t pol = policy_evict_first();
-    uint32_t n = 0;      // pages issued into this ring
-    uint32_t items = 0;  // items started (the query buffer is refilled once per item)
-    bool stop = false;
-    auto acquire_slot = [&](int slot) -> bool {  // wait until the consumer freed `slot`
-      if (n < C::NSLOT) return true;
-      const bool ok = mbar_wait_bounded(&empty[slot], ((n / C::NSLOT) - 1) & 1u, kWaitLimit);
-      return __all_sync(FULL, ok) && !*abort_flag;
-    };
-    while (!stop) {
-      unsigned w = 0;
-      if (lane == 0) w = atomicAdd(&p.counters[0], 1u);
-      w = __shfl_sync(FULL, w, 0);
-      if (w >= total) break;
-      const WorkItem it = p.items[w / Hkv];
-      const int kvh = static_cast<int>(w % Hkv);
-      const int part = it.pm & 0xffff, members = (it.pm >> 16) & 0xff;
-      const int tok0 = it.tok0, tok1 = it.tok1;
-      const int npages = (tok1 - tok0 + BS - 1) / BS;
-      const int t0 = it.t0, tq = it.tq;
-      const int rows = members * tq;  // (member, query token) pairs of the item: G query rows each
-      // key positions relative to the item's first query token, at position len - T + t0
-      // (causal masking of several query tokens)
-      const int rel0 = T > 1 ? tok0 - (p.seq_lens[it.seq] - T + t0) : 0;
-      int bt = 0;
-      bool bad = false, mismatch = false;
-      if (lane < npages) {
-        const int64_t col = tok0 / BS + lane;
-        bt = p.block_tables[static_cast<int64_t>(it.seq) * p.max_blocks_per_seq + col];
-        bad = bt < 0 || bt >= p.num_blocks;
-        // the members of a shared item must hold the same blocks
-        for (int m = 1; m < members; ++m)
-          mismatch |= p.block_tables[static_cast<int64_t>(it.seq + m) * p.max_blocks_per_seq + col] != bt;
-      }
-      bad = __any_sync(FULL, bad);
-      mismatch = __any_sync(FULL, mismatch);
-      if (lane == 0) {
-        if (bad) record_error(DEV_BAD_BLOCK_ID);
-        if (mismatch) record_error(DEV_BAD_PREFIX);
-      }
-      bad |= mismatch;
-      const uint32_t qb = items % C::QN;
-      if (items >= C::QN) {  // the consumers have taken the query rows of item `items - QN`
-        const bool ok = mbar_wait_bounded(&qfree[qb], ((items / C::QN) - 1) & 1u, kWaitLimit);
-        if (!__all_sync(FULL, ok) || *abort_flag) {
-          stop = true;
-          break;
-        }
-      }
-      for (int pg = 0; pg < npages; ++pg) {
-        const int phys = __shfl_sync(FULL, bt, pg);
-        const int slot = static_cast<int>(n % C::NSLOT);
-        if (!acquire_slot(slot)) {
-          stop = true;
-          break;
-        }
-        const bool first = pg == 0;
-        if (lane == 0) {
-          uint8_t* sb = ring + slot * C::SLOT_BYTES;
-          const int ntok = min(BS, tok1 - (tok0 + pg * BS));
-          const int flags = (first ? F_FIRST : 0) | (pg == npages - 1 ? F_LAST : 0) | (bad ? F_BAD : 0) |
-                            ((it.pm & WI_DIRECT) ? F_DIRECT : 0);
-          meta[2 * slot] = make_int4(it.seq, part | (pg << 16), kvh | (ntok << 8) | (rows << 16) | (flags << 24),
-                                     rel0 + pg * BS);
-          meta[2 * slot + 1] = make_int4(t0, 0, 0, 0);
-          if (bad) {
-            mbar_arrive(&full[slot]);
-          } else {
-            const uint32_t qbytes = first ? static_cast<uint32_t>(rows * G * D * C::QE) : 0u;
-            mbar_arrive_expect_tx(&full[slot], 2 * C::PAGE_BYTES + qbytes);
-#pragma unroll
-            for (int h = 0; h < C::HALVES; ++h) {
-              tma_load_3d(sb + h * C::BOX_BYTES, &tmk, 0, kvh * C::HALVES + h, phys * BS, &full[slot], pol);
-              tma_load_3d(sb + C::PAGE_BYTES + h * C::BOX_BYTES, &tmv, 0, kvh * C::HALVES + h, phys * BS,
-                          &full[slot], pol);
-            }
-          }
-        }
-        if (first && !bad) {
-          __syncwarp();  // the expected byte count is set before any copy can complete
-          if (lane < rows) {  // query rows of (member, token) lane: G contiguous heads
-            const int m = lane / tq, t = t0 + lane - m * tq;
-            bulk_load(qbufs + qb * C::QBUF_BYTES + lane * G * D * C::QE,
-                      static_cast<const uint8_t*>(p.q) +
-                          ((static_cast<int64_t>(it.seq + m) * T + t) * Hq + kvh * G) * D * C::QE,
-                      static_cast<uint32_t>(G * D * C::QE), &full[slot]);
-          }
-        }
-        ++n;
-      }
-      ++items;
-    }
-    if (!stop) {  // tell the consumer there is no more work
-      const int slot = static_cast<int>(n % C::NSLOT);
-      if (acquire_slot(slot)) {
-        if (lane == 0) {
-          meta[2 * slot] = make_int4(0, 0, F_END << 24, 0);
-          mbar_arrive(&full[slot]);
-        }
-      } else {
-        stop = true;
-      }
-    }
-    if (stop) {
-      if (lane == 0) record_error(DEV_TIMEOUT);
-      // copies this warp issued may still be landing: wait for them before the CTA exits
-      for (uint32_t k = n > C::NSLOT ? n - C::NSLOT : 0; k < n; ++k)
-        mbar_wait_bounded(&full[k % C::NSLOT], (k / C::NSLOT) & 1u, kWaitLimit);
-    }
+    produce<C, BS, D>(p, tmk, tmv, ring, qbufs, full, empty, qfree, meta, abort_flag, lane);
     return;
   }
 

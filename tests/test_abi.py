@@ -169,3 +169,16 @@ def test_prefix_argument_validation(lib):
 def test_selftest_argument_checks(lib):
     assert lib.pa_selftest_wait_timeout(0, ctypes.c_void_p(0)) == B.PA_ERR_INVALID
     assert lib.pa_selftest_wait_timeout((1 << 20) + 1, ctypes.c_void_p(0)) == B.PA_ERR_INVALID
+
+
+def test_set_option(lib):
+    """The wide-kernel option takes its two values and rejects others (no GPU needed)."""
+    assert lib.pa_set_option(B.PA_OPT_WIDE_KERNEL, 1) == B.PA_OK
+    assert lib.pa_set_option(B.PA_OPT_WIDE_KERNEL, 0) == B.PA_OK
+    assert lib.pa_set_option(B.PA_OPT_WIDE_KERNEL, 2) == B.PA_ERR_INVALID
+    assert lib.pa_set_option(B.PA_OPT_WIDE_KERNEL, -1) == B.PA_ERR_INVALID
+    assert lib.pa_set_option(0, 0) == B.PA_ERR_INVALID
+    with pytest.raises(ValueError):
+        B.set_wide_kernel("wgmma")
+    B.set_wide_kernel("tcgen05")
+    B.set_wide_kernel("mma")

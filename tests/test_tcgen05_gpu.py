@@ -1,0 +1,134 @@
+"""The 5th-generation tensor-core kernel for wide work items (PA_WIDE_TCGEN05) vs the fp64 oracle.
+
+Items of more than 8 query rows per KV head (several query tokens, or the members of a shared
+prefix) on a 16-bit cache with head_dim 128 and block size 16 run on this kernel once
+pa_set_option(PA_OPT_WIDE_KERNEL, PA_WIDE_TCGEN05) is called.  The cases mirror the warp-MMA
+kernel's: 9..32 query rows (N = 16 and N = 32 instantiations), column groups, short partitions
+(one chunk of 8 pages) and long ones (several chunks, a ragged last chunk and page), empty
+sequences, causal tails, shared prefixes, a bad block id and members whose tables differ.
+Tolerances are the attention ones (2e-3 with fp16 KV, 1e-2 with bf16 KV, plus half an ulp of a
+16-bit output).
+"""
+import numpy as np
+import pytest
+import torch
+
+from paged_kv_cache_327_b200 import binding as B
+from paged_kv_cache_327_b200 import block_manager as BM
+from paged_kv_cache_327_b200 import workload as W
+from tests import test_multi_gpu as TM
+from tests import test_prefix_gpu as TP
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _tcgen05_kernel():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    B.load_library()
+    B.set_wide_kernel("tcgen05")
+    yield
+    B.set_wide_kernel("mma")
+
+
+MULTI = [
+    # Hq, Hkv, T, D, bs, q_dtype, out_dtype, partition   (query rows per item = T * Hq / Hkv)
+    (32, 8, 3, 128, 16, "bf16", "bf16", 0),    # 12 rows: N = 16
+    (16, 4, 4, 128, 16, "f16", "f16", 0),      # 16 rows, fp16
+    (32, 8, 5, 128, 16, "bf16", "f32", 0),     # 20 rows: N = 32
+    (64, 8, 4, 128, 16, "bf16", "bf16", 0),    # 32 rows (G = 8)
+    (32, 8, 8, 128, 16, "bf16", "f32", 128),   # 32 rows, one chunk per partition
+    (32, 8, 16, 128, 16, "bf16", "f32", 0),    # 64 rows: 2 column groups of 8 tokens
+    (64, 8, 9, 128, 16, "bf16", "bf16", 0),    # G = 8: column groups of 4, 4 and 1 tokens
+    (8, 8, 40, 128, 16, "f16", "f32", 256),    # MHA: column groups of 32 and 8 tokens, 2 chunks per partition
+]
+
+
+@pytest.mark.parametrize("case", MULTI, ids=lambda c: "-".join(map(str, c)))
+def test_multi_matches_oracle(case):
+    Hq, Hkv, T, D, bs, qd, od, P = case
+    lens = TM.lens_for(T)
+    w = W.independent("multi", lens, num_q_tokens=T, num_q_heads=Hq, num_kv_heads=Hkv, head_dim=D, block_size=bs,
+                      q_dtype=qd, kv_dtype=qd, seed=4700 + MULTI.index(case))
+    dw, out = TM.gpu_multi(w, od, P)
+    assert B.pa_get_device_error() == B.PA_DEV_OK
+    _, ref, _, _ = TM.oracle_multi(w)
+    got = out.float().cpu().numpy()
+    TM.assert_close(got, ref, qd, od, f"case {case}")
+    assert np.all(got[lens.index(0)] == 0.0), "an empty sequence gives zero rows"
+
+
+def test_multi_8b_full_size():
+    """The 8B-shaped batch (256 sequences, lognormal lengths) with T = 5: sampled sequences
+    against the oracle, every row finite, and every row within tolerance of the warp-MMA kernel."""
+    w = W.make_config("8b", num_q_tokens=5)
+    dw, out = TM.gpu_multi(w, "bf16")
+    assert B.pa_get_device_error() == B.PA_DEV_OK
+    rng = np.random.default_rng(85)
+    L = w.seq_lens
+    seqs = sorted({int(np.argmax(L)), int(np.argmin(L))} | set(int(i) for i in rng.choice(w.num_seqs, 10,
+                                                                                              replace=False)))
+    idx, ref, _, _ = TM.oracle_multi(w, seqs)
+    TM.assert_close(out.float().cpu().numpy()[idx], ref, w.kv_dtype, "bf16", "8b T=5")
+    assert torch.isfinite(out.float()).all()
+    # the same decode (the cache already holds the step's tokens) on both kernels
+    ws = B.DecodeWorkspace.for_workload(dw)
+    a = torch.empty_like(out, dtype=torch.float32)
+    b = torch.empty_like(a)
+    B.pa_decode_multi(a, dw.q, dw.k_cache, dw.v_cache, dw.block_tables, dw.seq_lens, w.scale, ws.tensor)
+    B.set_wide_kernel("mma")
+    try:
+        B.pa_decode_multi(b, dw.q, dw.k_cache, dw.v_cache, dw.block_tables, dw.seq_lens, w.scale, ws.tensor)
+    finally:
+        B.set_wide_kernel("tcgen05")
+    torch.cuda.synchronize()
+    assert float((a - b).abs().max()) <= 2 * TM.TOL[w.kv_dtype]
+
+
+def test_multi_is_deterministic():
+    w = W.make_config("8b", num_seqs=24, num_q_tokens=4)
+    dw, a = TM.gpu_multi(w)
+    ws = B.DecodeWorkspace.for_workload(dw)
+    b = torch.empty_like(a)
+    B.pa_decode_multi(b, dw.q, dw.k_cache, dw.v_cache, dw.block_tables, dw.seq_lens, w.scale, ws.tensor)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)
+
+
+def test_bad_block_id_poisons_only_its_sequence():
+    T = 4
+    w = W.independent("bad", [40, 700, 1300, 20], num_q_tokens=T, num_q_heads=32, num_kv_heads=8, head_dim=128,
+                      block_size=16, q_dtype="bf16", kv_dtype="bf16", seed=4790)
+    dw = B.device_workload(w)
+    dw.block_tables[2, 40] = w.num_blocks + 5   # in the sequence's second partition
+    out = torch.zeros((4, T, 32, 128), dtype=torch.float32, device="cuda")
+    ws = B.DecodeWorkspace.for_workload(dw)
+    B.run_step(dw, out, ws)
+    assert B.pa_get_device_error() == B.PA_DEV_BAD_BLOCK_ID
+    assert torch.isnan(out[2]).all()
+    assert torch.isfinite(out[[0, 1, 3]]).all()
+
+
+@pytest.mark.parametrize("case", [c for c in TP.CASES if c[2] == 16 and c[3] != "f32"],
+                         ids=lambda c: "-".join(map(str, c[:7])))
+def test_prefix_decode_matches_oracle(case):
+    Hq, Hkv, bs, qd, od, P, mm, spec = case
+    kvd = qd
+    groups = [W.Group(p, st) for p, st in spec]
+    w = W.build_groups("prefix", groups, num_q_heads=Hq, num_kv_heads=Hkv, head_dim=128, block_size=bs, q_dtype=qd,
+                       kv_dtype=kvd, seed=5100 + TP.CASES.index(case))
+    pg = BM.find_prefix_groups(w.block_tables, w.seq_lens, bs)
+    dw, kc, vc = TP.stepped(w)
+    out = TP.prefix_decode(w, dw, pg, mm, od, P)
+    assert B.pa_get_device_error() == B.PA_DEV_OK
+    _, ref = TP.oracle_decode(w, kc, vc)
+    TP.assert_close(out.float().cpu().numpy(), ref, kvd, od, f"case {case[:7]}")
+
+
+def test_prefix_70b_batch():
+    TP.test_prefix_70b_batch_matches_decode_and_oracle()
+
+
+def test_prefix_members_with_different_tables_get_nan():
+    TP.test_members_with_different_tables_get_nan()
