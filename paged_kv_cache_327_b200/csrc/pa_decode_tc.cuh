@@ -15,11 +15,13 @@
 //                     A = the staged V page read in place (MN-major), B = P^T in shared memory
 // At the item's end the partial row sums are reduced across the 128 threads and thread d writes
 // element d of every output row (coalesced).  The MMAs are issued by one thread and complete on
-// mbarriers; the O product also releases the chunk's buffer to the producer.
+// mbarriers; the O product also releases the chunk's buffer to the producer.  The warp-MMA kernel
+// of pa_decode.cuh is the default for these items (faster on B200); this one is chosen with
+// pa_set_option(PA_OPT_WIDE_KERNEL, PA_WIDE_TCGEN05).
 //
-// CTA: one ring of 3 chunk buffers (64 KB each); warps 0-3 consume (TMEM lane quarters 0-3),
-// warp 4 produces (TMA for K/V, plain loads for the query rows).  Block size 16, head_dim 128,
-// 16-bit cache and query.
+// CTA (one per SM): 3 chunk buffers of 64 KB; warps 0-3 run the softmax and the output (TMEM lane
+// quarters 0-3), warp 4 produces (the work list, TMA for K/V, plain loads for the query rows),
+// warp 5 issues every MMA.  Block size 16, head_dim 128, 16-bit cache and query.
 #pragma once
 
 #include "pa_decode.cuh"
@@ -50,15 +52,6 @@ __device__ __forceinline__ void umma_ss(uint32_t d_tmem, uint64_t a_desc, uint64
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
-// D[tmem] = A[tmem] . B[smem] (+ D when accumulate)
-__device__ __forceinline__ void umma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
-                                        uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
 // the mbarrier gets one arrival when every tcgen05 operation this thread issued before has completed
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
@@ -79,11 +72,6 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16
       "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]),
       "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
       : "memory");
-}
-__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&v)[8]) {
-  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
-               "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
-               : "memory");
 }
 
 // Shared-memory matrix descriptor (sm_100): start address, leading / stride byte offsets (all in
