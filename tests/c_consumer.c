@@ -41,6 +41,11 @@ int main(void) {
                          PA_BF16, PA_BF16, 0, ifake, 1, 5, fake, 0, NULL) == PA_ERR_UNSUPPORTED); /* 40 rows */
   CHECK(pa_copy_blocks(fake, fake, ifake, 1, 10, 4008, NULL, NULL) == PA_ERR_INVALID); /* not 16-byte units */
   CHECK(pa_selftest_wait_timeout(0, NULL) == PA_ERR_INVALID);
+  /* the wide-item kernel option: its two values, nothing else */
+  CHECK(pa_set_option(PA_OPT_WIDE_KERNEL, PA_WIDE_TCGEN05) == PA_OK);
+  CHECK(pa_set_option(PA_OPT_WIDE_KERNEL, PA_WIDE_MMA) == PA_OK);
+  CHECK(pa_set_option(PA_OPT_WIDE_KERNEL, 7) == PA_ERR_INVALID);
+  CHECK(pa_set_option(99, PA_WIDE_MMA) == PA_ERR_INVALID);
   puts("ok");
   return 0;
 }
