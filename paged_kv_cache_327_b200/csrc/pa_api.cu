@@ -1,7 +1,8 @@
 // pa_api.cu -- the C ABI of libpa.so (declared in include/pa.h): host-side validation,
 // workspace layout, TMA descriptor encoding and kernel launches.  Every step of the
 // computation runs in the CUDA kernels of pa_decode.cuh / pa_cache.cuh; there is no CPU
-// fallback.  The library allocates no device memory.
+// fallback.  No call allocates device memory: the library's only device memory is static (the
+// error word and the fixed scratch buffer of pa_decode_static_workspace).
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
@@ -40,8 +41,26 @@ int64_t max_parts_for(int64_t max_len, int P, bool groups = true) {
   return std::max<int64_t>(1, (max_len + P - 1) / P + (groups ? 1 : 0));
 }
 
-// num_q_heads: query heads x query tokens.  Items: one per (sequence, partition, column group);
-// a column group holds at least a sixteenth of the query rows, hence the factor.
+// Query rows one work item holds per KV head: 32 with head_dim 128, 8 with head_dim 64.
+int max_item_rows(int head_dim) { return head_dim == 128 ? 32 : 8; }
+
+// Query tokens of one work item (a column group): all qtok when their G rows per token fit one
+// item, otherwise as many whole tokens as fit (at least one).
+int qtok_per_item(int qtok, int G, int head_dim) {
+  const int max_rows = max_item_rows(head_dim);
+  return qtok * G <= max_rows ? qtok : std::max(1, max_rows / G);
+}
+
+// Work items of one partition of one sequence, bounded from num_q_heads (= query tokens x query
+// heads) alone.  A split item holds floor(max_rows / G) * G >= 28 rows with head_dim 128 and
+// >= 5 with head_dim 64 (G <= 8), so ceil(num_q_heads / 16), resp. ceil(num_q_heads / 4), items
+// cover every column group; an unsplit partition has one item.
+int64_t items_per_partition_bound(int64_t num_q_heads, int64_t head_dim) {
+  const int64_t min_rows = head_dim == 128 ? 16 : 4;
+  return std::max<int64_t>(1, (num_q_heads + min_rows - 1) / min_rows);
+}
+
+// num_q_heads: query heads x query tokens.  Items: one per (sequence, partition, column group).
 WsLayout ws_layout(int64_t num_seqs, int64_t num_q_heads, int64_t head_dim, int64_t max_parts) {
   WsLayout L{};
   size_t o = 0;
@@ -54,7 +73,8 @@ WsLayout ws_layout(int64_t num_seqs, int64_t num_q_heads, int64_t head_dim, int6
   L.seq_sub = o;
   o += align256(static_cast<size_t>(num_seqs) * sizeof(int));
   L.items = o;
-  o += align256(static_cast<size_t>(num_seqs * max_parts * ((num_q_heads + 15) / 16)) * sizeof(pa::WorkItem));
+  o += align256(static_cast<size_t>(num_seqs * max_parts * items_per_partition_bound(num_q_heads, head_dim)) *
+                sizeof(pa::WorkItem));
   L.part_ml = o;
   o += align256(static_cast<size_t>(num_seqs * max_parts * num_q_heads) * sizeof(float2));
   L.part_acc = o;
@@ -310,8 +330,7 @@ int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cac
   if (qtok > 65536 || static_cast<int64_t>(qtok) * num_q_heads * head_dim > INT_MAX) return PA_ERR_UNSUPPORTED;
   // query tokens per item: all of them, or column groups of up to 32 query rows per KV head
   // (8 with head_dim 64, whose items run on the one-consumer kernels)
-  const int max_rows = head_dim == 128 ? 32 : 8;
-  const int qtok_item = qtok * G <= max_rows ? qtok : std::max(1, max_rows / G);
+  const int qtok_item = qtok_per_item(qtok, G, head_dim);
   // an item holds qtok_item * G (or max_members * G) query rows: up to 8 on every dtype pair, up to
   // 32 on a 16-bit cache with a query of its own type and head_dim 128
   const int64_t cols = static_cast<int64_t>(qtok_item) * max_members * G;
@@ -342,6 +361,12 @@ int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cac
   // partial results are kept per (query token, query head): the workspace of qtok * num_q_heads heads
   const WsLayout L = ws_layout(num_seqs, static_cast<int64_t>(qtok) * num_q_heads, head_dim, max_parts);
   if (!workspace || workspace_bytes < L.total) return PA_ERR_WORKSPACE;
+  // the plan writes up to num_seqs * max_parts * ncg items (shared items of prefix groups take
+  // partitions of their leader): they must fit the region the layout reserved for them
+  const int64_t ncg = (qtok + qtok_item - 1) / qtok_item;
+  if (static_cast<int64_t>(num_seqs) * max_parts * ncg * static_cast<int64_t>(sizeof(pa::WorkItem)) >
+      static_cast<int64_t>(L.part_ml - L.items))
+    return PA_ERR_WORKSPACE;
   if (reinterpret_cast<uintptr_t>(workspace) & 255u) return PA_ERR_INVALID;
 
   int dev;
@@ -389,8 +414,7 @@ int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cac
   pa::pa_decode_plan_kernel<<<1, pa::kPlanThreads, 0, st>>>(p);
   if (cudaPeekAtLastError() != cudaSuccess) return PA_ERR_CUDA;
 
-  const int64_t max_items =
-      static_cast<int64_t>(num_seqs) * max_parts * ((qtok + qtok_item - 1) / qtok_item) * num_kv_heads;
+  const int64_t max_items = static_cast<int64_t>(num_seqs) * max_parts * ncg * num_kv_heads;
   int rc;
   const int c = static_cast<int>(cols);
   if (block_size == 16)

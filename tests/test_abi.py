@@ -182,3 +182,24 @@ def test_set_option(lib):
         B.set_wide_kernel("wgmma")
     B.set_wide_kernel("tcgen05")
     B.set_wide_kernel("mma")
+
+
+def test_workspace_reserves_every_work_item(lib):
+    """Every multi-token shape that the library accepts fits its work list in the workspace that
+    pa_decode_workspace_size() advertises.  The library refuses (PA_ERR_WORKSPACE) a call whose
+    plan could write more work items than the layout reserved, so a call that passes every host
+    check reaches the device lookup, which fails here without a GPU (PA_ERR_CUDA).  The grid
+    includes the shapes whose column groups hold only 5 to 8 query rows (head_dim 64, few KV
+    heads), the worst case for the reservation."""
+    checked = 0
+    for D in (64, 128):
+        for Hkv in (1, 2, 3):
+            for G in range(1, 9):
+                for T in list(range(1, 41)) + [64, 100, 1000]:
+                    for N, MB in ((1, 1), (3, 8), (64, 130)):
+                        need = B.pa_decode_workspace_size(N, T * G * Hkv, D, MB * 16)
+                        rc = multi_call(lib, N=N, T=T, Hq=G * Hkv, Hkv=Hkv, D=D, MB=MB, NB=64, qd=2, kd=2,
+                                        ws=0x100000, wsb=need)
+                        assert rc == B.PA_ERR_CUDA, (D, Hkv, G, T, N, MB, rc)
+                        checked += 1
+    assert checked == 6192

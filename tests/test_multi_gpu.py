@@ -121,19 +121,17 @@ def test_one_query_token_is_decode():
     assert torch.equal(a, b[:, 0])
 
 
-def test_multi_8b_full_size():
-    """The 8B-shaped batch (256 sequences, lognormal lengths) with T = 5 query tokens:
-    sampled sequences against the oracle, every row finite."""
-    w = W.make_config("8b", num_q_tokens=5)
+@pytest.mark.parametrize("T", [5, 8, 16])
+def test_multi_8b_full_size(T):
+    """The 8B-shaped batch (256 sequences, lognormal lengths) with T query tokens, as the bench
+    runs it (T = 16 takes two column groups per partition): the step's stored tokens bit-exact
+    and every output row of every sequence against the oracle."""
+    w = W.make_config("8b", num_q_tokens=T)
     dw, out = gpu_multi(w, "bf16")
     assert B.pa_get_device_error() == B.PA_DEV_OK
-    L = w.seq_lens
-    rng = np.random.default_rng(8)
-    seqs = sorted({int(np.argmax(L)), int(np.argmin(L))} | set(int(i) for i in rng.choice(w.num_seqs, 10,
-                                                                                              replace=False)))
-    idx, ref, _, _ = oracle_multi(w, seqs)
-    got = out.float().cpu().numpy()[idx]
-    assert_close(got, ref, w.kv_dtype, "bf16", "8b T=5")
+    _, ref, kc, vc = oracle_multi(w)
+    assert np.array_equal(B.from_torch(dw.k_cache), kc) and np.array_equal(B.from_torch(dw.v_cache), vc)
+    assert_close(out.float().cpu().numpy(), ref, w.kv_dtype, "bf16", f"8b T={T}")
     assert torch.isfinite(out.float()).all()
 
 
@@ -172,3 +170,22 @@ def test_sequence_shorter_than_its_queries_is_flagged():
     assert torch.isnan(out[2]).all()
     _, ref, _, _ = oracle_multi(w, [0, 1])
     assert_close(out[:2].cpu().numpy(), ref, "bf16", "f32", "valid sequences beside an invalid one")
+
+
+@pytest.mark.parametrize("case", [(2, 1, 16, "f16"), (6, 2, 9, "bf16"), (5, 1, 7, "f16")],
+                         ids=lambda c: "-".join(map(str, c)))
+def test_multi_head_dim_64_many_column_groups(case):
+    """head_dim 64 with few KV heads: items of 5 to 8 query rows, so a sequence's T query tokens
+    make several column groups per partition.  64 sequences of up to 2048 tokens give a work
+    list far larger than the workspace's alignment padding: every group must have its own
+    reserved work item (none may spill into the partial results)."""
+    Hq, Hkv, T, dt = case
+    rng = np.random.default_rng(4300 + Hq)
+    lens = [int(x) for x in rng.integers(T, 2049, size=64)]
+    lens[:3] = [0, T, 2048]
+    w = W.independent("d64", lens, num_q_tokens=T, num_q_heads=Hq, num_kv_heads=Hkv, head_dim=64, block_size=16,
+                      q_dtype=dt, kv_dtype=dt, seed=4300 + Hq)
+    dw, out = gpu_multi(w, "f32")
+    assert B.pa_get_device_error() == B.PA_DEV_OK
+    _, ref, _, _ = oracle_multi(w)
+    assert_close(out.float().cpu().numpy(), ref, dt, "f32", f"head_dim 64 case {case}")
