@@ -50,8 +50,12 @@ def parse_args():
     ap.add_argument("--steps", type=int, default=3000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--op", choices=["step", "swap"], default="step",
-                    help="step: the decode step (default); swap: swap_blocks to / from pinned host memory")
+    ap.add_argument("--op", choices=["step", "swap", "cache"], default="step",
+                    help="step: the decode step (default); swap: swap_blocks to / from pinned host memory; "
+                         "cache: reshape_and_cache and copy_blocks alone (default workload: the 70b fork step)")
+    ap.add_argument("--step", choices=list(W.STEPS_70B), default=None,
+                    help="70b only: 'decode' (default: one new token per sequence) or 'fork' (every sample's "
+                         "whole suffix stored in the step, with all 192 copy-on-write pairs)")
     ap.add_argument("--config", default="8b", choices=list(W.CONFIG_NAMES))
     ap.add_argument("--block-size", type=int, default=None)
     ap.add_argument("--num-seqs", type=int, default=None,
@@ -73,6 +77,33 @@ def parse_args():
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target oracle time for cpu_baseline")
     ap.add_argument("--ref-seconds", type=float, default=150.0, help="target total time of --impl reference")
     return ap.parse_args()
+
+
+def make_workload(args, seed=None, num_seqs=None):
+    """The bench's workload: the config (with --block-size, --kv-dtype, --qtok, --step) and, for
+    profiling, a smaller batch of it (70b: that many shared-prefix samples, in groups of 4)."""
+    extra = {}
+    if num_seqs:
+        extra = {"num_groups": max(1, num_seqs // 4)} if args.config == "70b" else {"num_seqs": num_seqs}
+    if args.qtok > 1:
+        extra["num_q_tokens"] = args.qtok
+    if args.step:
+        if args.config != "70b":
+            raise SystemExit("--step applies to the 70b config")
+        extra["step"] = args.step
+    return W.make_config(args.config, block_size=args.block_size, seed=seed, kv_dtype=args.kv_dtype, **extra)
+
+
+def cpu_model() -> str:
+    """The host CPU's model name (from /proc/cpuinfo), or the platform's processor string."""
+    try:
+        for line in open("/proc/cpuinfo", encoding="utf-8"):
+            if line.lower().startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
 
 
 def workload_label(w: W.Workload) -> str:
@@ -127,7 +158,8 @@ def profile_name(args) -> str:
     """Name of the committed ncu summary of this run's partition kernel: config, cache dtype and
     query tokens (pa_decode_partition_8b, pa_decode_partition_8b_e4m3, pa_decode_partition_8b_T5)."""
     return (f"pa_decode_partition_{args.config}" + (f"_{args.kv_dtype}" if args.kv_dtype else "")
-            + (f"_T{args.qtok}" if args.qtok > 1 else "") + ("_prefix" if args.prefix else "")
+            + (f"_T{args.qtok}" if args.qtok > 1 else "") + ("_fork" if getattr(args, "step", None) == "fork" else "")
+            + ("_prefix" if args.prefix else "")
             + ("_tcgen05" if getattr(args, "wide_kernel", "mma") == "tcgen05" else ""))
 
 
@@ -215,13 +247,14 @@ def oracle_post_step(w: W.Workload):
     return kc, vc
 
 
-def oracle_sample_rate(w: W.Workload, seconds: float, start: int = 0):
-    """Time the fp64 oracle on consecutive sequences (from `start`, wrapping) until ~`seconds` of work.
+def oracle_sample_rate(w: W.Workload, seconds: float, start: int = 0, threads: int = 0):
+    """Time the fp64 oracle on consecutive sequences (from `start`, wrapping) until ~`seconds` of work,
+    on `threads` threads (0: every core the process may run on).
 
     Returns (KV bytes processed, seconds, threads, sequence count)."""
     import oracle
 
-    threads = oracle.default_threads()
+    threads = threads or oracle.default_threads()
     kc, vc = oracle_post_step(w)
     if w.num_q_tokens > 1:
         def run(q, bt, sl, num_threads):
@@ -261,8 +294,7 @@ def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
-    qkw = {"num_q_tokens": args.qtok} if args.qtok > 1 else {}
-    w = W.make_config(args.config, block_size=args.block_size, kv_dtype=args.kv_dtype, **qkw)
+    w = make_workload(args)
     per_step = max(0.5, args.ref_seconds / max(1, args.steps + args.warmup))
     start = 0
     for _ in range(args.warmup):
@@ -282,6 +314,7 @@ def run_reference(args):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": workload_label(w)},
         "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
+                         "cpu_model": cpu_model(),
                          "sample": f"{seqs} sequences over {args.steps} steps (consecutive windows of the batch), "
                                    f"fp64 two-pass softmax, attention only"},
         "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -311,12 +344,7 @@ def run_ours(args):
                                 device_id=torch.device("cuda", local))
 
     seed = rank_seed(args.config, rank)
-    extra = {}
-    if args.num_seqs:  # the 70b batch shrinks by whole groups of 4 samples
-        extra = {"num_groups": max(1, args.num_seqs // 4)} if args.config == "70b" else {"num_seqs": args.num_seqs}
-    if args.qtok > 1:
-        extra["num_q_tokens"] = args.qtok
-    w = W.make_config(args.config, block_size=args.block_size, seed=seed, kv_dtype=args.kv_dtype, **extra)
+    w = make_workload(args, seed, args.num_seqs)
     out_dtype = args.out_dtype or w.q_dtype
     dw = B.device_workload(w, f"cuda:{local}")
     ws = B.DecodeWorkspace.for_workload(dw, args.partition_size)
@@ -516,9 +544,12 @@ def run_ours(args):
     cpu = None
     if not args.no_cpu_baseline and world == 1:
         b, t, threads, n = oracle_sample_rate(w, args.cpu_seconds)
+        b1, t1, _, n1 = oracle_sample_rate(w, args.cpu_seconds / 3, threads=1)
         cpu = {"value": round(b / t / 1e9, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
+               "single_core_gbs": round(b1 / t1 / 1e9, 5), "cpu_model": cpu_model(),
                "sample": f"{n} sequence decodes from the start of the batch of {w.num_seqs} "
-                         f"({b / 1e9:.3f} GB of K+V), attention only, fp64 two-pass softmax, {t:.1f} s"}
+                         f"({b / 1e9:.3f} GB of K+V), attention only, fp64 two-pass softmax, {t:.1f} s on "
+                         f"{threads} threads; single core: {n1} sequence decodes ({b1 / 1e9:.3f} GB) in {t1:.1f} s"}
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_step, 5), "higher_is_better": True, "scaling": "weak",
@@ -526,6 +557,7 @@ def run_ours(args):
         "config": {"workload": workload_label(w), "kv_bytes_per_step": kv_bytes, "kv_bytes_unique": kv_unique,
                    "seq_tokens_per_step": w.total_tokens(), "new_tokens_per_step": int(len(w.slot_mapping)),
                    "cow_pairs_per_step": int(len(w.copy_pairs)), "out_dtype": out_dtype,
+                   "step": w.notes.get("step"),
                    "partition_size": args.partition_size or 512,
                    "wide_kernel": args.wide_kernel if (w.num_q_tokens > 1 or args.prefix) else None,
                    "prefix_groups": (f"{len(groups_np)} groups, {int(groups_np[:, 1].sum())} sequences, shared "
@@ -564,7 +596,7 @@ def run_swap(args):
     from paged_kv_cache_327_b200 import build as pkg_build
 
     pkg_build.build()
-    w = W.make_config(args.config, block_size=args.block_size, kv_dtype=args.kv_dtype)
+    w = make_workload(args)
     dw = B.device_workload(w)
     bs = w.block_size
     seqs = range(w.num_seqs // 4)
@@ -613,12 +645,106 @@ def run_swap(args):
     return 0
 
 
+def run_cache(args):
+    """reshape_and_cache and copy_blocks, each timed on its own (CUDA events around every launch,
+    L2 flushed before each), against the measured HBM copy bandwidth.  Default workload: the 70b
+    fork step (every sample's whole suffix stored, 192 copy-on-write pairs)."""
+    from paged_kv_cache_327_b200 import binding as B
+    from paged_kv_cache_327_b200 import build as pkg_build
+
+    pkg_build.build()
+    if args.config == "70b" and args.step is None:
+        args.step = "fork"
+    w = make_workload(args, num_seqs=args.num_seqs)
+    dw = B.device_workload(w)
+    stream = torch.cuda.current_stream()
+    fp8 = w.kv_dtype == "e4m3"
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    peak, peak_src = measured_peak()
+
+    def store():
+        if fp8:
+            B.pa_reshape_and_cache_fp8(dw.new_k, dw.new_v, dw.k_cache, dw.v_cache, dw.slot_mapping, w.k_scale,
+                                       w.v_scale, stream=stream)
+        else:
+            B.pa_reshape_and_cache(dw.new_k, dw.new_v, dw.k_cache, dw.v_cache, dw.slot_mapping, stream=stream)
+
+    def copy():
+        B.pa_copy_blocks(dw.k_cache, dw.v_cache, dw.copy_pairs, stream=stream)
+
+    def timed(fn, reps):
+        for _ in range(max(3, args.warmup)):
+            fn()
+        torch.cuda.synchronize()
+        flushed, back = [], []
+        for _ in range(reps):
+            flush.fill_(1)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            torch.cuda.synchronize()
+            flushed.append(a.elapsed_time(b))
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(reps):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        return float(np.median(flushed)), a.elapsed_time(b) / reps
+
+    reps = max(5, min(args.steps, 200))
+    T = int(len(w.slot_mapping))
+    new_es = W.ELEM_BYTES[w.new_kv_dtype]
+    # K and V rows read in their input dtype and written in the cache dtype, plus the slots
+    store_bytes = T * w.num_kv_heads * w.head_dim * 2 * (new_es + W.ELEM_BYTES[w.kv_dtype]) + 8 * T
+    P = int(len(w.copy_pairs))
+    copy_bytes = 2 * 2 * P * w.block_bytes + 8 * P  # K and V blocks read and written, plus the pairs
+    ops = {}
+    if T:
+        med, mean = timed(store, reps)
+        ops["reshape_and_cache"] = {"tokens": T, "algorithmic_bytes": store_bytes, "ms_l2_flushed_median": round(med, 5),
+                                    "ms_back_to_back_mean": round(mean, 5),
+                                    "achieved_gbs": round(store_bytes / (med * 1e-3) / 1e9, 2),
+                                    "frac": round(store_bytes / (med * 1e-3) / 1e9 / peak, 4)}
+    if P:
+        med, mean = timed(copy, reps)
+        ops["copy_blocks"] = {"pairs": P, "algorithmic_bytes": copy_bytes, "ms_l2_flushed_median": round(med, 5),
+                              "ms_back_to_back_mean": round(mean, 5),
+                              "achieved_gbs": round(copy_bytes / (med * 1e-3) / 1e9, 2),
+                              "frac": round(copy_bytes / (med * 1e-3) / 1e9 / peak, 4)}
+    if B.pa_get_device_error() != B.PA_DEV_OK:
+        raise RuntimeError("device error in the cache operations")
+    # the step's state is reproducible: check the caches against plain numpy indexing once
+    if not fp8:
+        kc, vc = W.apply_step_host(w)
+        if not (np.array_equal(B.from_torch(dw.k_cache), kc) and np.array_equal(B.from_torch(dw.v_cache), vc)):
+            raise RuntimeError("cache state after the timed cache operations differs from the expected state")
+    main_op = "reshape_and_cache" if T else "copy_blocks"
+    m = ops[main_op]
+    line = {
+        "metric": "reshape_and_cache / copy_blocks GB/s (% of HBM peak)", "op": "cache",
+        "value": m["achieved_gbs"], "unit": "GB/s", "n_gpus": 1, "steps": reps, "warmup": max(3, args.warmup),
+        "higher_is_better": True, "data": "synthetic", "dtype": w.kv_dtype,
+        "config": {"workload": workload_label(w), "step": w.notes.get("step"),
+                   "l2": "256 MB written before every timed launch"},
+        "ops": ops,
+        "roofline": {"bound": "hbm", "kernel": main_op, "achieved": m["achieved_gbs"], "peak": peak, "unit": "GB/s",
+                     "frac": m["frac"], "traffic": None, "peak_source": peak_src},
+        "gpu_launches": 2 * reps * len(ops),
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     args = parse_args()
     if args.impl == "reference":
         return run_reference(args)
     if args.op == "swap":
         return run_swap(args)
+    if args.op == "cache":
+        return run_cache(args)
     return run_ours(args)
 
 

@@ -13,8 +13,11 @@
  *
  * Conventions shared by every entry point
  *   - Every pointer argument is a DEVICE pointer unless its name starts with host_.
- *     The caller owns all memory (including the decode workspace); the library never
- *     allocates device memory and keeps no per-call state.
+ *     The caller owns all memory (including the decode workspace); no call allocates
+ *     device memory and none keeps per-call state.  The library's own device memory is
+ *     static, fixed in size and held from load to exit on every GPU that loads it: the
+ *     device error word and the PA_DECODE_STATIC_WORKSPACE_BYTES scratch buffer that only
+ *     pa_decode_static_workspace uses.
  *   - Tensors are dense and row-major (C order) unless a stride argument says otherwise.
  *   - Element types are pa_dtype values.  Caches and the decode query must start on a
  *     16-byte boundary.

@@ -2,7 +2,13 @@
 
 The CUDA runtime is linked statically, so the library loads on a machine without a GPU
 (for symbol checks); the driver's tensor-map encoder is looked up at run time.
+
+Several processes may build at once (one per GPU rank): they take turns under an exclusive
+file lock beside the library, the freshness check is repeated under the lock (so only the
+first one compiles), and each compiles into a temporary file of its own that is renamed over
+the library in one step.
 """
+import fcntl
 import os
 import subprocess
 import sys
@@ -29,18 +35,33 @@ def nvcc():
     return path if os.path.exists(path) else "nvcc"
 
 
-def build(force: bool = False, verbose: bool = False, extra=()) -> str:
-    if not force and os.path.exists(LIB):
-        mtime = os.path.getmtime(LIB)
-        if all(os.path.getmtime(f) <= mtime for f in DEPENDS):
-            return LIB
-    cmd = [nvcc(), *NVCC_FLAGS, *extra, "-I", os.path.join(ROOT, "include"), "-I", CSRC,
-           *SOURCES, "-o", LIB + ".tmp"]
-    if verbose:
-        cmd.insert(1, "-Xptxas=-v")
-    subprocess.run(cmd, check=True)
-    os.replace(LIB + ".tmp", LIB)
-    return LIB
+def _fresh(lib: str) -> bool:
+    if not os.path.exists(lib):
+        return False
+    mtime = os.path.getmtime(lib)
+    return all(os.path.getmtime(f) <= mtime for f in DEPENDS)
+
+
+def build(force: bool = False, verbose: bool = False, extra=(), lib: str = LIB) -> str:
+    """Compile `lib` (default: the in-tree libpa.so) unless it is newer than every source."""
+    if not force and _fresh(lib):
+        return lib
+    with open(lib + ".lock", "w") as lock:
+        fcntl.flock(lock, fcntl.LOCK_EX)  # released when the file closes
+        if not force and _fresh(lib):      # another process built it while this one waited
+            return lib
+        tmp = f"{lib}.{os.getpid()}.tmp"
+        cmd = [nvcc(), *NVCC_FLAGS, *extra, "-I", os.path.join(ROOT, "include"), "-I", CSRC,
+               *SOURCES, "-o", tmp]
+        if verbose:
+            cmd.insert(1, "-Xptxas=-v")
+        try:
+            subprocess.run(cmd, check=True)
+            os.replace(tmp, lib)
+        finally:
+            if os.path.exists(tmp):
+                os.unlink(tmp)
+    return lib
 
 
 if __name__ == "__main__":

@@ -120,9 +120,13 @@ class Group:
 
     prefix: tokens cached before the step (shared by every member).
     step_tokens: tokens each member appends in this step (through reshape_and_cache).
+    own_history: tokens each member appended after the fork and before the step (None: none).
+        Their first write into a shared partial block went through copy-on-write then, so
+        those copies are part of the cache state before the step, not of the step.
     """
     prefix: int
     step_tokens: List[int]
+    own_history: Optional[List[int]] = None
 
 
 @dataclasses.dataclass
@@ -224,12 +228,17 @@ def build_groups(name: str, groups: Sequence[Group], *, num_q_heads: int, num_kv
     for g in groups:
         if g.prefix < 0 or not g.step_tokens or min(g.step_tokens) < 0:
             raise ValueError("bad group")
+        if g.own_history is not None and (len(g.own_history) != len(g.step_tokens) or min(g.own_history) < 0):
+            raise ValueError("own_history needs one non-negative count per member")
     bs = block_size
 
     def run(allocator: BlockAllocator):
         tables: List[BlockTable] = []
         prefix_slots: List[np.ndarray] = []
+        own_slots: List[np.ndarray] = []
         step_slots: List[List[np.ndarray]] = []
+        hist_pairs: List[np.ndarray] = []
+        step_pairs: List[np.ndarray] = []
         for g in groups:
             parent = BlockTable(bs)
             prefix_slots.append(parent.append_tokens(g.prefix, allocator))
@@ -238,12 +247,18 @@ def build_groups(name: str, groups: Sequence[Group], *, num_q_heads: int, num_kv
                 child = BlockTable(bs)
                 child.fork_from(parent, allocator)
                 members.append(child)
+            if g.own_history is not None:
+                own_slots.extend(m.append_tokens(n, allocator) for m, n in zip(members, g.own_history))
+            hist_pairs.append(allocator.take_pending_copies())
             step_slots.append([m.append_tokens(n, allocator) for m, n in zip(members, g.step_tokens)])
+            step_pairs.append(allocator.take_pending_copies())
             tables.extend(members)
-        return tables, prefix_slots, step_slots
+        return (tables, prefix_slots, own_slots, step_slots, np.concatenate(hist_pairs + [np.zeros((0, 2), np.int32)]),
+                np.concatenate(step_pairs + [np.zeros((0, 2), np.int32)]))
 
     # dry run on an identity-ordered pool large enough for anything: counts the blocks needed
-    upper = sum(-(-g.prefix // bs) + sum(-(-n // bs) + 1 for n in g.step_tokens) for g in groups) + 1
+    upper = sum(-(-g.prefix // bs) + sum(-(-n // bs) + 1 for n in g.step_tokens) +
+                sum(-(-n // bs) + 1 for n in (g.own_history or [])) for g in groups) + 1
     probe = BlockAllocator(upper, bs)
     run(probe)
     need = upper - probe.get_num_free_blocks()
@@ -254,8 +269,7 @@ def build_groups(name: str, groups: Sequence[Group], *, num_q_heads: int, num_kv
 
     place_rng = np.random.default_rng([seed, _S_PLACE])
     allocator = BlockAllocator(num_blocks, bs, rng=place_rng)
-    tables, prefix_slots, step_slots = run(allocator)
-    pairs = allocator.take_pending_copies()
+    tables, prefix_slots, own_slots, step_slots, hist_pairs, pairs = run(allocator)
 
     N = len(tables)
     Hkv, D = num_kv_heads, head_dim
@@ -279,6 +293,14 @@ def build_groups(name: str, groups: Sequence[Group], *, num_q_heads: int, num_kv
     if H:
         k_cache.reshape(num_blocks * bs, Hkv, D)[hist_slots] = _draw((seed, _S_HIST, 0), (H, Hkv, D), kdt)
         v_cache.reshape(num_blocks * bs, Hkv, D)[hist_slots] = _draw((seed, _S_HIST, 1), (H, Hkv, D), vdt)
+    # members' own history: the copy-on-write copies of their first writes, then the tokens
+    for src, dst in hist_pairs:
+        k_cache[dst] = k_cache[src]
+        v_cache[dst] = v_cache[src]
+    own = np.concatenate([np.zeros(0, np.int64)] + own_slots)
+    if len(own):
+        k_cache.reshape(num_blocks * bs, Hkv, D)[own] = _draw((seed, _S_HIST, 2), (len(own), Hkv, D), kdt)
+        v_cache.reshape(num_blocks * bs, Hkv, D)[own] = _draw((seed, _S_HIST, 3), (len(own), Hkv, D), vdt)
 
     all_slots = np.concatenate([np.zeros(0, np.int64)] +
                                [s for per_group in step_slots for s in per_group]).astype(np.int64)
@@ -290,7 +312,7 @@ def build_groups(name: str, groups: Sequence[Group], *, num_q_heads: int, num_kv
     seq_lens = np.asarray([t.num_tokens for t in tables], dtype=np.int32)
     block_tables = tables_to_array(tables)
     info = {"groups": len(groups), "blocks_needed": int(need), "cow_pairs": int(len(pairs)),
-            "new_tokens": int(T), "pool_factor": pool_factor}
+            "cow_pairs_before_step": int(len(hist_pairs)), "new_tokens": int(T), "pool_factor": pool_factor}
     if notes:
         info.update(notes)
     return Workload(name=name, num_seqs=N, num_q_heads=num_q_heads, num_kv_heads=num_kv_heads,
@@ -312,9 +334,9 @@ def independent(name: str, seq_lens: Sequence[int], num_q_tokens: int = 1, **kw)
     return build_groups(name, groups, num_q_tokens=T, **kw)
 
 
-def _fp8_kw(kw: dict) -> dict:
-    """Inside make_config(kv_dtype="e4m3"): the config's own dtype becomes the new tokens' dtype."""
-    if _FP8_OVERRIDE:
+def _fp8_kw(kw: dict, fp8: bool) -> dict:
+    """A config over an FP8 cache: the config's own dtype becomes the new tokens' dtype."""
+    if fp8:
         kw = dict(kw, new_dtype=kw["kv_dtype"], kv_dtype="e4m3")
     return kw
 
@@ -330,7 +352,7 @@ def config_seed(name: str) -> int:
     return 3270 + CONFIG_INDEX[name]
 
 
-def _tiny(seed: int, block_size: int) -> Workload:
+def _tiny(seed: int, block_size: int, fp8: bool = False) -> Workload:
     # 4 sequences, post-step lengths uniform in [1, 64]; sequence 3 is a fork of sequence 2
     # (parallel sampling), so the step's first write into their shared partial block is the
     # one copy-on-write pair.  Fixed pool of 64 blocks.
@@ -341,25 +363,27 @@ def _tiny(seed: int, block_size: int) -> Workload:
         if (L2 - 1) % block_size != 0:
             break
     groups = [Group(L[0] - 1, [1]), Group(L[1] - 1, [1]), Group(L2 - 1, [1, 1])]
+    if fp8:
+        raise ValueError("the tiny config (head_dim 64) has no FP8 variant")
     return build_groups("tiny", groups, num_q_heads=2, num_kv_heads=2, head_dim=64,
                         block_size=block_size, q_dtype="f32", kv_dtype="f16", seed=seed,
                         num_blocks=64, notes={"lens": "uniform[1,64]; seq 3 forks seq 2"})
 
 
-def _7b(seed: int, block_size: int, num_seqs: int = 64, num_q_tokens: int = 1) -> Workload:
+def _7b(seed: int, block_size: int, num_seqs: int = 64, num_q_tokens: int = 1, fp8: bool = False) -> Workload:
     rng = np.random.default_rng([seed, _S_LENS])
     L = np.maximum(rng.integers(128, 2049, size=num_seqs), num_q_tokens)
-    return independent("7b", L, num_q_tokens, **_fp8_kw(dict(num_q_heads=32, num_kv_heads=32, head_dim=128, block_size=block_size,
-                                               q_dtype="bf16", kv_dtype="bf16", seed=seed,
-                                               notes={"lens": "uniform[128,2048]"})))
+    kw = dict(num_q_heads=32, num_kv_heads=32, head_dim=128, block_size=block_size, q_dtype="bf16",
+              kv_dtype="bf16", seed=seed, notes={"lens": "uniform[128,2048]"})
+    return independent("7b", L, num_q_tokens, **_fp8_kw(kw, fp8))
 
 
-def _13b(seed: int, block_size: int, num_seqs: int = 128, num_q_tokens: int = 1) -> Workload:
+def _13b(seed: int, block_size: int, num_seqs: int = 128, num_q_tokens: int = 1, fp8: bool = False) -> Workload:
     rng = np.random.default_rng([seed, _S_LENS])
     L = np.maximum(rng.integers(16, 2049, size=num_seqs), num_q_tokens)
-    return independent(f"13b-bs{block_size}", L, num_q_tokens, **_fp8_kw(dict(num_q_heads=40, num_kv_heads=40, head_dim=128,
-                                                             block_size=block_size, q_dtype="f16", kv_dtype="f16",
-                                                             seed=seed, notes={"lens": "uniform[16,2048]"})))
+    kw = dict(num_q_heads=40, num_kv_heads=40, head_dim=128, block_size=block_size, q_dtype="f16",
+              kv_dtype="f16", seed=seed, notes={"lens": "uniform[16,2048]"})
+    return independent(f"13b-bs{block_size}", L, num_q_tokens, **_fp8_kw(kw, fp8))
 
 
 def lognormal_lengths(rng: np.random.Generator, n: int, median: float = 1024.0, sigma: float = 1.0,
@@ -368,35 +392,48 @@ def lognormal_lengths(rng: np.random.Generator, n: int, median: float = 1024.0, 
     return np.clip(np.rint(np.exp(math.log(median) + sigma * z)), lo, hi).astype(np.int64)
 
 
-def _8b(seed: int, block_size: int, num_seqs: int = 256, num_q_tokens: int = 1) -> Workload:
+def _8b(seed: int, block_size: int, num_seqs: int = 256, num_q_tokens: int = 1, fp8: bool = False) -> Workload:
     rng = np.random.default_rng([seed, _S_LENS])
     L = np.maximum(lognormal_lengths(rng, num_seqs), num_q_tokens)
-    return independent("8b", L, num_q_tokens, **_fp8_kw(dict(num_q_heads=32, num_kv_heads=8, head_dim=128, block_size=block_size,
-                                               q_dtype="bf16", kv_dtype="bf16", seed=seed,
-                                               notes={"lens": "lognormal(median 1024, sigma 1.0) clipped to "
-                                                              "[32, 8192]"})))
+    kw = dict(num_q_heads=32, num_kv_heads=8, head_dim=128, block_size=block_size, q_dtype="bf16",
+              kv_dtype="bf16", seed=seed, notes={"lens": "lognormal(median 1024, sigma 1.0) clipped to [32, 8192]"})
+    return independent("8b", L, num_q_tokens, **_fp8_kw(kw, fp8))
+
+
+STEPS_70B = ("decode", "fork")
 
 
 def _70b(seed: int, block_size: int, num_groups: int = 64, samples: int = 4,
-         prefix: int = 4096, long_len: int = 32768, num_long: int = 4) -> Workload:
+         prefix: int = 4096, long_len: int = 32768, num_long: int = 4, step: str = "decode",
+         fp8: bool = False) -> Workload:
     # 64 groups x 4 samples.  Each group's parent holds prefix + r_g tokens, r_g uniform in
-    # [1, bs-1], so its last shared block is partial; the samples fork from it and each
-    # appends its own suffix (uniform in [1, 512] tokens) in the step: the first three
-    # writers into the shared partial block copy it, the fourth writes in place.  Four
-    # standalone 32768-token sequences ride in the same batch.
+    # [1, bs-1], so its last shared block is partial; the samples fork from it and each has a
+    # divergent suffix of uniform [1, 512] tokens: the first three writers into the shared
+    # partial block copy it, the fourth writes in place.  Four standalone 32768-token
+    # sequences ride in the same batch.
+    #   step "decode": one decode step of every sequence -- each stores one new token (256 + 4
+    #     new tokens); a sample's earlier suffix tokens, and the copy-on-write of its first
+    #     write, precede the step (a sample whose suffix is that one token copies in the step);
+    #   step "fork": every sample's whole suffix is stored in the step, so all 192 copies
+    #     (64 groups x 3) are part of it.
+    if step not in STEPS_70B:
+        raise ValueError(f"step must be one of {STEPS_70B}")
     rng = np.random.default_rng([seed, _S_LENS])
     groups = []
     for _ in range(num_groups):
         r = int(rng.integers(1, block_size))
         suffix = [int(x) for x in rng.integers(1, 513, size=samples)]
-        groups.append(Group(prefix + r, suffix))
+        if step == "fork":
+            groups.append(Group(prefix + r, suffix))
+        else:
+            groups.append(Group(prefix + r, [1] * samples, own_history=[n - 1 for n in suffix]))
     groups += [Group(long_len - 1, [1]) for _ in range(num_long)]
-    return build_groups("70b", groups, **_fp8_kw(dict(num_q_heads=64, num_kv_heads=8, head_dim=128,
-                                                      block_size=block_size, q_dtype="bf16", kv_dtype="bf16",
-                                                      seed=seed,
-                                                      notes={"lens": "64 groups x 4 samples: prefix 4096+r "
-                                                                     "(r in [1,bs-1]) + suffix uniform[1,512]; "
-                                                                     "plus 4 x 32768"})))
+    stored = "one token per sequence" if step == "decode" else "each sample's whole suffix"
+    kw = dict(num_q_heads=64, num_kv_heads=8, head_dim=128, block_size=block_size, q_dtype="bf16",
+              kv_dtype="bf16", seed=seed,
+              notes={"lens": "64 groups x 4 samples: prefix 4096+r (r in [1,bs-1]) + suffix uniform[1,512]; "
+                             "plus 4 x 32768", "step": f"{step}: the step stores {stored}"})
+    return build_groups("70b" if step == "decode" else "70b-fork", groups, **_fp8_kw(kw, fp8))
 
 
 _BUILDERS = {"tiny": _tiny, "7b": _7b, "13b": _13b, "8b": _8b, "70b": _70b}
@@ -411,20 +448,15 @@ def make_config(name: str, block_size: Optional[int] = None, seed: Optional[int]
     history is stored as FP8 codes, the step's new tokens stay in the config's dtype.
     num_q_tokens=T ("7b", "13b", "8b") gives the multi-token step: the same lengths (raised to T
     where shorter), the last T tokens of every sequence stored in the step and attended to
-    causally by T queries.
+    causally by T queries.  step="fork" ("70b") stores every sample's whole suffix in the step
+    instead of one token per sequence.
     """
     if name not in _BUILDERS:
         raise KeyError(f"unknown config {name!r}; choose from {CONFIG_NAMES}")
+    if kv_dtype not in (None, "e4m3"):
+        raise ValueError("kv_dtype is None (the config's own) or 'e4m3'")
     bs = block_size or _DEFAULT_BS[name]
-    global _FP8_OVERRIDE
-    _FP8_OVERRIDE = kv_dtype == "e4m3"
-    try:
-        return _BUILDERS[name](config_seed(name) if seed is None else seed, bs, **overrides)
-    finally:
-        _FP8_OVERRIDE = False
-
-
-_FP8_OVERRIDE = False
+    return _BUILDERS[name](config_seed(name) if seed is None else seed, bs, fp8=kv_dtype == "e4m3", **overrides)
 
 
 def apply_step_host(w: Workload) -> Tuple[np.ndarray, np.ndarray]:

@@ -158,7 +158,11 @@ def test_named_config_shapes(name):
         assert w.num_seqs == 256 and L.min() >= 32 and L.max() <= 8192
         assert 700 < np.median(L) < 1400
     if name == "70b":
-        assert w.num_seqs == 260 and len(w.copy_pairs) == 192
+        # one decode step: one new token per sequence; the 64 x 3 copy-on-write copies of the
+        # samples' first writes precede it (a sample whose whole suffix is the step's token
+        # copies in the step)
+        assert w.num_seqs == 260 and len(w.slot_mapping) == 260
+        assert len(w.copy_pairs) + w.notes["cow_pairs_before_step"] == 192
         assert sorted(L)[-4:] == [32768] * 4
         assert w.kv_bytes_unique() < w.kv_bytes_logical() / 2
     assert w.num_blocks >= int(np.ceil(1.25 * w.notes["blocks_needed"]))
@@ -166,6 +170,32 @@ def test_named_config_shapes(name):
     if name != "70b":
         used = np.concatenate([w.block_tables[i, :-(-int(l) // w.block_size)] for i, l in enumerate(L)])
         assert len(np.unique(used)) == len(used)
+
+
+def test_70b_fork_step_stores_every_suffix():
+    """The fork-step variant of the 70B batch: the same sequences, but every sample's whole
+    suffix (and so every copy-on-write) lies in the step."""
+    a = W.make_config("70b")
+    b = W.make_config("70b", step="fork")
+    assert np.array_equal(a.seq_lens, b.seq_lens)
+    assert len(b.copy_pairs) == 192 and b.notes["cow_pairs_before_step"] == 0
+    # a group's samples store their suffixes (1..512 tokens each), a long sequence one token
+    assert 256 + 4 < len(b.slot_mapping) <= 256 * 512 + 4
+    # the step's tokens of the decode variant are the last token of every sequence; in the fork
+    # variant each sample stores its whole suffix, which ends with that token
+    assert a.kv_bytes_unique() == b.kv_bytes_unique()
+    with pytest.raises(ValueError):
+        W.make_config("70b", step="prefill")
+
+
+def test_fp8_configs_are_reentrant():
+    """An FP8 config build leaves no state behind: the next plain build is the plain config."""
+    f = W.make_config("8b", kv_dtype="e4m3", num_seqs=4)
+    p = W.make_config("8b", num_seqs=4)
+    assert f.kv_dtype == "e4m3" and f.new_kv_dtype == "bf16"
+    assert p.kv_dtype == "bf16" and p.new_kv_dtype == "bf16"
+    with pytest.raises(ValueError):
+        W.make_config("tiny", kv_dtype="e4m3")
 
 
 def test_swap_out_and_in_move_groups_and_keep_sharing():

@@ -109,13 +109,13 @@ def test_fp8_decode_matches_oracle(case):
     assert np.all(out.float().cpu().numpy()[LENS.index(0)] == 0.0)
 
 
-def test_fp8_8b_full_size():
-    w = W.make_config("8b", kv_dtype="e4m3")
+@pytest.mark.parametrize("name,bs", [("8b", 16), ("7b", 16), ("13b", 32)])
+def test_fp8_full_size(name, bs):
+    """A named config over an FP8 cache, as the bench runs it: the quantising store bit-exact over
+    the whole cache and every output row of every sequence against the oracle."""
+    w = W.make_config(name, block_size=bs, kv_dtype="e4m3")
     dw, out = run(w, "bf16")
-    L = w.seq_lens
-    rng = np.random.default_rng(6)
-    seqs = sorted({int(np.argmax(L)), int(np.argmin(L))} | set(int(i) for i in rng.choice(w.num_seqs, 10, replace=False)))
-    check(w, dw, out, "bf16", seqs)
+    check(w, dw, out, "bf16")
     assert torch.isfinite(out.float()).all()
 
 

@@ -103,7 +103,8 @@ def test_prefix_decode_matches_oracle(case):
 
 
 def test_prefix_70b_batch_matches_decode_and_oracle():
-    """The 70B-shaped batch: every row agrees with pa_decode; sampled rows with the oracle."""
+    """The 70B-shaped batch as the bench runs it: every row agrees with pa_decode and, element by
+    element, with the oracle."""
     w = W.make_config("70b")
     pg = BM.find_prefix_groups(w.block_tables, w.seq_lens, w.block_size)
     dw, kc, vc = stepped(w)
@@ -114,10 +115,8 @@ def test_prefix_70b_batch_matches_decode_and_oracle():
     B.pa_decode(plain, dw.q, dw.k_cache, dw.v_cache, dw.block_tables, dw.seq_lens, w.scale, ws.tensor)
     torch.cuda.synchronize()
     assert float((out - plain).abs().max()) <= TOL[w.kv_dtype]
-    rng = np.random.default_rng(70)
-    seqs = sorted({0, 1, 2, 3, 255, w.num_seqs - 1} | set(int(i) for i in rng.choice(w.num_seqs, 6, replace=False)))
-    idx, ref = oracle_decode(w, kc, vc, seqs)
-    assert_close(out.float().cpu().numpy()[idx], ref, w.kv_dtype, "f32", "70b sample")
+    _, ref = oracle_decode(w, kc, vc)
+    assert_close(out.float().cpu().numpy(), ref, w.kv_dtype, "f32", "70b")
 
 
 def test_prefix_decode_is_deterministic():

@@ -5,8 +5,10 @@ already given nearly all free HBM to its KV-cache pool, or a plugin with no allo
 own.  This entry point takes its scratch from a buffer built into the library.  Its results
 must match pa_decode (which takes a caller workspace) within the parity tolerance, call
 after call, since every call reuses the same buffer and finds the previous call's contents
-in it.  This file is collected last so that a stop at its first failure leaves every other
-test already run; it also passes on its own in a fresh process.
+in it.  Both entry points run the same kernels on the same inputs, and their arithmetic does
+not depend on where the scratch lives, so the outputs must be bit-identical.  This file is
+collected last so that a stop at its first failure leaves every other test already run; it
+also passes on its own in a fresh process.
 """
 import ctypes
 
@@ -56,6 +58,7 @@ def test_static_workspace_matches_caller_workspace_twice(name, kw):
         assert B.pa_get_device_error() == B.PA_DEV_OK
         err = float((out - ref).abs().max())
         assert err <= TOL[w.kv_dtype], f"call {call}: max|err| vs pa_decode = {err}"
+        assert torch.equal(out, ref), f"call {call}: not bit-identical to pa_decode (max|err| {err})"
 
 
 def test_static_workspace_rejects_oversized_calls():
