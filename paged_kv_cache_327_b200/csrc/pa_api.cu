@@ -41,15 +41,10 @@ int64_t max_parts_for(int64_t max_len, int P, bool groups = true) {
   return std::max<int64_t>(1, (max_len + P - 1) / P + (groups ? 1 : 0));
 }
 
-// Query rows one work item holds per KV head: 32 with head_dim 128, 8 with head_dim 64.
+// Query rows one work item holds per KV head on the warp-MMA kernels: 32 with head_dim 128, 8 with
+// head_dim 64; the tensor-core kernel holds up to kTcMaxRows.
 int max_item_rows(int head_dim) { return head_dim == 128 ? 32 : 8; }
-
-// Query tokens of one work item (a column group): all qtok when their G rows per token fit one
-// item, otherwise as many whole tokens as fit (at least one).
-int qtok_per_item(int qtok, int G, int head_dim) {
-  const int max_rows = max_item_rows(head_dim);
-  return qtok * G <= max_rows ? qtok : std::max(1, max_rows / G);
-}
+constexpr int kTcMaxRows = 64;
 
 // Work items of one partition of one sequence, bounded from num_q_heads (= query tokens x query
 // heads) alone.  A split item holds floor(max_rows / G) * G >= 28 rows with head_dim 128 and
@@ -138,6 +133,23 @@ int encode_kv_map(CUtensorMap* map, const void* base, int kv_dtype, int64_t num_
   return r == CUDA_SUCCESS ? PA_OK : PA_ERR_CUDA;
 }
 
+// The query [num_seqs * qtok rows, num_q_heads, head_dim] (16-bit) seen as a 4-D tensor (64
+// elements, 2 halves of head_dim, heads, rows); one box = the 64-element half of `box_rows` rows of
+// G consecutive heads, 128-byte swizzle: the K-major A operand of the tensor-core kernel.
+int encode_q_map(CUtensorMap* map, const void* q, int q_dtype, int64_t rows, int num_q_heads, int G, int box_rows) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+  if (!enc) return PA_ERR_CUDA;
+  const cuuint64_t dims[4] = {64, 2, static_cast<cuuint64_t>(num_q_heads), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[3] = {128, 256, static_cast<cuuint64_t>(num_q_heads) * 256};
+  const cuuint32_t box[4] = {64, 1, static_cast<cuuint32_t>(G), static_cast<cuuint32_t>(box_rows)};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  const CUtensorMapDataType dt = q_dtype == PA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  const CUresult r = enc(map, dt, 4, const_cast<void*>(q), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? PA_OK : PA_ERR_CUDA;
+}
+
 template <int BS, int D, typename KT, typename QT, int NT, bool PAIR, bool CAUSAL, int NR>
 int launch_partition(const pa::DecodeParams& p, const CUtensorMap& tmk, const CUtensorMap& tmv,
                      int64_t max_items, int dev, DeviceInfo* info, cudaStream_t stream) {
@@ -179,11 +191,11 @@ int launch_partition(const pa::DecodeParams& p, const CUtensorMap& tmk, const CU
 // kernel for items of more than 8 query rows (PA_OPT_WIDE_KERNEL)
 std::atomic<int> g_wide_kernel{PA_WIDE_MMA};
 
-template <typename KT, int N>
-int launch_tc(const pa::DecodeParams& p, const CUtensorMap& tmk, const CUtensorMap& tmv, int64_t max_items,
-              int dev, DeviceInfo* info, cudaStream_t stream) {
-  using C = pa::TcCfg<KT, N>;
-  auto kern = pa::pa_decode_tc_kernel<KT, N, true>;
+template <typename KT>
+int launch_tc(const pa::DecodeParams& p, const CUtensorMap& tmk, const CUtensorMap& tmv, const CUtensorMap& tmq,
+              int64_t max_items, int dev, DeviceInfo* info, cudaStream_t stream) {
+  using C = pa::TcCfg<KT>;
+  auto kern = pa::pa_decode_tc_kernel<KT, true>;
   static std::atomic<bool> smem_set[kMaxDevices];
   if (!smem_set[dev].load(std::memory_order_acquire)) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
@@ -203,7 +215,7 @@ int launch_tc(const pa::DecodeParams& p, const CUtensorMap& tmk, const CUtensorM
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, kern, tmk, tmv, p) != cudaSuccess) return PA_ERR_CUDA;
+  if (cudaLaunchKernelEx(&cfg, kern, tmk, tmv, tmq, p) != cudaSuccess) return PA_ERR_CUDA;
   return cudaPeekAtLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
@@ -214,8 +226,9 @@ int launch_tc(const pa::DecodeParams& p, const CUtensorMap& tmk, const CUtensorM
 // cache with a query of the same type, head_dim 128, with two consumer warps per ring of 1 or 2
 // eight-row tiles.
 template <int BS, int D>
-int dispatch_kv(const pa::DecodeParams& p, const CUtensorMap& tmk, const CUtensorMap& tmv, int64_t max_items,
-                int dev, DeviceInfo* info, int kv_dtype, int q_dtype, int cols, cudaStream_t stream) {
+int dispatch_kv(const pa::DecodeParams& p, const CUtensorMap& tmk, const CUtensorMap& tmv, const CUtensorMap* tmq,
+                int64_t max_items, int dev, DeviceInfo* info, int kv_dtype, int q_dtype, int cols,
+                cudaStream_t stream) {
   const bool qf32 = q_dtype == PA_F32;
   const int nt = (cols + 7) / 8;
   // one instantiation: KV element type K, query type Q, tiles per consumer N, paired, causal;
@@ -240,13 +253,9 @@ int dispatch_kv(const pa::DecodeParams& p, const CUtensorMap& tmk, const CUtenso
   }
   if (nt > 1) {
     if constexpr (D == 128 && BS == 16) {  // 5th-generation tensor-core kernel, when chosen
-      if (g_wide_kernel.load(std::memory_order_relaxed) == PA_WIDE_TCGEN05) {
-        if (kv_dtype == PA_BF16 && q_dtype == PA_BF16)
-          return cols <= 16 ? launch_tc<bf16, 16>(p, tmk, tmv, max_items, dev, info, stream)
-                            : launch_tc<bf16, 32>(p, tmk, tmv, max_items, dev, info, stream);
-        if (kv_dtype == PA_F16 && q_dtype == PA_F16)
-          return cols <= 16 ? launch_tc<f16, 16>(p, tmk, tmv, max_items, dev, info, stream)
-                            : launch_tc<f16, 32>(p, tmk, tmv, max_items, dev, info, stream);
+      if (tmq) {
+        if (kv_dtype == PA_BF16 && q_dtype == PA_BF16) return launch_tc<bf16>(p, tmk, tmv, *tmq, max_items, dev, info, stream);
+        if (kv_dtype == PA_F16 && q_dtype == PA_F16) return launch_tc<f16>(p, tmk, tmv, *tmq, max_items, dev, info, stream);
       }
     }
     if constexpr (D == 128) {
@@ -328,13 +337,19 @@ int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cac
   // several query tokens: a 16-bit cache with a query of the same type
   if (qtok > 1 && (kv_dtype == PA_FP8_E4M3 || q_dtype != kv_dtype)) return PA_ERR_UNSUPPORTED;
   if (qtok > 65536 || static_cast<int64_t>(qtok) * num_q_heads * head_dim > INT_MAX) return PA_ERR_UNSUPPORTED;
-  // query tokens per item: all of them, or column groups of up to 32 query rows per KV head
+  // items of more than 8 query rows run on the tensor-core kernel when it is chosen (block size 16,
+  // head_dim 128, a 16-bit cache with a query of its own type): it holds up to 64 rows per item
+  const bool tc_ok = g_wide_kernel.load(std::memory_order_relaxed) == PA_WIDE_TCGEN05 && head_dim == 128 &&
+                     block_size == 16 && (kv_dtype == PA_F16 || kv_dtype == PA_BF16) && q_dtype == kv_dtype;
+  const int max_rows = tc_ok ? kTcMaxRows : max_item_rows(head_dim);
+  // query tokens per item: all of them, or column groups of up to max_rows query rows per KV head
   // (8 with head_dim 64, whose items run on the one-consumer kernels)
-  const int qtok_item = qtok_per_item(qtok, G, head_dim);
+  const int qtok_item = qtok * G <= max_rows ? qtok : std::max(1, max_rows / G);
   // an item holds qtok_item * G (or max_members * G) query rows: up to 8 on every dtype pair, up to
-  // 32 on a 16-bit cache with a query of its own type and head_dim 128
+  // 32 (64 on the tensor-core kernel) on a 16-bit cache with a query of its own type and head_dim 128
   const int64_t cols = static_cast<int64_t>(qtok_item) * max_members * G;
-  if (cols > 32) return PA_ERR_UNSUPPORTED;
+  if (cols > max_rows) return PA_ERR_UNSUPPORTED;
+  const bool use_tc = tc_ok && cols > 8;
   if (cols > 8 && (head_dim != 128 || kv_dtype == PA_FP8_E4M3 || q_dtype != kv_dtype)) return PA_ERR_UNSUPPORTED;
   if (head_dim != 64 && head_dim != 128) return PA_ERR_UNSUPPORTED;
   if (block_size != 16 && block_size != 32) return PA_ERR_UNSUPPORTED;
@@ -367,6 +382,8 @@ int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cac
   if (static_cast<int64_t>(num_seqs) * max_parts * ncg * static_cast<int64_t>(sizeof(pa::WorkItem)) >
       static_cast<int64_t>(L.part_ml - L.items))
     return PA_ERR_WORKSPACE;
+  const int64_t max_items = static_cast<int64_t>(num_seqs) * max_parts * ncg * num_kv_heads;
+  if (max_items > INT_MAX) return PA_ERR_UNSUPPORTED;  // the kernels count (item, KV head) pairs in 32 bits
   if (reinterpret_cast<uintptr_t>(workspace) & 255u) return PA_ERR_INVALID;
 
   int dev;
@@ -396,6 +413,7 @@ int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cac
   p.out_dtype = out_dtype;
   p.qtok = qtok;
   p.qtok_item = qtok_item;
+  p.qbox_rows = qtok > 1 ? qtok_item : max_members;
   p.groups = groups;
   p.num_groups = num_groups;
   p.max_members = max_members;
@@ -414,15 +432,19 @@ int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cac
   pa::pa_decode_plan_kernel<<<1, pa::kPlanThreads, 0, st>>>(p);
   if (cudaPeekAtLastError() != cudaSuccess) return PA_ERR_CUDA;
 
-  const int64_t max_items = static_cast<int64_t>(num_seqs) * max_parts * ncg * num_kv_heads;
   int rc;
   const int c = static_cast<int>(cols);
+  CUtensorMap tmq;
+  if (use_tc && encode_q_map(&tmq, q, q_dtype, static_cast<int64_t>(num_seqs) * qtok, num_q_heads, G,
+                             p.qbox_rows) != PA_OK)
+    return PA_ERR_CUDA;
+  const CUtensorMap* tq = use_tc ? &tmq : nullptr;
   if (block_size == 16)
-    rc = head_dim == 128 ? dispatch_kv<16, 128>(p, tmk, tmv, max_items, dev, info, kv_dtype, q_dtype, c, st)
-                         : dispatch_kv<16, 64>(p, tmk, tmv, max_items, dev, info, kv_dtype, q_dtype, c, st);
+    rc = head_dim == 128 ? dispatch_kv<16, 128>(p, tmk, tmv, tq, max_items, dev, info, kv_dtype, q_dtype, c, st)
+                         : dispatch_kv<16, 64>(p, tmk, tmv, tq, max_items, dev, info, kv_dtype, q_dtype, c, st);
   else
-    rc = head_dim == 128 ? dispatch_kv<32, 128>(p, tmk, tmv, max_items, dev, info, kv_dtype, q_dtype, c, st)
-                         : dispatch_kv<32, 64>(p, tmk, tmv, max_items, dev, info, kv_dtype, q_dtype, c, st);
+    rc = head_dim == 128 ? dispatch_kv<32, 128>(p, tmk, tmv, tq, max_items, dev, info, kv_dtype, q_dtype, c, st)
+                         : dispatch_kv<32, 64>(p, tmk, tmv, tq, max_items, dev, info, kv_dtype, q_dtype, c, st);
   if (rc != PA_OK) return rc;
   {  // merge kernel: waits (griddepcontrol.wait) for the partition kernel's partial results
     const int64_t warps = static_cast<int64_t>(num_seqs) * qtok * num_q_heads;
@@ -578,6 +600,7 @@ int pa_copy_blocks(void* k_cache, void* v_cache, const int32_t* src_dst_pairs, i
       if (srcs.count(d)) return PA_ERR_INVALID;
   }
   const int64_t vecs = static_cast<int64_t>(block_bytes / 16);
+  // chunks of 4 vectors per thread (a 32 KB block: 2 chunks of 256 threads)
   const int chunks = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(16, vecs / (256 * 4))));
   pa::pa_copy_blocks_kernel<<<dim3(static_cast<unsigned>(num_pairs), 2, static_cast<unsigned>(chunks)), 256, 0,
                               static_cast<cudaStream_t>(stream)>>>(static_cast<uint8_t*>(k_cache),

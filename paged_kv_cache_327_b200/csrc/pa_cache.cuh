@@ -20,21 +20,37 @@ __global__ void __launch_bounds__(128)
                                 const int64_t* __restrict__ slots, int num_tokens, int64_t row_bytes,
                                 int64_t k_stride_bytes, int64_t v_stride_bytes, int64_t num_slots) {
   const int64_t vecs = row_bytes >> 4;
-  for (int t = blockIdx.x; t < num_tokens; t += gridDim.x) {
-    const int64_t s = slots[t];
-    if (s < 0) continue;
-    if (s >= num_slots) {
-      if (threadIdx.x == 0) record_error(DEV_BAD_SLOT);
-      continue;
-    }
+  // two tokens per iteration (t and t + gridDim.x): their rows are read together with their slots
+  // (the loads do not wait for each other); a slot only decides whether, and where, a row is stored
+  for (int t = blockIdx.x; t < num_tokens; t += 2 * gridDim.x) {
+    const int t2 = t + gridDim.x;
+    const bool two = t2 < num_tokens;
+    const int64_t s = slots[t], s2 = two ? slots[t2] : -1;
+    const bool st = s >= 0 && s < num_slots, st2 = s2 >= 0 && s2 < num_slots;
+    if (threadIdx.x == 0 && (s >= num_slots || s2 >= num_slots)) record_error(DEV_BAD_SLOT);
     const uint4* ks = reinterpret_cast<const uint4*>(k + t * k_stride_bytes);
     const uint4* vs = reinterpret_cast<const uint4*>(v + t * v_stride_bytes);
-    uint4* kd = reinterpret_cast<uint4*>(kc + s * row_bytes);
-    uint4* vd = reinterpret_cast<uint4*>(vc + s * row_bytes);
+    const uint4* ks2 = reinterpret_cast<const uint4*>(k + (two ? t2 : t) * k_stride_bytes);
+    const uint4* vs2 = reinterpret_cast<const uint4*>(v + (two ? t2 : t) * v_stride_bytes);
+    uint4* kd = reinterpret_cast<uint4*>(kc + (st ? s : 0) * row_bytes);
+    uint4* vd = reinterpret_cast<uint4*>(vc + (st ? s : 0) * row_bytes);
+    uint4* kd2 = reinterpret_cast<uint4*>(kc + (st2 ? s2 : 0) * row_bytes);
+    uint4* vd2 = reinterpret_cast<uint4*>(vc + (st2 ? s2 : 0) * row_bytes);
     for (int64_t i = threadIdx.x; i < vecs; i += blockDim.x) {
       const uint4 a = __ldg(ks + i), b = __ldg(vs + i);
-      kd[i] = a;
-      vd[i] = b;
+      uint4 a2 = a, b2 = b;
+      if (two) {
+        a2 = __ldg(ks2 + i);
+        b2 = __ldg(vs2 + i);
+      }
+      if (st) {
+        kd[i] = a;
+        vd[i] = b;
+      }
+      if (st2) {
+        kd2[i] = a2;
+        vd2[i] = b2;
+      }
     }
   }
 }
@@ -69,21 +85,22 @@ __global__ void __launch_bounds__(128)
                                     int64_t k_stride, int64_t v_stride, int64_t num_slots, float k_scale,
                                     float v_scale) {
   for (int t = blockIdx.x; t < num_tokens; t += gridDim.x) {
+    // as in the 16-bit store, the rows are read together with the slot, which only guards the stores
     const int64_t s = slots[t];
-    if (s < 0) continue;
-    if (s >= num_slots) {
-      if (threadIdx.x == 0) record_error(DEV_BAD_SLOT);
-      continue;
-    }
+    const bool store = s >= 0 && s < num_slots;
+    if (s >= num_slots && threadIdx.x == 0) record_error(DEV_BAD_SLOT);
     for (int64_t i = threadIdx.x * 8; i < row; i += blockDim.x * 8) {
+      float x[2][8];
+      load8(k + t * k_stride + i, x[0]);
+      load8(v + t * v_stride + i, x[1]);
+      if (!store) continue;
 #pragma unroll
       for (int which = 0; which < 2; ++which) {
-        float x[8];
-        load8((which ? v + t * v_stride : k + t * k_stride) + i, x);
         const float sc = which ? v_scale : k_scale;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) x[j] = __fdiv_rn(x[j], sc);
-        const uint2 w = make_uint2(e4m3x4(x[0], x[1], x[2], x[3]), e4m3x4(x[4], x[5], x[6], x[7]));
+        for (int j = 0; j < 8; ++j) x[which][j] = __fdiv_rn(x[which][j], sc);
+        const uint2 w = make_uint2(e4m3x4(x[which][0], x[which][1], x[which][2], x[which][3]),
+                                   e4m3x4(x[which][4], x[which][5], x[which][6], x[which][7]));
         *reinterpret_cast<uint2*>((which ? vc : kc) + s * row + i) = w;
       }
     }
@@ -104,9 +121,16 @@ __global__ void __launch_bounds__(256)
   const uint4* s = reinterpret_cast<const uint4*>(base + src * block_bytes);
   uint4* d = reinterpret_cast<uint4*>(base + dst * block_bytes);
   const int64_t vecs = block_bytes >> 4;
-  for (int64_t i = threadIdx.x + static_cast<int64_t>(blockIdx.z) * blockDim.x; i < vecs;
-       i += static_cast<int64_t>(blockDim.x) * gridDim.z)
-    d[i] = s[i];
+  const int64_t stride = static_cast<int64_t>(blockDim.x) * gridDim.z;
+  int64_t i = threadIdx.x + static_cast<int64_t>(blockIdx.z) * blockDim.x;
+  for (; i + 3 * stride < vecs; i += 4 * stride) {  // four 16-byte loads in flight per thread
+    const uint4 a = s[i], b = s[i + stride], c = s[i + 2 * stride], e = s[i + 3 * stride];
+    d[i] = a;
+    d[i + stride] = b;
+    d[i + 2 * stride] = c;
+    d[i + 3 * stride] = e;
+  }
+  for (; i < vecs; i += stride) d[i] = s[i];
 }
 
 }  // namespace pa

@@ -87,6 +87,7 @@ struct DecodeParams {
   int head_dim, block_size, max_blocks_per_seq, num_blocks;
   int partition_size, max_parts, out_dtype, qtok;  // qtok: query tokens per sequence (1 = decode)
   int qtok_item;     // query tokens of one item (qtok, or fewer: then several column groups)
+  int qbox_rows;     // query rows per grouped head that the tensor-core kernel stages for an item
   // prefix groups, int32 [num_groups][3] = (first sequence, members, shared tokens): sequences
   // first .. first + members - 1 hold the same blocks for their first `shared` tokens
   const int32_t* groups;
@@ -113,33 +114,47 @@ __device__ __forceinline__ void store_out(void* out, int64_t idx, float v, int d
 }
 
 // ------------------------------------------------------------------------------ plan
-template <typename T>
-__device__ __forceinline__ T warp_inclusive_scan(T v) {
+struct ScanSum {
+  template <typename T>
+  __device__ __forceinline__ T operator()(T a, T b) const { return a + b; }
+};
+struct ScanMax {
+  template <typename T>
+  __device__ __forceinline__ T operator()(T a, T b) const { return a > b ? a : b; }
+};
+
+template <typename T, typename Op>
+__device__ __forceinline__ T warp_inclusive_scan(T v, Op op) {
   const int lane = threadIdx.x & 31;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
     const T n = __shfl_up_sync(0xffffffffu, v, o);
-    if (lane >= o) v += n;
+    if (lane >= o) v = op(n, v);
   }
   return v;
 }
 
-// Exclusive prefix sum over the block (blockDim.x a multiple of 32, at most 1024);
-// *total receives the block sum.  A 64-bit T scans two 32-bit counts at once (low + high << 32).
-template <typename T>
-__device__ T block_exclusive_scan(T v, T* s_warp, T* total) {
+// Exclusive scan over the block (blockDim.x a multiple of 32, at most 1024) with an associative,
+// commutative op whose identity is id; *total receives the reduction of all values.  A 64-bit T
+// under ScanSum scans two 32-bit counts at once (low + high << 32).
+template <typename T, typename Op>
+__device__ T block_exclusive_scan(T v, T id, Op op, T* s_warp, T* total) {
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
-  const T inc = warp_inclusive_scan(v);
+  const T inc = warp_inclusive_scan(v, op);
+  T exc = __shfl_up_sync(0xffffffffu, inc, 1);
+  if (lane == 0) exc = id;
   if (lane == 31) s_warp[w] = inc;
   __syncthreads();
   if (w == 0) {
-    const T x = lane < nw ? s_warp[lane] : T(0);
-    const T xi = warp_inclusive_scan(x);
-    if (lane < nw) s_warp[lane] = xi - x;
+    const T x = lane < nw ? s_warp[lane] : id;
+    const T xi = warp_inclusive_scan(x, op);
+    T xe = __shfl_up_sync(0xffffffffu, xi, 1);
+    if (lane == 0) xe = id;
+    if (lane < nw) s_warp[lane] = xe;
     if (lane == 31) s_warp[32] = xi;
   }
   __syncthreads();
-  const T r = s_warp[w] + inc - v;
+  const T r = op(s_warp[w], exc);
   *total = s_warp[32];
   __syncthreads();
   return r;
@@ -151,8 +166,11 @@ __device__ __forceinline__ long long pack2x32(int lo, int hi) {
 __device__ __forceinline__ int lo32(long long v) { return static_cast<int>(v & 0xffffffffll); }
 __device__ __forceinline__ int hi32(long long v) { return static_cast<int>(v >> 32); }
 
-constexpr int kPlanThreads = 256;
+constexpr int kPlanThreads = 1024;
 
+// seq_parts values besides the partial-result count (0: the sequence's item writes `out`):
+// rows the merge kernel fills, with zeros (an empty sequence) or NaN (an invalid length)
+constexpr int kPartsEmpty = -1, kPartsInvalid = -2;
 
 // Work list of one call.  Per sequence i of length L (valid: 0 <= L <= max_len and L = 0 or
 // L >= qtok) with S shared tokens (0 outside a prefix group):
@@ -161,7 +179,9 @@ constexpr int kPlanThreads = 256;
 //   * own items: tokens [S, L) in partitions of P tokens (full ones, then a ragged tail).
 // The partial results of sequence i are numbered shared partitions first, then its own; a
 // sequence with no shared tokens and one partition writes `out` directly.  Items are listed
-// shared first (the widest), then full partitions, then tails.
+// shared first (the widest), then full partitions, then tails, each kind in sequence order.
+// Thread t plans the contiguous run of sequences [t * chunk, (t + 1) * chunk): every count
+// is one block-wide scan, whatever the batch size.
 __global__ void __launch_bounds__(kPlanThreads) pa_decode_plan_kernel(const DecodeParams p) {
   // the partition kernel may start its prologue now; it waits for this grid before
   // touching anything written here
@@ -169,56 +189,98 @@ __global__ void __launch_bounds__(kPlanThreads) pa_decode_plan_kernel(const Deco
   __shared__ long long s_warp[33];
   const int N = p.num_seqs, P = p.partition_size, BS = p.block_size;
   const int max_len = p.max_blocks_per_seq * p.block_size;
+  const int chunk = (N + blockDim.x - 1) / blockDim.x;
+  const int lo = min(N, static_cast<int>(threadIdx.x) * chunk), hi = min(N, lo + chunk);
   auto valid_len = [&](int L) { return L >= 0 && L <= max_len && (L == 0 || L >= p.qtok); };
 
   if (p.num_groups > 0) {
     // A group is used if it is in range, its shared tokens are whole blocks that every member
     // holds, and no other group claims any of its sequences; otherwise it is reported and its
-    // sequences decode alone.  seq_sub first counts the claims on each sequence; each group's
-    // verdict is kept in the (not yet written) work list, one int per group (num_groups <= N).
+    // sequences decode alone.  Every group in range claims its members: claims start as a
+    // difference array (+1 at first, -1 after the last member) whose prefix sum counts the
+    // claims on each sequence; (1 + group index) is written at each group's first sequence, and a
+    // prefix maximum of the positions that hold one finds, for a sequence claimed once, the
+    // latest group start at or before it: the group that claims it.  A member rules its group out
+    // if it is claimed more than once, its length is invalid or it holds fewer than the shared
+    // tokens; an exclusive prefix count of such members gives each group's verdict in one
+    // subtraction.  The verdicts are kept in the (not yet written) work list, one int per group
+    // (num_groups <= N); seq_sub, seq_parts and seq_shared serve as scratch until their final
+    // values are written.
     int* verdict = reinterpret_cast<int*>(p.items);
-    for (int i = threadIdx.x; i < N; i += blockDim.x) p.seq_shared[i] = p.seq_sub[i] = 0;
+    int* claim = p.seq_sub;     // claims, then the claiming group of a sequence claimed once (or -1)
+    int* cover = p.seq_parts;   // 1 + index of the group that starts at the sequence (0: none)
+    int* badpre = p.seq_shared;
+    const int* gr = p.groups;
+    for (int i = threadIdx.x; i < N; i += blockDim.x) claim[i] = cover[i] = 0;
     __syncthreads();
     for (int g = threadIdx.x; g < p.num_groups; g += blockDim.x) {
-      const int first = p.groups[3 * g], M = p.groups[3 * g + 1], S = p.groups[3 * g + 2];
-      bool ok = first >= 0 && M >= 1 && first <= N - M && S >= 0 && S % BS == 0;
-      if (ok) {
-#pragma unroll 4
-        for (int m = 0; m < M; ++m) {  // independent loads: no early exit
-          const int L = p.seq_lens[first + m];
-          ok &= valid_len(L) && S <= L;
-        }
-      }
+      const int first = gr[3 * g], M = gr[3 * g + 1], S = gr[3 * g + 2];
+      const bool ok = first >= 0 && M >= 1 && first <= N - M && S >= 0 && S % BS == 0;
       verdict[g] = ok;
       if (!ok) {
         record_error(DEV_BAD_PREFIX);
         continue;
       }
-      for (int m = 0; m < M; ++m) atomicAdd(&p.seq_sub[first + m], 1);
+      atomicAdd(&claim[first], 1);
+      if (first + M < N) atomicSub(&claim[first + M], 1);
+      atomicMax(&cover[first], g + 1);
+    }
+    __syncthreads();
+    int csum = 0, smax = 0;  // smax: 1 + the latest position holding a group start
+    for (int i = lo; i < hi; ++i) {
+      csum += claim[i];
+      if (cover[i] > 0) smax = i + 1;
+    }
+    long long tot;
+    int c = static_cast<int>(block_exclusive_scan<long long>(csum, 0, ScanSum{}, s_warp, &tot));
+    int sp = static_cast<int>(block_exclusive_scan<long long>(smax, 0, ScanMax{}, s_warp, &tot));
+    int nbad = 0;
+    for (int i = lo; i < hi; ++i) {
+      c += claim[i];
+      if (cover[i] > 0) sp = i + 1;
+      // a sequence claimed once lies in the group that starts last at or before it (cover is
+      // only read here, so any thread may look up any start)
+      const int g = c == 1 ? cover[sp - 1] - 1 : -1;
+      bool bad = c > 1;
+      if (g >= 0) {
+        const int L = p.seq_lens[i];
+        bad = !valid_len(L) || gr[3 * g + 2] > L;
+      }
+      claim[i] = g;
+      badpre[i] = bad;
+      nbad += bad;
+    }
+    int b = static_cast<int>(block_exclusive_scan<long long>(nbad, 0, ScanSum{}, s_warp, &tot));
+    const int bad_total = static_cast<int>(tot);
+    for (int i = lo; i < hi; ++i) {
+      const int x = badpre[i];
+      badpre[i] = b;
+      b += x;
     }
     __syncthreads();
     for (int g = threadIdx.x; g < p.num_groups; g += blockDim.x) {
       if (!verdict[g]) continue;
-      const int first = p.groups[3 * g], M = p.groups[3 * g + 1], S = p.groups[3 * g + 2];
-      bool alone = true;
-#pragma unroll 4
-      for (int m = 0; m < M; ++m) alone &= p.seq_sub[first + m] == 1;
-      if (!alone) {
+      const int first = gr[3 * g], end = first + gr[3 * g + 1];
+      if ((end < N ? badpre[end] : bad_total) != badpre[first]) {
         verdict[g] = 0;
         record_error(DEV_BAD_PREFIX);
-        continue;
       }
-      if (S > 0 && M > 1)
-        for (int m = 0; m < M; ++m) p.seq_shared[first + m] = S;
     }
     __syncthreads();
-    for (int i = threadIdx.x; i < N; i += blockDim.x) p.seq_sub[i] = 0;
-    __syncthreads();
-    for (int g = threadIdx.x; g < p.num_groups; g += blockDim.x) {
-      if (!verdict[g]) continue;
-      const int first = p.groups[3 * g], M = p.groups[3 * g + 1], S = p.groups[3 * g + 2];
-      if (S == 0 || M == 1) continue;
-      for (int m = 0; m < M; m += p.max_members) p.seq_sub[first + m] = min(p.max_members, M - m);
+    // the sequences' shared tokens, and the members each leader of a shared pass covers
+    for (int i = lo; i < hi; ++i) {
+      int sh = 0, sub = 0;
+      const int g = claim[i];
+      if (g >= 0 && verdict[g]) {
+        const int first = gr[3 * g], M = gr[3 * g + 1], S = gr[3 * g + 2];
+        if (S > 0 && M > 1) {
+          sh = S;
+          const int k = i - first;
+          if (k % p.max_members == 0) sub = min(p.max_members, M - k);
+        }
+      }
+      p.seq_shared[i] = sh;
+      p.seq_sub[i] = sub;
     }
     __syncthreads();  // the verdicts are dead from here on: the work list overwrites them
   }
@@ -241,62 +303,45 @@ __global__ void __launch_bounds__(kPlanThreads) pa_decode_plan_kernel(const Deco
     return c;
   };
 
-  int loc_s = 0, loc_f = 0;
-  for (int i = threadIdx.x; i < N; i += blockDim.x) {
+  int loc_s = 0, loc_f = 0, loc_t = 0;
+  for (int i = lo; i < hi; ++i) {
     const Counts c = counts(i);
     loc_s += c.ns;
     loc_f += c.nf * ncg;
+    loc_t += c.nt * ncg;
   }
-  long long tot;
-  block_exclusive_scan(pack2x32(loc_f, loc_s), s_warp, &tot);
-  const int n_full = lo32(tot), n_shared = hi32(tot);
-  int base_s = 0, base_f = 0, base_t = 0;
-  for (int start = 0; start < N; start += blockDim.x) {
-    const int i = start + threadIdx.x;
-    Counts c{};
-    if (i < N) {
-      c = counts(i);
-      const bool valid = valid_len(c.L);
-      if (!valid) record_error(DEV_BAD_SEQ_LEN);
-      if (!valid || c.L == 0) {  // no work item: the rows are zero (empty) or NaN (invalid)
-        const float v = valid ? 0.f : CUDART_NAN_F;
-        const int64_t row = static_cast<int64_t>(p.qtok) * p.num_q_heads * p.head_dim;
-        for (int64_t e = 0; e < row; ++e) store_out(p.out, i * row + e, v, p.out_dtype);
-      }
-      const int parts = c.nps + c.nf + c.nt;
-      const bool direct = c.S == 0 && parts == 1;
-      p.seq_parts[i] = direct ? 0 : parts;
-    }
-    long long tft;
-    const long long oft = block_exclusive_scan(pack2x32(c.nf * ncg, c.nt * ncg), s_warp, &tft);
-    const int of = lo32(oft), ot = hi32(oft), tf = lo32(tft), tt = hi32(tft);
-    int os = 0, ts = 0;
-    if (n_shared > 0) {  // block-uniform
-      long long tsl;
-      os = static_cast<int>(block_exclusive_scan(static_cast<long long>(c.ns), s_warp, &tsl));
-      ts = static_cast<int>(tsl);
-    }
+  long long tft;
+  const long long oft = block_exclusive_scan<long long>(pack2x32(loc_f, loc_t), 0, ScanSum{}, s_warp, &tft);
+  int of = lo32(oft), ot = hi32(oft), os = 0, n_shared = 0;
+  const int n_full = lo32(tft), n_tail = hi32(tft);
+  if (p.num_groups > 0) {  // block-uniform
+    long long tsl;
+    os = static_cast<int>(block_exclusive_scan<long long>(loc_s, 0, ScanSum{}, s_warp, &tsl));
+    n_shared = static_cast<int>(tsl);
+  }
+  for (int i = lo; i < hi; ++i) {
+    const Counts c = counts(i);
+    const bool valid = valid_len(c.L);
+    if (!valid) record_error(DEV_BAD_SEQ_LEN);
+    const int parts = c.nps + c.nf + c.nt;
+    const bool direct = c.S == 0 && parts == 1;
+    p.seq_parts[i] = !valid ? kPartsInvalid : c.L == 0 ? kPartsEmpty : direct ? 0 : parts;
     const int dflag = (c.S == 0 && c.nf + c.nt == 1) ? WI_DIRECT : 0;
     // shared items have one query token (prefix groups are single-token decode)
     for (int k = 0; k < c.ns; ++k)
-      p.items[base_s + os + k] = WorkItem{i, k * P, min(c.S, (k + 1) * P), k | (c.sub << 16), 0, 1, 0, 0};
+      p.items[os++] = WorkItem{i, k * P, min(c.S, (k + 1) * P), k | (c.sub << 16), 0, 1, 0, 0};
     for (int k = 0; k < c.nf; ++k)
       for (int j = 0; j < ncg; ++j)
-        p.items[n_shared + base_f + of + k * ncg + j] =
-            WorkItem{i, c.S + k * P, c.S + (k + 1) * P, (c.nps + k) | (1 << 16) | dflag, j * Tc,
-                     min(Tc, p.qtok - j * Tc), 0, 0};
+        p.items[n_shared + of++] = WorkItem{i, c.S + k * P, c.S + (k + 1) * P, (c.nps + k) | (1 << 16) | dflag,
+                                            j * Tc, min(Tc, p.qtok - j * Tc), 0, 0};
     if (c.nt)
       for (int j = 0; j < ncg; ++j)
-        p.items[n_shared + n_full + base_t + ot + j] =
-            WorkItem{i, c.S + c.nf * P, c.L, (c.nps + c.nf) | (1 << 16) | dflag, j * Tc,
-                     min(Tc, p.qtok - j * Tc), 0, 0};
-    base_s += ts;
-    base_f += tf;
-    base_t += tt;
+        p.items[n_shared + n_full + ot++] = WorkItem{i, c.S + c.nf * P, c.L, (c.nps + c.nf) | (1 << 16) | dflag,
+                                                     j * Tc, min(Tc, p.qtok - j * Tc), 0, 0};
   }
   if (threadIdx.x == 0) {
     p.counters[0] = 0;
-    p.counters[1] = static_cast<unsigned>(n_shared + n_full + base_t);
+    p.counters[1] = static_cast<unsigned>(n_shared + n_full + n_tail);
   }
 }
 
@@ -1001,12 +1046,18 @@ __global__ void __launch_bounds__(kMergeWarps * 32) pa_decode_merge_kernel(const
   int np;
   if (p.num_groups == 0) {  // the partitions follow from the length alone
     const int L = p.seq_lens[seq], P = p.partition_size;
-    if (L <= P || L > p.max_blocks_per_seq * p.block_size) return;  // direct, empty or invalid rows
-    np = (L + P - 1) / P;
+    const bool valid = L >= 0 && L <= p.max_blocks_per_seq * p.block_size && (L == 0 || L >= p.qtok);
+    np = !valid ? kPartsInvalid : L == 0 ? kPartsEmpty : L <= P ? 0 : (L + P - 1) / P;
   } else {
     np = p.seq_parts[seq];
-    if (np == 0) return;  // written directly, or empty / invalid
   }
+  if (np < 0) {  // no work item: the row is zero (empty sequence) or NaN (invalid length)
+    const float v = np == kPartsEmpty ? 0.f : CUDART_NAN_F;
+    const int64_t o = (static_cast<int64_t>(seq) * Hq + hq) * D;
+    for (int d = lane; d < D; d += 32) store_out(p.out, o + d, v, p.out_dtype);
+    return;
+  }
+  if (np == 0) return;  // written directly by the sequence's only item
   const int64_t base = static_cast<int64_t>(seq) * p.max_parts;
   float M = -CUDART_INF_F;
   for (int k = lane; k < np; k += 32) M = fmaxf(M, __ldcg(&p.part_ml[(base + k) * Hq + hq].x));

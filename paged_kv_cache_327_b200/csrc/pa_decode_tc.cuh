@@ -1,27 +1,30 @@
 // pa_decode_tc.cuh -- the partition kernel for wide work items on the 5th-generation tensor cores.
 //
-// Items with 9 to 32 query rows per KV head (several query tokens of a sequence, or the members of
-// a shared prefix) carry 2-4x decode's math per K/V byte.  The kernel works on chunks of 8 pages
-// (128 tokens) of one item, in the transposed form, so that both products have M = 128 with no
-// padding and the softmax spreads over 128 threads:
-//   S^T = K . Q^T     tcgen05.mma, M = 128 tokens, N = the item's query rows (16 or 32),
-//                     K = head_dim; A = the chunk's K rows (TMA-staged, 128-byte swizzle),
-//                     B = the query rows (written swizzled by the producer), D in tensor memory
-//   softmax           thread t of the 128 consumer threads owns token t of the chunk (TMEM lane t)
-//                     and holds, per query row, the running maximum and its own partial row sum;
-//                     the maximum is raised (a CTA-wide vote) only when a score exceeds it by more
-//                     than 2^8, and the O columns are then rescaled in tensor memory
-//   O^T += V^T . P^T  tcgen05.mma per page, M = head_dim, N = query rows, K = 16 tokens;
-//                     A = the staged V page read in place (MN-major), B = P^T in shared memory
-// At the item's end the partial row sums are reduced across the 128 threads and thread d writes
-// element d of every output row (coalesced).  The MMAs are issued by one thread and complete on
-// mbarriers; the O product also releases the chunk's buffer to the producer.  The warp-MMA kernel
-// of pa_decode.cuh is the default for these items (faster on B200); this one is chosen with
-// pa_set_option(PA_OPT_WIDE_KERNEL, PA_WIDE_TCGEN05).
+// Items with several query rows per KV head (the query tokens of a sequence, or the members of a
+// shared prefix: up to 64 rows) carry up to 8x decode's math per K/V byte.  The query rows sit on
+// the M dimension of the products, so that every softmax reduction stays on the row's lane:
+//   S = Q . K^T      tcgen05.mma, M = 64 query rows, N = 64 tokens (a chunk of 4 pages), K =
+//                    head_dim; A = the item's query rows (TMA-staged once per item), B = the
+//                    chunk's K rows (TMA-staged, 128-byte swizzle), D in tensor memory
+//   softmax          two warps share each TMEM lane quarter; the lane of query row r in each owns
+//                    half of the row's 64 scores: it keeps the row's running maximum (agreed with
+//                    the other half through shared memory) and its half of the running sum, raises
+//                    the maximum (and rescales the O row in tensor memory) only when a score
+//                    exceeds it by more than 2^8, and writes its half of the row's weights P,
+//                    rounded to the operand type, to shared memory
+//   O += P . V       tcgen05.mma per page, M = 64, N = head_dim, K = 16 tokens; A = P, B = the
+//                    staged V page read in place (MN-major)
+// At the item's end each half-row's lane writes half of the row's head_dim outputs, divided by the
+// row's sum.  S and O products are issued by two warps of their own, so that neither waits for the
+// other's issue, and complete on mbarriers.  Double buffers keep every stage busy: two S buffers
+// and two P buffers (chunk n's softmax runs while the tensor core works on chunk n - 1's O and
+// chunk n + 1's S), two O buffers (an item's output is read while the next item accumulates), two
+// query buffers and five chunk buffers of 32 KB in flight per SM.
 //
-// CTA (one per SM): 3 chunk buffers of 64 KB; warps 0-3 run the softmax and the output (TMEM lane
-// quarters 0-3), warp 4 produces (the work list, TMA for K/V, plain loads for the query rows),
-// warp 5 issues every MMA.  Block size 16, head_dim 128, 16-bit cache and query.
+// CTA (one per SM): warps 0-7 run the softmax and the output (warp w on TMEM lane quarter w % 4,
+// columns 32 (w / 4) .. 32 (w / 4) + 31 of each chunk), warp 8 produces (the work list, TMA for the
+// K/V pages and the query rows), warp 9 issues the S products, warp 10 the O products.
+// Block size 16, head_dim 128, 16-bit cache and query.
 #pragma once
 
 #include "pa_decode.cuh"
@@ -133,69 +136,90 @@ __device__ __forceinline__ void tmem_stn(uint32_t taddr, const uint32_t (&v)[N])
 }
 
 // ---------------------------------------------------------------- configuration
-template <typename KT, int N>
+template <typename KT>
 struct TcCfg {
-  static_assert(N == 16 || N == 32, "query rows per item");
-  static constexpr int BS = 16, D = 128, QE = 2;
-  static constexpr int CH = 8;                             // pages per chunk: 128 tokens
-  static constexpr int NCH = 3;                            // chunk buffers
-  static constexpr int BOX = BS * 128;                     // one TMA box: 16 rows x 128 bytes
-  static constexpr int KH_BYTES = CH * BOX;                // one 64-element half of the chunk's K rows
-  static constexpr int VPAGE = 2 * BOX;                    // a V page: two halves
+  static constexpr int BS = 16, D = 128;
+  static constexpr int M = 64;                              // MMA rows: the item's query rows
+  static constexpr int CH = 4;                              // pages per chunk
+  static constexpr int CT = CH * BS;                        // tokens per chunk: N of S
+  static constexpr int NCH = 5;                             // chunk buffers
+  static constexpr int BOX = BS * 128;                      // one TMA box: 16 rows x 128 bytes
+  static constexpr int KH_BYTES = CH * BOX;                 // one 64-element half of the chunk's K rows
+  static constexpr int VPAGE = 2 * BOX;                     // a V page: two halves
   static constexpr int CHUNK_BYTES = 2 * KH_BYTES + CH * VPAGE;
-  static constexpr int OPB = 2 * N * 128;                  // Q or P^T operand: 2 halves of N rows x 128 bytes
-  static constexpr int QN = 2;                             // query buffers
+  static constexpr int QHALF = M * 128;                     // one 64-element half of the query rows
+  static constexpr int QBUF = 2 * QHALF;
+  static constexpr int QN = 2;                              // query buffers
+  static constexpr int PBUF = M * 128;                      // P: M rows x 64 tokens (one swizzle atom wide)
   static constexpr int OFF_Q = NCH * CHUNK_BYTES;
-  static constexpr int OFF_P = OFF_Q + QN * OPB;
-  static constexpr int OFF_BAR = OFF_P + OPB;
-  // mbarriers: chunk full / empty, query buffer free, S^T buffer full / free, P^T full, O product
-  // done, final drain of the tensor pipe
+  static constexpr int OFF_P = OFF_Q + QN * QBUF;
+  static constexpr int OFF_BAR = OFF_P + 2 * PBUF;
+  // mbarriers: chunk full / empty, query buffer free, S full / free, P full / free (the O product
+  // that read it is done), O buffer free (its item's output has been read), final drain
   static constexpr int B_FULL = 0, B_EMPTY = NCH, B_QFREE = 2 * NCH, B_SFULL = B_QFREE + QN, B_SFREE = B_SFULL + 2,
-                       B_PFULL = B_SFREE + 2, B_ODONE = B_PFULL + 1, B_FIN = B_ODONE + 1, NBAR = B_FIN + 1;
+                       B_PFULL = B_SFREE + 2, B_PFREE = B_PFULL + 2, B_OFREE = B_PFREE + 2, B_FIN = B_OFREE + 2,
+                       NBAR = B_FIN + 1;
   static constexpr int OFF_META = OFF_BAR + ((NBAR * 8 + 15) & ~15);
-  static constexpr int OFF_RED = OFF_META + NCH * 32;
-  // reductions: per-warp partials [4][N], row maxima [N], rescale factors [N], output scales [N],
-  // output offsets [N] (int64)
-  static constexpr int OFF_MISC = OFF_RED + 7 * N * 4 + N * 8;
+  // exchange between the two softmax warps of a lane quarter: chunk maxima [2 S buffers][2 halves][M]
+  // and item sums [2 items][2 halves][M]
+  static constexpr int OFF_XCH = OFF_META + NCH * 32;
+  static constexpr int OFF_MISC = OFF_XCH + 8 * M * 4;
   static constexpr int SMEM_BYTES = 1024 + OFF_MISC + 16;
-  // warps 0-3 consume (softmax, output), warp 4 loads, warp 5 issues the MMAs
-  static constexpr int NCONS = 128, NTHREADS = NCONS + 64;
-  // TMEM columns: O^T, then two S^T buffers
-  static constexpr uint32_t TM_COLS = 3 * N <= 64 ? 64 : 128, TM_O = 0, TM_S = N;
+  // warps 0-7: softmax and output, warp 8 loads, warp 9 issues the S products, warp 10 the O products
+  static constexpr int NSM = 256, W_LOAD = 8, W_S = 9, W_O = 10, NTHREADS = NSM + 96;
+  static constexpr int HC = CT / 2;  // chunk columns per softmax warp
+  // TMEM columns: two O buffers (head_dim columns each), then two S buffers (one chunk each)
+  static constexpr uint32_t TM_COLS = 512, TM_O = 0, TM_S = 2 * D;
   static constexpr uint32_t AB = std::is_same<KT, __nv_bfloat16>::value ? 1u : 0u;
-  static constexpr uint32_t IDESC_S = umma_idesc(AB, 0, 0, 128, N);  // K (K-major) . Q^T (K-major)
-  static constexpr uint32_t IDESC_O = umma_idesc(AB, 1, 0, 128, N);  // V^T (MN-major) . P^T (K-major)
-  static_assert(CHUNK_BYTES % 1024 == 0 && OFF_Q % 1024 == 0 && OPB % 1024 == 0 && (N * 128) % 1024 == 0,
+  static constexpr uint32_t IDESC_S = umma_idesc(AB, 0, 0, M, CT);  // Q (K-major) . K^T (K-major)
+  static constexpr uint32_t IDESC_O = umma_idesc(AB, 0, 1, M, D);   // P (K-major) . V (MN-major)
+  static_assert(CHUNK_BYTES % 1024 == 0 && OFF_Q % 1024 == 0 && QHALF % 1024 == 0 && OFF_P % 1024 == 0,
                 "128-byte swizzle atoms");
+  static_assert(TM_S + 2 * CT <= TM_COLS, "tensor memory");
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
 };
 
-// ---------------------------------------------------------------- producer (warp 4)
-// The loads that place an item (its work-list entry, block-table row, sequence length and query
-// rows) form a chain of dependent global reads.  The producer runs it ahead of the ring: while the
-// chunks of item k are issued, the entry of item k + 2 and the rest of item k + 1 are in flight.
-template <int QPL>
+// TMEM lane of row r of an M = 64 product (and of its operand A): rows 16 q .. 16 q + 15 occupy
+// lanes 0-15 of lane quarter q.  Returns -1 for a lane that holds no row.
+__device__ __forceinline__ int tc_lane_row(int lane128) {
+  return (lane128 & 31) < 16 ? (lane128 >> 5) * 16 + (lane128 & 31) : -1;
+}
+
+// 4-D tiled TMA load global -> shared, completion counted on `bar` in bytes (no cache hint).
+__device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, int x, int y, int z, int w,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(w), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// ---------------------------------------------------------------- producer (warp 8)
+// The loads that place an item (its work-list entry, block-table row) form a chain of dependent
+// global reads.  The producer runs it ahead of the ring: while the chunks of item k are issued,
+// the entry of item k + 2 and the block-table row of item k + 1 are in flight.
 struct TcItemLoads {
   bool valid;
   WorkItem it;
   int kvh, bt, rel0;
   bool mismatch;
-  uint4 qv[QPL];
 };
 
-template <typename C, int N>
+template <typename C>
 __device__ __forceinline__ void tc_produce(const DecodeParams& p, const CUtensorMap& tmk, const CUtensorMap& tmv,
-                                           uint8_t* smem, uint64_t* bars, int4* meta, volatile int* abort_flag,
-                                           int lane) {
+                                           const CUtensorMap& tmq, uint8_t* smem, uint64_t* bars, int4* meta,
+                                           volatile int* abort_flag, int lane) {
   constexpr unsigned FULL = 0xffffffffu;
-  constexpr int BS = C::BS, D = C::D, QPL = N / 2;  // query chunks (16 bytes) per lane
+  constexpr int BS = C::BS;
   uint64_t* full = bars + C::B_FULL;
   uint64_t* empty = bars + C::B_EMPTY;
   uint64_t* qfree = bars + C::B_QFREE;
-  const int G = p.group, Hkv = p.num_kv_heads, Hq = p.num_q_heads, T = p.qtok;
+  const int G = p.group, Hkv = p.num_kv_heads, T = p.qtok;
   const unsigned total = p.counters[1] * static_cast<unsigned>(Hkv);
   const uint64_t pol = policy_evict_first();
-  const uint8_t* qsrc = static_cast<const uint8_t*>(p.q);
+  // bytes of the query rows of one item: the box is G heads x (query tokens or members) rows, both halves
+  const uint32_t qbytes = static_cast<uint32_t>(2 * G * p.qbox_rows * 128);
   uint32_t nchunks = 0, items = 0;
   bool stop = false;
   auto acquire = [&](int c) -> bool {  // wait until the chunk buffer c was released
@@ -208,13 +232,11 @@ __device__ __forceinline__ void tc_produce(const DecodeParams& p, const CUtensor
     if (lane == 0) w = atomicAdd(&p.counters[0], 1u);
     return w;
   };
-  // q / d for 0 <= q < 1024 and 1 <= d <= 64: (q * ceil(2^16 / d)) >> 16 is exact there
-  const uint32_t inv_g = (65536u + G - 1) / G;
   auto entry = [&](unsigned w) -> WorkItem {
     return w < total ? p.items[w / Hkv] : WorkItem{0, 0, 0, 0, 0, 1, 0, 0};
   };
-  // issue every load of item w (entry `it`); nothing here waits for them
-  auto issue_loads = [&](unsigned w, const WorkItem& it, TcItemLoads<QPL>& L) {
+  // issue the block-table (and sequence-length) loads of item w (entry `it`); nothing waits here
+  auto issue_loads = [&](unsigned w, const WorkItem& it, TcItemLoads& L) {
     L.valid = w < total;
     L.it = it;
     L.kvh = static_cast<int>(w % Hkv);
@@ -232,21 +254,9 @@ __device__ __forceinline__ void tc_produce(const DecodeParams& p, const CUtensor
     }
     // key positions relative to the item's first query token, at position len - T + t0
     if (T > 1) L.rel0 = it.tok0 - (p.seq_lens[it.seq] - T + it.t0);
-    const int ncol = members * it.tq * G;
-    const uint32_t inv_tq = (65536u + it.tq - 1) / it.tq;
-#pragma unroll
-    for (int k = 0; k < QPL; ++k) {
-      const int idx = lane + 32 * k;  // row idx / 16, 16-byte chunk idx % 16
-      if (idx < ncol * 16) {
-        const int r = idx >> 4, mt = static_cast<int>((r * inv_g) >> 16), g = r - mt * G;
-        const int m = static_cast<int>((mt * inv_tq) >> 16), t = it.t0 + mt - m * it.tq;
-        const int64_t qrow = (static_cast<int64_t>(it.seq + m) * T + t) * Hq + L.kvh * G + g;
-        L.qv[k] = __ldg(reinterpret_cast<const uint4*>(qsrc + (qrow * D + (idx & 15) * 8) * C::QE));
-      }
-    }
   };
 
-  TcItemLoads<QPL> cur, nxt;
+  TcItemLoads cur, nxt;
   const unsigned c0 = claim();
   const unsigned c1 = claim();
   const unsigned w0 = __shfl_sync(FULL, c0, 0);
@@ -266,7 +276,7 @@ __device__ __forceinline__ void tc_produce(const DecodeParams& p, const CUtensor
     const int part = it.pm & 0xffff, members = (it.pm >> 16) & 0xff;
     const int tok0 = it.tok0, tok1 = it.tok1;
     const int npages = (tok1 - tok0 + BS - 1) / BS;
-    const int rows = members * it.tq, ncol = rows * G;
+    const int rows = members * it.tq;
     bool bad = lane < npages && (cur.bt < 0 || cur.bt >= p.num_blocks);
     bad = __any_sync(FULL, bad);
     const bool mismatch = __any_sync(FULL, cur.mismatch);
@@ -283,19 +293,6 @@ __device__ __forceinline__ void tc_produce(const DecodeParams& p, const CUtensor
         break;
       }
     }
-    if (!bad) {
-      // query row r -> half h, row r, 16-byte chunk ch at h * N * 128 + r * 128 + ((ch ^ (r & 7)) << 4):
-      // the 128-byte-swizzled K-major B operand
-      uint8_t* qdst = smem + C::OFF_Q + qb * C::OPB;
-#pragma unroll
-      for (int k = 0; k < QPL; ++k) {
-        const int idx = lane + 32 * k, r = idx >> 4, c16 = idx & 15;
-        if (idx < ncol * 16)
-          *reinterpret_cast<uint4*>(qdst + (c16 >> 3) * (N * 128) + r * 128 + (((c16 & 7) ^ (r & 7)) << 4)) = cur.qv[k];
-      }
-      fence_proxy_async_smem();
-    }
-    __syncwarp();
     const int nch = (npages + C::CH - 1) / C::CH;
     for (int cc = 0; cc < nch; ++cc) {
       const int c = static_cast<int>(nchunks % C::NCH);
@@ -304,7 +301,6 @@ __device__ __forceinline__ void tc_produce(const DecodeParams& p, const CUtensor
         break;
       }
       const int pg0 = cc * C::CH, npg = min(C::CH, npages - pg0);
-      const int phys = __shfl_sync(FULL, cur.bt, (pg0 + lane) & 31);
       if (lane == 0) {
         const int ntok_last = min(BS, tok1 - (tok0 + (pg0 + npg - 1) * BS));
         const int flags = (cc == 0 ? F_FIRST : 0) | (cc == nch - 1 ? F_LAST : 0) | (bad ? F_BAD : 0) |
@@ -314,17 +310,24 @@ __device__ __forceinline__ void tc_produce(const DecodeParams& p, const CUtensor
         if (bad)
           mbar_arrive(&full[c]);
         else
-          mbar_arrive_expect_tx(&full[c], static_cast<uint32_t>(npg * 2 * C::VPAGE));
+          mbar_arrive_expect_tx(&full[c], static_cast<uint32_t>(npg * 2 * C::VPAGE) + (cc == 0 ? qbytes : 0u));
       }
       __syncwarp();  // the expected byte count is set before any copy can complete
-      // one box per lane: page lane / 4, K half 0 / K half 1 / V half 0 / V half 1
-      const int lp = lane >> 2, lh = lane & 1;
-      const bool lv = (lane & 2) != 0;
-      const int lphys = __shfl_sync(FULL, phys, lp);
-      if (!bad && lp < npg) {
+      if (!bad) {
+        // one box per lane: page lane / 4, K half 0 / K half 1 / V half 0 / V half 1
+        const int lp = lane >> 2, lh = lane & 1;
+        const bool lv = (lane & 2) != 0;
+        const int lphys = __shfl_sync(FULL, cur.bt, (pg0 + lp) & 31);
         uint8_t* cb = smem + c * C::CHUNK_BYTES;
-        uint8_t* dst = lv ? cb + 2 * C::KH_BYTES + lp * C::VPAGE + lh * C::BOX : cb + lh * C::KH_BYTES + lp * C::BOX;
-        tma_load_3d(dst, lv ? &tmv : &tmk, 0, kvh * 2 + lh, lphys * BS, &full[c], pol);
+        if (lp < npg) {
+          uint8_t* dst = lv ? cb + 2 * C::KH_BYTES + lp * C::VPAGE + lh * C::BOX : cb + lh * C::KH_BYTES + lp * C::BOX;
+          tma_load_3d(dst, lv ? &tmv : &tmk, 0, kvh * 2 + lh, lphys * BS, &full[c], pol);
+        }
+        // the item's query rows with its first chunk: rows (query token or member) x G heads, one
+        // box per 64-element half, landing as the K-major A operand
+        if (cc == 0 && (lane == 16 || lane == 17))
+          tma_load_4d(smem + C::OFF_Q + qb * C::QBUF + (lane - 16) * C::QHALF, &tmq, 0, lane - 16, kvh * G,
+                      it.seq * T + it.t0, &full[c]);
       }
       ++nchunks;
     }
@@ -354,13 +357,19 @@ __device__ __forceinline__ void tc_produce(const DecodeParams& p, const CUtensor
   }
 }
 
-// ---------------------------------------------------------------- MMA issue (warp 5)
-// For chunk n: S^T(n) as soon as the chunk is in and its S^T buffer is free; O^T += V^T . P^T(n)
-// once the consumers have written P^T(n).  S^T(n + 1) is issued before O(n), so that it runs
-// during chunk n's softmax.
-template <typename C, int N>
-__device__ __forceinline__ void tc_mma(uint8_t* smem, uint64_t* bars, const int4* meta, volatile int* abort_flag,
-                                       uint32_t tm, int lane) {
+// ---------------------------------------------------------------- MMA issue (warps 9 and 10)
+// Chunk meta as the MMA warps need it.
+struct TcChunk {
+  int c, npg, qb, item;
+  bool end, poisoned, first, last;
+};
+
+// Warp 9: S(n) = Q . K(n)^T as soon as chunk n is in and its S buffer is free.  It also releases the
+// query buffer once an item's last S is done, and takes part in releasing each chunk buffer (it
+// has read the chunk's meta).
+template <typename C>
+__device__ __forceinline__ void tc_mma_s(uint8_t* smem, uint64_t* bars, const int4* meta, volatile int* abort_flag,
+                                         uint32_t tm, int lane) {
   constexpr unsigned FULL = 0xffffffffu;
   constexpr int D = C::D;
   uint64_t* full = bars + C::B_FULL;
@@ -368,162 +377,170 @@ __device__ __forceinline__ void tc_mma(uint8_t* smem, uint64_t* bars, const int4
   uint64_t* qfree = bars + C::B_QFREE;
   uint64_t* s_full = bars + C::B_SFULL;
   uint64_t* s_free = bars + C::B_SFREE;
-  uint64_t* p_full = bars + C::B_PFULL;
-  uint64_t* o_done = bars + C::B_ODONE;
-  struct Chunk {
-    int c, npg, qb;
-    bool end, poisoned, first, last;
-  };
-  uint32_t ns = 0, np = 0;  // S^T and O products issued
-  bool item_bad = false;
+  uint32_t ns = 0;  // S products issued
+  bool item_bad = false, ok = true;
   int item_qb = 0;
-  bool ok = true;
-  auto prepare = [&](uint32_t k) -> Chunk {
-    Chunk ch{static_cast<int>(k % C::NCH), 0, 0, true, false, false, false};
-    const bool ready = mbar_wait_bounded(&full[ch.c], (k / C::NCH) & 1u, kWaitLimit);
+  for (uint32_t k = 0;; ++k) {
+    const int c = static_cast<int>(k % C::NCH);
+    const bool ready = mbar_wait_bounded(&full[c], (k / C::NCH) & 1u, kWaitLimit);
     if (!__all_sync(FULL, ready && !*abort_flag)) {
       ok = false;
-      return ch;
+      break;
     }
-    const int4 m0 = meta[2 * ch.c], m1 = meta[2 * ch.c + 1];
+    const int4 m0 = meta[2 * c], m1 = meta[2 * c + 1];
     const int flags = (m0.z >> 24) & 0xff;
-    if (flags & F_END) return ch;
-    ch.end = false;
-    ch.first = (flags & F_FIRST) != 0;
-    ch.last = (flags & F_LAST) != 0;
-    if (ch.first) {
+    if (flags & F_END) break;
+    if (flags & F_FIRST) {
       item_bad = (flags & F_BAD) != 0;
       item_qb = m1.z;
     }
-    ch.poisoned = item_bad;
-    ch.qb = item_qb;
-    ch.npg = (m0.z >> 8) & 0xff;
-    if (!ch.poisoned) {
+    const bool last = (flags & F_LAST) != 0;
+    if (!item_bad) {
       const uint32_t b = ns & 1u;
-      if (ns >= 2) {  // the consumers have read S^T(ns - 2) out of this buffer
+      if (ns >= 2) {  // the softmax warps have read S(ns - 2) out of this buffer
         const bool fr = mbar_wait_bounded(&s_free[b], ((ns >> 1) - 1) & 1u, kWaitLimit);
         if (!__all_sync(FULL, fr)) {
           ok = false;
-          ch.end = true;
-          return ch;
+          break;
         }
       }
       if (lane == 0) {
         tc_fence_after();
-        const uint32_t kb = smem_u32(smem + ch.c * C::CHUNK_BYTES);
-        const uint32_t qa = smem_u32(smem + C::OFF_Q + ch.qb * C::OPB);
+        const uint32_t kb = smem_u32(smem + c * C::CHUNK_BYTES);
+        const uint32_t qa = smem_u32(smem + C::OFF_Q + item_qb * C::QBUF);
 #pragma unroll
         for (int k2 = 0; k2 < D / 16; ++k2) {
-          const uint32_t a = kb + (k2 >> 2) * C::KH_BYTES + (k2 & 3) * 32;
-          const uint32_t bq = qa + (k2 >> 2) * (N * 128) + (k2 & 3) * 32;
-          umma_ss(tm + C::TM_S + b * N, smem_desc_sw128(a, 16, 1024), smem_desc_sw128(bq, 16, 1024), C::IDESC_S,
+          const uint32_t a = qa + (k2 >> 2) * C::QHALF + (k2 & 3) * 32;
+          const uint32_t bk = kb + (k2 >> 2) * C::KH_BYTES + (k2 & 3) * 32;
+          umma_ss(tm + C::TM_S + b * C::CT, smem_desc_sw128(a, 16, 1024), smem_desc_sw128(bk, 16, 1024), C::IDESC_S,
                   k2 > 0);
         }
         umma_commit(&s_full[b]);
-        if (ch.last) umma_commit(&qfree[ch.qb]);  // the query rows are read once the item's last S^T is done
+        if (last) umma_commit(&qfree[item_qb]);  // the query rows are read once the item's last S is done
       }
       __syncwarp();
       ++ns;
+    } else if (last && lane == 0) {
+      mbar_arrive(&qfree[item_qb]);
     }
-    return ch;
-  };
-
-  // chunk k is in (no waiting)
-  auto arrived = [&](uint32_t k) -> bool {
-    uint32_t done = 0;
-    if (lane == 0) done = mbar_test(&full[k % C::NCH], (k / C::NCH) & 1u) ? 1u : 0u;
-    return __shfl_sync(FULL, done, 0) != 0;
-  };
-
-  uint32_t n = 0;
-  Chunk cur = prepare(0);
-  while (ok && !cur.end) {
-    // S^T(n + 1) goes first when its chunk is already in; O(n) never waits for the next chunk
-    bool have_next = false;
-    Chunk nxt;
-    if (arrived(n + 1)) {
-      nxt = prepare(n + 1);
-      have_next = true;
-      if (!ok) break;
-    }
-    if (!cur.poisoned) {
-      const bool pf = mbar_wait_bounded(p_full, np & 1u, kWaitLimit);
-      if (!__all_sync(FULL, pf)) {
-        ok = false;
-        break;
-      }
-      if (lane == 0) {
-        tc_fence_after();
-        const uint32_t vb = smem_u32(smem + cur.c * C::CHUNK_BYTES + 2 * C::KH_BYTES);
-        const uint32_t pb = smem_u32(smem + C::OFF_P);
-        for (int j = 0; j < cur.npg; ++j) {
-          const uint64_t a = smem_desc_sw128(vb + j * C::VPAGE, C::BOX, 1024);
-          const uint64_t b = smem_desc_sw128(pb + (j >> 2) * (N * 128) + (j & 3) * 32, 16, 1024);
-          umma_ss(tm + C::TM_O, a, b, C::IDESC_O, (cur.first && j == 0) ? 0u : 1u);
-        }
-        umma_commit(o_done);
-        umma_commit(&empty[cur.c]);  // the chunk buffer is free once these products are done
-      }
-      __syncwarp();
-      ++np;
-    } else if (lane == 0) {
-      mbar_arrive(&empty[cur.c]);
-      if (cur.last) mbar_arrive(&qfree[cur.qb]);
-    }
-    if (!have_next) {
-      nxt = prepare(n + 1);
-      if (!ok) break;
-    }
-    cur = nxt;
-    ++n;
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[c]);  // this warp is done with the chunk's meta
   }
   if (!ok && lane == 0) {
     record_error(DEV_TIMEOUT);
     *abort_flag = 1;
   }
   // every product issued here completes before the tensor memory is released
-  if (lane == 0) {
-    umma_commit(bars + C::B_FIN);
+  if (lane == 0) umma_commit(bars + C::B_FIN);
+  __syncwarp();
+  mbar_wait_bounded(bars + C::B_FIN, 0u, kWaitLimit);
+}
+
+// Warp 10: O(n) += P(n) . V(n) once the softmax warps have written P(n); its completion releases the
+// P buffer and the chunk buffer.  An item's first O product overwrites its O buffer, once the item
+// before the previous one has been read out of it.
+template <typename C>
+__device__ __forceinline__ void tc_mma_o(uint8_t* smem, uint64_t* bars, const int4* meta, volatile int* abort_flag,
+                                         uint32_t tm, int lane) {
+  constexpr unsigned FULL = 0xffffffffu;
+  constexpr int D = C::D;
+  uint64_t* full = bars + C::B_FULL;
+  uint64_t* empty = bars + C::B_EMPTY;
+  uint64_t* p_full = bars + C::B_PFULL;
+  uint64_t* p_free = bars + C::B_PFREE;
+  uint64_t* o_free = bars + C::B_OFREE;
+  uint32_t np = 0;  // O products issued
+  int items = -1;
+  bool item_bad = false, ok = true;
+  for (uint32_t k = 0;; ++k) {
+    const int c = static_cast<int>(k % C::NCH);
+    const bool ready = mbar_wait_bounded(&full[c], (k / C::NCH) & 1u, kWaitLimit);
+    if (!__all_sync(FULL, ready && !*abort_flag)) {
+      ok = false;
+      break;
+    }
+    const int4 m0 = meta[2 * c];
+    const int flags = (m0.z >> 24) & 0xff;
+    if (flags & F_END) break;
+    const bool first = (flags & F_FIRST) != 0;
+    if (first) {
+      ++items;
+      item_bad = (flags & F_BAD) != 0;
+    }
+    const int npg = (m0.z >> 8) & 0xff;
+    if (item_bad) {
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[c]);
+      continue;
+    }
+    const uint32_t pb = np & 1u, ob = static_cast<uint32_t>(items) & 1u;
+    bool good = mbar_wait_bounded(&p_full[pb], (np >> 1) & 1u, kWaitLimit);
+    if (good && first && items >= 2)  // the output of item - 2 has been read out of this O buffer
+      good = mbar_wait_bounded(&o_free[ob], ((items >> 1) - 1) & 1u, kWaitLimit);
+    if (!__all_sync(FULL, good)) {
+      ok = false;
+      break;
+    }
+    if (lane == 0) {
+      tc_fence_after();
+      const uint32_t vb = smem_u32(smem + c * C::CHUNK_BYTES + 2 * C::KH_BYTES);
+      const uint32_t pa = smem_u32(smem + C::OFF_P + pb * C::PBUF);
+      for (int j = 0; j < npg; ++j) {
+        const uint64_t a = smem_desc_sw128(pa + j * 32, 16, 1024);
+        const uint64_t b = smem_desc_sw128(vb + j * C::VPAGE, C::BOX, 1024);
+        umma_ss(tm + C::TM_O + ob * D, a, b, C::IDESC_O, (first && j == 0) ? 0u : 1u);
+      }
+      umma_commit(&p_free[pb]);
+      umma_commit(&empty[c]);  // the chunk buffer is free once these products are done
+    }
+    __syncwarp();
+    ++np;
   }
+  if (!ok && lane == 0) {
+    record_error(DEV_TIMEOUT);
+    *abort_flag = 1;
+  }
+  if (lane == 0) umma_commit(bars + C::B_FIN);
   __syncwarp();
   mbar_wait_bounded(bars + C::B_FIN, 0u, kWaitLimit);
 }
 
 // ---------------------------------------------------------------- kernel
-template <typename KT, int N, bool CAUSAL>
-__global__ void __launch_bounds__(TcCfg<KT, N>::NTHREADS, 1)
+template <typename KT, bool CAUSAL>
+__global__ void __launch_bounds__(TcCfg<KT>::NTHREADS, 1)
     pa_decode_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
-                        const DecodeParams p) {
-  using C = TcCfg<KT, N>;
-  constexpr int D = C::D, NC = C::NCONS;
-  constexpr int BAR_C = 1;     // named barrier of the consumer warps
-  constexpr int BAR_EXIT = 2;  // consumers and the MMA warp, before the tensor memory is released
+                        const __grid_constant__ CUtensorMap tmq, const DecodeParams p) {
+  using C = TcCfg<KT>;
+  constexpr int D = C::D, CT = C::CT, HC = C::HC, M = C::M;
+  // named barriers: 1 + q for the two softmax warps of lane quarter q; the softmax warps and the
+  // MMA warps before the tensor memory is released
+  constexpr int BAR_EXIT = 5;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
   int4* meta = reinterpret_cast<int4*>(smem + C::OFF_META);
-  float* red = reinterpret_cast<float*>(smem + C::OFF_RED);  // [4][N] per-warp partials
-  float* msm = red + 4 * N;                                  // [N] running row maxima
-  float* asm_ = msm + N;                                     // [N] rescale factors
-  float* fscale = asm_ + N;                                  // [N] output scale of each row
-  int64_t* fofs = reinterpret_cast<int64_t*>(fscale + N);    // [N] output offset of each row
+  float* xmax = reinterpret_cast<float*>(smem + C::OFF_XCH);  // [S buffer][half][M]
+  float* xsum = xmax + 4 * M;                                  // [item parity][half][M]
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC + 4);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::NBAR; ++s) {
-      // S^T free and P^T full: one arrival per consumer warp; a chunk buffer is free once the
-      // consumer warps have read its meta and the MMA warp has finished with it (or skipped it)
-      const bool four = s == C::B_SFREE || s == C::B_SFREE + 1 || s == C::B_PFULL;
+      // S free, P full and O free: one arrival per softmax warp; a chunk buffer is free once the
+      // softmax warps and the S warp have read its meta and the O warp has finished with it (or
+      // skipped it); the final drain: one commit per MMA warp
+      const bool sm = (s >= C::B_SFREE && s < C::B_SFREE + 2) || (s >= C::B_PFULL && s < C::B_PFULL + 2) ||
+                      (s >= C::B_OFREE && s < C::B_OFREE + 2);
       const bool empty = s >= C::B_EMPTY && s < C::B_EMPTY + C::NCH;
-      mbar_init(&bars[s], four ? 4 : empty ? 5 : 1);
+      mbar_init(&bars[s], sm ? C::NSM / 32 : empty ? C::NSM / 32 + 2 : s == C::B_FIN ? 2 : 1);
     }
     *abort_flag = 0;
     fence_mbar_init();
     prefetch_tensormap(&tmk);
     prefetch_tensormap(&tmv);
+    prefetch_tensormap(&tmq);
   }
   if (warp == 0) tmem_alloc(tmem_slot, C::TM_COLS);
   tc_fence_before();
@@ -532,82 +549,81 @@ __global__ void __launch_bounds__(TcCfg<KT, N>::NTHREADS, 1)
   const uint32_t tm = *reinterpret_cast<volatile uint32_t*>(tmem_slot);
   pdl_wait();  // the plan kernel's work list and counters are visible from here on
 
-  if (warp == 4) {
-    tc_produce<C, N>(p, tmk, tmv, smem, bars, meta, abort_flag, lane);
+  if (warp == C::W_LOAD) {
+    tc_produce<C>(p, tmk, tmv, tmq, smem, bars, meta, abort_flag, lane);
     return;
   }
-  if (warp == 5) {
-    tc_mma<C, N>(smem, bars, meta, abort_flag, tm, lane);
+  if (warp == C::W_S || warp == C::W_O) {
+    if (warp == C::W_S)
+      tc_mma_s<C>(smem, bars, meta, abort_flag, tm, lane);
+    else
+      tc_mma_o<C>(smem, bars, meta, abort_flag, tm, lane);
     tc_fence_before();
-    bar_sync(BAR_EXIT, NC + 32);
+    bar_sync(BAR_EXIT, C::NSM + 64);
     return;
   }
 
-  // ============================== consumers (warps 0-3) ==============================
+  // ============================== softmax and output (warps 0-7) ==============================
   constexpr unsigned FULL = 0xffffffffu;
   constexpr float kNone = -1e30f;  // running maximum of a row with no score yet (finite: no NaN from -inf - -inf)
   uint64_t* full = bars + C::B_FULL;
+  uint64_t* empty = bars + C::B_EMPTY;
   uint64_t* s_full = bars + C::B_SFULL;
   uint64_t* s_free = bars + C::B_SFREE;
   uint64_t* p_full = bars + C::B_PFULL;
-  uint64_t* o_done = bars + C::B_ODONE;
-  const int ct = threadIdx.x;  // token of the chunk (S^T lane), element of head_dim (O^T lane)
-  const uint32_t tl = tm + (static_cast<uint32_t>(warp * 32) << 16);  // this warp's lane quarter
-  uint8_t* pbuf = smem + C::OFF_P;
-
+  uint64_t* p_free = bars + C::B_PFREE;
+  uint64_t* o_free = bars + C::B_OFREE;
+  const int ct = threadIdx.x;
+  const int quarter = warp & 3, half = warp >> 2;  // TMEM lane quarter; chunk columns 32 half .. + 31
+  const int bar_pair = 1 + quarter;
+  const int row = tc_lane_row(quarter * 32 + lane);                     // this lane's query row, or -1
+  const uint32_t tl = tm + (static_cast<uint32_t>(quarter * 32) << 16);  // the lane quarter
   const int G = p.group, Hq = p.num_q_heads, T = p.qtok, HV = T * Hq;
   const float sl = p.scale_log2;
-  uint32_t n = 0, ns = 0, o_phase = 0;
-  bool o_pending = false, ok = true;
-  float m[N], lp[N];
-  int ncol = 0, item_t0 = 0;
-  bool poisoned = false, o_fresh = true;
+  uint32_t n = 0, ns = 0, np = 0;
+  int items = -1;
+  bool ok = true;
+  float m = kNone, l = 0.f;  // the row's running maximum (log2 units); this half's running sum
+  int ncol = 0, item_t0 = 0, first_np = 0;
+  bool poisoned = false, live = false;
 
-  // completion of the last O product
-  auto wait_o = [&]() -> bool {
-    bool fin = true;
-    if (o_pending) {
-      fin = mbar_wait_bounded(o_done, o_phase, kWaitLimit);
-      o_phase ^= 1u;
-      o_pending = false;
-      tc_fence_after();
-    }
-    return fin;
+  // completion of O product k (the P buffer it read is free again)
+  auto wait_o = [&](uint32_t k) -> bool {
+    const bool done = mbar_wait_bounded(&p_free[k & 1u], (k >> 1) & 1u, kWaitLimit);
+    tc_fence_after();
+    return done;
   };
 
   while (true) {
     const int c = static_cast<int>(n % C::NCH);
     const bool ready = mbar_wait_bounded(&full[c], (n / C::NCH) & 1u, kWaitLimit);
-    if (!bar_and(ready && !*abort_flag, BAR_C, NC)) {
+    if (!__all_sync(FULL, ready && !*abort_flag)) {
       ok = false;
       break;
     }
     const int4 m0 = meta[2 * c], m1 = meta[2 * c + 1];
     const int flags = (m0.z >> 24) & 0xff;
     if (flags & F_END) break;
-    if (flags & F_FIRST) {
+    const bool first = (flags & F_FIRST) != 0, last = (flags & F_LAST) != 0;
+    if (first) {
+      ++items;
       poisoned = (flags & F_BAD) != 0;
       ncol = ((m0.z >> 16) & 0xff) * G;
       item_t0 = m1.x;
-      o_fresh = true;
-#pragma unroll
-      for (int r = 0; r < N; ++r) {
-        m[r] = kNone;
-        lp[r] = 0.f;
-      }
-      if (ct < N) msm[ct] = kNone;  // read only after the next barrier
+      live = row >= 0 && row < ncol;
+      m = kNone;
+      l = 0.f;
+      first_np = static_cast<int>(np);
     }
     const int npg = (m0.z >> 8) & 0xff, ntok_last = m1.y;
-    const bool last = (flags & F_LAST) != 0;
     uint8_t* cb = smem + c * C::CHUNK_BYTES;
+    const uint32_t ob = static_cast<uint32_t>(items) & 1u;
 
     if (!poisoned) {
-      const int pg = ct >> 4, ti = ct & 15;
-      const bool valid = pg < npg && (pg < npg - 1 || ti < ntok_last);
-      if (pg == npg - 1 && ti >= ntok_last) {
-        // V rows past the end of the item may hold anything (even NaN) and would meet zero
-        // weights in the MMA: zero this token's row
-        uint8_t* vrow = cb + 2 * C::KH_BYTES + pg * C::VPAGE + ti * 128;
+      if (ct < CT && ct / C::BS == npg - 1 && (ct & (C::BS - 1)) >= ntok_last) {
+        // V rows past the end of the item may hold anything (even NaN) and would meet zero weights
+        // in the MMA: zero this token's row
+        uint8_t* vrow = cb + 2 * C::KH_BYTES + (npg - 1) * C::VPAGE + (ct & (C::BS - 1)) * 128;
 #pragma unroll
         for (int h = 0; h < 2; ++h)
 #pragma unroll
@@ -617,192 +633,181 @@ __global__ void __launch_bounds__(TcCfg<KT, N>::NTHREADS, 1)
       const uint32_t b = ns & 1u;
       bool good = mbar_wait_bounded(&s_full[b], (ns >> 1) & 1u, kWaitLimit);
       tc_fence_after();
-      uint32_t sr[N];
-      tmem_ldn<N>(tl + C::TM_S + b * N, sr);
+      uint32_t sr[HC];
+      tmem_ldn<HC>(tl + C::TM_S + b * CT + half * HC, sr);
       tc_wait_ld();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&s_free[b]);
       ++ns;
 
-      // scores in log2 units, -inf where masked: rows r < ncol; with several query tokens, row r
-      // (query token r / G) sees keys at relative positions <= r / G, i.e. r >= rel * G
-      const int lo = CAUSAL && T > 1 ? (m0.w + ct) * G : 0;
-      float x[N];
-      bool big = false;
+      // scores in log2 units, -inf where masked: tokens past the item's end; with several query
+      // tokens, row r (query token r / G of the item) sees keys at relative positions <= r / G.
+      // This lane holds chunk columns j0 .. j0 + HC - 1 of its row.
+      const int ntok = (npg - 1) * C::BS + ntok_last;
+      const int jend = live ? (CAUSAL && T > 1 ? min(ntok, row / G - m0.w + 1) : ntok) : 0;
+      const int jn = jend - half * HC;  // valid columns of this half: j < jn
+      // the maximum of this half's valid scores, as a tree (no long dependent chain)
+      float xv[HC];
 #pragma unroll
-      for (int r = 0; r < N; ++r) {
-        const bool keep = valid && r < ncol && r >= lo;
-        x[r] = keep ? __uint_as_float(sr[r]) * sl : -CUDART_INF_F;
-        big |= x[r] > m[r] + kRescaleThreshold;
-      }
-      // the previous O product is done: O may be rescaled and P^T overwritten
-      good = wait_o() && good;
-      if (bar_or(big || !good, BAR_C, NC)) {
-        if (!bar_and(good, BAR_C, NC)) {
-          ok = false;
-          break;
-        }
-        big = bar_or(big, BAR_C, NC);
-      }
-      if (big) {  // uniform here
-        // raise the maximum of every row whose chunk maximum exceeds it by more than the
-        // threshold: a butterfly leaves row lane % N's warp maximum in each lane, thread r < N
-        // decides row r
-        float v[N];
+      for (int j = 0; j < HC; ++j) xv[j] = j < jn ? __uint_as_float(sr[j]) : -CUDART_INF_F;
 #pragma unroll
-        for (int r = 0; r < N; ++r) v[r] = x[r];
-        if (N == 16) {
+      for (int w = HC / 2; w >= 1; w >>= 1)
 #pragma unroll
-          for (int r = 0; r < N; ++r) v[r] = fmaxf(v[r], __shfl_xor_sync(FULL, v[r], 16));
-        }
+        for (int j = 0; j < w; ++j) xv[j] = fmaxf(xv[j], xv[j + w]);
+      float mx = xv[0];
+      // the row's chunk maximum: both halves' (exchanged through shared memory, one buffer per S
+      // buffer: it is rewritten two products later, once both warps have passed the barrier of the
+      // product in between -- S products are counted alike in both warps, poisoned chunks have none)
+      float* xm = xmax + b * 2 * M;
+      if (row >= 0) xm[half * M + row] = mx;
+      bar_sync(bar_pair, 64);
+      if (row >= 0) mx = fmaxf(mx, xm[(half ^ 1) * M + row]);
+      mx *= sl;  // scale > 0 commutes with max
+      const bool raise = mx > m + kRescaleThreshold;
+      const float mnew = raise ? mx : m;
+      const float alpha = raise ? fast_exp2(m - mnew) : 1.f;  // 0 for a row without scores so far
+      // an O row that already holds this item's products is rescaled in tensor memory (by the first
+      // half's warp); the products issued so far must be done (the tcgen05.ld / st are warp-wide, so
+      // the warp votes)
+      if (half == 0 && __any_sync(FULL, raise) && static_cast<int>(np) > first_np) {
+        good = wait_o(np - 1) && good;
+        uint32_t ov[64];
 #pragma unroll
-        for (int s2 = N / 2; s2 >= 1; s2 >>= 1) {
-          const bool upper = (lane & s2) != 0;
-#pragma unroll
-          for (int i = 0; i < s2; ++i) {
-            const float send = upper ? v[i] : v[i + s2];
-            const float keep = upper ? v[i + s2] : v[i];
-            v[i] = fmaxf(keep, __shfl_xor_sync(FULL, send, s2));
-          }
-        }
-        if (lane < N) red[warp * N + lane] = v[0];
-        bar_sync(BAR_C, NC);
-        if (ct < N) {
-          const float mo = msm[ct];
-          const float cm = fmaxf(fmaxf(red[ct], red[N + ct]), fmaxf(red[2 * N + ct], red[3 * N + ct]));
-          float a = 1.f;
-          if (cm > mo + kRescaleThreshold) {
-            a = fast_exp2(mo - cm);  // 0 for a row without scores so far
-            msm[ct] = cm;
-          }
-          asm_[ct] = a;
-        }
-        bar_sync(BAR_C, NC);
-        bool rescale = false;
-        float alpha[N];
-#pragma unroll
-        for (int r = 0; r < N; ++r) {
-          alpha[r] = asm_[r];
-          m[r] = msm[r];
-          lp[r] *= alpha[r];
-          rescale |= alpha[r] != 1.f;
-        }
-        // (rescale is the same in every thread; O is idle: the previous product is done and this
-        // chunk's is not issued before the consumers signal P^T)
-        if (rescale && !o_fresh) {
-          uint32_t ov[N];
-          tmem_ldn<N>(tl + C::TM_O, ov);
+        for (int h = 0; h < D / 64; ++h) {
+          tmem_ldn<64>(tl + C::TM_O + ob * D + h * 64, ov);
           tc_wait_ld();
 #pragma unroll
-          for (int r = 0; r < N; ++r) ov[r] = __float_as_uint(__uint_as_float(ov[r]) * alpha[r]);
-          tmem_stn<N>(tl + C::TM_O, ov);
-          tc_wait_st();
+          for (int i = 0; i < 64; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
+          tmem_stn<64>(tl + C::TM_O + ob * D + h * 64, ov);
         }
+        tc_wait_st();
       }
-      // P^T (K-major: row r = query row, 128 tokens in two 64-token halves, 128-byte swizzle)
-      const uint32_t prow = smem_u32(pbuf) + (ct >> 6) * (N * 128) + (ct & 7) * 2;
-      const int pch = (ct & 63) >> 3;
+      m = mnew;
+      l *= alpha;
+      // this half of the P row: the weights the MMA sees, their sum taken over the same rounded values
+      uint32_t pk[HC / 2];
+      float ls[HC / 2];
 #pragma unroll
-      for (int r = 0; r < N; r += 2) {
-        const uint32_t pk = pack2<KT>(fast_exp2(x[r] - m[r]), fast_exp2(x[r + 1] - m[r + 1]));
-        const float2 w2 = unpack2<KT>(pk);  // the weights the MMA sees
-        lp[r] += w2.x;
-        lp[r + 1] += w2.y;
-        sts_u16(prow + r * 128 + ((pch ^ (r & 7)) << 4), static_cast<uint16_t>(pk & 0xffffu));
-        sts_u16(prow + (r + 1) * 128 + ((pch ^ ((r + 1) & 7)) << 4), static_cast<uint16_t>(pk >> 16));
+      for (int j = 0; j < HC; j += 2) {
+        const float e0 = j < jn ? fast_exp2(fmaf(__uint_as_float(sr[j]), sl, -m)) : 0.f;
+        const float e1 = j + 1 < jn ? fast_exp2(fmaf(__uint_as_float(sr[j + 1]), sl, -m)) : 0.f;
+        pk[j / 2] = pack2<KT>(e0, e1);
+        const float2 w2 = unpack2<KT>(pk[j / 2]);
+        ls[j / 2] = w2.x + w2.y;
+      }
+#pragma unroll
+      for (int w = HC / 4; w >= 1; w >>= 1)  // their sum, as a tree
+#pragma unroll
+        for (int j = 0; j < w; ++j) ls[j] += ls[j + w];
+      l += ls[0];
+      // the P buffer is free once O(np - 2) is done
+      if (np >= 2) good = wait_o(np - 2) && good;
+      if (!__all_sync(FULL, good)) {
+        ok = false;
+        break;
+      }
+      if (row >= 0) {  // K-major A operand: row `row`, 16-byte chunk q at ((q ^ (row & 7)) << 4)
+        uint8_t* prow = smem + C::OFF_P + (np & 1u) * C::PBUF + row * 128;
+#pragma unroll
+        for (int q = 0; q < HC / 8; ++q) {
+          const int qc = half * (HC / 8) + q;
+          *reinterpret_cast<uint4*>(prow + ((qc ^ (row & 7)) << 4)) =
+              make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+        }
       }
       fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(p_full);
-        mbar_arrive(&bars[C::B_EMPTY + c]);
-      }
-      o_pending = true;
-      o_fresh = false;
-    } else {
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars[C::B_EMPTY + c]);
+      if (lane == 0) mbar_arrive(&p_full[np & 1u]);
+      ++np;
     }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[c]);  // this warp is done with the chunk's meta and V rows
 
     if (last) {
-      // output of the item: reduce the row sums over the 128 threads
-      const bool good = wait_o();
-      if (!bar_and(good, BAR_C, NC)) {
+      // output of the item: each half-row's lane writes half of the row's head_dim columns
+      const bool o_any = static_cast<int>(np) > first_np;
+      bool good = true;
+      if (!poisoned && o_any) good = wait_o(np - 1);
+      if (!__all_sync(FULL, good)) {
         ok = false;
         break;
       }
-      const bool bad = poisoned || o_fresh;  // uniform
-      float v[N];
-#pragma unroll
-      for (int r = 0; r < N; ++r) v[r] = lp[r];
-      if (N == 16) {
-#pragma unroll
-        for (int r = 0; r < N; ++r) v[r] += __shfl_xor_sync(FULL, v[r], 16);
-      }
-#pragma unroll
-      for (int s2 = N / 2; s2 >= 1; s2 >>= 1) {
-        const bool upper = (lane & s2) != 0;
-#pragma unroll
-        for (int i = 0; i < s2; ++i) {
-          const float send = upper ? v[i] : v[i + s2];
-          const float keep = upper ? v[i + s2] : v[i];
-          v[i] = keep + __shfl_xor_sync(FULL, send, s2);
-        }
-      }
-      if (lane < N) red[warp * N + lane] = v[0];
-      bar_sync(BAR_C, NC);
+      const bool bad = poisoned || !o_any;
+      // the row's sum: both halves' (one buffer per item parity: every item, poisoned or not, ends
+      // with this barrier, so a buffer is rewritten only after both warps have read it)
+      float* xs = xsum + (items & 1) * 2 * M;
+      if (row >= 0) xs[half * M + row] = l;
+      bar_sync(bar_pair, 64);
+      const float lt = row >= 0 ? l + xs[(half ^ 1) * M + row] : 0.f;
       const int seq = m0.x, part = m0.y & 0xffff, kvh = m0.z & 0xff;
       const bool direct = (flags & F_DIRECT) != 0;
-      if (ct < ncol) {  // row ct: where it goes and how it is scaled
-        const float l = red[ct] + red[N + ct] + red[2 * N + ct] + red[3 * N + ct];
-        const int g = ct % G, mq = ct / G;
+      int64_t ofs = 0;
+      float fs = 0.f;
+      if (live) {
+        const int g = row % G, mq = row / G;
         const int mb = T > 1 ? 0 : mq, t = T > 1 ? item_t0 + mq : 0;
         const int vh = t * Hq + kvh * G + g;
         if (direct) {
-          fofs[ct] = (static_cast<int64_t>(seq + mb) * HV + vh) * D;
-          fscale[ct] = bad ? CUDART_NAN_F : p.v_scale / l;
+          ofs = (static_cast<int64_t>(seq + mb) * HV + vh) * D;
+          fs = bad ? CUDART_NAN_F : p.v_scale / lt;
         } else {
           const int64_t pidx = static_cast<int64_t>(seq + mb) * p.max_parts + part;
-          fofs[ct] = (pidx * HV + vh) * D;
-          fscale[ct] = bad ? CUDART_NAN_F : p.v_scale;
-          __stcg(&p.part_ml[pidx * HV + vh], bad ? make_float2(0.f, CUDART_NAN_F) : make_float2(msm[ct], l));
+          ofs = (pidx * HV + vh) * D;
+          fs = bad ? CUDART_NAN_F : p.v_scale;
+          if (half == 0)
+            __stcg(&p.part_ml[pidx * HV + vh], bad ? make_float2(0.f, CUDART_NAN_F) : make_float2(m, lt));
         }
       }
-      bar_sync(BAR_C, NC);
-      uint32_t ov[N];
+      const int h = half;  // this warp's 64 of the head_dim columns
+      uint32_t ov[64];
       if (!bad) {
-        tmem_ldn<N>(tl + C::TM_O, ov);
+        tmem_ldn<64>(tl + C::TM_O + ob * D + h * 64, ov);
         tc_wait_ld();
       } else {
 #pragma unroll
-        for (int r = 0; r < N; ++r) ov[r] = 0u;
+        for (int i = 0; i < 64; ++i) ov[i] = 0u;
       }
-      auto emit = [&](auto store) {
+      if (live) {
+        if (!direct) {
+          float4* dst = reinterpret_cast<float4*>(p.part_acc + ofs + h * 64);
 #pragma unroll
-        for (int r = 0; r < N; ++r)
-          if (r < ncol) store(fofs[r] + ct, __uint_as_float(ov[r]) * fscale[r]);
-      };
-      if (!direct)
-        emit([&](int64_t i, float val) { __stcg(p.part_acc + i, val); });
-      else if (p.out_dtype == DT_BF16)
-        emit([&](int64_t i, float val) { static_cast<__nv_bfloat16*>(p.out)[i] = __float2bfloat16_rn(val); });
-      else if (p.out_dtype == DT_F16)
-        emit([&](int64_t i, float val) { static_cast<__half*>(p.out)[i] = __float2half_rn(val); });
-      else
-        emit([&](int64_t i, float val) { static_cast<float*>(p.out)[i] = val; });
+          for (int i = 0; i < 16; ++i)
+            __stcg(dst + i, make_float4(__uint_as_float(ov[4 * i]) * fs, __uint_as_float(ov[4 * i + 1]) * fs,
+                                        __uint_as_float(ov[4 * i + 2]) * fs, __uint_as_float(ov[4 * i + 3]) * fs));
+        } else if (p.out_dtype == DT_F32) {
+          float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + ofs + h * 64);
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            dst[i] = make_float4(__uint_as_float(ov[4 * i]) * fs, __uint_as_float(ov[4 * i + 1]) * fs,
+                                 __uint_as_float(ov[4 * i + 2]) * fs, __uint_as_float(ov[4 * i + 3]) * fs);
+        } else {
+          uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) + ofs + h * 64);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            uint32_t w[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const float a = __uint_as_float(ov[8 * i + 2 * k]) * fs, b2 = __uint_as_float(ov[8 * i + 2 * k + 1]) * fs;
+              w[k] = p.out_dtype == DT_BF16 ? pack2<__nv_bfloat16>(a, b2) : pack2<__half>(a, b2);
+            }
+            dst[i] = make_uint4(w[0], w[1], w[2], w[3]);
+          }
+        }
+      }
       tc_fence_before();
-      bar_sync(BAR_C, NC);  // red[], fofs[] and the O columns are reused by the next item
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&o_free[ob]);  // the next item but one may overwrite this O buffer
     }
     ++n;
   }
-  if (!ok && ct == 0) {
+  if (!ok && lane == 0) {
     record_error(DEV_TIMEOUT);
     *abort_flag = 1;
   }
   tc_fence_before();
-  bar_sync(BAR_EXIT, NC + 32);  // the MMA warp has drained the tensor pipe
+  bar_sync(BAR_EXIT, C::NSM + 64);  // the MMA warps have drained the tensor pipe
   if (warp == 0) {
     tc_fence_after();
     tmem_dealloc(tm, C::TM_COLS);

@@ -192,6 +192,17 @@ def test_workspace_reserves_every_work_item(lib):
     includes the shapes whose column groups hold only 5 to 8 query rows (head_dim 64, few KV
     heads), the worst case for the reservation."""
     checked = 0
+    for wide in ("mma", "tcgen05"):  # the tensor-core kernel's items hold up to 64 rows
+        B.set_wide_kernel(wide)
+        try:
+            checked += _reservation_grid(lib)
+        finally:
+            B.set_wide_kernel("mma")
+    assert checked == 2 * 6192
+
+
+def _reservation_grid(lib):
+    checked = 0
     for D in (64, 128):
         for Hkv in (1, 2, 3):
             for G in range(1, 9):
@@ -202,4 +213,4 @@ def test_workspace_reserves_every_work_item(lib):
                                         ws=0x100000, wsb=need)
                         assert rc == B.PA_ERR_CUDA, (D, Hkv, G, T, N, MB, rc)
                         checked += 1
-    assert checked == 6192
+    return checked

@@ -254,3 +254,44 @@ def test_copy_blocks_host_validation():
     with pytest.raises(B.PAError):
         bad = np.asarray([[1, 2], [2, 3]], np.int32)          # a destination that is also a source
         B.pa_copy_blocks(dw.k_cache, dw.v_cache, torch.from_numpy(bad).cuda(), host_pairs=bad)
+
+
+def test_thousands_of_short_and_empty_sequences():
+    """4096 sequences of 0 to 40 tokens (8B shapes): the plan spreads its work over the whole
+    CTA, the merge kernel writes the rows of empty sequences, and every row matches the oracle."""
+    rng = np.random.default_rng(4096)
+    lens = [int(x) for x in rng.integers(0, 41, size=4096)]
+    w = W.independent("short", lens, num_q_heads=32, num_kv_heads=8, head_dim=128, block_size=16, q_dtype="bf16",
+                      kv_dtype="bf16", seed=4096)
+    dw, out = gpu_step(w, "f32")
+    kc, vc = oracle_post_step(w)
+    _, ref = oracle_decode(w, kc, vc)
+    assert_close(out_f32(out), ref, "bf16", "f32", "4096 short sequences")
+    empty = np.asarray(lens) == 0
+    assert empty.sum() > 50 and np.all(out_f32(out)[empty] == 0.0)
+
+
+def test_invalid_lengths_in_a_large_batch_give_nan_rows():
+    """Invalid lengths scattered over 3000 sequences: exactly those rows are NaN (written by the
+    merge kernel), the error is reported, and every other row matches the oracle."""
+    rng = np.random.default_rng(3000)
+    lens = [int(x) for x in rng.integers(0, 70, size=3000)]
+    w = W.independent("inv", lens, num_q_heads=8, num_kv_heads=2, head_dim=64, block_size=16, q_dtype="f16",
+                      kv_dtype="f16", seed=3000)
+    dw = B.device_workload(w)
+    B.pa_reshape_and_cache(dw.new_k, dw.new_v, dw.k_cache, dw.v_cache, dw.slot_mapping)
+    bad = rng.choice(3000, 40, replace=False)
+    sl = dw.seq_lens.clone()
+    sl[torch.from_numpy(bad).cuda()] = -1 - torch.arange(40, dtype=torch.int32, device="cuda")
+    out = torch.zeros((3000, 8, 64), device="cuda")
+    ws = B.DecodeWorkspace.for_workload(dw)
+    B.pa_decode(out, dw.q, dw.k_cache, dw.v_cache, dw.block_tables, sl, w.scale, ws.tensor)
+    assert B.pa_get_device_error() == B.PA_DEV_BAD_SEQ_LEN
+    got = out_f32(out)
+    mask = np.zeros(3000, bool)
+    mask[bad] = True
+    assert np.isnan(got[mask]).all() and not np.isnan(got[~mask]).any()
+    kc, vc = oracle_post_step(w)
+    good = np.flatnonzero(~mask)
+    _, ref = oracle_decode(w, kc, vc, good)
+    assert_close(got[good], ref, "f16", "f32", "valid rows beside invalid ones")

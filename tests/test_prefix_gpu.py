@@ -160,3 +160,22 @@ def test_members_with_different_tables_get_nan():
     assert np.isnan(got[0]).all() and np.isnan(got[1]).all()
     _, ref = oracle_decode(w, kc, vc, [2, 3])
     assert_close(got[2:], ref, "bf16", "f32", "sequences outside the bad group")
+
+
+def test_large_group_beside_many_small_groups():
+    """One system prompt shared by 600 requests, beside 150 forks of 2 to 4 samples: the plan
+    validates every group in parallel over its members; all groups are valid, so none may be
+    dropped (no PA_DEV_BAD_PREFIX), and every row matches the oracle."""
+    rng = np.random.default_rng(5500)
+    groups = [W.Group(1500, [1] * 600)]
+    groups += [W.Group(int(rng.integers(16, 600)), [int(x) for x in rng.integers(1, 30, size=int(rng.integers(2, 5)))])
+               for _ in range(150)]
+    w = W.build_groups("big", groups, num_q_heads=32, num_kv_heads=8, head_dim=128, block_size=16, q_dtype="bf16",
+                       kv_dtype="bf16", seed=5500)
+    pg = BM.find_prefix_groups(w.block_tables, w.seq_lens, 16)
+    assert pg[0].tolist() == [0, 600, 1488] and len(pg) > 100
+    dw, kc, vc = stepped(w)
+    out = prefix_decode(w, dw, pg, 8)
+    assert B.pa_get_device_error() == B.PA_DEV_OK
+    _, ref = oracle_decode(w, kc, vc)
+    assert_close(out.float().cpu().numpy(), ref, "bf16", "f32", "large group")

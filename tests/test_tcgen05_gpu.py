@@ -2,10 +2,11 @@
 
 Items of more than 8 query rows per KV head (several query tokens, or the members of a shared
 prefix) on a 16-bit cache with head_dim 128 and block size 16 run on this kernel once
-pa_set_option(PA_OPT_WIDE_KERNEL, PA_WIDE_TCGEN05) is called.  The cases mirror the warp-MMA
-kernel's: 9..32 query rows (N = 16 and N = 32 instantiations), column groups, short partitions
-(one chunk of 8 pages) and long ones (several chunks, a ragged last chunk and page), empty
-sequences, causal tails, shared prefixes, a bad block id and members whose tables differ.
+pa_set_option(PA_OPT_WIDE_KERNEL, PA_WIDE_TCGEN05) is called.  An item holds up to 64 query rows
+(the M of its products); wider sequences are split into column groups.  The cases mirror the
+warp-MMA kernel's: 12..64 query rows, column groups, short partitions (two chunks of 4 pages) and
+long ones (several chunks, a ragged last chunk and page), empty sequences, causal tails, shared
+prefixes of up to 64 rows, a bad block id and members whose tables differ.
 Tolerances are the attention ones (2e-3 with fp16 KV, 1e-2 with bf16 KV, plus half an ulp of a
 16-bit output).
 """
@@ -34,14 +35,16 @@ def _tcgen05_kernel():
 
 MULTI = [
     # Hq, Hkv, T, D, bs, q_dtype, out_dtype, partition   (query rows per item = T * Hq / Hkv)
-    (32, 8, 3, 128, 16, "bf16", "bf16", 0),    # 12 rows: N = 16
+    (32, 8, 3, 128, 16, "bf16", "bf16", 0),    # 12 rows
     (16, 4, 4, 128, 16, "f16", "f16", 0),      # 16 rows, fp16
-    (32, 8, 5, 128, 16, "bf16", "f32", 0),     # 20 rows: N = 32
+    (32, 8, 5, 128, 16, "bf16", "f32", 0),     # 20 rows
     (64, 8, 4, 128, 16, "bf16", "bf16", 0),    # 32 rows (G = 8)
-    (32, 8, 8, 128, 16, "bf16", "f32", 128),   # 32 rows, one chunk per partition
-    (32, 8, 16, 128, 16, "bf16", "f32", 0),    # 64 rows: 2 column groups of 8 tokens
-    (64, 8, 9, 128, 16, "bf16", "bf16", 0),    # G = 8: column groups of 4, 4 and 1 tokens
-    (8, 8, 40, 128, 16, "f16", "f32", 256),    # MHA: column groups of 32 and 8 tokens, 2 chunks per partition
+    (32, 8, 8, 128, 16, "bf16", "f32", 128),   # 32 rows, two chunks per partition
+    (32, 8, 16, 128, 16, "bf16", "f32", 0),    # 64 rows: one item per partition
+    (64, 8, 9, 128, 16, "bf16", "bf16", 0),    # G = 8, 72 rows: column groups of 8 and 1 tokens
+    (8, 8, 40, 128, 16, "f16", "f32", 256),    # MHA, 40 rows, four chunks per partition
+    (8, 8, 100, 128, 16, "bf16", "f32", 0),    # MHA, 100 rows: column groups of 64 and 36 tokens
+    (32, 8, 20, 128, 16, "f16", "bf16", 64),   # 80 rows: groups of 16 and 4 tokens, one-chunk partitions
 ]
 
 
@@ -130,3 +133,16 @@ def test_prefix_70b_batch():
 
 def test_prefix_members_with_different_tables_get_nan():
     TP.test_members_with_different_tables_get_nan()
+
+
+def test_prefix_64_rows():
+    """A shared pass of 8 members x G = 8 = 64 query rows (the tensor-core kernel's widest item)."""
+    groups = [W.Group(1100, [1, 3, 9, 27, 2, 5, 40, 1]), W.Group(600, [1] * 11), W.Group(70, [4])]
+    w = W.build_groups("p64", groups, num_q_heads=64, num_kv_heads=8, head_dim=128, block_size=16, q_dtype="bf16",
+                       kv_dtype="bf16", seed=5600)
+    pg = BM.find_prefix_groups(w.block_tables, w.seq_lens, 16)
+    dw, kc, vc = TP.stepped(w)
+    out = TP.prefix_decode(w, dw, pg, 8)
+    assert B.pa_get_device_error() == B.PA_DEV_OK
+    _, ref = TP.oracle_decode(w, kc, vc)
+    TP.assert_close(out.float().cpu().numpy(), ref, "bf16", "f32", "64-row shared passes")
