@@ -56,10 +56,14 @@ def parse_args():
     ap.add_argument("--step", choices=list(W.STEPS_70B), default=None,
                     help="70b only: 'decode' (default: one new token per sequence) or 'fork' (every sample's "
                          "whole suffix stored in the step, with all 192 copy-on-write pairs)")
-    ap.add_argument("--config", default="8b", choices=list(W.CONFIG_NAMES))
+    ap.add_argument("--config", default=None, choices=list(W.CONFIG_NAMES),
+                    help="workload (default: 8b; 70b with --op cache)")
     ap.add_argument("--block-size", type=int, default=None)
     ap.add_argument("--num-seqs", type=int, default=None,
                     help="smaller batch of the same config (profiling; 70b: that many shared-prefix samples)")
+    ap.add_argument("--uniform-lens", default=None, metavar="LO,HI",
+                    help="8b only: lengths uniform in [LO, HI] instead of the lognormal mix (with --num-seqs: "
+                         "e.g. 4096 sequences of 0 to 40 tokens)")
     ap.add_argument("--partition-size", type=int, default=0)
     ap.add_argument("--out-dtype", default=None, help="f32 | f16 | bf16 (default: the query dtype)")
     ap.add_argument("--kv-dtype", default=None, choices=["e4m3"],
@@ -74,9 +78,14 @@ def parse_args():
                     help="kernel for items of more than 8 query rows per KV head (--qtok, --prefix): the warp-MMA "
                          "kernel (default) or the 5th-generation tensor-core kernel")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-paths", action="store_true",
+                    help="skip the compact measurement of the other decode paths (default run at N=1 only)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target oracle time for cpu_baseline")
     ap.add_argument("--ref-seconds", type=float, default=150.0, help="target total time of --impl reference")
-    return ap.parse_args()
+    args = ap.parse_args()
+    if args.config is None:
+        args.config = "70b" if args.op == "cache" else "8b"
+    return args
 
 
 def make_workload(args, seed=None, num_seqs=None):
@@ -91,6 +100,11 @@ def make_workload(args, seed=None, num_seqs=None):
         if args.config != "70b":
             raise SystemExit("--step applies to the 70b config")
         extra["step"] = args.step
+    if getattr(args, "uniform_lens", None):
+        if args.config != "8b":
+            raise SystemExit("--uniform-lens applies to the 8b config")
+        lo, hi = (int(x) for x in args.uniform_lens.split(","))
+        extra["uniform_lens"] = (lo, hi)
     return W.make_config(args.config, block_size=args.block_size, seed=seed, kv_dtype=args.kv_dtype, **extra)
 
 
@@ -323,6 +337,72 @@ def run_reference(args):
     return 0
 
 
+# The other decode paths, measured after the headline step in the same run (N = 1): config, flags
+PATHS = [
+    ("8b_e4m3", dict(config="8b", kv_dtype="e4m3")),
+    ("8b_e4m3_bs32", dict(config="8b", kv_dtype="e4m3", block_size=32)),
+    ("8b_T5", dict(config="8b", qtok=5)),
+    ("8b_T8", dict(config="8b", qtok=8)),
+    ("8b_T16", dict(config="8b", qtok=16)),
+    ("8b_T5_bs32", dict(config="8b", qtok=5, block_size=32)),
+    ("70b_prefix", dict(config="70b", prefix=True)),
+    ("70b", dict(config="70b")),
+    ("7b", dict(config="7b")),
+    ("13b", dict(config="13b")),
+    ("13b_bs32", dict(config="13b", block_size=32)),
+]
+
+
+def measure_path(args, overrides: dict, calls: int = 200, warm: int = 10) -> dict:
+    """One decode path (after its step's cache writes): the mean CUDA-event time of `calls`
+    back-to-back decode calls (inputs larger than L2), as GB/s of algorithmic bytes (distinct
+    K+V, q, out, tables) and as a fraction of the measured HBM peak."""
+    from paged_kv_cache_327_b200 import binding as B
+    from paged_kv_cache_327_b200 import block_manager as BM
+
+    a = argparse.Namespace(**{**vars(args), "block_size": None, "kv_dtype": None, "qtok": 1, "prefix": False,
+                              "step": None, "uniform_lens": None, **overrides})
+    w = make_workload(a)
+    dw = B.device_workload(w)
+    ws = B.DecodeWorkspace.for_workload(dw)
+    out = torch.empty(tuple(dw.q.shape), dtype=B._NAME_TORCH[w.q_dtype], device="cuda")
+    B.run_step(dw, out, ws)
+    if a.prefix:
+        groups = torch.from_numpy(BM.find_prefix_groups(w.block_tables, w.seq_lens, w.block_size)).cuda()
+        mm = B.max_prefix_members(w.num_q_heads, w.num_kv_heads)
+        f = lambda: B.pa_decode_prefix(out, dw.q, dw.k_cache, dw.v_cache, dw.block_tables, dw.seq_lens, w.scale,
+                                       ws.tensor, groups, mm)
+    elif w.num_q_tokens > 1:
+        f = lambda: B.pa_decode_multi(out, dw.q, dw.k_cache, dw.v_cache, dw.block_tables, dw.seq_lens, w.scale,
+                                      ws.tensor)
+    elif w.kv_dtype == "e4m3":
+        f = lambda: B.pa_decode_fp8(out, dw.q, dw.k_cache, dw.v_cache, dw.block_tables, dw.seq_lens, w.scale,
+                                    w.k_scale, w.v_scale, ws.tensor)
+    else:
+        f = lambda: B.pa_decode(out, dw.q, dw.k_cache, dw.v_cache, dw.block_tables, dw.seq_lens, w.scale, ws.tensor)
+    for _ in range(warm):
+        f()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(calls):
+        f()
+    e1.record()
+    torch.cuda.synchronize()
+    if B.pa_get_device_error() != B.PA_DEV_OK:
+        raise RuntimeError(f"device error on path {overrides}")
+    ms = e0.elapsed_time(e1) / calls
+    io = w.io_bytes()
+    nbytes = w.kv_bytes_unique() + io["q"] + io["block_tables"] + io["seq_lens"] + out.numel() * out.element_size()
+    peak, _ = measured_peak()
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    res = {"ms": round(ms, 5), "achieved_gbs": round(gbs, 1), "frac": round(gbs / peak, 4),
+           "algorithmic_bytes": int(nbytes), "seq_tokens_per_s": round(w.total_tokens() / (ms * 1e-3), 1)}
+    del dw, ws, out
+    torch.cuda.empty_cache()
+    return res
+
+
 def run_ours(args):
     from paged_kv_cache_327_b200 import binding as B
     from paged_kv_cache_327_b200 import build as pkg_build
@@ -363,7 +443,7 @@ def run_ours(args):
     kv_bytes = w.kv_bytes_logical()
     # with shared prefix blocks a physical byte is read once per sharer but fetched from HBM
     # about once (L2 hits): the roofline counts distinct physical bytes
-    kv_unique = w.kv_bytes_unique() if len(w.copy_pairs) else kv_bytes
+    kv_unique = w.kv_bytes_unique()
     io = w.io_bytes()
     out_bytes = out.numel() * out.element_size()
     decode_bytes = kv_unique + io["q"] + io["block_tables"] + io["seq_lens"] + out_bytes
@@ -536,6 +616,21 @@ def run_ours(args):
     if rank != 0:
         return 0
 
+    paths = None
+    if world == 1 and not args.no_paths and args.config == "8b" and args.qtok == 1 and not args.kv_dtype \
+            and not args.num_seqs and not args.block_size and not getattr(args, "uniform_lens", None):
+        # the default run also measures every other decode path on the same GPU, clocks and peak
+        del dw, ws
+        torch.cuda.empty_cache()
+        paths = {}
+        for name, ov in PATHS:
+            try:
+                paths[name] = measure_path(args, ov)
+            except torch.cuda.OutOfMemoryError as e:
+                paths[name] = {"skipped": f"out of memory: {e}"[:120]}
+        paths["_method"] = ("mean CUDA-event time of 200 back-to-back decode calls after 10 warm-up calls "
+                            "(inputs larger than L2); frac of the same peak as roofline")
+
     ms_step = elapsed_ms / args.steps
     value = job_throughput(kv_bytes, world, ms_step * 1e-3)
     peak, peak_src = measured_peak()
@@ -584,6 +679,7 @@ def run_ours(args):
         "cpu_baseline": cpu,
         "clocks": clock_info,
         "gpu_launches": launches_per_step * args.steps,
+        "paths": paths,
     }
     print(json.dumps(line), flush=True)
     return 0
@@ -701,18 +797,20 @@ def run_cache(args):
     P = int(len(w.copy_pairs))
     copy_bytes = 2 * 2 * P * w.block_bytes + 8 * P  # K and V blocks read and written, plus the pairs
     ops = {}
-    if T:
-        med, mean = timed(store, reps)
-        ops["reshape_and_cache"] = {"tokens": T, "algorithmic_bytes": store_bytes, "ms_l2_flushed_median": round(med, 5),
-                                    "ms_back_to_back_mean": round(mean, 5),
-                                    "achieved_gbs": round(store_bytes / (med * 1e-3) / 1e9, 2),
-                                    "frac": round(store_bytes / (med * 1e-3) / 1e9 / peak, 4)}
+    # in the step's order: the copies (repeated, they read blocks no store has touched yet), then
+    # the stores (repeated, idempotent), so the final state is the step's
     if P:
         med, mean = timed(copy, reps)
         ops["copy_blocks"] = {"pairs": P, "algorithmic_bytes": copy_bytes, "ms_l2_flushed_median": round(med, 5),
                               "ms_back_to_back_mean": round(mean, 5),
                               "achieved_gbs": round(copy_bytes / (med * 1e-3) / 1e9, 2),
                               "frac": round(copy_bytes / (med * 1e-3) / 1e9 / peak, 4)}
+    if T:
+        med, mean = timed(store, reps)
+        ops["reshape_and_cache"] = {"tokens": T, "algorithmic_bytes": store_bytes, "ms_l2_flushed_median": round(med, 5),
+                                    "ms_back_to_back_mean": round(mean, 5),
+                                    "achieved_gbs": round(store_bytes / (med * 1e-3) / 1e9, 2),
+                                    "frac": round(store_bytes / (med * 1e-3) / 1e9 / peak, 4)}
     if B.pa_get_device_error() != B.PA_DEV_OK:
         raise RuntimeError("device error in the cache operations")
     # the step's state is reproducible: check the caches against plain numpy indexing once

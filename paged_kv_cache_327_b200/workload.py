@@ -392,11 +392,21 @@ def lognormal_lengths(rng: np.random.Generator, n: int, median: float = 1024.0, 
     return np.clip(np.rint(np.exp(math.log(median) + sigma * z)), lo, hi).astype(np.int64)
 
 
-def _8b(seed: int, block_size: int, num_seqs: int = 256, num_q_tokens: int = 1, fp8: bool = False) -> Workload:
+def _8b(seed: int, block_size: int, num_seqs: int = 256, num_q_tokens: int = 1, fp8: bool = False,
+        uniform_lens: Optional[Tuple[int, int]] = None) -> Workload:
+    # uniform_lens=(lo, hi): the same shapes with lengths uniform in [lo, hi] (e.g. thousands of short
+    # or empty sequences, for the plan kernel's scaling) instead of the lognormal mix
     rng = np.random.default_rng([seed, _S_LENS])
-    L = np.maximum(lognormal_lengths(rng, num_seqs), num_q_tokens)
+    if uniform_lens is None:
+        L = np.maximum(lognormal_lengths(rng, num_seqs), num_q_tokens)
+        lens = "lognormal(median 1024, sigma 1.0) clipped to [32, 8192]"
+    else:
+        lo, hi = uniform_lens
+        L = rng.integers(lo, hi + 1, size=num_seqs)
+        L = np.where(L > 0, np.maximum(L, num_q_tokens), 0)
+        lens = f"uniform[{lo},{hi}]"
     kw = dict(num_q_heads=32, num_kv_heads=8, head_dim=128, block_size=block_size, q_dtype="bf16",
-              kv_dtype="bf16", seed=seed, notes={"lens": "lognormal(median 1024, sigma 1.0) clipped to [32, 8192]"})
+              kv_dtype="bf16", seed=seed, notes={"lens": lens})
     return independent("8b", L, num_q_tokens, **_fp8_kw(kw, fp8))
 
 
