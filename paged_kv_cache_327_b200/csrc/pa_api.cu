@@ -109,20 +109,30 @@ int current_device_info(int* dev, DeviceInfo** info) {
   return PA_OK;
 }
 
-// KV cache [num_blocks, block_size, num_kv_heads, head_dim] seen as a 3-D tensor
-// (128 bytes of a row, head_dim * elem / 128 * num_kv_heads 128-byte column blocks,
-// num_blocks * block_size rows); one box = block_size rows of one 128-byte column block,
-// 128-byte swizzle.
+// KV cache [num_blocks, block_size, num_kv_heads, head_dim] seen as a 3-D tensor of 128-byte
+// column blocks (head_dim * elem / 128 of them per KV head), 128-byte swizzle:
+//  * per block: dims (128 bytes of a row, column blocks, num_blocks * block_size rows); one box =
+//    block_size rows of one column block, coordinates (0, column block, row);
+//  * whole rows (two_blocks, a KV head row of two column blocks): dims (128 bytes, rows, column
+//    blocks) with strides (row pitch, 128 bytes) -- the outer stride below the middle one; one box
+//    = block_size rows of both column blocks of a KV head, landing as [block][row][128 bytes], the
+//    layout two per-block boxes give; coordinates (0, row, column block).
 int encode_kv_map(CUtensorMap* map, const void* base, int kv_dtype, int64_t num_blocks, int block_size,
-                  int num_kv_heads, int head_dim) {
+                  int num_kv_heads, int head_dim, bool two_blocks = false) {
   PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
   if (!enc) return PA_ERR_CUDA;
   const int es = elem_bytes(kv_dtype);
   const cuuint64_t inner = 128 / es;
-  const cuuint64_t dims[3] = {inner, static_cast<cuuint64_t>(head_dim * es / 128) * num_kv_heads,
-                              static_cast<cuuint64_t>(num_blocks) * block_size};
-  const cuuint64_t strides[2] = {128, static_cast<cuuint64_t>(num_kv_heads) * head_dim * es};
-  const cuuint32_t box[3] = {static_cast<cuuint32_t>(inner), 1, static_cast<cuuint32_t>(block_size)};
+  const cuuint64_t nblk = static_cast<cuuint64_t>(head_dim * es / 128) * num_kv_heads;
+  const cuuint64_t rows = static_cast<cuuint64_t>(num_blocks) * block_size;
+  const cuuint64_t pitch = static_cast<cuuint64_t>(num_kv_heads) * head_dim * es;
+  const cuuint64_t dims_b[3] = {inner, nblk, rows}, dims_r[3] = {inner, rows, nblk};
+  const cuuint64_t strides_b[2] = {128, pitch}, strides_r[2] = {pitch, 128};
+  const cuuint32_t box_b[3] = {static_cast<cuuint32_t>(inner), 1, static_cast<cuuint32_t>(block_size)};
+  const cuuint32_t box_r[3] = {static_cast<cuuint32_t>(inner), static_cast<cuuint32_t>(block_size), 2};
+  const cuuint64_t* dims = two_blocks ? dims_r : dims_b;
+  const cuuint64_t* strides = two_blocks ? strides_r : strides_b;
+  const cuuint32_t* box = two_blocks ? box_r : box_b;
   const cuuint32_t estr[3] = {1, 1, 1};
   const CUtensorMapDataType dt = kv_dtype == PA_BF16   ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
                                  : kv_dtype == PA_F16  ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
@@ -227,8 +237,8 @@ int launch_tc(const pa::DecodeParams& p, const CUtensorMap& tmk, const CUtensorM
 // eight-row tiles.
 template <int BS, int D>
 int dispatch_kv(const pa::DecodeParams& p, const CUtensorMap& tmk, const CUtensorMap& tmv, const CUtensorMap* tmq,
-                int64_t max_items, int dev, DeviceInfo* info, int kv_dtype, int q_dtype, int cols,
-                cudaStream_t stream) {
+                const CUtensorMap* tmk_blocks, int64_t max_items, int dev, DeviceInfo* info, int kv_dtype,
+                int q_dtype, int cols, cudaStream_t stream) {
   const bool qf32 = q_dtype == PA_F32;
   const int nt = (cols + 7) / 8;
   // one instantiation: KV element type K, query type Q, tiles per consumer N, paired, causal;
@@ -254,8 +264,10 @@ int dispatch_kv(const pa::DecodeParams& p, const CUtensorMap& tmk, const CUtenso
   if (nt > 1) {
     if constexpr (D == 128 && BS == 16) {  // 5th-generation tensor-core kernel, when chosen
       if (tmq) {
-        if (kv_dtype == PA_BF16 && q_dtype == PA_BF16) return launch_tc<bf16>(p, tmk, tmv, *tmq, max_items, dev, info, stream);
-        if (kv_dtype == PA_F16 && q_dtype == PA_F16) return launch_tc<f16>(p, tmk, tmv, *tmq, max_items, dev, info, stream);
+        if (kv_dtype == PA_BF16 && q_dtype == PA_BF16)
+          return launch_tc<bf16>(p, *tmk_blocks, tmv, *tmq, max_items, dev, info, stream);
+        if (kv_dtype == PA_F16 && q_dtype == PA_F16)
+          return launch_tc<f16>(p, *tmk_blocks, tmv, *tmq, max_items, dev, info, stream);
       }
     }
     if constexpr (D == 128) {
@@ -389,9 +401,12 @@ int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cac
   int dev;
   DeviceInfo* info;
   if (current_device_info(&dev, &info) != PA_OK) return PA_ERR_CUDA;
-  CUtensorMap tmk, tmv;
-  if (encode_kv_map(&tmk, k_cache, kv_dtype, num_blocks, block_size, num_kv_heads, head_dim) != PA_OK ||
-      encode_kv_map(&tmv, v_cache, kv_dtype, num_blocks, block_size, num_kv_heads, head_dim) != PA_OK)
+  // a KV head row of two 128-byte column blocks (16-bit, head_dim 128) is fetched one page per box;
+  // the tensor-core kernel reads K per column block (its S products take a chunk's rows of one block)
+  const bool two = elem_bytes(kv_dtype) * head_dim == 256;
+  CUtensorMap tmk, tmv, tmk_blocks;
+  if (encode_kv_map(&tmk, k_cache, kv_dtype, num_blocks, block_size, num_kv_heads, head_dim, two) != PA_OK ||
+      encode_kv_map(&tmv, v_cache, kv_dtype, num_blocks, block_size, num_kv_heads, head_dim, two) != PA_OK)
     return PA_ERR_CUDA;
 
   uint8_t* ws = static_cast<uint8_t*>(workspace);
@@ -435,16 +450,20 @@ int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cac
   int rc;
   const int c = static_cast<int>(cols);
   CUtensorMap tmq;
-  if (use_tc && encode_q_map(&tmq, q, q_dtype, static_cast<int64_t>(num_seqs) * qtok, num_q_heads, G,
-                             p.qbox_rows) != PA_OK)
+  if (use_tc && (encode_q_map(&tmq, q, q_dtype, static_cast<int64_t>(num_seqs) * qtok, num_q_heads, G,
+                              p.qbox_rows) != PA_OK ||
+                 encode_kv_map(&tmk_blocks, k_cache, kv_dtype, num_blocks, block_size, num_kv_heads, head_dim) !=
+                     PA_OK))
     return PA_ERR_CUDA;
   const CUtensorMap* tq = use_tc ? &tmq : nullptr;
   if (block_size == 16)
-    rc = head_dim == 128 ? dispatch_kv<16, 128>(p, tmk, tmv, tq, max_items, dev, info, kv_dtype, q_dtype, c, st)
-                         : dispatch_kv<16, 64>(p, tmk, tmv, tq, max_items, dev, info, kv_dtype, q_dtype, c, st);
+    rc = head_dim == 128
+             ? dispatch_kv<16, 128>(p, tmk, tmv, tq, &tmk_blocks, max_items, dev, info, kv_dtype, q_dtype, c, st)
+             : dispatch_kv<16, 64>(p, tmk, tmv, tq, &tmk_blocks, max_items, dev, info, kv_dtype, q_dtype, c, st);
   else
-    rc = head_dim == 128 ? dispatch_kv<32, 128>(p, tmk, tmv, tq, max_items, dev, info, kv_dtype, q_dtype, c, st)
-                         : dispatch_kv<32, 64>(p, tmk, tmv, tq, max_items, dev, info, kv_dtype, q_dtype, c, st);
+    rc = head_dim == 128
+             ? dispatch_kv<32, 128>(p, tmk, tmv, tq, &tmk_blocks, max_items, dev, info, kv_dtype, q_dtype, c, st)
+             : dispatch_kv<32, 64>(p, tmk, tmv, tq, &tmk_blocks, max_items, dev, info, kv_dtype, q_dtype, c, st);
   if (rc != PA_OK) return rc;
   {  // merge kernel: waits (griddepcontrol.wait) for the partition kernel's partial results
     const int64_t warps = static_cast<int64_t>(num_seqs) * qtok * num_q_heads;

@@ -535,11 +535,12 @@ __device__ __forceinline__ void produce(const DecodeParams& p, const CUtensorMap
         } else {
           const uint32_t qbytes = first ? static_cast<uint32_t>(rows * G * D * C::QE) : 0u;
           mbar_arrive_expect_tx(&full[slot], 2 * C::PAGE_BYTES + qbytes);
-#pragma unroll
-          for (int h = 0; h < C::HALVES; ++h) {
-            tma_load_3d(sb + h * C::BOX_BYTES, &tmk, 0, kvh * C::HALVES + h, phys * BS, &full[slot], pol);
-            tma_load_3d(sb + C::PAGE_BYTES + h * C::BOX_BYTES, &tmv, 0, kvh * C::HALVES + h, phys * BS,
-                        &full[slot], pol);
+          if constexpr (C::HALVES == 2) {  // one box per page: both column blocks of the KV head row
+            tma_load_3d(sb, &tmk, 0, phys * BS, kvh * 2, &full[slot], pol);
+            tma_load_3d(sb + C::PAGE_BYTES, &tmv, 0, phys * BS, kvh * 2, &full[slot], pol);
+          } else {
+            tma_load_3d(sb, &tmk, 0, kvh, phys * BS, &full[slot], pol);
+            tma_load_3d(sb + C::PAGE_BYTES, &tmv, 0, kvh, phys * BS, &full[slot], pol);
           }
         }
       }

@@ -6,24 +6,27 @@
 //   S = Q . K^T      tcgen05.mma, M = 64 query rows, N = 64 tokens (a chunk of 4 pages), K =
 //                    head_dim; A = the item's query rows (TMA-staged once per item), B = the
 //                    chunk's K rows (TMA-staged, 128-byte swizzle), D in tensor memory
-//   softmax          two warps share each TMEM lane quarter; the lane of query row r in each owns
-//                    half of the row's 64 scores: it keeps the row's running maximum (agreed with
-//                    the other half through shared memory) and its half of the running sum, raises
-//                    the maximum (and rescales the O row in tensor memory) only when a score
-//                    exceeds it by more than 2^8, and writes its half of the row's weights P,
-//                    rounded to the operand type, to shared memory
+//   softmax          an M = 64 product keeps 16 rows in each TMEM lane quarter; two warps share a
+//                    quarter, each reading half of the chunk's 64 columns in the 16x256b shape, so
+//                    every lane holds scores of two rows (a quad of lanes shares a row): the rows'
+//                    running maxima are agreed across the quad (shuffles) and the two warps (shared
+//                    memory), each lane keeps its part of the rows' running sums, the maximum is
+//                    raised (and the O rows rescaled in tensor memory) only when a score exceeds it
+//                    by more than 2^8, and the weights P, rounded to the operand type, go to shared
+//                    memory
 //   O += P . V       tcgen05.mma per page, M = 64, N = head_dim, K = 16 tokens; A = P, B = the
 //                    staged V page read in place (MN-major)
-// At the item's end each half-row's lane writes half of the row's head_dim outputs, divided by the
-// row's sum.  S and O products are issued by two warps of their own, so that neither waits for the
+// At the item's end each warp writes half of the head_dim outputs of its 16 rows, divided by the
+// rows' sums.  S and O products are issued by two warps of their own, so that neither waits for the
 // other's issue, and complete on mbarriers.  Double buffers keep every stage busy: two S buffers
 // and two P buffers (chunk n's softmax runs while the tensor core works on chunk n - 1's O and
 // chunk n + 1's S), two O buffers (an item's output is read while the next item accumulates), two
 // query buffers and five chunk buffers of 32 KB in flight per SM.
 //
 // CTA (one per SM): warps 0-7 run the softmax and the output (warp w on TMEM lane quarter w % 4,
-// columns 32 (w / 4) .. 32 (w / 4) + 31 of each chunk), warp 8 produces (the work list, TMA for the
-// K/V pages and the query rows), warp 9 issues the S products, warp 10 the O products.
+// columns 32 (w / 4) .. 32 (w / 4) + 31 of each chunk; a quarter without the item's rows skips the
+// arithmetic), warp 8 produces (the work list, TMA for the K/V pages and the query rows), warp 9
+// issues the S products, warp 10 the O products.
 // Block size 16, head_dim 128, 16-bit cache and query.
 #pragma once
 
@@ -92,6 +95,40 @@ __host__ __device__ constexpr uint32_t umma_idesc(uint32_t ab_type, uint32_t a_m
          ((M >> 4) << 24);
 }
 
+// 16 TMEM lanes x 256 bits per repetition (8 columns of 32 bits): in each 8-column block j, thread t
+// holds (lane t / 4, columns 8 j + 2 (t % 4), + 1) in registers 4 j, 4 j + 1 and (lane t / 4 + 8,
+// the same columns) in 4 j + 2, 4 j + 3 -- the lanes counted from the address's lane field.
+__device__ __forceinline__ void tmem_ld16x256_x4(uint32_t taddr, uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.16x256b.x4.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
+      "%14, %15}, [%16];"
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]), "=r"(v[8]),
+        "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_st16x256_x4(uint32_t taddr, const uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.16x256b.x4.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
+      "%14, %15, %16};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]),
+      "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+      : "memory");
+}
+// N / 4 repetitions of the x4 form: N registers, columns 0 .. 2 N - 1 from the address
+template <int N>
+__device__ __forceinline__ void tmem_ld16x256(uint32_t taddr, uint32_t (&v)[N]) {
+  static_assert(N % 16 == 0, "registers");
+#pragma unroll
+  for (int i = 0; i < N / 16; ++i)
+    tmem_ld16x256_x4(taddr + 32 * i, *reinterpret_cast<uint32_t(*)[16]>(&v[16 * i]));
+}
+template <int N>
+__device__ __forceinline__ void tmem_st16x256(uint32_t taddr, const uint32_t (&v)[N]) {
+#pragma unroll
+  for (int i = 0; i < N / 16; ++i)
+    tmem_st16x256_x4(taddr + 32 * i, *reinterpret_cast<const uint32_t(*)[16]>(&v[16 * i]));
+}
+
 // ---------------------------------------------------------------- helpers
 // named barrier of the consumer warps, reducing a predicate (each warp reconverges first: the
 // barrier instructions are warp-aligned)
@@ -156,34 +193,32 @@ struct TcCfg {
   static constexpr int OFF_BAR = OFF_P + 2 * PBUF;
   // mbarriers: chunk full / empty, query buffer free, S full / free, P full / free (the O product
   // that read it is done), O buffer free (its item's output has been read), final drain
-  static constexpr int B_FULL = 0, B_EMPTY = NCH, B_QFREE = 2 * NCH, B_SFULL = B_QFREE + QN, B_SFREE = B_SFULL + 2,
-                       B_PFULL = B_SFREE + 2, B_PFREE = B_PFULL + 2, B_OFREE = B_PFREE + 2, B_FIN = B_OFREE + 2,
+  static constexpr int NSB = 3;  // S buffers: S products run up to NSB - 1 chunks ahead of the softmax
+  static constexpr int B_FULL = 0, B_EMPTY = NCH, B_QFREE = 2 * NCH, B_SFULL = B_QFREE + QN, B_SFREE = B_SFULL + NSB,
+                       B_PFULL = B_SFREE + NSB, B_PFREE = B_PFULL + 2, B_OFREE = B_PFREE + 2, B_FIN = B_OFREE + 2,
                        NBAR = B_FIN + 1;
   static constexpr int OFF_META = OFF_BAR + ((NBAR * 8 + 15) & ~15);
-  // exchange between the two softmax warps of a lane quarter: chunk maxima [2 S buffers][2 halves][M]
+  // exchange between the two softmax warps of a lane quarter: chunk maxima [NSB S buffers][2 halves][M]
   // and item sums [2 items][2 halves][M]
   static constexpr int OFF_XCH = OFF_META + NCH * 32;
-  static constexpr int OFF_MISC = OFF_XCH + 8 * M * 4;
+  static constexpr int OFF_MISC = OFF_XCH + (2 * NSB + 4) * M * 4;
   static constexpr int SMEM_BYTES = 1024 + OFF_MISC + 16;
   // warps 0-7: softmax and output, warp 8 loads, warp 9 issues the S products, warp 10 the O products
   static constexpr int NSM = 256, W_LOAD = 8, W_S = 9, W_O = 10, NTHREADS = NSM + 96;
   static constexpr int HC = CT / 2;  // chunk columns per softmax warp
-  // TMEM columns: two O buffers (head_dim columns each), then two S buffers (one chunk each)
+  // TMEM columns: two O buffers (head_dim columns each), then NSB S buffers (one chunk each)
   static constexpr uint32_t TM_COLS = 512, TM_O = 0, TM_S = 2 * D;
   static constexpr uint32_t AB = std::is_same<KT, __nv_bfloat16>::value ? 1u : 0u;
   static constexpr uint32_t IDESC_S = umma_idesc(AB, 0, 0, M, CT);  // Q (K-major) . K^T (K-major)
   static constexpr uint32_t IDESC_O = umma_idesc(AB, 0, 1, M, D);   // P (K-major) . V (MN-major)
   static_assert(CHUNK_BYTES % 1024 == 0 && OFF_Q % 1024 == 0 && QHALF % 1024 == 0 && OFF_P % 1024 == 0,
                 "128-byte swizzle atoms");
-  static_assert(TM_S + 2 * CT <= TM_COLS, "tensor memory");
+  static_assert(TM_S + NSB * CT <= TM_COLS, "tensor memory");
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
 };
 
-// TMEM lane of row r of an M = 64 product (and of its operand A): rows 16 q .. 16 q + 15 occupy
-// lanes 0-15 of lane quarter q.  Returns -1 for a lane that holds no row.
-__device__ __forceinline__ int tc_lane_row(int lane128) {
-  return (lane128 & 31) < 16 ? (lane128 >> 5) * 16 + (lane128 & 31) : -1;
-}
+// An M = 64 product (and its operand A) keeps rows 16 q .. 16 q + 15 in lanes 0-15 of TMEM lane
+// quarter q.
 
 // 4-D tiled TMA load global -> shared, completion counted on `bar` in bytes (no cache hint).
 __device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, int x, int y, int z, int w,
@@ -314,14 +349,16 @@ __device__ __forceinline__ void tc_produce(const DecodeParams& p, const CUtensor
       }
       __syncwarp();  // the expected byte count is set before any copy can complete
       if (!bad) {
-        // one box per lane: page lane / 4, K half 0 / K half 1 / V half 0 / V half 1
-        const int lp = lane >> 2, lh = lane & 1;
-        const bool lv = (lane & 2) != 0;
-        const int lphys = __shfl_sync(FULL, cur.bt, (pg0 + lp) & 31);
+        // one box per lane: K column block 0 / K column block 1 / the whole V page, of page lane / 3
+        // (K rows go to the chunk's block-major K operand, a V page lands as [block][row])
+        const int lp = lane / 3, lk = lane - 3 * lp;
+        const int lphys = __shfl_sync(FULL, cur.bt, (pg0 + min(lp, C::CH - 1)) & 31);
         uint8_t* cb = smem + c * C::CHUNK_BYTES;
         if (lp < npg) {
-          uint8_t* dst = lv ? cb + 2 * C::KH_BYTES + lp * C::VPAGE + lh * C::BOX : cb + lh * C::KH_BYTES + lp * C::BOX;
-          tma_load_3d(dst, lv ? &tmv : &tmk, 0, kvh * 2 + lh, lphys * BS, &full[c], pol);
+          if (lk < 2)
+            tma_load_3d(cb + lk * C::KH_BYTES + lp * C::BOX, &tmk, 0, kvh * 2 + lk, lphys * BS, &full[c], pol);
+          else
+            tma_load_3d(cb + 2 * C::KH_BYTES + lp * C::VPAGE, &tmv, 0, lphys * BS, kvh * 2, &full[c], pol);
         }
         // the item's query rows with its first chunk: rows (query token or member) x G heads, one
         // box per 64-element half, landing as the K-major A operand
@@ -396,9 +433,9 @@ __device__ __forceinline__ void tc_mma_s(uint8_t* smem, uint64_t* bars, const in
     }
     const bool last = (flags & F_LAST) != 0;
     if (!item_bad) {
-      const uint32_t b = ns & 1u;
-      if (ns >= 2) {  // the softmax warps have read S(ns - 2) out of this buffer
-        const bool fr = mbar_wait_bounded(&s_free[b], ((ns >> 1) - 1) & 1u, kWaitLimit);
+      const uint32_t b = ns % C::NSB;
+      if (ns >= C::NSB) {  // the softmax warps have read S(ns - NSB) out of this buffer
+        const bool fr = mbar_wait_bounded(&s_free[b], ((ns / C::NSB) - 1) & 1u, kWaitLimit);
         if (!__all_sync(FULL, fr)) {
           ok = false;
           break;
@@ -522,7 +559,7 @@ __global__ void __launch_bounds__(TcCfg<KT>::NTHREADS, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
   int4* meta = reinterpret_cast<int4*>(smem + C::OFF_META);
   float* xmax = reinterpret_cast<float*>(smem + C::OFF_XCH);  // [S buffer][half][M]
-  float* xsum = xmax + 4 * M;                                  // [item parity][half][M]
+  float* xsum = xmax + 2 * C::NSB * M;                         // [item parity][half][M]
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC + 4);
 
@@ -531,7 +568,7 @@ __global__ void __launch_bounds__(TcCfg<KT>::NTHREADS, 1)
       // S free, P full and O free: one arrival per softmax warp; a chunk buffer is free once the
       // softmax warps and the S warp have read its meta and the O warp has finished with it (or
       // skipped it); the final drain: one commit per MMA warp
-      const bool sm = (s >= C::B_SFREE && s < C::B_SFREE + 2) || (s >= C::B_PFULL && s < C::B_PFULL + 2) ||
+      const bool sm = (s >= C::B_SFREE && s < C::B_SFREE + C::NSB) || (s >= C::B_PFULL && s < C::B_PFULL + 2) ||
                       (s >= C::B_OFREE && s < C::B_OFREE + 2);
       const bool empty = s >= C::B_EMPTY && s < C::B_EMPTY + C::NCH;
       mbar_init(&bars[s], sm ? C::NSM / 32 : empty ? C::NSM / 32 + 2 : s == C::B_FIN ? 2 : 1);
@@ -564,8 +601,13 @@ __global__ void __launch_bounds__(TcCfg<KT>::NTHREADS, 1)
   }
 
   // ============================== softmax and output (warps 0-7) ==============================
+  // Warp w reads the 16 rows of lane quarter q = w % 4 in the 16x256b shape: lane t holds rows
+  // 16 q + t / 4 and 16 q + t / 4 + 8 at the chunk columns 32 h + 8 j + 2 (t % 4), + 1 (j < 4) of
+  // its half h = w / 4.  The four lanes of a quad share their rows, and the two warps of the
+  // quarter share them through shared memory.
   constexpr unsigned FULL = 0xffffffffu;
   constexpr float kNone = -1e30f;  // running maximum of a row with no score yet (finite: no NaN from -inf - -inf)
+  constexpr int NJ = HC / 8;       // 8-column blocks of this warp's half chunk
   uint64_t* full = bars + C::B_FULL;
   uint64_t* empty = bars + C::B_EMPTY;
   uint64_t* s_full = bars + C::B_SFULL;
@@ -574,18 +616,20 @@ __global__ void __launch_bounds__(TcCfg<KT>::NTHREADS, 1)
   uint64_t* p_free = bars + C::B_PFREE;
   uint64_t* o_free = bars + C::B_OFREE;
   const int ct = threadIdx.x;
-  const int quarter = warp & 3, half = warp >> 2;  // TMEM lane quarter; chunk columns 32 half .. + 31
+  const int quarter = warp & 3, half = warp >> 2;
   const int bar_pair = 1 + quarter;
-  const int row = tc_lane_row(quarter * 32 + lane);                     // this lane's query row, or -1
-  const uint32_t tl = tm + (static_cast<uint32_t>(quarter * 32) << 16);  // the lane quarter
+  const int rq = lane >> 2, cq = lane & 3;                 // row in the quarter's first eight, column pair
+  const int row0 = quarter * 16 + rq, row1 = row0 + 8;     // this lane's two query rows
+  const uint32_t tl = tm + (static_cast<uint32_t>(quarter * 32) << 16);  // the lane quarter (rows in lanes 0-15)
   const int G = p.group, Hq = p.num_q_heads, T = p.qtok, HV = T * Hq;
   const float sl = p.scale_log2;
   uint32_t n = 0, ns = 0, np = 0;
   int items = -1;
   bool ok = true;
-  float m = kNone, l = 0.f;  // the row's running maximum (log2 units); this half's running sum
+  float m0r = kNone, m1r = kNone;  // the rows' running maxima (log2 units)
+  float l0 = 0.f, l1 = 0.f;        // this lane's part of the rows' running sums
   int ncol = 0, item_t0 = 0, first_np = 0;
-  bool poisoned = false, live = false;
+  bool poisoned = false, busy = false;  // busy: the quarter holds at least one of the item's rows
 
   // completion of O product k (the P buffer it read is free again)
   auto wait_o = [&](uint32_t k) -> bool {
@@ -601,21 +645,21 @@ __global__ void __launch_bounds__(TcCfg<KT>::NTHREADS, 1)
       ok = false;
       break;
     }
-    const int4 m0 = meta[2 * c], m1 = meta[2 * c + 1];
-    const int flags = (m0.z >> 24) & 0xff;
+    const int4 mt0 = meta[2 * c], mt1 = meta[2 * c + 1];
+    const int flags = (mt0.z >> 24) & 0xff;
     if (flags & F_END) break;
     const bool first = (flags & F_FIRST) != 0, last = (flags & F_LAST) != 0;
     if (first) {
       ++items;
       poisoned = (flags & F_BAD) != 0;
-      ncol = ((m0.z >> 16) & 0xff) * G;
-      item_t0 = m1.x;
-      live = row >= 0 && row < ncol;
-      m = kNone;
-      l = 0.f;
+      ncol = ((mt0.z >> 16) & 0xff) * G;
+      item_t0 = mt1.x;
+      busy = quarter * 16 < ncol;
+      m0r = m1r = kNone;
+      l0 = l1 = 0.f;
       first_np = static_cast<int>(np);
     }
-    const int npg = (m0.z >> 8) & 0xff, ntok_last = m1.y;
+    const int npg = (mt0.z >> 8) & 0xff, ntok_last = mt1.y;
     uint8_t* cb = smem + c * C::CHUNK_BYTES;
     const uint32_t ob = static_cast<uint32_t>(items) & 1u;
 
@@ -630,90 +674,106 @@ __global__ void __launch_bounds__(TcCfg<KT>::NTHREADS, 1)
           for (int q = 0; q < 8; ++q) *reinterpret_cast<uint4*>(vrow + h * C::BOX + q * 16) = make_uint4(0u, 0u, 0u, 0u);
         fence_proxy_async_smem();
       }
-      const uint32_t b = ns & 1u;
-      bool good = mbar_wait_bounded(&s_full[b], (ns >> 1) & 1u, kWaitLimit);
+      const uint32_t b = ns % C::NSB;
+      bool good = mbar_wait_bounded(&s_full[b], (ns / C::NSB) & 1u, kWaitLimit);
       tc_fence_after();
-      uint32_t sr[HC];
-      tmem_ldn<HC>(tl + C::TM_S + b * CT + half * HC, sr);
-      tc_wait_ld();
+      uint32_t sr[HC / 2];
+      if (busy) {
+        tmem_ld16x256<HC / 2>(tl + C::TM_S + b * CT + half * HC, sr);
+        tc_wait_ld();
+      }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&s_free[b]);
       ++ns;
 
-      // scores in log2 units, -inf where masked: tokens past the item's end; with several query
-      // tokens, row r (query token r / G of the item) sees keys at relative positions <= r / G.
-      // This lane holds chunk columns j0 .. j0 + HC - 1 of its row.
-      const int ntok = (npg - 1) * C::BS + ntok_last;
-      const int jend = live ? (CAUSAL && T > 1 ? min(ntok, row / G - m0.w + 1) : ntok) : 0;
-      const int jn = jend - half * HC;  // valid columns of this half: j < jn
-      // the maximum of this half's valid scores, as a tree (no long dependent chain)
-      float xv[HC];
+      uint32_t pk[2][NJ];  // this lane's packed weights: [row][block]
+      if (busy) {
+        // scores in log2 units, -inf where masked: tokens past the item's end; with several query
+        // tokens, row r (query token r / G of the item) sees keys at relative positions <= r / G
+        const int ntok = (npg - 1) * C::BS + ntok_last;
+        auto jend_of = [&](int r) {
+          return r < ncol ? (CAUSAL && T > 1 ? min(ntok, r / G - mt0.w + 1) : ntok) : 0;
+        };
+        const int j0 = half * HC + 2 * cq;  // chunk column of this lane's first value
+        const int e0 = jend_of(row0) - j0, e1 = jend_of(row1) - j0;  // valid iff 8 j (+1) < e
+        float x0 = -CUDART_INF_F, x1 = -CUDART_INF_F;
 #pragma unroll
-      for (int j = 0; j < HC; ++j) xv[j] = j < jn ? __uint_as_float(sr[j]) : -CUDART_INF_F;
-#pragma unroll
-      for (int w = HC / 2; w >= 1; w >>= 1)
-#pragma unroll
-        for (int j = 0; j < w; ++j) xv[j] = fmaxf(xv[j], xv[j + w]);
-      float mx = xv[0];
-      // the row's chunk maximum: both halves' (exchanged through shared memory, one buffer per S
-      // buffer: it is rewritten two products later, once both warps have passed the barrier of the
-      // product in between -- S products are counted alike in both warps, poisoned chunks have none)
-      float* xm = xmax + b * 2 * M;
-      if (row >= 0) xm[half * M + row] = mx;
-      bar_sync(bar_pair, 64);
-      if (row >= 0) mx = fmaxf(mx, xm[(half ^ 1) * M + row]);
-      mx *= sl;  // scale > 0 commutes with max
-      const bool raise = mx > m + kRescaleThreshold;
-      const float mnew = raise ? mx : m;
-      const float alpha = raise ? fast_exp2(m - mnew) : 1.f;  // 0 for a row without scores so far
-      // an O row that already holds this item's products is rescaled in tensor memory (by the first
-      // half's warp); the products issued so far must be done (the tcgen05.ld / st are warp-wide, so
-      // the warp votes)
-      if (half == 0 && __any_sync(FULL, raise) && static_cast<int>(np) > first_np) {
-        good = wait_o(np - 1) && good;
-        uint32_t ov[64];
-#pragma unroll
-        for (int h = 0; h < D / 64; ++h) {
-          tmem_ldn<64>(tl + C::TM_O + ob * D + h * 64, ov);
-          tc_wait_ld();
-#pragma unroll
-          for (int i = 0; i < 64; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
-          tmem_stn<64>(tl + C::TM_O + ob * D + h * 64, ov);
+        for (int j = 0; j < NJ; ++j) {
+          x0 = fmaxf(x0, fmaxf(8 * j < e0 ? __uint_as_float(sr[4 * j]) : -CUDART_INF_F,
+                               8 * j + 1 < e0 ? __uint_as_float(sr[4 * j + 1]) : -CUDART_INF_F));
+          x1 = fmaxf(x1, fmaxf(8 * j < e1 ? __uint_as_float(sr[4 * j + 2]) : -CUDART_INF_F,
+                               8 * j + 1 < e1 ? __uint_as_float(sr[4 * j + 3]) : -CUDART_INF_F));
         }
-        tc_wait_st();
+        x0 = fmaxf(x0, __shfl_xor_sync(FULL, x0, 1));
+        x1 = fmaxf(x1, __shfl_xor_sync(FULL, x1, 1));
+        x0 = fmaxf(x0, __shfl_xor_sync(FULL, x0, 2));
+        x1 = fmaxf(x1, __shfl_xor_sync(FULL, x1, 2));
+        // the rows' chunk maxima: both halves' (exchanged through shared memory, one buffer per S
+        // buffer: it is rewritten NSB products later, once both warps have passed the barriers of
+        // the products in between -- S products are counted alike in both warps)
+        float* xm = xmax + b * 2 * M;
+        if (cq == 0) {
+          xm[half * M + row0] = x0;
+          xm[half * M + row1] = x1;
+        }
+        bar_sync(bar_pair, 64);
+        x0 = fmaxf(x0, xm[(half ^ 1) * M + row0]) * sl;  // scale > 0 commutes with max
+        x1 = fmaxf(x1, xm[(half ^ 1) * M + row1]) * sl;
+        const bool up0 = x0 > m0r + kRescaleThreshold, up1 = x1 > m1r + kRescaleThreshold;
+        const float n0 = up0 ? x0 : m0r, n1 = up1 ? x1 : m1r;
+        const float a0 = up0 ? fast_exp2(m0r - n0) : 1.f, a1 = up1 ? fast_exp2(m1r - n1) : 1.f;  // 0 for a fresh row
+        // O rows that already hold this item's products are rescaled in tensor memory (by the first
+        // half's warp) once the products issued so far are done (warp-wide ld / st: the warp votes)
+        if (half == 0 && __any_sync(FULL, up0 || up1) && static_cast<int>(np) > first_np) {
+          good = wait_o(np - 1) && good;
+#pragma unroll
+          for (int h = 0; h < D / 32; ++h) {  // 32 columns of the O rows per pass
+            uint32_t ov[16];
+            tmem_ld16x256_x4(tl + C::TM_O + ob * D + h * 32, ov);
+            tc_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 16; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * ((i & 2) ? a1 : a0));
+            tmem_st16x256_x4(tl + C::TM_O + ob * D + h * 32, ov);
+          }
+          tc_wait_st();
+        }
+        m0r = n0;
+        m1r = n1;
+        l0 *= a0;
+        l1 *= a1;
+        // the weights the MMA sees; the sums are taken over the same rounded values
+        float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+        for (int j = 0; j < NJ; ++j) {
+          const float w0 = 8 * j < e0 ? fast_exp2(fmaf(__uint_as_float(sr[4 * j]), sl, -m0r)) : 0.f;
+          const float w1 = 8 * j + 1 < e0 ? fast_exp2(fmaf(__uint_as_float(sr[4 * j + 1]), sl, -m0r)) : 0.f;
+          const float w2 = 8 * j < e1 ? fast_exp2(fmaf(__uint_as_float(sr[4 * j + 2]), sl, -m1r)) : 0.f;
+          const float w3 = 8 * j + 1 < e1 ? fast_exp2(fmaf(__uint_as_float(sr[4 * j + 3]), sl, -m1r)) : 0.f;
+          pk[0][j] = pack2<KT>(w0, w1);
+          pk[1][j] = pack2<KT>(w2, w3);
+          const float2 r0 = unpack2<KT>(pk[0][j]), r1 = unpack2<KT>(pk[1][j]);
+          s0 += r0.x + r0.y;
+          s1 += r1.x + r1.y;
+        }
+        l0 += s0;
+        l1 += s1;
       }
-      m = mnew;
-      l *= alpha;
-      // this half of the P row: the weights the MMA sees, their sum taken over the same rounded values
-      uint32_t pk[HC / 2];
-      float ls[HC / 2];
-#pragma unroll
-      for (int j = 0; j < HC; j += 2) {
-        const float e0 = j < jn ? fast_exp2(fmaf(__uint_as_float(sr[j]), sl, -m)) : 0.f;
-        const float e1 = j + 1 < jn ? fast_exp2(fmaf(__uint_as_float(sr[j + 1]), sl, -m)) : 0.f;
-        pk[j / 2] = pack2<KT>(e0, e1);
-        const float2 w2 = unpack2<KT>(pk[j / 2]);
-        ls[j / 2] = w2.x + w2.y;
-      }
-#pragma unroll
-      for (int w = HC / 4; w >= 1; w >>= 1)  // their sum, as a tree
-#pragma unroll
-        for (int j = 0; j < w; ++j) ls[j] += ls[j + w];
-      l += ls[0];
       // the P buffer is free once O(np - 2) is done
       if (np >= 2) good = wait_o(np - 2) && good;
       if (!__all_sync(FULL, good)) {
         ok = false;
         break;
       }
-      if (row >= 0) {  // K-major A operand: row `row`, 16-byte chunk q at ((q ^ (row & 7)) << 4)
-        uint8_t* prow = smem + C::OFF_P + (np & 1u) * C::PBUF + row * 128;
+      {  // K-major A operand: row r at r * 128, 16-byte chunk q at ((q ^ (r & 7)) << 4); this lane's
+         // pair of columns is 4 bytes at 4 (t % 4) in chunk (32 h + 8 j) / 8.  Rows of a quarter
+         // without the item's rows get zero weights (their products are not read).
+        uint8_t* pb = smem + C::OFF_P + (np & 1u) * C::PBUF;
 #pragma unroll
-        for (int q = 0; q < HC / 8; ++q) {
-          const int qc = half * (HC / 8) + q;
-          *reinterpret_cast<uint4*>(prow + ((qc ^ (row & 7)) << 4)) =
-              make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+        for (int j = 0; j < NJ; ++j) {
+          const int qc = half * NJ + j;
+          *reinterpret_cast<uint32_t*>(pb + row0 * 128 + ((qc ^ (row0 & 7)) << 4) + 4 * cq) = busy ? pk[0][j] : 0u;
+          *reinterpret_cast<uint32_t*>(pb + row1 * 128 + ((qc ^ (row1 & 7)) << 4) + 4 * cq) = busy ? pk[1][j] : 0u;
         }
       }
       fence_proxy_async_smem();
@@ -726,7 +786,7 @@ __global__ void __launch_bounds__(TcCfg<KT>::NTHREADS, 1)
     if (lane == 0) mbar_arrive(&empty[c]);  // this warp is done with the chunk's meta and V rows
 
     if (last) {
-      // output of the item: each half-row's lane writes half of the row's head_dim columns
+      // output of the item: each warp writes its half of the head_dim columns of its 16 rows
       const bool o_any = static_cast<int>(np) > first_np;
       bool good = true;
       if (!poisoned && o_any) good = wait_o(np - 1);
@@ -735,64 +795,72 @@ __global__ void __launch_bounds__(TcCfg<KT>::NTHREADS, 1)
         break;
       }
       const bool bad = poisoned || !o_any;
-      // the row's sum: both halves' (one buffer per item parity: every item, poisoned or not, ends
-      // with this barrier, so a buffer is rewritten only after both warps have read it)
+      // the rows' sums: the quad's parts, then both halves' (one buffer per item parity: every item,
+      // poisoned or not, ends with this barrier, so a buffer is rewritten only after both warps
+      // have read it)
+      l0 += __shfl_xor_sync(FULL, l0, 1);
+      l1 += __shfl_xor_sync(FULL, l1, 1);
+      l0 += __shfl_xor_sync(FULL, l0, 2);
+      l1 += __shfl_xor_sync(FULL, l1, 2);
       float* xs = xsum + (items & 1) * 2 * M;
-      if (row >= 0) xs[half * M + row] = l;
+      if (cq == 0) {
+        xs[half * M + row0] = l0;
+        xs[half * M + row1] = l1;
+      }
       bar_sync(bar_pair, 64);
-      const float lt = row >= 0 ? l + xs[(half ^ 1) * M + row] : 0.f;
-      const int seq = m0.x, part = m0.y & 0xffff, kvh = m0.z & 0xff;
-      const bool direct = (flags & F_DIRECT) != 0;
-      int64_t ofs = 0;
-      float fs = 0.f;
-      if (live) {
-        const int g = row % G, mq = row / G;
-        const int mb = T > 1 ? 0 : mq, t = T > 1 ? item_t0 + mq : 0;
-        const int vh = t * Hq + kvh * G + g;
-        if (direct) {
-          ofs = (static_cast<int64_t>(seq + mb) * HV + vh) * D;
-          fs = bad ? CUDART_NAN_F : p.v_scale / lt;
-        } else {
-          const int64_t pidx = static_cast<int64_t>(seq + mb) * p.max_parts + part;
-          ofs = (pidx * HV + vh) * D;
-          fs = bad ? CUDART_NAN_F : p.v_scale;
-          if (half == 0)
-            __stcg(&p.part_ml[pidx * HV + vh], bad ? make_float2(0.f, CUDART_NAN_F) : make_float2(m, lt));
+      const float lt0 = l0 + xs[(half ^ 1) * M + row0], lt1 = l1 + xs[(half ^ 1) * M + row1];
+      if (busy) {
+        const int seq = mt0.x, part = mt0.y & 0xffff, kvh = mt0.z & 0xff;
+        const bool direct = (flags & F_DIRECT) != 0;
+        int64_t ofs[2];
+        float fs[2];
+        bool live[2];
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+          const int r = i ? row1 : row0;
+          const float lt = i ? lt1 : lt0, mr = i ? m1r : m0r;
+          live[i] = r < ncol;
+          const int g = r % G, mq = r / G;
+          const int mb = T > 1 ? 0 : mq, t = T > 1 ? item_t0 + mq : 0;
+          const int vh = t * Hq + kvh * G + g;
+          if (direct) {
+            ofs[i] = (static_cast<int64_t>(seq + mb) * HV + vh) * D;
+            fs[i] = bad ? CUDART_NAN_F : p.v_scale / lt;
+          } else {
+            const int64_t pidx = static_cast<int64_t>(seq + mb) * p.max_parts + part;
+            ofs[i] = (pidx * HV + vh) * D;
+            fs[i] = bad ? CUDART_NAN_F : p.v_scale;
+            if (live[i] && half == 0 && cq == 0)
+              __stcg(&p.part_ml[pidx * HV + vh], bad ? make_float2(0.f, CUDART_NAN_F) : make_float2(mr, lt));
+          }
         }
-      }
-      const int h = half;  // this warp's 64 of the head_dim columns
-      uint32_t ov[64];
-      if (!bad) {
-        tmem_ldn<64>(tl + C::TM_O + ob * D + h * 64, ov);
-        tc_wait_ld();
-      } else {
 #pragma unroll
-        for (int i = 0; i < 64; ++i) ov[i] = 0u;
-      }
-      if (live) {
-        if (!direct) {
-          float4* dst = reinterpret_cast<float4*>(p.part_acc + ofs + h * 64);
+        for (int h2 = 0; h2 < 2; ++h2) {  // this warp's 64 columns, 32 per pass
+          const int col0 = half * 64 + h2 * 32;
+          uint32_t ov[16];
+          if (!bad) {
+            tmem_ld16x256_x4(tl + C::TM_O + ob * D + col0, ov);
+            tc_wait_ld();
+          } else {
 #pragma unroll
-          for (int i = 0; i < 16; ++i)
-            __stcg(dst + i, make_float4(__uint_as_float(ov[4 * i]) * fs, __uint_as_float(ov[4 * i + 1]) * fs,
-                                        __uint_as_float(ov[4 * i + 2]) * fs, __uint_as_float(ov[4 * i + 3]) * fs));
-        } else if (p.out_dtype == DT_F32) {
-          float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + ofs + h * 64);
+            for (int i = 0; i < 16; ++i) ov[i] = 0u;
+          }
 #pragma unroll
-          for (int i = 0; i < 16; ++i)
-            dst[i] = make_float4(__uint_as_float(ov[4 * i]) * fs, __uint_as_float(ov[4 * i + 1]) * fs,
-                                 __uint_as_float(ov[4 * i + 2]) * fs, __uint_as_float(ov[4 * i + 3]) * fs);
-        } else {
-          uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) + ofs + h * 64);
+          for (int i = 0; i < 2; ++i) {
+            if (!live[i]) continue;
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            uint32_t w[4];
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              const float a = __uint_as_float(ov[8 * i + 2 * k]) * fs, b2 = __uint_as_float(ov[8 * i + 2 * k + 1]) * fs;
-              w[k] = p.out_dtype == DT_BF16 ? pack2<__nv_bfloat16>(a, b2) : pack2<__half>(a, b2);
+            for (int j = 0; j < 4; ++j) {
+              const int64_t e = ofs[i] + col0 + 8 * j + 2 * cq;
+              const float a = __uint_as_float(ov[4 * j + 2 * i]) * fs[i];
+              const float b2 = __uint_as_float(ov[4 * j + 2 * i + 1]) * fs[i];
+              if (!direct)
+                __stcg(reinterpret_cast<float2*>(p.part_acc + e), make_float2(a, b2));
+              else if (p.out_dtype == DT_F32)
+                *reinterpret_cast<float2*>(static_cast<float*>(p.out) + e) = make_float2(a, b2);
+              else
+                *reinterpret_cast<uint32_t*>(static_cast<uint16_t*>(p.out) + e) =
+                    p.out_dtype == DT_BF16 ? pack2<__nv_bfloat16>(a, b2) : pack2<__half>(a, b2);
             }
-            dst[i] = make_uint4(w[0], w[1], w[2], w[3]);
           }
         }
       }
