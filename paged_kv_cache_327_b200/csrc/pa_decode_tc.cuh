@@ -622,6 +622,7 @@ __global__ void __launch_bounds__(TcCfg<KT>::NTHREADS, 1)
   const int row0 = quarter * 16 + rq, row1 = row0 + 8;     // this lane's two query rows
   const uint32_t tl = tm + (static_cast<uint32_t>(quarter * 32) << 16);  // the lane quarter (rows in lanes 0-15)
   const int G = p.group, Hq = p.num_q_heads, T = p.qtok, HV = T * Hq;
+  const int rt0 = row0 / G, rt1 = row1 / G;  // the rows' query token (or member) in an item
   const float sl = p.scale_log2;
   uint32_t n = 0, ns = 0, np = 0;
   int items = -1;
@@ -692,11 +693,11 @@ __global__ void __launch_bounds__(TcCfg<KT>::NTHREADS, 1)
         // scores in log2 units, -inf where masked: tokens past the item's end; with several query
         // tokens, row r (query token r / G of the item) sees keys at relative positions <= r / G
         const int ntok = (npg - 1) * C::BS + ntok_last;
-        auto jend_of = [&](int r) {
-          return r < ncol ? (CAUSAL && T > 1 ? min(ntok, r / G - mt0.w + 1) : ntok) : 0;
+        auto jend_of = [&](int r, int rt) {
+          return r < ncol ? (CAUSAL && T > 1 ? min(ntok, rt - mt0.w + 1) : ntok) : 0;
         };
         const int j0 = half * HC + 2 * cq;  // chunk column of this lane's first value
-        const int e0 = jend_of(row0) - j0, e1 = jend_of(row1) - j0;  // valid iff 8 j (+1) < e
+        const int e0 = jend_of(row0, rt0) - j0, e1 = jend_of(row1, rt1) - j0;  // valid iff 8 j (+1) < e
         float x0 = -CUDART_INF_F, x1 = -CUDART_INF_F;
 #pragma unroll
         for (int j = 0; j < NJ; ++j) {
@@ -820,7 +821,7 @@ __global__ void __launch_bounds__(TcCfg<KT>::NTHREADS, 1)
           const int r = i ? row1 : row0;
           const float lt = i ? lt1 : lt0, mr = i ? m1r : m0r;
           live[i] = r < ncol;
-          const int g = r % G, mq = r / G;
+          const int mq = i ? rt1 : rt0, g = r - mq * G;
           const int mb = T > 1 ? 0 : mq, t = T > 1 ? item_t0 + mq : 0;
           const int vh = t * Hq + kvh * G + g;
           if (direct) {
