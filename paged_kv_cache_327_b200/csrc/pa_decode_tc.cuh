@@ -6,27 +6,29 @@
 //   S = Q . K^T      tcgen05.mma, M = 64 query rows, N = 64 tokens (a chunk of 4 pages), K =
 //                    head_dim; A = the item's query rows (TMA-staged once per item), B = the
 //                    chunk's K rows (TMA-staged, 128-byte swizzle), D in tensor memory
-//   softmax          an M = 64 product keeps 16 rows in each TMEM lane quarter; two warps share a
-//                    quarter, each reading half of the chunk's 64 columns in the 16x256b shape, so
-//                    every lane holds scores of two rows (a quad of lanes shares a row): the rows'
-//                    running maxima are agreed across the quad (shuffles) and the two warps (shared
-//                    memory), each lane keeps its part of the rows' running sums, the maximum is
-//                    raised (and the O rows rescaled in tensor memory) only when a score exceeds it
-//                    by more than 2^8, and the weights P, rounded to the operand type, go to shared
-//                    memory
+//   softmax          an M = 64 product keeps 16 rows in each TMEM lane quarter; a warp reads all
+//                    64 columns of its quarter's rows in the 16x256b shape, so every lane holds
+//                    scores of two rows (a quad of lanes shares a row) and the rows' chunk maxima
+//                    are agreed by shuffles in the quad; the maximum is raised (and the O rows
+//                    rescaled in tensor memory) only when a score exceeds it by more than 2^8, and
+//                    the weights P, rounded to the operand type, go to shared memory
 //   O += P . V       tcgen05.mma per page, M = 64, N = head_dim, K = 16 tokens; A = P, B = the
 //                    staged V page read in place (MN-major)
-// At the item's end each warp writes half of the head_dim outputs of its 16 rows, divided by the
-// rows' sums.  S and O products are issued by two warps of their own, so that neither waits for the
-// other's issue, and complete on mbarriers.  Double buffers keep every stage busy: two S buffers
-// and two P buffers (chunk n's softmax runs while the tensor core works on chunk n - 1's O and
-// chunk n + 1's S), two O buffers (an item's output is read while the next item accumulates), two
-// query buffers and five chunk buffers of 32 KB in flight per SM.
+// Two groups of four softmax warps take the chunks (S products) in turn, so that two chunks are
+// in the softmax at once.  The running maximum stays one sequence per item: the owner of chunk k
+// decides its maxima from those decided for chunk k - 1 (handed over per lane quarter through
+// shared memory and an mbarrier), so every P is relative to the maximum O holds and one O
+// accumulator suffices; each group sums the weights of its own chunks, and the two parts meet at
+// the item's end, where each warp writes half of the head_dim outputs of its 16 rows.  S and O
+// products are issued by two warps of their own, so that neither waits for the other's issue, and
+// complete on mbarriers.  Buffers keep every stage busy: three S buffers, a P buffer per group,
+// two O buffers (an item's output is read while the next item accumulates), two query buffers and
+// five chunk buffers of 32 KB in flight per SM.
 //
 // CTA (one per SM): warps 0-7 run the softmax and the output (warp w on TMEM lane quarter w % 4,
-// columns 32 (w / 4) .. 32 (w / 4) + 31 of each chunk; a quarter without the item's rows skips the
-// arithmetic), warp 8 produces (the work list, TMA for the K/V pages and the query rows), warp 9
-// issues the S products, warp 10 the O products.
+// the chunks whose S product index has the parity of w / 4; a quarter without the item's rows
+// skips the arithmetic), warp 8 produces (the work list, TMA for the K/V pages and the query
+// rows), warp 9 issues the S products, warp 10 the O products.
 // Block size 16, head_dim 128, 16-bit cache and query.
 #pragma once
 
@@ -192,20 +194,22 @@ struct TcCfg {
   static constexpr int OFF_P = OFF_Q + QN * QBUF;
   static constexpr int OFF_BAR = OFF_P + 2 * PBUF;
   // mbarriers: chunk full / empty, query buffer free, S full / free, P full / free (the O product
-  // that read it is done), O buffer free (its item's output has been read), final drain
+  // that read it is done), O buffer free (its item's output has been read), final drain, and per
+  // lane quarter: the running maximum a chunk's owner decided [quarter][chunk parity], the item
+  // sums of the two softmax groups [quarter][item parity]
   static constexpr int NSB = 3;  // S buffers: S products run up to NSB - 1 chunks ahead of the softmax
   static constexpr int B_FULL = 0, B_EMPTY = NCH, B_QFREE = 2 * NCH, B_SFULL = B_QFREE + QN, B_SFREE = B_SFULL + NSB,
                        B_PFULL = B_SFREE + NSB, B_PFREE = B_PFULL + 2, B_OFREE = B_PFREE + 2, B_FIN = B_OFREE + 2,
-                       NBAR = B_FIN + 1;
+                       B_MAX = B_FIN + 1, B_SUM = B_MAX + 8, NBAR = B_SUM + 8;
   static constexpr int OFF_META = OFF_BAR + ((NBAR * 8 + 15) & ~15);
-  // exchange between the two softmax warps of a lane quarter: chunk maxima [NSB S buffers][2 halves][M]
-  // and item sums [2 items][2 halves][M]
+  // exchange between the two softmax warps of a lane quarter: the decided running maxima
+  // [chunk parity][M] and the groups' item sums [item parity][group][M]
   static constexpr int OFF_XCH = OFF_META + NCH * 32;
-  static constexpr int OFF_MISC = OFF_XCH + (2 * NSB + 4) * M * 4;
+  static constexpr int OFF_MISC = OFF_XCH + (2 + 4) * M * 4;
   static constexpr int SMEM_BYTES = 1024 + OFF_MISC + 16;
   // warps 0-7: softmax and output, warp 8 loads, warp 9 issues the S products, warp 10 the O products
   static constexpr int NSM = 256, W_LOAD = 8, W_S = 9, W_O = 10, NTHREADS = NSM + 96;
-  static constexpr int HC = CT / 2;  // chunk columns per softmax warp
+  static constexpr int HC = CT;  // chunk columns per softmax warp: all of them (groups alternate chunks)
   // TMEM columns: two O buffers (head_dim columns each), then NSB S buffers (one chunk each)
   static constexpr uint32_t TM_COLS = 512, TM_O = 0, TM_S = 2 * D;
   static constexpr uint32_t AB = std::is_same<KT, __nv_bfloat16>::value ? 1u : 0u;
@@ -558,20 +562,22 @@ __global__ void __launch_bounds__(TcCfg<KT>::NTHREADS, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
   int4* meta = reinterpret_cast<int4*>(smem + C::OFF_META);
-  float* xmax = reinterpret_cast<float*>(smem + C::OFF_XCH);  // [S buffer][half][M]
-  float* xsum = xmax + 2 * C::NSB * M;                         // [item parity][half][M]
+  float* xmax = reinterpret_cast<float*>(smem + C::OFF_XCH);               // [chunk parity][M]
+  float* xsum = xmax + 2 * M;                                              // [item parity][group][M]
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC + 4);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::NBAR; ++s) {
-      // S free, P full and O free: one arrival per softmax warp; a chunk buffer is free once the
-      // softmax warps and the S warp have read its meta and the O warp has finished with it (or
-      // skipped it); the final drain: one commit per MMA warp
-      const bool sm = (s >= C::B_SFREE && s < C::B_SFREE + C::NSB) || (s >= C::B_PFULL && s < C::B_PFULL + 2) ||
-                      (s >= C::B_OFREE && s < C::B_OFREE + 2);
+      // S free and P full: one arrival per warp of the chunk's softmax group; O free: one per
+      // softmax warp; a chunk buffer is free once the softmax warps and the S warp have read its
+      // meta and the O warp has finished with it (or skipped it); the final drain: one commit per
+      // MMA warp; a decided maximum: its owner warp; item sums: both warps of the quarter
+      const bool grp = (s >= C::B_SFREE && s < C::B_SFREE + C::NSB) || (s >= C::B_PFULL && s < C::B_PFULL + 2);
+      const bool all = s >= C::B_OFREE && s < C::B_OFREE + 2;
       const bool empty = s >= C::B_EMPTY && s < C::B_EMPTY + C::NCH;
-      mbar_init(&bars[s], sm ? C::NSM / 32 : empty ? C::NSM / 32 + 2 : s == C::B_FIN ? 2 : 1);
+      const bool sums = s >= C::B_SUM && s < C::B_SUM + 8;
+      mbar_init(&bars[s], grp ? C::NSM / 64 : all ? C::NSM / 32 : empty ? C::NSM / 32 + 2 : (s == C::B_FIN || sums) ? 2 : 1);
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -601,13 +607,17 @@ __global__ void __launch_bounds__(TcCfg<KT>::NTHREADS, 1)
   }
 
   // ============================== softmax and output (warps 0-7) ==============================
-  // Warp w reads the 16 rows of lane quarter q = w % 4 in the 16x256b shape: lane t holds rows
-  // 16 q + t / 4 and 16 q + t / 4 + 8 at the chunk columns 32 h + 8 j + 2 (t % 4), + 1 (j < 4) of
-  // its half h = w / 4.  The four lanes of a quad share their rows, and the two warps of the
-  // quarter share them through shared memory.
+  // Two groups of four warps take the S products in turn: group g = w / 4 the products whose index
+  // has parity g, so that two chunks are in the softmax at once.  Warp w reads the 16 rows of lane
+  // quarter q = w % 4 in the 16x256b shape: lane t holds rows 16 q + t / 4 and 16 q + t / 4 + 8 at
+  // the chunk columns 8 j + 2 (t % 4), + 1 (j < 8).  A row's running maximum is one sequence over
+  // the item's chunks: the owner of chunk k takes the maximum decided for chunk k - 1 from the
+  // other group's warp of its quarter, decides chunk k's and passes it on (shared memory and a
+  // per-quarter mbarrier), so O keeps one accumulator.  Each group sums its own chunks' weights;
+  // the two parts meet in the item's output.
   constexpr unsigned FULL = 0xffffffffu;
   constexpr float kNone = -1e30f;  // running maximum of a row with no score yet (finite: no NaN from -inf - -inf)
-  constexpr int NJ = HC / 8;       // 8-column blocks of this warp's half chunk
+  constexpr int NJ = HC / 8;       // 8-column blocks of a chunk
   uint64_t* full = bars + C::B_FULL;
   uint64_t* empty = bars + C::B_EMPTY;
   uint64_t* s_full = bars + C::B_SFULL;
@@ -615,9 +625,11 @@ __global__ void __launch_bounds__(TcCfg<KT>::NTHREADS, 1)
   uint64_t* p_full = bars + C::B_PFULL;
   uint64_t* p_free = bars + C::B_PFREE;
   uint64_t* o_free = bars + C::B_OFREE;
+  uint64_t* max_bar = bars + C::B_MAX + 2 * (warp & 3);  // [chunk parity] of this quarter
+  uint64_t* sum_bar = bars + C::B_SUM + 2 * (warp & 3);  // [item parity] of this quarter
   const int ct = threadIdx.x;
-  const int quarter = warp & 3, half = warp >> 2;
-  const int bar_pair = 1 + quarter;
+  const int quarter = warp & 3, grp = warp >> 2;
+  const int gt = ct & 127;                                 // thread of the group
   const int rq = lane >> 2, cq = lane & 3;                 // row in the quarter's first eight, column pair
   const int row0 = quarter * 16 + rq, row1 = row0 + 8;     // this lane's two query rows
   const uint32_t tl = tm + (static_cast<uint32_t>(quarter * 32) << 16);  // the lane quarter (rows in lanes 0-15)
@@ -627,9 +639,11 @@ __global__ void __launch_bounds__(TcCfg<KT>::NTHREADS, 1)
   uint32_t n = 0, ns = 0, np = 0;
   int items = -1;
   bool ok = true;
-  float m0r = kNone, m1r = kNone;  // the rows' running maxima (log2 units)
-  float l0 = 0.f, l1 = 0.f;        // this lane's part of the rows' running sums
+  float mf0 = kNone, mf1 = kNone;  // the maxima this warp decided for the last chunk it took (log2 units)
+  float ml0 = kNone, ml1 = kNone;  // the maxima this group's part of the row sums is relative to
+  float l0 = 0.f, l1 = 0.f;        // this lane's part of the group's row sums
   int ncol = 0, item_t0 = 0, first_np = 0;
+  uint32_t last_k = 0;             // the item's latest S product
   bool poisoned = false, busy = false;  // busy: the quarter holds at least one of the item's rows
 
   // completion of O product k (the P buffer it read is free again)
@@ -637,6 +651,13 @@ __global__ void __launch_bounds__(TcCfg<KT>::NTHREADS, 1)
     const bool done = mbar_wait_bounded(&p_free[k & 1u], (k >> 1) & 1u, kWaitLimit);
     tc_fence_after();
     return done;
+  };
+  // the maxima decided for chunk k, once its owner has passed them on
+  auto read_max = [&](uint32_t k, float& a, float& b) -> bool {
+    const bool got = mbar_wait_bounded(&max_bar[k & 1u], (k >> 1) & 1u, kWaitLimit);
+    a = xmax[(k & 1u) * M + row0];
+    b = xmax[(k & 1u) * M + row1];
+    return got;
   };
 
   while (true) {
@@ -656,7 +677,7 @@ __global__ void __launch_bounds__(TcCfg<KT>::NTHREADS, 1)
       ncol = ((mt0.z >> 16) & 0xff) * G;
       item_t0 = mt1.x;
       busy = quarter * 16 < ncol;
-      m0r = m1r = kNone;
+      ml0 = ml1 = kNone;
       l0 = l1 = 0.f;
       first_np = static_cast<int>(np);
     }
@@ -665,68 +686,80 @@ __global__ void __launch_bounds__(TcCfg<KT>::NTHREADS, 1)
     const uint32_t ob = static_cast<uint32_t>(items) & 1u;
 
     if (!poisoned) {
-      if (ct < CT && ct / C::BS == npg - 1 && (ct & (C::BS - 1)) >= ntok_last) {
-        // V rows past the end of the item may hold anything (even NaN) and would meet zero weights
-        // in the MMA: zero this token's row
-        uint8_t* vrow = cb + 2 * C::KH_BYTES + (npg - 1) * C::VPAGE + (ct & (C::BS - 1)) * 128;
+      const uint32_t k = ns++;  // this chunk's S product (np == k here)
+      last_k = k;
+      if ((k & 1u) == static_cast<uint32_t>(grp)) {
+        if (gt < CT && gt / C::BS == npg - 1 && (gt & (C::BS - 1)) >= ntok_last) {
+          // V rows past the end of the item may hold anything (even NaN) and would meet zero
+          // weights in the MMA: zero this token's row
+          uint8_t* vrow = cb + 2 * C::KH_BYTES + (npg - 1) * C::VPAGE + (gt & (C::BS - 1)) * 128;
 #pragma unroll
-        for (int h = 0; h < 2; ++h)
+          for (int h = 0; h < 2; ++h)
 #pragma unroll
-          for (int q = 0; q < 8; ++q) *reinterpret_cast<uint4*>(vrow + h * C::BOX + q * 16) = make_uint4(0u, 0u, 0u, 0u);
-        fence_proxy_async_smem();
-      }
-      const uint32_t b = ns % C::NSB;
-      bool good = mbar_wait_bounded(&s_full[b], (ns / C::NSB) & 1u, kWaitLimit);
-      tc_fence_after();
-      uint32_t sr[HC / 2];
-      if (busy) {
-        tmem_ld16x256<HC / 2>(tl + C::TM_S + b * CT + half * HC, sr);
-        tc_wait_ld();
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&s_free[b]);
-      ++ns;
+            for (int q = 0; q < 8; ++q) *reinterpret_cast<uint4*>(vrow + h * C::BOX + q * 16) = make_uint4(0u, 0u, 0u, 0u);
+          fence_proxy_async_smem();
+        }
+        const uint32_t b = k % C::NSB;
+        bool good = mbar_wait_bounded(&s_full[b], (k / C::NSB) & 1u, kWaitLimit);
+        tc_fence_after();
+        uint32_t sr[HC / 2];
+        if (busy) {
+          tmem_ld16x256<HC / 2>(tl + C::TM_S + b * CT, sr);
+          tc_wait_ld();
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s_free[b]);
 
-      uint32_t pk[2][NJ];  // this lane's packed weights: [row][block]
-      if (busy) {
         // scores in log2 units, -inf where masked: tokens past the item's end; with several query
         // tokens, row r (query token r / G of the item) sees keys at relative positions <= r / G
         const int ntok = (npg - 1) * C::BS + ntok_last;
         auto jend_of = [&](int r, int rt) {
           return r < ncol ? (CAUSAL && T > 1 ? min(ntok, rt - mt0.w + 1) : ntok) : 0;
         };
-        const int j0 = half * HC + 2 * cq;  // chunk column of this lane's first value
-        const int e0 = jend_of(row0, rt0) - j0, e1 = jend_of(row1, rt1) - j0;  // valid iff 8 j (+1) < e
+        const int e0 = jend_of(row0, rt0) - 2 * cq, e1 = jend_of(row1, rt1) - 2 * cq;  // valid iff 8 j (+1) < e
         float x0 = -CUDART_INF_F, x1 = -CUDART_INF_F;
+        if (busy) {
 #pragma unroll
-        for (int j = 0; j < NJ; ++j) {
-          x0 = fmaxf(x0, fmaxf(8 * j < e0 ? __uint_as_float(sr[4 * j]) : -CUDART_INF_F,
-                               8 * j + 1 < e0 ? __uint_as_float(sr[4 * j + 1]) : -CUDART_INF_F));
-          x1 = fmaxf(x1, fmaxf(8 * j < e1 ? __uint_as_float(sr[4 * j + 2]) : -CUDART_INF_F,
-                               8 * j + 1 < e1 ? __uint_as_float(sr[4 * j + 3]) : -CUDART_INF_F));
+          for (int j = 0; j < NJ; ++j) {
+            x0 = fmaxf(x0, fmaxf(8 * j < e0 ? __uint_as_float(sr[4 * j]) : -CUDART_INF_F,
+                                 8 * j + 1 < e0 ? __uint_as_float(sr[4 * j + 1]) : -CUDART_INF_F));
+            x1 = fmaxf(x1, fmaxf(8 * j < e1 ? __uint_as_float(sr[4 * j + 2]) : -CUDART_INF_F,
+                                 8 * j + 1 < e1 ? __uint_as_float(sr[4 * j + 3]) : -CUDART_INF_F));
+          }
+          x0 = fmaxf(x0, __shfl_xor_sync(FULL, x0, 1));
+          x1 = fmaxf(x1, __shfl_xor_sync(FULL, x1, 1));
+          x0 = fmaxf(x0, __shfl_xor_sync(FULL, x0, 2));
+          x1 = fmaxf(x1, __shfl_xor_sync(FULL, x1, 2));
         }
-        x0 = fmaxf(x0, __shfl_xor_sync(FULL, x0, 1));
-        x1 = fmaxf(x1, __shfl_xor_sync(FULL, x1, 1));
-        x0 = fmaxf(x0, __shfl_xor_sync(FULL, x0, 2));
-        x1 = fmaxf(x1, __shfl_xor_sync(FULL, x1, 2));
-        // the rows' chunk maxima: both halves' (exchanged through shared memory, one buffer per S
-        // buffer: it is rewritten NSB products later, once both warps have passed the barriers of
-        // the products in between -- S products are counted alike in both warps)
-        float* xm = xmax + b * 2 * M;
+        // the maxima decided for chunk k - 1 (always waited for: its owner has then read the
+        // slot this chunk's maxima go to); an item's first chunk starts from none
+        float p0 = kNone, p1 = kNone;
+        if (k > 0) {
+          float a, bb;
+          good = read_max(k - 1, a, bb) && good;
+          if (!first) {
+            p0 = a;
+            p1 = bb;
+          }
+        }
+        x0 *= sl;  // scale > 0 commutes with max
+        x1 *= sl;
+        const bool up0 = x0 > p0 + kRescaleThreshold, up1 = x1 > p1 + kRescaleThreshold;
+        const float n0 = up0 ? x0 : p0, n1 = up1 ? x1 : p1;
         if (cq == 0) {
-          xm[half * M + row0] = x0;
-          xm[half * M + row1] = x1;
+          xmax[(k & 1u) * M + row0] = n0;
+          xmax[(k & 1u) * M + row1] = n1;
         }
-        bar_sync(bar_pair, 64);
-        x0 = fmaxf(x0, xm[(half ^ 1) * M + row0]) * sl;  // scale > 0 commutes with max
-        x1 = fmaxf(x1, xm[(half ^ 1) * M + row1]) * sl;
-        const bool up0 = x0 > m0r + kRescaleThreshold, up1 = x1 > m1r + kRescaleThreshold;
-        const float n0 = up0 ? x0 : m0r, n1 = up1 ? x1 : m1r;
-        const float a0 = up0 ? fast_exp2(m0r - n0) : 1.f, a1 = up1 ? fast_exp2(m1r - n1) : 1.f;  // 0 for a fresh row
-        // O rows that already hold this item's products are rescaled in tensor memory (by the first
-        // half's warp) once the products issued so far are done (warp-wide ld / st: the warp votes)
-        if (half == 0 && __any_sync(FULL, up0 || up1) && static_cast<int>(np) > first_np) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&max_bar[k & 1u]);
+        mf0 = n0;
+        mf1 = n1;
+        // O rows that already hold this item's products (relative to the maxima of chunk k - 1)
+        // are rescaled in tensor memory once the products issued so far are done (warp-wide ld /
+        // st: the warp votes)
+        if (__any_sync(FULL, up0 || up1) && static_cast<int>(np) > first_np) {
+          const float a0 = up0 ? fast_exp2(p0 - n0) : 1.f, a1 = up1 ? fast_exp2(p1 - n1) : 1.f;
           good = wait_o(np - 1) && good;
 #pragma unroll
           for (int h = 0; h < D / 32; ++h) {  // 32 columns of the O rows per pass
@@ -739,77 +772,88 @@ __global__ void __launch_bounds__(TcCfg<KT>::NTHREADS, 1)
           }
           tc_wait_st();
         }
-        m0r = n0;
-        m1r = n1;
-        l0 *= a0;
-        l1 *= a1;
+        // this group's part of the sums follows the maxima (0 from none)
+        if (n0 > ml0) l0 *= fast_exp2(ml0 - n0);
+        if (n1 > ml1) l1 *= fast_exp2(ml1 - n1);
+        ml0 = n0;
+        ml1 = n1;
         // the weights the MMA sees; the sums are taken over the same rounded values
-        float s0 = 0.f, s1 = 0.f;
+        uint32_t pk[2][NJ];
+        if (busy) {
+          float s0 = 0.f, s1 = 0.f;
 #pragma unroll
-        for (int j = 0; j < NJ; ++j) {
-          const float w0 = 8 * j < e0 ? fast_exp2(fmaf(__uint_as_float(sr[4 * j]), sl, -m0r)) : 0.f;
-          const float w1 = 8 * j + 1 < e0 ? fast_exp2(fmaf(__uint_as_float(sr[4 * j + 1]), sl, -m0r)) : 0.f;
-          const float w2 = 8 * j < e1 ? fast_exp2(fmaf(__uint_as_float(sr[4 * j + 2]), sl, -m1r)) : 0.f;
-          const float w3 = 8 * j + 1 < e1 ? fast_exp2(fmaf(__uint_as_float(sr[4 * j + 3]), sl, -m1r)) : 0.f;
-          pk[0][j] = pack2<KT>(w0, w1);
-          pk[1][j] = pack2<KT>(w2, w3);
-          const float2 r0 = unpack2<KT>(pk[0][j]), r1 = unpack2<KT>(pk[1][j]);
-          s0 += r0.x + r0.y;
-          s1 += r1.x + r1.y;
+          for (int j = 0; j < NJ; ++j) {
+            const float w0 = 8 * j < e0 ? fast_exp2(fmaf(__uint_as_float(sr[4 * j]), sl, -n0)) : 0.f;
+            const float w1 = 8 * j + 1 < e0 ? fast_exp2(fmaf(__uint_as_float(sr[4 * j + 1]), sl, -n0)) : 0.f;
+            const float w2 = 8 * j < e1 ? fast_exp2(fmaf(__uint_as_float(sr[4 * j + 2]), sl, -n1)) : 0.f;
+            const float w3 = 8 * j + 1 < e1 ? fast_exp2(fmaf(__uint_as_float(sr[4 * j + 3]), sl, -n1)) : 0.f;
+            pk[0][j] = pack2<KT>(w0, w1);
+            pk[1][j] = pack2<KT>(w2, w3);
+            const float2 r0 = unpack2<KT>(pk[0][j]), r1 = unpack2<KT>(pk[1][j]);
+            s0 += r0.x + r0.y;
+            s1 += r1.x + r1.y;
+          }
+          l0 += s0;
+          l1 += s1;
         }
-        l0 += s0;
-        l1 += s1;
-      }
-      // the P buffer is free once O(np - 2) is done
-      if (np >= 2) good = wait_o(np - 2) && good;
-      if (!__all_sync(FULL, good)) {
-        ok = false;
-        break;
-      }
-      {  // K-major A operand: row r at r * 128, 16-byte chunk q at ((q ^ (r & 7)) << 4); this lane's
-         // pair of columns is 4 bytes at 4 (t % 4) in chunk (32 h + 8 j) / 8.  Rows of a quarter
-         // without the item's rows get zero weights (their products are not read).
-        uint8_t* pb = smem + C::OFF_P + (np & 1u) * C::PBUF;
+        // this group's P buffer is free once O(k - 2) is done
+        if (np >= 2) good = wait_o(np - 2) && good;
+        if (!__all_sync(FULL, good)) {
+          ok = false;
+          break;
+        }
+        {  // K-major A operand: row r at r * 128, 16-byte chunk q at ((q ^ (r & 7)) << 4); this lane's
+           // pair of columns is 4 bytes at 4 (t % 4) in chunk j.  Rows of a quarter without the
+           // item's rows get zero weights (their products are not read).
+          uint8_t* pb = smem + C::OFF_P + (np & 1u) * C::PBUF;
 #pragma unroll
-        for (int j = 0; j < NJ; ++j) {
-          const int qc = half * NJ + j;
-          *reinterpret_cast<uint32_t*>(pb + row0 * 128 + ((qc ^ (row0 & 7)) << 4) + 4 * cq) = busy ? pk[0][j] : 0u;
-          *reinterpret_cast<uint32_t*>(pb + row1 * 128 + ((qc ^ (row1 & 7)) << 4) + 4 * cq) = busy ? pk[1][j] : 0u;
+          for (int j = 0; j < NJ; ++j) {
+            *reinterpret_cast<uint32_t*>(pb + row0 * 128 + ((j ^ (row0 & 7)) << 4) + 4 * cq) = busy ? pk[0][j] : 0u;
+            *reinterpret_cast<uint32_t*>(pb + row1 * 128 + ((j ^ (row1 & 7)) << 4) + 4 * cq) = busy ? pk[1][j] : 0u;
+          }
         }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&p_full[np & 1u]);
       }
-      fence_proxy_async_smem();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&p_full[np & 1u]);
       ++np;
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[c]);  // this warp is done with the chunk's meta and V rows
 
     if (last) {
-      // output of the item: each warp writes its half of the head_dim columns of its 16 rows
+      // output of the item: each warp writes its group's half of the head_dim columns of its 16 rows
       const bool o_any = static_cast<int>(np) > first_np;
       bool good = true;
-      if (!poisoned && o_any) good = wait_o(np - 1);
-      if (!__all_sync(FULL, good)) {
-        ok = false;
-        break;
+      float fin0 = mf0, fin1 = mf1;  // the maxima decided for the item's last chunk
+      if (!poisoned && o_any) {
+        good = wait_o(np - 1);
+        if ((last_k & 1u) != static_cast<uint32_t>(grp)) good = read_max(last_k, fin0, fin1) && good;
       }
       const bool bad = poisoned || !o_any;
-      // the rows' sums: the quad's parts, then both halves' (one buffer per item parity: every item,
-      // poisoned or not, ends with this barrier, so a buffer is rewritten only after both warps
-      // have read it)
+      // the rows' sums: this group's (the quad's parts, brought to the final maxima), then both
+      // groups' (one buffer per item parity: every item, poisoned or not, ends with this exchange,
+      // so a buffer is rewritten only after both warps have read it)
       l0 += __shfl_xor_sync(FULL, l0, 1);
       l1 += __shfl_xor_sync(FULL, l1, 1);
       l0 += __shfl_xor_sync(FULL, l0, 2);
       l1 += __shfl_xor_sync(FULL, l1, 2);
-      float* xs = xsum + (items & 1) * 2 * M;
+      const float g0 = bad ? 0.f : l0 * fast_exp2(ml0 - fin0), g1 = bad ? 0.f : l1 * fast_exp2(ml1 - fin1);
+      const uint32_t ip = static_cast<uint32_t>(items) & 1u;
+      float* xs = xsum + ip * 2 * M;
       if (cq == 0) {
-        xs[half * M + row0] = l0;
-        xs[half * M + row1] = l1;
+        xs[grp * M + row0] = g0;
+        xs[grp * M + row1] = g1;
       }
-      bar_sync(bar_pair, 64);
-      const float lt0 = l0 + xs[(half ^ 1) * M + row0], lt1 = l1 + xs[(half ^ 1) * M + row1];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sum_bar[ip]);
+      good = mbar_wait_bounded(&sum_bar[ip], (static_cast<uint32_t>(items) >> 1) & 1u, kWaitLimit) && good;
+      if (!__all_sync(FULL, good)) {
+        ok = false;
+        break;
+      }
+      const float lt0 = g0 + xs[(grp ^ 1) * M + row0], lt1 = g1 + xs[(grp ^ 1) * M + row1];
       if (busy) {
         const int seq = mt0.x, part = mt0.y & 0xffff, kvh = mt0.z & 0xff;
         const bool direct = (flags & F_DIRECT) != 0;
@@ -819,7 +863,7 @@ __global__ void __launch_bounds__(TcCfg<KT>::NTHREADS, 1)
 #pragma unroll
         for (int i = 0; i < 2; ++i) {
           const int r = i ? row1 : row0;
-          const float lt = i ? lt1 : lt0, mr = i ? m1r : m0r;
+          const float lt = i ? lt1 : lt0, mr = i ? fin1 : fin0;
           live[i] = r < ncol;
           const int mq = i ? rt1 : rt0, g = r - mq * G;
           const int mb = T > 1 ? 0 : mq, t = T > 1 ? item_t0 + mq : 0;
@@ -831,13 +875,13 @@ __global__ void __launch_bounds__(TcCfg<KT>::NTHREADS, 1)
             const int64_t pidx = static_cast<int64_t>(seq + mb) * p.max_parts + part;
             ofs[i] = (pidx * HV + vh) * D;
             fs[i] = bad ? CUDART_NAN_F : p.v_scale;
-            if (live[i] && half == 0 && cq == 0)
+            if (live[i] && grp == 0 && cq == 0)
               __stcg(&p.part_ml[pidx * HV + vh], bad ? make_float2(0.f, CUDART_NAN_F) : make_float2(mr, lt));
           }
         }
 #pragma unroll
         for (int h2 = 0; h2 < 2; ++h2) {  // this warp's 64 columns, 32 per pass
-          const int col0 = half * 64 + h2 * 32;
+          const int col0 = grp * 64 + h2 * 32;
           uint32_t ov[16];
           if (!bad) {
             tmem_ld16x256_x4(tl + C::TM_O + ob * D + col0, ov);
