@@ -194,13 +194,13 @@ struct TcCfg {
   static constexpr int OFF_P = OFF_Q + QN * QBUF;
   static constexpr int OFF_BAR = OFF_P + 2 * PBUF;
   // mbarriers: chunk full / empty, query buffer free, S full / free, P full / free (the O product
-  // that read it is done), O buffer free (its item's output has been read), final drain, and per
-  // lane quarter: the running maximum a chunk's owner decided [quarter][chunk parity], the item
-  // sums of the two softmax groups [quarter][item parity]
+  // that read it is done), O buffer free (its item's output has been read), final drain, per lane
+  // quarter: the running maximum a chunk's owner decided [quarter][chunk parity], the item sums of
+  // the two softmax groups [quarter][item parity]; and chunk meta written (before its copies land)
   static constexpr int NSB = 3;  // S buffers: S products run up to NSB - 1 chunks ahead of the softmax
   static constexpr int B_FULL = 0, B_EMPTY = NCH, B_QFREE = 2 * NCH, B_SFULL = B_QFREE + QN, B_SFREE = B_SFULL + NSB,
                        B_PFULL = B_SFREE + NSB, B_PFREE = B_PFULL + 2, B_OFREE = B_PFREE + 2, B_FIN = B_OFREE + 2,
-                       B_MAX = B_FIN + 1, B_SUM = B_MAX + 8, NBAR = B_SUM + 8;
+                       B_MAX = B_FIN + 1, B_SUM = B_MAX + 8, B_META = B_SUM + 8, NBAR = B_META + NCH;
   static constexpr int OFF_META = OFF_BAR + ((NBAR * 8 + 15) & ~15);
   // exchange between the two softmax warps of a lane quarter: the decided running maxima
   // [chunk parity][M] and the groups' item sums [item parity][group][M]
@@ -350,6 +350,7 @@ __device__ __forceinline__ void tc_produce(const DecodeParams& p, const CUtensor
           mbar_arrive(&full[c]);
         else
           mbar_arrive_expect_tx(&full[c], static_cast<uint32_t>(npg * 2 * C::VPAGE) + (cc == 0 ? qbytes : 0u));
+        mbar_arrive(&bars[C::B_META + c]);  // roles that need only the meta go ahead
       }
       __syncwarp();  // the expected byte count is set before any copy can complete
       if (!bad) {
@@ -382,6 +383,7 @@ __device__ __forceinline__ void tc_produce(const DecodeParams& p, const CUtensor
       if (lane == 0) {
         meta[2 * c] = make_int4(0, 0, F_END << 24, 0);
         mbar_arrive(&full[c]);
+        mbar_arrive(&bars[C::B_META + c]);
       }
     } else {
       stop = true;
@@ -485,7 +487,7 @@ __device__ __forceinline__ void tc_mma_o(uint8_t* smem, uint64_t* bars, const in
                                          uint32_t tm, int lane) {
   constexpr unsigned FULL = 0xffffffffu;
   constexpr int D = C::D;
-  uint64_t* full = bars + C::B_FULL;
+  uint64_t* meta_ready = bars + C::B_META;  // P full implies the chunk's copies landed (its S read them)
   uint64_t* empty = bars + C::B_EMPTY;
   uint64_t* p_full = bars + C::B_PFULL;
   uint64_t* p_free = bars + C::B_PFREE;
@@ -495,7 +497,7 @@ __device__ __forceinline__ void tc_mma_o(uint8_t* smem, uint64_t* bars, const in
   bool item_bad = false, ok = true;
   for (uint32_t k = 0;; ++k) {
     const int c = static_cast<int>(k % C::NCH);
-    const bool ready = mbar_wait_bounded(&full[c], (k / C::NCH) & 1u, kWaitLimit);
+    const bool ready = mbar_wait_bounded(&meta_ready[c], (k / C::NCH) & 1u, kWaitLimit);
     if (!__all_sync(FULL, ready && !*abort_flag)) {
       ok = false;
       break;
@@ -619,6 +621,7 @@ __global__ void __launch_bounds__(TcCfg<KT>::NTHREADS, 1)
   constexpr float kNone = -1e30f;  // running maximum of a row with no score yet (finite: no NaN from -inf - -inf)
   constexpr int NJ = HC / 8;       // 8-column blocks of a chunk
   uint64_t* full = bars + C::B_FULL;
+  uint64_t* meta_ready = bars + C::B_META;
   uint64_t* empty = bars + C::B_EMPTY;
   uint64_t* s_full = bars + C::B_SFULL;
   uint64_t* s_free = bars + C::B_SFREE;
@@ -662,7 +665,7 @@ __global__ void __launch_bounds__(TcCfg<KT>::NTHREADS, 1)
 
   while (true) {
     const int c = static_cast<int>(n % C::NCH);
-    const bool ready = mbar_wait_bounded(&full[c], (n / C::NCH) & 1u, kWaitLimit);
+    const bool ready = mbar_wait_bounded(&meta_ready[c], (n / C::NCH) & 1u, kWaitLimit);
     if (!__all_sync(FULL, ready && !*abort_flag)) {
       ok = false;
       break;
@@ -689,6 +692,8 @@ __global__ void __launch_bounds__(TcCfg<KT>::NTHREADS, 1)
       const uint32_t k = ns++;  // this chunk's S product (np == k here)
       last_k = k;
       if ((k & 1u) == static_cast<uint32_t>(grp)) {
+        bool good = true;
+        if (ntok_last < C::BS) good = mbar_wait_bounded(&full[c], (n / C::NCH) & 1u, kWaitLimit);  // copies landed
         if (gt < CT && gt / C::BS == npg - 1 && (gt & (C::BS - 1)) >= ntok_last) {
           // V rows past the end of the item may hold anything (even NaN) and would meet zero
           // weights in the MMA: zero this token's row
@@ -700,7 +705,7 @@ __global__ void __launch_bounds__(TcCfg<KT>::NTHREADS, 1)
           fence_proxy_async_smem();
         }
         const uint32_t b = k % C::NSB;
-        bool good = mbar_wait_bounded(&s_full[b], (k / C::NSB) & 1u, kWaitLimit);
+        good = mbar_wait_bounded(&s_full[b], (k / C::NSB) & 1u, kWaitLimit) && good;
         tc_fence_after();
         uint32_t sr[HC / 2];
         if (busy) {
