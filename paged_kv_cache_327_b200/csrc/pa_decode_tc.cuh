@@ -132,6 +132,13 @@ __device__ __forceinline__ void tmem_st16x256(uint32_t taddr, const uint32_t (&v
 }
 
 // ---------------------------------------------------------------- helpers
+// four 8x8 matrices of 16-bit elements to shared memory: register i of thread t holds row t / 4,
+// columns 2 (t % 4) and + 1 of matrix i; threads 8 i .. 8 i + 7 give the addresses of its 8 rows
+__device__ __forceinline__ void stsm_x4(uint32_t addr, uint32_t r0, uint32_t r1, uint32_t r2, uint32_t r3) {
+  asm volatile("stmatrix.sync.aligned.m8n8.x4.shared.b16 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(r0), "r"(r1),
+               "r"(r2), "r"(r3)
+               : "memory");
+}
 // named barrier of the consumer warps, reducing a predicate (each warp reconverges first: the
 // barrier instructions are warp-aligned)
 __device__ __forceinline__ bool bar_and(bool v, int id, int nthreads) {
@@ -722,16 +729,26 @@ __global__ void __launch_bounds__(TcCfg<KT>::NTHREADS, 1)
         auto jend_of = [&](int r, int rt) {
           return r < ncol ? (CAUSAL && T > 1 ? min(ntok, rt - mt0.w + 1) : ntok) : 0;
         };
-        const int e0 = jend_of(row0, rt0) - 2 * cq, e1 = jend_of(row1, rt1) - 2 * cq;  // valid iff 8 j (+1) < e
+        const int je0 = jend_of(row0, rt0), je1 = jend_of(row1, rt1);
+        const int e0 = je0 - 2 * cq, e1 = je1 - 2 * cq;  // valid iff 8 j (+1) < e
+        // the usual chunk: every row of the warp sees all its columns (no mask to apply)
+        const bool whole = __all_sync(FULL, je0 >= CT && je1 >= CT);
         float x0 = -CUDART_INF_F, x1 = -CUDART_INF_F;
-        if (busy) {
+        auto chunk_max = [&](auto masked) {
+          constexpr bool MK = decltype(masked)::value;
 #pragma unroll
           for (int j = 0; j < NJ; ++j) {
-            x0 = fmaxf(x0, fmaxf(8 * j < e0 ? __uint_as_float(sr[4 * j]) : -CUDART_INF_F,
-                                 8 * j + 1 < e0 ? __uint_as_float(sr[4 * j + 1]) : -CUDART_INF_F));
-            x1 = fmaxf(x1, fmaxf(8 * j < e1 ? __uint_as_float(sr[4 * j + 2]) : -CUDART_INF_F,
-                                 8 * j + 1 < e1 ? __uint_as_float(sr[4 * j + 3]) : -CUDART_INF_F));
+            x0 = fmaxf(x0, fmaxf(!MK || 8 * j < e0 ? __uint_as_float(sr[4 * j]) : -CUDART_INF_F,
+                                 !MK || 8 * j + 1 < e0 ? __uint_as_float(sr[4 * j + 1]) : -CUDART_INF_F));
+            x1 = fmaxf(x1, fmaxf(!MK || 8 * j < e1 ? __uint_as_float(sr[4 * j + 2]) : -CUDART_INF_F,
+                                 !MK || 8 * j + 1 < e1 ? __uint_as_float(sr[4 * j + 3]) : -CUDART_INF_F));
           }
+        };
+        if (busy) {
+          if (whole)
+            chunk_max(std::false_type{});
+          else
+            chunk_max(std::true_type{});
           x0 = fmaxf(x0, __shfl_xor_sync(FULL, x0, 1));
           x1 = fmaxf(x1, __shfl_xor_sync(FULL, x1, 1));
           x0 = fmaxf(x0, __shfl_xor_sync(FULL, x0, 2));
@@ -784,14 +801,15 @@ __global__ void __launch_bounds__(TcCfg<KT>::NTHREADS, 1)
         ml1 = n1;
         // the weights the MMA sees; the sums are taken over the same rounded values
         uint32_t pk[2][NJ];
-        if (busy) {
+        auto chunk_weights = [&](auto masked) {
+          constexpr bool MK = decltype(masked)::value;
           float s0 = 0.f, s1 = 0.f;
 #pragma unroll
           for (int j = 0; j < NJ; ++j) {
-            const float w0 = 8 * j < e0 ? fast_exp2(fmaf(__uint_as_float(sr[4 * j]), sl, -n0)) : 0.f;
-            const float w1 = 8 * j + 1 < e0 ? fast_exp2(fmaf(__uint_as_float(sr[4 * j + 1]), sl, -n0)) : 0.f;
-            const float w2 = 8 * j < e1 ? fast_exp2(fmaf(__uint_as_float(sr[4 * j + 2]), sl, -n1)) : 0.f;
-            const float w3 = 8 * j + 1 < e1 ? fast_exp2(fmaf(__uint_as_float(sr[4 * j + 3]), sl, -n1)) : 0.f;
+            const float w0 = !MK || 8 * j < e0 ? fast_exp2(fmaf(__uint_as_float(sr[4 * j]), sl, -n0)) : 0.f;
+            const float w1 = !MK || 8 * j + 1 < e0 ? fast_exp2(fmaf(__uint_as_float(sr[4 * j + 1]), sl, -n0)) : 0.f;
+            const float w2 = !MK || 8 * j < e1 ? fast_exp2(fmaf(__uint_as_float(sr[4 * j + 2]), sl, -n1)) : 0.f;
+            const float w3 = !MK || 8 * j + 1 < e1 ? fast_exp2(fmaf(__uint_as_float(sr[4 * j + 3]), sl, -n1)) : 0.f;
             pk[0][j] = pack2<KT>(w0, w1);
             pk[1][j] = pack2<KT>(w2, w3);
             const float2 r0 = unpack2<KT>(pk[0][j]), r1 = unpack2<KT>(pk[1][j]);
@@ -800,6 +818,15 @@ __global__ void __launch_bounds__(TcCfg<KT>::NTHREADS, 1)
           }
           l0 += s0;
           l1 += s1;
+        };
+        if (busy) {
+          if (whole)
+            chunk_weights(std::false_type{});
+          else
+            chunk_weights(std::true_type{});
+        } else {
+#pragma unroll
+          for (int j = 0; j < NJ; ++j) pk[0][j] = pk[1][j] = 0u;  // rows without the item's rows: zero weights
         }
         // this group's P buffer is free once O(k - 2) is done
         if (np >= 2) good = wait_o(np - 2) && good;
@@ -807,15 +834,17 @@ __global__ void __launch_bounds__(TcCfg<KT>::NTHREADS, 1)
           ok = false;
           break;
         }
-        {  // K-major A operand: row r at r * 128, 16-byte chunk q at ((q ^ (r & 7)) << 4); this lane's
-           // pair of columns is 4 bytes at 4 (t % 4) in chunk j.  Rows of a quarter without the
-           // item's rows get zero weights (their products are not read).
-          uint8_t* pb = smem + C::OFF_P + (np & 1u) * C::PBUF;
+        {  // K-major A operand: row r at r * 128, 16-byte chunk j (columns 8 j .. 8 j + 7) at
+           // ((j ^ (r & 7)) << 4).  The warp's 16 rows x 64 columns are 16 matrices of 8 x 8 in the
+           // fragment layout of pk (rows 0-7 in pk[0], 8-15 in pk[1]): four stmatrix.x4, the i-th
+           // taking blocks 2 i and 2 i + 1; lane l gives row l % 8 of matrix l / 8 (rows + 8 for odd
+           // l / 8, block + 1 for l / 8 >= 2).
+          const int mrow = quarter * 16 + ((lane >> 3) & 1) * 8 + (lane & 7);
+          const uint32_t rbase = smem_u32(smem + C::OFF_P + (np & 1u) * C::PBUF) + mrow * 128;
+          const int jsel = lane >> 4, rx = lane & 7;
 #pragma unroll
-          for (int j = 0; j < NJ; ++j) {
-            *reinterpret_cast<uint32_t*>(pb + row0 * 128 + ((j ^ (row0 & 7)) << 4) + 4 * cq) = busy ? pk[0][j] : 0u;
-            *reinterpret_cast<uint32_t*>(pb + row1 * 128 + ((j ^ (row1 & 7)) << 4) + 4 * cq) = busy ? pk[1][j] : 0u;
-          }
+          for (int i = 0; i < NJ / 2; ++i)
+            stsm_x4(rbase + (((2 * i + jsel) ^ rx) << 4), pk[0][2 * i], pk[1][2 * i], pk[0][2 * i + 1], pk[1][2 * i + 1]);
         }
         fence_proxy_async_smem();
         tc_fence_before();
