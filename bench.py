@@ -74,7 +74,7 @@ def parse_args():
     ap.add_argument("--prefix", action="store_true",
                     help="prefix-aware decode (pa_decode_prefix): sequences sharing their first blocks read them "
                          "once; the groups come from the block tables")
-    ap.add_argument("--wide-kernel", choices=["mma", "tcgen05"], default="mma",
+    ap.add_argument("--wide-kernel", choices=["auto", "mma", "tcgen05"], default="auto",
                     help="kernel for items of more than 8 query rows per KV head (--qtok, --prefix): the warp-MMA "
                          "kernel (default) or the 5th-generation tensor-core kernel")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -168,13 +168,28 @@ def sources_digest():
     return h.hexdigest()[:16]
 
 
-def profile_name(args) -> str:
+def wide_kernel_used(w, wide: str, max_members: int = 1):
+    """The kernel the library runs for this workload's wide items (None: items of at most 8 query
+    rows, which run on the decode kernel): the rule of include/pa.h's PA_OPT_WIDE_KERNEL."""
+    rows = w.num_q_tokens * max_members * (w.num_q_heads // w.num_kv_heads)
+    if rows <= 8:
+        return None
+    tc_shape = (w.head_dim == 128 and w.block_size == 16 and w.kv_dtype in ("bf16", "f16")
+                and w.q_dtype == w.kv_dtype)
+    if tc_shape and (wide == "tcgen05" or (wide == "auto" and rows > 32)):
+        return "tcgen05"
+    return "mma"
+
+
+def profile_name(args, kernel=None) -> str:
     """Name of the committed ncu summary of this run's partition kernel: config, cache dtype and
-    query tokens (pa_decode_partition_8b, pa_decode_partition_8b_e4m3, pa_decode_partition_8b_T5)."""
+    query tokens (pa_decode_partition_8b, pa_decode_partition_8b_e4m3, pa_decode_partition_8b_T5),
+    with _tcgen05 when the wide items run on the tensor-core kernel (`kernel`, else the flag)."""
+    kernel = kernel or getattr(args, "wide_kernel", "mma")
     return (f"pa_decode_partition_{args.config}" + (f"_{args.kv_dtype}" if args.kv_dtype else "")
             + (f"_T{args.qtok}" if args.qtok > 1 else "") + ("_fork" if getattr(args, "step", None) == "fork" else "")
             + ("_prefix" if args.prefix else "")
-            + ("_tcgen05" if getattr(args, "wide_kernel", "mma") == "tcgen05" else ""))
+            + ("_tcgen05" if kernel == "tcgen05" else ""))
 
 
 def recorded_traffic(name: str):
@@ -344,6 +359,8 @@ PATHS = [
     ("8b_T5", dict(config="8b", qtok=5)),
     ("8b_T8", dict(config="8b", qtok=8)),
     ("8b_T16", dict(config="8b", qtok=16)),
+    ("8b_T16_mma", dict(config="8b", qtok=16, wide_kernel="mma")),
+    ("8b_T8_tcgen05", dict(config="8b", qtok=8, wide_kernel="tcgen05")),
     ("8b_T5_bs32", dict(config="8b", qtok=5, block_size=32)),
     ("70b_prefix", dict(config="70b", prefix=True)),
     ("70b", dict(config="70b")),
@@ -358,11 +375,21 @@ def measure_path(args, overrides: dict, calls: int = 200, warm: int = 10) -> dic
     back-to-back decode calls (inputs larger than L2), as GB/s of algorithmic bytes (distinct
     K+V, q, out, tables) and as a fraction of the measured HBM peak."""
     from paged_kv_cache_327_b200 import binding as B
-    from paged_kv_cache_327_b200 import block_manager as BM
 
     a = argparse.Namespace(**{**vars(args), "block_size": None, "kv_dtype": None, "qtok": 1, "prefix": False,
                               "step": None, "uniform_lens": None, **overrides})
     w = make_workload(a)
+    B.set_wide_kernel(a.wide_kernel)  # a path may name its own wide-item kernel
+    try:
+        return _measure_path(a, w, calls, warm)
+    finally:
+        B.set_wide_kernel(args.wide_kernel)
+
+
+def _measure_path(a, w, calls, warm) -> dict:
+    from paged_kv_cache_327_b200 import binding as B
+    from paged_kv_cache_327_b200 import block_manager as BM
+
     dw = B.device_workload(w)
     ws = B.DecodeWorkspace.for_workload(dw)
     out = torch.empty(tuple(dw.q.shape), dtype=B._NAME_TORCH[w.q_dtype], device="cuda")
@@ -397,7 +424,9 @@ def measure_path(args, overrides: dict, calls: int = 200, warm: int = 10) -> dic
     peak, _ = measured_peak()
     gbs = nbytes / (ms * 1e-3) / 1e9
     res = {"ms": round(ms, 5), "achieved_gbs": round(gbs, 1), "frac": round(gbs / peak, 4),
-           "algorithmic_bytes": int(nbytes), "seq_tokens_per_s": round(w.total_tokens() / (ms * 1e-3), 1)}
+           "algorithmic_bytes": int(nbytes), "seq_tokens_per_s": round(w.total_tokens() / (ms * 1e-3), 1),
+           "wide_kernel": wide_kernel_used(w, a.wide_kernel,
+                                           B.max_prefix_members(w.num_q_heads, w.num_kv_heads) if a.prefix else 1)}
     del dw, ws, out
     torch.cuda.empty_cache()
     return res
@@ -439,6 +468,7 @@ def run_ours(args):
         groups_np = BM.find_prefix_groups(w.block_tables, w.seq_lens, w.block_size)
     groups = torch.from_numpy(groups_np).to(f"cuda:{local}")
     max_members = B.max_prefix_members(w.num_q_heads, w.num_kv_heads)
+    wide_used = wide_kernel_used(w, args.wide_kernel, max_members if args.prefix else 1)
 
     kv_bytes = w.kv_bytes_logical()
     # with shared prefix blocks a physical byte is read once per sharer but fetched from HBM
@@ -654,7 +684,7 @@ def run_ours(args):
                    "cow_pairs_per_step": int(len(w.copy_pairs)), "out_dtype": out_dtype,
                    "step": w.notes.get("step"),
                    "partition_size": args.partition_size or 512,
-                   "wide_kernel": args.wide_kernel if (w.num_q_tokens > 1 or args.prefix) else None,
+                   "wide_kernel": (f"{args.wide_kernel} ({wide_used})" if wide_used else None),
                    "prefix_groups": (f"{len(groups_np)} groups, {int(groups_np[:, 1].sum())} sequences, shared "
                                      f"tokens {sorted(set(int(x) for x in groups_np[:, 2]))}, max_members "
                                      f"{max_members}") if args.prefix else None,
@@ -669,7 +699,7 @@ def run_ours(args):
                           "the copies of neighbouring steps overlap a step's kernels (two copy streams, "
                           "double-buffered device inputs and outputs)"},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
-                     "frac": round(achieved / peak, 4), "traffic": recorded_traffic(profile_name(args)),
+                     "frac": round(achieved / peak, 4), "traffic": recorded_traffic(profile_name(args, wide_used or "mma")),
                      "kernel": ("pa_decode_prefix" if args.prefix else
                                 "pa_decode_multi" if w.num_q_tokens > 1 else "pa_decode")
                                + " call (plan + partition + merge kernels)",

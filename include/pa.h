@@ -138,8 +138,10 @@ PA_API int pa_decode_fp8(void* out, const void* q, const void* k_cache, const vo
  *   are NaN and pa_get_device_error reports PA_DEV_BAD_SEQ_LEN).
  *   supported: q_dtype == kv_dtype (f16 or bf16) for num_q_tokens > 1 (num_q_tokens 1: every
  *   dtype pair of pa_decode), num_q_tokens up to 65536.  A work item holds up to 32 query rows
- *   (query tokens x grouped heads) per KV head, 8 with head_dim 64: with more query tokens, the
- *   tokens are split into column groups and each K/V page is read once per group.
+ *   (query tokens x grouped heads) per KV head on the warp-MMA kernel, 64 on the tensor-core
+ *   kernel (head_dim 128, block_size 16; see PA_OPT_WIDE_KERNEL), 8 with head_dim 64: with more
+ *   query tokens, the tokens are split into column groups and each K/V page is read once per
+ *   group.
  *   Everything else as pa_decode; the
  *   workspace is pa_decode_workspace_size(num_seqs, num_q_tokens * num_q_heads, head_dim,
  *   max_blocks_per_seq * block_size, partition_size).  num_q_tokens 1 is pa_decode. */
@@ -167,8 +169,9 @@ PA_API int pa_decode_multi(void* out, const void* q, const void* k_cache, const 
  *                  block-table entries differ inside the shared tokens get NaN rows and the
  *                  same error.
  *   max_members    members one shared pass serves (larger groups are split): max_members * G
- *                  query rows per KV head, at most 32; above 8 rows only with head_dim 128 and
- *                  q_dtype == kv_dtype (f16 or bf16).
+ *                  query rows per KV head, at most 32 (64 where the tensor-core kernel takes the
+ *                  call: block_size 16 and the PA_OPT_WIDE_KERNEL rule); above 8 rows only with
+ *                  head_dim 128 and q_dtype == kv_dtype (f16 or bf16).
  * Caches f16 or bf16; everything else, the workspace included, as pa_decode.  num_groups 0 is
  * pa_decode. */
 PA_API int pa_decode_prefix(void* out, const void* q, const void* k_cache, const void* v_cache,
@@ -251,19 +254,25 @@ PA_API int pa_selftest_wait_timeout(int polls, void* stream);
 /* Process-wide options.
  *
  * PA_OPT_WIDE_KERNEL chooses the kernel for work items of more than 8 query rows per KV head (the
- * query tokens of pa_decode_multi, or the members of a pa_decode_prefix group) on a 16-bit cache
- * with head_dim 128 and block_size 16:
- *   PA_WIDE_MMA (default)  the persistent warp-MMA kernel: two consumer warps per ring share
- *                          each staged page;
- *   PA_WIDE_TCGEN05        the 5th-generation tensor-core kernel: chunks of 8 pages, S^T = K.Q^T
- *                          and O^T += V^T.P^T accumulate in tensor memory, one loading warp, one
- *                          MMA-issuing warp and four softmax warps per CTA.
- * Both match the same oracle within the attention tolerances; on B200 the first is the faster
- * of the two for every shape measured.  Other paths ignore the option.
+ * query tokens of pa_decode_multi times the grouped heads, or the members of a pa_decode_prefix
+ * group times the grouped heads) on a 16-bit cache with a query of its own type, head_dim 128 and
+ * block_size 16:
+ *   PA_WIDE_AUTO (default) the tensor-core kernel for calls whose rows per KV head exceed 32 (the
+ *                          warp-MMA kernel would split them into column groups and read every
+ *                          K/V page once per group), the warp-MMA kernel otherwise;
+ *   PA_WIDE_MMA            always the persistent warp-MMA kernel (items of up to 32 rows: two
+ *                          consumer warps per ring share each staged page);
+ *   PA_WIDE_TCGEN05        always the 5th-generation tensor-core kernel (items of up to 64 rows:
+ *                          S = Q.K^T and O += P.V accumulate in tensor memory over chunks of 4
+ *                          pages; one loading warp, two MMA-issuing warps and two groups of four
+ *                          softmax warps that take the chunks in turn).
+ * All three match the same oracle within the attention tolerances.  Other shapes and paths ignore
+ * the option.
  * Returns PA_OK, or PA_ERR_INVALID for an unknown option or value (nothing changes then). */
 #define PA_OPT_WIDE_KERNEL 1
 #define PA_WIDE_MMA 0
 #define PA_WIDE_TCGEN05 1
+#define PA_WIDE_AUTO 2
 PA_API int pa_set_option(int option, int value);
 
 /* ABI version of this header (major * 100 + minor). */

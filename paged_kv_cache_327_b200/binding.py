@@ -301,7 +301,7 @@ def pa_selftest_wait_timeout(polls: int, stream=None) -> None:
 
 
 PA_OPT_WIDE_KERNEL = 1
-WIDE_KERNELS = {"mma": 0, "tcgen05": 1}
+WIDE_KERNELS = {"mma": 0, "tcgen05": 1, "auto": 2}
 
 
 def pa_set_option(option: int, value: int) -> None:
@@ -310,7 +310,8 @@ def pa_set_option(option: int, value: int) -> None:
 
 
 def set_wide_kernel(name: str) -> None:
-    """Kernel for items of more than 8 query rows per KV head: "mma" (default) or "tcgen05"."""
+    """Kernel for items of more than 8 query rows per KV head: "auto" (default: tcgen05 for items of
+    more than 32 rows, the warp-MMA kernel below that), "mma" or "tcgen05"."""
     if name not in WIDE_KERNELS:
         raise ValueError(f"wide kernel must be one of {sorted(WIDE_KERNELS)}, not {name!r}")
     pa_set_option(PA_OPT_WIDE_KERNEL, WIDE_KERNELS[name])

@@ -199,7 +199,7 @@ int launch_partition(const pa::DecodeParams& p, const CUtensorMap& tmk, const CU
 
 // The tensor-core kernel for wide items (block size 16, head_dim 128, 16-bit cache and query).
 // kernel for items of more than 8 query rows (PA_OPT_WIDE_KERNEL)
-std::atomic<int> g_wide_kernel{PA_WIDE_MMA};
+std::atomic<int> g_wide_kernel{PA_WIDE_AUTO};
 
 template <typename KT>
 int launch_tc(const pa::DecodeParams& p, const CUtensorMap& tmk, const CUtensorMap& tmv, const CUtensorMap& tmq,
@@ -295,7 +295,7 @@ int dispatch_kv(const pa::DecodeParams& p, const CUtensorMap& tmk, const CUtenso
 extern "C" {
 
 int pa_set_option(int option, int value) {
-  if (option == PA_OPT_WIDE_KERNEL && (value == PA_WIDE_MMA || value == PA_WIDE_TCGEN05)) {
+  if (option == PA_OPT_WIDE_KERNEL && (value == PA_WIDE_MMA || value == PA_WIDE_TCGEN05 || value == PA_WIDE_AUTO)) {
     g_wide_kernel.store(value, std::memory_order_relaxed);
     return PA_OK;
   }
@@ -349,10 +349,16 @@ int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cac
   // several query tokens: a 16-bit cache with a query of the same type
   if (qtok > 1 && (kv_dtype == PA_FP8_E4M3 || q_dtype != kv_dtype)) return PA_ERR_UNSUPPORTED;
   if (qtok > 65536 || static_cast<int64_t>(qtok) * num_q_heads * head_dim > INT_MAX) return PA_ERR_UNSUPPORTED;
-  // items of more than 8 query rows run on the tensor-core kernel when it is chosen (block size 16,
-  // head_dim 128, a 16-bit cache with a query of its own type): it holds up to 64 rows per item
-  const bool tc_ok = g_wide_kernel.load(std::memory_order_relaxed) == PA_WIDE_TCGEN05 && head_dim == 128 &&
-                     block_size == 16 && (kv_dtype == PA_F16 || kv_dtype == PA_BF16) && q_dtype == kv_dtype;
+  // items of more than 8 query rows may run on the tensor-core kernel (block size 16, head_dim 128,
+  // a 16-bit cache with a query of its own type), which holds up to 64 rows per item: when it is
+  // chosen, or by default when the rows per KV head exceed what the warp-MMA kernel's items hold
+  // (that kernel would split the query tokens into column groups and read every page once per group)
+  const int wide = g_wide_kernel.load(std::memory_order_relaxed);
+  const bool tc_shape = head_dim == 128 && block_size == 16 && (kv_dtype == PA_F16 || kv_dtype == PA_BF16) &&
+                        q_dtype == kv_dtype;
+  const int64_t rows_wanted = static_cast<int64_t>(qtok) * max_members * G;
+  const bool tc_ok = tc_shape && (wide == PA_WIDE_TCGEN05 ||
+                                  (wide == PA_WIDE_AUTO && rows_wanted > max_item_rows(head_dim)));
   const int max_rows = tc_ok ? kTcMaxRows : max_item_rows(head_dim);
   // query tokens per item: all of them, or column groups of up to max_rows query rows per KV head
   // (8 with head_dim 64, whose items run on the one-consumer kernels)

@@ -154,7 +154,15 @@ def test_prefix_argument_validation(lib):
     assert prefix_call(lib, mm=0) == B.PA_ERR_INVALID
     assert prefix_call(lib, groups=0) == B.PA_ERR_INVALID          # groups promised, none given
     assert prefix_call(lib, ng=5) == B.PA_ERR_INVALID              # more groups than sequences
-    assert prefix_call(lib, mm=5) == B.PA_ERR_UNSUPPORTED           # 5 members x 8 heads > 32 rows
+    # 5 members x 8 heads = 40 rows: beyond the warp-MMA kernel's 32, within the tensor-core
+    # kernel's 64 (which the default option takes for it); 9 members: beyond both
+    assert prefix_call(lib, mm=5) == B.PA_ERR_WORKSPACE
+    assert prefix_call(lib, mm=9) == B.PA_ERR_UNSUPPORTED
+    B.set_wide_kernel("mma")
+    try:
+        assert prefix_call(lib, mm=5) == B.PA_ERR_UNSUPPORTED
+    finally:
+        B.set_wide_kernel("auto")
     assert prefix_call(lib, kd=3) == B.PA_ERR_UNSUPPORTED           # FP8 cache
     assert prefix_call(lib, qd=0) == B.PA_ERR_UNSUPPORTED           # 32 rows need q_dtype == kv_dtype
     assert prefix_call(lib, Hq=512, Hkv=256) == B.PA_ERR_UNSUPPORTED  # more than 255 KV heads
@@ -172,16 +180,18 @@ def test_selftest_argument_checks(lib):
 
 
 def test_set_option(lib):
-    """The wide-kernel option takes its two values and rejects others (no GPU needed)."""
+    """The wide-kernel option takes its three values and rejects others (no GPU needed)."""
     assert lib.pa_set_option(B.PA_OPT_WIDE_KERNEL, 1) == B.PA_OK
     assert lib.pa_set_option(B.PA_OPT_WIDE_KERNEL, 0) == B.PA_OK
-    assert lib.pa_set_option(B.PA_OPT_WIDE_KERNEL, 2) == B.PA_ERR_INVALID
+    assert lib.pa_set_option(B.PA_OPT_WIDE_KERNEL, 2) == B.PA_OK
+    assert lib.pa_set_option(B.PA_OPT_WIDE_KERNEL, 3) == B.PA_ERR_INVALID
     assert lib.pa_set_option(B.PA_OPT_WIDE_KERNEL, -1) == B.PA_ERR_INVALID
     assert lib.pa_set_option(0, 0) == B.PA_ERR_INVALID
     with pytest.raises(ValueError):
         B.set_wide_kernel("wgmma")
     B.set_wide_kernel("tcgen05")
     B.set_wide_kernel("mma")
+    B.set_wide_kernel("auto")
 
 
 def test_workspace_reserves_every_work_item(lib):
@@ -192,13 +202,13 @@ def test_workspace_reserves_every_work_item(lib):
     includes the shapes whose column groups hold only 5 to 8 query rows (head_dim 64, few KV
     heads), the worst case for the reservation."""
     checked = 0
-    for wide in ("mma", "tcgen05"):  # the tensor-core kernel's items hold up to 64 rows
+    for wide in ("mma", "tcgen05", "auto"):  # the tensor-core kernel's items hold up to 64 rows
         B.set_wide_kernel(wide)
         try:
             checked += _reservation_grid(lib)
         finally:
-            B.set_wide_kernel("mma")
-    assert checked == 2 * 6192
+            B.set_wide_kernel("auto")
+    assert checked == 3 * 6192
 
 
 def _reservation_grid(lib):

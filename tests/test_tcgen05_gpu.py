@@ -2,7 +2,8 @@
 
 Items of more than 8 query rows per KV head (several query tokens, or the members of a shared
 prefix) on a 16-bit cache with head_dim 128 and block size 16 run on this kernel once
-pa_set_option(PA_OPT_WIDE_KERNEL, PA_WIDE_TCGEN05) is called.  An item holds up to 64 query rows
+pa_set_option(PA_OPT_WIDE_KERNEL, PA_WIDE_TCGEN05) is called, and by default (PA_WIDE_AUTO) when a
+call's rows per KV head exceed the warp-MMA kernel's 32.  An item holds up to 64 query rows
 (the M of its products); wider sequences are split into column groups.  The cases mirror the
 warp-MMA kernel's: 12..64 query rows, column groups, short partitions (two chunks of 4 pages) and
 long ones (several chunks, a ragged last chunk and page), empty sequences, causal tails, shared
@@ -30,7 +31,7 @@ def _tcgen05_kernel():
     B.load_library()
     B.set_wide_kernel("tcgen05")
     yield
-    B.set_wide_kernel("mma")
+    B.set_wide_kernel("auto")
 
 
 MULTI = [
@@ -146,3 +147,25 @@ def test_prefix_64_rows():
     assert B.pa_get_device_error() == B.PA_DEV_OK
     _, ref = TP.oracle_decode(w, kc, vc)
     TP.assert_close(out.float().cpu().numpy(), ref, "bf16", "f32", "64-row shared passes")
+
+
+@pytest.mark.parametrize("T,kernel", [(16, "tcgen05"), (8, "mma")])
+def test_default_option_picks_by_rows(T, kernel):
+    """PA_WIDE_AUTO (the default) runs items of more than 32 query rows per KV head (8B shapes:
+    4 grouped heads, so T = 16 gives 64 rows) on the tensor-core kernel and narrower ones on the
+    warp-MMA kernel: its result is bit-identical to the kernel it picks (both are deterministic)."""
+    w = W.make_config("8b", num_seqs=48, num_q_tokens=T)
+    dw, _ = TM.gpu_multi(w)  # the step's tokens are stored
+    ws = B.DecodeWorkspace.for_workload(dw)
+    outs = {}
+    try:
+        for mode in ("auto", kernel):
+            B.set_wide_kernel(mode)
+            o = torch.empty(tuple(dw.q.shape), dtype=torch.float32, device="cuda")
+            B.pa_decode_multi(o, dw.q, dw.k_cache, dw.v_cache, dw.block_tables, dw.seq_lens, w.scale, ws.tensor)
+            outs[mode] = o
+    finally:
+        B.set_wide_kernel("tcgen05")
+    torch.cuda.synchronize()
+    assert B.pa_get_device_error() == B.PA_DEV_OK
+    assert torch.equal(outs["auto"], outs[kernel])
