@@ -1033,11 +1033,70 @@ __global__ void __launch_bounds__(32) pa_selftest_wait_kernel(uint32_t polls) {
 // ------------------------------------------------------------------------------ merge
 // One warp per (sequence, virtual head = query token x query head) of a sequence whose items
 // wrote partial results (shared partitions first, then its own):
-// out = sum_k 2^(m_k - M) O_k / sum_k 2^(m_k - M) l_k, M = max_k m_k, partitions in order (a
-// fixed interleaved order for sequences of more than kMergeSplit partitions).
+// out = sum_k 2^(m_k - M) O_k / sum_k 2^(m_k - M) l_k, M = max_k m_k, taken in one pass over the
+// partitions in order: a running maximum, with the numerator and denominator relative to it
+// rescaled whenever a later partition raises it (the same quotient).  The loads of kMergeBatch
+// partitions are in flight at once; each lane holds head_dim / 32 consecutive columns.
 constexpr int kMergeWarps = 8;
-constexpr int kMergeSplit = 16;  // above this many partitions a warp merges four at a time
-__global__ void __launch_bounds__(kMergeWarps * 32) pa_decode_merge_kernel(const DecodeParams p) {
+constexpr int kMergeBatch = 4;
+
+__device__ __forceinline__ float neg_inf() { return -CUDART_INF_F; }
+
+template <int V>  // columns per lane
+struct MergeRow {
+  float m, den, num[V];
+  __device__ __forceinline__ MergeRow() : m(neg_inf()), den(0.f) {
+#pragma unroll
+    for (int j = 0; j < V; ++j) num[j] = 0.f;
+  }
+  // partition k: (maximum, sum, this lane's columns of the unnormalised output).  A partition in
+  // which the row saw no key is (-inf, 0, 0) and adds nothing; a poisoned one carries NaN.
+  __device__ __forceinline__ void add(float mk, float lk, const float (&a)[V]) {
+    if (mk == neg_inf()) return;
+    if (mk > m) {
+      const float r = fast_exp2(m - mk);  // 0 while nothing has been added (m = -inf)
+      den *= r;
+#pragma unroll
+      for (int j = 0; j < V; ++j) num[j] *= r;
+      m = mk;
+    }
+    const float w = fast_exp2(mk - m);
+    den += w * lk;
+#pragma unroll
+    for (int j = 0; j < V; ++j) num[j] += w * a[j];
+  }
+};
+
+template <int V>
+__device__ __forceinline__ void merge_row(const DecodeParams& p, int64_t base, int np, int64_t vrow, int HV,
+                                          int64_t o, int lane) {
+  using VT = typename std::conditional<V == 4, float4, float2>::type;
+  constexpr int D = 32 * V;
+  MergeRow<V> acc;
+  for (int k0 = 0; k0 < np; k0 += kMergeBatch) {
+    float2 ml[kMergeBatch];
+    float a[kMergeBatch][V];
+#pragma unroll
+    for (int u = 0; u < kMergeBatch; ++u) {
+      if (k0 + u < np) {
+        const int64_t row = (base + k0 + u) * HV + vrow;
+        ml[u] = __ldcg(&p.part_ml[row]);
+        const VT x = __ldcg(reinterpret_cast<const VT*>(p.part_acc + row * D) + lane);
+        const float* xf = reinterpret_cast<const float*>(&x);
+#pragma unroll
+        for (int j = 0; j < V; ++j) a[u][j] = xf[j];
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kMergeBatch; ++u)
+      if (k0 + u < np) acc.add(ml[u].x, ml[u].y, a[u]);
+  }
+  const float inv = 1.f / acc.den;
+#pragma unroll
+  for (int j = 0; j < V; ++j) store_out(p.out, o + lane * V + j, acc.num[j] * inv, p.out_dtype);
+}
+
+__global__ void __launch_bounds__(kMergeWarps * 32, 4) pa_decode_merge_kernel(const DecodeParams p) {
   pdl_wait();  // the partition kernel's partial results are visible from here on
   const int lane = threadIdx.x & 31;
   const int64_t pair = static_cast<int64_t>(blockIdx.x) * kMergeWarps + (threadIdx.x >> 5);
@@ -1052,86 +1111,18 @@ __global__ void __launch_bounds__(kMergeWarps * 32) pa_decode_merge_kernel(const
   } else {
     np = p.seq_parts[seq];
   }
+  const int64_t o = (static_cast<int64_t>(seq) * Hq + hq) * D;
   if (np < 0) {  // no work item: the row is zero (empty sequence) or NaN (invalid length)
     const float v = np == kPartsEmpty ? 0.f : CUDART_NAN_F;
-    const int64_t o = (static_cast<int64_t>(seq) * Hq + hq) * D;
     for (int d = lane; d < D; d += 32) store_out(p.out, o + d, v, p.out_dtype);
     return;
   }
   if (np == 0) return;  // written directly by the sequence's only item
   const int64_t base = static_cast<int64_t>(seq) * p.max_parts;
-  float M = -CUDART_INF_F;
-  for (int k = lane; k < np; k += 32) M = fmaxf(M, __ldcg(&p.part_ml[(base + k) * Hq + hq].x));
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-  float num[4] = {0.f, 0.f, 0.f, 0.f}, den = 0.f;
-  const int per = D >> 5;  // 2 or 4 elements per lane
-  if (np > kMergeSplit) {
-    // many partitions: four groups of 8 lanes take every fourth partition, a lane holding D / 8
-    // consecutive elements, so that several partitions are in flight; the groups' sums are added
-    // in a fixed order
-    const int grp = lane >> 3, cl = lane & 7, nv = D >> 5;  // float4 per lane
-    float4 acc4[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) acc4[j] = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 2
-    for (int k = grp; k < np; k += 4) {
-      const float2 ml = __ldcg(&p.part_ml[(base + k) * Hq + hq]);
-      const float4* src = reinterpret_cast<const float4*>(p.part_acc + ((base + k) * Hq + hq) * D) + cl * nv;
-      float4 a[4];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) a[j] = j < nv ? __ldcg(src + j) : make_float4(0.f, 0.f, 0.f, 0.f);
-      const float w = fast_exp2(ml.x - M);
-      den += w * ml.y;
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        acc4[j].x += w * a[j].x;
-        acc4[j].y += w * a[j].y;
-        acc4[j].z += w * a[j].z;
-        acc4[j].w += w * a[j].w;
-      }
-    }
-#pragma unroll
-    for (int o = 8; o < 32; o <<= 1) {
-      den += __shfl_xor_sync(0xffffffffu, den, o);
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        acc4[j].x += __shfl_xor_sync(0xffffffffu, acc4[j].x, o);
-        acc4[j].y += __shfl_xor_sync(0xffffffffu, acc4[j].y, o);
-        acc4[j].z += __shfl_xor_sync(0xffffffffu, acc4[j].z, o);
-        acc4[j].w += __shfl_xor_sync(0xffffffffu, acc4[j].w, o);
-      }
-    }
-    if (grp != 0) return;
-    const float inv = 1.f / den;
-    const int64_t o = (static_cast<int64_t>(seq) * Hq + hq) * D + cl * nv * 4;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      if (j >= nv) break;
-      store_out(p.out, o + 4 * j + 0, acc4[j].x * inv, p.out_dtype);
-      store_out(p.out, o + 4 * j + 1, acc4[j].y * inv, p.out_dtype);
-      store_out(p.out, o + 4 * j + 2, acc4[j].z * inv, p.out_dtype);
-      store_out(p.out, o + 4 * j + 3, acc4[j].w * inv, p.out_dtype);
-    }
-    return;
-  }
-#pragma unroll 4
-  for (int k = 0; k < np; ++k) {
-    const float2 ml = __ldcg(&p.part_ml[(base + k) * Hq + hq]);
-    const float* src = p.part_acc + ((base + k) * Hq + hq) * D + lane;
-    float a[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) a[j] = j < per ? __ldcg(src + 32 * j) : 0.f;
-    const float w = fast_exp2(ml.x - M);
-    den += w * ml.y;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) num[j] += w * a[j];
-  }
-  const float inv = 1.f / den;
-  const int64_t o = (static_cast<int64_t>(seq) * Hq + hq) * D + lane;
-#pragma unroll
-  for (int j = 0; j < 4; ++j)
-    if (j < per) store_out(p.out, o + 32 * j, num[j] * inv, p.out_dtype);
+  if (D == 128)
+    merge_row<4>(p, base, np, hq, Hq, o, lane);
+  else
+    merge_row<2>(p, base, np, hq, Hq, o, lane);
 }
 
 }  // namespace pa
