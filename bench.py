@@ -858,7 +858,10 @@ def run_cache(args):
                    "l2": "256 MB written before every timed launch"},
         "ops": ops,
         "roofline": {"bound": "hbm", "kernel": main_op, "achieved": m["achieved_gbs"], "peak": peak, "unit": "GB/s",
-                     "frac": m["frac"], "traffic": None, "peak_source": peak_src},
+                     "frac": m["frac"],
+                     "traffic": recorded_traffic(f"pa_{main_op}_{args.config}" + (f"_{args.kv_dtype}" if fp8 else "")
+                                                 + (f"_{args.step}" if args.step else "")),
+                     "peak_source": peak_src},
         "gpu_launches": 2 * reps * len(ops),
     }
     print(json.dumps(line), flush=True)
