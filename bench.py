@@ -188,8 +188,18 @@ def profile_name(args, kernel=None) -> str:
     kernel = kernel or getattr(args, "wide_kernel", "mma")
     return (f"pa_decode_partition_{args.config}" + (f"_{args.kv_dtype}" if args.kv_dtype else "")
             + (f"_T{args.qtok}" if args.qtok > 1 else "") + ("_fork" if getattr(args, "step", None) == "fork" else "")
-            + ("_prefix" if args.prefix else "")
+            + ("_prefix" if args.prefix else "") + resized_suffix(args)
             + ("_tcgen05" if kernel == "tcgen05" else ""))
+
+
+def resized_suffix(args) -> str:
+    """A resized workload (sequences, lengths, block or partition size) has a summary of its own
+    name, so it never takes the full-size summary's traffic."""
+    lens = getattr(args, "uniform_lens", None)
+    return ((f"_n{args.num_seqs}" if getattr(args, "num_seqs", None) else "")
+            + (f"_u{lens.replace(',', '-')}" if lens else "")
+            + (f"_bs{args.block_size}" if getattr(args, "block_size", None) else "")
+            + (f"_p{args.partition_size}" if getattr(args, "partition_size", 0) else ""))
 
 
 def recorded_traffic(name: str):
@@ -860,7 +870,7 @@ def run_cache(args):
         "roofline": {"bound": "hbm", "kernel": main_op, "achieved": m["achieved_gbs"], "peak": peak, "unit": "GB/s",
                      "frac": m["frac"],
                      "traffic": recorded_traffic(f"pa_{main_op}_{args.config}" + (f"_{args.kv_dtype}" if fp8 else "")
-                                                 + (f"_{args.step}" if args.step else "")),
+                                                 + (f"_{args.step}" if args.step else "") + resized_suffix(args)),
                      "peak_source": peak_src},
         "gpu_launches": 2 * reps * len(ops),
     }

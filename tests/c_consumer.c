@@ -37,13 +37,20 @@ int main(void) {
                   PA_BF16, 0, fake, 100, NULL) == PA_ERR_WORKSPACE);
   CHECK(pa_decode_multi(fake, fake, fake, fake, ifake, ifake, 4, 0, 32, 8, 128, 16, 0.088f, 512, 1000, PA_BF16,
                         PA_BF16, PA_BF16, 0, fake, 0, NULL) == PA_ERR_INVALID); /* no query tokens */
+  /* 5 members x 8 heads = 40 rows: the default option takes the tensor-core kernel (up to 64 rows),
+     so the call passes the row check and stops at the missing workspace; the warp-MMA kernel
+     holds 32 rows and refuses it */
   CHECK(pa_decode_prefix(fake, fake, fake, fake, ifake, ifake, 4, 64, 8, 128, 16, 0.088f, 512, 1000, PA_BF16,
-                         PA_BF16, PA_BF16, 0, ifake, 1, 5, fake, 0, NULL) == PA_ERR_UNSUPPORTED); /* 40 rows */
+                         PA_BF16, PA_BF16, 0, ifake, 1, 5, fake, 0, NULL) == PA_ERR_WORKSPACE);
+  CHECK(pa_set_option(PA_OPT_WIDE_KERNEL, PA_WIDE_MMA) == PA_OK);
+  CHECK(pa_decode_prefix(fake, fake, fake, fake, ifake, ifake, 4, 64, 8, 128, 16, 0.088f, 512, 1000, PA_BF16,
+                         PA_BF16, PA_BF16, 0, ifake, 1, 5, fake, 0, NULL) == PA_ERR_UNSUPPORTED);
   CHECK(pa_copy_blocks(fake, fake, ifake, 1, 10, 4008, NULL, NULL) == PA_ERR_INVALID); /* not 16-byte units */
   CHECK(pa_selftest_wait_timeout(0, NULL) == PA_ERR_INVALID);
-  /* the wide-item kernel option: its two values, nothing else */
+  /* the wide-item kernel option: its three values, nothing else */
   CHECK(pa_set_option(PA_OPT_WIDE_KERNEL, PA_WIDE_TCGEN05) == PA_OK);
   CHECK(pa_set_option(PA_OPT_WIDE_KERNEL, PA_WIDE_MMA) == PA_OK);
+  CHECK(pa_set_option(PA_OPT_WIDE_KERNEL, PA_WIDE_AUTO) == PA_OK);
   CHECK(pa_set_option(PA_OPT_WIDE_KERNEL, 7) == PA_ERR_INVALID);
   CHECK(pa_set_option(99, PA_WIDE_MMA) == PA_ERR_INVALID);
   puts("ok");

@@ -26,6 +26,10 @@ def test_profile_names():
     assert bench.profile_name(args(kv_dtype="e4m3")) == "pa_decode_partition_8b_e4m3"
     assert bench.profile_name(args(config="70b", prefix=True)) == "pa_decode_partition_70b_prefix"
     assert bench.profile_name(args(qtok=4, wide_kernel="tcgen05")) == "pa_decode_partition_8b_T4_tcgen05"
+    assert bench.profile_name(args(qtok=16), "tcgen05") == "pa_decode_partition_8b_T16_tcgen05"
+    # a resized workload never takes the full-size summary's traffic
+    assert bench.profile_name(args(num_seqs=4096, uniform_lens="0,40")) == "pa_decode_partition_8b_n4096_u0-40"
+    assert bench.profile_name(args(block_size=32)) == "pa_decode_partition_8b_bs32"
 
 
 def test_every_summary_has_traffic_and_digest():
