@@ -92,6 +92,8 @@ struct DecodeParams {
   // first .. first + members - 1 hold the same blocks for their first `shared` tokens
   const int32_t* groups;
   int num_groups, max_members;  // a shared item covers at most max_members sequences
+  int shared_partition;  // tokens of a shared item when there are many (a multiple of block_size)
+  int rings;             // page pipelines of the partition kernel (CTAs x rings per CTA)
   float scale_log2;  // scale * log2(e) (* k_scale for an FP8 cache)
   float v_scale;     // multiplies the output (FP8 cache); 1 otherwise
   // workspace views
@@ -287,6 +289,17 @@ __global__ void __launch_bounds__(kPlanThreads) pa_decode_plan_kernel(const Deco
 
   // column groups: the qtok query tokens of a sequence are split into items of qtok_item tokens
   const int Tc = p.qtok_item, ncg = (p.qtok + Tc - 1) / Tc;
+  // Shared items take P tokens each, or shared_partition tokens when, at P, they would outnumber
+  // the page pipelines four to one: fewer partial results per member for the merge, with the
+  // parallelism still ample.  The choice is block-uniform.
+  int Ps = P;
+  if (p.num_groups > 0 && p.shared_partition > P) {
+    long long loc = 0, tot;
+    for (int i = lo; i < hi; ++i)
+      if (valid_len(p.seq_lens[i]) && p.seq_sub[i] > 0) loc += (p.seq_shared[i] + P - 1) / P;
+    (void)block_exclusive_scan<long long>(loc, 0, ScanSum{}, s_warp, &tot);
+    if (tot * p.num_kv_heads >= 4LL * p.rings) Ps = p.shared_partition;
+  }
   struct Counts {
     int L, S, sub, ns, nf, nt, nps;
   };
@@ -296,7 +309,7 @@ __global__ void __launch_bounds__(kPlanThreads) pa_decode_plan_kernel(const Deco
     if (!valid_len(c.L)) return c;
     c.S = p.num_groups > 0 ? p.seq_shared[i] : 0;
     c.sub = p.num_groups > 0 ? p.seq_sub[i] : 0;
-    c.nps = (c.S + P - 1) / P;
+    c.nps = (c.S + Ps - 1) / Ps;
     c.ns = c.sub > 0 ? c.nps : 0;
     c.nf = (c.L - c.S) / P;
     c.nt = ((c.L - c.S) % P) ? 1 : 0;
@@ -329,7 +342,7 @@ __global__ void __launch_bounds__(kPlanThreads) pa_decode_plan_kernel(const Deco
     const int dflag = (c.S == 0 && c.nf + c.nt == 1) ? WI_DIRECT : 0;
     // shared items have one query token (prefix groups are single-token decode)
     for (int k = 0; k < c.ns; ++k)
-      p.items[os++] = WorkItem{i, k * P, min(c.S, (k + 1) * P), k | (c.sub << 16), 0, 1, 0, 0};
+      p.items[os++] = WorkItem{i, k * Ps, min(c.S, (k + 1) * Ps), k | (c.sub << 16), 0, 1, 0, 0};
     for (int k = 0; k < c.nf; ++k)
       for (int j = 0; j < ncg; ++j)
         p.items[n_shared + of++] = WorkItem{i, c.S + k * P, c.S + (k + 1) * P, (c.nps + k) | (1 << 16) | dflag,
@@ -489,16 +502,22 @@ __device__ __forceinline__ void produce(const DecodeParams& p, const CUtensorMap
     // key positions relative to the item's first query token, at position len - T + t0
     // (causal masking of several query tokens)
     const int rel0 = T > 1 ? tok0 - (p.seq_lens[it.seq] - T + t0) : 0;
-    int bt = 0;
+    // the item's block-table entries, one per lane for each 32-page window (items of up to 64
+    // pages; all of them are checked before the first page goes out)
     bool bad = false, mismatch = false;
-    if (lane < npages) {
-      const int64_t col = tok0 / BS + lane;
-      bt = p.block_tables[static_cast<int64_t>(it.seq) * p.max_blocks_per_seq + col];
-      bad = bt < 0 || bt >= p.num_blocks;
-      // the members of a shared item must hold the same blocks
-      for (int m = 1; m < members; ++m)
-        mismatch |= p.block_tables[static_cast<int64_t>(it.seq + m) * p.max_blocks_per_seq + col] != bt;
-    }
+    auto entry = [&](int pgi) -> int {
+      int v = 0;
+      if (pgi < npages) {
+        const int64_t col = tok0 / BS + pgi;
+        v = p.block_tables[static_cast<int64_t>(it.seq) * p.max_blocks_per_seq + col];
+        bad |= v < 0 || v >= p.num_blocks;
+        // the members of a shared item must hold the same blocks
+        for (int m = 1; m < members; ++m)
+          mismatch |= p.block_tables[static_cast<int64_t>(it.seq + m) * p.max_blocks_per_seq + col] != v;
+      }
+      return v;
+    };
+    const int bt = entry(lane), bt2 = entry(lane + 32);
     bad = __any_sync(FULL, bad);
     mismatch = __any_sync(FULL, mismatch);
     if (lane == 0) {
@@ -515,7 +534,7 @@ __device__ __forceinline__ void produce(const DecodeParams& p, const CUtensorMap
       }
     }
     for (int pg = 0; pg < npages; ++pg) {
-      const int phys = __shfl_sync(FULL, bt, pg);
+      const int phys = __shfl_sync(FULL, pg < 32 ? bt : bt2, pg & 31);
       const int slot = static_cast<int>(n % C::NSLOT);
       if (!acquire_slot(slot)) {
         stop = true;

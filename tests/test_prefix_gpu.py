@@ -179,3 +179,37 @@ def test_large_group_beside_many_small_groups():
     assert B.pa_get_device_error() == B.PA_DEV_OK
     _, ref = oracle_decode(w, kc, vc)
     assert_close(out.float().cpu().numpy(), ref, "bf16", "f32", "large group")
+
+
+def test_long_shared_items_check_every_page():
+    """Many groups (160 pairs sharing 1040 tokens, 8 KV heads) make the plan take shared items of
+    1024 tokens: 64 pages, whose block-table entries the producer reads in two windows of 32.  A
+    member whose table differs from its leader's only in the second window (page 40) poisons its
+    group's item (NaN rows, PA_DEV_BAD_PREFIX); every other row matches the oracle."""
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    groups = [W.Group(1040, [1, 1]) for _ in range(160)]
+    w = W.build_groups("long", groups, num_q_heads=32, num_kv_heads=8, head_dim=128, block_size=16, q_dtype="bf16",
+                       kv_dtype="bf16", seed=5600)
+    pg = BM.find_prefix_groups(w.block_tables, w.seq_lens, 16)
+    assert len(pg) == 160 and (pg[:, 2] == 1040).all()
+    # at 512 tokens the shared items would outnumber the partition kernel's page pipelines four to one
+    assert 160 * 3 * 8 >= 4 * 4 * sms
+    # member 1 of group 0 reads a different (valid) block at page 40 of the shared tokens
+    s0, s1 = int(pg[0, 0]), int(pg[0, 0]) + 1
+    other = int(w.block_tables[int(pg[1, 0]), 3])
+    w.block_tables[s1, 40] = other
+    dw, kc, vc = stepped(w)
+    out = prefix_decode(w, dw, pg, 8)
+    assert B.pa_get_device_error() == B.PA_DEV_BAD_PREFIX
+    got = out.float().cpu().numpy()
+    assert np.isnan(got[s0]).all() and np.isnan(got[s1]).all()
+    rest = [i for i in range(w.num_seqs) if i not in (s0, s1)]
+    _, ref = oracle_decode(w, kc, vc, rest)
+    assert_close(got[rest], ref, "bf16", "f32", "groups with consistent tables")
+    # the same batch without the inconsistency: every row matches
+    w.block_tables[s1, 40] = w.block_tables[s0, 40]
+    dw, kc, vc = stepped(w)
+    out = prefix_decode(w, dw, pg, 8)
+    assert B.pa_get_device_error() == B.PA_DEV_OK
+    _, ref = oracle_decode(w, kc, vc)
+    assert_close(out.float().cpu().numpy(), ref, "bf16", "f32", "long shared items")
