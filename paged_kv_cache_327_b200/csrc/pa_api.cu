@@ -438,9 +438,9 @@ int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cac
   p.groups = groups;
   p.num_groups = num_groups;
   p.max_members = max_members;
-  // shared items of twice the partition (up to the 64 pages a warp-MMA producer takes per item)
+  // shared items of up to four partitions (and the 128 pages a warp-MMA producer takes per item)
   // where the plan finds many of them; the tensor-core kernel's producer takes 32 pages per item
-  p.shared_partition = use_tc ? P : std::min(2 * P, 64 * block_size);
+  p.shared_partition = use_tc ? P : std::min(4 * P, 128 * block_size);
   p.rings = info->sm_count * 4;  // one CTA per SM, 4 rings each (prefix groups are 16-bit)
   const bool fp8 = kv_dtype == PA_FP8_E4M3;
   p.scale_log2 = scale * (fp8 ? k_scale : 1.f) * 1.4426950408889634f;

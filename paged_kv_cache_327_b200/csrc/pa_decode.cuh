@@ -289,16 +289,18 @@ __global__ void __launch_bounds__(kPlanThreads) pa_decode_plan_kernel(const Deco
 
   // column groups: the qtok query tokens of a sequence are split into items of qtok_item tokens
   const int Tc = p.qtok_item, ncg = (p.qtok + Tc - 1) / Tc;
-  // Shared items take P tokens each, or shared_partition tokens when, at P, they would outnumber
-  // the page pipelines four to one: fewer partial results per member for the merge, with the
-  // parallelism still ample.  The choice is block-uniform.
+  // Shared items take m P tokens each: m = 1, or more (up to shared_partition / P) while the
+  // shared items, counted at P, still number at least 2 m times the page pipelines -- fewer
+  // partial results per member for the merge, with the parallelism still ample.  The choice is
+  // block-uniform.
   int Ps = P;
   if (p.num_groups > 0 && p.shared_partition > P) {
     long long loc = 0, tot;
     for (int i = lo; i < hi; ++i)
       if (valid_len(p.seq_lens[i]) && p.seq_sub[i] > 0) loc += (p.seq_shared[i] + P - 1) / P;
     (void)block_exclusive_scan<long long>(loc, 0, ScanSum{}, s_warp, &tot);
-    if (tot * p.num_kv_heads >= 4LL * p.rings) Ps = p.shared_partition;
+    const long long m = min(static_cast<long long>(p.shared_partition / P), tot * p.num_kv_heads / (2LL * p.rings));
+    if (m > 1) Ps = static_cast<int>(m) * P;
   }
   struct Counts {
     int L, S, sub, ns, nf, nt, nps;
@@ -502,7 +504,7 @@ __device__ __forceinline__ void produce(const DecodeParams& p, const CUtensorMap
     // key positions relative to the item's first query token, at position len - T + t0
     // (causal masking of several query tokens)
     const int rel0 = T > 1 ? tok0 - (p.seq_lens[it.seq] - T + t0) : 0;
-    // the item's block-table entries, one per lane for each 32-page window (items of up to 64
+    // the item's block-table entries, one per lane for each 32-page window (items of up to 128
     // pages; all of them are checked before the first page goes out)
     bool bad = false, mismatch = false;
     auto entry = [&](int pgi) -> int {
@@ -517,7 +519,7 @@ __device__ __forceinline__ void produce(const DecodeParams& p, const CUtensorMap
       }
       return v;
     };
-    const int bt = entry(lane), bt2 = entry(lane + 32);
+    const int bt0 = entry(lane), bt1 = entry(lane + 32), bt2 = entry(lane + 64), bt3 = entry(lane + 96);
     bad = __any_sync(FULL, bad);
     mismatch = __any_sync(FULL, mismatch);
     if (lane == 0) {
@@ -534,7 +536,8 @@ __device__ __forceinline__ void produce(const DecodeParams& p, const CUtensorMap
       }
     }
     for (int pg = 0; pg < npages; ++pg) {
-      const int phys = __shfl_sync(FULL, pg < 32 ? bt : bt2, pg & 31);
+      const int win = pg >> 5;  // warp-uniform
+      const int phys = __shfl_sync(FULL, win == 0 ? bt0 : win == 1 ? bt1 : win == 2 ? bt2 : bt3, pg & 31);
       const int slot = static_cast<int>(n % C::NSLOT);
       if (!acquire_slot(slot)) {
         stop = true;

@@ -183,9 +183,10 @@ def test_large_group_beside_many_small_groups():
 
 def test_long_shared_items_check_every_page():
     """Many groups (160 pairs sharing 1040 tokens, 8 KV heads) make the plan take shared items of
-    1024 tokens: 64 pages, whose block-table entries the producer reads in two windows of 32.  A
-    member whose table differs from its leader's only in the second window (page 40) poisons its
-    group's item (NaN rows, PA_DEV_BAD_PREFIX); every other row matches the oracle."""
+    several partitions: here the whole 1040-token prefix, 65 pages, whose block-table entries the
+    producer reads in windows of 32.  A member whose table differs from its leader's only in the
+    second window (page 40) poisons its group's item (NaN rows, PA_DEV_BAD_PREFIX); every other
+    row matches the oracle."""
     sms = torch.cuda.get_device_properties(0).multi_processor_count
     groups = [W.Group(1040, [1, 1]) for _ in range(160)]
     w = W.build_groups("long", groups, num_q_heads=32, num_kv_heads=8, head_dim=128, block_size=16, q_dtype="bf16",
