@@ -95,8 +95,9 @@ PA_API size_t pa_decode_workspace_size(int num_seqs, int num_q_heads, int head_d
  *   supported: head_dim 64 or 128, block_size 16 or 32, G = num_q_heads / num_kv_heads
  *   from 1 to 8, num_kv_heads up to 255.  partition_size (0 = 512) must be a multiple of
  *   block_size and at most 32 * block_size: sequences longer than one partition are split into
- *   partitions whose partial softmax states are merged by a second kernel
- *   (deterministic: the split depends only on seq_lens[i]).
+ *   pieces of whole partitions (see PA_OPT_ITEM_SPLIT) whose partial softmax states are merged
+ *   by a second kernel (deterministic: the split depends on the call's arguments and the
+ *   device's SM count, never on timing).
  *   workspace    device scratch of >= pa_decode_workspace_size(num_seqs, num_q_heads,
  *                head_dim, max_blocks_per_seq * block_size, partition_size) bytes, 256-byte
  *                aligned; its contents need no initialisation and are overwritten.
@@ -268,11 +269,27 @@ PA_API int pa_selftest_wait_timeout(int polls, void* stream);
  *                          softmax warps that take the chunks in turn).
  * All three match the same oracle within the attention tolerances.  Other shapes and paths ignore
  * the option.
+ *
+ * PA_OPT_ITEM_SPLIT chooses how the decode calls cut the sequences into work items:
+ *   PA_SPLIT_ADAPTIVE (default) pieces of one to four partitions (at most 128 blocks).  Counted
+ *                     at one partition each, the call's items come to n per page pipeline of
+ *                     the device (SMs x pipelines per SM); shared prefixes, and each sequence's
+ *                     leading tokens, go in pieces of min(4, n / 2) partitions, its following
+ *                     tokens in pieces of min(4, n / 8), and its ragged tail last, so that the
+ *                     items that end a launch are short.  Fewer pieces leave less for the merge
+ *                     kernel; the split, and so the rounding of a row, then depends on the batch
+ *                     and the device's SM count as well as on the sequence;
+ *   PA_SPLIT_FIXED    pieces of exactly partition_size tokens (and a ragged tail): a sequence's
+ *                     output is then the same bits in every batch.
+ * Both match the oracle within the attention tolerances.
  * Returns PA_OK, or PA_ERR_INVALID for an unknown option or value (nothing changes then). */
 #define PA_OPT_WIDE_KERNEL 1
 #define PA_WIDE_MMA 0
 #define PA_WIDE_TCGEN05 1
 #define PA_WIDE_AUTO 2
+#define PA_OPT_ITEM_SPLIT 2
+#define PA_SPLIT_ADAPTIVE 0
+#define PA_SPLIT_FIXED 1
 PA_API int pa_set_option(int option, int value);
 
 /* ABI version of this header (major * 100 + minor). */

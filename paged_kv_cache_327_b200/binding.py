@@ -302,6 +302,8 @@ def pa_selftest_wait_timeout(polls: int, stream=None) -> None:
 
 PA_OPT_WIDE_KERNEL = 1
 WIDE_KERNELS = {"mma": 0, "tcgen05": 1, "auto": 2}
+PA_OPT_ITEM_SPLIT = 2
+ITEM_SPLITS = {"adaptive": 0, "fixed": 1}
 
 
 def pa_set_option(option: int, value: int) -> None:
@@ -315,6 +317,14 @@ def set_wide_kernel(name: str) -> None:
     if name not in WIDE_KERNELS:
         raise ValueError(f"wide kernel must be one of {sorted(WIDE_KERNELS)}, not {name!r}")
     pa_set_option(PA_OPT_WIDE_KERNEL, WIDE_KERNELS[name])
+
+
+def set_item_split(name: str) -> None:
+    """How decode calls cut sequences into work items: "adaptive" (default: pieces of one to four
+    partitions, sized to the batch) or "fixed" (one partition each: batch-invariant bits)."""
+    if name not in ITEM_SPLITS:
+        raise ValueError(f"item split must be one of {sorted(ITEM_SPLITS)}, not {name!r}")
+    pa_set_option(PA_OPT_ITEM_SPLIT, ITEM_SPLITS[name])
 
 
 def pa_get_device_error(stream=None) -> int:

@@ -200,6 +200,8 @@ int launch_partition(const pa::DecodeParams& p, const CUtensorMap& tmk, const CU
 // The tensor-core kernel for wide items (block size 16, head_dim 128, 16-bit cache and query).
 // kernel for items of more than 8 query rows (PA_OPT_WIDE_KERNEL)
 std::atomic<int> g_wide_kernel{PA_WIDE_AUTO};
+// how the calls cut sequences into work items (PA_OPT_ITEM_SPLIT)
+std::atomic<int> g_item_split{PA_SPLIT_ADAPTIVE};
 
 template <typename KT>
 int launch_tc(const pa::DecodeParams& p, const CUtensorMap& tmk, const CUtensorMap& tmv, const CUtensorMap& tmq,
@@ -299,10 +301,14 @@ int pa_set_option(int option, int value) {
     g_wide_kernel.store(value, std::memory_order_relaxed);
     return PA_OK;
   }
+  if (option == PA_OPT_ITEM_SPLIT && (value == PA_SPLIT_ADAPTIVE || value == PA_SPLIT_FIXED)) {
+    g_item_split.store(value, std::memory_order_relaxed);
+    return PA_OK;
+  }
   return PA_ERR_INVALID;
 }
 
-int pa_version(void) { return 100; }
+int pa_version(void) { return 101; }
 
 const char* pa_strerror(int status) {
   switch (status) {
@@ -438,11 +444,13 @@ int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cac
   p.groups = groups;
   p.num_groups = num_groups;
   p.max_members = max_members;
-  // shared items of up to four partitions (and the 128 pages a warp-MMA producer takes per item)
-  // where the plan finds many of them; the tensor-core kernel's producer takes 32 pages per item
-  p.shared_partition = use_tc ? P : std::min(4 * P, 128 * block_size);
-  p.rings = info->sm_count * 4;  // one CTA per SM, 4 rings each (prefix groups are 16-bit)
+  // items of up to four partitions, and the 128 pages a producer takes per item, where the plan
+  // finds enough of them; one CTA per SM, with 4 rings (8 with an FP8 cache) or, on the
+  // tensor-core kernel, one chunk pipeline
   const bool fp8 = kv_dtype == PA_FP8_E4M3;
+  const bool fixed = g_item_split.load(std::memory_order_relaxed) == PA_SPLIT_FIXED;
+  p.long_partition = fixed ? P : std::min(4 * P, 128 * block_size);
+  p.rings = info->sm_count * (use_tc ? 1 : fp8 ? 8 : 4);
   p.scale_log2 = scale * (fp8 ? k_scale : 1.f) * 1.4426950408889634f;
   p.v_scale = fp8 ? v_scale : 1.f;
   p.counters = reinterpret_cast<unsigned int*>(ws + L.counters);

@@ -92,8 +92,8 @@ struct DecodeParams {
   // first .. first + members - 1 hold the same blocks for their first `shared` tokens
   const int32_t* groups;
   int num_groups, max_members;  // a shared item covers at most max_members sequences
-  int shared_partition;  // tokens of a shared item when there are many (a multiple of block_size)
-  int rings;             // page pipelines of the partition kernel (CTAs x rings per CTA)
+  int long_partition;  // the longest item the partition kernel takes (a multiple of partition_size)
+  int rings;           // page pipelines of the partition kernel (CTAs x rings per CTA)
   float scale_log2;  // scale * log2(e) (* k_scale for an FP8 cache)
   float v_scale;     // multiplies the output (FP8 cache); 1 otherwise
   // workspace views
@@ -178,10 +178,12 @@ constexpr int kPartsEmpty = -1, kPartsInvalid = -2;
 // L >= qtok) with S shared tokens (0 outside a prefix group):
 //   * shared items: a sequence that leads up to max_members members of a group gets one item
 //     per partition of tokens [0, S), covering all those members;
-//   * own items: tokens [S, L) in partitions of P tokens (full ones, then a ragged tail).
+//   * own items: tokens [S, L) in long partitions of Pb tokens, then partitions of Pm tokens,
+//     then a ragged tail (Pb >= Pm >= P, all multiples of P, chosen below from the batch).
 // The partial results of sequence i are numbered shared partitions first, then its own; a
 // sequence with no shared tokens and one partition writes `out` directly.  Items are listed
-// shared first (the widest), then full partitions, then tails, each kind in sequence order.
+// shared first (the widest), then long, then middle partitions, then tails, each kind in
+// sequence order, so that the items that finish a launch are the shortest.
 // Thread t plans the contiguous run of sequences [t * chunk, (t + 1) * chunk): every count
 // is one block-wide scan, whatever the batch size.
 __global__ void __launch_bounds__(kPlanThreads) pa_decode_plan_kernel(const DecodeParams p) {
@@ -289,21 +291,31 @@ __global__ void __launch_bounds__(kPlanThreads) pa_decode_plan_kernel(const Deco
 
   // column groups: the qtok query tokens of a sequence are split into items of qtok_item tokens
   const int Tc = p.qtok_item, ncg = (p.qtok + Tc - 1) / Tc;
-  // Shared items take m P tokens each: m = 1, or more (up to shared_partition / P) while the
-  // shared items, counted at P, still number at least 2 m times the page pipelines -- fewer
-  // partial results per member for the merge, with the parallelism still ample.  The choice is
+  // Item lengths.  A longer item leaves fewer partial results for the merge and fewer item
+  // starts and ends in the partition kernel, but the items that finish a launch set its tail.
+  // Counted at P tokens, n items fall to each page pipeline; then shared items and long own
+  // items take m P tokens (m up to long_partition / P) while at least 2 of them per pipeline
+  // remain, and middle own items take m P tokens while at least 8 remain.  The choice is
   // block-uniform.
-  int Ps = P;
-  if (p.num_groups > 0 && p.shared_partition > P) {
-    long long loc = 0, tot;
-    for (int i = lo; i < hi; ++i)
-      if (valid_len(p.seq_lens[i]) && p.seq_sub[i] > 0) loc += (p.seq_shared[i] + P - 1) / P;
+  int Ps = P, Pb = P, Pm = P;
+  if (p.long_partition > P) {
+    long long loc = 0, tot;  // shared items (low 32 bits) and own items (high 32 bits) at P
+    for (int i = lo; i < hi; ++i) {
+      const int L = p.seq_lens[i];
+      if (!valid_len(L)) continue;
+      const int S = p.num_groups > 0 ? p.seq_shared[i] : 0;
+      if (p.num_groups > 0 && p.seq_sub[i] > 0) loc += (S + P - 1) / P;
+      loc += static_cast<long long>((L - S + P - 1) / P * ncg) << 32;
+    }
     (void)block_exclusive_scan<long long>(loc, 0, ScanSum{}, s_warp, &tot);
-    const long long m = min(static_cast<long long>(p.shared_partition / P), tot * p.num_kv_heads / (2LL * p.rings));
-    if (m > 1) Ps = static_cast<int>(m) * P;
+    const long long mmax = p.long_partition / P, hk = p.num_kv_heads, r = p.rings;
+    const long long n_sh = (tot & 0xffffffffll) * hk, n_own = (tot >> 32) * hk;
+    Ps = static_cast<int>(max(1ll, min(mmax, n_sh / (2 * r)))) * P;
+    Pb = static_cast<int>(max(1ll, min(mmax, n_own / (2 * r)))) * P;
+    Pm = static_cast<int>(max(1ll, min(mmax, n_own / (8 * r)))) * P;
   }
   struct Counts {
-    int L, S, sub, ns, nf, nt, nps;
+    int L, S, sub, ns, nb, nm, nt, nps;
   };
   auto counts = [&](int i) {
     Counts c{};
@@ -313,50 +325,54 @@ __global__ void __launch_bounds__(kPlanThreads) pa_decode_plan_kernel(const Deco
     c.sub = p.num_groups > 0 ? p.seq_sub[i] : 0;
     c.nps = (c.S + Ps - 1) / Ps;
     c.ns = c.sub > 0 ? c.nps : 0;
-    c.nf = (c.L - c.S) / P;
-    c.nt = ((c.L - c.S) % P) ? 1 : 0;
+    const int own = c.L - c.S;
+    c.nb = Pb > Pm ? own / Pb : 0;
+    c.nm = (own - c.nb * Pb) / Pm;
+    c.nt = ((own - c.nb * Pb) % Pm) ? 1 : 0;
     return c;
   };
 
-  int loc_s = 0, loc_f = 0, loc_t = 0;
+  int loc_s = 0, loc_b = 0, loc_m = 0, loc_t = 0;
   for (int i = lo; i < hi; ++i) {
     const Counts c = counts(i);
     loc_s += c.ns;
-    loc_f += c.nf * ncg;
+    loc_b += c.nb * ncg;
+    loc_m += c.nm * ncg;
     loc_t += c.nt * ncg;
   }
-  long long tft;
-  const long long oft = block_exclusive_scan<long long>(pack2x32(loc_f, loc_t), 0, ScanSum{}, s_warp, &tft);
-  int of = lo32(oft), ot = hi32(oft), os = 0, n_shared = 0;
-  const int n_full = lo32(tft), n_tail = hi32(tft);
-  if (p.num_groups > 0) {  // block-uniform
-    long long tsl;
-    os = static_cast<int>(block_exclusive_scan<long long>(loc_s, 0, ScanSum{}, s_warp, &tsl));
-    n_shared = static_cast<int>(tsl);
-  }
+  long long t_bm, t_ts;
+  const long long o_bm = block_exclusive_scan<long long>(pack2x32(loc_b, loc_m), 0, ScanSum{}, s_warp, &t_bm);
+  const long long o_ts = block_exclusive_scan<long long>(pack2x32(loc_t, loc_s), 0, ScanSum{}, s_warp, &t_ts);
+  int ob = lo32(o_bm), om = hi32(o_bm), ot = lo32(o_ts), os = hi32(o_ts);
+  const int n_long = lo32(t_bm), n_mid = hi32(t_bm), n_tail = lo32(t_ts), n_shared = hi32(t_ts);
+  // own items follow the shared ones: long, then middle, then tails
+  ob += n_shared;
+  om += n_shared + n_long;
+  ot += n_shared + n_long + n_mid;
   for (int i = lo; i < hi; ++i) {
     const Counts c = counts(i);
     const bool valid = valid_len(c.L);
     if (!valid) record_error(DEV_BAD_SEQ_LEN);
-    const int parts = c.nps + c.nf + c.nt;
+    const int parts = c.nps + c.nb + c.nm + c.nt;
     const bool direct = c.S == 0 && parts == 1;
     p.seq_parts[i] = !valid ? kPartsInvalid : c.L == 0 ? kPartsEmpty : direct ? 0 : parts;
-    const int dflag = (c.S == 0 && c.nf + c.nt == 1) ? WI_DIRECT : 0;
+    const int dflag = direct ? WI_DIRECT : 0;
     // shared items have one query token (prefix groups are single-token decode)
     for (int k = 0; k < c.ns; ++k)
       p.items[os++] = WorkItem{i, k * Ps, min(c.S, (k + 1) * Ps), k | (c.sub << 16), 0, 1, 0, 0};
-    for (int k = 0; k < c.nf; ++k)
+    // own partitions: [tok0, tok1) as partial result `part`, one item per column group
+    auto own_item = [&](int& o, int tok0, int tok1, int part) {
       for (int j = 0; j < ncg; ++j)
-        p.items[n_shared + of++] = WorkItem{i, c.S + k * P, c.S + (k + 1) * P, (c.nps + k) | (1 << 16) | dflag,
-                                            j * Tc, min(Tc, p.qtok - j * Tc), 0, 0};
-    if (c.nt)
-      for (int j = 0; j < ncg; ++j)
-        p.items[n_shared + n_full + ot++] = WorkItem{i, c.S + c.nf * P, c.L, (c.nps + c.nf) | (1 << 16) | dflag,
-                                                     j * Tc, min(Tc, p.qtok - j * Tc), 0, 0};
+        p.items[o++] = WorkItem{i, tok0, tok1, part | (1 << 16) | dflag, j * Tc, min(Tc, p.qtok - j * Tc), 0, 0};
+    };
+    int tok = c.S, part = c.nps;
+    for (int k = 0; k < c.nb; ++k, tok += Pb) own_item(ob, tok, tok + Pb, part++);
+    for (int k = 0; k < c.nm; ++k, tok += Pm) own_item(om, tok, tok + Pm, part++);
+    if (c.nt) own_item(ot, tok, c.L, part);
   }
   if (threadIdx.x == 0) {
     p.counters[0] = 0;
-    p.counters[1] = static_cast<unsigned>(n_shared + n_full + n_tail);
+    p.counters[1] = static_cast<unsigned>(n_shared + n_long + n_mid + n_tail);
   }
 }
 
@@ -1125,14 +1141,7 @@ __global__ void __launch_bounds__(kMergeWarps * 32, 4) pa_decode_merge_kernel(co
   const int Hq = p.qtok * p.num_q_heads, D = p.head_dim;
   if (pair >= static_cast<int64_t>(p.num_seqs) * Hq) return;
   const int seq = static_cast<int>(pair / Hq), hq = static_cast<int>(pair % Hq);
-  int np;
-  if (p.num_groups == 0) {  // the partitions follow from the length alone
-    const int L = p.seq_lens[seq], P = p.partition_size;
-    const bool valid = L >= 0 && L <= p.max_blocks_per_seq * p.block_size && (L == 0 || L >= p.qtok);
-    np = !valid ? kPartsInvalid : L == 0 ? kPartsEmpty : L <= P ? 0 : (L + P - 1) / P;
-  } else {
-    np = p.seq_parts[seq];
-  }
+  const int np = p.seq_parts[seq];  // the plan's count of the sequence's partial results
   const int64_t o = (static_cast<int64_t>(seq) * Hq + hq) * D;
   if (np < 0) {  // no work item: the row is zero (empty sequence) or NaN (invalid length)
     const float v = np == kPartsEmpty ? 0.f : CUDART_NAN_F;

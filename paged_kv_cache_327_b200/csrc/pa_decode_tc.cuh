@@ -222,6 +222,7 @@ struct TcCfg {
   static constexpr uint32_t AB = std::is_same<KT, __nv_bfloat16>::value ? 1u : 0u;
   static constexpr uint32_t IDESC_S = umma_idesc(AB, 0, 0, M, CT);  // Q (K-major) . K^T (K-major)
   static constexpr uint32_t IDESC_O = umma_idesc(AB, 0, 1, M, D);   // P (K-major) . V (MN-major)
+  static_assert(32 % CH == 0, "a chunk's pages lie in one 32-page window of the block table");
   static_assert(CHUNK_BYTES % 1024 == 0 && OFF_Q % 1024 == 0 && QHALF % 1024 == 0 && OFF_P % 1024 == 0,
                 "128-byte swizzle atoms");
   static_assert(TM_S + NSB * CT <= TM_COLS, "tensor memory");
@@ -248,7 +249,8 @@ __device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, i
 struct TcItemLoads {
   bool valid;
   WorkItem it;
-  int kvh, bt, rel0;
+  int kvh, rel0;
+  int bt[4];  // block-table entries, one per lane for each 32-page window (items of up to 128 pages)
   bool mismatch;
 };
 
@@ -286,17 +288,21 @@ __device__ __forceinline__ void tc_produce(const DecodeParams& p, const CUtensor
     L.valid = w < total;
     L.it = it;
     L.kvh = static_cast<int>(w % Hkv);
-    L.bt = 0;
+    L.bt[0] = L.bt[1] = L.bt[2] = L.bt[3] = 0;
     L.mismatch = false;
     L.rel0 = 0;
     if (!L.valid) return;
     const int members = (it.pm >> 16) & 0xff;
     const int npages = (it.tok1 - it.tok0 + BS - 1) / BS;
-    if (lane < npages) {
-      const int64_t col = it.tok0 / BS + lane;
-      L.bt = p.block_tables[static_cast<int64_t>(it.seq) * p.max_blocks_per_seq + col];
-      for (int m = 1; m < members; ++m)  // the members of a shared item must hold the same blocks
-        L.mismatch |= p.block_tables[static_cast<int64_t>(it.seq + m) * p.max_blocks_per_seq + col] != L.bt;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int pgi = lane + 32 * k;
+      if (pgi < npages) {
+        const int64_t col = it.tok0 / BS + pgi;
+        L.bt[k] = p.block_tables[static_cast<int64_t>(it.seq) * p.max_blocks_per_seq + col];
+        for (int m = 1; m < members; ++m)  // the members of a shared item must hold the same blocks
+          L.mismatch |= p.block_tables[static_cast<int64_t>(it.seq + m) * p.max_blocks_per_seq + col] != L.bt[k];
+      }
     }
     // key positions relative to the item's first query token, at position len - T + t0
     if (T > 1) L.rel0 = it.tok0 - (p.seq_lens[it.seq] - T + it.t0);
@@ -323,7 +329,9 @@ __device__ __forceinline__ void tc_produce(const DecodeParams& p, const CUtensor
     const int tok0 = it.tok0, tok1 = it.tok1;
     const int npages = (tok1 - tok0 + BS - 1) / BS;
     const int rows = members * it.tq;
-    bool bad = lane < npages && (cur.bt < 0 || cur.bt >= p.num_blocks);
+    bool bad = false;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) bad |= lane + 32 * k < npages && (cur.bt[k] < 0 || cur.bt[k] >= p.num_blocks);
     bad = __any_sync(FULL, bad);
     const bool mismatch = __any_sync(FULL, cur.mismatch);
     if (lane == 0) {
@@ -364,7 +372,10 @@ __device__ __forceinline__ void tc_produce(const DecodeParams& p, const CUtensor
         // one box per lane: K column block 0 / K column block 1 / the whole V page, of page lane / 3
         // (K rows go to the chunk's block-major K operand, a V page lands as [block][row])
         const int lp = lane / 3, lk = lane - 3 * lp;
-        const int lphys = __shfl_sync(FULL, cur.bt, (pg0 + min(lp, C::CH - 1)) & 31);
+        // the chunk lies in one 32-page window (CH divides 32), so the window is warp-uniform
+        const int win = pg0 >> 5;
+        const int lphys = __shfl_sync(FULL, win == 0 ? cur.bt[0] : win == 1 ? cur.bt[1] : win == 2 ? cur.bt[2] : cur.bt[3],
+                                      (pg0 + min(lp, C::CH - 1)) & 31);
         uint8_t* cb = smem + c * C::CHUNK_BYTES;
         if (lp < npg) {
           if (lk < 2)

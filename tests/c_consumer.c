@@ -15,7 +15,7 @@
   } while (0)
 
 int main(void) {
-  CHECK(pa_version() == 100);
+  CHECK(pa_version() == 101);
   CHECK(strlen(pa_strerror(PA_OK)) > 0);
   CHECK(strstr(pa_strerror(12345), "unknown") != NULL);
 
@@ -53,6 +53,10 @@ int main(void) {
   CHECK(pa_set_option(PA_OPT_WIDE_KERNEL, PA_WIDE_AUTO) == PA_OK);
   CHECK(pa_set_option(PA_OPT_WIDE_KERNEL, 7) == PA_ERR_INVALID);
   CHECK(pa_set_option(99, PA_WIDE_MMA) == PA_ERR_INVALID);
+  /* the item-split option: its two values, nothing else */
+  CHECK(pa_set_option(PA_OPT_ITEM_SPLIT, PA_SPLIT_FIXED) == PA_OK);
+  CHECK(pa_set_option(PA_OPT_ITEM_SPLIT, PA_SPLIT_ADAPTIVE) == PA_OK);
+  CHECK(pa_set_option(PA_OPT_ITEM_SPLIT, 2) == PA_ERR_INVALID);
   puts("ok");
   return 0;
 }

@@ -37,7 +37,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_version_and_strerror(lib):
-    assert lib.pa_version() == 100
+    assert lib.pa_version() == 101
     for st in (B.PA_OK, B.PA_ERR_INVALID, B.PA_ERR_UNSUPPORTED, B.PA_ERR_WORKSPACE, B.PA_ERR_CUDA):
         assert len(B.pa_strerror(st)) > 5
     assert "unknown" in B.pa_strerror(12345)
@@ -180,7 +180,8 @@ def test_selftest_argument_checks(lib):
 
 
 def test_set_option(lib):
-    """The wide-kernel option takes its three values and rejects others (no GPU needed)."""
+    """The wide-kernel option takes its three values, the item-split option its two, and both
+    reject others (no GPU needed)."""
     assert lib.pa_set_option(B.PA_OPT_WIDE_KERNEL, 1) == B.PA_OK
     assert lib.pa_set_option(B.PA_OPT_WIDE_KERNEL, 0) == B.PA_OK
     assert lib.pa_set_option(B.PA_OPT_WIDE_KERNEL, 2) == B.PA_OK
@@ -192,6 +193,15 @@ def test_set_option(lib):
     B.set_wide_kernel("tcgen05")
     B.set_wide_kernel("mma")
     B.set_wide_kernel("auto")
+    assert lib.pa_set_option(B.PA_OPT_ITEM_SPLIT, 1) == B.PA_OK
+    assert lib.pa_set_option(B.PA_OPT_ITEM_SPLIT, 0) == B.PA_OK
+    assert lib.pa_set_option(B.PA_OPT_ITEM_SPLIT, 2) == B.PA_ERR_INVALID
+    assert lib.pa_set_option(B.PA_OPT_ITEM_SPLIT, -1) == B.PA_ERR_INVALID
+    assert lib.pa_set_option(3, 0) == B.PA_ERR_INVALID
+    with pytest.raises(ValueError):
+        B.set_item_split("longest")
+    B.set_item_split("fixed")
+    B.set_item_split("adaptive")
 
 
 def test_workspace_reserves_every_work_item(lib):

@@ -29,4 +29,4 @@ def test_two_concurrent_builders_produce_a_loadable_library(tmp_path):
     assert os.path.exists(lib)
     # no temporary file is left behind, and the library is whole: it loads and answers
     assert not [f for f in os.listdir(tmp_path) if f.endswith(".tmp")]
-    assert ctypes.CDLL(lib).pa_version() == 100
+    assert ctypes.CDLL(lib).pa_version() == 101

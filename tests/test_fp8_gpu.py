@@ -120,6 +120,15 @@ def test_fp8_full_size(name, bs):
 
 
 def test_fp8_is_deterministic_and_batch_invariant():
+    """Same bits on a second call, and (PA_SPLIT_FIXED) for a sequence decoded on its own."""
+    B.set_item_split("fixed")
+    try:
+        check_deterministic_and_batch_invariant()
+    finally:
+        B.set_item_split("adaptive")
+
+
+def check_deterministic_and_batch_invariant():
     w = W.make_config("8b", kv_dtype="e4m3", num_seqs=24)
     dw, a = run(w)
     ws = B.DecodeWorkspace.for_workload(dw)

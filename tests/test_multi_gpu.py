@@ -136,6 +136,15 @@ def test_multi_8b_full_size(T):
 
 
 def test_multi_is_deterministic_and_batch_invariant():
+    """Same bits on a second call, and (PA_SPLIT_FIXED) for a sequence decoded on its own."""
+    B.set_item_split("fixed")
+    try:
+        check_deterministic_and_batch_invariant()
+    finally:
+        B.set_item_split("adaptive")
+
+
+def check_deterministic_and_batch_invariant():
     w = W.make_config("8b", num_seqs=24, num_q_tokens=4)
     dw, a = gpu_multi(w)
     ws = B.DecodeWorkspace.for_workload(dw)
