@@ -15,15 +15,13 @@
 //   O += P . V       tcgen05.mma per page, M = 64, N = head_dim, K = 16 tokens; A = P, B = the
 //                    staged V page read in place (MN-major)
 // Two groups of four softmax warps take the chunks (S products) in turn, so that two chunks are
-// in the softmax at once.  The running maximum stays one sequence per item: the owner of chunk k
-// decides its maxima from those decided for chunk k - 1 (handed over per lane quarter through
-// shared memory and an mbarrier), so every P is relative to the maximum O holds and one O
-// accumulator suffices; each group sums the weights of its own chunks, and the two parts meet at
-// the item's end, where each warp writes half of the head_dim outputs of its 16 rows.  S and O
-// products are issued by two warps of their own, so that neither waits for the other's issue, and
-// complete on mbarriers.  Buffers keep every stage busy: three S buffers, a P buffer per group,
-// two O buffers (an item's output is read while the next item accumulates), two query buffers and
-// five chunk buffers of 32 KB in flight per SM.
+// in the softmax at once.  Each group keeps its own online softmax over its chunks of an item --
+// running maxima, row sums, and an O accumulator in tensor memory -- so neither waits for the
+// other's maxima; the two states meet at the item's end, where the two warps of a lane quarter
+// exchange (maximum, sum) per row and each writes half of the head_dim outputs of the quarter's 16
+// rows.  S and O products are issued by two warps of their own, so that neither waits for the
+// other's issue, and complete on mbarriers.  Buffers keep every stage busy: three S buffers, a P
+// buffer per group, two query buffers and five chunk buffers of 32 KB in flight per SM.
 //
 // CTA (one per SM): warps 0-7 run the softmax and the output (warp w on TMEM lane quarter w % 4,
 // the chunks whose S product index has the parity of w / 4; a quarter without the item's rows
@@ -201,23 +199,24 @@ struct TcCfg {
   static constexpr int OFF_P = OFF_Q + QN * QBUF;
   static constexpr int OFF_BAR = OFF_P + 2 * PBUF;
   // mbarriers: chunk full / empty, query buffer free, S full / free, P full / free (the O product
-  // that read it is done), O buffer free (its item's output has been read), final drain, per lane
-  // quarter: the running maximum a chunk's owner decided [quarter][chunk parity], the item sums of
-  // the two softmax groups [quarter][item parity]; and chunk meta written (before its copies land)
+  // that read it is done), O accumulators free (the item's output has been read), final drain,
+  // the two softmax groups' item states [quarter][item parity]; and chunk meta written (before
+  // its copies land)
   static constexpr int NSB = 3;  // S buffers: S products run up to NSB - 1 chunks ahead of the softmax
   static constexpr int B_FULL = 0, B_EMPTY = NCH, B_QFREE = 2 * NCH, B_SFULL = B_QFREE + QN, B_SFREE = B_SFULL + NSB,
-                       B_PFULL = B_SFREE + NSB, B_PFREE = B_PFULL + 2, B_OFREE = B_PFREE + 2, B_FIN = B_OFREE + 2,
-                       B_MAX = B_FIN + 1, B_SUM = B_MAX + 8, B_META = B_SUM + 8, NBAR = B_META + NCH;
+                       B_PFULL = B_SFREE + NSB, B_PFREE = B_PFULL + 2, B_OFREE = B_PFREE + 2, B_FIN = B_OFREE + 1,
+                       B_SUM = B_FIN + 1, B_META = B_SUM + 8, NBAR = B_META + NCH;
   static constexpr int OFF_META = OFF_BAR + ((NBAR * 8 + 15) & ~15);
-  // exchange between the two softmax warps of a lane quarter: the decided running maxima
-  // [chunk parity][M] and the groups' item sums [item parity][group][M]
+  // exchange between the two softmax warps of a lane quarter: each group's (running maximum,
+  // sum) of a row at the item's end, [item parity][group][M]
   static constexpr int OFF_XCH = OFF_META + NCH * 32;
-  static constexpr int OFF_MISC = OFF_XCH + (2 + 4) * M * 4;
+  static constexpr int OFF_MISC = OFF_XCH + 2 * 2 * M * 8;
   static constexpr int SMEM_BYTES = 1024 + OFF_MISC + 16;
   // warps 0-7: softmax and output, warp 8 loads, warp 9 issues the S products, warp 10 the O products
   static constexpr int NSM = 256, W_LOAD = 8, W_S = 9, W_O = 10, NTHREADS = NSM + 96;
   static constexpr int HC = CT;  // chunk columns per softmax warp: all of them (groups alternate chunks)
-  // TMEM columns: two O buffers (head_dim columns each), then NSB S buffers (one chunk each)
+  // TMEM columns: the two softmax groups' O accumulators (head_dim columns each), then NSB S
+  // buffers (one chunk each)
   static constexpr uint32_t TM_COLS = 512, TM_O = 0, TM_S = 2 * D;
   static constexpr uint32_t AB = std::is_same<KT, __nv_bfloat16>::value ? 1u : 0u;
   static constexpr uint32_t IDESC_S = umma_idesc(AB, 0, 0, M, CT);  // Q (K-major) . K^T (K-major)
@@ -497,9 +496,10 @@ __device__ __forceinline__ void tc_mma_s(uint8_t* smem, uint64_t* bars, const in
   mbar_wait_bounded(bars + C::B_FIN, 0u, kWaitLimit);
 }
 
-// Warp 10: O(n) += P(n) . V(n) once the softmax warps have written P(n); its completion releases the
-// P buffer and the chunk buffer.  An item's first O product overwrites its O buffer, once the item
-// before the previous one has been read out of it.
+// Warp 10: O_g += P(n) . V(n) once the softmax warps have written P(n), g the parity of n (the
+// softmax group that took the chunk); its completion releases the P buffer and the chunk buffer.
+// A group's first O product of an item overwrites its accumulator, once the item before has been
+// read out of both.
 template <typename C>
 __device__ __forceinline__ void tc_mma_o(uint8_t* smem, uint64_t* bars, const int4* meta, volatile int* abort_flag,
                                          uint32_t tm, int lane) {
@@ -511,7 +511,8 @@ __device__ __forceinline__ void tc_mma_o(uint8_t* smem, uint64_t* bars, const in
   uint64_t* p_free = bars + C::B_PFREE;
   uint64_t* o_free = bars + C::B_OFREE;
   uint32_t np = 0;  // O products issued
-  int items = -1;
+  // items with O products (the others leave the accumulators alone), and the chunk's place in its item
+  int items = -1, cc = 0;
   bool item_bad = false, ok = true;
   for (uint32_t k = 0;; ++k) {
     const int c = static_cast<int>(k % C::NCH);
@@ -523,10 +524,10 @@ __device__ __forceinline__ void tc_mma_o(uint8_t* smem, uint64_t* bars, const in
     const int4 m0 = meta[2 * c];
     const int flags = (m0.z >> 24) & 0xff;
     if (flags & F_END) break;
-    const bool first = (flags & F_FIRST) != 0;
-    if (first) {
-      ++items;
+    if (flags & F_FIRST) {
       item_bad = (flags & F_BAD) != 0;
+      if (!item_bad) ++items;
+      cc = 0;
     }
     const int npg = (m0.z >> 8) & 0xff;
     if (item_bad) {
@@ -534,10 +535,15 @@ __device__ __forceinline__ void tc_mma_o(uint8_t* smem, uint64_t* bars, const in
       if (lane == 0) mbar_arrive(&empty[c]);
       continue;
     }
-    const uint32_t pb = np & 1u, ob = static_cast<uint32_t>(items) & 1u;
+    // the item's chunks alternate between the groups, so its first two open the two accumulators
+    const bool opens = cc < 2;
+    ++cc;
+    const uint32_t pb = np & 1u, ob = np & 1u;
     bool good = mbar_wait_bounded(&p_full[pb], (np >> 1) & 1u, kWaitLimit);
-    if (good && first && items >= 2)  // the output of item - 2 has been read out of this O buffer
-      good = mbar_wait_bounded(&o_free[ob], ((items >> 1) - 1) & 1u, kWaitLimit);
+    // the output of the item before (with O products: only those complete o_free, and an item's
+    // output needs its own products, so o_free is never two items ahead) has been read out
+    if (good && opens && items >= 1)
+      good = mbar_wait_bounded(o_free, static_cast<uint32_t>(items - 1) & 1u, kWaitLimit);
     if (!__all_sync(FULL, good)) {
       ok = false;
       break;
@@ -549,7 +555,7 @@ __device__ __forceinline__ void tc_mma_o(uint8_t* smem, uint64_t* bars, const in
       for (int j = 0; j < npg; ++j) {
         const uint64_t a = smem_desc_sw128(pa + j * 32, 16, 1024);
         const uint64_t b = smem_desc_sw128(vb + j * C::VPAGE, C::BOX, 1024);
-        umma_ss(tm + C::TM_O + ob * D, a, b, C::IDESC_O, (first && j == 0) ? 0u : 1u);
+        umma_ss(tm + C::TM_O + ob * D, a, b, C::IDESC_O, (opens && j == 0) ? 0u : 1u);
       }
       umma_commit(&p_free[pb]);
       umma_commit(&empty[c]);  // the chunk buffer is free once these products are done
@@ -582,8 +588,7 @@ __global__ void __launch_bounds__(TcCfg<KT>::NTHREADS, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
   int4* meta = reinterpret_cast<int4*>(smem + C::OFF_META);
-  float* xmax = reinterpret_cast<float*>(smem + C::OFF_XCH);               // [chunk parity][M]
-  float* xsum = xmax + 2 * M;                                              // [item parity][group][M]
+  float2* xstate = reinterpret_cast<float2*>(smem + C::OFF_XCH);  // [item parity][group][M]
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC + 4);
 
@@ -592,9 +597,9 @@ __global__ void __launch_bounds__(TcCfg<KT>::NTHREADS, 1)
       // S free and P full: one arrival per warp of the chunk's softmax group; O free: one per
       // softmax warp; a chunk buffer is free once the softmax warps and the S warp have read its
       // meta and the O warp has finished with it (or skipped it); the final drain: one commit per
-      // MMA warp; a decided maximum: its owner warp; item sums: both warps of the quarter
+      // MMA warp; item states: both warps of the quarter
       const bool grp = (s >= C::B_SFREE && s < C::B_SFREE + C::NSB) || (s >= C::B_PFULL && s < C::B_PFULL + 2);
-      const bool all = s >= C::B_OFREE && s < C::B_OFREE + 2;
+      const bool all = s == C::B_OFREE;
       const bool empty = s >= C::B_EMPTY && s < C::B_EMPTY + C::NCH;
       const bool sums = s >= C::B_SUM && s < C::B_SUM + 8;
       mbar_init(&bars[s], grp ? C::NSM / 64 : all ? C::NSM / 32 : empty ? C::NSM / 32 + 2 : (s == C::B_FIN || sums) ? 2 : 1);
@@ -630,11 +635,11 @@ __global__ void __launch_bounds__(TcCfg<KT>::NTHREADS, 1)
   // Two groups of four warps take the S products in turn: group g = w / 4 the products whose index
   // has parity g, so that two chunks are in the softmax at once.  Warp w reads the 16 rows of lane
   // quarter q = w % 4 in the 16x256b shape: lane t holds rows 16 q + t / 4 and 16 q + t / 4 + 8 at
-  // the chunk columns 8 j + 2 (t % 4), + 1 (j < 8).  A row's running maximum is one sequence over
-  // the item's chunks: the owner of chunk k takes the maximum decided for chunk k - 1 from the
-  // other group's warp of its quarter, decides chunk k's and passes it on (shared memory and a
-  // per-quarter mbarrier), so O keeps one accumulator.  Each group sums its own chunks' weights;
-  // the two parts meet in the item's output.
+  // the chunk columns 8 j + 2 (t % 4), + 1 (j < 8).  Each group runs its own online softmax over its
+  // chunks of the item, into its own O accumulator (O_g): its running maxima, raised lazily, its
+  // row sums relative to them.  At the item's end the two warps of a quarter exchange their
+  // groups' (maximum, sum) per row and each writes half of the head_dim columns of the combined
+  // output, O = O_0 2^(m_0 - m) + O_1 2^(m_1 - m) with m the larger maximum.
   constexpr unsigned FULL = 0xffffffffu;
   constexpr float kNone = -1e30f;  // running maximum of a row with no score yet (finite: no NaN from -inf - -inf)
   constexpr int NJ = HC / 8;       // 8-column blocks of a chunk
@@ -646,7 +651,6 @@ __global__ void __launch_bounds__(TcCfg<KT>::NTHREADS, 1)
   uint64_t* p_full = bars + C::B_PFULL;
   uint64_t* p_free = bars + C::B_PFREE;
   uint64_t* o_free = bars + C::B_OFREE;
-  uint64_t* max_bar = bars + C::B_MAX + 2 * (warp & 3);  // [chunk parity] of this quarter
   uint64_t* sum_bar = bars + C::B_SUM + 2 * (warp & 3);  // [item parity] of this quarter
   const int ct = threadIdx.x;
   const int quarter = warp & 3, grp = warp >> 2;
@@ -660,11 +664,9 @@ __global__ void __launch_bounds__(TcCfg<KT>::NTHREADS, 1)
   uint32_t n = 0, ns = 0, np = 0;
   int items = -1;
   bool ok = true;
-  float mf0 = kNone, mf1 = kNone;  // the maxima this warp decided for the last chunk it took (log2 units)
-  float ml0 = kNone, ml1 = kNone;  // the maxima this group's part of the row sums is relative to
-  float l0 = 0.f, l1 = 0.f;        // this lane's part of the group's row sums
-  int ncol = 0, item_t0 = 0, first_np = 0;
-  uint32_t last_k = 0;             // the item's latest S product
+  float ml0 = kNone, ml1 = kNone;  // this group's running maxima of the item (log2 units)
+  float l0 = 0.f, l1 = 0.f;        // this lane's part of the group's row sums, relative to them
+  int ncol = 0, item_t0 = 0, first_np = 0, gk = 0;  // gk: this group's chunks of the item so far
   bool poisoned = false, busy = false;  // busy: the quarter holds at least one of the item's rows
 
   // completion of O product k (the P buffer it read is free again)
@@ -672,13 +674,6 @@ __global__ void __launch_bounds__(TcCfg<KT>::NTHREADS, 1)
     const bool done = mbar_wait_bounded(&p_free[k & 1u], (k >> 1) & 1u, kWaitLimit);
     tc_fence_after();
     return done;
-  };
-  // the maxima decided for chunk k, once its owner has passed them on
-  auto read_max = [&](uint32_t k, float& a, float& b) -> bool {
-    const bool got = mbar_wait_bounded(&max_bar[k & 1u], (k >> 1) & 1u, kWaitLimit);
-    a = xmax[(k & 1u) * M + row0];
-    b = xmax[(k & 1u) * M + row1];
-    return got;
   };
 
   while (true) {
@@ -701,14 +696,13 @@ __global__ void __launch_bounds__(TcCfg<KT>::NTHREADS, 1)
       ml0 = ml1 = kNone;
       l0 = l1 = 0.f;
       first_np = static_cast<int>(np);
+      gk = 0;
     }
     const int npg = (mt0.z >> 8) & 0xff, ntok_last = mt1.y;
     uint8_t* cb = smem + c * C::CHUNK_BYTES;
-    const uint32_t ob = static_cast<uint32_t>(items) & 1u;
 
     if (!poisoned) {
       const uint32_t k = ns++;  // this chunk's S product (np == k here)
-      last_k = k;
       if ((k & 1u) == static_cast<uint32_t>(grp)) {
         bool good = true;
         if (ntok_last < C::BS) good = mbar_wait_bounded(&full[c], (n / C::NCH) & 1u, kWaitLimit);  // copies landed
@@ -765,51 +759,33 @@ __global__ void __launch_bounds__(TcCfg<KT>::NTHREADS, 1)
           x0 = fmaxf(x0, __shfl_xor_sync(FULL, x0, 2));
           x1 = fmaxf(x1, __shfl_xor_sync(FULL, x1, 2));
         }
-        // the maxima decided for chunk k - 1 (always waited for: its owner has then read the
-        // slot this chunk's maxima go to); an item's first chunk starts from none
-        float p0 = kNone, p1 = kNone;
-        if (k > 0) {
-          float a, bb;
-          good = read_max(k - 1, a, bb) && good;
-          if (!first) {
-            p0 = a;
-            p1 = bb;
-          }
-        }
         x0 *= sl;  // scale > 0 commutes with max
         x1 *= sl;
-        const bool up0 = x0 > p0 + kRescaleThreshold, up1 = x1 > p1 + kRescaleThreshold;
-        const float n0 = up0 ? x0 : p0, n1 = up1 ? x1 : p1;
-        if (cq == 0) {
-          xmax[(k & 1u) * M + row0] = n0;
-          xmax[(k & 1u) * M + row1] = n1;
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&max_bar[k & 1u]);
-        mf0 = n0;
-        mf1 = n1;
-        // O rows that already hold this item's products (relative to the maxima of chunk k - 1)
-        // are rescaled in tensor memory once the products issued so far are done (warp-wide ld /
-        // st: the warp votes)
-        if (__any_sync(FULL, up0 || up1) && static_cast<int>(np) > first_np) {
-          const float a0 = up0 ? fast_exp2(p0 - n0) : 1.f, a1 = up1 ? fast_exp2(p1 - n1) : 1.f;
-          good = wait_o(np - 1) && good;
+        // the group's maxima are raised only when a score exceeds them by more than the threshold
+        const bool up0 = x0 > ml0 + kRescaleThreshold, up1 = x1 > ml1 + kRescaleThreshold;
+        const float n0 = up0 ? x0 : ml0, n1 = up1 ? x1 : ml1;
+        // O_g rows that already hold this item's products (those of the group's chunk k - 2) are
+        // rescaled in tensor memory once that product is done (warp-wide ld / st: the warp votes)
+        if (__any_sync(FULL, up0 || up1) && gk > 0) {
+          const float a0 = up0 ? fast_exp2(ml0 - n0) : 1.f, a1 = up1 ? fast_exp2(ml1 - n1) : 1.f;
+          good = wait_o(np - 2) && good;
 #pragma unroll
           for (int h = 0; h < D / 32; ++h) {  // 32 columns of the O rows per pass
             uint32_t ov[16];
-            tmem_ld16x256_x4(tl + C::TM_O + ob * D + h * 32, ov);
+            tmem_ld16x256_x4(tl + C::TM_O + grp * D + h * 32, ov);
             tc_wait_ld();
 #pragma unroll
             for (int i = 0; i < 16; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * ((i & 2) ? a1 : a0));
-            tmem_st16x256_x4(tl + C::TM_O + ob * D + h * 32, ov);
+            tmem_st16x256_x4(tl + C::TM_O + grp * D + h * 32, ov);
           }
           tc_wait_st();
         }
-        // this group's part of the sums follows the maxima (0 from none)
-        if (n0 > ml0) l0 *= fast_exp2(ml0 - n0);
-        if (n1 > ml1) l1 *= fast_exp2(ml1 - n1);
+        // the sums follow the maxima (0 from none)
+        if (up0) l0 *= fast_exp2(ml0 - n0);
+        if (up1) l1 *= fast_exp2(ml1 - n1);
         ml0 = n0;
         ml1 = n1;
+        ++gk;
         // the weights the MMA sees; the sums are taken over the same rounded values
         uint32_t pk[2][NJ];
         auto chunk_weights = [&](auto masked) {
@@ -868,28 +844,28 @@ __global__ void __launch_bounds__(TcCfg<KT>::NTHREADS, 1)
     if (lane == 0) mbar_arrive(&empty[c]);  // this warp is done with the chunk's meta and V rows
 
     if (last) {
-      // output of the item: each warp writes its group's half of the head_dim columns of its 16 rows
-      const bool o_any = static_cast<int>(np) > first_np;
+      // output of the item: each warp writes half of the head_dim columns of its 16 rows
+      const int nk = static_cast<int>(np) - first_np;  // the item's O products
+      const bool bad = poisoned || nk == 0;
       bool good = true;
-      float fin0 = mf0, fin1 = mf1;  // the maxima decided for the item's last chunk
-      if (!poisoned && o_any) {
-        good = wait_o(np - 1);
-        if ((last_k & 1u) != static_cast<uint32_t>(grp)) good = read_max(last_k, fin0, fin1) && good;
-      }
-      const bool bad = poisoned || !o_any;
-      // the rows' sums: this group's (the quad's parts, brought to the final maxima), then both
-      // groups' (one buffer per item parity: every item, poisoned or not, ends with this exchange,
-      // so a buffer is rewritten only after both warps have read it)
+      if (!bad) good = wait_o(np - 1);  // all of them done (they complete in order)
+      // the accumulators that hold the item's products: the group of its first chunk, and the
+      // other one when it has two or more
+      const bool even_me = (first_np & 1) == grp;  // this group took the item's chunks 0, 2, 4, ...
+      const bool has_me = !bad && (nk >= 2 || even_me);
+      const bool has_other = !bad && (nk >= 2 || !even_me);
+      // this group's (maximum, sum) of the rows to the other warp of the quarter (one buffer per
+      // item parity: every item, poisoned or not, ends with this exchange, so a buffer is
+      // rewritten only after both warps have read it)
       l0 += __shfl_xor_sync(FULL, l0, 1);
       l1 += __shfl_xor_sync(FULL, l1, 1);
       l0 += __shfl_xor_sync(FULL, l0, 2);
       l1 += __shfl_xor_sync(FULL, l1, 2);
-      const float g0 = bad ? 0.f : l0 * fast_exp2(ml0 - fin0), g1 = bad ? 0.f : l1 * fast_exp2(ml1 - fin1);
       const uint32_t ip = static_cast<uint32_t>(items) & 1u;
-      float* xs = xsum + ip * 2 * M;
+      float2* xs = xstate + ip * 2 * M;
       if (cq == 0) {
-        xs[grp * M + row0] = g0;
-        xs[grp * M + row1] = g1;
+        xs[grp * M + row0] = make_float2(ml0, l0);
+        xs[grp * M + row1] = make_float2(ml1, l1);
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&sum_bar[ip]);
@@ -898,51 +874,66 @@ __global__ void __launch_bounds__(TcCfg<KT>::NTHREADS, 1)
         ok = false;
         break;
       }
-      const float lt0 = g0 + xs[(grp ^ 1) * M + row0], lt1 = g1 + xs[(grp ^ 1) * M + row1];
+      const float2 ot0 = xs[(grp ^ 1) * M + row0], ot1 = xs[(grp ^ 1) * M + row1];
       if (busy) {
         const int seq = mt0.x, part = mt0.y & 0xffff, kvh = mt0.z & 0xff;
         const bool direct = (flags & F_DIRECT) != 0;
         int64_t ofs[2];
-        float fs[2];
+        // the factors of the accumulators of the item's even- and odd-place chunks, output scale
+        // included: the two states are always combined in that order (which group takes which
+        // chunks depends on the CTA's earlier items; the result does not)
+        float fev[2], fod[2];
         bool live[2];
 #pragma unroll
         for (int i = 0; i < 2; ++i) {
           const int r = i ? row1 : row0;
-          const float lt = i ? lt1 : lt0, mr = i ? fin1 : fin0;
+          const float mm = i ? ml1 : ml0, lm = i ? l1 : l0;
+          const float2 ot = i ? ot1 : ot0;
+          const float me = has_me ? mm : kNone, mo = has_other ? ot.x : kNone;
+          const float mr = even_me ? fmaxf(me, mo) : fmaxf(mo, me);
+          const float am = has_me ? fast_exp2(mm - mr) : 0.f, ao = has_other ? fast_exp2(ot.x - mr) : 0.f;
+          const float ae = even_me ? am : ao, aod = even_me ? ao : am;
+          const float lt = (even_me ? lm : ot.y) * ae + (even_me ? ot.y : lm) * aod;
           live[i] = r < ncol;
           const int mq = i ? rt1 : rt0, g = r - mq * G;
           const int mb = T > 1 ? 0 : mq, t = T > 1 ? item_t0 + mq : 0;
           const int vh = t * Hq + kvh * G + g;
+          float f;
           if (direct) {
             ofs[i] = (static_cast<int64_t>(seq + mb) * HV + vh) * D;
-            fs[i] = bad ? CUDART_NAN_F : p.v_scale / lt;
+            f = bad ? CUDART_NAN_F : p.v_scale / lt;
           } else {
             const int64_t pidx = static_cast<int64_t>(seq + mb) * p.max_parts + part;
             ofs[i] = (pidx * HV + vh) * D;
-            fs[i] = bad ? CUDART_NAN_F : p.v_scale;
+            f = bad ? CUDART_NAN_F : p.v_scale;
             if (live[i] && grp == 0 && cq == 0)
               __stcg(&p.part_ml[pidx * HV + vh], bad ? make_float2(0.f, CUDART_NAN_F) : make_float2(mr, lt));
           }
+          fev[i] = ae * f;
+          fod[i] = aod * f;
         }
 #pragma unroll
         for (int h2 = 0; h2 < 2; ++h2) {  // this warp's 64 columns, 32 per pass
           const int col0 = grp * 64 + h2 * 32;
-          uint32_t ov[16];
-          if (!bad) {
-            tmem_ld16x256_x4(tl + C::TM_O + ob * D + col0, ov);
-            tc_wait_ld();
-          } else {
+          uint32_t oe[16], oq[16];  // the even- and odd-place accumulators' columns
 #pragma unroll
-            for (int i = 0; i < 16; ++i) ov[i] = 0u;
-          }
+          for (int i = 0; i < 16; ++i) oe[i] = oq[i] = 0u;
+          const uint32_t ce = tl + C::TM_O + (grp ^ (even_me ? 0 : 1)) * D + col0;
+          const uint32_t cqd = tl + C::TM_O + (grp ^ (even_me ? 1 : 0)) * D + col0;
+          if (even_me ? has_me : has_other) tmem_ld16x256_x4(ce, oe);
+          if (even_me ? has_other : has_me) tmem_ld16x256_x4(cqd, oq);
+          tc_wait_ld();
 #pragma unroll
           for (int i = 0; i < 2; ++i) {
             if (!live[i]) continue;
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
               const int64_t e = ofs[i] + col0 + 8 * j + 2 * cq;
-              const float a = __uint_as_float(ov[4 * j + 2 * i]) * fs[i];
-              const float b2 = __uint_as_float(ov[4 * j + 2 * i + 1]) * fs[i];
+              // an accumulator without the item's products contributes an exact zero (its
+              // registers stay 0: tensor memory may hold anything there)
+              const float a = __uint_as_float(oe[4 * j + 2 * i]) * fev[i] + __uint_as_float(oq[4 * j + 2 * i]) * fod[i];
+              const float b2 =
+                  __uint_as_float(oe[4 * j + 2 * i + 1]) * fev[i] + __uint_as_float(oq[4 * j + 2 * i + 1]) * fod[i];
               if (!direct)
                 __stcg(reinterpret_cast<float2*>(p.part_acc + e), make_float2(a, b2));
               else if (p.out_dtype == DT_F32)
@@ -956,7 +947,9 @@ __global__ void __launch_bounds__(TcCfg<KT>::NTHREADS, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&o_free[ob]);  // the next item but one may overwrite this O buffer
+      // the next item with O products may overwrite the accumulators (only such items complete
+      // o_free: its phases then follow the O warp's count)
+      if (!bad && lane == 0) mbar_arrive(o_free);
     }
     ++n;
   }
