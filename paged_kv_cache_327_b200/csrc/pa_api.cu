@@ -143,6 +143,28 @@ int encode_kv_map(CUtensorMap* map, const void* base, int kv_dtype, int64_t num_
   return r == CUDA_SUCCESS ? PA_OK : PA_ERR_CUDA;
 }
 
+// A 16-bit K cache with head_dim 128 for the tensor-core kernel, seen as a 4-D tensor (64 elements,
+// 8 rows, column blocks of 64 elements of every KV head, groups of 8 rows): one box = the page of
+// one KV head (2 column blocks x 16 rows), landing as [row half][column block][8 rows][128 bytes]
+// with the 128-byte swizzle.  Consecutive pages of a chunk then hold each column block's 8-row
+// groups 2048 bytes apart: the K-major operand of a 64-token S product, one box per page.
+int encode_k_tc_map(CUtensorMap* map, const void* base, int kv_dtype, int64_t num_blocks, int block_size,
+                    int num_kv_heads) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+  if (!enc) return PA_ERR_CUDA;
+  const cuuint64_t pitch = static_cast<cuuint64_t>(num_kv_heads) * 256;  // bytes of a token row
+  const cuuint64_t groups = static_cast<cuuint64_t>(num_blocks) * block_size / 8;
+  const cuuint64_t dims[4] = {64, 8, static_cast<cuuint64_t>(num_kv_heads) * 2, groups};
+  const cuuint64_t strides[3] = {pitch, 128, 8 * pitch};
+  const cuuint32_t box[4] = {64, 8, 2, static_cast<cuuint32_t>(block_size / 8)};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  const CUtensorMapDataType dt = kv_dtype == PA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  const CUresult r = enc(map, dt, 4, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? PA_OK : PA_ERR_CUDA;
+}
+
 // The query [num_seqs * qtok rows, num_q_heads, head_dim] (16-bit) seen as a 4-D tensor (64
 // elements, 2 halves of head_dim, heads, rows); one box = the 64-element half of `box_rows` rows of
 // G consecutive heads, 128-byte swizzle: the K-major A operand of the tensor-core kernel.
@@ -470,8 +492,7 @@ int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cac
   CUtensorMap tmq;
   if (use_tc && (encode_q_map(&tmq, q, q_dtype, static_cast<int64_t>(num_seqs) * qtok, num_q_heads, G,
                               p.qbox_rows) != PA_OK ||
-                 encode_kv_map(&tmk_blocks, k_cache, kv_dtype, num_blocks, block_size, num_kv_heads, head_dim) !=
-                     PA_OK))
+                 encode_k_tc_map(&tmk_blocks, k_cache, kv_dtype, num_blocks, block_size, num_kv_heads) != PA_OK))
     return PA_ERR_CUDA;
   const CUtensorMap* tq = use_tc ? &tmq : nullptr;
   if (block_size == 16)

@@ -188,9 +188,10 @@ struct TcCfg {
   static constexpr int CT = CH * BS;                        // tokens per chunk: N of S
   static constexpr int NCH = 5;                             // chunk buffers
   static constexpr int BOX = BS * 128;                      // one TMA box: 16 rows x 128 bytes
-  static constexpr int KH_BYTES = CH * BOX;                 // one 64-element half of the chunk's K rows
-  static constexpr int VPAGE = 2 * BOX;                     // a V page: two halves
-  static constexpr int CHUNK_BYTES = 2 * KH_BYTES + CH * VPAGE;
+  static constexpr int KPAGE = 2 * BOX;                     // a K page: [row half][column block][8 rows][128 B]
+  static constexpr int VPAGE = 2 * BOX;                     // a V page: [column block][16 rows][128 B]
+  static constexpr int KC_BYTES = CH * KPAGE;               // the chunk's K rows
+  static constexpr int CHUNK_BYTES = KC_BYTES + CH * VPAGE;
   static constexpr int QHALF = M * 128;                     // one 64-element half of the query rows
   static constexpr int QBUF = 2 * QHALF;
   static constexpr int QN = 2;                              // query buffers
@@ -238,6 +239,16 @@ __device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, i
       "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
       " [%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(smem_u32(dst)),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(w), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// The same with an L2 cache policy.
+__device__ __forceinline__ void tma_load_4d_hint(void* dst, const CUtensorMap* map, int x, int y, int z, int w,
+                                                 uint64_t* bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%2, %3, %4, %5}], [%6], %7;" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(w), "r"(smem_u32(bar)), "l"(policy)
       : "memory");
 }
 
@@ -368,19 +379,20 @@ __device__ __forceinline__ void tc_produce(const DecodeParams& p, const CUtensor
       }
       __syncwarp();  // the expected byte count is set before any copy can complete
       if (!bad) {
-        // one box per lane: K column block 0 / K column block 1 / the whole V page, of page lane / 3
-        // (K rows go to the chunk's block-major K operand, a V page lands as [block][row])
-        const int lp = lane / 3, lk = lane - 3 * lp;
+        // one box per lane: the K page / the V page, of page lane / 2 (a K page lands as [row
+        // half][column block][8 rows], so the chunk's pages form the K operand with 8-row groups
+        // 2048 bytes apart; a V page lands as [block][row])
+        const int lp = lane >> 1, lk = lane & 1;
         // the chunk lies in one 32-page window (CH divides 32), so the window is warp-uniform
         const int win = pg0 >> 5;
         const int lphys = __shfl_sync(FULL, win == 0 ? cur.bt[0] : win == 1 ? cur.bt[1] : win == 2 ? cur.bt[2] : cur.bt[3],
                                       (pg0 + min(lp, C::CH - 1)) & 31);
         uint8_t* cb = smem + c * C::CHUNK_BYTES;
         if (lp < npg) {
-          if (lk < 2)
-            tma_load_3d(cb + lk * C::KH_BYTES + lp * C::BOX, &tmk, 0, kvh * 2 + lk, lphys * BS, &full[c], pol);
+          if (lk == 0)
+            tma_load_4d_hint(cb + lp * C::KPAGE, &tmk, 0, 0, kvh * 2, lphys * (BS / 8), &full[c], pol);
           else
-            tma_load_3d(cb + 2 * C::KH_BYTES + lp * C::VPAGE, &tmv, 0, lphys * BS, kvh * 2, &full[c], pol);
+            tma_load_3d(cb + C::KC_BYTES + lp * C::VPAGE, &tmv, 0, lphys * BS, kvh * 2, &full[c], pol);
         }
         // the item's query rows with its first chunk: rows (query token or member) x G heads, one
         // box per 64-element half, landing as the K-major A operand
@@ -471,8 +483,8 @@ __device__ __forceinline__ void tc_mma_s(uint8_t* smem, uint64_t* bars, const in
 #pragma unroll
         for (int k2 = 0; k2 < D / 16; ++k2) {
           const uint32_t a = qa + (k2 >> 2) * C::QHALF + (k2 & 3) * 32;
-          const uint32_t bk = kb + (k2 >> 2) * C::KH_BYTES + (k2 & 3) * 32;
-          umma_ss(tm + C::TM_S + b * C::CT, smem_desc_sw128(a, 16, 1024), smem_desc_sw128(bk, 16, 1024), C::IDESC_S,
+          const uint32_t bk = kb + (k2 >> 2) * 1024 + (k2 & 3) * 32;  // column block k2 / 4
+          umma_ss(tm + C::TM_S + b * C::CT, smem_desc_sw128(a, 16, 1024), smem_desc_sw128(bk, 16, 2048), C::IDESC_S,
                   k2 > 0);
         }
         umma_commit(&s_full[b]);
@@ -550,7 +562,7 @@ __device__ __forceinline__ void tc_mma_o(uint8_t* smem, uint64_t* bars, const in
     }
     if (lane == 0) {
       tc_fence_after();
-      const uint32_t vb = smem_u32(smem + c * C::CHUNK_BYTES + 2 * C::KH_BYTES);
+      const uint32_t vb = smem_u32(smem + c * C::CHUNK_BYTES + C::KC_BYTES);
       const uint32_t pa = smem_u32(smem + C::OFF_P + pb * C::PBUF);
       for (int j = 0; j < npg; ++j) {
         const uint64_t a = smem_desc_sw128(pa + j * 32, 16, 1024);
@@ -709,7 +721,7 @@ __global__ void __launch_bounds__(TcCfg<KT>::NTHREADS, 1)
         if (gt < CT && gt / C::BS == npg - 1 && (gt & (C::BS - 1)) >= ntok_last) {
           // V rows past the end of the item may hold anything (even NaN) and would meet zero
           // weights in the MMA: zero this token's row
-          uint8_t* vrow = cb + 2 * C::KH_BYTES + (npg - 1) * C::VPAGE + (gt & (C::BS - 1)) * 128;
+          uint8_t* vrow = cb + C::KC_BYTES + (npg - 1) * C::VPAGE + (gt & (C::BS - 1)) * 128;
 #pragma unroll
           for (int h = 0; h < 2; ++h)
 #pragma unroll
@@ -875,6 +887,28 @@ __global__ void __launch_bounds__(TcCfg<KT>::NTHREADS, 1)
         break;
       }
       const float2 ot0 = xs[(grp ^ 1) * M + row0], ot1 = xs[(grp ^ 1) * M + row1];
+      // this warp's 64 columns of both accumulators, read at once (an accumulator without the
+      // item's products is not read: its registers stay 0, tensor memory may hold anything there)
+      uint32_t oe[2][16], oq[2][16];  // the even- and odd-place accumulators, 32 columns per pass
+#pragma unroll
+      for (int h2 = 0; h2 < 2; ++h2)
+#pragma unroll
+        for (int i = 0; i < 16; ++i) oe[h2][i] = oq[h2][i] = 0u;
+      if (busy) {
+        const uint32_t ce = tl + C::TM_O + (grp ^ (even_me ? 0 : 1)) * D + grp * 64;
+        const uint32_t cqd = tl + C::TM_O + (grp ^ (even_me ? 1 : 0)) * D + grp * 64;
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2) {
+          if (even_me ? has_me : has_other) tmem_ld16x256_x4(ce + h2 * 32, oe[h2]);
+          if (even_me ? has_other : has_me) tmem_ld16x256_x4(cqd + h2 * 32, oq[h2]);
+        }
+      }
+      tc_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      // the next item with O products may overwrite the accumulators (only such items complete
+      // o_free: its phases then follow the O warp's count)
+      if (!bad && lane == 0) mbar_arrive(o_free);
       if (busy) {
         const int seq = mt0.x, part = mt0.y & 0xffff, kvh = mt0.z & 0xff;
         const bool direct = (flags & F_DIRECT) != 0;
@@ -913,27 +947,18 @@ __global__ void __launch_bounds__(TcCfg<KT>::NTHREADS, 1)
           fod[i] = aod * f;
         }
 #pragma unroll
-        for (int h2 = 0; h2 < 2; ++h2) {  // this warp's 64 columns, 32 per pass
+        for (int h2 = 0; h2 < 2; ++h2) {
           const int col0 = grp * 64 + h2 * 32;
-          uint32_t oe[16], oq[16];  // the even- and odd-place accumulators' columns
-#pragma unroll
-          for (int i = 0; i < 16; ++i) oe[i] = oq[i] = 0u;
-          const uint32_t ce = tl + C::TM_O + (grp ^ (even_me ? 0 : 1)) * D + col0;
-          const uint32_t cqd = tl + C::TM_O + (grp ^ (even_me ? 1 : 0)) * D + col0;
-          if (even_me ? has_me : has_other) tmem_ld16x256_x4(ce, oe);
-          if (even_me ? has_other : has_me) tmem_ld16x256_x4(cqd, oq);
-          tc_wait_ld();
 #pragma unroll
           for (int i = 0; i < 2; ++i) {
             if (!live[i]) continue;
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
               const int64_t e = ofs[i] + col0 + 8 * j + 2 * cq;
-              // an accumulator without the item's products contributes an exact zero (its
-              // registers stay 0: tensor memory may hold anything there)
-              const float a = __uint_as_float(oe[4 * j + 2 * i]) * fev[i] + __uint_as_float(oq[4 * j + 2 * i]) * fod[i];
-              const float b2 =
-                  __uint_as_float(oe[4 * j + 2 * i + 1]) * fev[i] + __uint_as_float(oq[4 * j + 2 * i + 1]) * fod[i];
+              const float a = __uint_as_float(oe[h2][4 * j + 2 * i]) * fev[i] +
+                              __uint_as_float(oq[h2][4 * j + 2 * i]) * fod[i];
+              const float b2 = __uint_as_float(oe[h2][4 * j + 2 * i + 1]) * fev[i] +
+                               __uint_as_float(oq[h2][4 * j + 2 * i + 1]) * fod[i];
               if (!direct)
                 __stcg(reinterpret_cast<float2*>(p.part_acc + e), make_float2(a, b2));
               else if (p.out_dtype == DT_F32)
@@ -945,11 +970,6 @@ __global__ void __launch_bounds__(TcCfg<KT>::NTHREADS, 1)
           }
         }
       }
-      tc_fence_before();
-      __syncwarp();
-      // the next item with O products may overwrite the accumulators (only such items complete
-      // o_free: its phases then follow the O warp's count)
-      if (!bad && lane == 0) mbar_arrive(o_free);
     }
     ++n;
   }
