@@ -81,7 +81,7 @@ def parse_args():
     ap.add_argument("--no-paths", action="store_true",
                     help="skip the compact measurement of the other decode paths (default run at N=1 only)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target oracle time for cpu_baseline")
-    ap.add_argument("--ref-seconds", type=float, default=150.0, help="target total time of --impl reference")
+    ap.add_argument("--ref-seconds", type=float, default=120.0, help="target total time of --impl reference")
     args = ap.parse_args()
     if args.config is None:
         args.config = "70b" if args.op == "cache" else "8b"
@@ -286,11 +286,11 @@ def oracle_post_step(w: W.Workload):
     return kc, vc
 
 
-def oracle_sample_rate(w: W.Workload, seconds: float, start: int = 0, threads: int = 0):
-    """Time the fp64 oracle on consecutive sequences (from `start`, wrapping) until ~`seconds` of work,
-    on `threads` threads (0: every core the process may run on).
-
-    Returns (KV bytes processed, seconds, threads, sequence count)."""
+def oracle_sampler(w: W.Workload, threads: int = 0):
+    """The fp64 oracle made ready to time on w (the caches after the step, and a pilot run that sizes
+    the samples), on `threads` threads (0: every core the process may run on).  Returns
+    sample(seconds, start) -> (KV bytes processed, seconds, threads, sequence count), which times the
+    oracle on consecutive sequences (from `start`, wrapping) until ~`seconds` of work."""
     import oracle
 
     threads = threads or oracle.default_threads()
@@ -303,30 +303,42 @@ def oracle_sample_rate(w: W.Workload, seconds: float, start: int = 0, threads: i
             return oracle.decode(q, w.q_dtype, kc, vc, w.kv_dtype, bt, sl, w.scale, num_threads=num_threads,
                                  k_scale=w.k_scale, v_scale=w.v_scale)
     row = 2 * w.kv_row_bytes
-    order = [(start + i) % w.num_seqs for i in range(w.num_seqs)]
     # pilot: one sequence of median length to size the sample
     med = int(np.argsort(w.seq_lens)[w.num_seqs // 2])
     t = time.perf_counter()
     run(np.ascontiguousarray(w.q[[med]]), np.ascontiguousarray(w.block_tables[[med]]), w.seq_lens[[med]], 1)
     per_token = (time.perf_counter() - t) / max(1, int(w.seq_lens[med]))
-    budget_tokens = seconds * threads / max(per_token, 1e-12)
-    pick, tok = [], 0
-    for i in order:
-        if tok >= budget_tokens and pick:
-            break
-        pick.append(i)
-        tok += int(w.seq_lens[i])
-    idx = np.asarray(pick)
-    q, bt, sl = (np.ascontiguousarray(w.q[idx]), np.ascontiguousarray(w.block_tables[idx]),
-                 np.ascontiguousarray(w.seq_lens[idx]))
-    passes, t = 0, time.perf_counter()
-    while True:  # whole passes over the sample until the time budget is used
-        run(q, bt, sl, threads)
-        passes += 1
-        dt = time.perf_counter() - t
-        if dt >= 0.8 * seconds:
-            break
-    return passes * tok * row, dt, threads, passes * len(idx)
+    # tokens per second on all threads: first the pilot's estimate, then what the last sample measured
+    rate = [threads / max(per_token, 1e-12)]
+
+    def sample(seconds: float, start: int = 0):
+        budget_tokens = seconds * rate[0]
+        pick, tok = [], 0
+        for k in range(w.num_seqs):
+            i = (start + k) % w.num_seqs
+            if tok >= budget_tokens and pick:
+                break
+            pick.append(i)
+            tok += int(w.seq_lens[i])
+        idx = np.asarray(pick)
+        q, bt, sl = (np.ascontiguousarray(w.q[idx]), np.ascontiguousarray(w.block_tables[idx]),
+                     np.ascontiguousarray(w.seq_lens[idx]))
+        passes, t = 0, time.perf_counter()
+        while True:  # whole passes over the sample until the time budget is used
+            run(q, bt, sl, threads)
+            passes += 1
+            dt = time.perf_counter() - t
+            if dt >= 0.8 * seconds:
+                break
+        rate[0] = passes * tok / max(dt, 1e-9)
+        return passes * tok * row, dt, threads, passes * len(idx)
+
+    return sample
+
+
+def oracle_sample_rate(w: W.Workload, seconds: float, start: int = 0, threads: int = 0):
+    """One timed sample of the fp64 oracle on w (see oracle_sampler)."""
+    return oracle_sampler(w, threads)(seconds, start)
 
 
 def run_reference(args):
@@ -334,14 +346,17 @@ def run_reference(args):
     if rank != 0:
         return 0
     w = make_workload(args)
-    per_step = max(0.5, args.ref_seconds / max(1, args.steps + args.warmup))
+    # the caches and the pilot once; then every step is one timed sample, sized so that the whole run
+    # takes about --ref-seconds whatever --steps and --warmup are
+    sample = oracle_sampler(w)
+    per_step = args.ref_seconds / max(1, args.steps + args.warmup)
     start = 0
     for _ in range(args.warmup):
-        _, _, _, n = oracle_sample_rate(w, per_step, start)
+        _, _, _, n = sample(per_step, start)
         start += n
     total_b, total_t, threads, seqs = 0, 0.0, 1, 0
     for _ in range(args.steps):
-        b, t, threads, n = oracle_sample_rate(w, per_step, start)
+        b, t, threads, n = sample(per_step, start)
         start += n
         total_b += b
         total_t += t
