@@ -312,11 +312,12 @@ def oracle_sampler(w: W.Workload, threads: int = 0):
     rate = [threads / max(per_token, 1e-12)]
 
     def sample(seconds: float, start: int = 0):
+        # at least one sequence per thread, so that every core has work
         budget_tokens = seconds * rate[0]
         pick, tok = [], 0
         for k in range(w.num_seqs):
             i = (start + k) % w.num_seqs
-            if tok >= budget_tokens and pick:
+            if tok >= budget_tokens and len(pick) >= min(threads, w.num_seqs):
                 break
             pick.append(i)
             tok += int(w.seq_lens[i])
